@@ -1,0 +1,329 @@
+"""CPU oracle for rotated-token KV-cache quantization (TurboQuant form).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline / reference leg may import this package.  The
+product library never loads it, and it shares no code, header, table or
+constant generator with the CUDA path: the heavy loops live in
+``oracle.cc`` (plain single-threaded fp64 C++), this module only marshals
+numpy arrays and states the packed cache layout.
+
+Parity status of every function here is pinned by ``tests/test_oracle_*.py``
+(closed forms, textbook tables, published PRNG vectors, statistics and
+brute force); nothing is "parity unpinned".
+
+Packed cache layout (the pages give none; reading recorded in the design
+notes).  Per stream of vectors (one (batch, head) of the cache, or one call
+of the quantizer), for vector t:
+
+* ``codes[t, p, w]`` (uint32): bit i = bit p of the Lloyd-Max code of
+  coordinate 32*w + i, for planes p = 0..b-1 (bit-plane layout);
+* ``qjl[t, w]`` (uint32): bit i = QJL sign bit of projection row 32*w + i;
+* ``norms[t, 0:2]`` (fp16): (||x||, ||r||) -- for the NSN front end
+  (||x||, ||w||);
+* NSN only: ``block_mean[blk, j]`` (fp16), mean of block ``blk`` of 128
+  tokens on channel j.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cc")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+NSN_BLOCK = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.cc into liboracle.so next to it (g++, fp64, no fast-math)."""
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            L = ctypes.CDLL(_LIB_PATH)
+            P = ctypes.c_void_p
+            L.orc_splitmix64.restype = ctypes.c_uint64
+            L.orc_splitmix64.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
+            L.orc_rademacher_signs.argtypes = [ctypes.c_int, ctypes.c_uint64, P]
+            L.orc_double_to_half.restype = ctypes.c_uint16
+            L.orc_double_to_half.argtypes = [ctypes.c_double]
+            L.orc_half_to_double.restype = ctypes.c_double
+            L.orc_half_to_double.argtypes = [ctypes.c_uint16]
+            L.orc_gaussian_fp16.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, P, P]
+            L.orc_lloyd_max_gaussian.restype = ctypes.c_int
+            L.orc_lloyd_max_gaussian.argtypes = [ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_double]
+            L.orc_rht.argtypes = [ctypes.c_int, P, P, P]
+            L.orc_qjl_sketch.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P, P]
+            L.orc_qjl_estimate.restype = ctypes.c_double
+            L.orc_qjl_estimate.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P, ctypes.c_double]
+            L.orc_qjl_trials.argtypes = [ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int64, ctypes.c_uint64, P]
+            L.orc_quantize.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P,
+                                       P, ctypes.c_int64, P, P, P, P, P, P]
+            L.orc_dequantize.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P,
+                                         P, P, P, ctypes.c_int64, P]
+            L.orc_decode_attend.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P,
+                                            P, ctypes.c_int, P, P, P, P, P, P, P, P, ctypes.c_int64,
+                                            ctypes.c_double, P, P]
+            L.orc_nsn_quantize.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P,
+                                           ctypes.c_int64, P, P, P, P, P, P, P]
+            _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ----------------------------------------------------------------------------
+# Random numbers and number formats
+# ----------------------------------------------------------------------------
+def splitmix64(seed: int, i: int) -> int:
+    return int(lib().orc_splitmix64(seed & (2**64 - 1), i))
+
+
+def rademacher_signs(d: int, seed: int) -> np.ndarray:
+    out = np.empty(d, np.int8)
+    lib().orc_rademacher_signs(d, seed & (2**64 - 1), _p(out))
+    return out
+
+
+def gaussian_fp16(rows: int, cols: int, seed: int):
+    """Returns (fp16 bit patterns uint16 [rows, cols], unrounded fp64 draws)."""
+    bits = np.empty((rows, cols), np.uint16)
+    draws = np.empty((rows, cols), np.float64)
+    lib().orc_gaussian_fp16(rows, cols, seed & (2**64 - 1), _p(bits), _p(draws))
+    return bits, draws
+
+
+def double_to_half_bits(x) -> np.ndarray:
+    x = np.asarray(x, np.float64)
+    f = lib().orc_double_to_half
+    return np.array([f(float(v)) for v in x.ravel()], np.uint16).reshape(x.shape)
+
+
+def half_bits_to_double(h) -> np.ndarray:
+    h = np.asarray(h, np.uint16)
+    f = lib().orc_half_to_double
+    return np.array([f(int(v)) for v in h.ravel()], np.float64).reshape(h.shape)
+
+
+# ----------------------------------------------------------------------------
+# Codebook and per-handle constants
+# ----------------------------------------------------------------------------
+def lloyd_max(b: int, max_iter: int = 1_000_000, tol: float = 1e-15):
+    """Gaussian Lloyd-Max codebook: (centroids[2^b], thresholds[2^b-1], mse, steps)."""
+    L = 1 << b
+    c = np.empty(L, np.float64)
+    t = np.empty(max(L - 1, 1), np.float64)
+    mse = ctypes.c_double()
+    it = lib().orc_lloyd_max_gaussian(b, _p(c), _p(t), ctypes.byref(mse), max_iter, tol)
+    return c, t[: L - 1], mse.value, it
+
+
+@dataclass
+class Constants:
+    """Everything the method fixes for one (d, b, seed): signs, S, codebook.
+
+    Reading of the pages (which give no PRNG): the Rademacher signs use the
+    SplitMix64 stream seeded with ``seed``; the Gaussian projection S (m = d
+    rows) uses the stream seeded with ``seed + 1`` and is rounded to fp16.
+    """
+
+    d: int
+    b: int
+    seed: int
+    delta: np.ndarray          # int8 [d]
+    S_half: np.ndarray         # uint16 [m, d] fp16 patterns
+    S: np.ndarray              # float64 [m, d] (exact values of the fp16 entries)
+    centroids: np.ndarray      # float64 [2^b]
+    thresholds: np.ndarray     # float64 [2^b - 1]
+    mse: float
+
+    @property
+    def m(self) -> int:
+        return self.d
+
+
+def make_constants(d: int, b: int, seed: int) -> Constants:
+    delta = rademacher_signs(d, seed)
+    s_half, _ = gaussian_fp16(d, d, seed + 1)
+    S = half_bits_to_double_fast(s_half)
+    c, t, mse, _ = lloyd_max(b)
+    return Constants(d, b, seed, delta, s_half, S, c, t, mse)
+
+
+def half_bits_to_double_fast(h) -> np.ndarray:
+    """fp16 pattern -> value; via numpy's binary16 (exactly representable in fp64)."""
+    return np.asarray(h, np.uint16).view(np.float16).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------
+# The method
+# ----------------------------------------------------------------------------
+def rht(delta: np.ndarray, v: np.ndarray) -> np.ndarray:
+    v = _c(v, np.float64)
+    d = v.shape[-1]
+    y = np.empty(d, np.float64)
+    lib().orc_rht(d, _p(_c(delta, np.int8)), _p(v), _p(y))
+    return y
+
+
+def qjl_sketch(S: np.ndarray, r: np.ndarray):
+    S = _c(S, np.float64)
+    r = _c(r, np.float64)
+    m, d = S.shape
+    bits = np.empty(m, np.uint8)
+    u = np.empty(m, np.float64)
+    lib().orc_qjl_sketch(m, d, _p(S), _p(r), _p(bits), _p(u))
+    return bits, u
+
+
+def qjl_estimate(S: np.ndarray, q: np.ndarray, bits: np.ndarray, rnorm: float) -> float:
+    S = _c(S, np.float64)
+    m, d = S.shape
+    return float(lib().orc_qjl_estimate(m, d, _p(S), _p(_c(q, np.float64)), _p(_c(bits, np.uint8)),
+                                        float(rnorm)))
+
+
+def qjl_trials(m: int, q: np.ndarray, r: np.ndarray, T: int, seed0: int) -> np.ndarray:
+    """T independent QJL estimates of <q, r>, each with its own fp16 Gaussian S (m x d)."""
+    q = _c(q, np.float64)
+    r = _c(r, np.float64)
+    est = np.empty(T, np.float64)
+    lib().orc_qjl_trials(m, q.shape[0], _p(q), _p(r), T, seed0 & (2**64 - 1), _p(est))
+    return est
+
+
+def quantize(k: Constants, x: np.ndarray, use_qjl: bool = True) -> dict:
+    """Quantize rows of x ([n, d]) -> unpacked codes, bits, norms and intermediates."""
+    x = _c(x, np.float64)
+    n, d = x.shape
+    assert d == k.d
+    m = k.m if use_qjl else 0
+    codes = np.empty((n, d), np.int32)
+    bits = np.empty((n, max(m, 1)), np.uint8)
+    norm = np.empty(n, np.float64)
+    gamma = np.empty(n, np.float64)
+    z = np.empty((n, d), np.float64)
+    u = np.empty((n, max(m, 1)), np.float64)
+    lib().orc_quantize(d, k.b, m, int(use_qjl), _p(k.delta), _p(k.S), _p(k.centroids), _p(k.thresholds),
+                       _p(x), n, _p(codes), _p(bits), _p(norm), _p(gamma), _p(z), _p(u))
+    out = dict(codes=codes, norm=norm, gamma=gamma, z=z)
+    if use_qjl:
+        out.update(bits=bits, u=u)
+    return out
+
+
+def dequantize(k: Constants, codes, bits, norm, gamma, use_qjl: bool = True) -> np.ndarray:
+    codes = _c(codes, np.int32)
+    n, d = codes.shape
+    m = k.m if use_qjl else 0
+    bits = _c(bits if use_qjl else np.zeros((n, 1)), np.uint8)
+    xhat = np.empty((n, d), np.float64)
+    lib().orc_dequantize(d, k.b, m, int(use_qjl), _p(k.delta), _p(k.S), _p(k.centroids), _p(codes), _p(bits),
+                         _p(_c(norm, np.float64)), _p(_c(gamma, np.float64)), n, _p(xhat))
+    return xhat
+
+
+def decode_attend(k: Constants, q, kcache: dict, vcache: dict, scale: float, use_qjl: bool = True,
+                  want_logits: bool = True):
+    """Attention of G queries ([G, d]) over one KV head's key and value caches.
+
+    Each cache is a dict with ``codes`` [T, d], ``bits`` [T, m] (when QJL is
+    on), ``norm`` and ``gamma`` [T] -- the stored (fp16-widened) values.
+    Returns (logits [G, T] or None, out [G, d]).
+    """
+    q = _c(np.atleast_2d(q), np.float64)
+    G, d = q.shape
+    m = k.m if use_qjl else 0
+
+    def arrays(c):
+        codes = _c(c["codes"], np.int32).reshape(-1, d)
+        T = codes.shape[0]
+        bits = _c(c["bits"] if use_qjl else np.zeros((max(T, 1), 1)), np.uint8)
+        return codes, bits, _c(c["norm"], np.float64), _c(c["gamma"], np.float64), T
+
+    kc, kb, kn, kg, T = arrays(kcache)
+    vc, vb, vn, vg, Tv = arrays(vcache)
+    assert T == Tv
+    logits = np.empty((G, max(T, 1)), np.float64) if want_logits else None
+    out = np.empty((G, d), np.float64)
+    lib().orc_decode_attend(d, k.b, m, int(use_qjl), _p(k.delta), _p(k.S), _p(k.centroids), _p(q), G,
+                            _p(kc), _p(kb), _p(kn), _p(kg), _p(vc), _p(vb), _p(vn), _p(vg), T,
+                            float(scale), _p(logits), _p(out))
+    return (logits[:, :T] if want_logits else None), out
+
+
+def nsn_quantize(k: Constants, x, mean_in=None) -> dict:
+    """NSN front end + quantizer (no QJL) on one head's tokens ([n_tok, d], n_tok % 128 == 0)."""
+    x = _c(x, np.float64)
+    n, d = x.shape
+    assert n % NSN_BLOCK == 0
+    nb = n // NSN_BLOCK
+    codes = np.empty((n, d), np.int32)
+    nx = np.empty(n, np.float64)
+    nw = np.empty(n, np.float64)
+    mean_half = np.empty((nb, d), np.uint16)
+    mean_f64 = np.empty((nb, d), np.float64)
+    z = np.empty((n, d), np.float64)
+    mi = None if mean_in is None else _c(mean_in, np.uint16)
+    lib().orc_nsn_quantize(d, k.b, NSN_BLOCK, _p(k.delta), _p(k.centroids), _p(k.thresholds), _p(x), n,
+                           _p(mi), _p(codes), _p(nx), _p(nw), _p(mean_half), _p(mean_f64), _p(z))
+    return dict(codes=codes, norm_x=nx, norm_w=nw, mean_half=mean_half, mean_f64=mean_f64, z=z)
+
+
+# ----------------------------------------------------------------------------
+# Packed cache layout (see module docstring)
+# ----------------------------------------------------------------------------
+def pack_codes(codes: np.ndarray, b: int) -> np.ndarray:
+    codes = np.asarray(codes, np.int64)
+    n, d = codes.shape
+    words = np.zeros((n, b, d // 32), np.uint32)
+    for p in range(b):
+        plane = ((codes >> p) & 1).astype(np.uint64).reshape(n, d // 32, 32)
+        words[:, p, :] = (plane << np.arange(32, dtype=np.uint64)).sum(axis=2).astype(np.uint32)
+    return words
+
+
+def unpack_codes(words: np.ndarray, b: int, d: int) -> np.ndarray:
+    words = np.asarray(words, np.uint32).reshape(-1, b, d // 32).astype(np.uint64)
+    n = words.shape[0]
+    codes = np.zeros((n, d), np.int32)
+    sh = np.arange(32, dtype=np.uint64)
+    for p in range(b):
+        plane = ((words[:, p, :, None] >> sh) & 1).reshape(n, d).astype(np.int32)
+        codes |= plane << p
+    return codes
+
+
+def pack_bits(bits: np.ndarray) -> np.ndarray:
+    bits = np.asarray(bits, np.uint64)
+    n, m = bits.shape
+    return (bits.reshape(n, m // 32, 32) << np.arange(32, dtype=np.uint64)).sum(axis=2).astype(np.uint32)
+
+
+def unpack_bits(words: np.ndarray, m: int) -> np.ndarray:
+    words = np.asarray(words, np.uint32).reshape(-1, m // 32).astype(np.uint64)
+    n = words.shape[0]
+    return ((words[:, :, None] >> np.arange(32, dtype=np.uint64)) & 1).reshape(n, m).astype(np.uint8)
