@@ -1,0 +1,456 @@
+"""Benchmark of the rotated-token KV-cache quantizer on B200.
+
+Headline line: KV quantize tokens/s on one Llama-3-8B-shaped layer (8 KV
+heads x 32768 tokens x head_dim 128, bf16 K and V, 2-bit Lloyd-Max codes +
+1-bit QJL with m = 128).  One step quantizes that layer's K and V (two
+launches of the quantize kernel); a token is one position of the layer
+(8 heads x (K + V) = 16 vectors).  The same JSON line carries the measured
+decode attention (batch 16, 32/8 heads, 131072-token packed contexts) in
+GB/s of packed cache and the NSN front end (8 x 65536 x 128) in tokens/s.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+quantizes its own layer (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV quantize tokens/s"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
+    ap.add_argument("--no-nsn", action="store_true", help="skip the NSN front-end measurement")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--cpu-vectors", type=int, default=163840, help="vectors in the CPU oracle sample")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# plumbing
+# ----------------------------------------------------------------------------
+class Dist:
+    def __init__(self, n_gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world != n_gpus:
+            raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={self.world}")
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class Clocks:
+    """nvidia-smi samples of the current GPU during a timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        for r in csv.reader(io.StringIO(out)):
+            if len(r) >= 9:
+                self.rows.append([c.strip() for c in r])
+
+    def summary(self):
+        rows = getattr(self, "rows", [])
+        if not rows:
+            return None
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return float("nan")
+        sm = [num(r[1]) for r in rows]
+        mx = max(num(r[2]) for r in rows)
+        loaded = [s for s in sm if s == s and s > 0.5 * mx] or sm
+        reasons = set()
+        for r in rows:
+            for name, col in (("hw_slowdown", 5), ("hw_thermal_slowdown", 6), ("sw_thermal_slowdown", 7),
+                              ("sw_power_cap", 8)):
+                if r[col].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(rows), "power_w_max": max(num(r[3]) for r in rows)}
+
+
+def timed(dist: Dist, fn, steps: int, stream) -> float:
+    """Milliseconds for `steps` calls of fn(i), device-timed, max over ranks."""
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    return dist.max(e0.elapsed_time(e1))
+
+
+def traffic_record(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current build."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    fp = os.path.join(ROOT, "_build", "libkvq.fingerprint")
+    if not (os.path.exists(p) and os.path.exists(fp)):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    rec = j.get(kernel)
+    if not rec or rec.get("fingerprint") != open(fp).read().strip():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# our implementation
+# ----------------------------------------------------------------------------
+def bench_quantize(args, dist):
+    from calibration_free_rotated_token_b200 import _abi as kvq
+    from calibration_free_rotated_token_b200 import workloads as wl
+
+    c = wl.LLAMA_LAYER
+    H, T, d, b = c["heads"], c["tokens"], c["d"], c["b"]
+    h = kvq.Handle(d, b, c["handle_seed"], qjl=True)
+    copies = []
+    for i in range(4):
+        K = wl.llama_keys(H, T, d, c["k_seed"] + 100 * i + 1000 * dist.rank, device="cuda").reshape(-1, d)
+        V = wl.llama_values(H, T, d, c["v_seed"] + 100 * i + 1000 * dist.rank, device="cuda").reshape(-1, d)
+        copies.append((K, V))
+    n = H * T
+    outK = kvq.alloc_packed(h, n)
+    outV = kvq.alloc_packed(h, n)
+    stream = torch.cuda.current_stream()
+    launch_ev = []
+
+    def step(i, record=False):
+        K, V = copies[i % 4]
+        if record:
+            a, bq, cq = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a.record(stream)
+            kvq.kvq_quantize(h, K, *outK, stream=stream)
+            bq.record(stream)
+            kvq.kvq_quantize(h, V, *outV, stream=stream)
+            cq.record(stream)
+            launch_ev.append((a, bq, cq))
+        else:
+            kvq.kvq_quantize(h, K, *outK, stream=stream)
+            kvq.kvq_quantize(h, V, *outV, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    code, bits = kvq.kvq_status(h)
+    if code != 0:
+        raise RuntimeError(f"quantize status {code} bits {bits}")
+    with Clocks(torch.cuda.current_device()) as clk:
+        ms = timed(dist, lambda i: step(i, record=True), args.steps, stream)
+    launch_ms = []
+    for a, bq, cq in launch_ev:
+        launch_ms += [a.elapsed_time(bq), bq.elapsed_time(cq)]
+    code, bits = kvq.kvq_status(h)
+    if code != 0:
+        raise RuntimeError(f"quantize status {code} bits {bits}")
+
+    bytes_per_vec = 2 * d + b * d // 8 + d // 8 + 4
+    per_launch_bytes = n * bytes_per_vec
+    avg_launch_s = float(np.mean(launch_ms)) / 1e3
+    hbm, src = peaks()
+    achieved = per_launch_bytes / avg_launch_s / 1e9
+    res = dict(ms=ms, tokens_per_step=T, vectors_per_step=2 * n, launches=2 * args.steps,
+               roofline={"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(achieved / hbm, 4), "traffic": traffic_record("quantize_llama_layer"),
+                         "peak_source": f"{src} hbm_gbs (copy)", "kernel": "quantize_kernel<128,2,qjl,bf16>",
+                         "algorithmic_bytes_per_launch": per_launch_bytes,
+                         "avg_launch_ms": round(avg_launch_s * 1e3, 5)},
+               clocks=clk.summary())
+
+    # ---- end to end through the binding with host buffers ----
+    Kh = copies[0][0].cpu().pin_memory()
+    Vh = copies[0][1].cpu().pin_memory()
+    Kd = torch.empty_like(copies[0][0])
+    Vd = torch.empty_like(copies[0][1])
+    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in o] for o in (outK, outV)]
+
+    def e2e_step(i):
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        kvq.kvq_quantize(h, Kd, *outK, stream=stream)
+        kvq.kvq_quantize(h, Vd, *outV, stream=stream)
+        for ho, do in zip(host_out, (outK, outV)):
+            for x, y in zip(ho, do):
+                x.copy_(y, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    ms_e2e = timed(dist, e2e_step, max(3, args.steps // 2), stream)
+    e2e_steps = max(3, args.steps // 2)
+    h2d = Kh.numel() * Kh.element_size() + Vh.numel() * Vh.element_size()
+    d2h = sum(t.numel() * t.element_size() for o in host_out for t in o)
+    res["e2e"] = {"value": dist.world * T * e2e_steps / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                  "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / e2e_steps,
+                  "path": "pinned host K,V -> kvq_quantize (C ABI) -> pinned host codes, qjl, norms"}
+    res["sample_input"] = (copies[0][0][: args.cpu_vectors // 2].cpu(), copies[0][1][: args.cpu_vectors // 2].cpu())
+    h.close()
+    return res
+
+
+def bench_decode(args, dist):
+    from calibration_free_rotated_token_b200 import _abi as kvq
+    from calibration_free_rotated_token_b200 import workloads as wl
+
+    c = wl.DECODE
+    B, hq, hkv, d, T = c["batch"], c["hq"], c["hkv"], c["d"], c["T"]
+    h = kvq.Handle(d, c["b"], c["handle_seed"], qjl=True)
+    S = B * hkv
+    kc = torch.empty((S, T, h.b, d // 32), dtype=torch.int32, device="cuda")
+    vc = torch.empty_like(kc)
+    kq = torch.empty((S, T, d // 32), dtype=torch.int32, device="cuda")
+    vq = torch.empty_like(kq)
+    kn = torch.empty((S, T, 2), dtype=torch.float16, device="cuda")
+    vn = torch.empty_like(kn)
+    for bi in range(B):
+        sl = slice(bi * hkv, (bi + 1) * hkv)
+        K = wl.llama_keys(hkv, T, d, wl.cache_slice_seed(c["handle_seed"], bi, dist.rank, 0), device="cuda")
+        kvq.kvq_quantize(h, K, kc[sl], kq[sl], kn[sl])
+        del K
+        V = wl.llama_values(hkv, T, d, wl.cache_slice_seed(c["handle_seed"], bi, dist.rank, 1), device="cuda")
+        kvq.kvq_quantize(h, V, vc[sl], vq[sl], vn[sl])
+        del V
+    q = wl.queries(B, hq, d, c["q_seed"], device="cuda", std=c["q_std"])
+    out = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(kvq.kvq_decode_workspace(h, B, hq, hkv, T), dtype=torch.uint8, device="cuda")
+    seq = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    kcache = kvq.make_cache(kc, kq, kn, T)
+    vcache = kvq.make_cache(vc, vq, vn, T)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        kvq.kvq_decode_attend(h, q, hkv, kcache, vcache, seq, T, c["scale"], out, ws, stream=stream)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    code, bits = kvq.kvq_status(h)
+    if code != 0:
+        raise RuntimeError(f"decode status {code} bits {bits}")
+    steps = max(5, args.steps // 2)
+    ms = timed(dist, step, steps, stream)
+    cache_bytes = S * T * 2 * (h.b * d // 8 + d // 8 + 4)
+    gbs = cache_bytes / (ms / steps / 1e3) / 1e9
+    hbm, src = peaks()
+    h.close()
+    return {"metric": "packed-cache decode-attn GB/s", "value": round(dist.world * gbs, 1), "unit": "GB/s",
+            "frac_of_hbm": round(gbs / hbm, 4), "ms_per_step": ms / steps, "steps": steps,
+            "workload": "batch 16, 32 query / 8 KV heads, d 128, 131072-token contexts, b=2 + QJL, one bf16 query token",
+            "cache_bytes_per_step": cache_bytes, "launches_per_step": 3,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "traffic": traffic_record("decode_split"),
+                         "peak_source": f"{src} hbm_gbs (copy)",
+                         "note": "whole decode call (qproj + split + combine); the split kernel dominates"}}
+
+
+def bench_nsn(args, dist):
+    from calibration_free_rotated_token_b200 import _abi as kvq
+    from calibration_free_rotated_token_b200 import workloads as wl
+
+    c = wl.NSN
+    H, T, d = c["heads"], c["tokens"], c["d"]
+    h = kvq.Handle(d, c["b"], c["handle_seed"], qjl=False)
+    xs = [wl.nsn_tokens(H, T, d, c["seed"] + i + 1000 * dist.rank, device="cuda") for i in range(4)]
+    codes = torch.empty((H, T, h.b, d // 32), dtype=torch.int32, device="cuda")
+    norms = torch.empty((H, T, 2), dtype=torch.float16, device="cuda")
+    means = torch.empty((H, T // 128, d), dtype=torch.float16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        kvq.kvq_nsn_quantize(h, xs[i % 4], codes, norms, means, stream=stream)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    code, bits = kvq.kvq_status(h)
+    if code != 0:
+        raise RuntimeError(f"nsn status {code} bits {bits}")
+    steps = args.steps
+    ms = timed(dist, step, steps, stream)
+    bytes_per_vec = 2 * d + h.b * d // 8 + 4 + 2 * d / 128
+    gbs = H * T * bytes_per_vec / (ms / steps / 1e3) / 1e9
+    hbm, src = peaks()
+    h.close()
+    return {"metric": "NSN quantize tokens/s", "value": dist.world * T * steps / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms / steps, "workload": "8 heads x 65536 tokens x d128 bf16, b=2, no QJL",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "traffic": traffic_record("nsn_quantize"),
+                         "peak_source": f"{src} hbm_gbs (copy)"}}
+
+
+def cpu_baseline(sample, n_vectors: int):
+    """The oracle, as it stands, on a bounded sample of the same workload (rank 0, N = 1)."""
+    import oracle
+    from calibration_free_rotated_token_b200 import workloads as wl
+
+    c = wl.LLAMA_LAYER
+    k = oracle.make_constants(c["d"], c["b"], c["handle_seed"])
+    K, V = sample
+    Kd = K.double().numpy()[: n_vectors // 2]
+    Vd = V.double().numpy()[: n_vectors // 2]
+    t0 = time.perf_counter()
+    oracle.quantize(k, Kd, True)
+    oracle.quantize(k, Vd, True)
+    dt = time.perf_counter() - t0
+    vec = Kd.shape[0] + Vd.shape[0]
+    return {"value": vec / 16 / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{vec} vectors ({vec // 16} tokens) of the layer's K and V, single-threaded fp64 C++, "
+                      f"{dt:.1f} s"}
+
+
+def run_ours(args):
+    dist = Dist(args.gpus)
+    torch.cuda.set_device(dist.local)
+    q = bench_quantize(args, dist)
+    extra = {}
+    if not args.no_decode:
+        extra["decode_attn"] = bench_decode(args, dist)
+    if not args.no_nsn:
+        extra["nsn_quantize"] = bench_nsn(args, dist)
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(q["sample_input"], args.cpu_vectors)
+    if dist.rank == 0:
+        value = dist.world * q["tokens_per_step"] * args.steps / (q["ms"] / 1e3)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": q["ms"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "llama3-8b-layer KV quantize: 8 KV heads x 32768 tokens x d128, bf16 K and V, "
+                                   "2-bit Lloyd-Max + 1-bit QJL (m=128)",
+                       "token": "one position of the layer = 8 heads x (K + V) = 16 vectors",
+                       "vectors_per_step": q["vectors_per_step"],
+                       "l2": "4 rotating input copies per rank (4 x 134 MB > 126 MB L2)",
+                       "parallelism": f"dp{dist.world} (independent layers per rank, no collective)"},
+            "roofline": q["roofline"], "cpu_baseline": cpu, "e2e": q["e2e"], "gpu_launches": q["launches"],
+            "clocks": q["clocks"],
+        }
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+def run_reference(args):
+    """The oracle on the host cores, same metric/unit/config, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from calibration_free_rotated_token_b200 import workloads as wl
+
+    c = wl.LLAMA_LAYER
+    k = oracle.make_constants(c["d"], c["b"], c["handle_seed"])
+    per_step = 1024  # vectors per step: 64 positions x 8 heads of K, and of V
+    K = wl.llama_keys(c["heads"], 64, c["d"], c["k_seed"]).reshape(-1, c["d"]).double().numpy()
+    V = wl.llama_values(c["heads"], 64, c["d"], c["v_seed"]).reshape(-1, c["d"]).double().numpy()
+    for i in range(args.warmup):
+        oracle.quantize(k, K[: per_step // 2], True)
+        oracle.quantize(k, V[: per_step // 2], True)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.quantize(k, K[: per_step // 2], True)
+        oracle.quantize(k, V[: per_step // 2], True)
+    dt = time.perf_counter() - t0
+    value = per_step / 16 * args.steps / dt
+    sample = f"{per_step} vectors ({per_step // 16} tokens) of the layer's K and V per step, single-threaded fp64 C++"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "llama3-8b-layer KV quantize: 8 KV heads x 32768 tokens x d128, bf16 K and V, "
+                                   "2-bit Lloyd-Max + 1-bit QJL (m=128)",
+                       "token": "one position of the layer = 8 heads x (K + V) = 16 vectors"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

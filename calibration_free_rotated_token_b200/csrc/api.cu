@@ -1,0 +1,406 @@
+// api.cu -- the C ABI of include/kvq.h: argument checks, the per-handle
+// constants (signs, Gaussian projection, Lloyd-Max codebook), TMA tensor
+// maps and kernel dispatch.  Host code only.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+
+#include "../../include/kvq.h"
+#include "kvq_internal.h"
+
+namespace kvq {
+// One per (d, b), from quantize_inst.cu.
+cudaError_t launch_quantize_d64_b1(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d64_b2(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d64_b3(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d64_b4(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d128_b1(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d128_b2(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d128_b3(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d128_b4(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d256_b1(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d256_b2(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d256_b3(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d256_b4(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                  const QuantArgs& a, int sms, cudaStream_t s);
+
+namespace {
+cudaError_t launch_quantize_any(int d, int b, bool qjl, bool nsn, const CUtensorMap& map, int dtype,
+                                const QuantArgs& a, int sms, cudaStream_t s) {
+#define KVQ_CASE(D, B) \
+    if (d == D && b == B) return launch_quantize_d##D##_b##B(qjl, nsn, map, dtype, a, sms, s);
+    KVQ_CASE(64, 1) KVQ_CASE(64, 2) KVQ_CASE(64, 3) KVQ_CASE(64, 4)
+    KVQ_CASE(128, 1) KVQ_CASE(128, 2) KVQ_CASE(128, 3) KVQ_CASE(128, 4)
+    KVQ_CASE(256, 1) KVQ_CASE(256, 2) KVQ_CASE(256, 3) KVQ_CASE(256, 4)
+#undef KVQ_CASE
+    return cudaErrorNotSupported;
+}
+}  // namespace
+}  // namespace kvq
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const std::string& msg) {
+    g_err = msg;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(KVQ_ECUDA, std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")");
+}
+
+// ---------------------------------------------------------------------------
+// Constants of a handle.  The pages draw random signs and a Gaussian
+// projection without naming a generator; this library uses SplitMix64
+// (Steele, Lea, Flood, OOPSLA 2014): output i of the stream seeded with s is
+// the finaliser applied to s + (i + 1) * 0x9E3779B97F4A7C15.
+// ---------------------------------------------------------------------------
+uint64_t sm64(uint64_t seed, uint64_t i) {
+    uint64_t x = seed + (i + 1) * 0x9E3779B97F4A7C15ULL;
+    x ^= x >> 30;
+    x *= 0xBF58476D1CE4E5B9ULL;
+    x ^= x >> 27;
+    x *= 0x94D049BB133111EBULL;
+    x ^= x >> 31;
+    return x;
+}
+
+// Normal draw number k of stream `seed`: Box-Muller (cosine branch) on the
+// top 53 bits of outputs 2k (shifted into (0, 1]) and 2k+1 (in [0, 1)).
+double normal_draw(uint64_t seed, uint64_t k) {
+    const double two53 = 9007199254740992.0;
+    const double u1 = static_cast<double>((sm64(seed, 2 * k) >> 11) + 1) / two53;
+    const double u2 = static_cast<double>(sm64(seed, 2 * k + 1) >> 11) / two53;
+    return std::sqrt(-2.0 * std::log(u1)) * std::cos(6.283185307179586476925286766559 * u2);
+}
+
+double phi(double x) { return std::isinf(x) ? 0.0 : 0.39894228040143267794 * std::exp(-0.5 * x * x); }
+double Phi(double x) {
+    if (std::isinf(x)) return x > 0 ? 1.0 : 0.0;
+    return 0.5 * std::erfc(-0.70710678118654752440 * x);
+}
+
+// Gaussian Lloyd-Max codebook with L = 2^b levels (PolarQuant section 2:
+// Lloyd-Max centroids for N(0, 1); TurboQuant "Como Implementar": codebooks
+// precomputed per bit width).  Fixed-point iteration on the interior
+// decision levels: given decision levels, each centroid is the conditional
+// mean of its cell; the new decision levels are the centroid midpoints.
+void lloyd_max_codebook(int b, std::vector<double>* cent, std::vector<double>* thr) {
+    const int L = 1 << b;
+    std::vector<double> t(L + 1), c(L);
+    for (int k = 0; k <= L; ++k) t[k] = (k == 0) ? -INFINITY : (k == L ? INFINITY : -3.0 + 6.0 * k / L);
+    for (int iter = 0; iter < 1000000; ++iter) {
+        for (int k = 0; k < L; ++k) c[k] = (phi(t[k]) - phi(t[k + 1])) / (Phi(t[k + 1]) - Phi(t[k]));
+        double change = 0.0;
+        for (int k = 1; k < L; ++k) {
+            const double nt = 0.5 * (c[k - 1] + c[k]);
+            change = std::fmax(change, std::fabs(nt - t[k]));
+            t[k] = nt;
+        }
+        if (change <= 1e-15) break;
+    }
+    for (int k = 0; k < L; ++k) c[k] = (phi(t[k]) - phi(t[k + 1])) / (Phi(t[k + 1]) - Phi(t[k]));
+    cent->assign(c.begin(), c.end());
+    thr->clear();
+    for (int k = 1; k < L; ++k) thr->push_back(0.5 * (c[k - 1] + c[k]));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D map over rows x d elements (row stride ld elements), box 128 bytes x
+// 128 rows, 128-byte swizzle, zero fill out of bounds.
+int make_row_map(CUtensorMap* map, const void* x, int dtype, int64_t rows, int d, int64_t ld) {
+    auto enc = encode_fn();
+    if (!enc) return fail(KVQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const int esz = dtype == KVQ_F32 ? 4 : 2;
+    const CUtensorMapDataType dt = dtype == KVQ_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : dtype == KVQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t gstride[1] = {static_cast<cuuint64_t>(ld) * esz};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 128u};
+    cuuint32_t estride[2] = {1u, 1u};
+    CUresult r = enc(map, dt, 2, const_cast<void*>(x), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KVQ_ECUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
+    return KVQ_OK;
+}
+
+int check_handle(const kvq_ctx* h) {
+    if (!h) return fail(KVQ_EINVAL, "null handle");
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != h->device)
+        return fail(KVQ_EINVAL, "handle was created on device " + std::to_string(h->device) +
+                                    " but the current device is " + std::to_string(dev));
+    return KVQ_OK;
+}
+
+void fill_common(const kvq_ctx* h, float* cent, float* thr, uint32_t* ps) {
+    for (int k = 0; k < kvq::kMaxLevels; ++k) {
+        cent[k] = k < static_cast<int>(h->centroids.size()) ? h->centroids[k] : 0.f;
+        thr[k] = k < static_cast<int>(h->thresholds.size()) ? h->thresholds[k] : INFINITY;
+    }
+    std::memcpy(ps, h->pair_sign, sizeof(h->pair_sign));
+}
+
+int quantize_common(kvq_handle h, const void* x, int dtype, int64_t rows, int64_t ld, uint32_t* codes,
+                    uint32_t* qjl, uint16_t* norms, uint16_t* block_mean, bool nsn, void* stream) {
+    if (int e = check_handle(h)) return e;
+    if (dtype != KVQ_F32 && dtype != KVQ_F16 && dtype != KVQ_BF16) return fail(KVQ_EINVAL, "unknown dtype");
+    if (rows < 0) return fail(KVQ_EINVAL, "negative vector count");
+    if (rows == 0) return KVQ_OK;
+    if (rows > (int64_t(1) << 31) - 128) return fail(KVQ_EINVAL, "more than 2^31 - 128 vectors in one call");
+    const int esz = dtype == KVQ_F32 ? 4 : 2;
+    if (ld < h->d) return fail(KVQ_EINVAL, "row stride ld is smaller than d");
+    if ((ld * esz) % 16 != 0) return fail(KVQ_EINVAL, "row stride ld * element size must be a multiple of 16 bytes");
+    if (!x || !aligned(x, 16)) return fail(KVQ_EINVAL, "x must be a non-null 16-byte aligned device pointer");
+    if (!codes || !aligned(codes, 16)) return fail(KVQ_EINVAL, "codes must be non-null and 16-byte aligned");
+    if (!norms || !aligned(norms, 4)) return fail(KVQ_EINVAL, "norms must be non-null and 4-byte aligned");
+    const bool has_qjl = (h->flags & KVQ_QJL) != 0;
+    if (!nsn) {
+        if (has_qjl && (!qjl || !aligned(qjl, 16))) return fail(KVQ_EINVAL, "qjl must be non-null and 16-byte aligned");
+        if (!has_qjl && qjl) return fail(KVQ_EINVAL, "qjl must be NULL for a handle without KVQ_QJL");
+    }
+    if (dtype == KVQ_F32 && h->d > 128) return fail(KVQ_EUNSUPPORTED, "fp32 input is built for d <= 128");
+    CUtensorMap map;
+    if (int e = make_row_map(&map, x, dtype, rows, h->d, ld)) return e;
+    kvq::QuantArgs a{};
+    a.n = rows;
+    a.ntiles = (rows + kvq::kTileRows - 1) / kvq::kTileRows;
+    a.codes = codes;
+    a.qjl = nsn ? nullptr : qjl;
+    a.norms = reinterpret_cast<__half2*>(norms);
+    a.block_mean = reinterpret_cast<__half*>(block_mean);
+    a.S = h->d_S;
+    a.status = h->d_status;
+    fill_common(h, a.centroid, a.threshold, a.pair_sign);
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t err = kvq::launch_quantize_any(h->d, h->b, has_qjl, nsn, map, dtype, a, sms, s);
+    if (err == cudaErrorNotSupported) return fail(KVQ_EUNSUPPORTED, "this (d, dtype, front end) is not built");
+    if (err != cudaSuccess) return cuda_fail(err, "quantize launch");
+    return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_last_error(void) { return g_err.c_str(); }
+
+int kvq_init(kvq_handle* out, int d, int b, uint64_t seed, uint32_t flags) {
+    g_err.clear();
+    if (!out) return fail(KVQ_EINVAL, "null output handle pointer");
+    *out = nullptr;
+    if (d != 64 && d != 128 && d != 256) return fail(KVQ_EINVAL, "d must be 64, 128 or 256");
+    if (b < 1 || b > 4) return fail(KVQ_EINVAL, "b must be in 1..4");
+    if (flags & ~KVQ_QJL) return fail(KVQ_EINVAL, "unknown flag bits");
+    kvq_ctx* h = new (std::nothrow) kvq_ctx();
+    if (!h) return fail(KVQ_ENOMEM, "host allocation failed");
+    cudaGetDevice(&h->device);
+    h->d = d;
+    h->b = b;
+    h->m = d;
+    h->flags = flags;
+    h->seed = seed;
+    h->signs.resize(d);
+    for (int j = 0; j < d; ++j) h->signs[j] = (sm64(seed, static_cast<uint64_t>(j)) >> 63) ? -1 : 1;
+    for (int k = 0; k < d / 2; ++k)
+        h->pair_sign[k] = (h->signs[2 * k] < 0 ? 0x8000u : 0u) | (h->signs[2 * k + 1] < 0 ? 0x80000000u : 0u);
+    h->S_half.resize(static_cast<size_t>(h->m) * d);
+    for (size_t k = 0; k < h->S_half.size(); ++k) {
+        const __half v = __double2half(normal_draw(seed + 1, k));
+        std::memcpy(&h->S_half[k], &v, 2);
+    }
+    std::vector<double> c, t;
+    lloyd_max_codebook(b, &c, &t);
+    h->centroids.assign(c.begin(), c.end());
+    h->thresholds.assign(t.begin(), t.end());
+    cudaError_t e = cudaMalloc(&h->d_S, h->S_half.size() * sizeof(__half));
+    if (e == cudaSuccess) e = cudaMalloc(&h->d_status, sizeof(uint32_t));
+    if (e == cudaSuccess)
+        e = cudaMemcpy(h->d_S, h->S_half.data(), h->S_half.size() * sizeof(__half), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) {
+        cudaFree(h->d_S);
+        cudaFree(h->d_status);
+        delete h;
+        return e == cudaErrorMemoryAllocation ? fail(KVQ_ENOMEM, "device allocation failed")
+                                              : cuda_fail(e, "kvq_init");
+    }
+    *out = h;
+    return KVQ_OK;
+}
+
+int kvq_destroy(kvq_handle h) {
+    g_err.clear();
+    if (!h) return KVQ_OK;
+    cudaFree(h->d_S);
+    cudaFree(h->d_status);
+    delete h;
+    return KVQ_OK;
+}
+
+int kvq_get_info(kvq_handle h, int* d, int* b, int* m, uint32_t* flags) {
+    g_err.clear();
+    if (!h) return fail(KVQ_EINVAL, "null handle");
+    if (d) *d = h->d;
+    if (b) *b = h->b;
+    if (m) *m = h->m;
+    if (flags) *flags = h->flags;
+    return KVQ_OK;
+}
+
+int kvq_get_constants(kvq_handle h, int8_t* signs, uint16_t* S, float* centroids, float* thresholds) {
+    g_err.clear();
+    if (!h) return fail(KVQ_EINVAL, "null handle");
+    if (signs) std::memcpy(signs, h->signs.data(), h->signs.size());
+    if (S) std::memcpy(S, h->S_half.data(), h->S_half.size() * 2);
+    if (centroids) std::memcpy(centroids, h->centroids.data(), h->centroids.size() * sizeof(float));
+    if (thresholds) std::memcpy(thresholds, h->thresholds.data(), h->thresholds.size() * sizeof(float));
+    return KVQ_OK;
+}
+
+int kvq_quantize(kvq_handle h, const void* x, int dtype, int64_t n, int64_t ld, uint32_t* codes, uint32_t* qjl,
+                 uint16_t* norms, void* stream) {
+    g_err.clear();
+    return quantize_common(h, x, dtype, n, ld, codes, qjl, norms, nullptr, false, stream);
+}
+
+int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, uint32_t* codes,
+                     uint16_t* norms, uint16_t* block_mean, void* stream) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "the NSN front end takes a handle without KVQ_QJL");
+    if (n_heads < 0 || n_tok < 0) return fail(KVQ_EINVAL, "negative size");
+    if (n_tok % 128 != 0) return fail(KVQ_EINVAL, "n_tok must be a multiple of 128 (NSN blocks of 128 tokens)");
+    if (h->d > 128) return fail(KVQ_EUNSUPPORTED, "the NSN front end is built for d <= 128");
+    if (n_heads * n_tok == 0) return KVQ_OK;
+    if (!block_mean || !aligned(block_mean, 2)) return fail(KVQ_EINVAL, "block_mean must be non-null");
+    return quantize_common(h, x, dtype, n_heads * n_tok, h->d, codes, nullptr, norms, block_mean, true, stream);
+}
+
+size_t kvq_decode_workspace(kvq_handle h, int batch, int hq, int hkv, int64_t max_T) {
+    if (!h || batch <= 0 || hq <= 0 || hkv <= 0 || max_T < 0) return 0;
+    int ns = 0;
+    int64_t chunk = 0;
+    size_t ws = 0;
+    kvq::decode_plan(h, batch, hq, hkv, max_T > 0 ? max_T : 1, &ns, &chunk, &ws);
+    return ws;
+}
+
+int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
+                      const kvq_cache* v, const int32_t* seq_len, int64_t max_T, float scale, float* logits,
+                      float* out, void* workspace, size_t ws_bytes, void* stream) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    if (dtype != KVQ_F32 && dtype != KVQ_F16 && dtype != KVQ_BF16) return fail(KVQ_EINVAL, "unknown dtype");
+    if (batch <= 0 || hq <= 0 || hkv <= 0) return fail(KVQ_EINVAL, "batch, hq and hkv must be positive");
+    if (hq % hkv != 0) return fail(KVQ_EINVAL, "hq must be a multiple of hkv");
+    const int G = hq / hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KVQ_EUNSUPPORTED, "hq / hkv must be 1, 2, 4 or 8");
+    if (max_T < 0) return fail(KVQ_EINVAL, "negative max_T");
+    if (!k || !v) return fail(KVQ_EINVAL, "null cache descriptor");
+    const bool has_qjl = (h->flags & KVQ_QJL) != 0;
+    for (const kvq_cache* c : {k, v}) {
+        if (!c->codes || !aligned(c->codes, 4) || !c->norms || !aligned(c->norms, 4))
+            return fail(KVQ_EINVAL, "cache codes/norms must be non-null and 4-byte aligned");
+        if (has_qjl && (!c->qjl || !aligned(c->qjl, 4))) return fail(KVQ_EINVAL, "cache qjl must be non-null");
+        if (c->capacity < max_T) return fail(KVQ_EINVAL, "cache capacity is smaller than max_T");
+    }
+    if (!q || !out || !seq_len) return fail(KVQ_EINVAL, "q, out and seq_len must be non-null");
+    if (!std::isfinite(scale)) return fail(KVQ_EINVAL, "scale must be finite");
+    int ns = 0;
+    int64_t chunk = 0;
+    size_t need = 0;
+    kvq::decode_plan(h, batch, hq, hkv, max_T > 0 ? max_T : 1, &ns, &chunk, &need);
+    if (!workspace || !aligned(workspace, 16)) return fail(KVQ_EINVAL, "workspace must be non-null and 16-byte aligned");
+    if (ws_bytes < need)
+        return fail(KVQ_EINVAL, "workspace too small: need " + std::to_string(need) + " bytes");
+    kvq::DecodeArgs a{};
+    a.batch = batch;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.G = G;
+    a.max_T = max_T;
+    a.nsplit = ns;
+    a.chunk = chunk;
+    a.q = q;
+    a.qdtype = dtype;
+    a.kcodes = k->codes;
+    a.kqjl = k->qjl;
+    a.knorms = reinterpret_cast<const __half2*>(k->norms);
+    a.vcodes = v->codes;
+    a.vqjl = v->qjl;
+    a.vnorms = reinterpret_cast<const __half2*>(v->norms);
+    a.kcap = k->capacity;
+    a.vcap = v->capacity;
+    a.seq_len = seq_len;
+    a.scale = scale;
+    a.logits = logits;
+    a.out = out;
+    const int64_t bh = static_cast<int64_t>(batch) * hq;
+    float* ws = static_cast<float*>(workspace);
+    a.qrot = ws;
+    a.qproj = ws + bh * h->d;
+    a.part = ws + bh * h->d + bh * h->m;
+    a.S = h->d_S;
+    float thr_unused[kvq::kMaxLevels];
+    fill_common(h, a.centroid, thr_unused, a.pair_sign);
+    std::string why;
+    cudaError_t e = kvq::launch_decode(h, a, static_cast<cudaStream_t>(stream), &why);
+    if (e != cudaSuccess) return cuda_fail(e, ("decode launch " + why).c_str());
+    return KVQ_OK;
+}
+
+int kvq_status(kvq_handle h, void* stream, uint32_t* bits) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpy(&v, h->d_status, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(h->d_status, 0, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "kvq_status");
+    if (bits) *bits = v;
+    if (v & KVQ_STATUS_TIMEOUT) return fail(KVQ_ETIMEOUT, "a kernel's bounded wait gave up");
+    if (v & (KVQ_STATUS_NONFINITE | KVQ_STATUS_NORM_OVERFLOW))
+        return fail(KVQ_ENONFINITE, "non-finite input or a norm above the fp16 range");
+    return KVQ_OK;
+}
+
+}  // extern "C"

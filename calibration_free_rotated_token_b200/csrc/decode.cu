@@ -1,0 +1,408 @@
+// decode.cu -- decode attention straight from the packed cache.
+//
+// Method (TurboQuant blog, "Como Implementar": the query is rotated once and
+// the logits come from the stored indices; PolarQuant section 2: the
+// dequantisation H^T/d, the centroid lookup and the stored norm, here moved
+// to the query side and to one final inverse rotation):
+//   q' = H (delta .* q), p = S q'                              (qproj_kernel)
+//   l_t = scale (n_t/d) (<q', c[code_t]> + sqrt(pi/2)/m gamma_t <p, sgn_t>)
+//   per split of the context: running max M, sum L, A = sum w n c[vcode],
+//   B = sum w n gamma sgn_v                                   (decode_split_kernel)
+//   merge the splits exactly, out = delta .* H (A + sqrt(pi/2)/m S^T B) / (d L)
+//                                                              (decode_combine_kernel)
+// Three launches on one stream; the split partials live in the caller's
+// workspace.  No kernel waits on another CTA.
+#include <cfloat>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+namespace {
+
+constexpr int kDecThreads = 256;
+constexpr int kTokTile = 256;  // tokens per split granule
+constexpr float kSqrtHalfPi = 1.2533141373155002512f;  // sqrt(pi/2)
+
+template <int DT>
+__device__ __forceinline__ float load_elem(const void* p, int64_t i) {
+    if (DT == 0) return reinterpret_cast<const float*>(p)[i];
+    if (DT == 1) return __half2float(reinterpret_cast<const __half*>(p)[i]);
+    const uint16_t u = reinterpret_cast<const uint16_t*>(p)[i];
+    return __uint_as_float(static_cast<uint32_t>(u) << 16);
+}
+
+__device__ __forceinline__ float sign_of(const uint32_t* pair_sign, int j) {
+    return ((pair_sign[j >> 1] >> ((j & 1) ? 31 : 15)) & 1u) ? -1.f : 1.f;
+}
+
+// In-place FWHT of D floats in shared memory by the whole block.
+template <int D>
+__device__ __forceinline__ void fwht_smem(float* s) {
+    for (int h = 1; h < D; h <<= 1) {
+        for (int p = threadIdx.x; p < D / 2; p += blockDim.x) {
+            const int i = (p / h) * 2 * h + (p % h);
+            const float x = s[i], y = s[i + h];
+            s[i] = x + y;
+            s[i + h] = x - y;
+        }
+        __syncthreads();
+    }
+}
+
+// q' = H (delta .* q) and p = S q' for one (batch, query head) per block.
+template <int D, int DT, bool QJL>
+__global__ void __launch_bounds__(kDecThreads) qproj_kernel(const __grid_constant__ DecodeArgs a) {
+    __shared__ float sq[D];
+    const int64_t bh = blockIdx.x;
+    for (int j = threadIdx.x; j < D; j += blockDim.x)
+        sq[j] = sign_of(a.pair_sign, j) * load_elem<DT>(a.q, bh * D + j);
+    __syncthreads();
+    fwht_smem<D>(sq);
+    for (int j = threadIdx.x; j < D; j += blockDim.x) a.qrot[bh * D + j] = sq[j];
+    if (QJL) {
+        for (int i = threadIdx.x; i < D; i += blockDim.x) {
+            const __half* Si = a.S + static_cast<int64_t>(i) * D;
+            float acc = 0.f;
+            for (int j = 0; j < D; ++j) acc = fmaf(__half2float(Si[j]), sq[j], acc);
+            a.qproj[bh * D + i] = acc;
+        }
+    }
+}
+
+template <int B>
+__device__ __forceinline__ int code_at(const uint32_t* planes, int words_per_plane, int j) {
+    int code = 0;
+#pragma unroll
+    for (int p = 0; p < B; ++p) code |= static_cast<int>((planes[p * words_per_plane + (j >> 5)] >> (j & 31)) & 1u) << p;
+    return code;
+}
+
+// One (split, kv head, batch) per block: tokens [split*chunk, (split+1)*chunk).
+template <int D, int B, bool QJL, int G>
+__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int M = D;                 // QJL rows
+    constexpr int WP = D / 32;           // words per plane
+    constexpr int KW = B * WP;           // code words per vector
+    constexpr int QW = QJL ? M / 32 : 0; // sign words per vector
+    constexpr int PART = 2 + D + M;
+    constexpr int TT = (D == 256) ? 128 : 256;  // tokens per tile (one per thread of phase A)
+    const int split = blockIdx.x, hk = blockIdx.y, bi = blockIdx.z;
+    const int tid = threadIdx.x;
+
+    __shared__ float sqr[G][D];
+    __shared__ float spq[G][QJL ? M : 1];
+    __shared__ float scb[1 << B];
+    __shared__ float sw[G][TT];                  // softmax weights of the tile
+    __shared__ uint32_t svc[TT][KW];             // value codes of the tile
+    __shared__ uint32_t svq[TT][QJL ? QW : 1];
+    __shared__ float svn[TT], svg[TT];
+    __shared__ float sred[G][kDecThreads / 32];
+    __shared__ float smax[G], salpha[G], ssum[G];
+
+    const int64_t T = min(static_cast<int64_t>(max(a.seq_len[bi], 0)), a.max_T);
+    const int64_t t0 = static_cast<int64_t>(split) * a.chunk;
+    const int64_t t1e = min(t0 + a.chunk, a.max_T);       // range this split owns (logit output)
+    const int64_t t1 = min(t1e, T);                        // tokens that exist
+    const int64_t stream = static_cast<int64_t>(bi) * a.hkv + hk;
+    const int64_t qh0 = static_cast<int64_t>(bi) * a.hq + static_cast<int64_t>(hk) * G;
+
+    for (int e = tid; e < G * D; e += blockDim.x) sqr[e / D][e % D] = a.qrot[(qh0 + e / D) * D + e % D];
+    if (QJL)
+        for (int e = tid; e < G * M; e += blockDim.x) spq[e / M][e % M] = a.qproj[(qh0 + e / M) * M + e % M];
+    if (tid < (1 << B)) scb[tid] = a.centroid[tid];
+    if (tid < G) {
+        smax[tid] = -INFINITY;
+        ssum[tid] = 0.f;
+    }
+    // value-side accumulators: thread role A (coordinate tid < D) and B (row tid - D < M)
+    float accA[G], accB[G], accA2[G], accB2[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) accA[g] = accB[g] = accA2[g] = accB2[g] = 0.f;
+    __syncthreads();
+
+    const uint32_t* kc = a.kcodes + stream * a.kcap * KW;
+    const uint32_t* kq = QJL ? a.kqjl + stream * a.kcap * QW : nullptr;
+    const __half2* kn = a.knorms + stream * a.kcap;
+    const uint32_t* vc = a.vcodes + stream * a.vcap * KW;
+    const uint32_t* vq = QJL ? a.vqjl + stream * a.vcap * QW : nullptr;
+    const __half2* vn = a.vnorms + stream * a.vcap;
+    const float kappa = kSqrtHalfPi / M;
+
+    for (int64_t tb = t0; tb < t1e; tb += TT) {
+        // ---- phase A: logits, one token per thread ----
+        const int64_t t = tb + tid;
+        const bool mine = tid < TT;
+        float l[G];
+        if (mine && t < t1) {
+            uint32_t cw[KW];
+#pragma unroll
+            for (int w = 0; w < KW; ++w) cw[w] = kc[t * KW + w];
+            float acc[G], accq[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) acc[g] = accq[g] = 0.f;
+#pragma unroll
+            for (int j = 0; j < D; ++j) {
+                const float c = scb[code_at<B>(cw, WP, j)];
+#pragma unroll
+                for (int g = 0; g < G; ++g) acc[g] = fmaf(sqr[g][j], c, acc[g]);
+            }
+            const float2 nk = __half22float2(kn[t]);
+            if (QJL) {
+                uint32_t qw[QJL ? QW : 1];
+#pragma unroll
+                for (int w = 0; w < QW; ++w) qw[w] = kq[t * QW + w];
+#pragma unroll
+                for (int i = 0; i < M; ++i) {
+                    const float s = ((qw[i >> 5] >> (i & 31)) & 1u) ? 1.f : -1.f;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) accq[g] = fmaf(spq[g][i], s, accq[g]);
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) l[g] = a.scale * (nk.x / D) * (acc[g] + (QJL ? kappa * nk.y * accq[g] : 0.f));
+        } else {
+#pragma unroll
+            for (int g = 0; g < G; ++g) l[g] = -INFINITY;
+        }
+        if (a.logits != nullptr && mine && t < t1e) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) a.logits[(qh0 + g) * a.max_T + t] = l[g];
+        }
+        // stage the value records of this tile
+        if (mine && t < t1) {
+#pragma unroll
+            for (int w = 0; w < KW; ++w) svc[tid][w] = vc[t * KW + w];
+            if (QJL)
+#pragma unroll
+                for (int w = 0; w < QW; ++w) svq[tid][w] = vq[t * QW + w];
+            const float2 nv = __half22float2(vn[t]);
+            svn[tid] = nv.x;
+            svg[tid] = nv.y;
+        }
+        // ---- phase B: tile max, running max, weights ----
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float mx = l[g];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if ((tid & 31) == 0) sred[g][tid >> 5] = mx;
+        }
+        __syncthreads();
+        if (tid < G) {
+            float mx = sred[tid][0];
+            for (int k = 1; k < kDecThreads / 32; ++k) mx = fmaxf(mx, sred[tid][k]);
+            const float mold = smax[tid];
+            const float mnew = fmaxf(mold, mx);
+            salpha[tid] = (mnew == -INFINITY) ? 1.f : __expf(mold - mnew);
+            smax[tid] = mnew;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float mnew = smax[g];
+            const float wgt = (l[g] == -INFINITY) ? 0.f : __expf(l[g] - mnew);
+            if (mine) sw[g][tid] = wgt;
+            float s = wgt;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if ((tid & 31) == 0) sred[g][tid >> 5] = s;
+        }
+        __syncthreads();
+        if (tid < G) {
+            float s = 0.f;
+            for (int k = 0; k < kDecThreads / 32; ++k) s += sred[tid][k];
+            ssum[tid] = ssum[tid] * salpha[tid] + s;
+        }
+        // ---- phase C: value sums, one coordinate (or QJL row) per thread ----
+        const int ntok = static_cast<int>(min(static_cast<int64_t>(TT), t1 - tb > 0 ? t1 - tb : 0));
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            accA[g] *= salpha[g];
+            accB[g] *= salpha[g];
+            accA2[g] *= salpha[g];
+            accB2[g] *= salpha[g];
+        }
+        for (int role = tid; role < D + (QJL ? M : 0); role += kDecThreads) {
+            const bool second = role >= kDecThreads;
+            if (role < D) {
+                const int j = role;
+                float acc[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) acc[g] = 0.f;
+                for (int tt = 0; tt < ntok; ++tt) {
+                    const float c = scb[code_at<B>(svc[tt], WP, j)] * svn[tt];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) acc[g] = fmaf(sw[g][tt], c, acc[g]);
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    if (second) accA2[g] += acc[g];
+                    else accA[g] += acc[g];
+                }
+            } else {
+                const int i = role - D;
+                float acc[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) acc[g] = 0.f;
+                for (int tt = 0; tt < ntok; ++tt) {
+                    const float s = ((svq[tt][i >> 5] >> (i & 31)) & 1u) ? 1.f : -1.f;
+                    const float c = s * svn[tt] * svg[tt];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) acc[g] = fmaf(sw[g][tt], c, acc[g]);
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    if (second) accB2[g] += acc[g];
+                    else accB[g] += acc[g];
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- partials: {M, L, A[D], B[M]} per query head ----
+    for (int role = tid, k = 0; role < D + (QJL ? M : 0); role += kDecThreads, ++k) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float* pp = a.part + ((qh0 + g) * a.nsplit + split) * PART;
+            if (role < D) pp[2 + role] = k ? accA2[g] : accA[g];
+            else pp[2 + role] = k ? accB2[g] : accB[g];
+        }
+    }
+    if (tid < G) {
+        float* pp = a.part + ((qh0 + tid) * a.nsplit + split) * PART;
+        pp[0] = smax[tid];
+        pp[1] = ssum[tid];
+    }
+}
+
+// Merge the splits of one (batch, query head) and rotate back.
+template <int D, bool QJL>
+__global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int M = D;
+    constexpr int PART = 2 + D + M;
+    __shared__ float sA[D], sB[M];
+    __shared__ float sf[512];
+    __shared__ float sL, sM;
+    const int64_t bh = blockIdx.x;
+    const float* pp = a.part + bh * a.nsplit * PART;
+    if (threadIdx.x == 0) {
+        float mx = -INFINITY;
+        for (int s = 0; s < a.nsplit; ++s)
+            if (pp[s * PART + 1] > 0.f) mx = fmaxf(mx, pp[s * PART]);
+        float L = 0.f;
+        for (int s = 0; s < a.nsplit; ++s) {
+            const float f = (pp[s * PART + 1] > 0.f) ? __expf(pp[s * PART] - mx) : 0.f;
+            sf[s] = f;
+            L += f * pp[s * PART + 1];
+        }
+        sL = L;
+        sM = mx;
+    }
+    __syncthreads();
+    const float L = sL;
+    if (!(L > 0.f)) {
+        for (int j = threadIdx.x; j < D; j += blockDim.x) a.out[bh * D + j] = 0.f;
+        return;
+    }
+    for (int e = threadIdx.x; e < D + (QJL ? M : 0); e += blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < a.nsplit; ++s) acc = fmaf(sf[s], pp[s * PART + 2 + e], acc);
+        if (e < D) sA[e] = acc;
+        else sB[e - D] = acc;
+    }
+    __syncthreads();
+    // v = A + sqrt(pi/2)/m S^T B, in place in sA
+    float vj[(D + kDecThreads - 1) / kDecThreads];
+    int k = 0;
+    for (int j = threadIdx.x; j < D; j += blockDim.x, ++k) {
+        float acc = sA[j];
+        if (QJL) {
+            float st = 0.f;
+            for (int i = 0; i < M; ++i) st = fmaf(__half2float(a.S[static_cast<int64_t>(i) * D + j]), sB[i], st);
+            acc = fmaf(kSqrtHalfPi / M, st, acc);
+        }
+        vj[k] = acc;
+    }
+    __syncthreads();
+    k = 0;
+    for (int j = threadIdx.x; j < D; j += blockDim.x, ++k) sA[j] = vj[k];
+    __syncthreads();
+    fwht_smem<D>(sA);
+    const float inv = 1.0f / (static_cast<float>(D) * L);
+    for (int j = threadIdx.x; j < D; j += blockDim.x) a.out[bh * D + j] = sign_of(a.pair_sign, j) * sA[j] * inv;
+}
+
+template <int D, int B, bool QJL>
+cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
+    const dim3 block(kDecThreads);
+    const int nbh = a.batch * a.hq;
+    switch (a.qdtype) {
+        case 0: qproj_kernel<D, 0, QJL><<<nbh, block, 0, s>>>(a); break;
+        case 1: qproj_kernel<D, 1, QJL><<<nbh, block, 0, s>>>(a); break;
+        default: qproj_kernel<D, 2, QJL><<<nbh, block, 0, s>>>(a); break;
+    }
+    const dim3 grid(a.nsplit, a.hkv, a.batch);
+    switch (a.G) {
+        case 1: decode_split_kernel<D, B, QJL, 1><<<grid, block, 0, s>>>(a); break;
+        case 2: decode_split_kernel<D, B, QJL, 2><<<grid, block, 0, s>>>(a); break;
+        case 4: decode_split_kernel<D, B, QJL, 4><<<grid, block, 0, s>>>(a); break;
+        default: decode_split_kernel<D, B, QJL, 8><<<grid, block, 0, s>>>(a); break;
+    }
+    decode_combine_kernel<D, QJL><<<nbh, block, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D, int B>
+cudaError_t launch_db(const DecodeArgs& a, bool qjl, cudaStream_t s) {
+    return qjl ? launch_d<D, B, true>(a, s) : launch_d<D, B, false>(a, s);
+}
+
+template <int D>
+cudaError_t launch_dd(const DecodeArgs& a, int b, bool qjl, cudaStream_t s) {
+    switch (b) {
+        case 1: return launch_db<D, 1>(a, qjl, s);
+        case 2: return launch_db<D, 2>(a, qjl, s);
+        case 3: return launch_db<D, 3>(a, qjl, s);
+        default: return launch_db<D, 4>(a, qjl, s);
+    }
+}
+
+}  // namespace
+
+void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, int* nsplit, int64_t* chunk,
+                 size_t* ws_bytes) {
+    (void)hq;
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
+    const int64_t streams = static_cast<int64_t>(batch) * hkv;
+    int64_t want = (4 * static_cast<int64_t>(sms) + streams - 1) / (streams > 0 ? streams : 1);
+    const int64_t tiles = (max_T + kTokTile - 1) / kTokTile;
+    if (want > tiles) want = tiles;
+    if (want > 512) want = 512;
+    if (want < 1) want = 1;
+    int64_t ch = (max_T + want - 1) / want;
+    ch = (ch + kTokTile - 1) / kTokTile * kTokTile;
+    if (ch < kTokTile) ch = kTokTile;
+    const int64_t ns = (max_T + ch - 1) / ch > 0 ? (max_T + ch - 1) / ch : 1;
+    *nsplit = static_cast<int>(ns);
+    *chunk = ch;
+    const int64_t bh = static_cast<int64_t>(batch) * hq;
+    const int64_t floats = bh * h->d + bh * h->m + bh * ns * (2 + h->d + h->m);
+    *ws_bytes = static_cast<size_t>(floats) * sizeof(float) + 256;
+}
+
+cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s, std::string* why) {
+    const bool qjl = (h->flags & 1u) != 0;
+    switch (h->d) {
+        case 64: return launch_dd<64>(a, h->b, qjl, s);
+        case 128: return launch_dd<128>(a, h->b, qjl, s);
+        case 256: return launch_dd<256>(a, h->b, qjl, s);
+        default:
+            if (why) *why = "unsupported head dimension";
+            return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace kvq

@@ -1,0 +1,90 @@
+// kvq_internal.h -- handle layout and kernel-launch interfaces shared by the
+// C-ABI layer (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+struct kvq_ctx {
+    int device = 0;
+    int d = 0, b = 0, m = 0;
+    uint32_t flags = 0;
+    uint64_t seed = 0;
+    // Host copies of the constants.
+    std::vector<int8_t> signs;        // [d]
+    std::vector<uint16_t> S_half;     // [m][d] fp16 patterns
+    std::vector<float> centroids;     // [2^b]
+    std::vector<float> thresholds;    // [2^b - 1]
+    // Sign masks of bf16/fp16 pairs: bit 15 = sign of coordinate 2k, bit 31 =
+    // sign of coordinate 2k+1 (1 = negative).  XOR flips both halves' signs.
+    uint32_t pair_sign[128] = {};
+    // Device constants.
+    __half* d_S = nullptr;            // [m][d]
+    uint32_t* d_status = nullptr;     // one word, ORed by kernels
+};
+
+namespace kvq {
+
+constexpr int kTileRows = 128;        // vectors per MMA tile (M of the S.r product)
+constexpr int kMaxLevels = 16;
+
+// Everything a quantize kernel needs besides the TMA tensor map.  Passed by
+// value as a __grid_constant__ parameter (lives in the constant bank).
+struct QuantArgs {
+    int64_t n;                        // vectors (rows)
+    int64_t ntiles;
+    uint32_t* codes;                  // [n][b][d/32]
+    uint32_t* qjl;                    // [n][d/32] or null
+    __half2* norms;                   // [n]
+    __half* block_mean;               // NSN: [n/128][d]
+    const __half* S;                  // [m][d] fp16 (global), copied to smem per CTA
+    uint32_t* status;
+    float centroid[kMaxLevels];
+    float threshold[kMaxLevels];
+    uint32_t pair_sign[128];
+};
+
+// Launch the quantizer (nsn = false) or the NSN front end + quantizer
+// (nsn = true) over n rows described by `map` (2-D TMA map, 128-byte swizzle,
+// box = 128 bytes x 128 rows).  Returns a cudaError_t.
+cudaError_t launch_quantize(const kvq_ctx* h, const CUtensorMap& map, int dtype, bool nsn, const QuantArgs& a,
+                            cudaStream_t s, std::string* why);
+
+struct DecodeArgs {
+    int batch, hq, hkv, G;            // G = hq / hkv
+    int64_t max_T;
+    int nsplit;
+    int64_t chunk;                    // tokens per split
+    const void* q;
+    int qdtype;
+    const uint32_t* kcodes;
+    const uint32_t* kqjl;
+    const __half2* knorms;
+    const uint32_t* vcodes;
+    const uint32_t* vqjl;
+    const __half2* vnorms;
+    int64_t kcap, vcap;               // vectors per stream
+    const int32_t* seq_len;
+    float scale;
+    float* logits;                    // nullable
+    float* out;
+    float* qrot;                      // workspace [batch*hq][d]   q' = H (delta.*q)
+    float* qproj;                     // workspace [batch*hq][m]   p = S q'
+    float* part;                      // workspace [batch*hq][nsplit][2 + d + m]
+    const __half* S;
+    float centroid[kMaxLevels];
+    uint32_t pair_sign[128];
+};
+
+// Bytes of workspace and number of splits for a decode of these sizes.
+void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, int* nsplit, int64_t* chunk,
+                 size_t* ws_bytes);
+
+cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s, std::string* why);
+
+}  // namespace kvq

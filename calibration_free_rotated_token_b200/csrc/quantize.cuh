@@ -1,0 +1,550 @@
+// quantize.cuh -- the quantize kernel (and its NSN front-end variant).
+//
+// Method (TurboQuant blog, "Estagio 1" and "Estagio 2"; PolarQuant section 2;
+// NSNQuant sections 1-2 for the front end), per vector x of dimension D:
+//   n = ||x||, z = H (delta .* x) / n, code_j = #{k : z_j >= t_k},
+//   r = z - c[code], gamma = ||r||, QJL bits = [S r >= 0], norms fp16.
+//
+// Design (sm_100a):
+// * Persistent CTAs, one per SM, two warpgroups (256 threads).  128-vector
+//   tiles stream through a ring of shared-memory stages with TMA (128-byte
+//   swizzle, so that a thread reading "its" row is bank-conflict free); as
+//   soon as a warpgroup has read a stage, its leader refills that stage with
+//   the tile kStages ahead, so loads run that far ahead of the compute.
+//   Tails past n are zero-filled by TMA and never stored.
+// * One thread owns one vector (D <= 128) or one half of it (D = 256: the two
+//   warpgroups cooperate on one tile and the top butterfly of the Hadamard
+//   transform is taken at load time).  The FWHT runs entirely in registers:
+//   no shuffles, no shared-memory round trips.
+// * Codes are written as bit planes built in registers; the residual r is
+//   split into fp16 hi + lo and stored into tensor memory (thread = TMEM lane
+//   = MMA row), and one elected thread issues tcgen05 MMAs
+//   D(128 x m) = A_hi S^T + A_lo S^T with S (fp16, exact) resident in shared
+//   memory.  The epilogue reads its own accumulator row back from TMEM and
+//   packs the sign bits.  S is an exact fp16 operand and r is carried to
+//   ~22 bits, so the sign of (S r)_i is exact wherever |(S r)_i| is above a
+//   few 1e-5 * ||r||.
+// * Every wait on an mbarrier is bounded; the outcome is agreed on by the
+//   whole warpgroup (barrier reduction) so no thread is left at a barrier.
+#pragma once
+
+#include <cfloat>
+
+#include "kvq_internal.h"
+#include "sm100.cuh"
+
+namespace kvq {
+
+enum { DT_F32 = 0, DT_F16 = 1, DT_BF16 = 2 };
+
+template <int D, int B, bool QJL, int DT, bool NSN>
+struct QCfg {
+    static constexpr int kEsz = (DT == DT_F32) ? 4 : 2;
+    static constexpr int kBoxCols = 128 / kEsz;            // elements per 128-byte box row
+    static constexpr int kBoxes = D * kEsz / 128;
+    static constexpr int kBoxBytes = 128 * kTileRows;      // 16 KB
+    static constexpr int kStageBytes = kBoxes * kBoxBytes;
+    static constexpr bool kCoop = (D == 256);              // two threads per vector
+    static constexpr int kNV = kCoop ? 128 : D;            // coordinates held per thread
+    static constexpr int kSBytes = QJL ? D * D * 2 : 0;    // S, fp16, m = D rows
+    static constexpr int kBudget = 200 * 1024;
+    static constexpr int kStagesRaw = (kBudget - kSBytes) / kStageBytes;
+    static constexpr int kStagesCap = kStagesRaw > 4 ? 4 : kStagesRaw;
+    // Without cooperation each warpgroup owns the stages of its tiles (tile i
+    // uses stage i % kStages and goes to warpgroup i % 2), so the count is even.
+    static constexpr int kStages = kCoop ? kStagesCap : (kStagesCap & ~1);
+    static constexpr int kThreads = 256;
+    static constexpr int kTmemCols = !QJL ? 0 : (kCoop ? 512 : (4 * D < 32 ? 32 : 4 * D));
+    static constexpr int kAuxBytes = 4096;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kSBytes + kAuxBytes;
+    static_assert(kStages >= 1, "input tile does not fit in shared memory");
+    static_assert(!(NSN && (QJL || kCoop)), "NSN front end: no QJL, D <= 128");
+};
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+// Load this thread's row (D <= 128) from a swizzled stage, applying the
+// Rademacher signs when SIGN (XOR of the element sign bits).
+template <int D, int DT, bool SIGN>
+__device__ __forceinline__ void load_row(const uint8_t* sp, int r, float (&v)[D], const uint32_t* psign) {
+    constexpr int kEsz = DT == DT_F32 ? 4 : 2;
+    constexpr int kEpc = 16 / kEsz;  // elements per 16-byte chunk
+#pragma unroll
+    for (int box = 0; box < D * kEsz / 128; ++box) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 q = *reinterpret_cast<const uint4*>(sp + box * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+            const int e0 = box * (128 / kEsz) + c * kEpc;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (DT == DT_F32) {
+                    const int e = e0 + k;
+                    uint32_t s = 0;
+                    if (SIGN) s = (psign[e >> 1] << ((e & 1) ? 0 : 16)) & 0x80000000u;
+                    v[e] = u2f(w[k] ^ s);
+                } else {
+                    const int pk = e0 / 2 + k;
+                    const uint32_t wd = w[k] ^ (SIGN ? psign[pk] : 0u);
+                    if (DT == DT_BF16) {
+                        v[2 * pk] = u2f(wd << 16);
+                        v[2 * pk + 1] = u2f(wd & 0xFFFF0000u);
+                    } else {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wd));
+                        v[2 * pk] = f.x;
+                        v[2 * pk + 1] = f.y;
+                    }
+                }
+            }
+        }
+    }
+}
+
+// D = 256, 16-bit input: half h of the rotated vector needs
+// v_j = delta_j x_j + (-1)^h delta_{j+128} x_{j+128}, j < 128 (the top
+// butterfly of the Sylvester transform), plus the full ||x||^2.
+template <int DT>
+__device__ __forceinline__ float load_row_coop(const uint8_t* sp, int r, int h, float (&v)[128],
+                                               const uint32_t* psign) {
+    float ss = 0.f;
+#pragma unroll
+    for (int box = 0; box < 2; ++box) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int off = r * 128 + ((c ^ (r & 7)) << 4);
+            const uint4 qa = *reinterpret_cast<const uint4*>(sp + box * 16384 + off);
+            const uint4 qb = *reinterpret_cast<const uint4*>(sp + (box + 2) * 16384 + off);
+            const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+            const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int pk = box * 32 + c * 4 + k;  // pair index within the half
+                const uint32_t xa = wa[k] ^ psign[pk];
+                const uint32_t xb = wb[k] ^ psign[pk + 64];
+                float a0, a1, b0, b1;
+                if (DT == DT_BF16) {
+                    a0 = u2f(xa << 16); a1 = u2f(xa & 0xFFFF0000u);
+                    b0 = u2f(xb << 16); b1 = u2f(xb & 0xFFFF0000u);
+                } else {
+                    const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&xa));
+                    const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&xb));
+                    a0 = fa.x; a1 = fa.y; b0 = fb.x; b1 = fb.y;
+                }
+                ss = fmaf(a0, a0, ss); ss = fmaf(a1, a1, ss);
+                ss = fmaf(b0, b0, ss); ss = fmaf(b1, b1, ss);
+                v[2 * pk] = h ? a0 - b0 : a0 + b0;
+                v[2 * pk + 1] = h ? a1 - b1 : a1 + b1;
+            }
+        }
+    }
+    return ss;
+}
+
+// In-register fast Walsh-Hadamard transform (Sylvester order, unnormalised).
+template <int N>
+__device__ __forceinline__ void fwht(float (&v)[N]) {
+#pragma unroll
+    for (int h = 1; h < N; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+        }
+    }
+}
+
+// code = #{k : z >= t_k}; c = centroid[code].
+template <int B>
+__device__ __forceinline__ uint32_t lm_code(float z, const float* th, const float* cb, float& c) {
+    uint32_t code = 0;
+    float cv = cb[0];
+#pragma unroll
+    for (int k = 0; k < (1 << B) - 1; ++k) {
+        const bool ge = z >= th[k];
+        code += ge ? 1u : 0u;
+        cv = ge ? cb[k + 1] : cv;
+    }
+    c = cv;
+    return code;
+}
+
+// z = v * inv; codes into bit planes; v <- r = z - c[code]; returns ||r||^2.
+template <int NV, int B>
+__device__ __forceinline__ float codes_and_residual(float (&v)[NV], float inv, const QuantArgs& a,
+                                                     uint32_t (&planes)[B][NV / 32]) {
+    float rr = 0.f;
+#pragma unroll
+    for (int p = 0; p < B; ++p)
+#pragma unroll
+        for (int w = 0; w < NV / 32; ++w) planes[p][w] = 0u;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        const float z = v[j] * inv;
+        float c;
+        const uint32_t code = lm_code<B>(z, a.threshold, a.centroid, c);
+#pragma unroll
+        for (int p = 0; p < B; ++p) planes[p][j / 32] |= ((code >> p) & 1u) << (j % 32);
+        const float r = z - c;
+        rr = fmaf(r, r, rr);
+        v[j] = r;
+    }
+    return rr;
+}
+
+// Residual (NV coordinates, starting at coordinate `k0` of the vector) as
+// fp16 hi/lo pairs into tensor memory: A_hi at column col_hi, A_lo at col_lo
+// (two fp16 per 32-bit column, even coordinate in the low half).
+template <int NV>
+__device__ __forceinline__ void store_residual_tmem(const float (&v)[NV], uint32_t t_hi, uint32_t t_lo) {
+#pragma unroll
+    for (int cc = 0; cc < NV / 64; ++cc) {
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float r0 = v[64 * cc + 2 * i], r1 = v[64 * cc + 2 * i + 1];
+            const __half2 hh = __floats2half2_rn(r0, r1);
+            const float2 hf = __half22float2(hh);
+            const __half2 ll = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
+            hi[i] = *reinterpret_cast<const uint32_t*>(&hh);
+            lo[i] = *reinterpret_cast<const uint32_t*>(&ll);
+        }
+        tmem_st32(t_hi + cc * 32, hi);
+        tmem_st32(t_lo + cc * 32, lo);
+    }
+    if (NV == 32) {
+        // not used: D >= 64
+    }
+}
+
+// Sign bits of NV accumulator columns of this thread's TMEM lane.
+template <int NV>
+__device__ __forceinline__ void qjl_bits_from_tmem(uint32_t taddr, uint32_t (&qw)[NV / 32]) {
+#pragma unroll
+    for (int cc = 0; cc < NV / 32; ++cc) {
+        uint32_t u[32];
+        tmem_ld32(taddr + cc * 32, u);
+        tmem_wait_ld();
+        uint32_t neg = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) neg |= (u[i] >> 31) << i;
+        qw[cc] = ~neg;  // bit = [u >= 0]
+    }
+}
+
+// Issue the QJL MMAs of one tile: acc(128 x N) = A_hi S^T + A_lo S^T.
+// K = KD coordinates, S resident in shared memory as KD/64 K-chunks of
+// N rows x 128 bytes (128-byte swizzle).
+template <int N, int KD>
+__device__ __forceinline__ void issue_qjl_mma(uint32_t acc, uint32_t a_hi, uint32_t a_lo, uint32_t s_smem) {
+    constexpr uint32_t idesc = idesc_f16_f32(kTileRows, N);
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+        for (int ks = 0; ks < KD / 16; ++ks) {
+            const uint32_t boff = (ks / 4) * (N * 128) + (ks % 4) * 32;
+            const uint64_t bd = smem_desc_sw128(s_smem + boff);
+            mma_f16_ts(acc, (pass ? a_lo : a_hi) + ks * 8, bd, idesc, (pass | ks) ? 1u : 0u);
+        }
+    }
+}
+
+template <int NWORDS>
+__device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t* src, uint32_t mask) {
+    if (NWORDS % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NWORDS; i += 4)
+            *reinterpret_cast<uint4*>(dst + i) =
+                make_uint4(src[i] & mask, src[i + 1] & mask, src[i + 2] & mask, src[i + 3] & mask);
+    } else {
+#pragma unroll
+        for (int i = 0; i < NWORDS; i += 2)
+            *reinterpret_cast<uint2*>(dst + i) = make_uint2(src[i] & mask, src[i + 1] & mask);
+    }
+}
+
+__device__ __forceinline__ void flag_norm(float ss, float nrm, uint32_t* status) {
+    if (!(ss < INFINITY)) atomicOr(status, kStatusNonFinite);
+    else if (nrm > 65504.f) atomicOr(status, kStatusNormOverflow);
+}
+
+template <int D, int B, bool QJL, int DT, bool NSN>
+__global__ void __launch_bounds__(256, 1)
+    quantize_kernel(const __grid_constant__ CUtensorMap map, const __grid_constant__ QuantArgs a) {
+    using C = QCfg<D, B, QJL, DT, NSN>;
+    constexpr int kStages = C::kStages;
+    constexpr int kWpp = D / 32;  // words per plane (whole vector)
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stage0 = smem;
+    uint8_t* sS = smem + kStages * C::kStageBytes;
+    uint8_t* aux = sS + C::kSBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(aux);   // [4]
+    uint64_t* mmadone = full + 4;                          // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mmadone + 2);
+    float* xch = reinterpret_cast<float*>(aux + 256);      // [2][128] floats
+    __half* so16 = reinterpret_cast<__half*>(aux + 256 + 1024);  // [2][128]
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int64_t G = gridDim.x;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        mbar_init(&mmadone[0], 1);
+        mbar_init(&mmadone[1], 1);
+        fence_mbar_init();
+    }
+    if (QJL) {
+        // S (m = D rows, K = D) into shared memory, K-major, 128-byte swizzle:
+        // K-chunk kc (64 fp16) of row n at sS + kc*D*128 + n*128, 16-byte
+        // chunk c stored at position c ^ (n & 7).
+        const uint4* gS = reinterpret_cast<const uint4*>(a.S);
+        for (int e = tid; e < D * D / 8; e += C::kThreads) {
+            const int n = e / (D / 8), cc = e % (D / 8);
+            const int kc = cc / 8, c16 = cc % 8;
+            *reinterpret_cast<uint4*>(sS + kc * (D * 128) + n * 128 + ((c16 ^ (n & 7)) << 4)) = gS[e];
+        }
+        fence_proxy_async_smem();
+        if (warp == 0) {
+            tmem_alloc(tmem_slot, C::kTmemCols);
+            tmem_relinquish();
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    uint32_t tmem = 0;
+    if (QJL) {
+        tc_fence_after();
+        tmem = *tmem_slot;
+    }
+
+    // Stage refill: tile i lives in stage i % kStages; the leader of the
+    // warpgroup that consumes it arms the stage's barrier and issues the TMA.
+    auto issue_tile = [&](int64_t i) {
+        const int64_t tile = blockIdx.x + i * G;
+        if (tile >= a.ntiles) return;
+        const int st = static_cast<int>(i % kStages);
+        mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+#pragma unroll
+        for (int box = 0; box < C::kBoxes; ++box)
+            tma_load_2d(stage0 + st * C::kStageBytes + box * C::kBoxBytes, &map, &full[st], box * C::kBoxCols,
+                        static_cast<int>(tile * kTileRows));
+    };
+    if (!C::kCoop) {
+        // ---------------- compute warpgroup w: one vector per thread ----------------
+        const int w = warp >> 2;
+        const int r = tid & 127;
+        const uint32_t bar_id = 1 + w;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tb = tmem + w * (2 * D);  // A_hi @ +0, A_lo @ +D/2, acc @ +D
+        if (r == 0) {
+            prefetch_tmap(&map);
+            for (int64_t i = w; i < kStages; i += 2) issue_tile(i);
+        }
+        int64_t jlocal = 0;
+        int64_t i = w;
+        for (;; i += 2, ++jlocal) {
+            const int64_t tile = blockIdx.x + i * G;
+            if (tile >= a.ntiles) break;
+            const int st = static_cast<int>(i % kStages);
+            const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((i / kStages) & 1), a.status);
+            if (named_bar_or(bar_id, 128, !ok)) break;
+            const uint8_t* sp = stage0 + st * C::kStageBytes;
+            const int64_t vidx = tile * kTileRows + r;
+            const bool valid = vidx < a.n;
+
+            float v[D];
+            float nx = 0.f, nrm;
+            if (NSN) {
+                load_row<D, DT, false>(sp, r, v, a.pair_sign);
+                float ss = 0.f;
+#pragma unroll
+                for (int j = 0; j < D; ++j) ss = fmaf(v[j], v[j], ss);
+                nx = sqrtf(ss);
+                flag_norm(ss, nx, a.status);
+                const float inv = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
+                xch[w * 128 + r] = inv;
+                named_bar_sync(bar_id, 128);
+                if (r < D) {
+                    // block mean of u = sqrt(D) x / ||x|| on channel j = r
+                    const int j = r;
+                    float acc = 0.f;
+                    for (int t = 0; t < kTileRows; ++t) {
+                        float xt;
+                        if (DT == DT_F32) {
+                            const uint8_t* p = sp + (j / 32) * 16384 + t * 128 + ((((j % 32) / 4) ^ (t & 7)) << 4) + (j % 4) * 4;
+                            xt = *reinterpret_cast<const float*>(p);
+                        } else {
+                            const uint8_t* p = sp + (j / 64) * 16384 + t * 128 + ((((j % 64) / 8) ^ (t & 7)) << 4) + (j % 8) * 2;
+                            const uint16_t hv = *reinterpret_cast<const uint16_t*>(p);
+                            xt = (DT == DT_BF16) ? u2f(static_cast<uint32_t>(hv) << 16)
+                                                 : __half2float(*reinterpret_cast<const __half*>(&hv));
+                        }
+                        acc = fmaf(xt, xch[w * 128 + t], acc);
+                    }
+                    const __half o16 = __float2half_rn(acc * (1.0f / kTileRows));
+                    so16[w * 128 + j] = o16;
+                    a.block_mean[tile * D + j] = o16;
+                }
+                named_bar_sync(bar_id, 128);
+                if (r == 0) issue_tile(i + kStages);
+                // w = u - fp16(o), then the Rademacher signs
+                float ws = 0.f;
+#pragma unroll
+                for (int j = 0; j < D; ++j) {
+                    float wv = v[j] * inv - __half2float(so16[w * 128 + j]);
+                    const uint32_t sbit = (a.pair_sign[j >> 1] << ((j & 1) ? 0 : 16)) & 0x80000000u;
+                    wv = u2f(__float_as_uint(wv) ^ sbit);
+                    ws = fmaf(wv, wv, ws);
+                    v[j] = wv;
+                }
+                nrm = sqrtf(ws);
+            } else {
+                load_row<D, DT, true>(sp, r, v, a.pair_sign);
+                named_bar_sync(bar_id, 128);
+                if (r == 0) issue_tile(i + kStages);
+                float ss = 0.f;
+#pragma unroll
+                for (int j = 0; j < D; ++j) ss = fmaf(v[j], v[j], ss);
+                nrm = sqrtf(ss);
+                flag_norm(ss, nrm, a.status);
+            }
+
+            fwht<D>(v);
+            const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+            uint32_t planes[B][kWpp];
+            const float rr = codes_and_residual<D, B>(v, inv, a, planes);
+            const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
+
+            if (QJL) {
+                store_residual_tmem<D>(v, tb + lane_base, tb + lane_base + D / 2);
+                tmem_wait_st();
+                tc_fence_before();
+                named_bar_sync(bar_id, 128);
+                if (r == 0) {
+                    tc_fence_after();
+                    issue_qjl_mma<D, D>(tb + D, tb, tb + D / 2, smem_u32(sS));
+                    mma_commit(&mmadone[w]);
+                }
+            }
+            if (valid) {
+                uint32_t* cp = a.codes + vidx * (B * kWpp);
+#pragma unroll
+                for (int p = 0; p < B; ++p) store_words<kWpp>(cp + p * kWpp, planes[p], zmask);
+                const float g = nrm > 0.f ? sqrtf(rr) : 0.f;
+                a.norms[vidx] = __halves2half2(__float2half_rn(NSN ? nx : nrm), __float2half_rn(NSN ? nrm : g));
+            }
+            if (QJL) {
+                const bool okm = mbar_wait(&mmadone[w], static_cast<uint32_t>(jlocal & 1), a.status);
+                if (named_bar_or(bar_id, 128, !okm)) break;
+                tc_fence_after();
+                uint32_t qw[kWpp];
+                qjl_bits_from_tmem<D>(tb + lane_base + D, qw);
+                tc_fence_before();
+                if (valid) store_words<kWpp>(a.qjl + vidx * kWpp, qw, zmask);
+            }
+        }
+        if (r == 0) {
+            // Loads issued for tiles i, i+2, ... (< i + kStages) that were not consumed.
+            for (int64_t k = i; k <= i + kStages; k += 2)
+                if (blockIdx.x + k * G < a.ntiles)
+                    mbar_wait(&full[k % kStages], static_cast<uint32_t>((k / kStages) & 1), a.status);
+        }
+    } else {
+        // ---------------- D = 256: both warpgroups on one tile, two threads per vector ----------------
+        const int h = warp >> 2;  // which half of the rotated vector
+        const int r = tid & 127;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        if (tid == 0) {
+            prefetch_tmap(&map);
+            for (int64_t i = 0; i < kStages; ++i) issue_tile(i);
+        }
+        int64_t jlocal = 0;
+        int64_t i = 0;
+        for (;; ++i, ++jlocal) {
+            const int64_t tile = blockIdx.x + i * G;
+            if (tile >= a.ntiles) break;
+            const int st = static_cast<int>(i % kStages);
+            const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((i / kStages) & 1), a.status);
+            if (named_bar_or(3, 256, !ok)) break;
+            const uint8_t* sp = stage0 + st * C::kStageBytes;
+            const int64_t vidx = tile * kTileRows + r;
+            const bool valid = vidx < a.n;
+
+            float v[128];
+            const float ss = load_row_coop<DT>(sp, r, h, v, a.pair_sign);
+            named_bar_sync(3, 256);
+            if (tid == 0) issue_tile(i + kStages);
+            const float nrm = sqrtf(ss);
+            if (h == 0) flag_norm(ss, nrm, a.status);
+            fwht<128>(v);
+            const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+            uint32_t planes[B][4];
+            const float rr = codes_and_residual<128, B>(v, inv, a, planes);
+            const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
+            xch[h * 128 + r] = rr;
+            if (QJL) {
+                // A_hi columns [0,128), A_lo [128,256), acc [256,512)
+                store_residual_tmem<128>(v, tmem + lane_base + h * 64, tmem + lane_base + 128 + h * 64);
+                tmem_wait_st();
+                tc_fence_before();
+            }
+            named_bar_sync(3, 256);
+            if (QJL && tid == 0) {
+                tc_fence_after();
+                issue_qjl_mma<256, 256>(tmem + 256, tmem, tmem + 128, smem_u32(sS));
+                mma_commit(&mmadone[0]);
+            }
+            if (valid) {
+                uint32_t* cp = a.codes + vidx * (B * 8) + h * 4;
+#pragma unroll
+                for (int p = 0; p < B; ++p) store_words<4>(cp + p * 8, planes[p], zmask);
+                if (h == 0) {
+                    const float g = nrm > 0.f ? sqrtf(xch[r] + xch[128 + r]) : 0.f;
+                    a.norms[vidx] = __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
+                }
+            }
+            if (QJL) {
+                const bool okm = mbar_wait(&mmadone[0], static_cast<uint32_t>(jlocal & 1), a.status);
+                if (named_bar_or(3, 256, !okm)) break;
+                tc_fence_after();
+                uint32_t qw[4];
+                qjl_bits_from_tmem<128>(tmem + lane_base + 256 + h * 128, qw);
+                tc_fence_before();
+                if (valid) store_words<4>(a.qjl + vidx * 8 + h * 4, qw, zmask);
+            }
+            // xch is rewritten next tile only after this barrier
+            named_bar_sync(3, 256);
+        }
+        if (tid == 0) {
+            for (int64_t k = i; k <= i + kStages; ++k)
+                if (blockIdx.x + k * G < a.ntiles)
+                    mbar_wait(&full[k % kStages], static_cast<uint32_t>((k / kStages) & 1), a.status);
+        }
+    }
+
+    __syncthreads();
+    if (QJL && warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int D, int B, bool QJL, int DT, bool NSN>
+cudaError_t launch_quantize_t(const CUtensorMap& map, const QuantArgs& a, int num_sms, cudaStream_t s) {
+    using C = QCfg<D, B, QJL, DT, NSN>;
+    auto kern = quantize_kernel<D, B, QJL, DT, NSN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = a.ntiles < num_sms ? a.ntiles : num_sms;
+    if (grid <= 0) return cudaSuccess;
+    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, s>>>(map, a);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -1,0 +1,44 @@
+// quantize_inst.cu -- instantiates the quantize kernels of one (d, b), given
+// as -DKVQ_D=<d> -DKVQ_B=<b> by the build; the build compiles this file once
+// per supported pair so that the twelve instantiations compile in parallel.
+#include "quantize.cuh"
+
+#ifndef KVQ_D
+#error "KVQ_D must be defined"
+#endif
+#ifndef KVQ_B
+#error "KVQ_B must be defined"
+#endif
+
+#define KVQ_CAT4(a, b, c, d) a##b##c##d
+#define KVQ_LAUNCH_NAME(D, B) KVQ_CAT4(launch_quantize_d, D, _b, B)
+
+namespace kvq {
+
+namespace {
+
+template <int D, int B, bool QJL, bool NSN>
+cudaError_t by_dtype(const CUtensorMap& map, int dtype, const QuantArgs& a, int sms, cudaStream_t s) {
+    if constexpr (NSN && (QJL || D > 128)) {
+        return cudaErrorNotSupported;
+    } else {
+        switch (dtype) {
+            case DT_F32:
+                if constexpr (D <= 128) return launch_quantize_t<D, B, QJL, DT_F32, NSN>(map, a, sms, s);
+                else return cudaErrorNotSupported;
+            case DT_F16: return launch_quantize_t<D, B, QJL, DT_F16, NSN>(map, a, sms, s);
+            default: return launch_quantize_t<D, B, QJL, DT_BF16, NSN>(map, a, sms, s);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t KVQ_LAUNCH_NAME(KVQ_D, KVQ_B)(bool qjl, bool nsn, const CUtensorMap& map, int dtype, const QuantArgs& a,
+                                           int sms, cudaStream_t s) {
+    if (nsn) return by_dtype<KVQ_D, KVQ_B, false, true>(map, dtype, a, sms, s);
+    return qjl ? by_dtype<KVQ_D, KVQ_B, true, false>(map, dtype, a, sms, s)
+               : by_dtype<KVQ_D, KVQ_B, false, false>(map, dtype, a, sms, s);
+}
+
+}  // namespace kvq

@@ -1,0 +1,208 @@
+/*
+ * kvq.h -- C ABI of the B200 (sm_100a) rotated-token KV-cache quantizer.
+ *
+ * The method (TurboQuant form, calibration free):
+ *   quantize  x -> ||x||, z = H (delta .* x) / ||x||, b-bit Gaussian Lloyd-Max
+ *             codes of z, residual r = z - c[code], 1-bit QJL sketch
+ *             sign(S r), fp16 norms (||x||, ||r||);
+ *   decode    rotate each query once, logits straight from the packed codes
+ *             plus the QJL correction, softmax, weighted sum of the decoded
+ *             values, all over the packed cache.
+ * Sources: "O Que E TurboQuant?" (TurboQuant blog), sections "Estagio 1:
+ * Rotacao Aleatoria + Compressao PolarQuant", "Estagio 2: Correcao Residual
+ * QJL" and "Como Implementar"; "PolarQuant: Optimal Gaussian Weight
+ * Quantization via Hadamard Rotation for LLM Compression", section 2
+ * (block normalisation, Walsh-Hadamard rotation, Gaussian Lloyd-Max,
+ * dequantisation); "NSNQuant: A Double Normalization Approach for
+ * Calibration-Free Low-Bit Vector Quantization of KV Cache", sections 1, 2
+ * and 4 (Normalize-Shift-Normalize front end, RHT, block flush).
+ *
+ * Conventions for every entry point:
+ *  - Return 0 (KVQ_OK) on success or a negative KVQ_E* code; the message of
+ *    the last failure on the calling thread is kvq_last_error().  Nothing is
+ *    thrown across the ABI and no kernel traps.
+ *  - Pointer arguments named as "device" must point to device memory of the
+ *    current CUDA device; the caller allocates and owns every input, output
+ *    and workspace buffer.  The handle owns only its constants.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls other than kvq_init / kvq_destroy / kvq_status /
+ *    kvq_get_constants are asynchronous on that stream and do not
+ *    synchronise.
+ *  - Errors in arguments are detected on the host before any launch
+ *    (KVQ_EINVAL / KVQ_EUNSUPPORTED) and leave outputs untouched.
+ *    Conditions found on the device (non-finite input, an fp16 norm
+ *    overflow, a bounded wait that gave up) are ORed into the handle's
+ *    device status word and reported by kvq_status().
+ *
+ * Packed cache layout.  A "stream" is a sequence of vectors of one head
+ * (one call of kvq_quantize, or one (batch, kv-head) of a cache).  For
+ * vector t of a stream, with L = 2^b levels, m = d projection rows:
+ *   codes  uint32 [t][b][d/32]  bit i of word (p, w) = bit p of the code of
+ *                               coordinate 32*w + i (bit planes);
+ *   qjl    uint32 [t][m/32]     bit i of word w = [ (S r)_{32w+i} >= 0 ];
+ *   norms  fp16   [t][2]        (||x||, ||r||)  -- NSN: (||x||, ||w||).
+ * Coordinates are in the rotated domain, Sylvester (natural) order.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+#define KVQ_OK 0
+#define KVQ_EINVAL (-1)       /* bad argument: null/misaligned pointer, size, dtype, layout */
+#define KVQ_EUNSUPPORTED (-2) /* valid by the method but not built (e.g. fp32 input at d = 256) */
+#define KVQ_ECUDA (-3)        /* a CUDA runtime/driver call failed (message has the CUDA error) */
+#define KVQ_ENOMEM (-4)       /* device or host allocation failed in kvq_init */
+#define KVQ_ENONFINITE (-5)   /* kvq_status: an input was NaN/Inf or a norm overflowed fp16 */
+#define KVQ_ETIMEOUT (-6)     /* kvq_status: a kernel's bounded wait gave up; outputs invalid */
+
+/* ---- flags of kvq_init ------------------------------------------------- */
+#define KVQ_QJL 1u            /* store the 1-bit QJL residual sketch (m = d rows) */
+
+/* ---- element types of inputs ------------------------------------------ */
+#define KVQ_F32 0
+#define KVQ_F16 1
+#define KVQ_BF16 2
+
+/* Device status word bits, as returned in *bits by kvq_status. */
+#define KVQ_STATUS_NONFINITE 1u
+#define KVQ_STATUS_NORM_OVERFLOW 2u
+#define KVQ_STATUS_TIMEOUT 4u
+
+typedef struct kvq_ctx* kvq_handle;
+
+/*
+ * kvq_init -- build the constants of one quantizer and upload them to the
+ * current device (TurboQuant blog, "Como Implementar": codebooks are
+ * precomputed per head dimension and bit width; no calibration data).
+ *   h      out: new handle (host pointer to a kvq_handle).
+ *   d      head dimension, one of 64, 128, 256 (power of two: FWHT).
+ *   b      Lloyd-Max bits per coordinate, 1..4.
+ *   seed   seeds the SplitMix64 streams: Rademacher signs use `seed`, the
+ *          Gaussian projection S (d x d, rounded to fp16) uses `seed + 1`.
+ *   flags  KVQ_QJL or 0.
+ * Synchronous.  Allocates device memory for the constants and a status
+ * word.  Errors: KVQ_EINVAL, KVQ_ENOMEM, KVQ_ECUDA.
+ */
+int kvq_init(kvq_handle* h, int d, int b, uint64_t seed, uint32_t flags);
+
+/* kvq_destroy -- free the handle and its device constants (synchronous).
+ * A NULL handle is accepted and ignored. */
+int kvq_destroy(kvq_handle h);
+
+/*
+ * kvq_quantize -- quantize n vectors (TurboQuant blog, Stages 1 and 2;
+ * PolarQuant section 2).  Per vector x (row i of x):
+ *   norm = ||x||; z = H (delta .* x) / norm; code_j = #{k : z_j >= t_k};
+ *   r = z - c[code]; gamma = ||r||; qjl bit_i = [(S r)_i >= 0];
+ *   norms = (fp16(norm), fp16(gamma)).  A zero vector stores all zeros.
+ *   x      device, n rows of d elements of `dtype`, row stride `ld`
+ *          elements (ld >= d; ld * element size a multiple of 16 bytes;
+ *          x 16-byte aligned).
+ *   n      number of vectors, >= 0 (0 is a no-op).
+ *   codes  device, n * b * d/32 uint32, 16-byte aligned.
+ *   qjl    device, n * d/32 uint32, 16-byte aligned; must be NULL when the
+ *          handle has no KVQ_QJL flag and non-NULL when it has.
+ *   norms  device, n * 2 fp16 (bit patterns), 4-byte aligned.
+ * fp32 input is built for d <= 128.  Non-finite inputs and norms above the
+ * fp16 range set status bits; those rows' outputs are unspecified.
+ */
+int kvq_quantize(kvq_handle h, const void* x, int dtype, int64_t n, int64_t ld, uint32_t* codes,
+                 uint32_t* qjl, uint16_t* norms, void* stream);
+
+/*
+ * kvq_nsn_quantize -- NSN front end then the quantizer without QJL
+ * (NSNQuant section 1 Normalize-Shift-Normalize, section 2 Hadamard, section
+ * 4 block flush).  For each head and each block of 128 consecutive tokens:
+ *   u_t = sqrt(d) x_t / ||x_t|| (0 for a zero token); o = mean_t u_t per
+ *   channel, stored as fp16; w_t = u_t - fp16(o); w_t is quantized as above
+ *   (codes of H (delta .* w_t) / ||w_t||); norms = (fp16 ||x_t||,
+ *   fp16 ||w_t||), i.e. s1 = ||x||/sqrt(d), s2 = ||w||/sqrt(d).
+ *   x           device, [n_heads][n_tok][d] contiguous, dtype as above.
+ *   n_tok       tokens per head, a multiple of 128 (the full-precision tail
+ *               of a real cache stays outside, NSNQuant section 4).
+ *   codes       device, n_heads * n_tok * b * d/32 uint32.
+ *   norms       device, n_heads * n_tok * 2 fp16.
+ *   block_mean  device, n_heads * (n_tok/128) * d fp16.
+ * Requires a handle without KVQ_QJL (KVQ_EINVAL otherwise).
+ */
+int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok,
+                     uint32_t* codes, uint16_t* norms, uint16_t* block_mean, void* stream);
+
+/* One packed cache (keys or values) of batch * hkv streams, each holding up
+ * to `capacity` vectors in the layout above; stream (bi, hi) starts at
+ * vector (bi * hkv + hi) * capacity. */
+typedef struct kvq_cache {
+    const uint32_t* codes;  /* device, streams * capacity * b * d/32 */
+    const uint32_t* qjl;    /* device, streams * capacity * d/32; NULL without KVQ_QJL */
+    const uint16_t* norms;  /* device, streams * capacity * 2 fp16 */
+    int64_t capacity;       /* vectors per stream, >= max_T */
+} kvq_cache;
+
+/* Bytes of device workspace kvq_decode_attend needs for these sizes. */
+size_t kvq_decode_workspace(kvq_handle h, int batch, int hq, int hkv, int64_t max_T);
+
+/*
+ * kvq_decode_attend -- one decode step of attention over packed K and V
+ * caches (TurboQuant blog, "Como Implementar": queries rotated once,
+ * logits computed straight from the indices; PolarQuant section 2
+ * dequantisation moved to the query side).  For query head g of batch bi,
+ * attending KV head hi = g / (hq / hkv) over tokens t < seq_len[bi]:
+ *   q' = H (delta .* q); p = S q'  (fp32)
+ *   l_t = scale * (n_t / d) * ( sum_j q'_j c[code_tj]
+ *                               + sqrt(pi/2)/m * gamma_t * sum_i p_i (2 bit_ti - 1) )
+ *   softmax over t (split over the context, merged exactly);
+ *   out = 1/(d sum_t w_t) * delta .* H ( sum_t w_t n_t c[vcode_t]
+ *           + sqrt(pi/2)/m * S^T sum_t w_t n_t gamma_t (2 vbit_t - 1) ).
+ *   q        device, [batch][hq][d] of `dtype`, contiguous.
+ *   hq, hkv  query and KV heads; hq a multiple of hkv, hq/hkv in {1,2,4,8}.
+ *   k, v     host pointers to cache descriptors (device buffers inside).
+ *   seq_len  device, int32 [batch], each in [0, max_T]; 0 gives a zero output.
+ *   max_T    bound on seq_len (sizes the split grid), <= capacity.
+ *   scale    logit scale (e.g. 1/sqrt(d)).
+ *   logits   device, fp32 [batch][hq][max_T] or NULL; entries past seq_len
+ *            are written as -inf.
+ *   out      device, fp32 [batch][hq][d].
+ *   workspace, ws_bytes  device scratch of at least
+ *            kvq_decode_workspace(h, batch, hq, hkv, max_T) bytes, 16-byte
+ *            aligned; contents on entry are ignored.
+ */
+int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv,
+                      const kvq_cache* k, const kvq_cache* v, const int32_t* seq_len, int64_t max_T,
+                      float scale, float* logits, float* out, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * kvq_status -- synchronise `stream`, read and clear the handle's device
+ * status word.  Returns KVQ_OK, KVQ_ENONFINITE or KVQ_ETIMEOUT (the most
+ * severe condition seen); *bits (nullable, host) receives the raw
+ * KVQ_STATUS_* bits.
+ */
+int kvq_status(kvq_handle h, void* stream, uint32_t* bits);
+
+/* kvq_last_error -- message of the last failure on this thread ("" if none).
+ * The string stays valid until the next kvq_* call on the same thread. */
+const char* kvq_last_error(void);
+
+/*
+ * kvq_get_constants -- copy the handle's constants to host buffers (any
+ * argument may be NULL): signs int8 [d] (+1/-1); S fp16 bit patterns
+ * [d][d] row-major; centroids fp32 [2^b] ascending; thresholds fp32
+ * [2^b - 1].  Synchronous.
+ */
+int kvq_get_constants(kvq_handle h, int8_t* signs, uint16_t* S, float* centroids, float* thresholds);
+
+/* kvq_get_info -- d, b, m and flags of a handle (host out-pointers, nullable). */
+int kvq_get_info(kvq_handle h, int* d, int* b, int* m, uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

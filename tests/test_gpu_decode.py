@@ -1,0 +1,171 @@
+"""Parity of the CUDA decode attention (through the C ABI) with the CPU oracle.
+
+Both sides decode the same packed cache, the oracle's own quantization of
+the seeded inputs, so only the attention arithmetic is compared."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from calibration_free_rotated_token_b200 import _abi as kvq
+from calibration_free_rotated_token_b200 import workloads as wl
+
+from .parity import assert_close, compare_quantize, oracle_cache, to_device_u32, to_np_f16bits, to_np_u32
+
+pytestmark = pytest.mark.gpu
+
+_consts = {}
+
+
+def constants(d, b, seed):
+    if (d, b, seed) not in _consts:
+        _consts[(d, b, seed)] = oracle.make_constants(d, b, seed)
+    return _consts[(d, b, seed)]
+
+
+def upload_streams(h, caches, capacity):
+    """caches: list over streams of (codes, qjl, norms) numpy arrays -> device KvqCache + tensors."""
+    S = len(caches)
+    codes = torch.zeros((S, capacity, h.b, h.d // 32), dtype=torch.int32, device="cuda")
+    qjl = torch.zeros((S, capacity, h.m // 32), dtype=torch.int32, device="cuda") if h.qjl else None
+    norms = torch.zeros((S, capacity, 2), dtype=torch.float16, device="cuda")
+    for s, (c, q, n) in enumerate(caches):
+        T = c.shape[0]
+        codes[s, :T] = to_device_u32(c)
+        if h.qjl:
+            qjl[s, :T] = to_device_u32(q)
+        norms[s, :T] = torch.from_numpy(np.ascontiguousarray(n)).cuda()
+    return kvq.make_cache(codes, qjl, norms, capacity), (codes, qjl, norms)
+
+
+def run_decode(h, q, hkv, kc, vc, seq_len, max_T, scale, want_logits=True):
+    B, hq, d = q.shape
+    out = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(kvq.kvq_decode_workspace(h, B, hq, hkv, max_T), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((B, hq, max_T), dtype=torch.float32, device="cuda") if want_logits else None
+    sl = torch.tensor(seq_len, dtype=torch.int32, device="cuda")
+    kvq.kvq_decode_attend(h, q, hkv, kc, vc, sl, max_T, scale, out, ws, logits)
+    code, bits = kvq.kvq_status(h)
+    assert code == 0, (code, bits)
+    return out.cpu().numpy(), (logits.cpu().numpy() if want_logits else None)
+
+
+def check_case(d, b, qjl, batch, hq, hkv, seq_len, capacity, scale, qdtype=torch.bfloat16, seed=3):
+    k = constants(d, b, seed)
+    G = hq // hkv
+    max_T = max(seq_len)
+    kcs, vcs, kst, vst = [], [], [], []
+    for bi in range(batch):
+        for hk in range(hkv):
+            T = seq_len[bi]
+            K = wl.llama_keys(1, T, d, seed=1000 + bi * 31 + hk)[0].double().numpy()
+            V = wl.llama_values(1, T, d, seed=2000 + bi * 31 + hk)[0].double().numpy()
+            c, q, n, st = oracle_cache(k, K, qjl)
+            kcs.append((c, q, n)); kst.append(st)
+            c, q, n, st = oracle_cache(k, V, qjl)
+            vcs.append((c, q, n)); vst.append(st)
+    qv = wl.queries(batch, hq, d, seed=77, dtype=qdtype)
+    with kvq.Handle(d, b, seed, qjl=qjl) as h:
+        kc, kt = upload_streams(h, kcs, capacity)
+        vc, vt = upload_streams(h, vcs, capacity)
+        out, logits = run_decode(h, qv.cuda(), hkv, kc, vc, seq_len, max_T, scale)
+    qd = qv.double().numpy()
+    for bi in range(batch):
+        for hk in range(hkv):
+            s = bi * hkv + hk
+            lr, orf = oracle.decode_attend(k, qd[bi, hk * G:(hk + 1) * G], kst[s], vst[s], scale, qjl)
+            assert_close(out[bi, hk * G:(hk + 1) * G], orf, f"out b{bi} kvh{hk}")
+            T = seq_len[bi]
+            if T > 0:
+                assert_close(logits[bi, hk * G:(hk + 1) * G, :T], lr, f"logits b{bi} kvh{hk}")
+            assert np.all(logits[bi, hk * G:(hk + 1) * G, T:] == -np.inf)
+
+
+def test_tiny_reference_workload():
+    """One query over 4096 fp32 N(0,1) keys/values, d=128, b=2 + QJL, scale 1/sqrt(128)."""
+    c = wl.TINY
+    k = constants(c["d"], c["b"], c["handle_seed"])
+    K = wl.gaussian(c["n"], c["d"], c["data_seed"]).double().numpy()
+    V = wl.gaussian(c["n"], c["d"], c["data_seed"] + 1000).double().numpy()
+    ck, qk, nk, sk = oracle_cache(k, K, True)
+    cv, qv_, nv, sv = oracle_cache(k, V, True)
+    q = wl.gaussian(1, c["d"], 7).reshape(1, 1, c["d"])
+    with kvq.Handle(c["d"], c["b"], c["handle_seed"], qjl=True) as h:
+        kc, _kt = upload_streams(h, [(ck, qk, nk)], c["n"])
+        vc, _vt = upload_streams(h, [(cv, qv_, nv)], c["n"])
+        out, logits = run_decode(h, q.cuda(), 1, kc, vc, [c["n"]], c["n"], c["scale"])
+    lr, orf = oracle.decode_attend(k, q[0].double().numpy(), sk, sv, c["scale"], True)
+    assert_close(logits[0], lr, "logits")
+    assert_close(out[0], orf, "out")
+
+
+@pytest.mark.parametrize("d,b,qjl,batch,hq,hkv,seq_len,cap,qdt", [
+    (128, 2, True, 2, 8, 2, [1000, 777], 1100, torch.bfloat16),      # GQA 4:1, ragged contexts
+    (128, 2, True, 1, 32, 8, [600], 600, torch.bfloat16),             # Llama-3-8B heads
+    (128, 3, False, 2, 2, 2, [513, 1], 520, torch.float16),           # GQA 1:1, one-token context
+    (64, 1, True, 1, 8, 1, [300], 300, torch.float32),                # GQA 8:1
+    (64, 4, False, 2, 4, 2, [0, 257], 300, torch.bfloat16),           # an empty context
+    (256, 2, True, 1, 4, 2, [400], 512, torch.bfloat16),
+    (256, 4, False, 1, 2, 1, [129], 129, torch.bfloat16),
+])
+def test_decode_matches_oracle(d, b, qjl, batch, hq, hkv, seq_len, cap, qdt):
+    check_case(d, b, qjl, batch, hq, hkv, seq_len, cap, scale=1 / np.sqrt(d), qdtype=qdt)
+
+
+def test_long_context_split_merge():
+    """A context long enough for many splits (exact merge of the split partials)."""
+    check_case(128, 2, True, 1, 4, 1, [20000], 20000, scale=1.0 / np.sqrt(128))
+
+
+def test_decode_workload_full_size_sampled():
+    """batch 16, 32/8 heads, d 128, 131072-token contexts, b=2 + QJL, q ~ N(0,1)/sqrt(128), scale 1.
+
+    The whole cache is produced by the CUDA quantizer from the Llama-layer
+    generator; for one sampled (sequence, KV head) the GPU quantizer is checked
+    against the oracle on sampled rows and that stream is then replaced by the
+    oracle's own cache, whose decode the oracle recomputes for the 4 query heads.
+    """
+    c = wl.DECODE
+    d, T, B, hq, hkv = c["d"], c["T"], c["batch"], c["hq"], c["hkv"]
+    G = hq // hkv
+    k = constants(d, c["b"], c["handle_seed"])
+    sample = (5, 3)
+    with kvq.Handle(d, c["b"], c["handle_seed"], qjl=True) as h:
+        S = B * hkv
+        kcodes = torch.empty((S, T, h.b, d // 32), dtype=torch.int32, device="cuda")
+        vcodes = torch.empty_like(kcodes)
+        kqjl = torch.empty((S, T, d // 32), dtype=torch.int32, device="cuda")
+        vqjl = torch.empty_like(kqjl)
+        knorm = torch.empty((S, T, 2), dtype=torch.float16, device="cuda")
+        vnorm = torch.empty_like(knorm)
+        for bi in range(B):
+            K = wl.llama_keys(hkv, T, d, wl.cache_slice_seed(c["handle_seed"], bi, 0, 0), device="cuda")
+            V = wl.llama_values(hkv, T, d, wl.cache_slice_seed(c["handle_seed"], bi, 0, 1), device="cuda")
+            sl = slice(bi * hkv, (bi + 1) * hkv)
+            kvq.kvq_quantize(h, K, kcodes[sl], kqjl[sl], knorm[sl])
+            kvq.kvq_quantize(h, V, vcodes[sl], vqjl[sl], vnorm[sl])
+            if bi == sample[0]:
+                Ks = K[sample[1]].double().cpu().numpy()
+                Vs = V[sample[1]].double().cpu().numpy()
+        assert kvq.kvq_status(h)[0] == 0
+        s = sample[0] * hkv + sample[1]
+        rows = np.sort(np.random.default_rng(1).choice(T, 1024, replace=False))
+        tr = torch.from_numpy(rows).cuda()
+        compare_quantize(k, Ks[rows], to_np_u32(kcodes[s][tr]), to_np_u32(kqjl[s][tr]),
+                         to_np_f16bits(knorm[s][tr]), True)
+        ck, qk, nk, sk = oracle_cache(k, Ks, True)
+        cv, qv_, nv, sv = oracle_cache(k, Vs, True)
+        kcodes[s] = to_device_u32(ck).reshape(T, h.b, d // 32)
+        kqjl[s] = to_device_u32(qk)
+        knorm[s] = torch.from_numpy(nk).cuda()
+        vcodes[s] = to_device_u32(cv).reshape(T, h.b, d // 32)
+        vqjl[s] = to_device_u32(qv_)
+        vnorm[s] = torch.from_numpy(nv).cuda()
+        q = wl.queries(B, hq, d, c["q_seed"], device="cuda", std=c["q_std"])
+        kc = kvq.make_cache(kcodes, kqjl, knorm, T)
+        vc = kvq.make_cache(vcodes, vqjl, vnorm, T)
+        out, _ = run_decode(h, q, hkv, kc, vc, [T] * B, T, c["scale"], want_logits=False)
+    qs = q[sample[0], sample[1] * G:(sample[1] + 1) * G].double().cpu().numpy()
+    _, orf = oracle.decode_attend(k, qs, sk, sv, c["scale"], True, want_logits=False)
+    assert_close(out[sample[0], sample[1] * G:(sample[1] + 1) * G], orf, "out (sampled stream)")
+    assert np.isfinite(out).all()

@@ -1,0 +1,171 @@
+"""Parity of the CUDA quantizer (through the C ABI) with the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from calibration_free_rotated_token_b200 import _abi as kvq
+from calibration_free_rotated_token_b200 import workloads as wl
+
+from .parity import compare_quantize, to_np_f16bits, to_np_u32
+
+pytestmark = pytest.mark.gpu
+
+_consts = {}
+
+
+def constants(d, b, seed):
+    key = (d, b, seed)
+    if key not in _consts:
+        _consts[key] = oracle.make_constants(d, b, seed)
+    return _consts[key]
+
+
+def run_quantize(h, x):
+    codes, qjl, norms = kvq.alloc_packed(h, x.shape[0])
+    kvq.kvq_quantize(h, x, codes, qjl, norms)
+    code, bits = kvq.kvq_status(h)
+    assert code == 0, (code, bits, kvq.kvq_last_error())
+    return codes, qjl, norms
+
+
+@pytest.mark.parametrize("d,b", [(64, 1), (128, 2), (256, 3), (128, 4)])
+def test_constants_match_oracle(d, b):
+    with kvq.Handle(d, b, 7, qjl=True) as h:
+        signs, S, cent, thr = kvq.kvq_get_constants(h)
+    k = constants(d, b, 7)
+    np.testing.assert_array_equal(signs.numpy(), k.delta)
+    np.testing.assert_array_equal(S.numpy().view(np.uint16), k.S_half)
+    np.testing.assert_array_equal(cent.numpy(), k.centroids.astype(np.float32))
+    np.testing.assert_array_equal(thr.numpy(), k.thresholds.astype(np.float32))
+
+
+def test_tiny_reference_workload():
+    """4096 fp32 N(0,1) keys, d=128, b=2 + QJL (m=128), data seed 0, signs seed 1, S seed 2."""
+    c = wl.TINY
+    x = wl.gaussian(c["n"], c["d"], c["data_seed"])
+    with kvq.Handle(c["d"], c["b"], c["handle_seed"], qjl=True) as h:
+        codes, qjl, norms = run_quantize(h, x.cuda())
+    k = constants(c["d"], c["b"], c["handle_seed"])
+    stats = compare_quantize(k, x.double().numpy(), to_np_u32(codes), to_np_u32(qjl), to_np_f16bits(norms), True)
+    print("tiny:", stats)
+
+
+CASES = [
+    # d, b, qjl, dtype, n  (n spans several tiles and a ragged tail)
+    (128, 2, True, torch.bfloat16, 1000),
+    (128, 2, False, torch.bfloat16, 777),
+    (128, 1, True, torch.float16, 515),
+    (128, 3, True, torch.float32, 300),
+    (128, 4, False, torch.bfloat16, 640),
+    (64, 1, True, torch.bfloat16, 1000),
+    (64, 2, True, torch.float32, 333),
+    (64, 3, False, torch.float16, 257),
+    (64, 4, True, torch.bfloat16, 129),
+    (256, 1, True, torch.bfloat16, 300),
+    (256, 2, True, torch.float16, 1000),
+    (256, 3, False, torch.bfloat16, 450),
+    (256, 4, True, torch.bfloat16, 129),
+]
+
+
+@pytest.mark.parametrize("d,b,qjl,dtype,n", CASES)
+def test_quantize_matches_oracle(d, b, qjl, dtype, n):
+    x = wl.sweep_tokens(n, d, seed=100 + d + b, dtype=dtype)
+    x[3] = 0  # a zero vector
+    with kvq.Handle(d, b, 5, qjl=qjl) as h:
+        codes, qj, norms = run_quantize(h, x.cuda())
+    k = constants(d, b, 5)
+    compare_quantize(k, x.double().numpy(), to_np_u32(codes), to_np_u32(qj) if qjl else None,
+                     to_np_f16bits(norms), qjl)
+    assert (to_np_u32(codes).reshape(n, -1)[3] == 0).all()
+    assert (to_np_f16bits(norms).reshape(n, 2)[3] == 0).all()
+
+
+def test_strided_rows_and_single_vector():
+    d = 128
+    base = wl.llama_keys(1, 300, 192, seed=3)[0]  # rows of 192, use the first 128 columns
+    x = base[:, :d]
+    with kvq.Handle(d, 2, 9, qjl=True) as h:
+        codes, qjl, norms = run_quantize(h, x.cuda())
+        c1, q1, n1 = run_quantize(h, x[:1].contiguous().cuda())
+    k = constants(d, 2, 9)
+    compare_quantize(k, x.double().numpy(), to_np_u32(codes), to_np_u32(qjl), to_np_f16bits(norms), True)
+    assert np.array_equal(to_np_u32(c1), to_np_u32(codes)[:1])
+    assert np.array_equal(to_np_u32(q1), to_np_u32(qjl)[:1])
+
+
+def test_empty_input_is_a_no_op():
+    with kvq.Handle(128, 2, 1, qjl=True) as h:
+        codes, qjl, norms = kvq.alloc_packed(h, 1)
+        codes.fill_(7)
+        kvq.kvq_quantize(h, torch.empty(0, 128, device="cuda", dtype=torch.bfloat16), codes, qjl, norms)
+        assert kvq.kvq_status(h)[0] == 0
+        assert (codes == 7).all()
+
+
+def test_nonfinite_input_sets_status():
+    with kvq.Handle(128, 2, 1, qjl=True) as h:
+        x = torch.randn(256, 128, device="cuda")
+        x[17, 5] = float("nan")
+        codes, qjl, norms = kvq.alloc_packed(h, 256)
+        kvq.kvq_quantize(h, x, codes, qjl, norms)
+        code, bits = kvq.kvq_status(h)
+        assert code == kvq.KVQ_ENONFINITE and bits & kvq.STATUS_NONFINITE
+        # the status word is cleared by the read
+        kvq.kvq_quantize(h, torch.randn(256, 128, device="cuda"), codes, qjl, norms)
+        assert kvq.kvq_status(h)[0] == 0
+
+
+def test_host_side_argument_errors():
+    with kvq.Handle(128, 2, 1, qjl=True) as h:
+        codes, qjl, norms = kvq.alloc_packed(h, 16)
+        x = torch.randn(16, 128, device="cuda")
+        # misaligned x, missing qjl on a QJL handle, row stride not a multiple of 16 bytes
+        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr() + 4, 0, 16, 128, codes.data_ptr(), qjl.data_ptr(),
+                                       norms.data_ptr(), None)
+        assert code == kvq.KVQ_EINVAL
+        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr(), 0, 16, 128, codes.data_ptr(), None,
+                                       norms.data_ptr(), None)
+        assert code == kvq.KVQ_EINVAL
+        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr(), 0, 16, 130, codes.data_ptr(), qjl.data_ptr(),
+                                       norms.data_ptr(), None)
+        assert code == kvq.KVQ_EINVAL
+        with pytest.raises(kvq.KvqError):
+            kvq.kvq_quantize(h, x[:, :64], codes, qjl, norms)
+    assert kvq.load().kvq_nsn_quantize(h.ptr if False else None, None, 0, 1, 128, None, None, None, None) \
+        == kvq.KVQ_EINVAL
+
+
+def test_llama_layer_full_size_sampled():
+    """8 KV heads x 32768 tokens x 128, bf16 keys with outlier channels, b=2 + QJL; oracle on sampled rows."""
+    c = wl.LLAMA_LAYER
+    K = wl.llama_keys(c["heads"], c["tokens"], c["d"], c["k_seed"], device="cuda")
+    V = wl.llama_values(c["heads"], c["tokens"], c["d"], c["v_seed"], device="cuda")
+    k = constants(c["d"], c["b"], c["handle_seed"])
+    rng = np.random.default_rng(0)
+    with kvq.Handle(c["d"], c["b"], c["handle_seed"], qjl=True) as h:
+        for X in (K, V):
+            X2 = X.reshape(-1, c["d"])
+            codes, qjl, norms = run_quantize(h, X2)
+            idx = np.sort(rng.choice(X2.shape[0], 2048, replace=False))
+            ti = torch.from_numpy(idx).cuda()
+            compare_quantize(k, X2[ti].double().cpu().numpy(), to_np_u32(codes[ti]), to_np_u32(qjl[ti]),
+                             to_np_f16bits(norms[ti]), True)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+@pytest.mark.parametrize("qjl", [True, False])
+def test_sweep_full_size_sampled(d, b, qjl):
+    """1,048,576 bf16 N(0,1) vectors with 1% of tokens x10; oracle on 256 sampled rows."""
+    n = wl.SWEEP["n"]
+    x = wl.sweep_tokens(n, d, seed=wl.SWEEP["seed"] + d, device="cuda")
+    k = constants(d, b, wl.SWEEP["handle_seed"])
+    with kvq.Handle(d, b, wl.SWEEP["handle_seed"], qjl=qjl) as h:
+        codes, qj, norms = run_quantize(h, x)
+    idx = np.sort(np.random.default_rng(d * 10 + b).choice(n, 256, replace=False))
+    idx[-1] = n - 1
+    ti = torch.from_numpy(idx).cuda()
+    compare_quantize(k, x[ti].double().cpu().numpy(), to_np_u32(codes[ti]), to_np_u32(qj[ti]) if qjl else None,
+                     to_np_f16bits(norms[ti]), qjl)
