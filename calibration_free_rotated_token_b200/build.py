@@ -2,7 +2,8 @@
 
 Compiles every translation unit of ``csrc/`` with nvcc for
 ``-gencode arch=compute_100a,code=sm_100a`` in parallel (the quantize kernels
-once per (d, b) pair from ``quantize_inst.cu``) and links them into
+once per (d, b) pair from ``quantize_inst.cu``), recompiling only objects
+whose source, shared headers or flags changed, and links them into
 ``calibration_free_rotated_token_b200/libkvq.so`` with the CUDA runtime
 linked statically.  Object files go to ``_build/`` at the repository root.
 
@@ -47,14 +48,30 @@ def _sources():
     return jobs
 
 
-def _fingerprint() -> str:
+def _headers_digest() -> bytes:
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
-        with open(os.path.join(CSRC, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        if name.endswith((".h", ".cuh")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + f.read())
     with open(os.path.join(ROOT, "include", "kvq.h"), "rb") as f:
         h.update(f.read())
     h.update(" ".join(ARCH + FLAGS).encode())
+    return h.digest()
+
+
+def _object_key(src: str, extra) -> str:
+    h = hashlib.sha256(_headers_digest())
+    with open(os.path.join(CSRC, src), "rb") as f:
+        h.update(f.read())
+    h.update(" ".join(extra).encode())
+    return h.hexdigest()
+
+
+def _fingerprint() -> str:
+    h = hashlib.sha256()
+    for obj, src, extra in _sources():
+        h.update(_object_key(src, extra).encode())
     return h.hexdigest()
 
 
@@ -71,12 +88,18 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -
     def compile_one(job):
         obj, src, extra = job
         out = os.path.join(BUILD, obj)
+        key = _object_key(src, extra)
+        keyfile = out + ".key"
+        if not force and os.path.exists(out) and os.path.exists(keyfile) and open(keyfile).read() == key:
+            return out
         cmd = [nvcc, *ARCH, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", out]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src} {' '.join(extra)}:\n{r.stderr}")
         if verbose and r.stderr.strip():
             print(r.stderr, file=sys.stderr)
+        with open(keyfile, "w") as f:
+            f.write(key)
         return out
 
     n = jobs or max(1, min(len(_sources()), os.cpu_count() or 4))

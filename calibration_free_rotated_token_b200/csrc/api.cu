@@ -118,6 +118,13 @@ void lloyd_max_codebook(int b, std::vector<double>* cent, std::vector<double>* t
         if (change <= 1e-15) break;
     }
     for (int k = 0; k < L; ++k) c[k] = (phi(t[k]) - phi(t[k + 1])) / (Phi(t[k + 1]) - Phi(t[k]));
+    // N(0, 1) is symmetric, so is its optimal codebook: remove the rounding
+    // asymmetry, which also makes the middle decision level exactly 0.
+    for (int k = 0; k < L / 2; ++k) {
+        const double m = 0.5 * (c[L - 1 - k] - c[k]);
+        c[k] = -m;
+        c[L - 1 - k] = m;
+    }
     cent->assign(c.begin(), c.end());
     thr->clear();
     for (int k = 1; k < L; ++k) thr->push_back(0.5 * (c[k - 1] + c[k]));

@@ -36,8 +36,9 @@ def test_constants_match_oracle(d, b):
     k = constants(d, b, 7)
     np.testing.assert_array_equal(signs.numpy(), k.delta)
     np.testing.assert_array_equal(S.numpy().view(np.uint16), k.S_half)
-    np.testing.assert_array_equal(cent.numpy(), k.centroids.astype(np.float32))
-    np.testing.assert_array_equal(thr.numpy(), k.thresholds.astype(np.float32))
+    # two independent Lloyd-Max computations: equal to fp32 rounding
+    np.testing.assert_allclose(cent.numpy(), k.centroids, rtol=2.0 ** -23, atol=1e-12)
+    np.testing.assert_allclose(thr.numpy(), k.thresholds, rtol=2.0 ** -23, atol=1e-12)
 
 
 def test_tiny_reference_workload():
@@ -131,7 +132,7 @@ def test_host_side_argument_errors():
         code = kvq.load().kvq_quantize(h.ptr, x.data_ptr(), 0, 16, 130, codes.data_ptr(), qjl.data_ptr(),
                                        norms.data_ptr(), None)
         assert code == kvq.KVQ_EINVAL
-        with pytest.raises(kvq.KvqError):
+        with pytest.raises(ValueError):
             kvq.kvq_quantize(h, x[:, :64], codes, qjl, norms)
     assert kvq.load().kvq_nsn_quantize(h.ptr if False else None, None, 0, 1, 128, None, None, None, None) \
         == kvq.KVQ_EINVAL
