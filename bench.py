@@ -45,6 +45,12 @@ def parse():
     ap.add_argument("--no-nsn", action="store_true", help="skip the NSN front-end measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-vectors", type=int, default=163840, help="vectors in the CPU oracle sample")
+    ap.add_argument("--only", choices=("quantize", "decode", "nsn"), default=None,
+                    help="run one part only (for profiler captures); prints that part's result")
+    ap.add_argument("--decode-T", type=int, default=None,
+                    help="context length of the decode measurement (default: the workload's 131072)")
+    ap.add_argument("--soak", type=float, default=1.5,
+                    help="seconds of untimed steps under the clock sampler before the timed region")
     return ap.parse_args()
 
 
@@ -216,7 +222,16 @@ def bench_quantize(args, dist):
     code, bits = kvq.kvq_status(h)
     if code != 0:
         raise RuntimeError(f"quantize status {code} bits {bits}")
+    # The K-step region lasts milliseconds, shorter than the sampler's period:
+    # the sampler runs over an untimed soak of the same step and the region.
     with Clocks(torch.cuda.current_device()) as clk:
+        t_end = time.time() + args.soak
+        i = 0
+        while time.time() < t_end:
+            step(i)
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
         ms = timed(dist, lambda i: step(i, record=True), args.steps, stream)
     launch_ms = []
     for a, bq, cq in launch_ev:
@@ -273,7 +288,7 @@ def bench_decode(args, dist):
     from calibration_free_rotated_token_b200 import workloads as wl
 
     c = wl.DECODE
-    B, hq, hkv, d, T = c["batch"], c["hq"], c["hkv"], c["d"], c["T"]
+    B, hq, hkv, d, T = c["batch"], c["hq"], c["hkv"], c["d"], (args.decode_T or c["T"])
     h = kvq.Handle(d, c["b"], c["handle_seed"], qjl=True)
     S = B * hkv
     kc = torch.empty((S, T, h.b, d // 32), dtype=torch.int32, device="cuda")
@@ -314,7 +329,7 @@ def bench_decode(args, dist):
     h.close()
     return {"metric": "packed-cache decode-attn GB/s", "value": round(dist.world * gbs, 1), "unit": "GB/s",
             "frac_of_hbm": round(gbs / hbm, 4), "ms_per_step": ms / steps, "steps": steps,
-            "workload": "batch 16, 32 query / 8 KV heads, d 128, 131072-token contexts, b=2 + QJL, one bf16 query token",
+            "workload": f"batch 16, 32 query / 8 KV heads, d 128, {T}-token contexts, b=2 + QJL, one bf16 query token",
             "cache_bytes_per_step": cache_bytes, "launches_per_step": 3,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "traffic": traffic_record("decode_split"),
@@ -379,6 +394,14 @@ def cpu_baseline(sample, n_vectors: int):
 def run_ours(args):
     dist = Dist(args.gpus)
     torch.cuda.set_device(dist.local)
+    if args.only:
+        fn = {"quantize": bench_quantize, "decode": bench_decode, "nsn": bench_nsn}[args.only]
+        r = fn(args, dist)
+        r.pop("sample_input", None)
+        if dist.rank == 0:
+            print(json.dumps({"only": args.only, **r}), flush=True)
+        dist.close()
+        return
     q = bench_quantize(args, dist)
     extra = {}
     if not args.no_decode:

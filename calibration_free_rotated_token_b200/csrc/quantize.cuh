@@ -62,11 +62,16 @@ struct QCfg {
 };
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+__device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
-// Load this thread's row (D <= 128) from a swizzled stage, applying the
-// Rademacher signs when SIGN (XOR of the element sign bits).
+// Collect the sign bit of `x` as the new low bit of w (shifting w up by one).
+__device__ __forceinline__ uint32_t push_sign(uint32_t w, float x) { return __funnelshift_l(f2u(x), w, 1); }
+
+// Load this thread's row (D <= 128) from a swizzled stage as coordinate pairs
+// v[k] = (x_2k, x_2k+1), applying the Rademacher signs when SIGN (XOR of the
+// element sign bits).
 template <int D, int DT, bool SIGN>
-__device__ __forceinline__ void load_row(const uint8_t* sp, int r, float (&v)[D], const uint32_t* psign) {
+__device__ __forceinline__ void load_row(const uint8_t* sp, int r, float2 (&v)[D / 2], const uint32_t* psign) {
     constexpr int kEsz = DT == DT_F32 ? 4 : 2;
     constexpr int kEpc = 16 / kEsz;  // elements per 16-byte chunk
 #pragma unroll
@@ -76,23 +81,26 @@ __device__ __forceinline__ void load_row(const uint8_t* sp, int r, float (&v)[D]
             const uint4 q = *reinterpret_cast<const uint4*>(sp + box * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
             const uint32_t w[4] = {q.x, q.y, q.z, q.w};
             const int e0 = box * (128 / kEsz) + c * kEpc;
+            if (DT == DT_F32) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                if (DT == DT_F32) {
-                    const int e = e0 + k;
-                    uint32_t s = 0;
-                    if (SIGN) s = (psign[e >> 1] << ((e & 1) ? 0 : 16)) & 0x80000000u;
-                    v[e] = u2f(w[k] ^ s);
-                } else {
+                for (int k = 0; k < 2; ++k) {
+                    const int e = e0 + 2 * k;
+                    uint32_t s0 = 0, s1 = 0;
+                    if (SIGN) {
+                        s0 = psign[e >> 1] << 16;
+                        s1 = psign[e >> 1] & 0x80000000u;
+                    }
+                    v[e >> 1] = make_float2(u2f(w[2 * k] ^ (s0 & 0x80000000u)), u2f(w[2 * k + 1] ^ s1));
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
                     const int pk = e0 / 2 + k;
                     const uint32_t wd = w[k] ^ (SIGN ? psign[pk] : 0u);
                     if (DT == DT_BF16) {
-                        v[2 * pk] = u2f(wd << 16);
-                        v[2 * pk + 1] = u2f(wd & 0xFFFF0000u);
+                        v[pk] = make_float2(u2f(wd << 16), u2f(wd & 0xFFFF0000u));
                     } else {
-                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wd));
-                        v[2 * pk] = f.x;
-                        v[2 * pk + 1] = f.y;
+                        v[pk] = __half22float2(*reinterpret_cast<const __half2*>(&wd));
                     }
                 }
             }
@@ -104,9 +112,10 @@ __device__ __forceinline__ void load_row(const uint8_t* sp, int r, float (&v)[D]
 // v_j = delta_j x_j + (-1)^h delta_{j+128} x_{j+128}, j < 128 (the top
 // butterfly of the Sylvester transform), plus the full ||x||^2.
 template <int DT>
-__device__ __forceinline__ float load_row_coop(const uint8_t* sp, int r, int h, float (&v)[128],
+__device__ __forceinline__ float load_row_coop(const uint8_t* sp, int r, int h, float2 (&v)[64],
                                                const uint32_t* psign) {
-    float ss = 0.f;
+    float2 ss = make_float2(0.f, 0.f);
+    const float2 sgn = h ? make_float2(-1.f, -1.f) : make_float2(1.f, 1.f);
 #pragma unroll
     for (int box = 0; box < 2; ++box) {
 #pragma unroll
@@ -121,116 +130,185 @@ __device__ __forceinline__ float load_row_coop(const uint8_t* sp, int r, int h, 
                 const int pk = box * 32 + c * 4 + k;  // pair index within the half
                 const uint32_t xa = wa[k] ^ psign[pk];
                 const uint32_t xb = wb[k] ^ psign[pk + 64];
-                float a0, a1, b0, b1;
+                float2 a, b;
                 if (DT == DT_BF16) {
-                    a0 = u2f(xa << 16); a1 = u2f(xa & 0xFFFF0000u);
-                    b0 = u2f(xb << 16); b1 = u2f(xb & 0xFFFF0000u);
+                    a = make_float2(u2f(xa << 16), u2f(xa & 0xFFFF0000u));
+                    b = make_float2(u2f(xb << 16), u2f(xb & 0xFFFF0000u));
                 } else {
-                    const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&xa));
-                    const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&xb));
-                    a0 = fa.x; a1 = fa.y; b0 = fb.x; b1 = fb.y;
+                    a = __half22float2(*reinterpret_cast<const __half2*>(&xa));
+                    b = __half22float2(*reinterpret_cast<const __half2*>(&xb));
                 }
-                ss = fmaf(a0, a0, ss); ss = fmaf(a1, a1, ss);
-                ss = fmaf(b0, b0, ss); ss = fmaf(b1, b1, ss);
-                v[2 * pk] = h ? a0 - b0 : a0 + b0;
-                v[2 * pk + 1] = h ? a1 - b1 : a1 + b1;
+                ss = __ffma2_rn(a, a, ss);
+                ss = __ffma2_rn(b, b, ss);
+                v[pk] = __ffma2_rn(sgn, b, a);
             }
         }
     }
-    return ss;
+    return ss.x + ss.y;
 }
 
-// In-register fast Walsh-Hadamard transform (Sylvester order, unnormalised).
-template <int N>
-__device__ __forceinline__ void fwht(float (&v)[N]) {
+template <int NP>
+__device__ __forceinline__ float sumsq(const float2 (&v)[NP]) {
+    float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int h = 1; h < N; h <<= 1) {
+    for (int k = 0; k < NP; k += 2) {
+        a = __ffma2_rn(v[k], v[k], a);
+        b = __ffma2_rn(v[k + 1], v[k + 1], b);
+    }
+    a = __fadd2_rn(a, b);
+    return a.x + a.y;
+}
+
+// In-register fast Walsh-Hadamard transform (Sylvester order, unnormalised)
+// of 2*NP coordinates held as pairs: the stride-1 butterflies inside each
+// pair, the others on whole pairs with packed fp32x2 adds.
+template <int NP>
+__device__ __forceinline__ void fwht(float2 (&v)[NP]) {
+    const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-            if ((i & h) == 0) {
-                const float a = v[i], b = v[i + h];
-                v[i] = a + b;
-                v[i + h] = a - b;
+    for (int k = 0; k < NP; ++k) v[k] = make_float2(v[k].x + v[k].y, v[k].x - v[k].y);
+#pragma unroll
+    for (int hp = 1; hp < NP; hp <<= 1) {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            if ((k & hp) == 0) {
+                const float2 a = v[k], b = v[k + hp];
+                v[k] = __fadd2_rn(a, b);
+                v[k + hp] = __ffma2_rn(b, m1, a);
             }
         }
     }
 }
 
-// code = #{k : z >= t_k}; c = centroid[code].
+// Lloyd-Max cell of one coordinate z on the symmetric codebook, by sign and
+// magnitude: the sign picks the half (the middle decision level is 0), and
+// the magnitude |z| is compared with the positive decision levels
+// tau_j = t[H-1+j] (binary search, H = 2^(B-1)); mu = c[H + idx] is the
+// magnitude of the centroid.  g[p] = |z| - (level compared at search step p):
+// its sign bit is the complement of magnitude-index bit p.
 template <int B>
-__device__ __forceinline__ uint32_t lm_code(float z, const float* th, const float* cb, float& c) {
-    uint32_t code = 0;
-    float cv = cb[0];
-#pragma unroll
-    for (int k = 0; k < (1 << B) - 1; ++k) {
-        const bool ge = z >= th[k];
-        code += ge ? 1u : 0u;
-        cv = ge ? cb[k + 1] : cv;
+__device__ __forceinline__ float mag_search(float az, const float* th, const float* cb, float (&g)[B > 1 ? B - 1 : 1]) {
+    constexpr int H = 1 << (B - 1);
+    const float* tau = th + (H - 1);  // tau[j], j >= 1
+    const float* mu = cb + H;
+    if constexpr (B == 1) {
+        g[0] = 0.f;
+        return mu[0];
+    } else if constexpr (B == 2) {
+        g[0] = az - tau[1];
+        return g[0] >= 0.f ? mu[1] : mu[0];
+    } else if constexpr (B == 3) {
+        g[1] = az - tau[2];
+        const bool m1 = g[1] >= 0.f;
+        g[0] = az - (m1 ? tau[3] : tau[1]);
+        const bool m0 = g[0] >= 0.f;
+        return m1 ? (m0 ? mu[3] : mu[2]) : (m0 ? mu[1] : mu[0]);
+    } else {
+        g[2] = az - tau[4];
+        const bool m2 = g[2] >= 0.f;
+        g[1] = az - (m2 ? tau[6] : tau[2]);
+        const bool m1 = g[1] >= 0.f;
+        g[0] = az - (m2 ? (m1 ? tau[7] : tau[5]) : (m1 ? tau[3] : tau[1]));
+        const bool m0 = g[0] >= 0.f;
+        const float hi = m1 ? (m0 ? mu[7] : mu[6]) : (m0 ? mu[5] : mu[4]);
+        const float lo = m1 ? (m0 ? mu[3] : mu[2]) : (m0 ? mu[1] : mu[0]);
+        return m2 ? hi : lo;
     }
-    c = cv;
-    return code;
 }
 
-// z = v * inv; codes into bit planes; v <- r = z - c[code]; returns ||r||^2.
+// z = v * inv; Lloyd-Max codes into bit planes; v <- r = z - c[code];
+// returns ||r||^2.  Bit planes: the top plane is [z >= 0]; plane p < B-1 is
+// bit p of the code, which equals (magnitude-index bit p) XNOR (sign), so
+// every plane is assembled from sign bits with one funnel shift per
+// coordinate.  Coordinates go from high to low within each 32-bit word.
 template <int NV, int B>
-__device__ __forceinline__ float codes_and_residual(float (&v)[NV], float inv, const QuantArgs& a,
+__device__ __forceinline__ float codes_and_residual(float2 (&v)[NV / 2], float inv, const QuantArgs& a,
                                                      uint32_t (&planes)[B][NV / 32]) {
-    float rr = 0.f;
+    constexpr int NG = B > 1 ? B - 1 : 1;
+    const float2 inv2 = make_float2(inv, inv);
+    const float2 m1 = make_float2(-1.f, -1.f);
+    float2 rr = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int p = 0; p < B; ++p)
+    for (int w = 0; w < NV / 32; ++w) {
+        // four independent chains of 8 coordinates (one byte each) per plane
+        uint32_t wz[4], wg[NG][4];
 #pragma unroll
-        for (int w = 0; w < NV / 32; ++w) planes[p][w] = 0u;
+        for (int q = 0; q < 4; ++q) {
+            wz[q] = 0;
 #pragma unroll
-    for (int j = 0; j < NV; ++j) {
-        const float z = v[j] * inv;
-        float c;
-        const uint32_t code = lm_code<B>(z, a.threshold, a.centroid, c);
+            for (int p = 0; p < NG; ++p) wg[p][q] = 0;
+        }
 #pragma unroll
-        for (int p = 0; p < B; ++p) planes[p][j / 32] |= ((code >> p) & 1u) << (j % 32);
-        const float r = z - c;
-        rr = fmaf(r, r, rr);
-        v[j] = r;
+        for (int kk = 3; kk >= 0; --kk) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int k = w * 16 + q * 4 + kk;  // pair index: coordinates 2k, 2k+1
+                const float2 z = __fmul2_rn(v[k], inv2);
+                float g1[NG], g0[NG];
+                const float mu1 = mag_search<B>(fabsf(z.y), a.threshold, a.centroid, g1);
+                const float mu0 = mag_search<B>(fabsf(z.x), a.threshold, a.centroid, g0);
+                wz[q] = push_sign(push_sign(wz[q], z.y), z.x);
+                if (B > 1) {
+#pragma unroll
+                    for (int p = 0; p < NG; ++p) wg[p][q] = push_sign(push_sign(wg[p][q], g1[p]), g0[p]);
+                }
+                const float2 c = make_float2(copysignf(mu0, z.x), copysignf(mu1, z.y));
+                const float2 r = __ffma2_rn(c, m1, z);
+                rr = __ffma2_rn(r, r, rr);
+                v[k] = r;
+            }
+        }
+        const uint32_t z32 = wz[0] | (wz[1] << 8) | (wz[2] << 16) | (wz[3] << 24);
+        planes[B - 1][w] = ~z32;
+#pragma unroll
+        for (int p = 0; p < B - 1; ++p)
+            planes[p][w] = ~(z32 ^ (wg[p][0] | (wg[p][1] << 8) | (wg[p][2] << 16) | (wg[p][3] << 24)));
     }
-    return rr;
+    return rr.x + rr.y;
 }
 
-// Residual (NV coordinates, starting at coordinate `k0` of the vector) as
-// fp16 hi/lo pairs into tensor memory: A_hi at column col_hi, A_lo at col_lo
-// (two fp16 per 32-bit column, even coordinate in the low half).
-template <int NV>
-__device__ __forceinline__ void store_residual_tmem(const float (&v)[NV], uint32_t t_hi, uint32_t t_lo) {
+// Residual (2*NP coordinates) as fp16 hi/lo pairs into tensor memory: A_hi
+// from column t_hi, A_lo from t_lo (two fp16 per 32-bit column, even
+// coordinate in the low half).
+template <int NP>
+__device__ __forceinline__ void store_residual_tmem(const float2 (&v)[NP], uint32_t t_hi, uint32_t t_lo) {
+    const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
-    for (int cc = 0; cc < NV / 64; ++cc) {
+    for (int cc = 0; cc < NP / 32; ++cc) {
         uint32_t hi[32], lo[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const float r0 = v[64 * cc + 2 * i], r1 = v[64 * cc + 2 * i + 1];
-            const __half2 hh = __floats2half2_rn(r0, r1);
-            const float2 hf = __half22float2(hh);
-            const __half2 ll = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
+            const float2 r = v[32 * cc + i];
+            const __half2 hh = __float22half2_rn(r);
+            const float2 rem = __ffma2_rn(__half22float2(hh), m1, r);
+            const __half2 ll = __float22half2_rn(rem);
             hi[i] = *reinterpret_cast<const uint32_t*>(&hh);
             lo[i] = *reinterpret_cast<const uint32_t*>(&ll);
         }
         tmem_st32(t_hi + cc * 32, hi);
         tmem_st32(t_lo + cc * 32, lo);
     }
-    if (NV == 32) {
-        // not used: D >= 64
-    }
 }
 
-// Sign bits of NV accumulator columns of this thread's TMEM lane.
-template <int NV>
+// Sign bits of NV accumulator columns of this thread's TMEM lane: 32-column
+// loads, one wait per 64 columns, four independent 8-bit chains per word.
+template <int NV, int PER_WAIT = 2>
 __device__ __forceinline__ void qjl_bits_from_tmem(uint32_t taddr, uint32_t (&qw)[NV / 32]) {
 #pragma unroll
-    for (int cc = 0; cc < NV / 32; ++cc) {
-        uint32_t u[32];
-        tmem_ld32(taddr + cc * 32, u);
-        tmem_wait_ld();
-        uint32_t neg = 0;
+    for (int cc = 0; cc < NV / 32; cc += PER_WAIT) {
+        uint32_t u[PER_WAIT][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) neg |= (u[i] >> 31) << i;
-        qw[cc] = ~neg;  // bit = [u >= 0]
+        for (int h = 0; h < PER_WAIT; ++h) tmem_ld32(taddr + (cc + h) * 32, u[h]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < PER_WAIT; ++h) {
+            uint32_t b[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int i = 7; i >= 0; --i)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) b[q] = __funnelshift_l(u[h][8 * q + i], b[q], 1);
+            qw[cc + h] = ~(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24));  // bit = [u >= 0]
+        }
     }
 }
 
@@ -348,6 +426,21 @@ __global__ void __launch_bounds__(256, 1)
         }
         int64_t jlocal = 0;
         int64_t i = w;
+        // Epilogue state of the tile whose QJL MMA is in flight.
+        bool pend = false, pend_valid = false;
+        int64_t pend_vidx = 0;
+        uint32_t pend_zmask = 0, pend_parity = 0;
+        auto finish_pending = [&]() -> bool {
+            const bool okm = mbar_wait(&mmadone[w], pend_parity, a.status);
+            if (named_bar_or(bar_id, 128, !okm)) return false;
+            tc_fence_after();
+            uint32_t qw[kWpp];
+            qjl_bits_from_tmem<D, 1>(tb + lane_base + D, qw);
+            tc_fence_before();
+            if (pend_valid) store_words<kWpp>(a.qjl + pend_vidx * kWpp, qw, pend_zmask);
+            pend = false;
+            return true;
+        };
         for (;; i += 2, ++jlocal) {
             const int64_t tile = blockIdx.x + i * G;
             if (tile >= a.ntiles) break;
@@ -358,13 +451,11 @@ __global__ void __launch_bounds__(256, 1)
             const int64_t vidx = tile * kTileRows + r;
             const bool valid = vidx < a.n;
 
-            float v[D];
+            float2 v[D / 2];
             float nx = 0.f, nrm;
             if (NSN) {
                 load_row<D, DT, false>(sp, r, v, a.pair_sign);
-                float ss = 0.f;
-#pragma unroll
-                for (int j = 0; j < D; ++j) ss = fmaf(v[j], v[j], ss);
+                const float ss = sumsq(v);
                 nx = sqrtf(ss);
                 flag_norm(ss, nx, a.status);
                 const float inv = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
@@ -394,44 +485,30 @@ __global__ void __launch_bounds__(256, 1)
                 named_bar_sync(bar_id, 128);
                 if (r == 0) issue_tile(i + kStages);
                 // w = u - fp16(o), then the Rademacher signs
-                float ws = 0.f;
+                const float2 inv2 = make_float2(inv, inv);
+                const __half2* o2 = reinterpret_cast<const __half2*>(so16 + w * 128);
 #pragma unroll
-                for (int j = 0; j < D; ++j) {
-                    float wv = v[j] * inv - __half2float(so16[w * 128 + j]);
-                    const uint32_t sbit = (a.pair_sign[j >> 1] << ((j & 1) ? 0 : 16)) & 0x80000000u;
-                    wv = u2f(__float_as_uint(wv) ^ sbit);
-                    ws = fmaf(wv, wv, ws);
-                    v[j] = wv;
+                for (int k = 0; k < D / 2; ++k) {
+                    const float2 wv = __ffma2_rn(v[k], inv2, __half22float2(__hneg2(o2[k])));
+                    const uint32_t ps = a.pair_sign[k];
+                    v[k] = make_float2(u2f(f2u(wv.x) ^ (ps << 16)), u2f(f2u(wv.y) ^ (ps & 0x80000000u)));
                 }
-                nrm = sqrtf(ws);
+                nrm = sqrtf(sumsq(v));
             } else {
                 load_row<D, DT, true>(sp, r, v, a.pair_sign);
                 named_bar_sync(bar_id, 128);
                 if (r == 0) issue_tile(i + kStages);
-                float ss = 0.f;
-#pragma unroll
-                for (int j = 0; j < D; ++j) ss = fmaf(v[j], v[j], ss);
+                const float ss = sumsq(v);
                 nrm = sqrtf(ss);
                 flag_norm(ss, nrm, a.status);
             }
 
-            fwht<D>(v);
+            fwht<D / 2>(v);
             const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
             uint32_t planes[B][kWpp];
             const float rr = codes_and_residual<D, B>(v, inv, a, planes);
             const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
 
-            if (QJL) {
-                store_residual_tmem<D>(v, tb + lane_base, tb + lane_base + D / 2);
-                tmem_wait_st();
-                tc_fence_before();
-                named_bar_sync(bar_id, 128);
-                if (r == 0) {
-                    tc_fence_after();
-                    issue_qjl_mma<D, D>(tb + D, tb, tb + D / 2, smem_u32(sS));
-                    mma_commit(&mmadone[w]);
-                }
-            }
             if (valid) {
                 uint32_t* cp = a.codes + vidx * (B * kWpp);
 #pragma unroll
@@ -440,15 +517,27 @@ __global__ void __launch_bounds__(256, 1)
                 a.norms[vidx] = __halves2half2(__float2half_rn(NSN ? nx : nrm), __float2half_rn(NSN ? nrm : g));
             }
             if (QJL) {
-                const bool okm = mbar_wait(&mmadone[w], static_cast<uint32_t>(jlocal & 1), a.status);
-                if (named_bar_or(bar_id, 128, !okm)) break;
-                tc_fence_after();
-                uint32_t qw[kWpp];
-                qjl_bits_from_tmem<D>(tb + lane_base + D, qw);
+                // Software pipeline: the MMA of the previous tile ran while this
+                // tile was computed; finish its epilogue now, which also frees the
+                // A and accumulator columns for this tile.
+                if (pend && !finish_pending()) break;
+                store_residual_tmem<D / 2>(v, tb + lane_base, tb + lane_base + D / 2);
+                tmem_wait_st();
                 tc_fence_before();
-                if (valid) store_words<kWpp>(a.qjl + vidx * kWpp, qw, zmask);
+                named_bar_sync(bar_id, 128);
+                if (r == 0) {
+                    tc_fence_after();
+                    issue_qjl_mma<D, D>(tb + D, tb, tb + D / 2, smem_u32(sS));
+                    mma_commit(&mmadone[w]);
+                }
+                pend = true;
+                pend_vidx = vidx;
+                pend_valid = valid;
+                pend_zmask = zmask;
+                pend_parity = static_cast<uint32_t>(jlocal & 1);
             }
         }
+        if (QJL && pend) finish_pending();
         if (r == 0) {
             // Loads issued for tiles i, i+2, ... (< i + kStages) that were not consumed.
             for (int64_t k = i; k <= i + kStages; k += 2)
@@ -476,13 +565,13 @@ __global__ void __launch_bounds__(256, 1)
             const int64_t vidx = tile * kTileRows + r;
             const bool valid = vidx < a.n;
 
-            float v[128];
+            float2 v[64];
             const float ss = load_row_coop<DT>(sp, r, h, v, a.pair_sign);
             named_bar_sync(3, 256);
             if (tid == 0) issue_tile(i + kStages);
             const float nrm = sqrtf(ss);
             if (h == 0) flag_norm(ss, nrm, a.status);
-            fwht<128>(v);
+            fwht<64>(v);
             const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
             uint32_t planes[B][4];
             const float rr = codes_and_residual<128, B>(v, inv, a, planes);
@@ -490,7 +579,7 @@ __global__ void __launch_bounds__(256, 1)
             xch[h * 128 + r] = rr;
             if (QJL) {
                 // A_hi columns [0,128), A_lo [128,256), acc [256,512)
-                store_residual_tmem<128>(v, tmem + lane_base + h * 64, tmem + lane_base + 128 + h * 64);
+                store_residual_tmem<64>(v, tmem + lane_base + h * 64, tmem + lane_base + 128 + h * 64);
                 tmem_wait_st();
                 tc_fence_before();
             }
