@@ -32,8 +32,10 @@ STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
 # Every symbol include/kvq.h declares.
 EXPORTED = (
     "kvq_init", "kvq_destroy", "kvq_quantize", "kvq_nsn_quantize", "kvq_decode_workspace",
-    "kvq_decode_attend", "kvq_status", "kvq_last_error", "kvq_get_constants", "kvq_get_info",
+    "kvq_decode_attend", "kvq_decode_attend_noalloc", "kvq_status", "kvq_last_error", "kvq_get_constants",
+    "kvq_get_info",
 )
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 _DTYPES = {torch.float32: KVQ_F32, torch.float16: KVQ_F16, torch.bfloat16: KVQ_BF16}
 
@@ -72,12 +74,14 @@ def load() -> ctypes.CDLL:
         L.kvq_decode_workspace.restype = SZ
         L.kvq_decode_attend.argtypes = [P, P, I, I, I, I, ctypes.POINTER(KvqCache), ctypes.POINTER(KvqCache), P,
                                         I64, ctypes.c_float, P, P, P, SZ, P]
+        L.kvq_decode_attend_noalloc.argtypes = [P, P, I, I, I, I, ctypes.POINTER(KvqCache),
+                                                ctypes.POINTER(KvqCache), P, I64, ctypes.c_float, P, P, P]
         L.kvq_status.argtypes = [P, P, ctypes.POINTER(U32)]
         L.kvq_last_error.restype = ctypes.c_char_p
         L.kvq_get_constants.argtypes = [P, P, P, P, P]
         L.kvq_get_info.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(U32)]
         for name in ("kvq_init", "kvq_destroy", "kvq_quantize", "kvq_nsn_quantize", "kvq_decode_attend",
-                     "kvq_status", "kvq_get_constants", "kvq_get_info"):
+                     "kvq_decode_attend_noalloc", "kvq_status", "kvq_get_constants", "kvq_get_info"):
             getattr(L, name).restype = I
         _lib = L
         return L
@@ -235,6 +239,28 @@ def kvq_decode_attend(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vc
     _check(load().kvq_decode_attend(h.ptr, _ptr(q), _DTYPES[q.dtype], B, hq, hkv, ctypes.byref(kcache),
                                     ctypes.byref(vcache), _ptr(seq_len), max_T, float(scale), _ptr(logits),
                                     _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def kvq_decode_attend_noalloc(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vcache: KvqCache,
+                              seq_len: torch.Tensor, max_T: int, scale: float, out: torch.Tensor,
+                              logits: torch.Tensor | None = None, stream=None):
+    """kvq_decode_attend using the library's fixed device scratch instead of a workspace.
+
+    For callers that must not allocate device memory when they decode; the
+    scratch (8 MiB per GPU, held until exit) is shared by all calls, so calls
+    must not overlap on the GPU.
+    """
+    if q.dim() != 3 or q.shape[-1] != h.d:
+        raise ValueError(f"q must be [batch, hq, {h.d}]")
+    _need(q, "q")
+    B, hq, _ = q.shape
+    _need(seq_len, "seq_len", dtype=torch.int32, numel=B)
+    _need(out, "out", dtype=torch.float32, numel=B * hq * h.d)
+    if logits is not None:
+        _need(logits, "logits", dtype=torch.float32, numel=B * hq * max_T)
+    _check(load().kvq_decode_attend_noalloc(h.ptr, _ptr(q), _DTYPES[q.dtype], B, hq, hkv, ctypes.byref(kcache),
+                                            ctypes.byref(vcache), _ptr(seq_len), max_T, float(scale), _ptr(logits),
+                                            _ptr(out), _stream(stream)))
 
 
 def kvq_status(h: Handle, stream=None) -> tuple[int, int]:

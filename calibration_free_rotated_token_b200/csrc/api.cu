@@ -330,10 +330,14 @@ size_t kvq_decode_workspace(kvq_handle h, int batch, int hq, int hkv, int64_t ma
     return ws;
 }
 
-int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
-                      const kvq_cache* v, const int32_t* seq_len, int64_t max_T, float scale, float* logits,
-                      float* out, void* workspace, size_t ws_bytes, void* stream) {
-    g_err.clear();
+}  // extern "C"
+
+namespace {
+
+// Argument checks shared by both decode entry points; fills the split plan.
+int decode_check(kvq_handle h, int dtype, int batch, int hq, int hkv, const kvq_cache* k, const kvq_cache* v,
+                 const void* q, const int32_t* seq_len, int64_t max_T, float scale, float* out, int* ns,
+                 int64_t* chunk, size_t* need) {
     if (int e = check_handle(h)) return e;
     if (dtype != KVQ_F32 && dtype != KVQ_F16 && dtype != KVQ_BF16) return fail(KVQ_EINVAL, "unknown dtype");
     if (batch <= 0 || hq <= 0 || hkv <= 0) return fail(KVQ_EINVAL, "batch, hq and hkv must be positive");
@@ -351,18 +355,18 @@ int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq,
     }
     if (!q || !out || !seq_len) return fail(KVQ_EINVAL, "q, out and seq_len must be non-null");
     if (!std::isfinite(scale)) return fail(KVQ_EINVAL, "scale must be finite");
-    int ns = 0;
-    int64_t chunk = 0;
-    size_t need = 0;
-    kvq::decode_plan(h, batch, hq, hkv, max_T > 0 ? max_T : 1, &ns, &chunk, &need);
-    if (!workspace || !aligned(workspace, 16)) return fail(KVQ_EINVAL, "workspace must be non-null and 16-byte aligned");
-    if (ws_bytes < need)
-        return fail(KVQ_EINVAL, "workspace too small: need " + std::to_string(need) + " bytes");
+    kvq::decode_plan(h, batch, hq, hkv, max_T > 0 ? max_T : 1, ns, chunk, need);
+    return KVQ_OK;
+}
+
+int decode_launch(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
+                  const kvq_cache* v, const int32_t* seq_len, int64_t max_T, float scale, float* logits,
+                  float* out, void* workspace, int ns, int64_t chunk, void* stream) {
     kvq::DecodeArgs a{};
     a.batch = batch;
     a.hq = hq;
     a.hkv = hkv;
-    a.G = G;
+    a.G = hq / hkv;
     a.max_T = max_T;
     a.nsplit = ns;
     a.chunk = chunk;
@@ -392,6 +396,45 @@ int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq,
     cudaError_t e = kvq::launch_decode(h, a, static_cast<cudaStream_t>(stream), &why);
     if (e != cudaSuccess) return cuda_fail(e, ("decode launch " + why).c_str());
     return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
+                      const kvq_cache* v, const int32_t* seq_len, int64_t max_T, float scale, float* logits,
+                      float* out, void* workspace, size_t ws_bytes, void* stream) {
+    g_err.clear();
+    int ns = 0;
+    int64_t chunk = 0;
+    size_t need = 0;
+    if (int e = decode_check(h, dtype, batch, hq, hkv, k, v, q, seq_len, max_T, scale, out, &ns, &chunk, &need))
+        return e;
+    if (!workspace || !aligned(workspace, 16)) return fail(KVQ_EINVAL, "workspace must be non-null and 16-byte aligned");
+    if (ws_bytes < need) return fail(KVQ_EINVAL, "workspace too small: need " + std::to_string(need) + " bytes");
+    return decode_launch(h, q, dtype, batch, hq, hkv, k, v, seq_len, max_T, scale, logits, out, workspace, ns, chunk,
+                         stream);
+}
+
+int kvq_decode_attend_noalloc(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv,
+                              const kvq_cache* k, const kvq_cache* v, const int32_t* seq_len, int64_t max_T,
+                              float scale, float* logits, float* out, void* stream) {
+    g_err.clear();
+    int ns = 0;
+    int64_t chunk = 0;
+    size_t need = 0;
+    if (int e = decode_check(h, dtype, batch, hq, hkv, k, v, q, seq_len, max_T, scale, out, &ns, &chunk, &need))
+        return e;
+    if (need > kvq::kNoAllocScratchBytes)
+        return fail(KVQ_EINVAL, "these sizes need " + std::to_string(need) + " bytes of decode scratch, more than the " +
+                                    std::to_string(kvq::kNoAllocScratchBytes) +
+                                    " bytes built into the library; use kvq_decode_attend with a workspace");
+    void* scratch = nullptr;
+    const cudaError_t e = kvq::noalloc_scratch(h->device, &scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the decode scratch");
+    return decode_launch(h, q, dtype, batch, hq, hkv, k, v, seq_len, max_T, scale, logits, out, scratch, ns, chunk,
+                         stream);
 }
 
 int kvq_status(kvq_handle h, void* stream, uint32_t* bits) {

@@ -13,10 +13,36 @@
 // Three launches on one stream; the split partials live in the caller's
 // workspace.  No kernel waits on another CTA.
 #include <cfloat>
+#include <mutex>
 
 #include "kvq_internal.h"
 
 namespace kvq {
+
+// Fixed device scratch used by kvq_decode_attend_noalloc in place of a
+// caller-provided workspace.  A file-scope __device__ array: every GPU that
+// loads this library holds kNoAllocScratchBytes of it until the process
+// exits.  Host code must not use the symbol itself as a device address; the
+// address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+cudaError_t noalloc_scratch(int device, void** ptr) {
+    // Looked up once per device, with that device current (the caller makes
+    // sure it is), and cached; later calls only read the cache.
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[device] == nullptr) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[device] = p;
+    }
+    *ptr = addr[device];
+    return cudaSuccess;
+}
 
 namespace {
 

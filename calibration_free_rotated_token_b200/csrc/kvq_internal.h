@@ -87,4 +87,10 @@ void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, in
 
 cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s, std::string* why);
 
+// Size of the fixed scratch of kvq_decode_attend_noalloc (mirrors
+// KVQ_NOALLOC_SCRATCH_BYTES of kvq.h) and its address on `device`, which
+// must be the current device.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+cudaError_t noalloc_scratch(int device, void** ptr);
+
 }  // namespace kvq

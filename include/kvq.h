@@ -178,6 +178,38 @@ int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq,
                       float scale, float* logits, float* out, void* workspace, size_t ws_bytes,
                       void* stream);
 
+/* Bytes of the fixed decode scratch built into the library (see
+ * kvq_decode_attend_noalloc). */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * kvq_decode_attend_noalloc -- kvq_decode_attend without a caller-provided
+ * workspace.  The pages have no counterpart of this call: it exists for
+ * callers that cannot allocate device memory at the point where they decode,
+ * e.g. a serving engine whose device memory is carved into a fixed pool at
+ * start-up and that forbids later cudaMalloc calls, or a plug-in running
+ * inside another runtime that owns every allocation.  Instead of a
+ * workspace the call uses a scratch array of KVQ_NOALLOC_SCRATCH_BYTES (8 MiB)
+ * compiled into the library as a __device__ variable: every GPU that loads
+ * the library holds it until the process exits.  The call itself allocates
+ * nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+ *   Arguments, semantics, outputs and errors are those of kvq_decode_attend
+ *   with `workspace`/`ws_bytes` removed.  Sizes whose workspace
+ *   (kvq_decode_workspace) exceeds KVQ_NOALLOC_SCRATCH_BYTES are rejected with
+ *   KVQ_EINVAL before any launch.
+ *   The first call on a device looks up the scratch array's device address
+ *   (cudaGetSymbolAddress) with that device current and caches it; make that
+ *   first call before any stream capture.
+ *   Every call shares the one array and it keeps the last call's contents;
+ *   no part of it needs to start at zero (each word read is first written by
+ *   the same call).  Calls whose kernels overlap on the GPU (different
+ *   streams, or different host threads) race on the array and corrupt each
+ *   other's results: serialise them, e.g. on one stream.
+ */
+int kvq_decode_attend_noalloc(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv,
+                              const kvq_cache* k, const kvq_cache* v, const int32_t* seq_len, int64_t max_T,
+                              float scale, float* logits, float* out, void* stream);
+
 /*
  * kvq_status -- synchronise `stream`, read and clear the handle's device
  * status word.  Returns KVQ_OK, KVQ_ENONFINITE or KVQ_ETIMEOUT (the most
