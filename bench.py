@@ -198,8 +198,8 @@ def bench_quantize(args, dist):
         V = wl.llama_values(H, T, d, c["v_seed"] + 100 * i + 1000 * dist.rank, device="cuda").reshape(-1, d)
         copies.append((K, V))
     n = H * T
-    outK = kvq.alloc_packed(h, n)
-    outV = kvq.alloc_packed(h, n)
+    outK = kvq.alloc_packed(h, n)                                  # keys: one record per token
+    outV = kvq.alloc_packed(h, n, layout=kvq.KVQ_LAYOUT_BLOCK32)    # values: blocks of 32 tokens
     stream = torch.cuda.current_stream()
     launch_ev = []
 
@@ -210,12 +210,12 @@ def bench_quantize(args, dist):
             a.record(stream)
             kvq.kvq_quantize(h, K, *outK, stream=stream)
             bq.record(stream)
-            kvq.kvq_quantize(h, V, *outV, stream=stream)
+            kvq.kvq_quantize(h, V, *outV, stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
             cq.record(stream)
             launch_ev.append((a, bq, cq))
         else:
             kvq.kvq_quantize(h, K, *outK, stream=stream)
-            kvq.kvq_quantize(h, V, *outV, stream=stream)
+            kvq.kvq_quantize(h, V, *outV, stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
 
     for i in range(args.warmup):
         step(i)
@@ -264,7 +264,7 @@ def bench_quantize(args, dist):
         Kd.copy_(Kh, non_blocking=True)
         Vd.copy_(Vh, non_blocking=True)
         kvq.kvq_quantize(h, Kd, *outK, stream=stream)
-        kvq.kvq_quantize(h, Vd, *outV, stream=stream)
+        kvq.kvq_quantize(h, Vd, *outV, stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
         for ho, do in zip(host_out, (outK, outV)):
             for x, y in zip(ho, do):
                 x.copy_(y, non_blocking=True)
@@ -292,9 +292,9 @@ def bench_decode(args, dist):
     h = kvq.Handle(d, c["b"], c["handle_seed"], qjl=True)
     S = B * hkv
     kc = torch.empty((S, T, h.b, d // 32), dtype=torch.int32, device="cuda")
-    vc = torch.empty_like(kc)
+    vc = torch.empty((S, T // 32, h.b, d), dtype=torch.int32, device="cuda")
     kq = torch.empty((S, T, d // 32), dtype=torch.int32, device="cuda")
-    vq = torch.empty_like(kq)
+    vq = torch.empty((S, T // 32, d), dtype=torch.int32, device="cuda")
     kn = torch.empty((S, T, 2), dtype=torch.float16, device="cuda")
     vn = torch.empty_like(kn)
     for bi in range(B):
@@ -303,14 +303,16 @@ def bench_decode(args, dist):
         kvq.kvq_quantize(h, K, kc[sl], kq[sl], kn[sl])
         del K
         V = wl.llama_values(hkv, T, d, wl.cache_slice_seed(c["handle_seed"], bi, dist.rank, 1), device="cuda")
-        kvq.kvq_quantize(h, V, vc[sl], vq[sl], vn[sl])
+        for hk in range(hkv):
+            s_ = bi * hkv + hk
+            kvq.kvq_quantize(h, V[hk], vc[s_], vq[s_], vn[s_], layout=kvq.KVQ_LAYOUT_BLOCK32)
         del V
     q = wl.queries(B, hq, d, c["q_seed"], device="cuda", std=c["q_std"])
     out = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
     ws = torch.empty(kvq.kvq_decode_workspace(h, B, hq, hkv, T), dtype=torch.uint8, device="cuda")
     seq = torch.full((B,), T, dtype=torch.int32, device="cuda")
-    kcache = kvq.make_cache(kc, kq, kn, T)
-    vcache = kvq.make_cache(vc, vq, vn, T)
+    kcache = kvq.make_cache(kc, kq, kn, T, kvq.KVQ_LAYOUT_TOKEN)
+    vcache = kvq.make_cache(vc, vq, vn, T, kvq.KVQ_LAYOUT_BLOCK32)
     stream = torch.cuda.current_stream()
 
     def step(i):
@@ -420,6 +422,7 @@ def run_ours(args):
             "config": {"workload": "llama3-8b-layer KV quantize: 8 KV heads x 32768 tokens x d128, bf16 K and V, "
                                    "2-bit Lloyd-Max + 1-bit QJL (m=128)",
                        "token": "one position of the layer = 8 heads x (K + V) = 16 vectors",
+                       "layouts": "K one record per token, V bit planes in blocks of 32 tokens (what decode reads)",
                        "vectors_per_step": q["vectors_per_step"],
                        "l2": "4 rotating input copies per rank (4 x 134 MB > 126 MB L2)",
                        "parallelism": f"dp{dist.world} (independent layers per rank, no collective)"},

@@ -27,6 +27,7 @@ KVQ_ENONFINITE = -5
 KVQ_ETIMEOUT = -6
 KVQ_QJL = 1
 KVQ_F32, KVQ_F16, KVQ_BF16 = 0, 1, 2
+KVQ_LAYOUT_TOKEN, KVQ_LAYOUT_BLOCK32 = 0, 1
 STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
 
 # Every symbol include/kvq.h declares.
@@ -48,7 +49,7 @@ class KvqError(RuntimeError):
 
 class KvqCache(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("qjl", ctypes.c_void_p), ("norms", ctypes.c_void_p),
-                ("capacity", ctypes.c_int64)]
+                ("capacity", ctypes.c_int64), ("layout", ctypes.c_int32)]
 
 
 _lib = None
@@ -68,7 +69,7 @@ def load() -> ctypes.CDLL:
                                    ctypes.c_uint64, ctypes.c_size_t)
         L.kvq_init.argtypes = [ctypes.POINTER(P), I, I, U64, U32]
         L.kvq_destroy.argtypes = [P]
-        L.kvq_quantize.argtypes = [P, P, I, I64, I64, P, P, P, P]
+        L.kvq_quantize.argtypes = [P, P, I, I64, I64, I, P, P, P, P]
         L.kvq_nsn_quantize.argtypes = [P, P, I, I64, I64, P, P, P, P]
         L.kvq_decode_workspace.argtypes = [P, I, I, I, I64]
         L.kvq_decode_workspace.restype = SZ
@@ -169,20 +170,23 @@ def kvq_get_constants(h: Handle):
     return signs, S, cent, thr[: (1 << h.b) - 1]
 
 
-def packed_shapes(h: Handle, n: int):
-    """Shapes of (codes uint32, qjl uint32 or None, norms fp16) for n vectors."""
+def packed_shapes(h: Handle, n: int, layout: int = KVQ_LAYOUT_TOKEN):
+    """Shapes of (codes uint32, qjl uint32 or None, norms fp16) for n vectors in `layout`."""
+    if layout == KVQ_LAYOUT_BLOCK32:
+        nb = (n + 31) // 32
+        return (nb, h.b, h.d), ((nb, h.m) if h.qjl else None), (n, 2)
     return (n, h.b, h.d // 32), ((n, h.m // 32) if h.qjl else None), (n, 2)
 
 
-def alloc_packed(h: Handle, n: int, device="cuda"):
-    cs, qs, ns = packed_shapes(h, n)
+def alloc_packed(h: Handle, n: int, device="cuda", layout: int = KVQ_LAYOUT_TOKEN):
+    cs, qs, ns = packed_shapes(h, n, layout)
     codes = torch.empty(cs, dtype=torch.int32, device=device)
     qjl = torch.empty(qs, dtype=torch.int32, device=device) if qs else None
     norms = torch.empty(ns, dtype=torch.float16, device=device)
     return codes, qjl, norms
 
 
-def kvq_quantize(h: Handle, x: torch.Tensor, codes, qjl, norms, stream=None):
+def kvq_quantize(h: Handle, x: torch.Tensor, codes, qjl, norms, stream=None, layout: int = KVQ_LAYOUT_TOKEN):
     """x: [n, d] (any leading dims flattened), fp32/fp16/bf16, rows contiguous in the last dim."""
     if x.dim() < 2 or x.shape[-1] != h.d:
         raise ValueError(f"x must be [..., {h.d}]")
@@ -193,12 +197,13 @@ def kvq_quantize(h: Handle, x: torch.Tensor, codes, qjl, norms, stream=None):
     ld = x2.stride(0) if n > 1 else h.d
     if x.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {x.dtype}")
-    _need(codes, "codes", numel=n * h.b * h.d // 32)
+    rows = n if layout == KVQ_LAYOUT_TOKEN else 32 * ((n + 31) // 32)
+    _need(codes, "codes", numel=rows * h.b * h.d // 32)
     _need(norms, "norms", dtype=torch.float16, numel=2 * n)
     if h.qjl:
-        _need(qjl, "qjl", numel=n * h.m // 32)
-    _check(load().kvq_quantize(h.ptr, _ptr(x2), _DTYPES[x.dtype], n, ld, _ptr(codes), _ptr(qjl) if h.qjl else None,
-                               _ptr(norms), _stream(stream)))
+        _need(qjl, "qjl", numel=rows * h.m // 32)
+    _check(load().kvq_quantize(h.ptr, _ptr(x2), _DTYPES[x.dtype], n, ld, layout, _ptr(codes),
+                               _ptr(qjl) if h.qjl else None, _ptr(norms), _stream(stream)))
 
 
 def kvq_nsn_quantize(h: Handle, x: torch.Tensor, codes, norms, block_mean, stream=None):
@@ -218,8 +223,10 @@ def kvq_decode_workspace(h: Handle, batch: int, hq: int, hkv: int, max_T: int) -
     return int(load().kvq_decode_workspace(h.ptr, batch, hq, hkv, max_T))
 
 
-def make_cache(codes, qjl, norms, capacity: int) -> KvqCache:
-    return KvqCache(codes.data_ptr(), qjl.data_ptr() if qjl is not None else None, norms.data_ptr(), capacity)
+def make_cache(codes, qjl, norms, capacity: int, layout: int = KVQ_LAYOUT_TOKEN) -> KvqCache:
+    """Cache descriptor; keys use KVQ_LAYOUT_TOKEN, values KVQ_LAYOUT_BLOCK32."""
+    return KvqCache(codes.data_ptr(), qjl.data_ptr() if qjl is not None else None, norms.data_ptr(), capacity,
+                    layout)
 
 
 def kvq_decode_attend(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vcache: KvqCache,

@@ -183,10 +183,11 @@ void fill_common(const kvq_ctx* h, float* cent, float* thr, uint32_t* ps) {
     std::memcpy(ps, h->pair_sign, sizeof(h->pair_sign));
 }
 
-int quantize_common(kvq_handle h, const void* x, int dtype, int64_t rows, int64_t ld, uint32_t* codes,
+int quantize_common(kvq_handle h, const void* x, int dtype, int64_t rows, int64_t ld, int layout, uint32_t* codes,
                     uint32_t* qjl, uint16_t* norms, uint16_t* block_mean, bool nsn, void* stream) {
     if (int e = check_handle(h)) return e;
     if (dtype != KVQ_F32 && dtype != KVQ_F16 && dtype != KVQ_BF16) return fail(KVQ_EINVAL, "unknown dtype");
+    if (layout != KVQ_LAYOUT_TOKEN && layout != KVQ_LAYOUT_BLOCK32) return fail(KVQ_EINVAL, "unknown layout");
     if (rows < 0) return fail(KVQ_EINVAL, "negative vector count");
     if (rows == 0) return KVQ_OK;
     if (rows > (int64_t(1) << 31) - 128) return fail(KVQ_EINVAL, "more than 2^31 - 128 vectors in one call");
@@ -206,6 +207,7 @@ int quantize_common(kvq_handle h, const void* x, int dtype, int64_t rows, int64_
     if (int e = make_row_map(&map, x, dtype, rows, h->d, ld)) return e;
     kvq::QuantArgs a{};
     a.n = rows;
+    a.layout = layout;
     a.ntiles = (rows + kvq::kTileRows - 1) / kvq::kTileRows;
     a.codes = codes;
     a.qjl = nsn ? nullptr : qjl;
@@ -302,10 +304,10 @@ int kvq_get_constants(kvq_handle h, int8_t* signs, uint16_t* S, float* centroids
     return KVQ_OK;
 }
 
-int kvq_quantize(kvq_handle h, const void* x, int dtype, int64_t n, int64_t ld, uint32_t* codes, uint32_t* qjl,
-                 uint16_t* norms, void* stream) {
+int kvq_quantize(kvq_handle h, const void* x, int dtype, int64_t n, int64_t ld, int layout, uint32_t* codes,
+                 uint32_t* qjl, uint16_t* norms, void* stream) {
     g_err.clear();
-    return quantize_common(h, x, dtype, n, ld, codes, qjl, norms, nullptr, false, stream);
+    return quantize_common(h, x, dtype, n, ld, layout, codes, qjl, norms, nullptr, false, stream);
 }
 
 int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, uint32_t* codes,
@@ -318,7 +320,8 @@ int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, in
     if (h->d > 128) return fail(KVQ_EUNSUPPORTED, "the NSN front end is built for d <= 128");
     if (n_heads * n_tok == 0) return KVQ_OK;
     if (!block_mean || !aligned(block_mean, 2)) return fail(KVQ_EINVAL, "block_mean must be non-null");
-    return quantize_common(h, x, dtype, n_heads * n_tok, h->d, codes, nullptr, norms, block_mean, true, stream);
+    return quantize_common(h, x, dtype, n_heads * n_tok, h->d, KVQ_LAYOUT_TOKEN, codes, nullptr, norms, block_mean,
+                           true, stream);
 }
 
 size_t kvq_decode_workspace(kvq_handle h, int batch, int hq, int hkv, int64_t max_T) {
@@ -353,6 +356,9 @@ int decode_check(kvq_handle h, int dtype, int batch, int hq, int hkv, const kvq_
         if (has_qjl && (!c->qjl || !aligned(c->qjl, 4))) return fail(KVQ_EINVAL, "cache qjl must be non-null");
         if (c->capacity < max_T) return fail(KVQ_EINVAL, "cache capacity is smaller than max_T");
     }
+    if (k->layout != KVQ_LAYOUT_TOKEN) return fail(KVQ_EINVAL, "the key cache must use KVQ_LAYOUT_TOKEN");
+    if (v->layout != KVQ_LAYOUT_BLOCK32 || v->capacity % 32 != 0)
+        return fail(KVQ_EINVAL, "the value cache must use KVQ_LAYOUT_BLOCK32 with a capacity that is a multiple of 32");
     if (!q || !out || !seq_len) return fail(KVQ_EINVAL, "q, out and seq_len must be non-null");
     if (!std::isfinite(scale)) return fail(KVQ_EINVAL, "scale must be finite");
     kvq::decode_plan(h, batch, hq, hkv, max_T > 0 ? max_T : 1, ns, chunk, need);

@@ -120,8 +120,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     __shared__ float spq[G][QJL ? M : 1];
     __shared__ float scb[1 << B];
     __shared__ float sw[G][TT];                  // softmax weights of the tile
-    __shared__ uint32_t svc[TT][KW];             // value codes of the tile
-    __shared__ uint32_t svq[TT][QJL ? QW : 1];
+    __shared__ uint32_t svc[TT / 32][B][D];      // value code planes of the tile (block-32 layout)
+    __shared__ uint32_t svq[TT / 32][QJL ? M : 1];
     __shared__ float svn[TT], svg[TT];
     __shared__ float sred[G][kDecThreads / 32];
     __shared__ float smax[G], salpha[G], ssum[G];
@@ -150,8 +150,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     const uint32_t* kc = a.kcodes + stream * a.kcap * KW;
     const uint32_t* kq = QJL ? a.kqjl + stream * a.kcap * QW : nullptr;
     const __half2* kn = a.knorms + stream * a.kcap;
-    const uint32_t* vc = a.vcodes + stream * a.vcap * KW;
-    const uint32_t* vq = QJL ? a.vqjl + stream * a.vcap * QW : nullptr;
+    // values: block-32 layout, capacity a multiple of 32
+    const uint32_t* vc = a.vcodes + stream * (a.vcap / 32) * B * D;
+    const uint32_t* vq = QJL ? a.vqjl + stream * (a.vcap / 32) * M : nullptr;
     const __half2* vn = a.vnorms + stream * a.vcap;
     const float kappa = kSqrtHalfPi / M;
 
@@ -195,13 +196,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 #pragma unroll
             for (int g = 0; g < G; ++g) a.logits[(qh0 + g) * a.max_T + t] = l[g];
         }
-        // stage the value records of this tile
-        if (mine && t < t1) {
-#pragma unroll
-            for (int w = 0; w < KW; ++w) svc[tid][w] = vc[t * KW + w];
+        // stage the value bit planes (blocks of 32 tokens) and norms of this tile
+        {
+            const int64_t blk0 = tb / 32;
+            const int nblk = static_cast<int>(min(static_cast<int64_t>(TT / 32), (t1 - tb + 31) / 32 > 0 ? (t1 - tb + 31) / 32 : 0));
+            for (int e = tid; e < nblk * B * D; e += kDecThreads)
+                (&svc[0][0][0])[e] = vc[blk0 * B * D + e];
             if (QJL)
-#pragma unroll
-                for (int w = 0; w < QW; ++w) svq[tid][w] = vq[t * QW + w];
+                for (int e = tid; e < nblk * M; e += kDecThreads) (&svq[0][0])[e] = vq[blk0 * M + e];
+        }
+        if (mine && t < t1) {
             const float2 nv = __half22float2(vn[t]);
             svn[tid] = nv.x;
             svg[tid] = nv.y;
@@ -257,7 +261,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 #pragma unroll
                 for (int g = 0; g < G; ++g) acc[g] = 0.f;
                 for (int tt = 0; tt < ntok; ++tt) {
-                    const float c = scb[code_at<B>(svc[tt], WP, j)] * svn[tt];
+                    int code = 0;
+#pragma unroll
+                    for (int p = 0; p < B; ++p) code |= static_cast<int>((svc[tt >> 5][p][j] >> (tt & 31)) & 1u) << p;
+                    const float c = scb[code] * svn[tt];
 #pragma unroll
                     for (int g = 0; g < G; ++g) acc[g] = fmaf(sw[g][tt], c, acc[g]);
                 }
@@ -272,7 +279,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 #pragma unroll
                 for (int g = 0; g < G; ++g) acc[g] = 0.f;
                 for (int tt = 0; tt < ntok; ++tt) {
-                    const float s = ((svq[tt][i >> 5] >> (i & 31)) & 1u) ? 1.f : -1.f;
+                    const float s = ((svq[tt >> 5][i] >> (tt & 31)) & 1u) ? 1.f : -1.f;
                     const float c = s * svn[tt] * svg[tt];
 #pragma unroll
                     for (int g = 0; g < G; ++g) acc[g] = fmaf(sw[g][tt], c, acc[g]);

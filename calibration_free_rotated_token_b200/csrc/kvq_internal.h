@@ -37,6 +37,7 @@ constexpr int kMaxLevels = 16;
 // value as a __grid_constant__ parameter (lives in the constant bank).
 struct QuantArgs {
     int64_t n;                        // vectors (rows)
+    int layout;                       // 0: one record per vector, 1: blocks of 32 vectors transposed
     int64_t ntiles;
     uint32_t* codes;                  // [n][b][d/32]
     uint32_t* qjl;                    // [n][d/32] or null

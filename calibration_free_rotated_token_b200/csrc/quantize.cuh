@@ -329,6 +329,34 @@ __device__ __forceinline__ void issue_qjl_mma(uint32_t acc, uint32_t a_hi, uint3
     }
 }
 
+// 32 x 32 bit transpose across the warp: lane i enters with row i (bit j =
+// column j) and leaves with column i (bit j = row j).  Five stages of a
+// shuffle exchanging the off-diagonal sub-blocks.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const uint32_t m = s == 16 ? 0x0000FFFFu : s == 8 ? 0x00FF00FFu : s == 4 ? 0x0F0F0F0Fu : s == 2 ? 0x33333333u
+                                                                                                  : 0x55555555u;
+        const uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, s);
+        x = (lane & s) ? ((x & ~m) | ((y >> s) & m)) : ((x & m) | ((y << s) & ~m));
+    }
+    return x;
+}
+
+// Block-32 store of NW words per lane: the warp holds 32 consecutive vectors
+// (lane = vector); word w covers coordinates (or QJL rows) 32w .. 32w+31.
+// dst points at the block's word for coordinate 0; lane i writes
+// coordinate 32w + i.  Called by the whole warp.
+template <int NW>
+__device__ __forceinline__ void store_block32(uint32_t* dst, const uint32_t* words, uint32_t mask, int lane,
+                                              bool store) {
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const uint32_t t = warp_transpose32(words[w] & mask, lane);
+        if (store) dst[32 * w + lane] = t;
+    }
+}
+
 template <int NWORDS>
 __device__ __forceinline__ void store_words(uint32_t* dst, const uint32_t* src, uint32_t mask) {
     if (NWORDS % 4 == 0) {
@@ -428,7 +456,7 @@ __global__ void __launch_bounds__(256, 1)
         int64_t i = w;
         // Epilogue state of the tile whose QJL MMA is in flight.
         bool pend = false, pend_valid = false;
-        int64_t pend_vidx = 0;
+        int64_t pend_vidx = 0, pend_tile = 0;
         uint32_t pend_zmask = 0, pend_parity = 0;
         auto finish_pending = [&]() -> bool {
             const bool okm = mbar_wait(&mmadone[w], pend_parity, a.status);
@@ -437,7 +465,12 @@ __global__ void __launch_bounds__(256, 1)
             uint32_t qw[kWpp];
             qjl_bits_from_tmem<D, 1>(tb + lane_base + D, qw);
             tc_fence_before();
-            if (pend_valid) store_words<kWpp>(a.qjl + pend_vidx * kWpp, qw, pend_zmask);
+            if (a.layout == 0) {
+                if (pend_valid) store_words<kWpp>(a.qjl + pend_vidx * kWpp, qw, pend_zmask);
+            } else {
+                const int64_t blk = pend_tile * 4 + (warp & 3);
+                store_block32<kWpp>(a.qjl + blk * D, qw, pend_valid ? pend_zmask : 0u, lane, blk * 32 < a.n);
+            }
             pend = false;
             return true;
         };
@@ -509,10 +542,20 @@ __global__ void __launch_bounds__(256, 1)
             const float rr = codes_and_residual<D, B>(v, inv, a, planes);
             const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
 
-            if (valid) {
-                uint32_t* cp = a.codes + vidx * (B * kWpp);
+            if (a.layout == 0) {
+                if (valid) {
+                    uint32_t* cp = a.codes + vidx * (B * kWpp);
 #pragma unroll
-                for (int p = 0; p < B; ++p) store_words<kWpp>(cp + p * kWpp, planes[p], zmask);
+                    for (int p = 0; p < B; ++p) store_words<kWpp>(cp + p * kWpp, planes[p], zmask);
+                }
+            } else {
+                const int64_t blk = tile * 4 + (warp & 3);
+                const uint32_t m = valid ? zmask : 0u;
+#pragma unroll
+                for (int p = 0; p < B; ++p)
+                    store_block32<kWpp>(a.codes + (blk * B + p) * D, planes[p], m, lane, blk * 32 < a.n);
+            }
+            if (valid) {
                 const float g = nrm > 0.f ? sqrtf(rr) : 0.f;
                 a.norms[vidx] = __halves2half2(__float2half_rn(NSN ? nx : nrm), __float2half_rn(NSN ? nrm : g));
             }
@@ -531,6 +574,7 @@ __global__ void __launch_bounds__(256, 1)
                     mma_commit(&mmadone[w]);
                 }
                 pend = true;
+                pend_tile = tile;
                 pend_vidx = vidx;
                 pend_valid = valid;
                 pend_zmask = zmask;
@@ -589,10 +633,20 @@ __global__ void __launch_bounds__(256, 1)
                 issue_qjl_mma<256, 256>(tmem + 256, tmem, tmem + 128, smem_u32(sS));
                 mma_commit(&mmadone[0]);
             }
-            if (valid) {
-                uint32_t* cp = a.codes + vidx * (B * 8) + h * 4;
+            if (a.layout == 0) {
+                if (valid) {
+                    uint32_t* cp = a.codes + vidx * (B * 8) + h * 4;
 #pragma unroll
-                for (int p = 0; p < B; ++p) store_words<4>(cp + p * 8, planes[p], zmask);
+                    for (int p = 0; p < B; ++p) store_words<4>(cp + p * 8, planes[p], zmask);
+                }
+            } else {
+                const int64_t blk = tile * 4 + (warp & 3);
+#pragma unroll
+                for (int p = 0; p < B; ++p)
+                    store_block32<4>(a.codes + (blk * B + p) * 256 + h * 128, planes[p], valid ? zmask : 0u, lane,
+                                     blk * 32 < a.n);
+            }
+            if (valid) {
                 if (h == 0) {
                     const float g = nrm > 0.f ? sqrtf(xch[r] + xch[128 + r]) : 0.f;
                     a.norms[vidx] = __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
@@ -605,7 +659,12 @@ __global__ void __launch_bounds__(256, 1)
                 uint32_t qw[4];
                 qjl_bits_from_tmem<128>(tmem + lane_base + 256 + h * 128, qw);
                 tc_fence_before();
-                if (valid) store_words<4>(a.qjl + vidx * 8 + h * 4, qw, zmask);
+                if (a.layout == 0) {
+                    if (valid) store_words<4>(a.qjl + vidx * 8 + h * 4, qw, zmask);
+                } else {
+                    const int64_t blk = tile * 4 + (warp & 3);
+                    store_block32<4>(a.qjl + blk * 256 + h * 128, qw, valid ? zmask : 0u, lane, blk * 32 < a.n);
+                }
             }
             // xch is rewritten next tile only after this barrier
             named_bar_sync(3, 256);

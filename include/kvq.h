@@ -42,6 +42,17 @@
  *   qjl    uint32 [t][m/32]     bit i of word w = [ (S r)_{32w+i} >= 0 ];
  *   norms  fp16   [t][2]        (||x||, ||r||)  -- NSN: (||x||, ||w||).
  * Coordinates are in the rotated domain, Sylvester (natural) order.
+ *
+ * KVQ_LAYOUT_BLOCK32 stores the same bits transposed per block of 32
+ * consecutive vectors (vector t is bit t % 32 of block t / 32), the layout
+ * the decode kernel consumes for values (its value sums contract over
+ * tokens, four tokens per tensor-core register):
+ *   codes  uint32 [blk][b][d]   bit i of word (blk, p, j) = bit p of the code
+ *                               of coordinate j of vector 32*blk + i;
+ *   qjl    uint32 [blk][m]      bit i of word (blk, k) = QJL bit of row k of
+ *                               vector 32*blk + i;
+ *   norms  fp16   [t][2]        as above (one record per vector).
+ * Bits of vectors past the end of the input are 0.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -69,6 +80,10 @@ extern "C" {
 #define KVQ_F32 0
 #define KVQ_F16 1
 #define KVQ_BF16 2
+
+/* ---- packed layouts ------------------------------------------------------ */
+#define KVQ_LAYOUT_TOKEN 0    /* one record per vector (see "Packed cache layout") */
+#define KVQ_LAYOUT_BLOCK32 1  /* bit planes transposed in blocks of 32 consecutive vectors */
 
 /* Device status word bits, as returned in *bits by kvq_status. */
 #define KVQ_STATUS_NONFINITE 1u
@@ -106,14 +121,17 @@ int kvq_destroy(kvq_handle h);
  *          elements (ld >= d; ld * element size a multiple of 16 bytes;
  *          x 16-byte aligned).
  *   n      number of vectors, >= 0 (0 is a no-op).
- *   codes  device, n * b * d/32 uint32, 16-byte aligned.
- *   qjl    device, n * d/32 uint32, 16-byte aligned; must be NULL when the
- *          handle has no KVQ_QJL flag and non-NULL when it has.
+ *   layout KVQ_LAYOUT_TOKEN or KVQ_LAYOUT_BLOCK32 (codes and qjl).
+ *   codes  device, 16-byte aligned; n * b * d/32 uint32 (token layout) or
+ *          ceil(n/32) * b * d uint32 (block-32 layout).
+ *   qjl    device, 16-byte aligned, n * d/32 (token) or ceil(n/32) * d
+ *          (block-32) uint32; must be NULL when the handle has no KVQ_QJL
+ *          flag and non-NULL when it has.
  *   norms  device, n * 2 fp16 (bit patterns), 4-byte aligned.
  * fp32 input is built for d <= 128.  Non-finite inputs and norms above the
  * fp16 range set status bits; those rows' outputs are unspecified.
  */
-int kvq_quantize(kvq_handle h, const void* x, int dtype, int64_t n, int64_t ld, uint32_t* codes,
+int kvq_quantize(kvq_handle h, const void* x, int dtype, int64_t n, int64_t ld, int layout, uint32_t* codes,
                  uint32_t* qjl, uint16_t* norms, void* stream);
 
 /*
@@ -137,12 +155,14 @@ int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, in
 
 /* One packed cache (keys or values) of batch * hkv streams, each holding up
  * to `capacity` vectors in the layout above; stream (bi, hi) starts at
- * vector (bi * hkv + hi) * capacity. */
+ * vector (bi * hkv + hi) * capacity.  Keys use KVQ_LAYOUT_TOKEN, values
+ * KVQ_LAYOUT_BLOCK32 (capacity a multiple of 32). */
 typedef struct kvq_cache {
     const uint32_t* codes;  /* device, streams * capacity * b * d/32 */
     const uint32_t* qjl;    /* device, streams * capacity * d/32; NULL without KVQ_QJL */
     const uint16_t* norms;  /* device, streams * capacity * 2 fp16 */
     int64_t capacity;       /* vectors per stream, >= max_T */
+    int32_t layout;         /* KVQ_LAYOUT_TOKEN (keys) or KVQ_LAYOUT_BLOCK32 (values) */
 } kvq_cache;
 
 /* Bytes of device workspace kvq_decode_attend needs for these sizes. */

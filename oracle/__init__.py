@@ -22,6 +22,11 @@ of the quantizer), for vector t:
   (||x||, ||w||);
 * NSN only: ``block_mean[blk, j]`` (fp16), mean of block ``blk`` of 128
   tokens on channel j.
+
+Block-32 layout (values): the same bits transposed per block of 32
+consecutive vectors: ``codes[blk, p, j]`` bit i = bit p of the code of
+coordinate j of vector 32*blk + i; ``qjl[blk, k]`` bit i = QJL bit of row k of
+vector 32*blk + i; bits of vectors past the end are 0.
 """
 from __future__ import annotations
 
@@ -327,3 +332,44 @@ def unpack_bits(words: np.ndarray, m: int) -> np.ndarray:
     words = np.asarray(words, np.uint32).reshape(-1, m // 32).astype(np.uint64)
     n = words.shape[0]
     return ((words[:, :, None] >> np.arange(32, dtype=np.uint64)) & 1).reshape(n, m).astype(np.uint8)
+
+
+def pack_codes_block32(codes: np.ndarray, b: int) -> np.ndarray:
+    codes = np.asarray(codes, np.int64)
+    n, d = codes.shape
+    nb = (n + 31) // 32
+    full = np.zeros((nb * 32, d), np.int64)
+    full[:n] = codes
+    words = np.zeros((nb, b, d), np.uint32)
+    sh = np.arange(32, dtype=np.uint64)[None, :, None]
+    for p in range(b):
+        plane = ((full >> p) & 1).astype(np.uint64).reshape(nb, 32, d)
+        words[:, p, :] = (plane << sh).sum(axis=1).astype(np.uint32)
+    return words
+
+
+def unpack_codes_block32(words: np.ndarray, b: int, d: int, n: int) -> np.ndarray:
+    words = np.asarray(words, np.uint32).reshape(-1, b, d).astype(np.uint64)
+    nb = words.shape[0]
+    codes = np.zeros((nb * 32, d), np.int32)
+    sh = np.arange(32, dtype=np.uint64)[None, :, None]
+    for p in range(b):
+        plane = ((words[:, p, None, :] >> sh) & 1).reshape(nb * 32, d).astype(np.int32)
+        codes |= plane << p
+    return codes[:n]
+
+
+def pack_bits_block32(bits: np.ndarray) -> np.ndarray:
+    bits = np.asarray(bits, np.uint64)
+    n, m = bits.shape
+    nb = (n + 31) // 32
+    full = np.zeros((nb * 32, m), np.uint64)
+    full[:n] = bits
+    return (full.reshape(nb, 32, m) << np.arange(32, dtype=np.uint64)[None, :, None]).sum(axis=1).astype(np.uint32)
+
+
+def unpack_bits_block32(words: np.ndarray, m: int, n: int) -> np.ndarray:
+    words = np.asarray(words, np.uint32).reshape(-1, m).astype(np.uint64)
+    nb = words.shape[0]
+    bits = ((words[:, None, :] >> np.arange(32, dtype=np.uint64)[None, :, None]) & 1).reshape(nb * 32, m)
+    return bits[:n].astype(np.uint8)

@@ -46,13 +46,16 @@ def ulp_distance_f16(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
 
 
 def compare_quantize(k: oracle.Constants, x: np.ndarray, codes_g, qjl_g, norms_g, use_qjl: bool,
-                     ref: dict | None = None) -> dict:
-    """Checks one quantize call; returns counts (excluded coordinates, ulp cases)."""
+                     ref: dict | None = None, layout: int = 0) -> dict:
+    """Checks one quantize call (layout 0: one record per vector, 1: block-32); returns counts."""
     x = np.asarray(x, np.float64)
     n, d = x.shape
     if ref is None:
         ref = oracle.quantize(k, x, use_qjl)
-    codes = oracle.unpack_codes(codes_g.reshape(n, -1), k.b, d)
+    if layout == 0:
+        codes = oracle.unpack_codes(codes_g.reshape(n, -1), k.b, d)
+    else:
+        codes = oracle.unpack_codes_block32(codes_g, k.b, d, n)
     near = (np.abs(ref["z"][..., None] - k.thresholds[None, None, :]) < CODE_BAND).any(-1)
     near[ref["norm"] == 0] = False  # a zero vector has a defined all-zero record: compared exactly
     bad = (codes != ref["codes"]) & ~near
@@ -75,7 +78,7 @@ def compare_quantize(k: oracle.Constants, x: np.ndarray, codes_g, qjl_g, norms_g
     out = dict(excluded_coords=int(near.sum()), coords=int(near.size), norm_ulp=int((dn > 0).sum()),
                gamma_ulp=int((dg > 0).sum()))
     if use_qjl:
-        bits = oracle.unpack_bits(qjl_g.reshape(n, -1), k.m)
+        bits = oracle.unpack_bits(qjl_g.reshape(n, -1), k.m) if layout == 0 else oracle.unpack_bits_block32(qjl_g, k.m, n)
         tiny = np.abs(ref["u"]) < QJL_BAND * ref["gamma"][:, None]
         cmp = ~tiny & vec_ok[:, None]
         badb = (bits != ref["bits"]) & cmp
@@ -96,11 +99,15 @@ def assert_close(got: np.ndarray, want: np.ndarray, what: str):
     return worst
 
 
-def oracle_cache(k: oracle.Constants, x: np.ndarray, use_qjl: bool):
-    """The oracle's own packed cache of x: (codes u32, qjl u32 or None, norms fp16 bits, widened dict)."""
+def oracle_cache(k: oracle.Constants, x: np.ndarray, use_qjl: bool, layout: int = 0):
+    """The oracle's own packed cache of x: (codes u32, qjl u32 or None, norms fp16, widened dict)."""
     q = oracle.quantize(k, x, use_qjl)
-    codes = oracle.pack_codes(q["codes"], k.b)
-    qjl = oracle.pack_bits(q["bits"]) if use_qjl else None
+    if layout == 0:
+        codes = oracle.pack_codes(q["codes"], k.b)
+        qjl = oracle.pack_bits(q["bits"]) if use_qjl else None
+    else:
+        codes = oracle.pack_codes_block32(q["codes"], k.b)
+        qjl = oracle.pack_bits_block32(q["bits"]) if use_qjl else None
     nb = q["norm"].astype(np.float16)
     gb = q["gamma"].astype(np.float16)
     norms = np.stack([nb, gb], axis=1)

@@ -23,19 +23,24 @@ def constants(d, b, seed):
     return _consts[(d, b, seed)]
 
 
-def upload_streams(h, caches, capacity):
+def upload_streams(h, caches, capacity, layout):
     """caches: list over streams of (codes, qjl, norms) numpy arrays -> device KvqCache + tensors."""
     S = len(caches)
-    codes = torch.zeros((S, capacity, h.b, h.d // 32), dtype=torch.int32, device="cuda")
-    qjl = torch.zeros((S, capacity, h.m // 32), dtype=torch.int32, device="cuda") if h.qjl else None
+    if layout == 0:
+        codes = torch.zeros((S, capacity, h.b, h.d // 32), dtype=torch.int32, device="cuda")
+        qjl = torch.zeros((S, capacity, h.m // 32), dtype=torch.int32, device="cuda") if h.qjl else None
+    else:
+        codes = torch.zeros((S, capacity // 32, h.b, h.d), dtype=torch.int32, device="cuda")
+        qjl = torch.zeros((S, capacity // 32, h.m), dtype=torch.int32, device="cuda") if h.qjl else None
     norms = torch.zeros((S, capacity, 2), dtype=torch.float16, device="cuda")
     for s, (c, q, n) in enumerate(caches):
-        T = c.shape[0]
-        codes[s, :T] = to_device_u32(c)
+        T = n.shape[0]
+        rows = c.shape[0]
+        codes[s, :rows] = to_device_u32(c).reshape(codes[s, :rows].shape)
         if h.qjl:
-            qjl[s, :T] = to_device_u32(q)
+            qjl[s, :rows] = to_device_u32(q).reshape(qjl[s, :rows].shape)
         norms[s, :T] = torch.from_numpy(np.ascontiguousarray(n)).cuda()
-    return kvq.make_cache(codes, qjl, norms, capacity), (codes, qjl, norms)
+    return kvq.make_cache(codes, qjl, norms, capacity, layout), (codes, qjl, norms)
 
 
 def run_decode(h, q, hkv, kc, vc, seq_len, max_T, scale, want_logits=True):
@@ -62,12 +67,12 @@ def check_case(d, b, qjl, batch, hq, hkv, seq_len, capacity, scale, qdtype=torch
             V = wl.llama_values(1, T, d, seed=2000 + bi * 31 + hk)[0].double().numpy()
             c, q, n, st = oracle_cache(k, K, qjl)
             kcs.append((c, q, n)); kst.append(st)
-            c, q, n, st = oracle_cache(k, V, qjl)
+            c, q, n, st = oracle_cache(k, V, qjl, layout=1)
             vcs.append((c, q, n)); vst.append(st)
     qv = wl.queries(batch, hq, d, seed=77, dtype=qdtype)
     with kvq.Handle(d, b, seed, qjl=qjl) as h:
-        kc, kt = upload_streams(h, kcs, capacity)
-        vc, vt = upload_streams(h, vcs, capacity)
+        kc, kt = upload_streams(h, kcs, capacity, 0)
+        vc, vt = upload_streams(h, vcs, capacity, 1)
         out, logits = run_decode(h, qv.cuda(), hkv, kc, vc, seq_len, max_T, scale)
     qd = qv.double().numpy()
     for bi in range(batch):
@@ -88,11 +93,11 @@ def test_tiny_reference_workload():
     K = wl.gaussian(c["n"], c["d"], c["data_seed"]).double().numpy()
     V = wl.gaussian(c["n"], c["d"], c["data_seed"] + 1000).double().numpy()
     ck, qk, nk, sk = oracle_cache(k, K, True)
-    cv, qv_, nv, sv = oracle_cache(k, V, True)
+    cv, qv_, nv, sv = oracle_cache(k, V, True, layout=1)
     q = wl.gaussian(1, c["d"], 7).reshape(1, 1, c["d"])
     with kvq.Handle(c["d"], c["b"], c["handle_seed"], qjl=True) as h:
-        kc, _kt = upload_streams(h, [(ck, qk, nk)], c["n"])
-        vc, _vt = upload_streams(h, [(cv, qv_, nv)], c["n"])
+        kc, _kt = upload_streams(h, [(ck, qk, nk)], c["n"], 0)
+        vc, _vt = upload_streams(h, [(cv, qv_, nv)], c["n"], 1)
         out, logits = run_decode(h, q.cuda(), 1, kc, vc, [c["n"]], c["n"], c["scale"])
     lr, orf = oracle.decode_attend(k, q[0].double().numpy(), sk, sv, c["scale"], True)
     assert_close(logits[0], lr, "logits")
@@ -100,13 +105,13 @@ def test_tiny_reference_workload():
 
 
 @pytest.mark.parametrize("d,b,qjl,batch,hq,hkv,seq_len,cap,qdt", [
-    (128, 2, True, 2, 8, 2, [1000, 777], 1100, torch.bfloat16),      # GQA 4:1, ragged contexts
-    (128, 2, True, 1, 32, 8, [600], 600, torch.bfloat16),             # Llama-3-8B heads
-    (128, 3, False, 2, 2, 2, [513, 1], 520, torch.float16),           # GQA 1:1, one-token context
-    (64, 1, True, 1, 8, 1, [300], 300, torch.float32),                # GQA 8:1
-    (64, 4, False, 2, 4, 2, [0, 257], 300, torch.bfloat16),           # an empty context
+    (128, 2, True, 2, 8, 2, [1000, 777], 1120, torch.bfloat16),      # GQA 4:1, ragged contexts
+    (128, 2, True, 1, 32, 8, [600], 608, torch.bfloat16),             # Llama-3-8B heads
+    (128, 3, False, 2, 2, 2, [513, 1], 544, torch.float16),           # GQA 1:1, one-token context
+    (64, 1, True, 1, 8, 1, [300], 320, torch.float32),                # GQA 8:1
+    (64, 4, False, 2, 4, 2, [0, 257], 320, torch.bfloat16),           # an empty context
     (256, 2, True, 1, 4, 2, [400], 512, torch.bfloat16),
-    (256, 4, False, 1, 2, 1, [129], 129, torch.bfloat16),
+    (256, 4, False, 1, 2, 1, [129], 160, torch.bfloat16),
 ])
 def test_decode_matches_oracle(d, b, qjl, batch, hq, hkv, seq_len, cap, qdt):
     check_case(d, b, qjl, batch, hq, hkv, seq_len, cap, scale=1 / np.sqrt(d), qdtype=qdt)
@@ -133,9 +138,9 @@ def test_decode_workload_full_size_sampled():
     with kvq.Handle(d, c["b"], c["handle_seed"], qjl=True) as h:
         S = B * hkv
         kcodes = torch.empty((S, T, h.b, d // 32), dtype=torch.int32, device="cuda")
-        vcodes = torch.empty_like(kcodes)
+        vcodes = torch.empty((S, T // 32, h.b, d), dtype=torch.int32, device="cuda")
         kqjl = torch.empty((S, T, d // 32), dtype=torch.int32, device="cuda")
-        vqjl = torch.empty_like(kqjl)
+        vqjl = torch.empty((S, T // 32, d), dtype=torch.int32, device="cuda")
         knorm = torch.empty((S, T, 2), dtype=torch.float16, device="cuda")
         vnorm = torch.empty_like(knorm)
         for bi in range(B):
@@ -143,7 +148,9 @@ def test_decode_workload_full_size_sampled():
             V = wl.llama_values(hkv, T, d, wl.cache_slice_seed(c["handle_seed"], bi, 0, 1), device="cuda")
             sl = slice(bi * hkv, (bi + 1) * hkv)
             kvq.kvq_quantize(h, K, kcodes[sl], kqjl[sl], knorm[sl])
-            kvq.kvq_quantize(h, V, vcodes[sl], vqjl[sl], vnorm[sl])
+            for hk in range(hkv):
+                kvq.kvq_quantize(h, V[hk], vcodes[bi * hkv + hk], vqjl[bi * hkv + hk], vnorm[bi * hkv + hk],
+                                 layout=1)
             if bi == sample[0]:
                 Ks = K[sample[1]].double().cpu().numpy()
                 Vs = V[sample[1]].double().cpu().numpy()
@@ -154,16 +161,16 @@ def test_decode_workload_full_size_sampled():
         compare_quantize(k, Ks[rows], to_np_u32(kcodes[s][tr]), to_np_u32(kqjl[s][tr]),
                          to_np_f16bits(knorm[s][tr]), True)
         ck, qk, nk, sk = oracle_cache(k, Ks, True)
-        cv, qv_, nv, sv = oracle_cache(k, Vs, True)
+        cv, qv_, nv, sv = oracle_cache(k, Vs, True, layout=1)
         kcodes[s] = to_device_u32(ck).reshape(T, h.b, d // 32)
         kqjl[s] = to_device_u32(qk)
         knorm[s] = torch.from_numpy(nk).cuda()
-        vcodes[s] = to_device_u32(cv).reshape(T, h.b, d // 32)
+        vcodes[s] = to_device_u32(cv).reshape(T // 32, h.b, d)
         vqjl[s] = to_device_u32(qv_)
         vnorm[s] = torch.from_numpy(nv).cuda()
         q = wl.queries(B, hq, d, c["q_seed"], device="cuda", std=c["q_std"])
-        kc = kvq.make_cache(kcodes, kqjl, knorm, T)
-        vc = kvq.make_cache(vcodes, vqjl, vnorm, T)
+        kc = kvq.make_cache(kcodes, kqjl, knorm, T, 0)
+        vc = kvq.make_cache(vcodes, vqjl, vnorm, T, 1)
         out, _ = run_decode(h, q, hkv, kc, vc, [T] * B, T, c["scale"], want_logits=False)
     qs = q[sample[0], sample[1] * G:(sample[1] + 1) * G].double().cpu().numpy()
     _, orf = oracle.decode_attend(k, qs, sk, sv, c["scale"], True, want_logits=False)

@@ -21,9 +21,9 @@ def constants(d, b, seed):
     return _consts[key]
 
 
-def run_quantize(h, x):
-    codes, qjl, norms = kvq.alloc_packed(h, x.shape[0])
-    kvq.kvq_quantize(h, x, codes, qjl, norms)
+def run_quantize(h, x, layout=0):
+    codes, qjl, norms = kvq.alloc_packed(h, x.shape[0], layout=layout)
+    kvq.kvq_quantize(h, x, codes, qjl, norms, layout=layout)
     code, bits = kvq.kvq_status(h)
     assert code == 0, (code, bits, kvq.kvq_last_error())
     return codes, qjl, norms
@@ -83,6 +83,39 @@ def test_quantize_matches_oracle(d, b, qjl, dtype, n):
     assert (to_np_f16bits(norms).reshape(n, 2)[3] == 0).all()
 
 
+BLOCK_CASES = [
+    (128, 2, True, torch.bfloat16, 1000),
+    (128, 1, False, torch.float16, 70),
+    (64, 2, True, torch.float32, 333),
+    (64, 4, True, torch.bfloat16, 31),
+    (256, 2, True, torch.bfloat16, 300),
+    (256, 3, False, torch.bfloat16, 129),
+]
+
+
+@pytest.mark.parametrize("d,b,qjl,dtype,n", BLOCK_CASES)
+def test_quantize_block32_layout_matches_oracle(d, b, qjl, dtype, n):
+    x = wl.sweep_tokens(n, d, seed=200 + d + b, dtype=dtype)
+    x[min(5, n - 1)] = 0
+    with kvq.Handle(d, b, 6, qjl=qjl) as h:
+        codes, qj, norms = run_quantize(h, x.cuda(), layout=1)
+        # the same bits as the token layout
+        c0, q0, _ = run_quantize(h, x.cuda(), layout=0)
+    k = constants(d, b, 6)
+    compare_quantize(k, x.double().numpy(), to_np_u32(codes), to_np_u32(qj) if qjl else None,
+                     to_np_f16bits(norms), qjl, layout=1)
+    np.testing.assert_array_equal(oracle.unpack_codes_block32(to_np_u32(codes), b, d, n),
+                                  oracle.unpack_codes(to_np_u32(c0).reshape(n, -1), b, d))
+    if qjl:
+        np.testing.assert_array_equal(oracle.unpack_bits_block32(to_np_u32(qj), d, n),
+                                      oracle.unpack_bits(to_np_u32(q0).reshape(n, -1), d))
+    # bits of vectors past n in the last block are zero
+    tail = n % 32
+    if tail:
+        w = to_np_u32(codes)[-1]
+        assert np.all((w >> np.uint32(tail)) == 0)
+
+
 def test_strided_rows_and_single_vector():
     d = 128
     base = wl.llama_keys(1, 300, 192, seed=3)[0]  # rows of 192, use the first 128 columns
@@ -123,13 +156,16 @@ def test_host_side_argument_errors():
         codes, qjl, norms = kvq.alloc_packed(h, 16)
         x = torch.randn(16, 128, device="cuda")
         # misaligned x, missing qjl on a QJL handle, row stride not a multiple of 16 bytes
-        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr() + 4, 0, 16, 128, codes.data_ptr(), qjl.data_ptr(),
+        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr() + 4, 0, 16, 128, 0, codes.data_ptr(), qjl.data_ptr(),
                                        norms.data_ptr(), None)
         assert code == kvq.KVQ_EINVAL
-        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr(), 0, 16, 128, codes.data_ptr(), None,
+        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr(), 0, 16, 128, 0, codes.data_ptr(), None,
                                        norms.data_ptr(), None)
         assert code == kvq.KVQ_EINVAL
-        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr(), 0, 16, 130, codes.data_ptr(), qjl.data_ptr(),
+        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr(), 0, 16, 130, 0, codes.data_ptr(), qjl.data_ptr(),
+                                       norms.data_ptr(), None)
+        assert code == kvq.KVQ_EINVAL
+        code = kvq.load().kvq_quantize(h.ptr, x.data_ptr(), 0, 16, 128, 2, codes.data_ptr(), qjl.data_ptr(),
                                        norms.data_ptr(), None)
         assert code == kvq.KVQ_EINVAL
         with pytest.raises(ValueError):
@@ -146,13 +182,20 @@ def test_llama_layer_full_size_sampled():
     k = constants(c["d"], c["b"], c["handle_seed"])
     rng = np.random.default_rng(0)
     with kvq.Handle(c["d"], c["b"], c["handle_seed"], qjl=True) as h:
-        for X in (K, V):
+        for X, layout in ((K, 0), (V, 1)):
             X2 = X.reshape(-1, c["d"])
-            codes, qjl, norms = run_quantize(h, X2)
-            idx = np.sort(rng.choice(X2.shape[0], 2048, replace=False))
-            ti = torch.from_numpy(idx).cuda()
-            compare_quantize(k, X2[ti].double().cpu().numpy(), to_np_u32(codes[ti]), to_np_u32(qjl[ti]),
-                             to_np_f16bits(norms[ti]), True)
+            codes, qjl, norms = run_quantize(h, X2, layout=layout)
+            if layout == 0:
+                idx = np.sort(rng.choice(X2.shape[0], 2048, replace=False))
+                ti = torch.from_numpy(idx).cuda()
+                compare_quantize(k, X2[ti].double().cpu().numpy(), to_np_u32(codes[ti]), to_np_u32(qjl[ti]),
+                                 to_np_f16bits(norms[ti]), True)
+            else:
+                # sampled whole blocks of 32 vectors
+                for blk in np.sort(rng.choice(X2.shape[0] // 32, 64, replace=False)):
+                    sl = slice(blk * 32, blk * 32 + 32)
+                    compare_quantize(k, X2[sl].double().cpu().numpy(), to_np_u32(codes[blk:blk + 1]),
+                                     to_np_u32(qjl[blk:blk + 1]), to_np_f16bits(norms[sl]), True, layout=1)
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])

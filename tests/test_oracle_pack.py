@@ -31,3 +31,23 @@ def test_round_trips():
             np.testing.assert_array_equal(oracle.unpack_codes(oracle.pack_codes(codes, b), b, d), codes)
     bits = rng.integers(0, 2, (9, 128)).astype(np.uint8)
     np.testing.assert_array_equal(oracle.unpack_bits(oracle.pack_bits(bits), 128), bits)
+
+
+def test_block32_hand_worked_and_round_trip():
+    # vector i of a block is bit i of every word: 3 vectors, code of coordinate j of vector v = (v + j) % 4
+    codes = (np.arange(3)[:, None] + np.arange(64)[None, :]) % 4
+    w = oracle.pack_codes_block32(codes, 2)
+    assert w.shape == (1, 2, 64)
+    # coordinate 0: codes of vectors 0,1,2 = 0,1,2 -> plane 0 bits 0,1,0 -> 0b010; plane 1 bits 0,0,1 -> 0b100
+    assert w[0, 0, 0] == 0b010 and w[0, 1, 0] == 0b100
+    rng = np.random.default_rng(1)
+    for n in (1, 31, 32, 33, 100):
+        c = rng.integers(0, 8, (n, 128))
+        np.testing.assert_array_equal(oracle.unpack_codes_block32(oracle.pack_codes_block32(c, 3), 3, 128, n), c)
+        bits = rng.integers(0, 2, (n, 64)).astype(np.uint8)
+        np.testing.assert_array_equal(oracle.unpack_bits_block32(oracle.pack_bits_block32(bits), 64, n), bits)
+    # token and block layouts carry the same bits
+    c = rng.integers(0, 4, (64, 128))
+    tok = oracle.unpack_codes(oracle.pack_codes(c, 2), 2, 128)
+    blk = oracle.unpack_codes_block32(oracle.pack_codes_block32(c, 2), 2, 128, 64)
+    np.testing.assert_array_equal(tok, blk)

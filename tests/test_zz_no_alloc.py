@@ -19,23 +19,22 @@ from .parity import ATOL, RTOL
 pytestmark = pytest.mark.gpu
 
 
-def _cache(h, S, T, seed):
-    """S streams of T quantized tokens of the Llama-layer key/value generator, on the device."""
-    codes = torch.empty((S, T, h.b, h.d // 32), dtype=torch.int32, device="cuda")
-    qjl = torch.empty((S, T, h.m // 32), dtype=torch.int32, device="cuda")
-    norms = torch.empty((S, T, 2), dtype=torch.float16, device="cuda")
+def _cache(h, S, T, seed, layout):
+    """S streams of T quantized tokens of the Llama-layer key generator, on the device."""
     x = wl.llama_keys(S, T, h.d, seed, device="cuda")
-    kvq.kvq_quantize(h, x, codes, qjl, norms)
-    return codes, qjl, norms
+    parts = [kvq.alloc_packed(h, T, layout=layout) for _ in range(S)]
+    for s in range(S):
+        kvq.kvq_quantize(h, x[s], *parts[s], layout=layout)
+    return [torch.stack([p[i] for p in parts]) for i in range(3)]
 
 
 def test_noalloc_matches_workspace_entry_point_on_two_calls():
-    d, B, hq, hkv, T = 128, 2, 8, 2, 3000
+    d, B, hq, hkv, T = 128, 2, 8, 2, 3008
     with kvq.Handle(d, 2, 1, qjl=True) as h:
-        kt = _cache(h, B * hkv, T, seed=5)
-        vt = _cache(h, B * hkv, T, seed=6)
-        kc = kvq.make_cache(*kt, T)
-        vc = kvq.make_cache(*vt, T)
+        kt = _cache(h, B * hkv, T, seed=5, layout=0)
+        vt = _cache(h, B * hkv, T, seed=6, layout=1)
+        kc = kvq.make_cache(*kt, T, 0)
+        vc = kvq.make_cache(*vt, T, 1)
         seq = torch.tensor([T, 1777], dtype=torch.int32, device="cuda")
         ws = torch.empty(kvq.kvq_decode_workspace(h, B, hq, hkv, T), dtype=torch.uint8, device="cuda")
         assert ws.numel() <= kvq.NOALLOC_SCRATCH_BYTES
@@ -62,10 +61,11 @@ def test_noalloc_rejects_sizes_beyond_the_fixed_scratch():
     with kvq.Handle(d, 2, 1, qjl=True) as h:
         assert kvq.kvq_decode_workspace(h, B, hq, hkv, T) > kvq.NOALLOC_SCRATCH_BYTES
         dummy = torch.zeros(64, dtype=torch.int32, device="cuda")
-        c = kvq.make_cache(dummy, dummy, dummy.view(torch.float16), T)
+        kc = kvq.make_cache(dummy, dummy, dummy.view(torch.float16), T, 0)
+        vc = kvq.make_cache(dummy, dummy, dummy.view(torch.float16), T, 1)
         q = torch.zeros((B, hq, d), dtype=torch.bfloat16, device="cuda")
         out = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
         seq = torch.zeros(B, dtype=torch.int32, device="cuda")
         with pytest.raises(kvq.KvqError) as e:
-            kvq.kvq_decode_attend_noalloc(h, q, hkv, c, c, seq, T, 1.0, out)
+            kvq.kvq_decode_attend_noalloc(h, q, hkv, kc, vc, seq, T, 1.0, out)
         assert e.value.code == kvq.KVQ_EINVAL and "scratch" in str(e.value)
