@@ -41,7 +41,7 @@ def _nvcc() -> str:
 
 def _sources():
     """(object name, source, extra flags) of every compile job."""
-    jobs = [("api.o", "api.cu", []), ("decode.o", "decode.cu", [])]
+    jobs = [("api.o", "api.cu", []), ("decode.o", "decode.cu", []), ("decode_mma.o", "decode_mma.cu", [])]
     for d in DIMS:
         for b in BITS:
             jobs.append((f"quantize_d{d}_b{b}.o", "quantize_inst.cu", [f"-DKVQ_D={d}", f"-DKVQ_B={b}"]))

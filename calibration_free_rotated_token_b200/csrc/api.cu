@@ -357,8 +357,13 @@ int decode_check(kvq_handle h, int dtype, int batch, int hq, int hkv, const kvq_
         if (c->capacity < max_T) return fail(KVQ_EINVAL, "cache capacity is smaller than max_T");
     }
     if (k->layout != KVQ_LAYOUT_TOKEN) return fail(KVQ_EINVAL, "the key cache must use KVQ_LAYOUT_TOKEN");
-    if (v->layout != KVQ_LAYOUT_BLOCK32 || v->capacity % 32 != 0)
-        return fail(KVQ_EINVAL, "the value cache must use KVQ_LAYOUT_BLOCK32 with a capacity that is a multiple of 32");
+    if (v->layout != KVQ_LAYOUT_BLOCK32) return fail(KVQ_EINVAL, "the value cache must use KVQ_LAYOUT_BLOCK32");
+    if (k->capacity % 32 != 0 || v->capacity % 32 != 0)
+        return fail(KVQ_EINVAL, "cache capacities must be multiples of 32");
+    for (const kvq_cache* c : {k, v}) {
+        if (!aligned(c->codes, 16) || !aligned(c->norms, 16) || (c->qjl && !aligned(c->qjl, 16)))
+            return fail(KVQ_EINVAL, "cache buffers must be 16-byte aligned");
+    }
     if (!q || !out || !seq_len) return fail(KVQ_EINVAL, "q, out and seq_len must be non-null");
     if (!std::isfinite(scale)) return fail(KVQ_EINVAL, "scale must be finite");
     kvq::decode_plan(h, batch, hq, hkv, max_T > 0 ? max_T : 1, ns, chunk, need);
@@ -391,11 +396,23 @@ int decode_launch(kvq_handle h, const void* q, int dtype, int batch, int hq, int
     a.logits = logits;
     a.out = out;
     const int64_t bh = static_cast<int64_t>(batch) * hq;
-    float* ws = static_cast<float*>(workspace);
-    a.qrot = ws;
-    a.qproj = ws + bh * h->d;
-    a.part = ws + bh * h->d + bh * h->m;
+    const int64_t streams = static_cast<int64_t>(batch) * hkv;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    size_t off = static_cast<size_t>(bh * ns * (2 + h->d + h->m)) * sizeof(float);
+    off = (off + 255) / 256 * 256;
+    a.part = reinterpret_cast<float*>(ws);
+    if (kvq::decode_uses_mma(h)) {
+        a.qscal = reinterpret_cast<float*>(ws + off);
+        off += static_cast<size_t>(bh) * 4 * sizeof(float);
+        off = (off + 255) / 256 * 256;
+        a.qfrag = reinterpret_cast<uint2*>(ws + off);
+        (void)streams;
+    } else {
+        a.qrot = reinterpret_cast<float*>(ws + off);
+        a.qproj = a.qrot + bh * h->d;
+    }
     a.S = h->d_S;
+    a.status = h->d_status;
     float thr_unused[kvq::kMaxLevels];
     fill_common(h, a.centroid, thr_unused, a.pair_sign);
     std::string why;

@@ -406,7 +406,6 @@ cudaError_t launch_dd(const DecodeArgs& a, int b, bool qjl, cudaStream_t s) {
 
 void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, int* nsplit, int64_t* chunk,
                  size_t* ws_bytes) {
-    (void)hq;
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
     const int64_t streams = static_cast<int64_t>(batch) * hkv;
@@ -422,12 +421,34 @@ void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, in
     *nsplit = static_cast<int>(ns);
     *chunk = ch;
     const int64_t bh = static_cast<int64_t>(batch) * hq;
-    const int64_t floats = bh * h->d + bh * h->m + bh * ns * (2 + h->d + h->m);
-    *ws_bytes = static_cast<size_t>(floats) * sizeof(float) + 256;
+    // partials first (both paths), then the path's query data
+    size_t bytes = static_cast<size_t>(bh * ns * (2 + h->d + h->m)) * sizeof(float);
+    bytes = (bytes + 255) / 256 * 256;
+    if (decode_uses_mma(h)) {
+        bytes += static_cast<size_t>(bh) * 4 * sizeof(float);
+        bytes = (bytes + 255) / 256 * 256;
+        bytes += static_cast<size_t>(streams) * decode_mma_qfrag_bytes(h, hq / hkv);
+    } else {
+        bytes += static_cast<size_t>(bh) * (h->d + h->m) * sizeof(float);
+    }
+    *ws_bytes = bytes + 256;
 }
 
 cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s, std::string* why) {
     const bool qjl = (h->flags & 1u) != 0;
+    if (decode_uses_mma(h)) {
+        cudaError_t e = launch_decode_mma(h, a, s);
+        if (e != cudaSuccess) return e;
+        switch (h->d) {
+            case 64: qjl ? decode_combine_kernel<64, true><<<a.batch * a.hq, kDecThreads, 0, s>>>(a)
+                         : decode_combine_kernel<64, false><<<a.batch * a.hq, kDecThreads, 0, s>>>(a); break;
+            case 128: qjl ? decode_combine_kernel<128, true><<<a.batch * a.hq, kDecThreads, 0, s>>>(a)
+                          : decode_combine_kernel<128, false><<<a.batch * a.hq, kDecThreads, 0, s>>>(a); break;
+            default: qjl ? decode_combine_kernel<256, true><<<a.batch * a.hq, kDecThreads, 0, s>>>(a)
+                         : decode_combine_kernel<256, false><<<a.batch * a.hq, kDecThreads, 0, s>>>(a); break;
+        }
+        return cudaGetLastError();
+    }
     switch (h->d) {
         case 64: return launch_dd<64>(a, h->b, qjl, s);
         case 128: return launch_dd<128>(a, h->b, qjl, s);

@@ -77,6 +77,9 @@ struct DecodeArgs {
     float* qrot;                      // workspace [batch*hq][d]   q' = H (delta.*q)
     float* qproj;                     // workspace [batch*hq][m]   p = S q'
     float* part;                      // workspace [batch*hq][nsplit][2 + d + m]
+    uint2* qfrag;                     // tensor path: workspace, query fragments per (sequence, KV head)
+    uint32_t* status;                 // device status word of the handle
+    float* qscal;                     // tensor path: workspace [batch*hq][4] per-head scalars
     const __half* S;
     float centroid[kMaxLevels];
     uint32_t pair_sign[128];
@@ -87,6 +90,11 @@ void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, in
                  size_t* ws_bytes);
 
 cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s, std::string* why);
+
+// Tensor-core decode path (1- and 2-bit codebooks): query fragments + split kernel.
+cudaError_t launch_decode_mma(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s);
+size_t decode_mma_qfrag_bytes(const kvq_ctx* h, int G);
+inline bool decode_uses_mma(const kvq_ctx* h) { return h->b <= 2; }
 
 // Size of the fixed scratch of kvq_decode_attend_noalloc (mirrors
 // KVQ_NOALLOC_SCRATCH_BYTES of kvq.h) and its address on `device`, which

@@ -156,7 +156,8 @@ int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, in
 /* One packed cache (keys or values) of batch * hkv streams, each holding up
  * to `capacity` vectors in the layout above; stream (bi, hi) starts at
  * vector (bi * hkv + hi) * capacity.  Keys use KVQ_LAYOUT_TOKEN, values
- * KVQ_LAYOUT_BLOCK32 (capacity a multiple of 32). */
+ * KVQ_LAYOUT_BLOCK32; capacities are multiples of 32 and the buffers 16-byte
+ * aligned. */
 typedef struct kvq_cache {
     const uint32_t* codes;  /* device, streams * capacity * b * d/32 */
     const uint32_t* qjl;    /* device, streams * capacity * d/32; NULL without KVQ_QJL */

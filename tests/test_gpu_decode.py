@@ -122,19 +122,14 @@ def test_long_context_split_merge():
     check_case(128, 2, True, 1, 4, 1, [20000], 20000, scale=1.0 / np.sqrt(128))
 
 
-def test_decode_workload_full_size_sampled():
-    """batch 16, 32/8 heads, d 128, 131072-token contexts, b=2 + QJL, q ~ N(0,1)/sqrt(128), scale 1.
-
-    The whole cache is produced by the CUDA quantizer from the Llama-layer
-    generator; for one sampled (sequence, KV head) the GPU quantizer is checked
-    against the oracle on sampled rows and that stream is then replaced by the
-    oracle's own cache, whose decode the oracle recomputes for the 4 query heads.
-    """
+def _sampled_stream_decode(B, hq, hkv, T, sample, check_rows=1024):
+    """Cache of B x hkv streams of T tokens from the CUDA quantizer (Llama-layer generator);
+    one sampled (sequence, KV head) is checked against the oracle's quantization on sampled
+    rows and then replaced by the oracle's own cache, whose decode the oracle recomputes."""
     c = wl.DECODE
-    d, T, B, hq, hkv = c["d"], c["T"], c["batch"], c["hq"], c["hkv"]
+    d = c["d"]
     G = hq // hkv
     k = constants(d, c["b"], c["handle_seed"])
-    sample = (5, 3)
     with kvq.Handle(d, c["b"], c["handle_seed"], qjl=True) as h:
         S = B * hkv
         kcodes = torch.empty((S, T, h.b, d // 32), dtype=torch.int32, device="cuda")
@@ -156,7 +151,7 @@ def test_decode_workload_full_size_sampled():
                 Vs = V[sample[1]].double().cpu().numpy()
         assert kvq.kvq_status(h)[0] == 0
         s = sample[0] * hkv + sample[1]
-        rows = np.sort(np.random.default_rng(1).choice(T, 1024, replace=False))
+        rows = np.sort(np.random.default_rng(1).choice(T, min(check_rows, T), replace=False))
         tr = torch.from_numpy(rows).cuda()
         compare_quantize(k, Ks[rows], to_np_u32(kcodes[s][tr]), to_np_u32(kqjl[s][tr]),
                          to_np_f16bits(knorm[s][tr]), True)
@@ -176,3 +171,14 @@ def test_decode_workload_full_size_sampled():
     _, orf = oracle.decode_attend(k, qs, sk, sv, c["scale"], True, want_logits=False)
     assert_close(out[sample[0], sample[1] * G:(sample[1] + 1) * G], orf, "out (sampled stream)")
     assert np.isfinite(out).all()
+
+
+def test_decode_several_subchunks_per_split():
+    """4 sequences x 8 KV heads x 16384 tokens: 16 splits of 1024 tokens (four sub-chunks each)."""
+    _sampled_stream_decode(4, 32, 8, 16384, sample=(2, 5))
+
+
+def test_decode_workload_full_size_sampled():
+    """batch 16, 32/8 heads, d 128, 131072-token contexts, b=2 + QJL, q ~ N(0,1)/sqrt(128), scale 1."""
+    c = wl.DECODE
+    _sampled_stream_decode(c["batch"], c["hq"], c["hkv"], c["T"], sample=(5, 3))
