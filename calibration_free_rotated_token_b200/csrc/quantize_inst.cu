@@ -1,7 +1,10 @@
 // quantize_inst.cu -- instantiates the quantize kernels of one (d, b), given
 // as -DKVQ_D=<d> -DKVQ_B=<b> by the build; the build compiles this file once
 // per supported pair so that the twelve instantiations compile in parallel.
-#include "quantize.cuh"
+// 16-bit input with d <= 128 takes the tensor-core rotation kernel
+// (quantize_tc.cuh); fp32 input, d = 256 and the NSN front end take the
+// kernel with the in-register transform (quantize.cuh).
+#include "quantize_tc.cuh"
 
 #ifndef KVQ_D
 #error "KVQ_D must be defined"
@@ -26,8 +29,12 @@ cudaError_t by_dtype(const CUtensorMap& map, int dtype, const QuantArgs& a, int 
             case DT_F32:
                 if constexpr (D <= 128) return launch_quantize_t<D, B, QJL, DT_F32, NSN>(map, a, sms, s);
                 else return cudaErrorNotSupported;
-            case DT_F16: return launch_quantize_t<D, B, QJL, DT_F16, NSN>(map, a, sms, s);
-            default: return launch_quantize_t<D, B, QJL, DT_BF16, NSN>(map, a, sms, s);
+            case DT_F16:
+                if constexpr (D <= 128 && !NSN) return launch_quantize_tc<D, B, QJL, DT_F16>(map, a, sms, s);
+                else return launch_quantize_t<D, B, QJL, DT_F16, NSN>(map, a, sms, s);
+            default:
+                if constexpr (D <= 128 && !NSN) return launch_quantize_tc<D, B, QJL, DT_BF16>(map, a, sms, s);
+                else return launch_quantize_t<D, B, QJL, DT_BF16, NSN>(map, a, sms, s);
         }
     }
 }

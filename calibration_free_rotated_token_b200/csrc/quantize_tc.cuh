@@ -1,0 +1,336 @@
+// quantize_tc.cuh -- the quantize kernel with the rotation on the tensor
+// cores, for 16-bit input and d <= 128.
+//
+// Method (TurboQuant blog, "Estagio 1" and "Estagio 2"; PolarQuant section 2),
+// per vector x: y = H (delta .* x) (unnormalised Sylvester Hadamard, so
+// ||y||^2 = d ||x||^2), n = ||x||, z = y / n, code_j = #{k : z_j >= t_k},
+// r = z - c[code], gamma = ||r||, QJL bits = [S r >= 0], norms fp16.
+//
+// Design (sm_100a):
+// * The randomized Hadamard rotation is one dense product per 128-vector
+//   tile, Y(128 x d) = X(128 x d) (H D)^T, on tcgen05: X straight from the
+//   TMA stage (K-major, 128-byte swizzle), H D (entries +-1, exact in bf16
+//   and fp16, built in shared memory at start-up) as the B operand, fp32
+//   accumulation into tensor memory.  Every product x_k * (+-1) is exact,
+//   so y carries only fp32 summation rounding.
+// * Four warpgroups per CTA (one CTA per SM), each owning 128 TMEM columns
+//   and whole tiles; a thread owns one vector (its TMEM lane).  Each stage of
+//   the x ring belongs to one warpgroup; it is free as soon as the rotation
+//   MMA has read it, and the warpgroup refills it then.
+// * Pass 1 reads y back (32 columns at a time) for ||y||^2; pass 2 reads it
+//   again, forms codes and the residual chunk by chunk and writes the fp16
+//   residual into the already consumed columns [0, d/2).
+// * QJL: U(128 x 64) = R S_h^T for the two 64-row halves of S (d = 128; one
+//   half for d = 64), accumulated in columns [64, 128), and the sign bits are
+//   packed from there.  The residual enters as one fp16 term: with S exact in
+//   fp16 and fp32 accumulation the error of (S r)_i is about 2e-4 ||r|| (one
+//   standard deviation), so a sign can differ from the exact one only where
+//   |(S r)_i| is a few 1e-4 ||r||, inside the 1e-3 ||r|| band where the sign
+//   is not pinned (a flip outside it needs a 5-sigma error, ~1e-11 per bit).
+// * Every mbarrier wait is bounded and its outcome agreed on by the
+//   warpgroup; loads still in flight at exit are waited for.
+#pragma once
+
+#include "quantize.cuh"
+
+namespace kvq {
+
+template <int D, bool QJL>
+struct TcCfg {
+    static constexpr int kTileBytes = kTileRows * D * 2;   // 16-bit input
+    static constexpr int kBoxBytes = 128 * kTileRows;      // 64 elements x 128 rows
+    static constexpr int kBoxes = D * 2 / 128;
+    static constexpr int kMatBytes = D * D * 2;            // H D or S, 16-bit, K-major, swizzled
+    static constexpr int kWG = 4;
+    static constexpr int kThreads = 128 * kWG;
+    static constexpr int kAuxBytes = 1024;
+    static constexpr int kBudget = 225 * 1024;
+    static constexpr int kStagesRaw = (kBudget - kMatBytes - (QJL ? kMatBytes : 0) - kAuxBytes) / kTileBytes;
+    // Tile i goes to warpgroup i % 4 and stage i % kStages; with kStages a
+    // multiple of 4 every stage belongs to one warpgroup, which consumes its
+    // phases strictly in order (a parity wait can never see a stale phase).
+    static constexpr int kStages = (kStagesRaw > 8 ? 8 : kStagesRaw) / kWG * kWG;
+    static constexpr int kSmemBytes = 1024 + kStages * kTileBytes + kMatBytes + (QJL ? kMatBytes : 0) + kAuxBytes;
+    static constexpr int kQN = 64;                          // rows of S per QJL MMA
+    static_assert(D == 64 || D == 128, "tensor-core rotation: d in {64, 128}");
+    static_assert(kStages >= kWG, "one stage per warpgroup at least");
+};
+
+// Sign word of 32 accumulator values: bit i = [u_i >= 0].
+__device__ __forceinline__ uint32_t sign_word(const uint32_t (&u)[32]) {
+    uint32_t b[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int i = 7; i >= 0; --i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) b[q] = __funnelshift_l(u[8 * q + i], b[q], 1);
+    return ~(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24));
+}
+
+template <int D, int B, bool QJL, int DT>
+__global__ void __launch_bounds__(512, 1)
+    quantize_tc_kernel(const __grid_constant__ CUtensorMap map, const __grid_constant__ QuantArgs a) {
+    using C = TcCfg<D, QJL>;
+    constexpr int NS = C::kStages;
+    constexpr int kWpp = D / 32;
+    constexpr uint32_t kIdescH = idesc_16bit_f32(kTileRows, D, DT == DT_BF16);
+    constexpr uint32_t kIdescQ = idesc_16bit_f32(kTileRows, C::kQN, false);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stage0 = smem;
+    uint8_t* sHD = smem + NS * C::kTileBytes;
+    uint8_t* sS = sHD + C::kMatBytes;
+    uint8_t* aux = sS + (QJL ? C::kMatBytes : 0);
+    uint64_t* full = reinterpret_cast<uint64_t*>(aux);    // [8]
+    uint64_t* hbar = full + 8;                              // [4] rotation MMA done
+    uint64_t* qbar = hbar + 4;                              // [4] QJL MMA done
+    uint32_t* iss = reinterpret_cast<uint32_t*>(qbar + 4);  // [8] loads issued per stage
+    uint32_t* con = iss + 8;                                // [8] loads consumed per stage
+    uint32_t* tmem_slot = con + 8;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int wg = warp >> 2;
+    const int r = tid & 127;
+    const int64_t G = gridDim.x;
+
+    if (tid == 0) {
+        for (int s = 0; s < 8; ++s) {
+            mbar_init(&full[s], 1);
+            iss[s] = 0;
+            con[s] = 0;
+        }
+        for (int w = 0; w < 4; ++w) {
+            mbar_init(&hbar[w], 1);
+            mbar_init(&qbar[w], 1);
+        }
+        fence_mbar_init();
+    }
+    // H D as the B operand (row n = output coordinate, K = input coordinate):
+    // entry (n, k) = (-1)^popcount(n & k) delta_k.  K-chunk kc (64 entries)
+    // of row n at sHD + kc*D*128 + n*128, 16-byte chunk c at c ^ (n & 7).
+    {
+        const uint32_t one = (DT == DT_BF16) ? 0x3F80u : 0x3C00u;
+        for (int e = tid; e < D * D / 8; e += C::kThreads) {
+            const int n = e / (D / 8), cc = e % (D / 8);
+            const int kc = cc / 8, c16 = cc % 8;
+            uint32_t w4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int k = 8 * cc + 2 * q;
+                const uint32_t ps = a.pair_sign[k >> 1];
+                const uint32_t s0 = ((__popc(n & k) & 1u) << 15) ^ (ps & 0x8000u);
+                const uint32_t s1 = ((__popc(n & (k + 1)) & 1u) << 15) ^ ((ps >> 16) & 0x8000u);
+                w4[q] = (one | s0) | ((one | s1) << 16);
+            }
+            *reinterpret_cast<uint4*>(sHD + kc * (D * 128) + n * 128 + ((c16 ^ (n & 7)) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+    }
+    if (QJL) {
+        const uint4* gS = reinterpret_cast<const uint4*>(a.S);
+        for (int e = tid; e < D * D / 8; e += C::kThreads) {
+            const int n = e / (D / 8), cc = e % (D / 8);
+            const int kc = cc / 8, c16 = cc % 8;
+            *reinterpret_cast<uint4*>(sS + kc * (D * 128) + n * 128 + ((c16 ^ (n & 7)) << 4)) = gS[e];
+        }
+    }
+    fence_proxy_async_smem();
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // Tile i (local index) lives in stage i % NS.
+    auto issue_tile = [&](int64_t i) {
+        const int64_t tile = blockIdx.x + i * G;
+        if (tile >= a.ntiles) return;
+        const int st = static_cast<int>(i % NS);
+        iss[st] += 1;
+        mbar_arrive_expect_tx(&full[st], C::kTileBytes);
+#pragma unroll
+        for (int box = 0; box < C::kBoxes; ++box)
+            tma_load_2d(stage0 + st * C::kTileBytes + box * C::kBoxBytes, &map, &full[st], box * 64,
+                        static_cast<int>(tile * kTileRows));
+    };
+    if (tid == 0) {
+        prefetch_tmap(&map);
+        for (int64_t i = 0; i < NS; ++i) issue_tile(i);
+    }
+    __syncthreads();
+
+    const uint32_t bar_id = 1 + wg;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tcol = tmem + static_cast<uint32_t>(wg * 128);  // this warpgroup's 128 columns
+    const uint32_t tl = tcol + lane_base;                            // ... at this thread's lane
+    uint32_t hpar = 0, qpar = 0;
+
+    for (int64_t i = wg;; i += C::kWG) {
+        const int64_t tile = blockIdx.x + i * G;
+        if (tile >= a.ntiles) break;
+        const int st = static_cast<int>(i % NS);
+        const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((i / NS) & 1), a.status);
+        if (named_bar_or(bar_id, 128, !ok)) break;
+        if (r == 0) {
+            con[st] += 1;
+            // ---- rotation: Y = X (H D)^T into columns [0, D) ----
+            tc_fence_after();
+            const uint32_t xs = smem_u32(stage0 + st * C::kTileBytes);
+            const uint32_t hs = smem_u32(sHD);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t aoff = (ks / 4) * C::kBoxBytes + (ks % 4) * 32;
+                const uint32_t boff = (ks / 4) * (D * 128) + (ks % 4) * 32;
+                mma_f16_ss(tcol, smem_desc_sw128(xs + aoff), smem_desc_sw128(hs + boff), kIdescH, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(&hbar[wg]);
+        }
+        const bool okh = mbar_wait(&hbar[wg], hpar, a.status);
+        hpar ^= 1u;
+        if (named_bar_or(bar_id, 128, !okh)) break;
+        if (r == 0) issue_tile(i + NS);  // the stage has been read
+        tc_fence_after();
+
+        // ---- pass 1: ||y||^2 = D ||x||^2 ----
+        float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tmem_ld32(tl + 32 * c, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float2 y = make_float2(u2f(u[2 * k]), u2f(u[2 * k + 1]));
+                acc2 = __ffma2_rn(y, y, acc2);
+            }
+        }
+        const float ssx = (acc2.x + acc2.y) * (1.0f / D);
+        const float nrm = sqrtf(ssx);
+        flag_norm(ssx, nrm, a.status);
+        const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+
+        // ---- pass 2: codes, residual (fp16 into columns [16c, 16c + 16)) ----
+        uint32_t planes[B][kWpp];
+        float rr = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tmem_ld32(tl + 32 * c, u);
+            tmem_wait_ld();
+            float2 v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] = make_float2(u2f(u[2 * k]), u2f(u[2 * k + 1]));
+            uint32_t pl[B][1];
+            rr += codes_and_residual<32, B>(v, inv, a, pl);
+#pragma unroll
+            for (int p = 0; p < B; ++p) planes[p][c] = pl[p][0];
+            if (QJL) {
+                uint32_t hi[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const __half2 hh = __float22half2_rn(v[k]);
+                    hi[k] = *reinterpret_cast<const uint32_t*>(&hh);
+                }
+                tmem_st16(tl + 16 * c, hi);
+            }
+        }
+        const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
+        const int64_t vidx = tile * kTileRows + r;
+        const bool valid = vidx < a.n;
+        if (a.layout == 0) {
+            if (valid) {
+                uint32_t* cp = a.codes + vidx * (B * kWpp);
+#pragma unroll
+                for (int p = 0; p < B; ++p) store_words<kWpp>(cp + p * kWpp, planes[p], zmask);
+            }
+        } else {
+            const int64_t blk = tile * 4 + (warp & 3);
+            const uint32_t m = valid ? zmask : 0u;
+#pragma unroll
+            for (int p = 0; p < B; ++p)
+                store_block32<kWpp>(a.codes + (blk * B + p) * D, planes[p], m, lane, blk * 32 < a.n);
+        }
+        if (valid) {
+            const float g = nrm > 0.f ? sqrtf(rr) : 0.f;
+            a.norms[vidx] = __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
+        }
+
+        if (QJL) {
+            // ---- QJL: U = R S_h^T per 64-row half of S, in columns [64, 128) ----
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar_sync(bar_id, 128);
+            uint32_t qw[kWpp];
+            bool failed = false;
+#pragma unroll
+            for (int h = 0; h < D / C::kQN; ++h) {
+                if (r == 0) {
+                    tc_fence_after();
+                    const uint32_t ss0 = smem_u32(sS);
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t boff = (ks / 4) * (D * 128) + h * (C::kQN * 128) + (ks % 4) * 32;
+                        mma_f16_ts(tcol + 64, tcol + ks * 8, smem_desc_sw128(ss0 + boff), kIdescQ,
+                                   ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&qbar[wg]);
+                }
+                const bool okq = mbar_wait(&qbar[wg], qpar, a.status);
+                qpar ^= 1u;
+                if (named_bar_or(bar_id, 128, !okq)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t u0[32], u1[32];
+                tmem_ld32(tl + 64, u0);
+                tmem_ld32(tl + 96, u1);
+                tmem_wait_ld();
+                qw[2 * h] = sign_word(u0);
+                qw[2 * h + 1] = sign_word(u1);
+                tc_fence_before();
+                if (h + 1 < D / C::kQN) named_bar_sync(bar_id, 128);  // the next half reuses the columns
+            }
+            if (failed) break;
+            if (a.layout == 0) {
+                if (valid) store_words<kWpp>(a.qjl + vidx * kWpp, qw, zmask);
+            } else {
+                const int64_t blk = tile * 4 + (warp & 3);
+                store_block32<kWpp>(a.qjl + blk * D, qw, valid ? zmask : 0u, lane, blk * 32 < a.n);
+            }
+        }
+        // The next rotation MMA rewrites this warpgroup's columns; the barrier
+        // at the top of the next iteration orders it after these accesses.
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (tid == 0) {
+        // Loads issued but never consumed (only after a wait gave up).
+        for (int s = 0; s < NS; ++s)
+            if (iss[s] > con[s]) mbar_wait(&full[s], con[s] & 1u, a.status);
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D, int B, bool QJL, int DT>
+cudaError_t launch_quantize_tc(const CUtensorMap& map, const QuantArgs& a, int num_sms, cudaStream_t s) {
+    using C = TcCfg<D, QJL>;
+    auto kern = quantize_tc_kernel<D, B, QJL, DT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = a.ntiles < num_sms ? a.ntiles : num_sms;
+    if (grid <= 0) return cudaSuccess;
+    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, s>>>(map, a);
+    return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -215,6 +215,24 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor of kind::f16 with bf16 (bf16 = true) or fp16 A and
+// B (the two always share one type), fp32 accumulator, K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_16bit_f32(int M, int N, bool bf16) {
+    return idesc_f16_f32(M, N) | (bf16 ? ((1u << 7) | (1u << 10)) : 0u);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, both described by shared-memory
+// descriptors (M x 16 and N x 16, K-major).  Issued by one thread.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T, A M x 16 fp16 from tensor memory, B
 // described by bdesc (N x 16, K-major).  Issued by one thread.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
