@@ -153,12 +153,19 @@ class Clocks:
                 "samples": len(rows), "power_w_max": max(num(r[3]) for r in rows)}
 
 
+HEAD_START_CYCLES = 6_000_000  # ~3 ms at 1.97 GHz
+
+
 def timed(dist: Dist, fn, steps: int, stream) -> float:
     """Milliseconds for `steps` calls of fn(i), device-timed, max over ranks."""
     dist.barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    # A device-side sleep ahead of the region lets the host enqueue the steps
+    # before the GPU reaches them, so the device intervals hold no host
+    # launch latency (that is what the e2e figure measures).
+    torch.cuda._sleep(HEAD_START_CYCLES)
     e0.record(stream)
     for i in range(steps):
         fn(i)

@@ -196,7 +196,11 @@ __device__ __forceinline__ float mag_search(float az, const float* th, const flo
         return mu[0];
     } else if constexpr (B == 2) {
         g[0] = az - tau[1];
-        return g[0] >= 0.f ? mu[1] : mu[0];
+        // [g >= 0] as 0 or 1 on the FMA pipe: tau[1] = 0.98..., so a negative
+        // g is at least 2^-25 below 0 (exact difference near tau, or below
+        // -tau/2), and g * 2^32 + 1 saturates to exactly 0 or 1.
+        const float s = __saturatef(fmaf(g[0], 0x1p32f, 1.0f));
+        return fmaf(s, mu[1] - mu[0], mu[0]);
     } else if constexpr (B == 3) {
         g[1] = az - tau[2];
         const bool m1 = g[1] >= 0.f;

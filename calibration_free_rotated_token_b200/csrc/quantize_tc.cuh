@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(512, 1)
         }
     }
     if (QJL) {
+        // S is written once at handle creation, before any launch.
         const uint4* gS = reinterpret_cast<const uint4*>(a.S);
         for (int e = tid; e < D * D / 8; e += C::kThreads) {
             const int n = e / (D / 8), cc = e % (D / 8);
@@ -145,6 +146,10 @@ __global__ void __launch_bounds__(512, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+
+    // Launched as a programmatic dependent: the input may come from the grid
+    // before this one, so nothing global is read or written before this.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // Tile i (local index) lives in stage i % NS.
     auto issue_tile = [&](int64_t i) {
@@ -196,18 +201,21 @@ __global__ void __launch_bounds__(512, 1)
         if (r == 0) issue_tile(i + NS);  // the stage has been read
         tc_fence_after();
 
-        // ---- pass 1: ||y||^2 = D ||x||^2 ----
+        // ---- pass 1: ||y||^2 = D ||x||^2 (the next chunk loads while one is summed) ----
+        constexpr int NC = D / 32;
+        uint32_t ybuf[2][32];
         float2 acc2 = make_float2(0.f, 0.f);
+        tmem_ld32(tl, ybuf[0]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            uint32_t u[32];
-            tmem_ld32(tl + 32 * c, u);
-            tmem_wait_ld();
+        for (int c = 0; c < NC; ++c) {
+            if (c + 1 < NC) tmem_ld32(tl + 32 * (c + 1), ybuf[(c + 1) & 1]);
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const float2 y = make_float2(u2f(u[2 * k]), u2f(u[2 * k + 1]));
+                const float2 y = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
                 acc2 = __ffma2_rn(y, y, acc2);
             }
+            if (c + 1 < NC) tmem_wait_ld();
         }
         const float ssx = (acc2.x + acc2.y) * (1.0f / D);
         const float nrm = sqrtf(ssx);
@@ -215,16 +223,18 @@ __global__ void __launch_bounds__(512, 1)
         const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
 
         // ---- pass 2: codes, residual (fp16 into columns [16c, 16c + 16)) ----
+        // Chunk c + 1 loads while chunk c is coded; the residual of chunk c
+        // goes to columns that chunks 0 .. c/2 occupied, all read already.
         uint32_t planes[B][kWpp];
         float rr = 0.f;
+        tmem_ld32(tl, ybuf[0]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            uint32_t u[32];
-            tmem_ld32(tl + 32 * c, u);
-            tmem_wait_ld();
+        for (int c = 0; c < NC; ++c) {
+            if (c + 1 < NC) tmem_ld32(tl + 32 * (c + 1), ybuf[(c + 1) & 1]);
             float2 v[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = make_float2(u2f(u[2 * k]), u2f(u[2 * k + 1]));
+            for (int k = 0; k < 16; ++k) v[k] = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
             uint32_t pl[B][1];
             rr += codes_and_residual<32, B>(v, inv, a, pl);
 #pragma unroll
@@ -238,6 +248,7 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 tmem_st16(tl + 16 * c, hi);
             }
+            if (c + 1 < NC) tmem_wait_ld();
         }
         const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
         const int64_t vidx = tile * kTileRows + r;
@@ -329,8 +340,19 @@ cudaError_t launch_quantize_tc(const CUtensorMap& map, const QuantArgs& a, int n
     if (e != cudaSuccess) return e;
     const int64_t grid = a.ntiles < num_sms ? a.ntiles : num_sms;
     if (grid <= 0) return cudaSuccess;
-    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, s>>>(map, a);
-    return cudaGetLastError();
+    // Programmatic dependent launch: this grid may be scheduled while the
+    // previous one drains; the kernel waits for it before touching memory.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, map, a);
 }
 
 }  // namespace kvq
