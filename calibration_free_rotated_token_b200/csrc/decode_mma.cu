@@ -1,4 +1,4 @@
-// decode_mma.cu -- decode attention on the tensor cores (warp-level int8
+// decode_mma.cu -- decode attention on the tensor cores (warp-level integer
 // MMA), for 1- and 2-bit codebooks.
 //
 // Method (TurboQuant blog, "Como Implementar": the query is rotated once and
@@ -13,21 +13,24 @@
 //   planes: c[code] = c0 + (c1 - c0) bit0 + (c2 - c0) bit1 (the bit0*bit1
 //   coefficient c3 - c2 - c1 + c0 vanishes by symmetry).  So every dot
 //   product above is a constant plus plain sums of 0/1 planes, and both
-//   contractions run as exact integer tensor-core products:
-//   - keys: D(16 tokens x 8) += A(16 tokens x 32 coords, 0/1) B(32 coords x 8)
-//     where B holds the query (times the plane coefficient) as three signed
-//     8-bit digits per head (21-bit fixed point);
-//   - values: D(16 x 8 coords) += A(16 x 32 tokens) B(32 tokens x 8 coords,
-//     0/1) where A holds the softmax weights as three 8-bit digits per head.
-// * The 0/1 operands come straight from the packed words: one shift and one
-//   mask give four elements (bits t, t+8, t+16, t+24 of a word), so keys read
-//   one record per token and values read the block-32 layout (bits of 32
-//   tokens of one coordinate in a word).  The K-element order this implies is
-//   folded into the precomputed query fragments and the weight fragments.
-// * Per CTA: one (split, KV head, sequence); 256-token sub-chunks staged by
-//   1-D bulk copies into double-buffered shared memory; phase K (logits),
-//   phase S (softmax statistics, weight digits), phase V (value sums, int32
-//   per sub-chunk, merged into fp32 with the running-max rescale).
+//   contractions run as exact integer tensor-core products (m16n8k32):
+//   - keys:   D(16 tokens x 8) += A(16 tokens x 32 coords) B(32 coords x 8),
+//     B = the query (times the plane coefficient) in four signed base-128
+//     digits per head;
+//   - values: D(16 x 8 coords) += A(16 x 32 tokens) B(32 tokens x 8 coords),
+//     A = the softmax weights in four unsigned base-256 digits per head.
+// * The 0/1 operand is one AND of a packed word with a per-lane mask: byte
+//   i of (w & (0x01010101 << s)) is bit s + 8i of w, valued 2^s.  The
+//   factor 2^s is taken out on the other operand, which carries 2^(7 - s)
+//   (so every product is 2^7 times the intended one).
+// * The weight digits are the four bytes of one integer conversion,
+//   round(w 2^(7-s)/sigma) < 2^31 (s = 7 keeps 24 bits of the largest weight
+//   of the sub-chunk).
+// * A persistent grid walks (stream, split) items; per item, sub-chunks of
+//   TC tokens stream through two shared-memory stages by 1-D bulk copies;
+//   per sub-chunk: phase K (logits), phase S (softmax statistics and weight
+//   digits), phase V (value sums, int32 per sub-chunk, merged into fp32 with
+//   the running-max rescale).
 // * Every mbarrier wait is bounded; all threads take the same decision.
 #include <cfloat>
 
@@ -40,19 +43,31 @@ namespace {
 
 constexpr int kThreads = 128;                           // 4 warps
 constexpr float kSqrtHalfPi = 1.2533141373155002512f;  // sqrt(pi/2)
-constexpr float kDigitRange = 2.0e6f;                   // |X| <= 2e6 < 2^21: three balanced int8 digits
+constexpr float kQRange = 1.3e8f;                       // |X| <= 1.3e8: four balanced base-128 digits
+constexpr float kWCap = 2.0e9f;                         // weight integers stay below 2^31
+constexpr uint32_t kLowBits = 0x01010101u;
 
 template <int D>
 struct DTile {
     static constexpr int TC = (D == 256) ? 128 : 256;  // tokens per sub-chunk
 };
 
-// Balanced base-128 digits of an integer |X| <= kDigitRange: X = d0 2^14 + d1 2^7 + d2.
-__device__ __forceinline__ void digits3(int X, int& d0, int& d1, int& d2) {
-    d2 = ((X + 64) & 127) - 64;
-    const int X1 = (X - d2) >> 7;
-    d1 = ((X1 + 64) & 127) - 64;
-    d0 = (X1 - d1) >> 7;
+template <int G>
+struct HeadCfg {
+    static constexpr int NTK = (G <= 4) ? 2 : 4;  // key n-tiles: 4 digit columns per head
+    static constexpr int RT = (G <= 4) ? 1 : 2;   // value m-tiles: 4 digit rows per head
+    static constexpr int GP = (G <= 4) ? 4 : 8;   // heads incl. padding
+    static constexpr int CPL = (G <= 4) ? 1 : 2;  // value columns merged per lane
+};
+
+// Balanced base-128 digits of |X| <= kQRange: X = d0 2^21 + d1 2^14 + d2 2^7 + d3.
+__device__ __forceinline__ void digits4(int X, int (&d)[4]) {
+    d[3] = ((X + 64) & 127) - 64;
+    X = (X - d[3]) >> 7;
+    d[2] = ((X + 64) & 127) - 64;
+    X = (X - d[2]) >> 7;
+    d[1] = ((X + 64) & 127) - 64;
+    d[0] = (X - d[1]) >> 7;
 }
 
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
@@ -72,32 +87,35 @@ __device__ __forceinline__ float load_elem(const void* p, int64_t i) {
     return __uint_as_float(static_cast<uint32_t>(u) << 16);
 }
 
-// Key-side column map of the query fragments: n-tile nt, column n -> (head,
-// digit) or -1 for padding.  With G <= 4 thread t of the MMA ends up with
-// head t (columns 2t, 2t+1 of n-tile 0 = digits 0, 1; column 2t of n-tile 1 =
-// digit 2); with G = 8 it gets heads t and t+4.
-template <int G>
-__device__ __forceinline__ int key_col_head(int nt, int n, int* dig) {
-    if (G <= 4) {
-        if (nt == 0) { *dig = n & 1; return n >> 1; }
-        if (n & 1) return -1;
-        *dig = 2;
-        return n >> 1;
-    } else {
-        if (nt < 2) { *dig = n & 1; return (n >> 1) + 4 * nt; }
-        *dig = 2;
-        return (n >> 1) + 4 * (n & 1);
-    }
+// Warp-level integer products: d(16x8, s32) += a(16x32, u8, row) * b(32x8, s8 or u8, col).
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint2 b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y));
+}
+__device__ __forceinline__ void mma_u8u8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // Query preparation for one (sequence, KV head) group: q' = H (delta .* q),
-// p = S q' per query head, the three-digit fixed-point fragments of
-// coef_P q' (code planes) and p (QJL rows) in MMA B-fragment order, and the
-// per-head scalars {c0 sum q', sigma_code, sigma_qjl, sum p}.
+// p = S q' per query head, the digit fragments of coef_P q' (code planes)
+// and p (QJL rows) in MMA B-fragment order, and the per-head scalars
+// {c0 sum q', sigma_code/128, sigma_qjl/128, sum p}.
+//
+// B fragment of lane (g, t) in n-tile nt, K-step ks (32 coordinates 32w ..):
+// column g = (head (g >> 1) + 4 (nt >> 1), digit (g & 1) + 2 (nt & 1)); K
+// index 4t + i is coordinate 32w + t + 8i with factor 2^(7 - t), K index
+// 16 + 4t + i is coordinate 32w + t + 4 + 8i with factor 2^(3 - t).
 template <int D, int B, bool QJL, int G, int DT>
 __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int M = D;
-    constexpr int NTK = (G <= 4) ? 2 : 3;
+    constexpr int NTK = HeadCfg<G>::NTK;
     constexpr int KS = (B + (QJL ? 1 : 0)) * (D / 32);
     __shared__ float sq[G][D];
     __shared__ float sp[G][QJL ? M : 1];
@@ -136,7 +154,6 @@ __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__
     const float coef0 = a.centroid[1] - c0;
     const float coef1 = (B == 2) ? a.centroid[2] - c0 : 0.f;
     const float cmax = fmaxf(fabsf(coef0), fabsf(coef1));
-    // one warp per head: max |q'|, max |p|, sums
     for (int h = tid / 32; h < G; h += kThreads / 32) {
         const int ln = tid % 32;
         float mq = 0.f, mp = 0.f, s_q = 0.f, s_p = 0.f;
@@ -155,41 +172,41 @@ __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__
             s_p += __shfl_xor_sync(0xFFFFFFFFu, s_p, o);
         }
         if (ln == 0) {
-            const float sig_c = (mq * cmax > 0.f) ? mq * cmax / kDigitRange : 1.f;
-            const float sig_q = (mp > 0.f) ? mp / kDigitRange : 1.f;
+            // X = v 2^(7-s) / sig stays within kQRange for every s
+            const float sig_c = (mq * cmax > 0.f) ? mq * cmax * 128.f / kQRange : 1.f;
+            const float sig_q = (mp > 0.f) ? mp * 128.f / kQRange : 1.f;
             ssig[h][0] = sig_c;
             ssig[h][1] = sig_q;
             a.qscal[(qh0 + h) * 4 + 0] = c0 * s_q;
-            a.qscal[(qh0 + h) * 4 + 1] = sig_c;
-            a.qscal[(qh0 + h) * 4 + 2] = sig_q;
+            a.qscal[(qh0 + h) * 4 + 1] = sig_c * (1.f / 128.f);
+            a.qscal[(qh0 + h) * 4 + 2] = sig_q * (1.f / 128.f);
             a.qscal[(qh0 + h) * 4 + 3] = s_p;
         }
     }
     __syncthreads();
-    // B fragments: [k-step][n-tile][lane] of (b0, b1)
     uint2* frag = a.qfrag + static_cast<int64_t>(blockIdx.x) * KS * NTK * 32;
     for (int e = tid; e < KS * NTK * 32; e += kThreads) {
         const int lane = e % 32, nt = (e / 32) % NTK, ks = e / (32 * NTK);
         const int g = lane >> 2, t = lane & 3;
-        int dig = 0;
-        const int h = key_col_head<G>(nt, g, &dig);
+        const int h = (g >> 1) + 4 * (nt >> 1);
+        const int dig = (g & 1) + 2 * (nt & 1);
         uint32_t b[2] = {0u, 0u};
-        if (h >= 0 && h < G) {
+        if (h < G) {
             const int plane = ks / (D / 32), w = ks % (D / 32);
             const bool is_q = plane >= B;
             const float coef = (plane == 0) ? coef0 : coef1;
             const float sig = is_q ? ssig[h][1] : ssig[h][0];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
+                const float fac = static_cast<float>(1 << (7 - t - 4 * half));
                 int dd[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int j = 32 * w + t + 4 * half + 8 * i;
                     const float v = is_q ? sp[h][j] : coef * sq[h][j];
-                    const int X = __float2int_rn(v / sig);
-                    int d0, d1, d2;
-                    digits3(X, d0, d1, d2);
-                    dd[i] = dig == 0 ? d0 : (dig == 1 ? d1 : d2);
+                    int d4[4];
+                    digits4(__float2int_rn(v * fac / sig), d4);
+                    dd[i] = d4[dig];
                 }
                 b[half] = pack4(dd[0], dd[1], dd[2], dd[3]);
             }
@@ -203,10 +220,10 @@ template <int D, int B, bool QJL, int G>
 struct MmaSmem {
     static constexpr int M = D;
     static constexpr int TC = DTile<D>::TC;
-    static constexpr int NTK = (G <= 4) ? 2 : 3;
-    static constexpr int RT = (G <= 4) ? 1 : 2;
+    static constexpr int NTK = HeadCfg<G>::NTK;
+    static constexpr int RT = HeadCfg<G>::RT;
+    static constexpr int GP = HeadCfg<G>::GP;
     static constexpr int KS = (B + (QJL ? 1 : 0)) * (D / 32);
-    static constexpr int GP = (G <= 4) ? 4 : 8;            // heads incl. padding
     // staging of one sub-chunk
     static constexpr int kKc = TC * B * D / 8;             // key codes (token layout)
     static constexpr int kKq = QJL ? TC * M / 8 : 0;       // key sign bits
@@ -219,16 +236,19 @@ struct MmaSmem {
     static constexpr int kLog = GP * TC * 4;               // logits of the sub-chunk
     static constexpr int kWfrag = (TC / 32) * RT * 32 * 16;  // weight digits, per kind
     static constexpr int kBytes = 2 * kStage + kFrag + kLog + 2 * kWfrag + 1024;
+    static constexpr bool kQfReg = KS * NTK <= 24;         // query fragments held in registers
 };
 
 template <int D, int B, bool QJL, int G>
 __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_constant__ DecodeArgs a) {
     using L = MmaSmem<D, B, QJL, G>;
-    constexpr int M = D, TC = L::TC, NTK = L::NTK, RT = L::RT, KS = L::KS, GP = L::GP;
+    using HC = HeadCfg<G>;
+    constexpr int M = D, TC = L::TC, NTK = L::NTK, RT = L::RT, KS = L::KS, GP = L::GP, CPL = HC::CPL;
     constexpr int KWT = B * D / 32;           // code words per token (key layout)
     constexpr int QWT = QJL ? M / 32 : 0;     // sign words per token
-    constexpr int NTV = D / 32;               // value n-tiles per warp and plane (D/4 coordinates / 8)
+    constexpr int NTV = D / 32;               // value n-tiles per warp (D/4 coordinates / 8)
     constexpr int NPV = B + (QJL ? 1 : 0);
+    constexpr bool QF_REG = L::kQfReg;
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* stage[2] = {smem, smem + L::kStage};
     uint2* sfrag = reinterpret_cast<uint2*>(smem + 2 * L::kStage);
@@ -239,417 +259,508 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     uint64_t* bar = reinterpret_cast<uint64_t*>(misc);      // [2]
     float* sred = reinterpret_cast<float*>(misc + 16);      // [4 warps][GP][3]
     float* shead = sred + 4 * GP * 3;                        // [GP][8]: scalars, running state
+    float* sstat = shead + GP * 8;                           // [GP][8]: mnew, alpha, sig_w, sig_wq, inv_w, inv_wq
 
-    const int split = blockIdx.x, hk = blockIdx.y, bi = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int64_t T = min(static_cast<int64_t>(max(a.seq_len[bi], 0)), a.max_T);
-    const int64_t t0 = static_cast<int64_t>(split) * a.chunk;
-    const int64_t t1e = min(t0 + a.chunk, a.max_T);
-    const int64_t t1 = min(t1e, T);
-    const int64_t stream = static_cast<int64_t>(bi) * a.hkv + hk;
-    const int64_t qh0 = static_cast<int64_t>(bi) * a.hq + static_cast<int64_t>(hk) * G;
-    const int64_t grp = static_cast<int64_t>(bi) * a.hkv + hk;
-
-    // stream bases
-    const uint8_t* kc = reinterpret_cast<const uint8_t*>(a.kcodes) + stream * a.kcap * (B * D / 8);
-    const uint8_t* kq = QJL ? reinterpret_cast<const uint8_t*>(a.kqjl) + stream * a.kcap * (M / 8) : nullptr;
-    const uint8_t* kn = reinterpret_cast<const uint8_t*>(a.knorms) + stream * a.kcap * 4;
-    const uint8_t* vc = reinterpret_cast<const uint8_t*>(a.vcodes) + stream * (a.vcap / 32) * B * D * 4;
-    const uint8_t* vq = QJL ? reinterpret_cast<const uint8_t*>(a.vqjl) + stream * (a.vcap / 32) * M * 4 : nullptr;
-    const uint8_t* vn = reinterpret_cast<const uint8_t*>(a.vnorms) + stream * a.vcap * 4;
-
-    // ---- set-up: query fragments, per-head scalars, zero weight digits, barriers
-    {
-        const uint2* gf = a.qfrag + grp * KS * NTK * 32;
-        for (int e = tid; e < KS * NTK * 32; e += kThreads) sfrag[e] = gf[e];
-        for (int e = tid; e < 2 * L::kWfrag / 4; e += kThreads) swc[e] = 0u;
-        if (tid < GP) {
-            float* hs = shead + tid * 8;
-            if (tid < G) {
-                const float* qs = a.qscal + (qh0 + tid) * 4;
-                hs[0] = qs[0]; hs[1] = qs[1]; hs[2] = qs[2]; hs[3] = qs[3];
-            } else {
-                hs[0] = hs[1] = hs[2] = hs[3] = 0.f;
-            }
-            hs[4] = -INFINITY;  // running max
-            hs[5] = 0.f;        // running sum of exp
-            hs[6] = 0.f;        // running sum of code weights (Omega)
-            hs[7] = 0.f;        // running sum of QJL weights (Omega')
-        }
-        if (tid == 0) {
-            mbar_init(&bar[0], 1);
-            mbar_init(&bar[1], 1);
-            fence_mbar_init();
-        }
-    }
-    __syncthreads();
-
-    const int nsub = static_cast<int>((t1e - t0 + TC - 1) / TC);
-    // tokens of the sub-chunk that exist in the cache (rounded to whole blocks of 32)
-    auto issue = [&](int sc) {
-        const int64_t tb = t0 + static_cast<int64_t>(sc) * TC;
-        const int64_t have = min(static_cast<int64_t>(TC), t1 - tb);
-        if (have <= 0) return false;
-        const int64_t nt = (have + 31) / 32 * 32;  // <= capacity - tb (capacity is a multiple of 32)
-        uint8_t* st = stage[sc & 1];
-        uint64_t* b = &bar[sc & 1];
-        const uint32_t bytes = static_cast<uint32_t>(nt * (B * D / 8 + (QJL ? M / 8 : 0) + 4) +
-                                                     (nt / 32) * (B * D * 4 + (QJL ? M * 4 : 0)) + nt * 4);
-        mbar_arrive_expect_tx(b, bytes);
-        bulk_load(st, kc + tb * (B * D / 8), static_cast<uint32_t>(nt * (B * D / 8)), b);
-        if (QJL) bulk_load(st + L::kKc, kq + tb * (M / 8), static_cast<uint32_t>(nt * (M / 8)), b);
-        bulk_load(st + L::kKc + L::kKq, kn + tb * 4, static_cast<uint32_t>(nt * 4), b);
-        bulk_load(st + L::kKc + L::kKq + L::kKn, vc + (tb / 32) * B * D * 4, static_cast<uint32_t>((nt / 32) * B * D * 4),
-                  b);
-        if (QJL)
-            bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc, vq + (tb / 32) * M * 4,
-                      static_cast<uint32_t>((nt / 32) * M * 4), b);
-        bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq, vn + tb * 4, static_cast<uint32_t>(nt * 4), b);
-        return true;
-    };
-    bool armed0 = false, armed1 = false;
-    if (tid == 0) {
-        armed0 = issue(0);
-        armed1 = nsub > 1 ? issue(1) : false;
-    }
-    uint32_t phase[2] = {0u, 0u};
-    bool alive = true;
-
-    // fp32 running value sums: this thread's coordinates of warp `warp`
-    // (code part combined over planes; QJL part), head g (G <= 4, lanes g < 4)
-    // or head g (G = 8, all lanes).
-    float accA[NTV][2], accB[NTV][2];
-#pragma unroll
-    for (int nt = 0; nt < NTV; ++nt) accA[nt][0] = accA[nt][1] = accB[nt][0] = accB[nt][1] = 0.f;
-
+    const uint32_t msk_lo = kLowBits << t, msk_hi = kLowBits << (t + 4);
     const float kappa = kSqrtHalfPi / M;
     const float coef0 = a.centroid[1] - a.centroid[0];
     const float coef1 = (B == 2) ? a.centroid[2] - a.centroid[0] : 0.f;
 
-    for (int sc = 0; sc < nsub; ++sc) {
-        const int64_t tb = t0 + static_cast<int64_t>(sc) * TC;
-        const int64_t have = min(static_cast<int64_t>(TC), t1 - tb);  // may be <= 0 (split past the context)
-        const uint8_t* st = stage[sc & 1];
-        if (have > 0) {
-            const bool ok = mbar_wait(&bar[sc & 1], phase[sc & 1], a.status);
-            phase[sc & 1] ^= 1u;
-            if (__syncthreads_or(!ok)) { alive = false; break; }
-        }
-        const uint32_t* sKc = reinterpret_cast<const uint32_t*>(st);
-        const uint32_t* sKq = reinterpret_cast<const uint32_t*>(st + L::kKc);
-        const __half2* sKn = reinterpret_cast<const __half2*>(st + L::kKc + L::kKq);
-        const uint32_t* sVc = reinterpret_cast<const uint32_t*>(st + L::kKc + L::kKq + L::kKn);
-        const uint32_t* sVq = reinterpret_cast<const uint32_t*>(st + L::kKc + L::kKq + L::kKn + L::kVc);
-        const __half2* sVn = reinterpret_cast<const __half2*>(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq);
-
-        // ---------------- phase K: logits of the sub-chunk ----------------
-        for (int mt = warp; mt < TC / 16; mt += 4) {
-            const int tl0 = mt * 16 + g, tl1 = tl0 + 8;
-            int accc[NTK][4], accq[NTK][4];
-#pragma unroll
-            for (int nt = 0; nt < NTK; ++nt)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) accc[nt][r] = accq[nt][r] = 0;
-            if (tb + mt * 16 < t1) {
-#pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    const bool is_q = ks >= B * (D / 32);
-                    uint32_t w0, w1;
-                    if (!is_q) {
-                        w0 = sKc[tl0 * KWT + ks];
-                        w1 = sKc[tl1 * KWT + ks];
-                    } else {
-                        w0 = sKq[tl0 * QWT + (ks - B * (D / 32))];
-                        w1 = sKq[tl1 * QWT + (ks - B * (D / 32))];
-                    }
-                    const uint32_t af[4] = {(w0 >> t) & 0x01010101u, (w1 >> t) & 0x01010101u,
-                                            (w0 >> (t + 4)) & 0x01010101u, (w1 >> (t + 4)) & 0x01010101u};
-#pragma unroll
-                    for (int nt = 0; nt < NTK; ++nt) {
-                        const uint2 bq = sfrag[(ks * NTK + nt) * 32 + lane];
-                        if (!is_q) mma_s8_16832(accc[nt], af, bq.x, bq.y);
-                        else mma_s8_16832(accq[nt], af, bq.x, bq.y);
-                    }
-                }
-            }
-            // epilogue: thread t owns head t (and t + 4 when G = 8)
-#pragma unroll
-            for (int hh = 0; hh < (G == 8 ? 2 : 1); ++hh) {
-                const int h = t + 4 * hh;
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int tl = rr ? tl1 : tl0;
-                    const int64_t tg = tb + tl;
-                    float l = -INFINITY;
-                    if (h < G && tg < t1) {
-                        int ci, qi;
-                        if (G <= 4) {
-                            ci = accc[0][2 * rr] * 16384 + accc[0][2 * rr + 1] * 128 + accc[1][2 * rr];
-                            qi = accq[0][2 * rr] * 16384 + accq[0][2 * rr + 1] * 128 + accq[1][2 * rr];
-                        } else {
-                            ci = accc[hh][2 * rr] * 16384 + accc[hh][2 * rr + 1] * 128 + accc[2][2 * rr + hh];
-                            qi = accq[hh][2 * rr] * 16384 + accq[hh][2 * rr + 1] * 128 + accq[2][2 * rr + hh];
-                        }
-                        const float* hs = shead + h * 8;
-                        const float2 nk = __half22float2(sKn[tl]);
-                        float dot = hs[0] + hs[1] * static_cast<float>(ci);
-                        if (QJL) dot += kappa * nk.y * (2.f * hs[2] * static_cast<float>(qi) - hs[3]);
-                        l = a.scale * (nk.x / D) * dot;
-                    }
-                    if (h < GP) slog[h * TC + tl] = l;
-                    if (a.logits != nullptr && h < G && tg < t1e) a.logits[(qh0 + h) * a.max_T + tg] = l;
-                }
-            }
-        }
-        __syncthreads();
-
-        // ---------------- phase S: softmax statistics and weight digits ----------------
-        // pass 1: per head, the max logit and the max of l + log(n) (and of
-        // l + log(n gamma)): the largest weight of the sub-chunk, which sets
-        // the scale of its weight digits (so that small weights keep their
-        // resolution when the sub-chunk sits far below the running max).
-        {
-            float mx[GP], mw[GP], mq[GP];
-#pragma unroll
-            for (int h = 0; h < GP; ++h) mx[h] = mw[h] = mq[h] = -INFINITY;
-            for (int tl = tid; tl < TC; tl += kThreads) {
-                if (tb + tl < t1) {
-                    const float2 nv = __half22float2(sVn[tl]);
-                    const float ln = __logf(nv.x), lg = __logf(nv.x * nv.y);
-#pragma unroll
-                    for (int h = 0; h < GP; ++h) {
-                        const float l = slog[h * TC + tl];
-                        mx[h] = fmaxf(mx[h], l);
-                        mw[h] = fmaxf(mw[h], l + ln);
-                        mq[h] = fmaxf(mq[h], l + lg);
-                    }
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-                for (int h = 0; h < GP; ++h) {
-                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], o));
-                    mw[h] = fmaxf(mw[h], __shfl_xor_sync(0xFFFFFFFFu, mw[h], o));
-                    mq[h] = fmaxf(mq[h], __shfl_xor_sync(0xFFFFFFFFu, mq[h], o));
-                }
-            }
-            if (lane == 0) {
-#pragma unroll
-                for (int h = 0; h < GP; ++h) {
-                    sred[(warp * GP + h) * 3 + 0] = mx[h];
-                    sred[(warp * GP + h) * 3 + 1] = mw[h];
-                    sred[(warp * GP + h) * 3 + 2] = mq[h];
-                }
-            }
-        }
-        __syncthreads();
-        // per-head new running max, rescale factor and weight-digit scales
-        float* sstat = shead + GP * 8;  // [GP][4]: mnew, alpha, sig_w, sig_wq
-        if (tid < GP) {
-            const int h = tid;
-            float mx = -INFINITY, mw = -INFINITY, mq = -INFINITY;
-            for (int w = 0; w < 4; ++w) {
-                mx = fmaxf(mx, sred[(w * GP + h) * 3 + 0]);
-                mw = fmaxf(mw, sred[(w * GP + h) * 3 + 1]);
-                mq = fmaxf(mq, sred[(w * GP + h) * 3 + 2]);
-            }
-            float* hs = shead + h * 8;
-            const float mold = hs[4];
-            const float mnew = fmaxf(mold, mx);
-            const float alpha = (mnew == -INFINITY) ? 1.f : __expf(mold - mnew);
-            hs[4] = mnew;
-            const float wmax = (mw == -INFINITY) ? 0.f : __expf(mw - mnew);
-            const float qmax = (mq == -INFINITY) ? 0.f : __expf(mq - mnew);
-            sstat[h * 4 + 0] = mnew;
-            sstat[h * 4 + 1] = alpha;
-            sstat[h * 4 + 2] = wmax > 0.f ? wmax / kDigitRange : 1.f;
-            sstat[h * 4 + 3] = qmax > 0.f ? qmax / kDigitRange : 1.f;
-        }
-        __syncthreads();
-        // pass 2: weight digits into A-fragment order; sums of exp and weights
-        {
-            float sum_e[GP], sum_w[GP], sum_wq[GP];
-#pragma unroll
-            for (int h = 0; h < GP; ++h) sum_e[h] = sum_w[h] = sum_wq[h] = 0.f;
-            for (int tl = tid; tl < TC; tl += kThreads) {
-                const bool valid = tb + tl < t1;
-                const float2 nv = valid ? __half22float2(sVn[tl]) : make_float2(0.f, 0.f);
-                // K-element of token u in its block: u = t' + 8 i (+4 for the second half)
-                const int u = tl & 31, bb = tl >> 5;
-                const int tp = u & 3, half = (u >> 2) & 1, i = u >> 3;
-#pragma unroll
-                for (int h = 0; h < GP; ++h) {
-                    float wc = 0.f, wq = 0.f;
-                    if (valid && h < G) {
-                        const float e = __expf(slog[h * TC + tl] - sstat[h * 4 + 0]);
-                        sum_e[h] += e;
-                        wc = e * nv.x;
-                        wq = wc * nv.y;
-                        sum_w[h] += wc;
-                        sum_wq[h] += wq;
-                    }
-                    int dc[3], dq[3];
-                    const int xc = min(__float2int_rn(wc / sstat[h * 4 + 2]), static_cast<int>(kDigitRange) + 4096);
-                    const int xq = min(__float2int_rn(wq / sstat[h * 4 + 3]), static_cast<int>(kDigitRange) + 4096);
-                    digits3(xc, dc[0], dc[1], dc[2]);
-                    digits3(xq, dq[0], dq[1], dq[2]);
-#pragma unroll
-                    for (int dg = 0; dg < 3; ++dg) {
-                        // row r of the weight operand: G <= 4: r = h + 4 dg (one row tile);
-                        // G = 8: r = h + 8 dg (rows 16..23 -> second row tile)
-                        const int r = (G <= 4) ? h + 4 * dg : h + 8 * dg;
-                        const int rt = r >> 4, rl = r & 15;
-                        const int ln = 4 * (rl & 7) + tp;
-                        const int reg = (rl >> 3) + 2 * half;
-                        const int byte = ((((bb * RT + rt) * 32 + ln) * 4 + reg) << 2) + i;
-                        reinterpret_cast<uint8_t*>(swc)[byte] = static_cast<uint8_t>(dc[dg]);
-                        if (QJL) reinterpret_cast<uint8_t*>(swq)[byte] = static_cast<uint8_t>(dq[dg]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                for (int h = 0; h < GP; ++h) {
-                    sum_e[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_e[h], o);
-                    sum_w[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_w[h], o);
-                    sum_wq[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_wq[h], o);
-                }
-            if (lane == 0)
-#pragma unroll
-                for (int h = 0; h < GP; ++h) {
-                    sred[(warp * GP + h) * 3 + 0] = sum_e[h];
-                    sred[(warp * GP + h) * 3 + 1] = sum_w[h];
-                    sred[(warp * GP + h) * 3 + 2] = sum_wq[h];
-                }
-        }
-        __syncthreads();
-        if (tid < GP) {
-            const int h = tid;
-            float te = 0.f, tw = 0.f, twq = 0.f;
-            for (int w = 0; w < 4; ++w) {
-                te += sred[(w * GP + h) * 3 + 0];
-                tw += sred[(w * GP + h) * 3 + 1];
-                twq += sred[(w * GP + h) * 3 + 2];
-            }
-            float* hs = shead + h * 8;
-            const float alpha = sstat[h * 4 + 1];
-            hs[5] = hs[5] * alpha + te;
-            hs[6] = hs[6] * alpha + tw;
-            hs[7] = hs[7] * alpha + twq;
-        }
-
-        // ---------------- phase V: value sums of the sub-chunk ----------------
-        {
-            int accv[NPV][NTV][RT][4];
-#pragma unroll
-            for (int p = 0; p < NPV; ++p)
-#pragma unroll
-                for (int nt = 0; nt < NTV; ++nt)
-#pragma unroll
-                    for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) accv[p][nt][rt][r] = 0;
-            const int nblk = have > 0 ? static_cast<int>((have + 31) / 32) : 0;
-            for (int bb = 0; bb < nblk; ++bb) {
-                uint32_t aw[RT][4], aq[RT][4];
-#pragma unroll
-                for (int rt = 0; rt < RT; ++rt) {
-                    const uint4 x = reinterpret_cast<const uint4*>(swc)[(bb * RT + rt) * 32 + lane];
-                    aw[rt][0] = x.x; aw[rt][1] = x.y; aw[rt][2] = x.z; aw[rt][3] = x.w;
-                    if (QJL) {
-                        const uint4 y = reinterpret_cast<const uint4*>(swq)[(bb * RT + rt) * 32 + lane];
-                        aq[rt][0] = y.x; aq[rt][1] = y.y; aq[rt][2] = y.z; aq[rt][3] = y.w;
-                    }
-                }
-#pragma unroll
-                for (int p = 0; p < NPV; ++p) {
-#pragma unroll
-                    for (int nt = 0; nt < NTV; ++nt) {
-                        const int coord = warp * (D / 4) + nt * 8 + g;
-                        const uint32_t wv = (p < B) ? sVc[(bb * B + p) * D + coord] : sVq[bb * M + coord];
-                        const uint32_t b0 = (wv >> t) & 0x01010101u, b1 = (wv >> (t + 4)) & 0x01010101u;
-#pragma unroll
-                        for (int rt = 0; rt < RT; ++rt) {
-                            if (p < B) mma_s8_16832(accv[p][nt][rt], aw[rt], b0, b1);
-                            else mma_s8_16832(accv[p][nt][rt], aq[rt], b0, b1);
-                        }
-                    }
-                }
-            }
-            // merge into the fp32 running sums (rescaled by alpha of this sub-chunk)
-#pragma unroll
-            for (int nt = 0; nt < NTV; ++nt) {
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    int vi[NPV];
-                    int head;
-#pragma unroll
-                    for (int p = 0; p < NPV; ++p) {
-                        if (G <= 4) {
-                            // rows g (digit 0 or 1, head g & 3) and g + 8 (digit 2 or pad)
-                            const int d1 = __shfl_xor_sync(0xFFFFFFFFu, accv[p][nt][0][c], 16);
-                            vi[p] = accv[p][nt][0][c] * 16384 + d1 * 128 + accv[p][nt][0][2 + c];
-                        } else {
-                            vi[p] = accv[p][nt][0][c] * 16384 + accv[p][nt][0][2 + c] * 128 + accv[p][nt][1][c];
-                        }
-                    }
-                    head = g;
-                    const bool own = (G <= 4) ? (g < 4) : true;
-                    if (own && head < G) {
-                        const float alpha = sstat[head * 4 + 1];
-                        const float sgw = sstat[head * 4 + 2], sgq = sstat[head * 4 + 3];
-                        float code = coef0 * static_cast<float>(vi[0]);
-                        if (B == 2) code += coef1 * static_cast<float>(vi[1 % NPV]);
-                        accA[nt][c] = accA[nt][c] * alpha + sgw * code;
-                        if (QJL) accB[nt][c] = accB[nt][c] * alpha + sgq * 2.f * static_cast<float>(vi[NPV - 1]);
-                    }
-                }
-            }
-        }
-        __syncthreads();  // stage and weight digits are reused by the next sub-chunk
-        if (tid == 0 && sc + 2 < nsub) {
-            if (sc & 1) armed1 = issue(sc + 2);
-            else armed0 = issue(sc + 2);
-        }
-    }
+    for (int e = tid; e < 2 * L::kWfrag / 4; e += kThreads) swc[e] = 0u;  // padding rows stay zero
     if (tid == 0) {
-        // loads in flight are waited for before exit (only when a wait gave up)
-        if (!alive) {
-            if (armed0) mbar_wait(&bar[0], phase[0], a.status);
-            if (armed1) mbar_wait(&bar[1], phase[1], a.status);
-        }
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
     }
+    uint32_t phase[2] = {0u, 0u};
+    bool alive = true;
+    const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit;
 
-    // ---------------- partials: {M, L, A[D], B[M]} per query head ----------------
-    constexpr int PART = 2 + D + M;
-    const bool own = (G <= 4) ? (g < 4) : true;
-    const int head = g;
-    if (own && head < G) {
-        float* pp = a.part + ((qh0 + head) * a.nsplit + split) * PART;
-        const float* hs = shead + head * 8;
-        const float c0 = a.centroid[0];
+    for (int64_t item = blockIdx.x; item < items && alive; item += gridDim.x) {
+        const int split = static_cast<int>(item % a.nsplit);
+        const int64_t stream = item / a.nsplit;
+        const int hk = static_cast<int>(stream % a.hkv), bi = static_cast<int>(stream / a.hkv);
+        const int64_t T = min(static_cast<int64_t>(max(a.seq_len[bi], 0)), a.max_T);
+        const int64_t t0 = static_cast<int64_t>(split) * a.chunk;
+        const int64_t t1e = min(t0 + a.chunk, a.max_T);
+        const int64_t t1 = min(t1e, T);
+        const int64_t qh0 = static_cast<int64_t>(bi) * a.hq + static_cast<int64_t>(hk) * G;
+        const uint8_t* kc = reinterpret_cast<const uint8_t*>(a.kcodes) + stream * a.kcap * (B * D / 8);
+        const uint8_t* kq = QJL ? reinterpret_cast<const uint8_t*>(a.kqjl) + stream * a.kcap * (M / 8) : nullptr;
+        const uint8_t* kn = reinterpret_cast<const uint8_t*>(a.knorms) + stream * a.kcap * 4;
+        const uint8_t* vc = reinterpret_cast<const uint8_t*>(a.vcodes) + stream * (a.vcap / 32) * B * D * 4;
+        const uint8_t* vq = QJL ? reinterpret_cast<const uint8_t*>(a.vqjl) + stream * (a.vcap / 32) * M * 4 : nullptr;
+        const uint8_t* vn = reinterpret_cast<const uint8_t*>(a.vnorms) + stream * a.vcap * 4;
+
+        // ---- item set-up (the previous item is done with shared memory) ----
+        __syncthreads();
+        {
+            const uint2* gf = a.qfrag + stream * KS * NTK * 32;
+            for (int e = tid; e < KS * NTK * 32; e += kThreads) sfrag[e] = gf[e];
+            if (tid < GP) {
+                float* hs = shead + tid * 8;
+                if (tid < G) {
+                    const float* qs = a.qscal + (qh0 + tid) * 4;
+                    hs[0] = qs[0]; hs[1] = qs[1]; hs[2] = qs[2]; hs[3] = qs[3];
+                } else {
+                    hs[0] = hs[1] = hs[2] = hs[3] = 0.f;
+                }
+                hs[4] = -INFINITY;  // running max
+                hs[5] = 0.f;        // running sum of exp
+                hs[6] = 0.f;        // running sum of code weights (Omega)
+                hs[7] = 0.f;        // running sum of QJL weights (Omega')
+            }
+        }
+        const int nsub = static_cast<int>((t1e - t0 + TC - 1) / TC);
+        // tokens of the sub-chunk that exist in the cache (rounded to whole blocks of 32)
+        auto issue = [&](int sc) {
+            const int64_t tb = t0 + static_cast<int64_t>(sc) * TC;
+            const int64_t have = min(static_cast<int64_t>(TC), t1 - tb);
+            if (have <= 0) return false;
+            const int64_t nt = (have + 31) / 32 * 32;  // <= capacity - tb (capacity is a multiple of 32)
+            uint8_t* st = stage[sc & 1];
+            uint64_t* b = &bar[sc & 1];
+            const uint32_t bytes = static_cast<uint32_t>(nt * (B * D / 8 + (QJL ? M / 8 : 0) + 4) +
+                                                         (nt / 32) * (B * D * 4 + (QJL ? M * 4 : 0)) + nt * 4);
+            mbar_arrive_expect_tx(b, bytes);
+            bulk_load(st, kc + tb * (B * D / 8), static_cast<uint32_t>(nt * (B * D / 8)), b);
+            if (QJL) bulk_load(st + L::kKc, kq + tb * (M / 8), static_cast<uint32_t>(nt * (M / 8)), b);
+            bulk_load(st + L::kKc + L::kKq, kn + tb * 4, static_cast<uint32_t>(nt * 4), b);
+            bulk_load(st + L::kKc + L::kKq + L::kKn, vc + (tb / 32) * B * D * 4,
+                      static_cast<uint32_t>((nt / 32) * B * D * 4), b);
+            if (QJL)
+                bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc, vq + (tb / 32) * M * 4,
+                          static_cast<uint32_t>((nt / 32) * M * 4), b);
+            bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq, vn + tb * 4, static_cast<uint32_t>(nt * 4),
+                      b);
+            return true;
+        };
+        bool armed0 = false, armed1 = false;
+        if (tid == 0) {
+            armed0 = issue(0);
+            armed1 = nsub > 1 ? issue(1) : false;
+        }
+        __syncthreads();
+        uint2 qf[QF_REG ? KS : 1][QF_REG ? NTK : 1];
+        if (QF_REG) {
+#pragma unroll
+            for (int ks = 0; ks < (QF_REG ? KS : 1); ++ks)
+#pragma unroll
+                for (int nt = 0; nt < (QF_REG ? NTK : 1); ++nt) qf[ks][nt] = sfrag[(ks * NTK + nt) * 32 + lane];
+        }
+
+        // fp32 running value sums of this lane's (head, coordinate) pairs
+        float accA[NTV][CPL], accB[NTV][CPL];
 #pragma unroll
         for (int nt = 0; nt < NTV; ++nt)
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int coord = warp * (D / 4) + nt * 8 + 2 * t + c;
-                pp[2 + coord] = c0 * hs[6] + accA[nt][c];
-                if (QJL) pp[2 + D + coord] = accB[nt][c] - hs[7];
+            for (int c = 0; c < CPL; ++c) accA[nt][c] = accB[nt][c] = 0.f;
+
+        for (int sc = 0; sc < nsub; ++sc) {
+            const int64_t tb = t0 + static_cast<int64_t>(sc) * TC;
+            const int64_t have = min(static_cast<int64_t>(TC), t1 - tb);  // may be <= 0 (split past the context)
+            const uint8_t* st = stage[sc & 1];
+            if (have > 0) {
+                const bool ok = mbar_wait(&bar[sc & 1], phase[sc & 1], a.status);
+                phase[sc & 1] ^= 1u;
+                if (__syncthreads_or(!ok)) { alive = false; break; }
             }
-    }
-    if (tid < G) {
-        float* pp = a.part + ((qh0 + tid) * a.nsplit + split) * PART;
-        pp[0] = shead[tid * 8 + 4];
-        pp[1] = shead[tid * 8 + 5];
+            const uint32_t* sKc = reinterpret_cast<const uint32_t*>(st);
+            const uint32_t* sKq = reinterpret_cast<const uint32_t*>(st + L::kKc);
+            const __half2* sKn = reinterpret_cast<const __half2*>(st + L::kKc + L::kKq);
+            const uint32_t* sVc = reinterpret_cast<const uint32_t*>(st + L::kKc + L::kKq + L::kKn);
+            const uint32_t* sVq = reinterpret_cast<const uint32_t*>(st + L::kKc + L::kKq + L::kKn + L::kVc);
+            const __half2* sVn = reinterpret_cast<const __half2*>(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq);
+
+            // ---------------- phase K: logits of the sub-chunk ----------------
+            for (int mt = warp; mt < TC / 16; mt += 4) {
+                const int tl0 = mt * 16 + g, tl1 = tl0 + 8;
+                int accc[2][NTK][4], accq[2][NTK][4];  // even / odd K-steps (two dependency chains)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int nt = 0; nt < NTK; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) accc[e][nt][r] = accq[e][nt][r] = 0;
+                if (tb + mt * 16 < t1) {
+                    uint32_t w0[KS], w1[KS];
+#pragma unroll
+                    for (int q4 = 0; q4 < KWT / 4; ++q4) {
+                        const uint4 x0 = reinterpret_cast<const uint4*>(sKc + tl0 * KWT)[q4];
+                        const uint4 x1 = reinterpret_cast<const uint4*>(sKc + tl1 * KWT)[q4];
+                        w0[4 * q4] = x0.x; w0[4 * q4 + 1] = x0.y; w0[4 * q4 + 2] = x0.z; w0[4 * q4 + 3] = x0.w;
+                        w1[4 * q4] = x1.x; w1[4 * q4 + 1] = x1.y; w1[4 * q4 + 2] = x1.z; w1[4 * q4 + 3] = x1.w;
+                    }
+#pragma unroll
+                    for (int k = KWT / 4 * 4; k < KWT; ++k) {
+                        w0[k] = sKc[tl0 * KWT + k];
+                        w1[k] = sKc[tl1 * KWT + k];
+                    }
+                    if (QJL) {
+#pragma unroll
+                        for (int k = 0; k < QWT; k += 2) {
+                            const uint2 x0 = reinterpret_cast<const uint2*>(sKq + tl0 * QWT)[k / 2];
+                            const uint2 x1 = reinterpret_cast<const uint2*>(sKq + tl1 * QWT)[k / 2];
+                            w0[KWT + k] = x0.x; w0[KWT + k + 1] = x0.y;
+                            w1[KWT + k] = x1.x; w1[KWT + k + 1] = x1.y;
+                        }
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) {
+                        const uint32_t af[4] = {w0[ks] & msk_lo, w1[ks] & msk_lo, w0[ks] & msk_hi, w1[ks] & msk_hi};
+#pragma unroll
+                        for (int nt = 0; nt < NTK; ++nt) {
+                            const uint2 bq = QF_REG ? qf[QF_REG ? ks : 0][QF_REG ? nt : 0]
+                                                    : sfrag[(ks * NTK + nt) * 32 + lane];
+                            if (ks < B * (D / 32)) mma_u8s8(accc[ks & 1][nt], af, bq);
+                            else mma_u8s8(accq[ks & 1][nt], af, bq);
+                        }
+                    }
+                }
+                // epilogue: thread t owns head t (and t + 4 when G = 8); its
+                // columns hold the four digits of the head
+#pragma unroll
+                for (int hh = 0; hh < (G == 8 ? 2 : 1); ++hh) {
+                    const int h = t + 4 * hh;
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int tl = rr ? tl1 : tl0;
+                        const int64_t tg = tb + tl;
+                        float l = -INFINITY;
+                        if (h < G && tg < t1) {
+                            const int n0 = 2 * hh, n1 = 2 * hh + 1;
+                            const int c_hi = (accc[0][n0][2 * rr] + accc[1][n0][2 * rr]) * 128 +
+                                             accc[0][n0][2 * rr + 1] + accc[1][n0][2 * rr + 1];
+                            const int c_lo = (accc[0][n1][2 * rr] + accc[1][n1][2 * rr]) * 128 +
+                                             accc[0][n1][2 * rr + 1] + accc[1][n1][2 * rr + 1];
+                            const float xc = fmaf(static_cast<float>(c_hi), 16384.f, static_cast<float>(c_lo));
+                            const float* hs = shead + h * 8;
+                            const float2 nk = __half22float2(sKn[tl]);
+                            float dot = fmaf(hs[1], xc, hs[0]);
+                            if (QJL) {
+                                const int q_hi = (accq[0][n0][2 * rr] + accq[1][n0][2 * rr]) * 128 +
+                                                 accq[0][n0][2 * rr + 1] + accq[1][n0][2 * rr + 1];
+                                const int q_lo = (accq[0][n1][2 * rr] + accq[1][n1][2 * rr]) * 128 +
+                                                 accq[0][n1][2 * rr + 1] + accq[1][n1][2 * rr + 1];
+                                const float xq = fmaf(static_cast<float>(q_hi), 16384.f, static_cast<float>(q_lo));
+                                dot += kappa * nk.y * (2.f * hs[2] * xq - hs[3]);
+                            }
+                            l = a.scale * (nk.x / D) * dot;
+                        }
+                        if (h < GP) slog[h * TC + tl] = l;
+                        if (a.logits != nullptr && h < G && tg < t1e) a.logits[(qh0 + h) * a.max_T + tg] = l;
+                    }
+                }
+            }
+            __syncthreads();
+
+            // ---------------- phase S: softmax statistics and weight digits ----------------
+            // pass 1: per head, the max logit and the max of l + log(n) (and of
+            // l + log(n gamma)): the largest weight of the sub-chunk, which sets
+            // the scale of its weight digits.
+            {
+                float mx[GP], mw[GP], mq[GP];
+#pragma unroll
+                for (int h = 0; h < GP; ++h) mx[h] = mw[h] = mq[h] = -INFINITY;
+                for (int tl = tid; tl < TC; tl += kThreads) {
+                    if (tb + tl < t1) {
+                        const float2 nv = __half22float2(sVn[tl]);
+                        const float ln = __logf(nv.x), lg = __logf(nv.x * nv.y);
+#pragma unroll
+                        for (int h = 0; h < GP; ++h) {
+                            const float l = slog[h * TC + tl];
+                            mx[h] = fmaxf(mx[h], l);
+                            mw[h] = fmaxf(mw[h], l + ln);
+                            mq[h] = fmaxf(mq[h], l + lg);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+                    for (int h = 0; h < GP; ++h) {
+                        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], o));
+                        mw[h] = fmaxf(mw[h], __shfl_xor_sync(0xFFFFFFFFu, mw[h], o));
+                        mq[h] = fmaxf(mq[h], __shfl_xor_sync(0xFFFFFFFFu, mq[h], o));
+                    }
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int h = 0; h < GP; ++h) {
+                        sred[(warp * GP + h) * 3 + 0] = mx[h];
+                        sred[(warp * GP + h) * 3 + 1] = mw[h];
+                        sred[(warp * GP + h) * 3 + 2] = mq[h];
+                    }
+                }
+            }
+            __syncthreads();
+            // per-head new running max, rescale factor and weight-digit scales:
+            // weight w is the integer X = w 2^(7-s) inv < kWCap, and a value
+            // sum S of the MMA stands for S sig / 128 with sig = 1 / inv
+            if (tid < GP) {
+                const int h = tid;
+                float mx = -INFINITY, mw = -INFINITY, mq = -INFINITY;
+                for (int w = 0; w < 4; ++w) {
+                    mx = fmaxf(mx, sred[(w * GP + h) * 3 + 0]);
+                    mw = fmaxf(mw, sred[(w * GP + h) * 3 + 1]);
+                    mq = fmaxf(mq, sred[(w * GP + h) * 3 + 2]);
+                }
+                float* hs = shead + h * 8;
+                const float mold = hs[4];
+                const float mnew = fmaxf(mold, mx);
+                const float alpha = (mnew == -INFINITY) ? 1.f : __expf(mold - mnew);
+                hs[4] = mnew;
+                const float wmax = (mw == -INFINITY) ? 0.f : __expf(mw - mnew);
+                const float qmax = (mq == -INFINITY) ? 0.f : __expf(mq - mnew);
+                float* ss = sstat + h * 8;
+                ss[0] = mnew;
+                ss[1] = alpha;
+                ss[2] = wmax * (128.f / kWCap);
+                ss[3] = qmax * (128.f / kWCap);
+                ss[4] = wmax > 0.f ? kWCap / (128.f * wmax) : 0.f;
+                ss[5] = qmax > 0.f ? kWCap / (128.f * qmax) : 0.f;
+            }
+            __syncthreads();
+            // pass 2: weight digits into A-fragment bytes; sums of exp and weights.
+            // Token u of block bb is K index 4(u&7) + (u>>3) (u&7 < 4) or
+            // 16 + 4((u&7)-4) + (u>>3): lane 4(r&7) + (u&3), register
+            // (r>>3) + 2((u&7)>>2), byte u>>3 of row r's fragment.
+            {
+                float sum_e[GP], sum_w[GP], sum_wq[GP];
+#pragma unroll
+                for (int h = 0; h < GP; ++h) sum_e[h] = sum_w[h] = sum_wq[h] = 0.f;
+                for (int tl = tid; tl < TC; tl += kThreads) {
+                    const bool valid = tb + tl < t1;
+                    const float2 nv = valid ? __half22float2(sVn[tl]) : make_float2(0.f, 0.f);
+                    const int u = tl & 31, bb = tl >> 5, s = u & 7;
+                    const float fac = static_cast<float>(1 << (7 - s));
+                    uint8_t* bc = reinterpret_cast<uint8_t*>(swc) + (u >> 3);
+                    uint8_t* bq = reinterpret_cast<uint8_t*>(swq) + (u >> 3);
+#pragma unroll
+                    for (int h = 0; h < GP; ++h) {
+                        uint32_t xc = 0u, xq = 0u;
+                        if (valid && h < G) {
+                            const float* ss = sstat + h * 8;
+                            const float e = __expf(slog[h * TC + tl] - ss[0]);
+                            sum_e[h] += e;
+                            const float wc = e * nv.x;
+                            const float wq = wc * nv.y;
+                            sum_w[h] += wc;
+                            sum_wq[h] += wq;
+                            xc = __float2uint_rn(wc * (fac * ss[4]));
+                            if (QJL) xq = __float2uint_rn(wq * (fac * ss[5]));
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            // row r of the weight operand: G <= 4: r = h + 4k; G = 8: r = h + 8k
+                            const int r = (G <= 4) ? h + 4 * k : h + 8 * k;
+                            const int rt = r >> 4, rl = r & 15;
+                            const int off =
+                                ((((bb * RT + rt) * 32 + 4 * (rl & 7) + (s & 3)) * 4 + (rl >> 3) + 2 * (s >> 2)) << 2);
+                            bc[off] = static_cast<uint8_t>(xc >> (8 * k));
+                            if (QJL) bq[off] = static_cast<uint8_t>(xq >> (8 * k));
+                        }
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                    for (int h = 0; h < GP; ++h) {
+                        sum_e[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_e[h], o);
+                        sum_w[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_w[h], o);
+                        sum_wq[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_wq[h], o);
+                    }
+                if (lane == 0)
+#pragma unroll
+                    for (int h = 0; h < GP; ++h) {
+                        sred[(warp * GP + h) * 3 + 0] = sum_e[h];
+                        sred[(warp * GP + h) * 3 + 1] = sum_w[h];
+                        sred[(warp * GP + h) * 3 + 2] = sum_wq[h];
+                    }
+            }
+            __syncthreads();
+            if (tid < GP) {
+                const int h = tid;
+                float te = 0.f, tw = 0.f, twq = 0.f;
+                for (int w = 0; w < 4; ++w) {
+                    te += sred[(w * GP + h) * 3 + 0];
+                    tw += sred[(w * GP + h) * 3 + 1];
+                    twq += sred[(w * GP + h) * 3 + 2];
+                }
+                float* hs = shead + h * 8;
+                const float alpha = sstat[h * 8 + 1];
+                hs[5] = hs[5] * alpha + te;
+                hs[6] = hs[6] * alpha + tw;
+                hs[7] = hs[7] * alpha + twq;
+            }
+
+            // ---------------- phase V: value sums of the sub-chunk ----------------
+            // Lane (g, t) of warp w reads the words of coordinates
+            // w D/4 + NTV g + nt (nt < NTV) in one load: n-tile nt, column n is
+            // coordinate w D/4 + NTV n + nt.
+            {
+                int accv[NPV][NTV][RT][4];
+#pragma unroll
+                for (int p = 0; p < NPV; ++p)
+#pragma unroll
+                    for (int nt = 0; nt < NTV; ++nt)
+#pragma unroll
+                        for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) accv[p][nt][rt][r] = 0;
+                const int nblk = have > 0 ? static_cast<int>((have + 31) / 32) : 0;
+                const int cbase = warp * (D / 4) + NTV * g;
+                for (int bb = 0; bb < nblk; ++bb) {
+                    uint32_t aw[RT][4], aq[RT][4];
+#pragma unroll
+                    for (int rt = 0; rt < RT; ++rt) {
+                        const uint4 x = reinterpret_cast<const uint4*>(swc)[(bb * RT + rt) * 32 + lane];
+                        aw[rt][0] = x.x; aw[rt][1] = x.y; aw[rt][2] = x.z; aw[rt][3] = x.w;
+                        if (QJL) {
+                            const uint4 y = reinterpret_cast<const uint4*>(swq)[(bb * RT + rt) * 32 + lane];
+                            aq[rt][0] = y.x; aq[rt][1] = y.y; aq[rt][2] = y.z; aq[rt][3] = y.w;
+                        }
+                    }
+#pragma unroll
+                    for (int p = 0; p < NPV; ++p) {
+                        const uint32_t* src = (p < B) ? sVc + (bb * B + p) * D + cbase : sVq + bb * M + cbase;
+                        uint32_t wv[NTV];
+                        if (NTV % 4 == 0) {
+#pragma unroll
+                            for (int q4 = 0; q4 < NTV / 4; ++q4) {
+                                const uint4 x = reinterpret_cast<const uint4*>(src)[q4];
+                                wv[4 * q4] = x.x; wv[4 * q4 + 1] = x.y; wv[4 * q4 + 2] = x.z; wv[4 * q4 + 3] = x.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int q2 = 0; q2 < NTV / 2; ++q2) {
+                                const uint2 x = reinterpret_cast<const uint2*>(src)[q2];
+                                wv[2 * q2] = x.x; wv[2 * q2 + 1] = x.y;
+                            }
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < NTV; ++nt) {
+                            const uint32_t b0 = wv[nt] & msk_lo, b1 = wv[nt] & msk_hi;
+#pragma unroll
+                            for (int rt = 0; rt < RT; ++rt) {
+                                if (p < B) mma_u8u8(accv[p][nt][rt], aw[rt], b0, b1);
+                                else mma_u8u8(accv[p][nt][rt], aq[rt], b0, b1);
+                            }
+                        }
+                    }
+                }
+                // Merge into the fp32 running sums (rescaled by alpha).  Digit k
+                // of head h sits in row h + 4k (G <= 4): lane g < 4 holds digits
+                // 0, 2 of head g and lane + 16 digits 1, 3; lane g < 4 completes
+                // column 2t, lane g + 4 column 2t + 1, swapping the other two.
+                // With G = 8 (rows h + 8k, two row tiles) every lane holds all
+                // digits of head g, columns 2t and 2t + 1.  Each digit sum is
+                // non-negative and below 2^24.
+                const int head = (G <= 4) ? (g & 3) : g;
+                const bool hi = g >= 4;
+                const float* ss = sstat + (head < G ? head : 0) * 8;
+                const float alpha = ss[1];
+                const float sgw = ss[2] * (1.f / 128.f);
+                const float sgq = ss[3] * (1.f / 128.f);
+#pragma unroll
+                for (int nt = 0; nt < NTV; ++nt) {
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) {
+                        float vals[NPV];
+#pragma unroll
+                        for (int p = 0; p < NPV; ++p) {
+                            uint32_t d0, d1, d2, d3;
+                            if (G <= 4) {
+                                const int* x = accv[p][nt][0];
+                                const int s1 = __shfl_xor_sync(0xFFFFFFFFu, hi ? x[0] : x[1], 16);
+                                const int s3 = __shfl_xor_sync(0xFFFFFFFFu, hi ? x[2] : x[3], 16);
+                                d0 = static_cast<uint32_t>(hi ? s1 : x[0]);
+                                d1 = static_cast<uint32_t>(hi ? x[1] : s1);
+                                d2 = static_cast<uint32_t>(hi ? s3 : x[2]);
+                                d3 = static_cast<uint32_t>(hi ? x[3] : s3);
+                            } else {
+                                d0 = static_cast<uint32_t>(accv[p][nt][0][c]);
+                                d1 = static_cast<uint32_t>(accv[p][nt][0][2 + c]);
+                                d2 = static_cast<uint32_t>(accv[p][nt][RT - 1][c]);
+                                d3 = static_cast<uint32_t>(accv[p][nt][RT - 1][2 + c]);
+                            }
+                            vals[p] = fmaf(static_cast<float>(d3), 16777216.f,
+                                           fmaf(static_cast<float>(d2), 65536.f, static_cast<float>(d1 * 256u + d0)));
+                        }
+                        if (head < G) {
+                            float code = coef0 * vals[0];
+                            if (B == 2) code = fmaf(coef1, vals[1 % NPV], code);
+                            accA[nt][c] = fmaf(accA[nt][c], alpha, sgw * code);
+                            if (QJL) accB[nt][c] = fmaf(accB[nt][c], alpha, sgq * 2.f * vals[NPV - 1]);
+                        }
+                    }
+                }
+            }
+            __syncthreads();  // stage and weight digits are reused by the next sub-chunk
+            if (tid == 0 && sc + 2 < nsub) {
+                if (sc & 1) armed1 = issue(sc + 2);
+                else armed0 = issue(sc + 2);
+            }
+        }
+        if (!alive) {
+            if (tid == 0) {
+                // loads in flight are waited for before exit (only when a wait gave up)
+                if (armed0) mbar_wait(&bar[0], phase[0], a.status);
+                if (armed1) mbar_wait(&bar[1], phase[1], a.status);
+            }
+            break;
+        }
+
+        // ---------------- partials: {M, L, A[D], B[M]} per query head ----------------
+        constexpr int PART = 2 + D + M;
+        {
+            const int head = (G <= 4) ? (g & 3) : g;
+            if (head < G) {
+                float* pp = a.part + ((qh0 + head) * a.nsplit + split) * PART;
+                const float* hs = shead + head * 8;
+                const float c0 = a.centroid[0];
+#pragma unroll
+                for (int nt = 0; nt < NTV; ++nt)
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) {
+                        const int col = (G <= 4) ? 2 * t + (g >= 4 ? 1 : 0) : 2 * t + c;
+                        const int coord = warp * (D / 4) + NTV * col + nt;
+                        pp[2 + coord] = c0 * hs[6] + accA[nt][c];
+                        if (QJL) pp[2 + D + coord] = accB[nt][c] - hs[7];
+                    }
+            }
+            if (tid < G) {
+                float* pp = a.part + ((qh0 + tid) * a.nsplit + split) * PART;
+                pp[0] = shead[tid * 8 + 4];
+                pp[1] = shead[tid * 8 + 5];
+            }
+        }
     }
 }
 
-}  // namespace
+template <int D, int B, bool QJL, int G>
+int ctas_per_sm_g() {
+    using L = MmaSmem<D, B, QJL, G>;
+    auto kern = decode_mma_kernel<D, B, QJL, G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess) return 1;
+    int n = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, L::kBytes) != cudaSuccess || n < 1) n = 1;
+    return n;
+}
+
+template <int D, int B, bool QJL>
+int ctas_per_sm_d(int G) {
+    switch (G) {
+        case 1: return ctas_per_sm_g<D, B, QJL, 1>();
+        case 2: return ctas_per_sm_g<D, B, QJL, 2>();
+        case 4: return ctas_per_sm_g<D, B, QJL, 4>();
+        default: return ctas_per_sm_g<D, B, QJL, 8>();
+    }
+}
 
 template <int D, int B, bool QJL, int G>
-static cudaError_t launch_mma_g(const DecodeArgs& a, cudaStream_t s) {
+cudaError_t launch_mma_g(const DecodeArgs& a, int grid, cudaStream_t s) {
     const int groups = a.batch * a.hkv;
     switch (a.qdtype) {
         case 0: qfrag_kernel<D, B, QJL, G, 0><<<groups, kThreads, 0, s>>>(a); break;
@@ -660,34 +771,71 @@ static cudaError_t launch_mma_g(const DecodeArgs& a, cudaStream_t s) {
     auto kern = decode_mma_kernel<D, B, QJL, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(a.nsplit, a.hkv, a.batch), kThreads, L::kBytes, s>>>(a);
+    const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit;
+    const int64_t n = items < grid ? items : grid;
+    if (n <= 0) return cudaSuccess;
+    kern<<<static_cast<unsigned>(n), kThreads, L::kBytes, s>>>(a);
     return cudaGetLastError();
 }
 
 template <int D, int B, bool QJL>
-static cudaError_t launch_mma_d(const DecodeArgs& a, cudaStream_t s) {
+cudaError_t launch_mma_d(const DecodeArgs& a, int grid, cudaStream_t s) {
     switch (a.G) {
-        case 1: return launch_mma_g<D, B, QJL, 1>(a, s);
-        case 2: return launch_mma_g<D, B, QJL, 2>(a, s);
-        case 4: return launch_mma_g<D, B, QJL, 4>(a, s);
-        default: return launch_mma_g<D, B, QJL, 8>(a, s);
+        case 1: return launch_mma_g<D, B, QJL, 1>(a, grid, s);
+        case 2: return launch_mma_g<D, B, QJL, 2>(a, grid, s);
+        case 4: return launch_mma_g<D, B, QJL, 4>(a, grid, s);
+        default: return launch_mma_g<D, B, QJL, 8>(a, grid, s);
     }
+}
+
+}  // namespace
+
+#define KVQ_MMA_CASES(FN, ...)                                              \
+    switch (h->d * 16 + h->b * 4 + (qjl ? 1 : 0)) {                         \
+        case 64 * 16 + 4: return FN<64, 1, false>(__VA_ARGS__);             \
+        case 64 * 16 + 5: return FN<64, 1, true>(__VA_ARGS__);              \
+        case 64 * 16 + 8: return FN<64, 2, false>(__VA_ARGS__);             \
+        case 64 * 16 + 9: return FN<64, 2, true>(__VA_ARGS__);              \
+        case 128 * 16 + 4: return FN<128, 1, false>(__VA_ARGS__);           \
+        case 128 * 16 + 5: return FN<128, 1, true>(__VA_ARGS__);            \
+        case 128 * 16 + 8: return FN<128, 2, false>(__VA_ARGS__);           \
+        case 128 * 16 + 9: return FN<128, 2, true>(__VA_ARGS__);            \
+        case 256 * 16 + 4: return FN<256, 1, false>(__VA_ARGS__);           \
+        case 256 * 16 + 5: return FN<256, 1, true>(__VA_ARGS__);            \
+        case 256 * 16 + 8: return FN<256, 2, false>(__VA_ARGS__);           \
+        case 256 * 16 + 9: return FN<256, 2, true>(__VA_ARGS__);            \
+        default: break;                                                     \
+    }
+
+namespace {
+int ctas_per_sm(const kvq_ctx* h, int G) {
+    const bool qjl = (h->flags & 1u) != 0;
+    KVQ_MMA_CASES(ctas_per_sm_d, G)
+    return 1;
+}
+}  // namespace
+
+// Resident CTAs of the split kernel on the whole device: the persistent grid.
+int decode_mma_grid(const kvq_ctx* h, int G) {
+    const int gi = (G >= 1 && G <= 8) ? G : 8;
+    if (h->mma_grid[gi] > 0) return h->mma_grid[gi];
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
+    const int n = ctas_per_sm(h, G) * sms;
+    const_cast<kvq_ctx*>(h)->mma_grid[gi] = n;
+    return n;
 }
 
 // Query fragments + split kernel of the tensor-core path (b <= 2).
 cudaError_t launch_decode_mma(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s) {
     const bool qjl = (h->flags & 1u) != 0;
-#define KVQ_MMA_CASE(D_, B_)                                                                              \
-    if (h->d == D_ && h->b == B_)                                                                         \
-        return qjl ? launch_mma_d<D_, B_, true>(a, s) : launch_mma_d<D_, B_, false>(a, s);
-    KVQ_MMA_CASE(64, 1) KVQ_MMA_CASE(64, 2) KVQ_MMA_CASE(128, 1) KVQ_MMA_CASE(128, 2) KVQ_MMA_CASE(256, 1)
-    KVQ_MMA_CASE(256, 2)
-#undef KVQ_MMA_CASE
+    const int grid = decode_mma_grid(h, a.G);
+    KVQ_MMA_CASES(launch_mma_d, a, grid, s)
     return cudaErrorNotSupported;
 }
 
 size_t decode_mma_qfrag_bytes(const kvq_ctx* h, int G) {
-    const int NTK = (G <= 4) ? 2 : 3;
+    const int NTK = (G <= 4) ? 2 : 4;
     const int KS = (h->b + ((h->flags & 1u) ? 1 : 0)) * (h->d / 32);
     return static_cast<size_t>(KS) * NTK * 32 * 8;
 }

@@ -26,6 +26,9 @@ struct kvq_ctx {
     // Device constants.
     __half* d_S = nullptr;            // [m][d]
     uint32_t* d_status = nullptr;     // one word, ORed by kernels
+    // Resident CTAs of the tensor-core decode kernel per group size G (index
+    // G = 1, 2, 4, 8; 0 = not yet queried).
+    int mma_grid[9] = {};
 };
 
 namespace kvq {
@@ -94,6 +97,8 @@ cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s,
 // Tensor-core decode path (1- and 2-bit codebooks): query fragments + split kernel.
 cudaError_t launch_decode_mma(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s);
 size_t decode_mma_qfrag_bytes(const kvq_ctx* h, int G);
+// Resident CTAs of the tensor-core split kernel on the device (its persistent grid).
+int decode_mma_grid(const kvq_ctx* h, int G);
 inline bool decode_uses_mma(const kvq_ctx* h) { return h->b <= 2; }
 
 // Size of the fixed scratch of kvq_decode_attend_noalloc (mirrors
