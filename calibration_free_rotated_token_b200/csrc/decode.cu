@@ -412,13 +412,13 @@ void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, in
     int64_t ch;
     if (decode_uses_mma(h)) {
         // Persistent grid over (stream, split) items: about 16 items per
-        // resident CTA keeps the last round short; splits of at least 512
+        // resident CTA keeps the last round short; splits of at least 1024
         // tokens amortise the per-item set-up.
         const int64_t grid = decode_mma_grid(h, hkv > 0 ? hq / hkv : 1);
         const int64_t target = 16 * grid;
         ch = (streams * max_T + target - 1) / (target > 0 ? target : 1);
         ch = (ch + 255) / 256 * 256;
-        if (ch < 512) ch = 512;
+        if (ch < 1024) ch = 1024;
         if ((max_T + ch - 1) / ch > 4096) ch = ((max_T + 4095) / 4096 + 255) / 256 * 256;
     } else {
         int64_t want = (4 * static_cast<int64_t>(sms) + streams - 1) / (streams > 0 ? streams : 1);

@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     constexpr int NTV = D / 32;               // value n-tiles per warp (D/4 coordinates / 8)
     constexpr int NPV = B + (QJL ? 1 : 0);
     constexpr bool QF_REG = L::kQfReg;
+    constexpr int HH = (G == 8) ? 2 : 1;      // query heads per lane in the logit epilogue
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t* stage[2] = {smem, smem + L::kStage};
     uint2* sfrag = reinterpret_cast<uint2*>(smem + 2 * L::kStage);
@@ -257,9 +258,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     uint32_t* swq = swc + L::kWfrag / 4;                                                       // QJL-weight digits
     uint8_t* misc = smem + 2 * L::kStage + L::kFrag + L::kLog + 2 * L::kWfrag;
     uint64_t* bar = reinterpret_cast<uint64_t*>(misc);      // [2]
-    float* sred = reinterpret_cast<float*>(misc + 16);      // [4 warps][GP][3]
-    float* shead = sred + 4 * GP * 3;                        // [GP][8]: scalars, running state
-    float* sstat = shead + GP * 8;                           // [GP][8]: mnew, alpha, sig_w, sig_wq, inv_w, inv_wq
+    float* sred = reinterpret_cast<float*>(misc + 16);      // 96 floats: [4 warps][GP][3] or [4 warps][16]
+    float* shead = sred + 96;                                // [GP][8]: item sums (5..7)
+    float* sstat = shead + GP * 8;                           // [GP][8]: -, alpha, sig_w/128, sig_wq/128
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
     const uint32_t msk_lo = kLowBits << t, msk_hi = kLowBits << (t + 4);
@@ -298,19 +299,30 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
         {
             const uint2* gf = a.qfrag + stream * KS * NTK * 32;
             for (int e = tid; e < KS * NTK * 32; e += kThreads) sfrag[e] = gf[e];
-            if (tid < GP) {
-                float* hs = shead + tid * 8;
-                if (tid < G) {
-                    const float* qs = a.qscal + (qh0 + tid) * 4;
-                    hs[0] = qs[0]; hs[1] = qs[1]; hs[2] = qs[2]; hs[3] = qs[3];
-                } else {
-                    hs[0] = hs[1] = hs[2] = hs[3] = 0.f;
-                }
-                hs[4] = -INFINITY;  // running max
-                hs[5] = 0.f;        // running sum of exp
-                hs[6] = 0.f;        // running sum of code weights (Omega)
-                hs[7] = 0.f;        // running sum of QJL weights (Omega')
+        }
+        // logit constants of this lane's heads t (and t + 4):
+        // l = n (k0 + k1 xc + n_gamma (k2 xq - k3)), scale / d folded in
+        float hk0[HH], hk1[HH], hk2[HH], hk3[HH];
+#pragma unroll
+        for (int hh = 0; hh < HH; ++hh) {
+            const int h = t + 4 * hh;
+            hk0[hh] = hk1[hh] = hk2[hh] = hk3[hh] = 0.f;
+            if (h < G) {
+                const float* qs = a.qscal + (qh0 + h) * 4;
+                const float f = a.scale / D;
+                hk0[hh] = f * qs[0];
+                hk1[hh] = f * qs[1];
+                hk2[hh] = f * kappa * 2.f * qs[2];
+                hk3[hh] = f * kappa * qs[3];
             }
+        }
+        // running max per head (the same in every thread) and this thread's
+        // partial sums of exp, code weights and QJL weights (rescaled with it)
+        float mrun[GP], pe[GP], pw[GP], pq[GP];
+#pragma unroll
+        for (int h = 0; h < GP; ++h) {
+            mrun[h] = -INFINITY;
+            pe[h] = pw[h] = pq[h] = 0.f;
         }
         const int nsub = static_cast<int>((t1e - t0 + TC - 1) / TC);
         // tokens of the sub-chunk that exist in the cache (rounded to whole blocks of 32)
@@ -374,15 +386,16 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             const __half2* sVn = reinterpret_cast<const __half2*>(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq);
 
             // ---------------- phase K: logits of the sub-chunk ----------------
+            float lmax[HH];
+#pragma unroll
+            for (int hh = 0; hh < HH; ++hh) lmax[hh] = -INFINITY;
             for (int mt = warp; mt < TC / 16; mt += 4) {
                 const int tl0 = mt * 16 + g, tl1 = tl0 + 8;
-                int accc[2][NTK][4], accq[2][NTK][4];  // even / odd K-steps (two dependency chains)
+                int accc[2][NTK][4], accq[NTK][4];  // code K-steps alternate between two chains
 #pragma unroll
-                for (int e = 0; e < 2; ++e)
+                for (int nt = 0; nt < NTK; ++nt)
 #pragma unroll
-                    for (int nt = 0; nt < NTK; ++nt)
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) accc[e][nt][r] = accq[e][nt][r] = 0;
+                    for (int r = 0; r < 4; ++r) accc[0][nt][r] = accc[1][nt][r] = accq[nt][r] = 0;
                 if (tb + mt * 16 < t1) {
                     uint32_t w0[KS], w1[KS];
 #pragma unroll
@@ -406,22 +419,29 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                             w1[KWT + k] = x1.x; w1[KWT + k + 1] = x1.y;
                         }
                     }
+                    // code and QJL K-steps interleaved: 2 NTK independent accumulators
 #pragma unroll
-                    for (int ks = 0; ks < KS; ++ks) {
-                        const uint32_t af[4] = {w0[ks] & msk_lo, w1[ks] & msk_lo, w0[ks] & msk_hi, w1[ks] & msk_hi};
+                    for (int i = 0; i < KWT || i < QWT; ++i) {
 #pragma unroll
-                        for (int nt = 0; nt < NTK; ++nt) {
-                            const uint2 bq = QF_REG ? qf[QF_REG ? ks : 0][QF_REG ? nt : 0]
-                                                    : sfrag[(ks * NTK + nt) * 32 + lane];
-                            if (ks < B * (D / 32)) mma_u8s8(accc[ks & 1][nt], af, bq);
-                            else mma_u8s8(accq[ks & 1][nt], af, bq);
+                        for (int kind = 0; kind < 2; ++kind) {
+                            if (kind == 0 ? (i >= KWT) : (i >= QWT)) continue;
+                            const int ks = kind == 0 ? i : KWT + i;
+                            const uint32_t af[4] = {w0[ks] & msk_lo, w1[ks] & msk_lo, w0[ks] & msk_hi,
+                                                    w1[ks] & msk_hi};
+#pragma unroll
+                            for (int nt = 0; nt < NTK; ++nt) {
+                                const uint2 bq = QF_REG ? qf[QF_REG ? ks : 0][QF_REG ? nt : 0]
+                                                        : sfrag[(ks * NTK + nt) * 32 + lane];
+                                if (kind == 0) mma_u8s8(accc[i & 1][nt], af, bq);
+                                else mma_u8s8(accq[nt], af, bq);
+                            }
                         }
                     }
                 }
                 // epilogue: thread t owns head t (and t + 4 when G = 8); its
                 // columns hold the four digits of the head
 #pragma unroll
-                for (int hh = 0; hh < (G == 8 ? 2 : 1); ++hh) {
+                for (int hh = 0; hh < HH; ++hh) {
                     const int h = t + 4 * hh;
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr) {
@@ -430,170 +450,140 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                         float l = -INFINITY;
                         if (h < G && tg < t1) {
                             const int n0 = 2 * hh, n1 = 2 * hh + 1;
-                            const int c_hi = (accc[0][n0][2 * rr] + accc[1][n0][2 * rr]) * 128 +
-                                             accc[0][n0][2 * rr + 1] + accc[1][n0][2 * rr + 1];
-                            const int c_lo = (accc[0][n1][2 * rr] + accc[1][n1][2 * rr]) * 128 +
-                                             accc[0][n1][2 * rr + 1] + accc[1][n1][2 * rr + 1];
-                            const float xc = fmaf(static_cast<float>(c_hi), 16384.f, static_cast<float>(c_lo));
-                            const float* hs = shead + h * 8;
+                            const float xc = fmaf(static_cast<float>((accc[0][n0][2 * rr] + accc[1][n0][2 * rr]) * 128 +
+                                                                     accc[0][n0][2 * rr + 1] + accc[1][n0][2 * rr + 1]),
+                                                  16384.f,
+                                                  static_cast<float>((accc[0][n1][2 * rr] + accc[1][n1][2 * rr]) * 128 +
+                                                                     accc[0][n1][2 * rr + 1] + accc[1][n1][2 * rr + 1]));
                             const float2 nk = __half22float2(sKn[tl]);
-                            float dot = fmaf(hs[1], xc, hs[0]);
+                            float inner = fmaf(hk1[hh], xc, hk0[hh]);
                             if (QJL) {
-                                const int q_hi = (accq[0][n0][2 * rr] + accq[1][n0][2 * rr]) * 128 +
-                                                 accq[0][n0][2 * rr + 1] + accq[1][n0][2 * rr + 1];
-                                const int q_lo = (accq[0][n1][2 * rr] + accq[1][n1][2 * rr]) * 128 +
-                                                 accq[0][n1][2 * rr + 1] + accq[1][n1][2 * rr + 1];
-                                const float xq = fmaf(static_cast<float>(q_hi), 16384.f, static_cast<float>(q_lo));
-                                dot += kappa * nk.y * (2.f * hs[2] * xq - hs[3]);
+                                const float xq =
+                                    fmaf(static_cast<float>(accq[n0][2 * rr] * 128 + accq[n0][2 * rr + 1]), 16384.f,
+                                         static_cast<float>(accq[n1][2 * rr] * 128 + accq[n1][2 * rr + 1]));
+                                inner = fmaf(nk.y, fmaf(hk2[hh], xq, -hk3[hh]), inner);
                             }
-                            l = a.scale * (nk.x / D) * dot;
+                            l = nk.x * inner;
+                            lmax[hh] = fmaxf(lmax[hh], l);
                         }
                         if (h < GP) slog[h * TC + tl] = l;
                         if (a.logits != nullptr && h < G && tg < t1e) a.logits[(qh0 + h) * a.max_T + tg] = l;
                     }
                 }
             }
-            __syncthreads();
-
-            // ---------------- phase S: softmax statistics and weight digits ----------------
-            // pass 1: per head, the max logit and the max of l + log(n) (and of
-            // l + log(n gamma)): the largest weight of the sub-chunk, which sets
-            // the scale of its weight digits.
+            // Bounds for the weight digits: per head the max logit of the
+            // sub-chunk, and the max value norm n (and n gamma); the product
+            // bounds the largest weight.
             {
-                float mx[GP], mw[GP], mq[GP];
-#pragma unroll
-                for (int h = 0; h < GP; ++h) mx[h] = mw[h] = mq[h] = -INFINITY;
+                float nmx = 0.f, ngx = 0.f;
                 for (int tl = tid; tl < TC; tl += kThreads) {
                     if (tb + tl < t1) {
                         const float2 nv = __half22float2(sVn[tl]);
-                        const float ln = __logf(nv.x), lg = __logf(nv.x * nv.y);
-#pragma unroll
-                        for (int h = 0; h < GP; ++h) {
-                            const float l = slog[h * TC + tl];
-                            mx[h] = fmaxf(mx[h], l);
-                            mw[h] = fmaxf(mw[h], l + ln);
-                            mq[h] = fmaxf(mq[h], l + lg);
-                        }
+                        nmx = fmaxf(nmx, nv.x);
+                        ngx = fmaxf(ngx, nv.x * nv.y);
                     }
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
+                    nmx = fmaxf(nmx, __shfl_xor_sync(0xFFFFFFFFu, nmx, o));
+                    ngx = fmaxf(ngx, __shfl_xor_sync(0xFFFFFFFFu, ngx, o));
+                }
 #pragma unroll
-                    for (int h = 0; h < GP; ++h) {
-                        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xFFFFFFFFu, mx[h], o));
-                        mw[h] = fmaxf(mw[h], __shfl_xor_sync(0xFFFFFFFFu, mw[h], o));
-                        mq[h] = fmaxf(mq[h], __shfl_xor_sync(0xFFFFFFFFu, mq[h], o));
-                    }
+                for (int hh = 0; hh < HH; ++hh)
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) lmax[hh] = fmaxf(lmax[hh], __shfl_xor_sync(0xFFFFFFFFu, lmax[hh], o));
+                if (g == 0) {
+#pragma unroll
+                    for (int hh = 0; hh < HH; ++hh)
+                        if (t + 4 * hh < GP) sred[warp * 16 + t + 4 * hh] = lmax[hh];
                 }
                 if (lane == 0) {
+                    sred[warp * 16 + 8] = nmx;
+                    sred[warp * 16 + 9] = ngx;
+                }
+            }
+            __syncthreads();
+            // Softmax statistics of the sub-chunk, computed alike by every
+            // thread: new running max, rescale factor, digit scales (weight w
+            // is the integer w 2^(7-s) inv < kWCap; a digit sum S of the value
+            // MMA stands for S sig / 128 with sig = 1 / inv).
+            float mnew[GP], invw[GP], invq[GP];
+            {
+                // lane h < GP of every warp works out head h; the others take
+                // the values by shuffle
+                float nmax = 0.f, ngmax = 0.f;
 #pragma unroll
-                    for (int h = 0; h < GP; ++h) {
-                        sred[(warp * GP + h) * 3 + 0] = mx[h];
-                        sred[(warp * GP + h) * 3 + 1] = mw[h];
-                        sred[(warp * GP + h) * 3 + 2] = mq[h];
-                    }
-                }
-            }
-            __syncthreads();
-            // per-head new running max, rescale factor and weight-digit scales:
-            // weight w is the integer X = w 2^(7-s) inv < kWCap, and a value
-            // sum S of the MMA stands for S sig / 128 with sig = 1 / inv
-            if (tid < GP) {
-                const int h = tid;
-                float mx = -INFINITY, mw = -INFINITY, mq = -INFINITY;
                 for (int w = 0; w < 4; ++w) {
-                    mx = fmaxf(mx, sred[(w * GP + h) * 3 + 0]);
-                    mw = fmaxf(mw, sred[(w * GP + h) * 3 + 1]);
-                    mq = fmaxf(mq, sred[(w * GP + h) * 3 + 2]);
+                    nmax = fmaxf(nmax, sred[w * 16 + 8]);
+                    ngmax = fmaxf(ngmax, sred[w * 16 + 9]);
                 }
-                float* hs = shead + h * 8;
-                const float mold = hs[4];
-                const float mnew = fmaxf(mold, mx);
-                const float alpha = (mnew == -INFINITY) ? 1.f : __expf(mold - mnew);
-                hs[4] = mnew;
-                const float wmax = (mw == -INFINITY) ? 0.f : __expf(mw - mnew);
-                const float qmax = (mq == -INFINITY) ? 0.f : __expf(mq - mnew);
-                float* ss = sstat + h * 8;
-                ss[0] = mnew;
-                ss[1] = alpha;
-                ss[2] = wmax * (128.f / kWCap);
-                ss[3] = qmax * (128.f / kWCap);
-                ss[4] = wmax > 0.f ? kWCap / (128.f * wmax) : 0.f;
-                ss[5] = qmax > 0.f ? kWCap / (128.f * qmax) : 0.f;
+                const int hl = lane < GP ? lane : 0;
+                float msc = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) msc = fmaxf(msc, sred[w * 16 + hl]);
+                float mold = mrun[0];
+#pragma unroll
+                for (int h = 1; h < GP; ++h) mold = (hl == h) ? mrun[h] : mold;
+                const float mn = fmaxf(mold, msc);
+                const float al = (mn == -INFINITY) ? 1.f : __expf(mold - mn);
+                const float top = (msc == -INFINITY) ? 0.f : __expf(msc - mn);
+                const float wb = top * nmax, qb = top * ngmax;
+                const float iw = wb > 0.f ? __fdividef(kWCap / 128.f, wb) : 0.f;
+                const float iq = qb > 0.f ? __fdividef(kWCap / 128.f, qb) : 0.f;
+                if (warp == 0 && lane < GP) {
+                    sstat[lane * 8 + 1] = al;
+                    sstat[lane * 8 + 2] = iw > 0.f ? __fdividef(1.f / 128.f, iw) : 0.f;  // sig / 128
+                    sstat[lane * 8 + 3] = iq > 0.f ? __fdividef(1.f / 128.f, iq) : 0.f;
+                }
+#pragma unroll
+                for (int h = 0; h < GP; ++h) {
+                    mnew[h] = __shfl_sync(0xFFFFFFFFu, mn, h);
+                    invw[h] = __shfl_sync(0xFFFFFFFFu, iw, h);
+                    invq[h] = __shfl_sync(0xFFFFFFFFu, iq, h);
+                    const float alpha = __shfl_sync(0xFFFFFFFFu, al, h);
+                    mrun[h] = mnew[h];
+                    pe[h] *= alpha;
+                    pw[h] *= alpha;
+                    pq[h] *= alpha;
+                }
             }
-            __syncthreads();
-            // pass 2: weight digits into A-fragment bytes; sums of exp and weights.
+            // pass 2: weight digits into A-fragment bytes; partial sums.
             // Token u of block bb is K index 4(u&7) + (u>>3) (u&7 < 4) or
             // 16 + 4((u&7)-4) + (u>>3): lane 4(r&7) + (u&3), register
             // (r>>3) + 2((u&7)>>2), byte u>>3 of row r's fragment.
-            {
-                float sum_e[GP], sum_w[GP], sum_wq[GP];
+            for (int tl = tid; tl < TC; tl += kThreads) {
+                const bool valid = tb + tl < t1;
+                const float2 nv = valid ? __half22float2(sVn[tl]) : make_float2(0.f, 0.f);
+                const int u = tl & 31, bb = tl >> 5, s = u & 7;
+                const float fac = static_cast<float>(1 << (7 - s));
+                uint8_t* bc = reinterpret_cast<uint8_t*>(swc) + (u >> 3);
+                uint8_t* bq = reinterpret_cast<uint8_t*>(swq) + (u >> 3);
 #pragma unroll
-                for (int h = 0; h < GP; ++h) sum_e[h] = sum_w[h] = sum_wq[h] = 0.f;
-                for (int tl = tid; tl < TC; tl += kThreads) {
-                    const bool valid = tb + tl < t1;
-                    const float2 nv = valid ? __half22float2(sVn[tl]) : make_float2(0.f, 0.f);
-                    const int u = tl & 31, bb = tl >> 5, s = u & 7;
-                    const float fac = static_cast<float>(1 << (7 - s));
-                    uint8_t* bc = reinterpret_cast<uint8_t*>(swc) + (u >> 3);
-                    uint8_t* bq = reinterpret_cast<uint8_t*>(swq) + (u >> 3);
+                for (int h = 0; h < GP; ++h) {
+                    uint32_t xc = 0u, xq = 0u;
+                    if (valid && h < G) {
+                        const float e = __expf(slog[h * TC + tl] - mnew[h]);
+                        const float wc = e * nv.x;
+                        const float wq = wc * nv.y;
+                        pe[h] += e;
+                        pw[h] += wc;
+                        pq[h] += wq;
+                        xc = __float2uint_rn(wc * (fac * invw[h]));
+                        if (QJL) xq = __float2uint_rn(wq * (fac * invq[h]));
+                    }
 #pragma unroll
-                    for (int h = 0; h < GP; ++h) {
-                        uint32_t xc = 0u, xq = 0u;
-                        if (valid && h < G) {
-                            const float* ss = sstat + h * 8;
-                            const float e = __expf(slog[h * TC + tl] - ss[0]);
-                            sum_e[h] += e;
-                            const float wc = e * nv.x;
-                            const float wq = wc * nv.y;
-                            sum_w[h] += wc;
-                            sum_wq[h] += wq;
-                            xc = __float2uint_rn(wc * (fac * ss[4]));
-                            if (QJL) xq = __float2uint_rn(wq * (fac * ss[5]));
-                        }
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            // row r of the weight operand: G <= 4: r = h + 4k; G = 8: r = h + 8k
-                            const int r = (G <= 4) ? h + 4 * k : h + 8 * k;
-                            const int rt = r >> 4, rl = r & 15;
-                            const int off =
-                                ((((bb * RT + rt) * 32 + 4 * (rl & 7) + (s & 3)) * 4 + (rl >> 3) + 2 * (s >> 2)) << 2);
-                            bc[off] = static_cast<uint8_t>(xc >> (8 * k));
-                            if (QJL) bq[off] = static_cast<uint8_t>(xq >> (8 * k));
-                        }
+                    for (int k = 0; k < 4; ++k) {
+                        // row r of the weight operand: G <= 4: r = h + 4k; G = 8: r = h + 8k
+                        const int r = (G <= 4) ? h + 4 * k : h + 8 * k;
+                        const int rt = r >> 4, rl = r & 15;
+                        const int off =
+                            ((((bb * RT + rt) * 32 + 4 * (rl & 7) + (s & 3)) * 4 + (rl >> 3) + 2 * (s >> 2)) << 2);
+                        bc[off] = static_cast<uint8_t>(xc >> (8 * k));
+                        if (QJL) bq[off] = static_cast<uint8_t>(xq >> (8 * k));
                     }
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                    for (int h = 0; h < GP; ++h) {
-                        sum_e[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_e[h], o);
-                        sum_w[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_w[h], o);
-                        sum_wq[h] += __shfl_xor_sync(0xFFFFFFFFu, sum_wq[h], o);
-                    }
-                if (lane == 0)
-#pragma unroll
-                    for (int h = 0; h < GP; ++h) {
-                        sred[(warp * GP + h) * 3 + 0] = sum_e[h];
-                        sred[(warp * GP + h) * 3 + 1] = sum_w[h];
-                        sred[(warp * GP + h) * 3 + 2] = sum_wq[h];
-                    }
             }
             __syncthreads();
-            if (tid < GP) {
-                const int h = tid;
-                float te = 0.f, tw = 0.f, twq = 0.f;
-                for (int w = 0; w < 4; ++w) {
-                    te += sred[(w * GP + h) * 3 + 0];
-                    tw += sred[(w * GP + h) * 3 + 1];
-                    twq += sred[(w * GP + h) * 3 + 2];
-                }
-                float* hs = shead + h * 8;
-                const float alpha = sstat[h * 8 + 1];
-                hs[5] = hs[5] * alpha + te;
-                hs[6] = hs[6] * alpha + tw;
-                hs[7] = hs[7] * alpha + twq;
-            }
 
             // ---------------- phase V: value sums of the sub-chunk ----------------
             // Lane (g, t) of warp w reads the words of coordinates
@@ -661,8 +651,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                 const bool hi = g >= 4;
                 const float* ss = sstat + (head < G ? head : 0) * 8;
                 const float alpha = ss[1];
-                const float sgw = ss[2] * (1.f / 128.f);
-                const float sgq = ss[3] * (1.f / 128.f);
+                const float sgw = ss[2];
+                const float sgq = ss[3];
 #pragma unroll
                 for (int nt = 0; nt < NTV; ++nt) {
 #pragma unroll
@@ -713,6 +703,37 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
         }
 
         // ---------------- partials: {M, L, A[D], B[M]} per query head ----------------
+        // CTA-wide sums of this item's exp and weights (shead[h*8 + 5..7]).
+        {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int h = 0; h < GP; ++h) {
+                    pe[h] += __shfl_xor_sync(0xFFFFFFFFu, pe[h], o);
+                    pw[h] += __shfl_xor_sync(0xFFFFFFFFu, pw[h], o);
+                    pq[h] += __shfl_xor_sync(0xFFFFFFFFu, pq[h], o);
+                }
+            if (lane == 0)
+#pragma unroll
+                for (int h = 0; h < GP; ++h) {
+                    sred[(warp * GP + h) * 3 + 0] = pe[h];
+                    sred[(warp * GP + h) * 3 + 1] = pw[h];
+                    sred[(warp * GP + h) * 3 + 2] = pq[h];
+                }
+            __syncthreads();
+            if (tid < GP) {
+                float te = 0.f, tw = 0.f, twq = 0.f;
+                for (int w = 0; w < 4; ++w) {
+                    te += sred[(w * GP + tid) * 3 + 0];
+                    tw += sred[(w * GP + tid) * 3 + 1];
+                    twq += sred[(w * GP + tid) * 3 + 2];
+                }
+                shead[tid * 8 + 5] = te;
+                shead[tid * 8 + 6] = tw;
+                shead[tid * 8 + 7] = twq;
+            }
+            __syncthreads();
+        }
         constexpr int PART = 2 + D + M;
         {
             const int head = (G <= 4) ? (g & 3) : g;
@@ -730,10 +751,13 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                         if (QJL) pp[2 + D + coord] = accB[nt][c] - hs[7];
                     }
             }
-            if (tid < G) {
-                float* pp = a.part + ((qh0 + tid) * a.nsplit + split) * PART;
-                pp[0] = shead[tid * 8 + 4];
-                pp[1] = shead[tid * 8 + 5];
+#pragma unroll
+            for (int h = 0; h < GP; ++h) {
+                if (tid == h && h < G) {
+                    float* pp = a.part + ((qh0 + h) * a.nsplit + split) * PART;
+                    pp[0] = mrun[h];
+                    pp[1] = shead[h * 8 + 5];
+                }
             }
         }
     }
