@@ -58,21 +58,28 @@ def parse():
 # plumbing
 # ----------------------------------------------------------------------------
 class Dist:
-    def __init__(self, n_gpus: int):
+    """One process per GPU (torchrun env).  Only a barrier and a max-reduction of
+    timings cross ranks: each rank works on its own layer / sequences.  The
+    backend is NCCL on the GPUs ("gloo" on CPU for the multi-rank host tests)."""
+
+    def __init__(self, n_gpus: int, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         if self.world != n_gpus:
             raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={self.world}")
         self.pg = None
+        self.dev = torch.device("cuda", self.local) if backend == "nccl" else torch.device("cpu")
         if self.world > 1:
             import datetime
 
             import torch.distributed as dist
 
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {}
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = self.dev
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.pg = dist
 
     def barrier(self):
@@ -82,13 +89,18 @@ class Dist:
     def max(self, x: float) -> float:
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms_max: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (ms_max / 1e3)
 
 
 def peaks():
@@ -421,7 +433,7 @@ def run_ours(args):
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         cpu = cpu_baseline(q["sample_input"], args.cpu_vectors)
     if dist.rank == 0:
-        value = dist.world * q["tokens_per_step"] * args.steps / (q["ms"] / 1e3)
+        value = whole_job_rate(dist.world, q["tokens_per_step"] * args.steps, q["ms"])
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": q["ms"] / args.steps, "higher_is_better": True,
