@@ -1,9 +1,9 @@
 // quantize_inst.cu -- instantiates the quantize kernels of one (d, b), given
 // as -DKVQ_D=<d> -DKVQ_B=<b> by the build; the build compiles this file once
 // per supported pair so that the twelve instantiations compile in parallel.
-// 16-bit input with d <= 128 takes the tensor-core rotation kernel
-// (quantize_tc.cuh); fp32 input, d = 256 and the NSN front end take the
-// kernel with the in-register transform (quantize.cuh).
+// 16-bit input with d <= 128 (with or without the NSN front end) takes the
+// tensor-core rotation kernel (quantize_tc.cuh); fp32 input and d = 256 take
+// the kernel with the in-register transform (quantize.cuh).
 #include "quantize_tc.cuh"
 
 #ifndef KVQ_D
@@ -24,6 +24,12 @@ template <int D, int B, bool QJL, bool NSN>
 cudaError_t by_dtype(const CUtensorMap& map, int dtype, const QuantArgs& a, int sms, cudaStream_t s) {
     if constexpr (NSN && (QJL || D > 128)) {
         return cudaErrorNotSupported;
+    } else if constexpr (NSN) {
+        switch (dtype) {
+            case DT_F32: return launch_quantize_t<D, B, false, DT_F32, true>(map, a, sms, s);
+            case DT_F16: return launch_quantize_tc<D, B, false, DT_F16, true>(map, a, sms, s);
+            default: return launch_quantize_tc<D, B, false, DT_BF16, true>(map, a, sms, s);
+        }
     } else {
         switch (dtype) {
             case DT_F32:

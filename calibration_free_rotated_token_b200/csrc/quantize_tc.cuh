@@ -1,5 +1,5 @@
-// quantize_tc.cuh -- the quantize kernel with the rotation on the tensor
-// cores, for 16-bit input and d <= 128.
+// quantize_tc.cuh -- the quantize kernel (and its NSN front end) with the
+// rotation on the tensor cores, for 16-bit input and d <= 128.
 //
 // Method (TurboQuant blog, "Estagio 1" and "Estagio 2"; PolarQuant section 2),
 // per vector x: y = H (delta .* x) (unnormalised Sylvester Hadamard, so
@@ -27,6 +27,10 @@
 //   standard deviation), so a sign can differ from the exact one only where
 //   |(S r)_i| is a few 1e-4 ||r||, inside the 1e-3 ||r|| band where the sign
 //   is not pinned (a flip outside it needs a 5-sigma error, ~1e-11 per bit).
+// * NSN front end ([NSN] "NSNQuant" sections 1-2): the tile is one block of
+//   128 tokens; sc = sqrt(d)/||x|| from the staged tile, the channel means
+//   of u = sc x and their fp16 rounding o, and ho = H (delta .* o) by a
+//   one-warp FWHT; the rotation of w = u - o is then sc y - ho.
 // * Every mbarrier wait is bounded and its outcome agreed on by the
 //   warpgroup; loads still in flight at exit are waited for.
 #pragma once
@@ -35,7 +39,7 @@
 
 namespace kvq {
 
-template <int D, bool QJL>
+template <int D, bool QJL, bool NSN = false>
 struct TcCfg {
     static constexpr int kTileBytes = kTileRows * D * 2;   // 16-bit input
     static constexpr int kBoxBytes = 128 * kTileRows;      // 64 elements x 128 rows
@@ -43,7 +47,7 @@ struct TcCfg {
     static constexpr int kMatBytes = D * D * 2;            // H D or S, 16-bit, K-major, swizzled
     static constexpr int kWG = 4;
     static constexpr int kThreads = 128 * kWG;
-    static constexpr int kAuxBytes = 1024;
+    static constexpr int kAuxBytes = NSN ? 12288 : 1024;  // NSN: per-warpgroup scale, partial means, mean, rotated mean
     static constexpr int kBudget = 225 * 1024;
     static constexpr int kStagesRaw = (kBudget - kMatBytes - (QJL ? kMatBytes : 0) - kAuxBytes) / kTileBytes;
     // Tile i goes to warpgroup i % 4 and stage i % kStages; with kStages a
@@ -66,10 +70,44 @@ __device__ __forceinline__ uint32_t sign_word(const uint32_t (&u)[32]) {
     return ~(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24));
 }
 
-template <int D, int B, bool QJL, int DT>
+// Sum of squares of row r of a 16-bit stage (boxes of 64 elements x 128
+// rows, 128-byte swizzle: 16-byte chunk c of row r at c ^ (r & 7)).
+template <int D, int DT>
+__device__ __forceinline__ float stage_row_sumsq(const uint8_t* sp, int r) {
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int box = 0; box < D / 64; ++box) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 q = *reinterpret_cast<const uint4*>(sp + box * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 v;
+                if (DT == DT_BF16) v = make_float2(u2f(w[k] << 16), u2f(w[k] & 0xFFFF0000u));
+                else v = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+                if (k & 1) a1 = __ffma2_rn(v, v, a1);
+                else a0 = __ffma2_rn(v, v, a0);
+            }
+        }
+    }
+    a0 = __fadd2_rn(a0, a1);
+    return a0.x + a0.y;
+}
+
+// Element (t, j) of a 16-bit stage as fp32.
+template <int DT>
+__device__ __forceinline__ float stage_elem(const uint8_t* sp, int t, int j) {
+    const uint8_t* p = sp + (j / 64) * 16384 + t * 128 + ((((j % 64) / 8) ^ (t & 7)) << 4) + (j % 8) * 2;
+    const uint16_t hv = *reinterpret_cast<const uint16_t*>(p);
+    return (DT == DT_BF16) ? u2f(static_cast<uint32_t>(hv) << 16) : __half2float(*reinterpret_cast<const __half*>(&hv));
+}
+
+template <int D, int B, bool QJL, int DT, bool NSN = false>
 __global__ void __launch_bounds__(512, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap map, const __grid_constant__ QuantArgs a) {
-    using C = TcCfg<D, QJL>;
+    static_assert(!(NSN && QJL), "NSN front end: no QJL");
+    using C = TcCfg<D, QJL, NSN>;
     constexpr int NS = C::kStages;
     constexpr int kWpp = D / 32;
     constexpr uint32_t kIdescH = idesc_16bit_f32(kTileRows, D, DT == DT_BF16);
@@ -87,6 +125,7 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t* iss = reinterpret_cast<uint32_t*>(qbar + 4);  // [8] loads issued per stage
     uint32_t* con = iss + 8;                                // [8] loads consumed per stage
     uint32_t* tmem_slot = con + 8;
+    float* nsn_aux = reinterpret_cast<float*>(aux + 1024);  // NSN: [4 warpgroups][640]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -195,6 +234,82 @@ __global__ void __launch_bounds__(512, 1)
             }
             mma_commit(&hbar[wg]);
         }
+        // NSN front end on the tile (= one block of 128 tokens of one head):
+        // sc = sqrt(D)/||x||, block mean o of u = sc x per channel, fp16(o),
+        // and ho = H (delta .* fp16(o)), so that H D w = sc y - ho.
+        float nx = 0.f, sc = 0.f;
+        float* xch = nsn_aux + wg * 640;  // [128] sc per token
+        float* so = xch + 128;            // [D] delta .* fp16(o)
+        float* ho = xch + 256;            // [D] H (delta .* fp16(o))
+        float2* opart = reinterpret_cast<float2*>(xch + 384);  // [128 / (D/2)][D/2] partial channel sums
+        if constexpr (NSN) {
+            const uint8_t* sp = stage0 + st * C::kTileBytes;
+            const float ssx0 = stage_row_sumsq<D, DT>(sp, r);
+            nx = sqrtf(ssx0);
+            flag_norm(ssx0, nx, a.status);
+            sc = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
+            xch[r] = sc;
+            named_bar_sync(bar_id, 128);
+            {
+                // thread r: channel pair p, tokens of group q (fp32x2 sums)
+                constexpr int P = D / 2, Q = kTileRows / P, TPQ = kTileRows / Q;
+                const int p = r % P, q = r / P;
+                const int j0 = 2 * p;
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+                for (int t = q * TPQ; t < (q + 1) * TPQ; ++t) {
+                    const uint32_t wd = *reinterpret_cast<const uint32_t*>(
+                        sp + (j0 / 64) * 16384 + t * 128 + ((((j0 % 64) / 8) ^ (t & 7)) << 4) + (j0 % 8) * 2);
+                    const float2 xv = (DT == DT_BF16) ? make_float2(u2f(wd << 16), u2f(wd & 0xFFFF0000u))
+                                                      : __half22float2(*reinterpret_cast<const __half2*>(&wd));
+                    const float sct = xch[t];
+                    acc = __ffma2_rn(xv, make_float2(sct, sct), acc);
+                }
+                opart[q * P + p] = acc;
+            }
+            named_bar_sync(bar_id, 128);
+            if (r < D) {
+                constexpr int P = D / 2, Q = kTileRows / P;
+                float acc = 0.f;
+#pragma unroll
+                for (int q = 0; q < Q; ++q) {
+                    const float2 pq = opart[q * P + r / 2];
+                    acc += (r & 1) ? pq.y : pq.x;
+                }
+                const __half o16 = __float2half_rn(acc * (1.0f / kTileRows));
+                if (tile * kTileRows < a.n) a.block_mean[tile * D + r] = o16;
+                const uint32_t ps = a.pair_sign[r >> 1];
+                const bool neg = ((ps >> ((r & 1) ? 31 : 15)) & 1u) != 0;
+                so[r] = neg ? -__half2float(o16) : __half2float(o16);
+            }
+            named_bar_sync(bar_id, 128);
+            if ((warp & 3) == 0) {
+                // Sylvester FWHT of so in one warp: element VPL*lane + k
+                constexpr int VPL = D / 32;
+                float v[VPL];
+#pragma unroll
+                for (int k = 0; k < VPL; ++k) v[k] = so[VPL * lane + k];
+#pragma unroll
+                for (int h = 1; h < VPL; h <<= 1)
+#pragma unroll
+                    for (int k = 0; k < VPL; ++k)
+                        if ((k & h) == 0) {
+                            const float x0 = v[k], x1 = v[k + h];
+                            v[k] = x0 + x1;
+                            v[k + h] = x0 - x1;
+                        }
+#pragma unroll
+                for (int hl = 1; hl < 32; hl <<= 1)
+#pragma unroll
+                    for (int k = 0; k < VPL; ++k) {
+                        const float o = __shfl_xor_sync(0xFFFFFFFFu, v[k], hl);
+                        v[k] = (lane & hl) ? o - v[k] : v[k] + o;
+                    }
+#pragma unroll
+                for (int k = 0; k < VPL; ++k) ho[VPL * lane + k] = v[k];
+            }
+            named_bar_sync(bar_id, 128);
+        }
         const bool okh = mbar_wait(&hbar[wg], hpar, a.status);
         hpar ^= 1u;
         if (named_bar_or(bar_id, 128, !okh)) break;
@@ -212,14 +327,18 @@ __global__ void __launch_bounds__(512, 1)
             if (c + 1 < NC) tmem_ld32(tl + 32 * (c + 1), ybuf[(c + 1) & 1]);
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const float2 y = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
+                float2 y = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
+                if constexpr (NSN) {
+                    const float2 h2 = reinterpret_cast<const float2*>(ho)[16 * c + k];
+                    y = __ffma2_rn(y, make_float2(sc, sc), make_float2(-h2.x, -h2.y));  // H D w
+                }
                 acc2 = __ffma2_rn(y, y, acc2);
             }
             if (c + 1 < NC) tmem_wait_ld();
         }
         const float ssx = (acc2.x + acc2.y) * (1.0f / D);
-        const float nrm = sqrtf(ssx);
-        flag_norm(ssx, nrm, a.status);
+        const float nrm = sqrtf(ssx);  // ||x||, or ||w|| for NSN
+        if (!NSN) flag_norm(ssx, nrm, a.status);
         const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
 
         // ---- pass 2: codes, residual (fp16 into columns [16c, 16c + 16)) ----
@@ -234,7 +353,13 @@ __global__ void __launch_bounds__(512, 1)
             if (c + 1 < NC) tmem_ld32(tl + 32 * (c + 1), ybuf[(c + 1) & 1]);
             float2 v[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
+            for (int k = 0; k < 16; ++k) {
+                v[k] = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
+                if constexpr (NSN) {
+                    const float2 h2 = reinterpret_cast<const float2*>(ho)[16 * c + k];
+                    v[k] = __ffma2_rn(v[k], make_float2(sc, sc), make_float2(-h2.x, -h2.y));
+                }
+            }
             uint32_t pl[B][1];
             rr += codes_and_residual<32, B>(v, inv, a, pl);
 #pragma unroll
@@ -268,7 +393,8 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (valid) {
             const float g = nrm > 0.f ? sqrtf(rr) : 0.f;
-            a.norms[vidx] = __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
+            a.norms[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
+                                : __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
         }
 
         if (QJL) {
@@ -332,10 +458,10 @@ __global__ void __launch_bounds__(512, 1)
     }
 }
 
-template <int D, int B, bool QJL, int DT>
+template <int D, int B, bool QJL, int DT, bool NSN = false>
 cudaError_t launch_quantize_tc(const CUtensorMap& map, const QuantArgs& a, int num_sms, cudaStream_t s) {
-    using C = TcCfg<D, QJL>;
-    auto kern = quantize_tc_kernel<D, B, QJL, DT>;
+    using C = TcCfg<D, QJL, NSN>;
+    auto kern = quantize_tc_kernel<D, B, QJL, DT, NSN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t grid = a.ntiles < num_sms ? a.ntiles : num_sms;
