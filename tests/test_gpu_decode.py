@@ -112,6 +112,8 @@ def test_tiny_reference_workload():
     (64, 4, False, 2, 4, 2, [0, 257], 320, torch.bfloat16),           # an empty context
     (256, 2, True, 1, 4, 2, [400], 512, torch.bfloat16),
     (256, 4, False, 1, 2, 1, [129], 160, torch.bfloat16),
+    (128, 1, False, 1, 2, 2, [300], 320, torch.bfloat16),            # tensor-core path, GQA 1:1
+    (128, 2, False, 2, 4, 1, [900, 64], 960, torch.float16),          # tensor-core path without QJL
 ])
 def test_decode_matches_oracle(d, b, qjl, batch, hq, hkv, seq_len, cap, qdt):
     check_case(d, b, qjl, batch, hq, hkv, seq_len, cap, scale=1 / np.sqrt(d), qdtype=qdt)
@@ -182,3 +184,53 @@ def test_decode_workload_full_size_sampled():
     """batch 16, 32/8 heads, d 128, 131072-token contexts, b=2 + QJL, q ~ N(0,1)/sqrt(128), scale 1."""
     c = wl.DECODE
     _sampled_stream_decode(c["batch"], c["hq"], c["hkv"], c["T"], sample=(5, 3))
+
+
+@pytest.mark.parametrize("d,b,qjl", [(64, 1, False), (64, 3, True), (128, 2, True), (128, 4, False),
+                                     (256, 2, False)])
+def test_sweep_decode_full_size_sampled(d, b, qjl):
+    """Bit-width / head-dim sweep: the 1,048,576 bf16 vectors (1% x10) as 8 KV heads x 131072 tokens,
+    quantized as K and V by the CUDA path, one N(0,1) query per KV head; one sampled head is checked
+    against the oracle's quantization on sampled rows and then replaced by the oracle's own cache,
+    whose decode the oracle recomputes."""
+    c = wl.SWEEP
+    H, T = c["hkv"], c["T"]
+    k = constants(d, b, c["handle_seed"])
+    X = wl.sweep_tokens(c["n"], d, seed=c["seed"] + d, device="cuda").reshape(H, T, d)
+    Y = wl.sweep_tokens(c["n"], d, seed=c["seed"] + d + 500, device="cuda").reshape(H, T, d)
+    hs = 3
+    with kvq.Handle(d, b, c["handle_seed"], qjl=qjl) as h:
+        kcodes, kqjl, knorm = kvq.alloc_packed(h, H * T)
+        kvq.kvq_quantize(h, X.reshape(-1, d), kcodes, kqjl, knorm)
+        vcodes = torch.empty((H, T // 32, b, d), dtype=torch.int32, device="cuda")
+        vqjl = torch.empty((H, T // 32, d), dtype=torch.int32, device="cuda") if qjl else None
+        vnorm = torch.empty((H, T, 2), dtype=torch.float16, device="cuda")
+        for hk in range(H):
+            kvq.kvq_quantize(h, Y[hk], vcodes[hk], vqjl[hk] if qjl else None, vnorm[hk], layout=1)
+        assert kvq.kvq_status(h)[0] == 0
+        kcodes = kcodes.reshape(H, T, b, d // 32)
+        kqjl = kqjl.reshape(H, T, d // 32) if qjl else None
+        knorm = knorm.reshape(H, T, 2)
+        Xs = X[hs].double().cpu().numpy()
+        Ys = Y[hs].double().cpu().numpy()
+        rows = np.sort(np.random.default_rng(d + b).choice(T, 512, replace=False))
+        tr = torch.from_numpy(rows).cuda()
+        compare_quantize(k, Xs[rows], to_np_u32(kcodes[hs][tr]), to_np_u32(kqjl[hs][tr]) if qjl else None,
+                         to_np_f16bits(knorm[hs][tr]), qjl)
+        ck, qk, nk, sk = oracle_cache(k, Xs, qjl)
+        cv, qv_, nv, sv = oracle_cache(k, Ys, qjl, layout=1)
+        kcodes[hs] = to_device_u32(ck).reshape(T, b, d // 32)
+        knorm[hs] = torch.from_numpy(nk).cuda()
+        vcodes[hs] = to_device_u32(cv).reshape(T // 32, b, d)
+        vnorm[hs] = torch.from_numpy(nv).cuda()
+        if qjl:
+            kqjl[hs] = to_device_u32(qk)
+            vqjl[hs] = to_device_u32(qv_)
+        q = wl.queries(1, H, d, seed=c["seed"] + 7, device="cuda")
+        kc = kvq.make_cache(kcodes, kqjl, knorm, T, 0)
+        vc = kvq.make_cache(vcodes, vqjl, vnorm, T, 1)
+        out, _ = run_decode(h, q, H, kc, vc, [T], T, 1.0 / np.sqrt(d), want_logits=False)
+    _, orf = oracle.decode_attend(k, q[0, hs:hs + 1].double().cpu().numpy(), sk, sv, 1.0 / np.sqrt(d), qjl,
+                                  want_logits=False)
+    assert_close(out[0, hs:hs + 1], orf, "out (sampled head)")
+    assert np.isfinite(out).all()
