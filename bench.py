@@ -38,7 +38,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
@@ -101,6 +101,22 @@ class Dist:
 def whole_job_rate(world: int, units_per_rank: float, ms_max: float) -> float:
     """Whole-job throughput: the units every rank processed over the slowest rank's time."""
     return world * units_per_rank / (ms_max / 1e3)
+
+
+def tensor_record(n: int, d: int, launch_s: float) -> dict:
+    """Algorithmic tensor-core throughput of one quantize launch: the S r
+    projection (2 m d flop per vector, m = d) and the Hadamard rotation (2 d^2)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak, src = 1590.0, "fallback"
+    if os.path.exists(p):
+        with open(p) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured"
+    sr = 2.0 * d * d * n / launch_s / 1e12
+    rot = 2.0 * d * d * n / launch_s / 1e12
+    return {"sr_projection_tflops": round(sr, 1), "rotation_tflops": round(rot, 1),
+            "peak_bf16_tflops": peak, "peak_source": src, "frac": round((sr + rot) / peak, 4),
+            "note": "fp16 S r (one fp16 residual term) and bf16 x (H D)^T, fp32 accumulate; "
+                    "the S r contraction is the method's, the rotation is this kernel's choice"}
 
 
 def peaks():
@@ -267,9 +283,11 @@ def bench_quantize(args, dist):
     res = dict(ms=ms, tokens_per_step=T, vectors_per_step=2 * n, launches=2 * args.steps,
                roofline={"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(achieved / hbm, 4), "traffic": traffic_record("quantize_llama_layer"),
-                         "peak_source": f"{src} hbm_gbs (copy)", "kernel": "quantize_kernel<128,2,qjl,bf16>",
+                         "peak_source": f"{src} hbm_gbs (copy)", "kernel": "quantize_tc_kernel<128,2,qjl,bf16>",
                          "algorithmic_bytes_per_launch": per_launch_bytes,
-                         "avg_launch_ms": round(avg_launch_s * 1e3, 5)},
+                         "avg_launch_ms": round(avg_launch_s * 1e3, 5),
+                         "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4)},
+               tensor=tensor_record(n, d, avg_launch_s),
                clocks=clk.summary())
 
     # ---- end to end through the binding with host buffers ----
@@ -297,7 +315,8 @@ def bench_quantize(args, dist):
     res["e2e"] = {"value": dist.world * T * e2e_steps / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                   "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / e2e_steps,
                   "path": "pinned host K,V -> kvq_quantize (C ABI) -> pinned host codes, qjl, norms"}
-    res["sample_input"] = (copies[0][0][: args.cpu_vectors // 2].cpu(), copies[0][1][: args.cpu_vectors // 2].cpu())
+    rows = min(max(args.cpu_vectors, 8192 * (os.cpu_count() or 1)) // 2, n)  # enough for the sharded oracle run
+    res["sample_input"] = (copies[0][0][:rows].cpu(), copies[0][1][:rows].cpu())
     h.close()
     return res
 
@@ -353,7 +372,8 @@ def bench_decode(args, dist):
             "workload": f"batch 16, 32 query / 8 KV heads, d 128, {T}-token contexts, b=2 + QJL, one bf16 query token",
             "cache_bytes_per_step": cache_bytes, "launches_per_step": 3,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(gbs / hbm, 4), "traffic": traffic_record("decode_split"),
+                         "frac": round(gbs / hbm, 4), "frac_of_spec_8tbs": round(gbs / SPEC_HBM_GBS, 4),
+                         "traffic": traffic_record("decode_split"),
                          "peak_source": f"{src} hbm_gbs (copy)",
                          "note": "whole decode call (qproj + split + combine); the split kernel dominates"}}
 
@@ -388,8 +408,36 @@ def bench_nsn(args, dist):
     return {"metric": "NSN quantize tokens/s", "value": dist.world * T * steps / (ms / 1e3), "unit": "tokens/s",
             "ms_per_step": ms / steps, "workload": "8 heads x 65536 tokens x d128 bf16, b=2, no QJL",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                         "frac": round(gbs / hbm, 4), "traffic": traffic_record("nsn_quantize"),
+                         "frac": round(gbs / hbm, 4), "frac_of_spec_8tbs": round(gbs / SPEC_HBM_GBS, 4),
+                         "traffic": traffic_record("nsn_quantize"),
                          "peak_source": f"{src} hbm_gbs (copy)"}}
+
+
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e specification (DGX figure)
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_quantize_sharded(k, X, qjl: bool, threads: int):
+    """The oracle's quantize over row ranges of X on `threads` host threads
+    (the C oracle runs with the interpreter lock released; no shared state)."""
+    import concurrent.futures as cf
+
+    import oracle
+
+    chunks = [c for c in np.array_split(X, threads) if c.shape[0] > 0]
+    with cf.ThreadPoolExecutor(max_workers=len(chunks)) as ex:
+        list(ex.map(lambda c: oracle.quantize(k, c, qjl), chunks))
+    return len(chunks)
 
 
 def cpu_baseline(sample, n_vectors: int):
@@ -402,14 +450,28 @@ def cpu_baseline(sample, n_vectors: int):
     K, V = sample
     Kd = K.double().numpy()[: n_vectors // 2]
     Vd = V.double().numpy()[: n_vectors // 2]
+    # (i) one thread
     t0 = time.perf_counter()
     oracle.quantize(k, Kd, True)
     oracle.quantize(k, Vd, True)
-    dt = time.perf_counter() - t0
-    vec = Kd.shape[0] + Vd.shape[0]
-    return {"value": vec / 16 / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{vec} vectors ({vec // 16} tokens) of the layer's K and V, single-threaded fp64 C++, "
-                      f"{dt:.1f} s"}
+    dt1 = time.perf_counter() - t0
+    vec1 = Kd.shape[0] + Vd.shape[0]
+    # (ii) sharded over every host core (token ranges, no shared state)
+    cores = os.cpu_count() or 1
+    nsh = min(max(n_vectors, 8192 * cores), 2 * K.shape[0])
+    Ks = K.double().numpy()[: nsh // 2]
+    Vs = V.double().numpy()[: nsh // 2]
+    t0 = time.perf_counter()
+    used = oracle_quantize_sharded(k, Ks, True, cores)
+    oracle_quantize_sharded(k, Vs, True, cores)
+    dts = time.perf_counter() - t0
+    vecs = Ks.shape[0] + Vs.shape[0]
+    return {"value": vecs / 16 / dts, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"{vecs} vectors ({vecs // 16} tokens) of the layer's K and V, fp64 C++ oracle on {used} "
+                      f"host threads over token ranges, {dts:.1f} s",
+            "cpu_model": cpu_model(),
+            "single_thread": {"value": vec1 / 16 / dt1, "unit": UNIT, "cores": 1,
+                              "sample": f"{vec1} vectors, one thread, {dt1:.1f} s"}}
 
 
 def run_ours(args):
@@ -445,7 +507,8 @@ def run_ours(args):
                        "vectors_per_step": q["vectors_per_step"],
                        "l2": "4 rotating input copies per rank (4 x 134 MB > 126 MB L2)",
                        "parallelism": f"dp{dist.world} (independent layers per rank, no collective)"},
-            "roofline": q["roofline"], "cpu_baseline": cpu, "e2e": q["e2e"], "gpu_launches": q["launches"],
+            "roofline": q["roofline"], "tensor": q["tensor"], "cpu_baseline": cpu, "e2e": q["e2e"],
+            "gpu_launches": q["launches"],
             "clocks": q["clocks"],
         }
         line.update(extra)
@@ -463,26 +526,29 @@ def run_reference(args):
 
     c = wl.LLAMA_LAYER
     k = oracle.make_constants(c["d"], c["b"], c["handle_seed"])
-    per_step = 1024  # vectors per step: 64 positions x 8 heads of K, and of V
-    K = wl.llama_keys(c["heads"], 64, c["d"], c["k_seed"]).reshape(-1, c["d"]).double().numpy()
-    V = wl.llama_values(c["heads"], 64, c["d"], c["v_seed"]).reshape(-1, c["d"]).double().numpy()
+    cores = os.cpu_count() or 1
+    pos = 64 * cores                 # positions per step: 64 per host thread
+    per_step = 16 * pos              # vectors per step: 8 heads of K and of V per position
+    K = wl.llama_keys(c["heads"], pos, c["d"], c["k_seed"]).reshape(-1, c["d"]).double().numpy()
+    V = wl.llama_values(c["heads"], pos, c["d"], c["v_seed"]).reshape(-1, c["d"]).double().numpy()
     for i in range(args.warmup):
-        oracle.quantize(k, K[: per_step // 2], True)
-        oracle.quantize(k, V[: per_step // 2], True)
+        oracle_quantize_sharded(k, K, True, cores)
+        oracle_quantize_sharded(k, V, True, cores)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        oracle.quantize(k, K[: per_step // 2], True)
-        oracle.quantize(k, V[: per_step // 2], True)
+        used = oracle_quantize_sharded(k, K, True, cores)
+        oracle_quantize_sharded(k, V, True, cores)
     dt = time.perf_counter() - t0
     value = per_step / 16 * args.steps / dt
-    sample = f"{per_step} vectors ({per_step // 16} tokens) of the layer's K and V per step, single-threaded fp64 C++"
+    sample = (f"{per_step} vectors ({pos} tokens) of the layer's K and V per step, fp64 C++ oracle on {used} host "
+              f"threads over token ranges ({cpu_model()})")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": "llama3-8b-layer KV quantize: 8 KV heads x 32768 tokens x d128, bf16 K and V, "
                                    "2-bit Lloyd-Max + 1-bit QJL (m=128)",
                        "token": "one position of the layer = 8 heads x (K + V) = 16 vectors"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
