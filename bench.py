@@ -315,7 +315,7 @@ def bench_quantize(args, dist):
     res["e2e"] = {"value": dist.world * T * e2e_steps / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                   "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e / e2e_steps,
                   "path": "pinned host K,V -> kvq_quantize (C ABI) -> pinned host codes, qjl, norms"}
-    rows = min(max(args.cpu_vectors, 8192 * (os.cpu_count() or 1)) // 2, n)  # enough for the sharded oracle run
+    rows = min(max(args.cpu_vectors, 24576 * (os.cpu_count() or 1)) // 2, n)  # enough for the sharded oracle run
     res["sample_input"] = (copies[0][0][:rows].cpu(), copies[0][1][:rows].cpu())
     h.close()
     return res
@@ -458,7 +458,7 @@ def cpu_baseline(sample, n_vectors: int):
     vec1 = Kd.shape[0] + Vd.shape[0]
     # (ii) sharded over every host core (token ranges, no shared state)
     cores = os.cpu_count() or 1
-    nsh = min(max(n_vectors, 8192 * cores), 2 * K.shape[0])
+    nsh = min(max(n_vectors, 24576 * cores), 2 * K.shape[0])
     Ks = K.double().numpy()[: nsh // 2]
     Vs = V.double().numpy()[: nsh // 2]
     t0 = time.perf_counter()
