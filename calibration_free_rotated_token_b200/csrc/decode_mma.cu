@@ -95,6 +95,14 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y));
 }
+// The same with a zero accumulator input (first K-step of a chain).
+__device__ __forceinline__ void mma_u8s8_z(int (&d)[4], const uint32_t (&a)[4], uint2 b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y), "r"(0));
+}
 __device__ __forceinline__ void mma_u8u8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -251,7 +259,6 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     constexpr bool QF_REG = L::kQfReg;
     constexpr int HH = (G == 8) ? 2 : 1;      // query heads per lane in the logit epilogue
     extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t* stage[2] = {smem, smem + L::kStage};
     uint2* sfrag = reinterpret_cast<uint2*>(smem + 2 * L::kStage);
     float* slog = reinterpret_cast<float*>(smem + 2 * L::kStage + L::kFrag);  // [GP][TC]
     uint32_t* swc = reinterpret_cast<uint32_t*>(smem + 2 * L::kStage + L::kFrag + L::kLog);  // code-weight digits
@@ -331,7 +338,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             const int64_t have = min(static_cast<int64_t>(TC), t1 - tb);
             if (have <= 0) return false;
             const int64_t nt = (have + 31) / 32 * 32;  // <= capacity - tb (capacity is a multiple of 32)
-            uint8_t* st = stage[sc & 1];
+            uint8_t* st = smem + (sc & 1) * L::kStage;
             uint64_t* b = &bar[sc & 1];
             const uint32_t bytes = static_cast<uint32_t>(nt * (B * D / 8 + (QJL ? M / 8 : 0) + 4) +
                                                          (nt / 32) * (B * D * 4 + (QJL ? M * 4 : 0)) + nt * 4);
@@ -372,7 +379,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
         for (int sc = 0; sc < nsub; ++sc) {
             const int64_t tb = t0 + static_cast<int64_t>(sc) * TC;
             const int64_t have = min(static_cast<int64_t>(TC), t1 - tb);  // may be <= 0 (split past the context)
-            const uint8_t* st = stage[sc & 1];
+            const uint8_t* st = smem + (sc & 1) * L::kStage;
+            // tokens of the sub-chunk inside the context, and inside the split (32-bit)
+            const int nval = static_cast<int>(max(min(t1 - tb, static_cast<int64_t>(TC)), static_cast<int64_t>(0)));
+            const int nval_e = static_cast<int>(max(min(t1e - tb, static_cast<int64_t>(TC)), static_cast<int64_t>(0)));
             if (have > 0) {
                 const bool ok = mbar_wait(&bar[sc & 1], phase[sc & 1], a.status);
                 phase[sc & 1] ^= 1u;
@@ -392,11 +402,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             for (int mt = warp; mt < TC / 16; mt += 4) {
                 const int tl0 = mt * 16 + g, tl1 = tl0 + 8;
                 int accc[2][NTK][4], accq[NTK][4];  // code K-steps alternate between two chains
-#pragma unroll
-                for (int nt = 0; nt < NTK; ++nt)
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) accc[0][nt][r] = accc[1][nt][r] = accq[nt][r] = 0;
-                if (tb + mt * 16 < t1) {
+                if (mt * 16 < nval) {
                     uint32_t w0[KS], w1[KS];
 #pragma unroll
                     for (int q4 = 0; q4 < KWT / 4; ++q4) {
@@ -432,11 +438,27 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                             for (int nt = 0; nt < NTK; ++nt) {
                                 const uint2 bq = QF_REG ? qf[QF_REG ? ks : 0][QF_REG ? nt : 0]
                                                         : sfrag[(ks * NTK + nt) * 32 + lane];
-                                if (kind == 0) mma_u8s8(accc[i & 1][nt], af, bq);
-                                else mma_u8s8(accq[nt], af, bq);
+                                if (kind == 0) {
+                                    if (i < 2) mma_u8s8_z(accc[i & 1][nt], af, bq);
+                                    else mma_u8s8(accc[i & 1][nt], af, bq);
+                                } else {
+                                    if (i == 0) mma_u8s8_z(accq[nt], af, bq);
+                                    else mma_u8s8(accq[nt], af, bq);
+                                }
                             }
                         }
                     }
+                    if (KWT < 2) {
+#pragma unroll
+                        for (int nt = 0; nt < NTK; ++nt)
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) accc[1][nt][r] = 0;
+                    }
+                } else {
+#pragma unroll
+                    for (int nt = 0; nt < NTK; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) accc[0][nt][r] = accc[1][nt][r] = accq[nt][r] = 0;
                 }
                 // epilogue: thread t owns head t (and t + 4 when G = 8); its
                 // columns hold the four digits of the head
@@ -446,9 +468,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr) {
                         const int tl = rr ? tl1 : tl0;
-                        const int64_t tg = tb + tl;
-                        float l = -INFINITY;
-                        if (h < G && tg < t1) {
+                        float l;
+                        {
                             const int n0 = 2 * hh, n1 = 2 * hh + 1;
                             const float xc = fmaf(static_cast<float>((accc[0][n0][2 * rr] + accc[1][n0][2 * rr]) * 128 +
                                                                      accc[0][n0][2 * rr + 1] + accc[1][n0][2 * rr + 1]),
@@ -463,11 +484,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                                          static_cast<float>(accq[n1][2 * rr] * 128 + accq[n1][2 * rr + 1]));
                                 inner = fmaf(nk.y, fmaf(hk2[hh], xq, -hk3[hh]), inner);
                             }
-                            l = nk.x * inner;
+                            l = (h < G && tl < nval) ? nk.x * inner : -INFINITY;
                             lmax[hh] = fmaxf(lmax[hh], l);
                         }
                         if (h < GP) slog[h * TC + tl] = l;
-                        if (a.logits != nullptr && h < G && tg < t1e) a.logits[(qh0 + h) * a.max_T + tg] = l;
+                        if (a.logits != nullptr && h < G && tl < nval_e) a.logits[(qh0 + h) * a.max_T + tb + tl] = l;
                     }
                 }
             }
@@ -477,7 +498,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             {
                 float nmx = 0.f, ngx = 0.f;
                 for (int tl = tid; tl < TC; tl += kThreads) {
-                    if (tb + tl < t1) {
+                    if (tl < nval) {
                         const float2 nv = __half22float2(sVn[tl]);
                         nmx = fmaxf(nmx, nv.x);
                         ngx = fmaxf(ngx, nv.x * nv.y);
@@ -552,7 +573,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             // 16 + 4((u&7)-4) + (u>>3): lane 4(r&7) + (u&3), register
             // (r>>3) + 2((u&7)>>2), byte u>>3 of row r's fragment.
             for (int tl = tid; tl < TC; tl += kThreads) {
-                const bool valid = tb + tl < t1;
+                const bool valid = tl < nval;
                 const float2 nv = valid ? __half22float2(sVn[tl]) : make_float2(0.f, 0.f);
                 const int u = tl & 31, bb = tl >> 5, s = u & 7;
                 const float fac = static_cast<float>(1 << (7 - s));
@@ -560,9 +581,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                 uint8_t* bq = reinterpret_cast<uint8_t*>(swq) + (u >> 3);
 #pragma unroll
                 for (int h = 0; h < GP; ++h) {
-                    uint32_t xc = 0u, xq = 0u;
-                    if (valid && h < G) {
-                        const float e = __expf(slog[h * TC + tl] - mnew[h]);
+                    uint32_t xc, xq = 0u;
+                    {
+                        const float ex = __expf(slog[h * TC + tl] - mnew[h]);
+                        const float e = (valid && h < G) ? ex : 0.f;
                         const float wc = e * nv.x;
                         const float wq = wc * nv.y;
                         pe[h] += e;
