@@ -95,6 +95,37 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b.x), "r"(b.y));
 }
+// Operand quads as uint4 / pairs as uint2 (lets the allocator keep them in
+// aligned register groups).
+__device__ __forceinline__ void mma_u8s8_q(int (&d)[4], uint4 a, uint2 b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y));
+}
+__device__ __forceinline__ void mma_u8s8_qz(int (&d)[4], uint4 a, uint2 b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(0));
+}
+__device__ __forceinline__ void mma_u8u8_q(int (&d)[4], uint4 a, uint2 b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y));
+}
+__device__ __forceinline__ void mma_u8u8_qz(int (&d)[4], uint4 a, uint2 b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(0));
+}
+
 // The same with a zero accumulator input (first K-step of a chain).
 __device__ __forceinline__ void mma_u8s8_z(int (&d)[4], const uint32_t (&a)[4], uint2 b) {
     asm volatile(
@@ -432,18 +463,18 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                         for (int kind = 0; kind < 2; ++kind) {
                             if (kind == 0 ? (i >= KWT) : (i >= QWT)) continue;
                             const int ks = kind == 0 ? i : KWT + i;
-                            const uint32_t af[4] = {w0[ks] & msk_lo, w1[ks] & msk_lo, w0[ks] & msk_hi,
-                                                    w1[ks] & msk_hi};
+                            const uint4 af = make_uint4(w0[ks] & msk_lo, w1[ks] & msk_lo, w0[ks] & msk_hi,
+                                                        w1[ks] & msk_hi);
 #pragma unroll
                             for (int nt = 0; nt < NTK; ++nt) {
                                 const uint2 bq = QF_REG ? qf[QF_REG ? ks : 0][QF_REG ? nt : 0]
                                                         : sfrag[(ks * NTK + nt) * 32 + lane];
                                 if (kind == 0) {
-                                    if (i < 2) mma_u8s8_z(accc[i & 1][nt], af, bq);
-                                    else mma_u8s8(accc[i & 1][nt], af, bq);
+                                    if (i < 2) mma_u8s8_qz(accc[i & 1][nt], af, bq);
+                                    else mma_u8s8_q(accc[i & 1][nt], af, bq);
                                 } else {
-                                    if (i == 0) mma_u8s8_z(accq[nt], af, bq);
-                                    else mma_u8s8(accq[nt], af, bq);
+                                    if (i == 0) mma_u8s8_qz(accq[nt], af, bq);
+                                    else mma_u8s8_q(accq[nt], af, bq);
                                 }
                             }
                         }
@@ -613,26 +644,14 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             // coordinate w D/4 + NTV n + nt.
             {
                 int accv[NPV][NTV][RT][4];
-#pragma unroll
-                for (int p = 0; p < NPV; ++p)
-#pragma unroll
-                    for (int nt = 0; nt < NTV; ++nt)
-#pragma unroll
-                        for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-                            for (int r = 0; r < 4; ++r) accv[p][nt][rt][r] = 0;
-                const int nblk = have > 0 ? static_cast<int>((have + 31) / 32) : 0;
+                const int nblk = nval > 0 ? (nval + 31) / 32 : 0;
                 const int cbase = warp * (D / 4) + NTV * g;
-                for (int bb = 0; bb < nblk; ++bb) {
-                    uint32_t aw[RT][4], aq[RT][4];
+                auto vblock = [&](int bb, bool first) {
+                    uint4 aw[RT], aq[RT];
 #pragma unroll
                     for (int rt = 0; rt < RT; ++rt) {
-                        const uint4 x = reinterpret_cast<const uint4*>(swc)[(bb * RT + rt) * 32 + lane];
-                        aw[rt][0] = x.x; aw[rt][1] = x.y; aw[rt][2] = x.z; aw[rt][3] = x.w;
-                        if (QJL) {
-                            const uint4 y = reinterpret_cast<const uint4*>(swq)[(bb * RT + rt) * 32 + lane];
-                            aq[rt][0] = y.x; aq[rt][1] = y.y; aq[rt][2] = y.z; aq[rt][3] = y.w;
-                        }
+                        aw[rt] = reinterpret_cast<const uint4*>(swc)[(bb * RT + rt) * 32 + lane];
+                        if (QJL) aq[rt] = reinterpret_cast<const uint4*>(swq)[(bb * RT + rt) * 32 + lane];
                     }
 #pragma unroll
                     for (int p = 0; p < NPV; ++p) {
@@ -653,14 +672,28 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                         }
 #pragma unroll
                         for (int nt = 0; nt < NTV; ++nt) {
-                            const uint32_t b0 = wv[nt] & msk_lo, b1 = wv[nt] & msk_hi;
+                            const uint2 bv = make_uint2(wv[nt] & msk_lo, wv[nt] & msk_hi);
 #pragma unroll
                             for (int rt = 0; rt < RT; ++rt) {
-                                if (p < B) mma_u8u8(accv[p][nt][rt], aw[rt], b0, b1);
-                                else mma_u8u8(accv[p][nt][rt], aq[rt], b0, b1);
+                                const uint4 af = (p < B) ? aw[rt] : aq[(QJL ? rt : 0)];
+                                if (first) mma_u8u8_qz(accv[p][nt][rt], af, bv);
+                                else mma_u8u8_q(accv[p][nt][rt], af, bv);
                             }
                         }
                     }
+                };
+                if (nblk > 0) {
+                    vblock(0, true);
+                    for (int bb = 1; bb < nblk; ++bb) vblock(bb, false);
+                } else {
+#pragma unroll
+                    for (int p = 0; p < NPV; ++p)
+#pragma unroll
+                        for (int nt = 0; nt < NTV; ++nt)
+#pragma unroll
+                            for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                                for (int r = 0; r < 4; ++r) accv[p][nt][rt][r] = 0;
                 }
                 // Merge into the fp32 running sums (rescaled by alpha).  Digit k
                 // of head h sits in row h + 4k (G <= 4): lane g < 4 holds digits
