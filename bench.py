@@ -236,21 +236,11 @@ def bench_quantize(args, dist):
     outK = kvq.alloc_packed(h, n)                                  # keys: one record per token
     outV = kvq.alloc_packed(h, n, layout=kvq.KVQ_LAYOUT_BLOCK32)    # values: blocks of 32 tokens
     stream = torch.cuda.current_stream()
-    launch_ev = []
 
-    def step(i, record=False):
+    def step(i):
         K, V = copies[i % 4]
-        if record:
-            a, bq, cq = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-            a.record(stream)
-            kvq.kvq_quantize(h, K, *outK, stream=stream)
-            bq.record(stream)
-            kvq.kvq_quantize(h, V, *outV, stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
-            cq.record(stream)
-            launch_ev.append((a, bq, cq))
-        else:
-            kvq.kvq_quantize(h, K, *outK, stream=stream)
-            kvq.kvq_quantize(h, V, *outV, stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
+        kvq.kvq_quantize(h, K, *outK, stream=stream)
+        kvq.kvq_quantize(h, V, *outV, stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
 
     for i in range(args.warmup):
         step(i)
@@ -267,17 +257,17 @@ def bench_quantize(args, dist):
             i += 1
             if i % 64 == 0:
                 torch.cuda.synchronize()
-        ms = timed(dist, lambda i: step(i, record=True), args.steps, stream)
-    launch_ms = []
-    for a, bq, cq in launch_ev:
-        launch_ms += [a.elapsed_time(bq), bq.elapsed_time(cq)]
+        ms = timed(dist, step, args.steps, stream)
     code, bits = kvq.kvq_status(h)
     if code != 0:
         raise RuntimeError(f"quantize status {code} bits {bits}")
 
     bytes_per_vec = 2 * d + b * d // 8 + d // 8 + 4
     per_launch_bytes = n * bytes_per_vec
-    avg_launch_s = float(np.mean(launch_ms)) / 1e3
+    # The timed region holds nothing but the quantize launches (two per step,
+    # back to back on one stream, so each next launch's set-up overlaps the
+    # previous one's tail): the average launch is the region over the launches.
+    avg_launch_s = ms / (2 * args.steps) / 1e3
     hbm, src = peaks()
     achieved = per_launch_bytes / avg_launch_s / 1e9
     res = dict(ms=ms, tokens_per_step=T, vectors_per_step=2 * n, launches=2 * args.steps,

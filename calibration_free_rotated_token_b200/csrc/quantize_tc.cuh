@@ -189,6 +189,10 @@ __global__ void __launch_bounds__(512, 1)
     // Launched as a programmatic dependent: the input may come from the grid
     // before this one, so nothing global is read or written before this.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Let the next programmatic dependent be scheduled now: its CTAs take an
+    // SM as soon as one of ours exits, so their set-up overlaps our tail (it
+    // still waits for this whole grid before it reads or writes memory).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // Tile i (local index) lives in stage i % NS.
     auto issue_tile = [&](int64_t i) {
