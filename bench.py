@@ -44,8 +44,9 @@ def parse():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-attention measurement")
     ap.add_argument("--no-nsn", action="store_true", help="skip the NSN front-end measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the bit-width / head-dim sweep")
     ap.add_argument("--cpu-vectors", type=int, default=163840, help="vectors in the CPU oracle sample")
-    ap.add_argument("--only", choices=("quantize", "decode", "nsn"), default=None,
+    ap.add_argument("--only", choices=("quantize", "decode", "nsn", "sweep"), default=None,
                     help="run one part only (for profiler captures); prints that part's result")
     ap.add_argument("--decode-T", type=int, default=None,
                     help="context length of the decode measurement (default: the workload's 131072)")
@@ -403,6 +404,70 @@ def bench_nsn(args, dist):
                          "peak_source": f"{src} hbm_gbs (copy)"}}
 
 
+def bench_sweep(args, dist):
+    """Bit-width / head-dim sweep: per (d, b, QJL), the quantize of 2^20 keys and
+    2^20 values (bf16 N(0, 1), 1% of the tokens x10) and one decode over them as
+    8 KV heads x 131072 tokens with one query per head (scale 1/sqrt(d))."""
+    from calibration_free_rotated_token_b200 import _abi as kvq
+    from calibration_free_rotated_token_b200 import workloads as wl
+
+    c = wl.SWEEP
+    n, hkv, T = c["n"], c["hkv"], c["T"]
+    hbm, src = peaks()
+    stream = torch.cuda.current_stream()
+    steps = max(5, args.steps // 3)
+    rows = []
+    for d in c["dims"]:
+        X = [wl.sweep_tokens(n, d, c["seed"] + 2 * d + i + 1000 * dist.rank, device="cuda") for i in range(2)]
+        q = wl.queries(1, hkv, d, c["seed"] + 7 * d, device="cuda")
+        seq = torch.full((1,), T, dtype=torch.int32, device="cuda")
+        out = torch.empty((1, hkv, d), dtype=torch.float32, device="cuda")
+        for b in c["bits"]:
+            for qjl in c["qjl"]:
+                h = kvq.Handle(d, b, c["handle_seed"], qjl=qjl)
+                outK = kvq.alloc_packed(h, n)
+                outV = kvq.alloc_packed(h, n, layout=kvq.KVQ_LAYOUT_BLOCK32)
+
+                def qstep(i):
+                    kvq.kvq_quantize(h, X[0], *outK, stream=stream)
+                    kvq.kvq_quantize(h, X[1], *outV, stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
+
+                for i in range(3):
+                    qstep(i)
+                ms_q = timed(dist, qstep, steps, stream)
+                kcache = kvq.make_cache(*outK, T, kvq.KVQ_LAYOUT_TOKEN)
+                vcache = kvq.make_cache(*outV, T, kvq.KVQ_LAYOUT_BLOCK32)
+                ws = torch.empty(kvq.kvq_decode_workspace(h, 1, hkv, hkv, T), dtype=torch.uint8, device="cuda")
+
+                def dstep(i):
+                    kvq.kvq_decode_attend(h, q, hkv, kcache, vcache, seq, T, d ** -0.5, out, ws, stream=stream)
+
+                for i in range(3):
+                    dstep(i)
+                ms_d = timed(dist, dstep, steps, stream)
+                code, bits = kvq.kvq_status(h)
+                if code != 0:
+                    raise RuntimeError(f"sweep d={d} b={b} qjl={qjl}: status {code} bits {bits}")
+                rec = b * d // 8 + (d // 8 if qjl else 0) + 4  # packed bytes per vector
+                q_gbs = n * (2 * d + rec) / (ms_q / (2 * steps) / 1e3) / 1e9
+                d_gbs = 2 * n * rec / (ms_d / steps / 1e3) / 1e9
+                rows.append({"d": d, "b": b, "qjl": qjl,
+                             "quantize_us": round(ms_q / (2 * steps) * 1e3, 2), "quantize_gbs": round(q_gbs, 1),
+                             "quantize_frac": round(q_gbs / hbm, 4),
+                             "quantize_kernel": "quantize_tc_kernel" if d <= 128 else "quantize_kernel",
+                             "decode_us": round(ms_d / steps * 1e3, 2), "decode_gbs": round(d_gbs, 1),
+                             "decode_frac": round(d_gbs / hbm, 4),
+                             "decode_kernel": "decode_mma_kernel" if b <= 2 else "decode_split_kernel"})
+                h.close()
+                del outK, outV, kcache, vcache, ws
+        del X
+    return {"workload": "per (d, b, QJL): quantize 2^20 keys + 2^20 values (bf16 N(0,1), 1% of tokens x10; "
+                        "keys per token, values in blocks of 32), then one decode over them: 8 KV heads x "
+                        "131072 tokens, one bf16 query per head",
+            "bytes": "quantize: 2d in + the packed record out per vector; decode: the K and V records read",
+            "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "steps": steps, "rows": rows}
+
+
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e specification (DGX figure)
 
 
@@ -468,7 +533,7 @@ def run_ours(args):
     dist = Dist(args.gpus)
     torch.cuda.set_device(dist.local)
     if args.only:
-        fn = {"quantize": bench_quantize, "decode": bench_decode, "nsn": bench_nsn}[args.only]
+        fn = {"quantize": bench_quantize, "decode": bench_decode, "nsn": bench_nsn, "sweep": bench_sweep}[args.only]
         r = fn(args, dist)
         r.pop("sample_input", None)
         if dist.rank == 0:
@@ -481,6 +546,8 @@ def run_ours(args):
         extra["decode_attn"] = bench_decode(args, dist)
     if not args.no_nsn:
         extra["nsn_quantize"] = bench_nsn(args, dist)
+    if not args.no_sweep:
+        extra["sweep"] = bench_sweep(args, dist)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         cpu = cpu_baseline(q["sample_input"], args.cpu_vectors)

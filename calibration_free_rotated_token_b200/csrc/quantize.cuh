@@ -185,12 +185,27 @@ __device__ __forceinline__ void fwht(float2 (&v)[NP]) {
 // the magnitude |z| is compared with the positive decision levels
 // tau_j = t[H-1+j] (binary search, H = 2^(B-1)); mu = c[H + idx] is the
 // magnitude of the centroid.  g[p] = |z| - (level compared at search step p):
-// its sign bit is the complement of magnitude-index bit p.
+// its sign bit is the complement of magnitude-index bit p.  The levels and
+// magnitudes sit in registers (MagTab), so every step is a compare and a
+// register select: no branch and no indexed constant load.
 template <int B>
-__device__ __forceinline__ float mag_search(float az, const float* th, const float* cb, float (&g)[B > 1 ? B - 1 : 1]) {
-    constexpr int H = 1 << (B - 1);
-    const float* tau = th + (H - 1);  // tau[j], j >= 1
-    const float* mu = cb + H;
+struct MagTab {
+    static constexpr int H = 1 << (B - 1);
+    float tau[H];  // tau[0] unused
+    float mu[H];
+    __device__ __forceinline__ explicit MagTab(const QuantArgs& a) {
+#pragma unroll
+        for (int j = 0; j < H; ++j) {
+            tau[j] = j > 0 ? a.threshold[H - 1 + j] : 0.f;
+            mu[j] = a.centroid[H + j];
+        }
+    }
+};
+
+template <int B>
+__device__ __forceinline__ float mag_search(float az, const MagTab<B>& tb, float (&g)[B > 1 ? B - 1 : 1]) {
+    const float* tau = tb.tau;
+    const float* mu = tb.mu;
     if constexpr (B == 1) {
         g[0] = 0.f;
         return mu[0];
@@ -206,16 +221,22 @@ __device__ __forceinline__ float mag_search(float az, const float* th, const flo
         const bool m1 = g[1] >= 0.f;
         g[0] = az - (m1 ? tau[3] : tau[1]);
         const bool m0 = g[0] >= 0.f;
-        return m1 ? (m0 ? mu[3] : mu[2]) : (m0 ? mu[1] : mu[0]);
+        const float hi = m0 ? mu[3] : mu[2];
+        const float lo = m0 ? mu[1] : mu[0];
+        return m1 ? hi : lo;
     } else {
         g[2] = az - tau[4];
         const bool m2 = g[2] >= 0.f;
         g[1] = az - (m2 ? tau[6] : tau[2]);
         const bool m1 = g[1] >= 0.f;
-        g[0] = az - (m2 ? (m1 ? tau[7] : tau[5]) : (m1 ? tau[3] : tau[1]));
+        const float t_hi = m2 ? tau[7] : tau[3];
+        const float t_lo = m2 ? tau[5] : tau[1];
+        g[0] = az - (m1 ? t_hi : t_lo);
         const bool m0 = g[0] >= 0.f;
-        const float hi = m1 ? (m0 ? mu[7] : mu[6]) : (m0 ? mu[5] : mu[4]);
-        const float lo = m1 ? (m0 ? mu[3] : mu[2]) : (m0 ? mu[1] : mu[0]);
+        const float a3 = m0 ? mu[7] : mu[6], a2 = m0 ? mu[5] : mu[4];
+        const float a1 = m0 ? mu[3] : mu[2], a0 = m0 ? mu[1] : mu[0];
+        const float hi = m1 ? a3 : a2;
+        const float lo = m1 ? a1 : a0;
         return m2 ? hi : lo;
     }
 }
@@ -232,6 +253,7 @@ __device__ __forceinline__ float codes_and_residual(float2 (&v)[NV / 2], float i
     const float2 inv2 = make_float2(inv, inv);
     const float2 m1 = make_float2(-1.f, -1.f);
     float2 rr = make_float2(0.f, 0.f);
+    const MagTab<B> tab(a);
 #pragma unroll
     for (int w = 0; w < NV / 32; ++w) {
         // four independent chains of 8 coordinates (one byte each) per plane
@@ -249,8 +271,8 @@ __device__ __forceinline__ float codes_and_residual(float2 (&v)[NV / 2], float i
                 const int k = w * 16 + q * 4 + kk;  // pair index: coordinates 2k, 2k+1
                 const float2 z = __fmul2_rn(v[k], inv2);
                 float g1[NG], g0[NG];
-                const float mu1 = mag_search<B>(fabsf(z.y), a.threshold, a.centroid, g1);
-                const float mu0 = mag_search<B>(fabsf(z.x), a.threshold, a.centroid, g0);
+                const float mu1 = mag_search<B>(fabsf(z.y), tab, g1);
+                const float mu0 = mag_search<B>(fabsf(z.x), tab, g0);
                 wz[q] = push_sign(push_sign(wz[q], z.y), z.x);
                 if (B > 1) {
 #pragma unroll
