@@ -32,7 +32,7 @@ STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
 
 # Every symbol include/kvq.h declares.
 EXPORTED = (
-    "kvq_init", "kvq_destroy", "kvq_quantize", "kvq_nsn_quantize", "kvq_decode_workspace",
+    "kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize", "kvq_decode_workspace",
     "kvq_decode_attend", "kvq_decode_attend_noalloc", "kvq_status", "kvq_last_error", "kvq_get_constants",
     "kvq_get_info",
 )
@@ -50,6 +50,12 @@ class KvqError(RuntimeError):
 class KvqCache(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("qjl", ctypes.c_void_p), ("norms", ctypes.c_void_p),
                 ("capacity", ctypes.c_int64), ("layout", ctypes.c_int32)]
+
+
+class KvqQuantJob(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("n", ctypes.c_int64), ("ld", ctypes.c_int64),
+                ("layout", ctypes.c_int32), ("codes", ctypes.c_void_p), ("qjl", ctypes.c_void_p),
+                ("norms", ctypes.c_void_p)]
 
 
 _lib = None
@@ -71,6 +77,7 @@ def load() -> ctypes.CDLL:
         L.kvq_destroy.argtypes = [P]
         L.kvq_quantize.argtypes = [P, P, I, I64, I64, I, P, P, P, P]
         L.kvq_nsn_quantize.argtypes = [P, P, I, I64, I64, P, P, P, P]
+        L.kvq_quantize_batch.argtypes = [P, I, ctypes.POINTER(KvqQuantJob), P]
         L.kvq_decode_workspace.argtypes = [P, I, I, I, I64]
         L.kvq_decode_workspace.restype = SZ
         L.kvq_decode_attend.argtypes = [P, P, I, I, I, I, ctypes.POINTER(KvqCache), ctypes.POINTER(KvqCache), P,
@@ -81,7 +88,8 @@ def load() -> ctypes.CDLL:
         L.kvq_last_error.restype = ctypes.c_char_p
         L.kvq_get_constants.argtypes = [P, P, P, P, P]
         L.kvq_get_info.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(U32)]
-        for name in ("kvq_init", "kvq_destroy", "kvq_quantize", "kvq_nsn_quantize", "kvq_decode_attend",
+        for name in ("kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize",
+                     "kvq_decode_attend",
                      "kvq_decode_attend_noalloc", "kvq_status", "kvq_get_constants", "kvq_get_info"):
             getattr(L, name).restype = I
         _lib = L
@@ -204,6 +212,30 @@ def kvq_quantize(h: Handle, x: torch.Tensor, codes, qjl, norms, stream=None, lay
         _need(qjl, "qjl", numel=rows * h.m // 32)
     _check(load().kvq_quantize(h.ptr, _ptr(x2), _DTYPES[x.dtype], n, ld, layout, _ptr(codes),
                                _ptr(qjl) if h.qjl else None, _ptr(norms), _stream(stream)))
+
+
+def _job(h: Handle, x: torch.Tensor, codes, qjl, norms, layout: int) -> KvqQuantJob:
+    if x.dim() < 2 or x.shape[-1] != h.d:
+        raise ValueError(f"x must be [..., {h.d}]")
+    x2 = x.reshape(-1, h.d)
+    if x2.stride(-1) != 1:
+        raise ValueError("x rows must be contiguous")
+    n = x2.shape[0]
+    if x.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    rows = n if layout == KVQ_LAYOUT_TOKEN else 32 * ((n + 31) // 32)
+    _need(codes, "codes", numel=rows * h.b * h.d // 32)
+    _need(norms, "norms", dtype=torch.float16, numel=2 * n)
+    if h.qjl:
+        _need(qjl, "qjl", numel=rows * h.m // 32)
+    return KvqQuantJob(_ptr(x2), _DTYPES[x.dtype], n, x2.stride(0) if n > 1 else h.d, layout, _ptr(codes),
+                       _ptr(qjl) if h.qjl else None, _ptr(norms))
+
+
+def kvq_quantize_batch(h: Handle, jobs, stream=None):
+    """jobs: sequence of (x, codes, qjl, norms, layout) -- kvq_quantize of each, fused launches where possible."""
+    arr = (KvqQuantJob * max(len(jobs), 1))(*[_job(h, *j) for j in jobs])
+    _check(load().kvq_quantize_batch(h.ptr, len(jobs), arr, _stream(stream)))
 
 
 def kvq_nsn_quantize(h: Handle, x: torch.Tensor, codes, norms, block_mean, stream=None):

@@ -9,42 +9,43 @@
 #include <mutex>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "../../include/kvq.h"
 #include "kvq_internal.h"
 
 namespace kvq {
 // One per (d, b), from quantize_inst.cu.
-cudaError_t launch_quantize_d64_b1(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d64_b2(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d64_b3(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d64_b4(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d128_b1(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d128_b2(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d128_b3(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d128_b4(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d256_b1(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d256_b2(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d256_b3(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
-cudaError_t launch_quantize_d256_b4(bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                  const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d64_b1(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d64_b2(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d64_b3(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d64_b4(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d128_b1(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d128_b2(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d128_b3(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d128_b4(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d256_b1(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d256_b2(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d256_b3(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
+cudaError_t launch_quantize_d256_b4(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                  int dtype, const QuantArgs& a, int sms, cudaStream_t s);
 
 namespace {
-cudaError_t launch_quantize_any(int d, int b, bool qjl, bool nsn, const CUtensorMap& map, int dtype,
-                                const QuantArgs& a, int sms, cudaStream_t s) {
+cudaError_t launch_quantize_any(int d, int b, bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                int dtype, const QuantArgs& a, int sms, cudaStream_t s) {
 #define KVQ_CASE(D, B) \
-    if (d == D && b == B) return launch_quantize_d##D##_b##B(qjl, nsn, map, dtype, a, sms, s);
+    if (d == D && b == B) return launch_quantize_d##D##_b##B(qjl, nsn, map, map1, dtype, a, sms, s);
     KVQ_CASE(64, 1) KVQ_CASE(64, 2) KVQ_CASE(64, 3) KVQ_CASE(64, 4)
     KVQ_CASE(128, 1) KVQ_CASE(128, 2) KVQ_CASE(128, 3) KVQ_CASE(128, 4)
     KVQ_CASE(256, 1) KVQ_CASE(256, 2) KVQ_CASE(256, 3) KVQ_CASE(256, 4)
@@ -183,35 +184,60 @@ void fill_common(const kvq_ctx* h, float* cent, float* thr, uint32_t* ps) {
     std::memcpy(ps, h->pair_sign, sizeof(h->pair_sign));
 }
 
-int quantize_common(kvq_handle h, const void* x, int dtype, int64_t rows, int64_t ld, int layout, uint32_t* codes,
-                    uint32_t* qjl, uint16_t* norms, uint16_t* block_mean, bool nsn, void* stream) {
-    if (int e = check_handle(h)) return e;
-    if (dtype != KVQ_F32 && dtype != KVQ_F16 && dtype != KVQ_BF16) return fail(KVQ_EINVAL, "unknown dtype");
-    if (layout != KVQ_LAYOUT_TOKEN && layout != KVQ_LAYOUT_BLOCK32) return fail(KVQ_EINVAL, "unknown layout");
-    if (rows < 0) return fail(KVQ_EINVAL, "negative vector count");
-    if (rows == 0) return KVQ_OK;
-    if (rows > (int64_t(1) << 31) - 128) return fail(KVQ_EINVAL, "more than 2^31 - 128 vectors in one call");
-    const int esz = dtype == KVQ_F32 ? 4 : 2;
-    if (ld < h->d) return fail(KVQ_EINVAL, "row stride ld is smaller than d");
-    if ((ld * esz) % 16 != 0) return fail(KVQ_EINVAL, "row stride ld * element size must be a multiple of 16 bytes");
-    if (!x || !aligned(x, 16)) return fail(KVQ_EINVAL, "x must be a non-null 16-byte aligned device pointer");
-    if (!codes || !aligned(codes, 16)) return fail(KVQ_EINVAL, "codes must be non-null and 16-byte aligned");
-    if (!norms || !aligned(norms, 4)) return fail(KVQ_EINVAL, "norms must be non-null and 4-byte aligned");
+// One stream of vectors to quantize.
+struct QJob {
+    const void* x;
+    int dtype;
+    int64_t rows, ld;
+    int layout;
+    uint32_t* codes;
+    uint32_t* qjl;
+    uint16_t* norms;
+};
+
+// Argument checks of one stream; builds its tensor map when rows > 0.
+int check_job(kvq_handle h, const QJob& j, bool nsn, CUtensorMap* map) {
+    if (j.dtype != KVQ_F32 && j.dtype != KVQ_F16 && j.dtype != KVQ_BF16) return fail(KVQ_EINVAL, "unknown dtype");
+    if (j.layout != KVQ_LAYOUT_TOKEN && j.layout != KVQ_LAYOUT_BLOCK32) return fail(KVQ_EINVAL, "unknown layout");
+    if (j.rows < 0) return fail(KVQ_EINVAL, "negative vector count");
+    if (j.rows == 0) return KVQ_OK;
+    if (j.rows > (int64_t(1) << 31) - 128) return fail(KVQ_EINVAL, "more than 2^31 - 128 vectors in one call");
+    const int esz = j.dtype == KVQ_F32 ? 4 : 2;
+    if (j.ld < h->d) return fail(KVQ_EINVAL, "row stride ld is smaller than d");
+    if ((j.ld * esz) % 16 != 0) return fail(KVQ_EINVAL, "row stride ld * element size must be a multiple of 16 bytes");
+    if (!j.x || !aligned(j.x, 16)) return fail(KVQ_EINVAL, "x must be a non-null 16-byte aligned device pointer");
+    if (!j.codes || !aligned(j.codes, 16)) return fail(KVQ_EINVAL, "codes must be non-null and 16-byte aligned");
+    if (!j.norms || !aligned(j.norms, 4)) return fail(KVQ_EINVAL, "norms must be non-null and 4-byte aligned");
     const bool has_qjl = (h->flags & KVQ_QJL) != 0;
     if (!nsn) {
-        if (has_qjl && (!qjl || !aligned(qjl, 16))) return fail(KVQ_EINVAL, "qjl must be non-null and 16-byte aligned");
-        if (!has_qjl && qjl) return fail(KVQ_EINVAL, "qjl must be NULL for a handle without KVQ_QJL");
+        if (has_qjl && (!j.qjl || !aligned(j.qjl, 16)))
+            return fail(KVQ_EINVAL, "qjl must be non-null and 16-byte aligned");
+        if (!has_qjl && j.qjl) return fail(KVQ_EINVAL, "qjl must be NULL for a handle without KVQ_QJL");
     }
-    if (dtype == KVQ_F32 && h->d > 128) return fail(KVQ_EUNSUPPORTED, "fp32 input is built for d <= 128");
-    CUtensorMap map;
-    if (int e = make_row_map(&map, x, dtype, rows, h->d, ld)) return e;
+    if (j.dtype == KVQ_F32 && h->d > 128) return fail(KVQ_EUNSUPPORTED, "fp32 input is built for d <= 128");
+    return make_row_map(map, j.x, j.dtype, j.rows, h->d, j.ld);
+}
+
+// One launch over one stream (j1 == nullptr) or two streams of the same
+// dtype (the tensor-core kernel's tiles of j0, then those of j1).
+int launch_jobs(kvq_handle h, const QJob& j0, const CUtensorMap& m0, const QJob* j1, const CUtensorMap* m1,
+                uint16_t* block_mean, bool nsn, void* stream) {
     kvq::QuantArgs a{};
-    a.n = rows;
-    a.layout = layout;
-    a.ntiles = (rows + kvq::kTileRows - 1) / kvq::kTileRows;
-    a.codes = codes;
-    a.qjl = nsn ? nullptr : qjl;
-    a.norms = reinterpret_cast<__half2*>(norms);
+    a.n = j0.rows;
+    a.layout = j0.layout;
+    a.ntiles0 = (j0.rows + kvq::kTileRows - 1) / kvq::kTileRows;
+    a.ntiles = a.ntiles0;
+    a.codes = j0.codes;
+    a.qjl = nsn ? nullptr : j0.qjl;
+    a.norms = reinterpret_cast<__half2*>(j0.norms);
+    if (j1) {
+        a.n1 = j1->rows;
+        a.layout1 = j1->layout;
+        a.ntiles += (j1->rows + kvq::kTileRows - 1) / kvq::kTileRows;
+        a.codes1 = j1->codes;
+        a.qjl1 = j1->qjl;
+        a.norms1 = reinterpret_cast<__half2*>(j1->norms);
+    }
     a.block_mean = reinterpret_cast<__half*>(block_mean);
     a.S = h->d_S;
     a.status = h->d_status;
@@ -219,10 +245,22 @@ int quantize_common(kvq_handle h, const void* x, int dtype, int64_t rows, int64_
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, h->device);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t err = kvq::launch_quantize_any(h->d, h->b, has_qjl, nsn, map, dtype, a, sms, s);
+    const bool has_qjl = (h->flags & KVQ_QJL) != 0;
+    const cudaError_t err =
+        kvq::launch_quantize_any(h->d, h->b, has_qjl, nsn, m0, j1 ? *m1 : m0, j0.dtype, a, sms, s);
     if (err == cudaErrorNotSupported) return fail(KVQ_EUNSUPPORTED, "this (d, dtype, front end) is not built");
     if (err != cudaSuccess) return cuda_fail(err, "quantize launch");
     return KVQ_OK;
+}
+
+int quantize_common(kvq_handle h, const void* x, int dtype, int64_t rows, int64_t ld, int layout, uint32_t* codes,
+                    uint32_t* qjl, uint16_t* norms, uint16_t* block_mean, bool nsn, void* stream) {
+    if (int e = check_handle(h)) return e;
+    const QJob j{x, dtype, rows, ld, layout, codes, qjl, norms};
+    CUtensorMap map;
+    if (int e = check_job(h, j, nsn, &map)) return e;
+    if (rows == 0) return KVQ_OK;
+    return launch_jobs(h, j, map, nullptr, nullptr, block_mean, nsn, stream);
 }
 
 }  // namespace
@@ -308,6 +346,34 @@ int kvq_quantize(kvq_handle h, const void* x, int dtype, int64_t n, int64_t ld, 
                  uint32_t* qjl, uint16_t* norms, void* stream) {
     g_err.clear();
     return quantize_common(h, x, dtype, n, ld, layout, codes, qjl, norms, nullptr, false, stream);
+}
+
+int kvq_quantize_batch(kvq_handle h, int count, const kvq_quant_job* jobs, void* stream) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    if (count < 0 || (count > 0 && !jobs)) return fail(KVQ_EINVAL, "count must be >= 0 and jobs non-null");
+    std::vector<QJob> js;
+    std::vector<CUtensorMap> maps;
+    js.reserve(count);
+    maps.reserve(count);
+    for (int i = 0; i < count; ++i) {
+        const kvq_quant_job& u = jobs[i];
+        const QJob j{u.x, u.dtype, u.n, u.ld, u.layout, u.codes, u.qjl, u.norms};
+        CUtensorMap m;
+        if (int e = check_job(h, j, false, &m)) return fail(e, "job " + std::to_string(i) + ": " + g_err);
+        if (j.rows == 0) continue;
+        js.push_back(j);
+        maps.push_back(m);
+    }
+    for (size_t i = 0; i < js.size();) {
+        const bool pair = i + 1 < js.size() && js[i].dtype == js[i + 1].dtype &&
+                          kvq::quantize_pairs(h->d, js[i].dtype, false);
+        if (int e = launch_jobs(h, js[i], maps[i], pair ? &js[i + 1] : nullptr, pair ? &maps[i + 1] : nullptr,
+                                nullptr, false, stream))
+            return e;
+        i += pair ? 2 : 1;
+    }
+    return KVQ_OK;
 }
 
 int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, uint32_t* codes,

@@ -51,6 +51,15 @@ struct QuantArgs {
     float centroid[kMaxLevels];
     float threshold[kMaxLevels];
     uint32_t pair_sign[128];
+    // A second stream of vectors in the same launch (tensor-core kernel
+    // only): tiles [ntiles0, ntiles) read the second tensor map and write
+    // these outputs.  With one stream ntiles0 = ntiles.
+    int64_t ntiles0;
+    int64_t n1;
+    int layout1;
+    uint32_t* codes1;
+    uint32_t* qjl1;
+    __half2* norms1;
 };
 
 // Launch the quantizer (nsn = false) or the NSN front end + quantizer
@@ -58,6 +67,9 @@ struct QuantArgs {
 // box = 128 bytes x 128 rows).  Returns a cudaError_t.
 cudaError_t launch_quantize(const kvq_ctx* h, const CUtensorMap& map, int dtype, bool nsn, const QuantArgs& a,
                             cudaStream_t s, std::string* why);
+// True when two streams of vectors can share one launch (the tensor-core
+// kernel: 16-bit input, d <= 128, no NSN front end).
+inline bool quantize_pairs(int d, int dtype, bool nsn) { return d <= 128 && dtype != 0 && !nsn; }
 
 struct DecodeArgs {
     int batch, hq, hkv, G;            // G = hq / hkv

@@ -21,14 +21,15 @@ namespace kvq {
 namespace {
 
 template <int D, int B, bool QJL, bool NSN>
-cudaError_t by_dtype(const CUtensorMap& map, int dtype, const QuantArgs& a, int sms, cudaStream_t s) {
+cudaError_t by_dtype(const CUtensorMap& map, const CUtensorMap& map1, int dtype, const QuantArgs& a, int sms,
+                     cudaStream_t s) {
     if constexpr (NSN && (QJL || D > 128)) {
         return cudaErrorNotSupported;
     } else if constexpr (NSN) {
         switch (dtype) {
             case DT_F32: return launch_quantize_t<D, B, false, DT_F32, true>(map, a, sms, s);
-            case DT_F16: return launch_quantize_tc<D, B, false, DT_F16, true>(map, a, sms, s);
-            default: return launch_quantize_tc<D, B, false, DT_BF16, true>(map, a, sms, s);
+            case DT_F16: return launch_quantize_tc<D, B, false, DT_F16, true>(map, map1, a, sms, s);
+            default: return launch_quantize_tc<D, B, false, DT_BF16, true>(map, map1, a, sms, s);
         }
     } else {
         switch (dtype) {
@@ -36,10 +37,10 @@ cudaError_t by_dtype(const CUtensorMap& map, int dtype, const QuantArgs& a, int 
                 if constexpr (D <= 128) return launch_quantize_t<D, B, QJL, DT_F32, NSN>(map, a, sms, s);
                 else return cudaErrorNotSupported;
             case DT_F16:
-                if constexpr (D <= 128 && !NSN) return launch_quantize_tc<D, B, QJL, DT_F16>(map, a, sms, s);
+                if constexpr (D <= 128 && !NSN) return launch_quantize_tc<D, B, QJL, DT_F16>(map, map1, a, sms, s);
                 else return launch_quantize_t<D, B, QJL, DT_F16, NSN>(map, a, sms, s);
             default:
-                if constexpr (D <= 128 && !NSN) return launch_quantize_tc<D, B, QJL, DT_BF16>(map, a, sms, s);
+                if constexpr (D <= 128 && !NSN) return launch_quantize_tc<D, B, QJL, DT_BF16>(map, map1, a, sms, s);
                 else return launch_quantize_t<D, B, QJL, DT_BF16, NSN>(map, a, sms, s);
         }
     }
@@ -47,11 +48,14 @@ cudaError_t by_dtype(const CUtensorMap& map, int dtype, const QuantArgs& a, int 
 
 }  // namespace
 
-cudaError_t KVQ_LAUNCH_NAME(KVQ_D, KVQ_B)(bool qjl, bool nsn, const CUtensorMap& map, int dtype, const QuantArgs& a,
-                                           int sms, cudaStream_t s) {
-    if (nsn) return by_dtype<KVQ_D, KVQ_B, false, true>(map, dtype, a, sms, s);
-    return qjl ? by_dtype<KVQ_D, KVQ_B, true, false>(map, dtype, a, sms, s)
-               : by_dtype<KVQ_D, KVQ_B, false, false>(map, dtype, a, sms, s);
+// map1 describes the second stream of vectors (tiles [a.ntiles0, a.ntiles));
+// only the tensor-core kernel takes two streams (quantize_pairs).
+cudaError_t KVQ_LAUNCH_NAME(KVQ_D, KVQ_B)(bool qjl, bool nsn, const CUtensorMap& map, const CUtensorMap& map1,
+                                           int dtype, const QuantArgs& a, int sms, cudaStream_t s) {
+    if (a.ntiles0 != a.ntiles && !quantize_pairs(KVQ_D, dtype, nsn)) return cudaErrorNotSupported;
+    if (nsn) return by_dtype<KVQ_D, KVQ_B, false, true>(map, map1, dtype, a, sms, s);
+    return qjl ? by_dtype<KVQ_D, KVQ_B, true, false>(map, map1, dtype, a, sms, s)
+               : by_dtype<KVQ_D, KVQ_B, false, false>(map, map1, dtype, a, sms, s);
 }
 
 }  // namespace kvq

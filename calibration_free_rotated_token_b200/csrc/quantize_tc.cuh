@@ -105,7 +105,8 @@ __device__ __forceinline__ float stage_elem(const uint8_t* sp, int t, int j) {
 
 template <int D, int B, bool QJL, int DT, bool NSN = false>
 __global__ void __launch_bounds__(512, 1)
-    quantize_tc_kernel(const __grid_constant__ CUtensorMap map, const __grid_constant__ QuantArgs a) {
+    quantize_tc_kernel(const __grid_constant__ CUtensorMap map, const __grid_constant__ CUtensorMap map1,
+                       const __grid_constant__ QuantArgs a) {
     static_assert(!(NSN && QJL), "NSN front end: no QJL");
     using C = TcCfg<D, QJL, NSN>;
     constexpr int NS = C::kStages;
@@ -198,16 +199,19 @@ __global__ void __launch_bounds__(512, 1)
     auto issue_tile = [&](int64_t i) {
         const int64_t tile = blockIdx.x + i * G;
         if (tile >= a.ntiles) return;
+        const bool s1 = tile >= a.ntiles0;  // second stream of vectors
+        const int64_t lt = s1 ? tile - a.ntiles0 : tile;
         const int st = static_cast<int>(i % NS);
         iss[st] += 1;
         mbar_arrive_expect_tx(&full[st], C::kTileBytes);
 #pragma unroll
         for (int box = 0; box < C::kBoxes; ++box)
-            tma_load_2d(stage0 + st * C::kTileBytes + box * C::kBoxBytes, &map, &full[st], box * 64,
-                        static_cast<int>(tile * kTileRows));
+            tma_load_2d(stage0 + st * C::kTileBytes + box * C::kBoxBytes, s1 ? &map1 : &map, &full[st], box * 64,
+                        static_cast<int>(lt * kTileRows));
     };
     if (tid == 0) {
         prefetch_tmap(&map);
+        if (a.ntiles0 < a.ntiles) prefetch_tmap(&map1);
         for (int64_t i = 0; i < NS; ++i) issue_tile(i);
     }
     __syncthreads();
@@ -219,8 +223,16 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t hpar = 0, qpar = 0;
 
     for (int64_t i = wg;; i += C::kWG) {
-        const int64_t tile = blockIdx.x + i * G;
-        if (tile >= a.ntiles) break;
+        const int64_t tile_g = blockIdx.x + i * G;
+        if (tile_g >= a.ntiles) break;
+        // the tile's stream of vectors and its outputs
+        const bool s1 = tile_g >= a.ntiles0;
+        const int64_t tile = s1 ? tile_g - a.ntiles0 : tile_g;
+        const int64_t n_s = s1 ? a.n1 : a.n;
+        const int layout_s = s1 ? a.layout1 : a.layout;
+        uint32_t* const codes_s = s1 ? a.codes1 : a.codes;
+        uint32_t* const qjl_s = s1 ? a.qjl1 : a.qjl;
+        __half2* const norms_s = s1 ? a.norms1 : a.norms;
         const int st = static_cast<int>(i % NS);
         const bool ok = mbar_wait(&full[st], static_cast<uint32_t>((i / NS) & 1), a.status);
         if (named_bar_or(bar_id, 128, !ok)) break;
@@ -281,7 +293,7 @@ __global__ void __launch_bounds__(512, 1)
                     acc += (r & 1) ? pq.y : pq.x;
                 }
                 const __half o16 = __float2half_rn(acc * (1.0f / kTileRows));
-                if (tile * kTileRows < a.n) a.block_mean[tile * D + r] = o16;
+                if (tile * kTileRows < n_s) a.block_mean[tile * D + r] = o16;
                 const uint32_t ps = a.pair_sign[r >> 1];
                 const bool neg = ((ps >> ((r & 1) ? 31 : 15)) & 1u) != 0;
                 so[r] = neg ? -__half2float(o16) : __half2float(o16);
@@ -381,10 +393,10 @@ __global__ void __launch_bounds__(512, 1)
         }
         const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
         const int64_t vidx = tile * kTileRows + r;
-        const bool valid = vidx < a.n;
-        if (a.layout == 0) {
+        const bool valid = vidx < n_s;
+        if (layout_s == 0) {
             if (valid) {
-                uint32_t* cp = a.codes + vidx * (B * kWpp);
+                uint32_t* cp = codes_s + vidx * (B * kWpp);
 #pragma unroll
                 for (int p = 0; p < B; ++p) store_words<kWpp>(cp + p * kWpp, planes[p], zmask);
             }
@@ -393,11 +405,11 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t m = valid ? zmask : 0u;
 #pragma unroll
             for (int p = 0; p < B; ++p)
-                store_block32<kWpp>(a.codes + (blk * B + p) * D, planes[p], m, lane, blk * 32 < a.n);
+                store_block32<kWpp>(codes_s + (blk * B + p) * D, planes[p], m, lane, blk * 32 < n_s);
         }
         if (valid) {
             const float g = nrm > 0.f ? sqrtf(rr) : 0.f;
-            a.norms[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
+            norms_s[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
                                 : __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
         }
 
@@ -438,11 +450,11 @@ __global__ void __launch_bounds__(512, 1)
                 if (h + 1 < D / C::kQN) named_bar_sync(bar_id, 128);  // the next half reuses the columns
             }
             if (failed) break;
-            if (a.layout == 0) {
-                if (valid) store_words<kWpp>(a.qjl + vidx * kWpp, qw, zmask);
+            if (layout_s == 0) {
+                if (valid) store_words<kWpp>(qjl_s + vidx * kWpp, qw, zmask);
             } else {
                 const int64_t blk = tile * 4 + (warp & 3);
-                store_block32<kWpp>(a.qjl + blk * D, qw, valid ? zmask : 0u, lane, blk * 32 < a.n);
+                store_block32<kWpp>(qjl_s + blk * D, qw, valid ? zmask : 0u, lane, blk * 32 < n_s);
             }
         }
         // The next rotation MMA rewrites this warpgroup's columns; the barrier
@@ -463,7 +475,8 @@ __global__ void __launch_bounds__(512, 1)
 }
 
 template <int D, int B, bool QJL, int DT, bool NSN = false>
-cudaError_t launch_quantize_tc(const CUtensorMap& map, const QuantArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_quantize_tc(const CUtensorMap& map, const CUtensorMap& map1, const QuantArgs& a, int num_sms,
+                               cudaStream_t s) {
     using C = TcCfg<D, QJL, NSN>;
     auto kern = quantize_tc_kernel<D, B, QJL, DT, NSN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -482,7 +495,7 @@ cudaError_t launch_quantize_tc(const CUtensorMap& map, const QuantArgs& a, int n
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, map, a);
+    return cudaLaunchKernelEx(&cfg, kern, map, map1, a);
 }
 
 }  // namespace kvq

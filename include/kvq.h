@@ -134,6 +134,33 @@ int kvq_destroy(kvq_handle h);
 int kvq_quantize(kvq_handle h, const void* x, int dtype, int64_t n, int64_t ld, int layout, uint32_t* codes,
                  uint32_t* qjl, uint16_t* norms, void* stream);
 
+/* One stream of vectors for kvq_quantize_batch: the arguments of
+ * kvq_quantize, with the same meaning and rules. */
+typedef struct kvq_quant_job {
+    const void* x;
+    int dtype;
+    int64_t n;
+    int64_t ld;
+    int layout;
+    uint32_t* codes;
+    uint32_t* qjl;
+    uint16_t* norms;
+} kvq_quant_job;
+
+/*
+ * kvq_quantize_batch -- kvq_quantize of `count` streams of vectors (for
+ * instance the keys and the values of one layer) in as few launches as the
+ * kernels allow: two consecutive non-empty jobs of the same 16-bit dtype at
+ * d <= 128 share one launch, whose tiles are those of the first job then
+ * those of the second; the others take one launch each.  The outputs are
+ * exactly those of one kvq_quantize call per job.
+ *   count  >= 0; jobs  host array of `count` descriptors (read during the
+ *          call only).  Every job is checked before anything is launched;
+ *          an error names the job ("job i: ...") and launches nothing.
+ * Asynchronous on `stream`.  Errors: as kvq_quantize.
+ */
+int kvq_quantize_batch(kvq_handle h, int count, const kvq_quant_job* jobs, void* stream);
+
 /*
  * kvq_nsn_quantize -- NSN front end then the quantizer without QJL
  * (NSNQuant section 1 Normalize-Shift-Normalize, section 2 Hadamard, section

@@ -48,3 +48,10 @@ def test_invalid_arguments_are_rejected_on_host(lib):
     assert lib.kvq_init(ctypes.byref(h), 128, 2, 1, 8) == _abi.KVQ_EINVAL
     assert lib.kvq_init(None, 128, 2, 1, 1) == _abi.KVQ_EINVAL
     assert lib.kvq_destroy(None) == 0
+
+
+def test_quantize_batch_rejects_bad_arguments_on_host(lib):
+    lib.kvq_quantize_batch.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    lib.kvq_last_error.restype = ctypes.c_char_p
+    assert lib.kvq_quantize_batch(None, 0, None, None) == _abi.KVQ_EINVAL
+    assert b"null handle" in lib.kvq_last_error()

@@ -182,9 +182,14 @@ def test_llama_layer_full_size_sampled():
     k = constants(c["d"], c["b"], c["handle_seed"])
     rng = np.random.default_rng(0)
     with kvq.Handle(c["d"], c["b"], c["handle_seed"], qjl=True) as h:
+        # K and V of the layer in one fused launch, as the benchmark times them
+        outs = [kvq.alloc_packed(h, K.numel() // c["d"], layout=lay) for lay in (0, 1)]
+        kvq.kvq_quantize_batch(h, [(K, *outs[0], 0), (V, *outs[1], 1)])
+        code, bits = kvq.kvq_status(h)
+        assert code == 0, (code, bits)
         for X, layout in ((K, 0), (V, 1)):
             X2 = X.reshape(-1, c["d"])
-            codes, qjl, norms = run_quantize(h, X2, layout=layout)
+            codes, qjl, norms = outs[layout]
             if layout == 0:
                 idx = np.sort(rng.choice(X2.shape[0], 2048, replace=False))
                 ti = torch.from_numpy(idx).cuda()
@@ -213,3 +218,66 @@ def test_sweep_full_size_sampled(d, b, qjl):
     ti = torch.from_numpy(idx).cuda()
     compare_quantize(k, x[ti].double().cpu().numpy(), to_np_u32(codes[ti]), to_np_u32(qj[ti]) if qjl else None,
                      to_np_f16bits(norms[ti]), qjl)
+
+
+BATCH_CASES = [
+    # d, b, qjl, (dtype, n, layout) of the first and of the second job
+    (128, 2, True, (torch.bfloat16, 1000, 0), (torch.bfloat16, 300, 1)),  # one fused launch, ragged tails
+    (64, 1, False, (torch.float16, 129, 1), (torch.float16, 2000, 0)),    # fused, block-32 first
+    (128, 4, True, (torch.bfloat16, 31, 0), (torch.bfloat16, 33, 1)),     # fused, both under one tile
+    (128, 3, True, (torch.bfloat16, 515, 0), (torch.float16, 257, 1)),    # dtypes differ: two launches
+    (256, 2, True, (torch.bfloat16, 300, 0), (torch.bfloat16, 300, 1)),   # d = 256: two launches
+    (128, 2, False, (torch.float32, 100, 0), (torch.float32, 70, 1)),     # fp32: two launches
+]
+
+
+@pytest.mark.parametrize("d,b,qjl,j0,j1", BATCH_CASES)
+def test_quantize_batch_matches_oracle_and_single_calls(d, b, qjl, j0, j1):
+    xs = [wl.sweep_tokens(n, d, seed=300 + d + b + i, dtype=dt) for i, (dt, n, _) in enumerate((j0, j1))]
+    xs[0][min(2, j0[1] - 1)] = 0
+    k = constants(d, b, 8)
+    with kvq.Handle(d, b, 8, qjl=qjl) as h:
+        outs = [kvq.alloc_packed(h, x.shape[0], layout=j[2]) for x, j in zip(xs, (j0, j1))]
+        kvq.kvq_quantize_batch(h, [(x.cuda(), *o, j[2]) for x, o, j in zip(xs, outs, (j0, j1))])
+        code, bits = kvq.kvq_status(h)
+        assert code == 0, (code, bits)
+        for x, (codes, qj, norms), j in zip(xs, outs, (j0, j1)):
+            compare_quantize(k, x.double().numpy(), to_np_u32(codes), to_np_u32(qj) if qjl else None,
+                             to_np_f16bits(norms), qjl, layout=j[2])
+            # bit for bit what one kvq_quantize call per job writes
+            c1, q1, n1 = run_quantize(h, x.cuda(), layout=j[2])
+            assert torch.equal(c1, codes) and torch.equal(n1, norms)
+            if qjl:
+                assert torch.equal(q1, qj)
+
+
+def test_quantize_batch_empty_jobs_and_three_streams():
+    d, b = 128, 2
+    xs = [wl.sweep_tokens(n, d, seed=400 + n, dtype=torch.bfloat16) for n in (200, 0, 130, 64)]
+    with kvq.Handle(d, b, 8, qjl=True) as h:
+        lays = (0, 1, 1, 0)
+        outs = [kvq.alloc_packed(h, max(x.shape[0], 1), layout=l) for x, l in zip(xs, lays)]
+        kvq.kvq_quantize_batch(h, [(x.cuda(), *o, l) for x, o, l in zip(xs, outs, lays)])
+        kvq.kvq_quantize_batch(h, [])
+        assert kvq.kvq_status(h)[0] == 0
+        for x, o, l in zip(xs, outs, lays):
+            if x.shape[0] == 0:
+                continue
+            c1, q1, n1 = run_quantize(h, x.cuda(), layout=l)
+            assert torch.equal(c1, o[0]) and torch.equal(q1, o[1]) and torch.equal(n1, o[2])
+
+
+def test_quantize_batch_checks_every_job_before_launching():
+    with kvq.Handle(128, 2, 1, qjl=True) as h:
+        x = torch.randn(64, 128, device="cuda", dtype=torch.bfloat16)
+        good = kvq.alloc_packed(h, 64)
+        bad = kvq.alloc_packed(h, 64)
+        good[0].fill_(7)
+        jobs = (kvq.KvqQuantJob * 2)(kvq._job(h, x, *good, 0), kvq._job(h, x, *bad, 0))
+        jobs[1].qjl = None  # a QJL handle needs the sign buffer
+        code = kvq.load().kvq_quantize_batch(h.ptr, 2, jobs, None)
+        assert code == kvq.KVQ_EINVAL
+        assert kvq.load().kvq_last_error().decode().startswith("job 1")
+        torch.cuda.synchronize()
+        assert (good[0] == 7).all()  # nothing was launched
+        assert kvq.load().kvq_quantize_batch(h.ptr, -1, None, None) == kvq.KVQ_EINVAL
