@@ -26,6 +26,7 @@ KVQ_ENOMEM = -4
 KVQ_ENONFINITE = -5
 KVQ_ETIMEOUT = -6
 KVQ_QJL = 1
+KVQ_BETA_CODEBOOK = 2
 KVQ_F32, KVQ_F16, KVQ_BF16 = 0, 1, 2
 KVQ_LAYOUT_TOKEN, KVQ_LAYOUT_BLOCK32 = 0, 1
 STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
@@ -34,7 +35,7 @@ STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
 EXPORTED = (
     "kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize", "kvq_decode_workspace",
     "kvq_decode_attend", "kvq_decode_attend_noalloc", "kvq_status", "kvq_last_error", "kvq_get_constants",
-    "kvq_get_info",
+    "kvq_get_info", "kvq_codebook",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -88,9 +89,11 @@ def load() -> ctypes.CDLL:
         L.kvq_last_error.restype = ctypes.c_char_p
         L.kvq_get_constants.argtypes = [P, P, P, P, P]
         L.kvq_get_info.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(U32)]
+        L.kvq_codebook.argtypes = [I, I, U32, P, P]
         for name in ("kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize",
                      "kvq_decode_attend",
-                     "kvq_decode_attend_noalloc", "kvq_status", "kvq_get_constants", "kvq_get_info"):
+                     "kvq_decode_attend_noalloc", "kvq_status", "kvq_get_constants", "kvq_get_info",
+                     "kvq_codebook"):
             getattr(L, name).restype = I
         _lib = L
         return L
@@ -127,10 +130,11 @@ def _need(t, name, dtype=None, numel=None, device=True):
 class Handle:
     """Owns a kvq_handle; ``d``, ``b``, ``m``, ``qjl`` mirror kvq_get_info."""
 
-    def __init__(self, d: int, b: int, seed: int, qjl: bool = True):
+    def __init__(self, d: int, b: int, seed: int, qjl: bool = True, beta: bool = False):
         L = load()
         h = ctypes.c_void_p()
-        _check(L.kvq_init(ctypes.byref(h), d, b, seed & (2**64 - 1), KVQ_QJL if qjl else 0))
+        flags = (KVQ_QJL if qjl else 0) | (KVQ_BETA_CODEBOOK if beta else 0)
+        _check(L.kvq_init(ctypes.byref(h), d, b, seed & (2**64 - 1), flags))
         self._h = h
         dd, bb, mm, ff = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_uint32()
         _check(L.kvq_get_info(h, ctypes.byref(dd), ctypes.byref(bb), ctypes.byref(mm), ctypes.byref(ff)))
@@ -212,6 +216,15 @@ def kvq_quantize(h: Handle, x: torch.Tensor, codes, qjl, norms, stream=None, lay
         _need(qjl, "qjl", numel=rows * h.m // 32)
     _check(load().kvq_quantize(h.ptr, _ptr(x2), _DTYPES[x.dtype], n, ld, layout, _ptr(codes),
                                _ptr(qjl) if h.qjl else None, _ptr(norms), _stream(stream)))
+
+
+def kvq_codebook(d: int, b: int, beta: bool = False):
+    """(centroids, thresholds) as fp32 numpy arrays, computed by the library on the host."""
+    import numpy as np
+    c = np.zeros(1 << b, np.float32)
+    t = np.zeros(max((1 << b) - 1, 1), np.float32)
+    _check(load().kvq_codebook(d, b, KVQ_BETA_CODEBOOK if beta else 0, c.ctypes.data, t.ctypes.data))
+    return c, t[: (1 << b) - 1]
 
 
 def _job(h: Handle, x: torch.Tensor, codes, qjl, norms, layout: int) -> KvqQuantJob:

@@ -131,6 +131,65 @@ void lloyd_max_codebook(int b, std::vector<double>* cent, std::vector<double>* t
     for (int k = 1; k < L; ++k) thr->push_back(0.5 * (c[k - 1] + c[k]));
 }
 
+// Codebook for the exact law of one coordinate of a rotated unit vector,
+// scaled by sqrt(d) (TurboQuant blog, "Estágio 1": Beta((d-1)/2, (d-1)/2) on
+// [-1, 1], Lloyd-Max over it).  Density of z: f(z) ~ (1 - z^2/d)^a on
+// |z| < sqrt(d), a = (d-3)/2.  Cell moments in closed form:
+//   int_0^t f  ~ sqrt(d) I_n(asin(t/sqrt(d))),  I_n(th) = int_0^th cos^n,
+//                n = d - 2, by I_n = cos^(n-1) sin / n + (n-1)/n I_(n-2);
+//   int z f    ~ -d/(d-1) (1 - t^2/d)^((d-1)/2)  (antiderivative).
+// The common normalisation cancels in every centroid (a ratio of the two).
+double sphere_m0(int d, double t) {
+    const double r = std::sqrt(static_cast<double>(d));
+    const double x = std::fmin(std::fabs(t) / r, 1.0);
+    const double th = std::asin(x), sn = std::sin(th), cs = std::cos(th);
+    const int n = d - 2;
+    double I = (n % 2 == 0) ? th : sn;  // I_0 or I_1
+    double cp = (n % 2 == 0) ? cs : cs * cs;  // cos^(k-1) for the first step k = 2 or 3
+    for (int k = (n % 2 == 0) ? 2 : 3; k <= n; k += 2) {
+        I = cp * sn / k + (k - 1.0) / k * I;
+        cp *= cs * cs;
+    }
+    return std::copysign(r * I, t);
+}
+double sphere_f1(int d, double t) {
+    const double w = std::fmax(1.0 - t * t / d, 0.0);
+    return -static_cast<double>(d) / (d - 1) * std::pow(w, 0.5 * (d - 1));
+}
+
+void lloyd_max_sphere_codebook(int d, int b, std::vector<double>* cent, std::vector<double>* thr) {
+    const int L = 1 << b;
+    const double edge = std::sqrt(static_cast<double>(d));
+    std::vector<double> c, t0;
+    lloyd_max_codebook(b, &c, &t0);  // starting point: the Gaussian codebook, inside the support
+    double mx = 0.0;
+    for (double v : c) mx = std::fmax(mx, std::fabs(v));
+    if (mx > 0.9 * edge)
+        for (double& v : c) v *= 0.9 * edge / mx;
+    std::vector<double> t(L + 1);
+    for (int iter = 0; iter < 1000000; ++iter) {
+        t[0] = -edge;
+        t[L] = edge;
+        for (int k = 1; k < L; ++k) t[k] = 0.5 * (c[k - 1] + c[k]);
+        double change = 0.0;
+        for (int k = 0; k < L; ++k) {
+            const double m0 = sphere_m0(d, t[k + 1]) - sphere_m0(d, t[k]);
+            const double nc = (sphere_f1(d, t[k + 1]) - sphere_f1(d, t[k])) / m0;
+            change = std::fmax(change, std::fabs(nc - c[k]));
+            c[k] = nc;
+        }
+        if (change <= 1e-15) break;
+    }
+    for (int k = 0; k < L / 2; ++k) {
+        const double m = 0.5 * (c[L - 1 - k] - c[k]);
+        c[k] = -m;
+        c[L - 1 - k] = m;
+    }
+    cent->assign(c.begin(), c.end());
+    thr->clear();
+    for (int k = 1; k < L; ++k) thr->push_back(0.5 * (c[k - 1] + c[k]));
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -275,7 +334,7 @@ int kvq_init(kvq_handle* out, int d, int b, uint64_t seed, uint32_t flags) {
     *out = nullptr;
     if (d != 64 && d != 128 && d != 256) return fail(KVQ_EINVAL, "d must be 64, 128 or 256");
     if (b < 1 || b > 4) return fail(KVQ_EINVAL, "b must be in 1..4");
-    if (flags & ~KVQ_QJL) return fail(KVQ_EINVAL, "unknown flag bits");
+    if (flags & ~(KVQ_QJL | KVQ_BETA_CODEBOOK)) return fail(KVQ_EINVAL, "unknown flag bits");
     kvq_ctx* h = new (std::nothrow) kvq_ctx();
     if (!h) return fail(KVQ_ENOMEM, "host allocation failed");
     cudaGetDevice(&h->device);
@@ -294,7 +353,8 @@ int kvq_init(kvq_handle* out, int d, int b, uint64_t seed, uint32_t flags) {
         std::memcpy(&h->S_half[k], &v, 2);
     }
     std::vector<double> c, t;
-    lloyd_max_codebook(b, &c, &t);
+    if (flags & KVQ_BETA_CODEBOOK) lloyd_max_sphere_codebook(d, b, &c, &t);
+    else lloyd_max_codebook(b, &c, &t);
     h->centroids.assign(c.begin(), c.end());
     h->thresholds.assign(t.begin(), t.end());
     cudaError_t e = cudaMalloc(&h->d_S, h->S_half.size() * sizeof(__half));
@@ -310,6 +370,20 @@ int kvq_init(kvq_handle* out, int d, int b, uint64_t seed, uint32_t flags) {
                                               : cuda_fail(e, "kvq_init");
     }
     *out = h;
+    return KVQ_OK;
+}
+
+int kvq_codebook(int d, int b, uint32_t flags, float* centroids, float* thresholds) {
+    g_err.clear();
+    if (d != 64 && d != 128 && d != 256) return fail(KVQ_EINVAL, "d must be 64, 128 or 256");
+    if (b < 1 || b > 4) return fail(KVQ_EINVAL, "b must be in 1..4");
+    if (flags & ~(KVQ_QJL | KVQ_BETA_CODEBOOK)) return fail(KVQ_EINVAL, "unknown flag bits");
+    if (!centroids || !thresholds) return fail(KVQ_EINVAL, "centroids and thresholds must be non-null");
+    std::vector<double> c, t;
+    if (flags & KVQ_BETA_CODEBOOK) lloyd_max_sphere_codebook(d, b, &c, &t);
+    else lloyd_max_codebook(b, &c, &t);
+    for (size_t k = 0; k < c.size(); ++k) centroids[k] = static_cast<float>(c[k]);
+    for (size_t k = 0; k < t.size(); ++k) thresholds[k] = static_cast<float>(t[k]);
     return KVQ_OK;
 }
 

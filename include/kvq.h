@@ -75,6 +75,10 @@ extern "C" {
 
 /* ---- flags of kvq_init ------------------------------------------------- */
 #define KVQ_QJL 1u            /* store the 1-bit QJL residual sketch (m = d rows) */
+/* Codebook: Lloyd-Max for the exact law of one coordinate of a rotated unit
+ * vector scaled by sqrt(d) (Beta((d-1)/2, (d-1)/2) on [-1, 1], stretched to
+ * [-sqrt(d), sqrt(d)]; TurboQuant blog, "Estágio 1") instead of N(0, 1). */
+#define KVQ_BETA_CODEBOOK 2u
 
 /* ---- element types of inputs ------------------------------------------ */
 #define KVQ_F32 0
@@ -101,11 +105,20 @@ typedef struct kvq_ctx* kvq_handle;
  *   b      Lloyd-Max bits per coordinate, 1..4.
  *   seed   seeds the SplitMix64 streams: Rademacher signs use `seed`, the
  *          Gaussian projection S (d x d, rounded to fp16) uses `seed + 1`.
- *   flags  KVQ_QJL or 0.
+ *   flags  KVQ_QJL and/or KVQ_BETA_CODEBOOK, or 0.
  * Synchronous.  Allocates device memory for the constants and a status
  * word.  Errors: KVQ_EINVAL, KVQ_ENOMEM, KVQ_ECUDA.
  */
 int kvq_init(kvq_handle* h, int d, int b, uint64_t seed, uint32_t flags);
+
+/*
+ * kvq_codebook -- the codebook a handle with (d, b, flags) uses, computed on
+ * the host (no device needed): 2^b ascending centroids and the 2^b - 1
+ * decision levels between them (the midpoints), rounded to fp32.
+ *   centroids   host, 2^b floats;  thresholds  host, 2^b - 1 floats.
+ * Errors: KVQ_EINVAL (d, b, flags as kvq_init; null outputs).
+ */
+int kvq_codebook(int d, int b, uint32_t flags, float* centroids, float* thresholds);
 
 /* kvq_destroy -- free the handle and its device constants (synchronous).
  * A NULL handle is accepted and ignored. */

@@ -146,6 +146,65 @@ def lloyd_max(b: int, max_iter: int = 1_000_000, tol: float = 1e-15):
     return c, t[: L - 1], mse.value, it
 
 
+def sphere_coordinate_pdf(z, d: int):
+    """Density of z = sqrt(d) u_1, u uniform on the unit sphere of R^d (d >= 3).
+
+    TurboQuant blog, "Estágio 1": after the random rotation each coordinate of
+    the unit vector follows Beta((d-1)/2, (d-1)/2) stretched to [-1, 1], i.e.
+    f_u(u) = (1 - u^2)^((d-3)/2) / B(1/2, (d-1)/2); the quantizer works on
+    z = sqrt(d) u (unit variance), so f(z) = f_u(z / sqrt(d)) / sqrt(d) on
+    |z| < sqrt(d)."""
+    from math import lgamma
+    z = np.asarray(z, np.float64)
+    a = (d - 3) / 2.0
+    log_beta = lgamma(0.5) + lgamma((d - 1) / 2.0) - lgamma(d / 2.0)
+    w = np.clip(1.0 - z * z / d, 0.0, None)
+    return np.where(np.abs(z) < np.sqrt(d), w ** a, 0.0) / (np.exp(log_beta) * np.sqrt(d))
+
+
+_GL = {}
+
+
+def _cell_moments(d: int, lo: float, hi: float, nodes: int = 768):
+    """int f, int z f, int z^2 f over [lo, hi] by Gauss-Legendre quadrature."""
+    if nodes not in _GL:
+        _GL[nodes] = np.polynomial.legendre.leggauss(nodes)
+    x, w = _GL[nodes]
+    z = 0.5 * (hi - lo) * x + 0.5 * (hi + lo)
+    fw = 0.5 * (hi - lo) * w * sphere_coordinate_pdf(z, d)
+    return fw.sum(), (fw * z).sum(), (fw * z * z).sum()
+
+
+def lloyd_max_sphere(d: int, b: int, max_iter: int = 100_000, tol: float = 1e-14):
+    """Lloyd-Max codebook for one coordinate of a rotated unit vector scaled by
+    sqrt(d) (the d-exact law above instead of N(0, 1)): (centroids, thresholds,
+    mse, steps).  Lloyd's two conditions, in the order the method states them:
+    decision levels at the midpoints of adjacent centroids, each centroid the
+    mean of its cell; iterated from the Gaussian codebook to a fixed point."""
+    L = 1 << b
+    edge = float(np.sqrt(d))
+    c = lloyd_max(b)[0].copy()
+    c *= min(1.0, 0.9 * edge / np.max(np.abs(c)))  # start inside the support, cells non-empty
+    it = 0
+    for it in range(1, max_iter + 1):
+        t = np.concatenate(([-edge], 0.5 * (c[:-1] + c[1:]), [edge]))
+        cn = np.empty(L)
+        for k in range(L):
+            p, m1, _ = _cell_moments(d, t[k], t[k + 1])
+            cn[k] = m1 / p
+        move = np.max(np.abs(cn - c))
+        c = cn
+        if move <= tol:
+            break
+    c = 0.5 * (c - c[::-1])  # the law is symmetric, so is the codebook
+    t = np.concatenate(([-edge], 0.5 * (c[:-1] + c[1:]), [edge]))
+    mse = 0.0
+    for k in range(L):
+        p, m1, m2 = _cell_moments(d, t[k], t[k + 1])
+        mse += m2 - 2.0 * c[k] * m1 + c[k] * c[k] * p
+    return c, t[1:-1].copy(), mse, it
+
+
 @dataclass
 class Constants:
     """Everything the method fixes for one (d, b, seed): signs, S, codebook.
@@ -170,11 +229,18 @@ class Constants:
         return self.d
 
 
-def make_constants(d: int, b: int, seed: int) -> Constants:
+def make_constants(d: int, b: int, seed: int, codebook: str = "gaussian") -> Constants:
+    """codebook: "gaussian" (Lloyd-Max for N(0, 1)) or "beta" (for the exact
+    coordinate law of a rotated unit vector, lloyd_max_sphere)."""
     delta = rademacher_signs(d, seed)
     s_half, _ = gaussian_fp16(d, d, seed + 1)
     S = half_bits_to_double_fast(s_half)
-    c, t, mse, _ = lloyd_max(b)
+    if codebook == "gaussian":
+        c, t, mse, _ = lloyd_max(b)
+    elif codebook == "beta":
+        c, t, mse, _ = lloyd_max_sphere(d, b)
+    else:
+        raise ValueError(f"unknown codebook {codebook!r}")
     return Constants(d, b, seed, delta, s_half, S, c, t, mse)
 
 

@@ -55,3 +55,24 @@ def test_quantize_batch_rejects_bad_arguments_on_host(lib):
     lib.kvq_last_error.restype = ctypes.c_char_p
     assert lib.kvq_quantize_batch(None, 0, None, None) == _abi.KVQ_EINVAL
     assert b"null handle" in lib.kvq_last_error()
+
+
+
+@pytest.mark.parametrize("beta", [False, True])
+def test_library_codebook_matches_oracle_on_host(lib, beta):
+    """The library's codebook (computed on the host, no device) against the
+    oracle's: two independent computations, equal to fp32 rounding."""
+    import numpy as np
+
+    import oracle
+    for d in (64, 128, 256):
+        for b in (1, 2, 3, 4):
+            c, t = _abi.kvq_codebook(d, b, beta)
+            co, to, _, _ = oracle.lloyd_max_sphere(d, b) if beta else oracle.lloyd_max(b)
+            np.testing.assert_allclose(c, co, rtol=2.0 ** -23, atol=1e-12)
+            np.testing.assert_allclose(t, to, rtol=2.0 ** -23, atol=1e-12)
+    import ctypes as C
+    buf = (C.c_float * 16)()
+    assert lib.kvq_codebook(96, 2, 0, buf, buf) == _abi.KVQ_EINVAL
+    assert lib.kvq_codebook(128, 2, 8, buf, buf) == _abi.KVQ_EINVAL
+    assert lib.kvq_codebook(128, 2, 0, None, buf) == _abi.KVQ_EINVAL

@@ -17,10 +17,10 @@ pytestmark = pytest.mark.gpu
 _consts = {}
 
 
-def constants(d, b, seed):
-    if (d, b, seed) not in _consts:
-        _consts[(d, b, seed)] = oracle.make_constants(d, b, seed)
-    return _consts[(d, b, seed)]
+def constants(d, b, seed, codebook="gaussian"):
+    if (d, b, seed, codebook) not in _consts:
+        _consts[(d, b, seed, codebook)] = oracle.make_constants(d, b, seed, codebook)
+    return _consts[(d, b, seed, codebook)]
 
 
 def upload_streams(h, caches, capacity, layout):
@@ -55,8 +55,8 @@ def run_decode(h, q, hkv, kc, vc, seq_len, max_T, scale, want_logits=True):
     return out.cpu().numpy(), (logits.cpu().numpy() if want_logits else None)
 
 
-def check_case(d, b, qjl, batch, hq, hkv, seq_len, capacity, scale, qdtype=torch.bfloat16, seed=3):
-    k = constants(d, b, seed)
+def check_case(d, b, qjl, batch, hq, hkv, seq_len, capacity, scale, qdtype=torch.bfloat16, seed=3, beta=False):
+    k = constants(d, b, seed, "beta" if beta else "gaussian")
     G = hq // hkv
     max_T = max(seq_len)
     kcs, vcs, kst, vst = [], [], [], []
@@ -70,7 +70,7 @@ def check_case(d, b, qjl, batch, hq, hkv, seq_len, capacity, scale, qdtype=torch
             c, q, n, st = oracle_cache(k, V, qjl, layout=1)
             vcs.append((c, q, n)); vst.append(st)
     qv = wl.queries(batch, hq, d, seed=77, dtype=qdtype)
-    with kvq.Handle(d, b, seed, qjl=qjl) as h:
+    with kvq.Handle(d, b, seed, qjl=qjl, beta=beta) as h:
         kc, kt = upload_streams(h, kcs, capacity, 0)
         vc, vt = upload_streams(h, vcs, capacity, 1)
         out, logits = run_decode(h, qv.cuda(), hkv, kc, vc, seq_len, max_T, scale)
@@ -117,6 +117,16 @@ def test_tiny_reference_workload():
 ])
 def test_decode_matches_oracle(d, b, qjl, batch, hq, hkv, seq_len, cap, qdt):
     check_case(d, b, qjl, batch, hq, hkv, seq_len, cap, scale=1 / np.sqrt(d), qdtype=qdt)
+
+
+@pytest.mark.parametrize("d,b,qjl,batch,hq,hkv,seq_len,cap", [
+    (128, 2, True, 2, 8, 2, [1000, 300], 1024),   # tensor-core path
+    (64, 1, False, 1, 4, 4, [700], 704),          # tensor-core path, GQA 1:1
+    (128, 3, True, 1, 4, 1, [513], 544),          # 3-bit path
+    (256, 4, False, 1, 2, 1, [129], 160),
+])
+def test_decode_beta_codebook_matches_oracle(d, b, qjl, batch, hq, hkv, seq_len, cap):
+    check_case(d, b, qjl, batch, hq, hkv, seq_len, cap, scale=1 / np.sqrt(d), beta=True)
 
 
 def test_long_context_split_merge():

@@ -281,3 +281,24 @@ def test_quantize_batch_checks_every_job_before_launching():
         torch.cuda.synchronize()
         assert (good[0] == 7).all()  # nothing was launched
         assert kvq.load().kvq_quantize_batch(h.ptr, -1, None, None) == kvq.KVQ_EINVAL
+
+
+
+@pytest.mark.parametrize("d,b,qjl,dtype,n", [
+    (128, 2, True, torch.bfloat16, 1000),
+    (64, 3, False, torch.float16, 300),
+    (256, 4, True, torch.bfloat16, 257),
+    (128, 1, False, torch.float32, 200),
+    (128, 4, True, torch.bfloat16, 515),
+])
+def test_quantize_beta_codebook_matches_oracle(d, b, qjl, dtype, n):
+    """KVQ_BETA_CODEBOOK: the kernels are unchanged, the codebook is the d-exact one."""
+    x = wl.sweep_tokens(n, d, seed=500 + d + b, dtype=dtype)
+    k = oracle.make_constants(d, b, 5, codebook="beta")
+    with kvq.Handle(d, b, 5, qjl=qjl, beta=True) as h:
+        _, _, cent, thr = kvq.kvq_get_constants(h)
+        np.testing.assert_allclose(cent.numpy(), k.centroids, rtol=2.0 ** -23, atol=1e-12)
+        np.testing.assert_allclose(thr.numpy(), k.thresholds, rtol=2.0 ** -23, atol=1e-12)
+        codes, qj, norms = run_quantize(h, x.cuda())
+    compare_quantize(k, x.double().numpy(), to_np_u32(codes), to_np_u32(qj) if qjl else None,
+                     to_np_f16bits(norms), qjl)

@@ -69,3 +69,77 @@ def test_fixed_point_by_quadrature(b):
         D += integrate.quad(lambda x: (x - c[k]) ** 2 * stats.norm.pdf(x), a, e, epsabs=1e-14,
                             epsrel=1e-13)[0]
     assert abs(D - mse) < 1e-10
+
+
+
+# ---------------------------------------------------------------------------
+# d-exact codebook: Lloyd-Max for one coordinate of a rotated unit vector,
+# z = sqrt(d) u_1 with (u_1 + 1)/2 ~ Beta((d-1)/2, (d-1)/2).
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_sphere_codebook_d3_is_the_uniform_quantizer(b):
+    """d = 3: u_1 is uniform on [-1, 1] (Archimedes), so z is uniform on
+    [-sqrt(3), sqrt(3)] and Lloyd-Max is the uniform quantizer with MSE
+    (cell width)^2 / 12 = 1 / L^2."""
+    L = 1 << b
+    c, t, mse, _ = oracle.lloyd_max_sphere(3, b)
+    r = np.sqrt(3.0)
+    np.testing.assert_allclose(c, r * (-1 + (2 * np.arange(L) + 1) / L), atol=1e-10)
+    np.testing.assert_allclose(t, r * (-1 + 2 * np.arange(1, L) / L), atol=1e-10)
+    assert abs(mse - 1.0 / L ** 2) < 1e-10
+
+
+@pytest.mark.parametrize("d", [5, 64, 128, 256])
+def test_sphere_codebook_one_bit_closed_form(d):
+    """1 bit: the centroids are +-E|z| = sqrt(d) Gamma(d/2) / (sqrt(pi) Gamma((d+1)/2))
+    and the MSE is E[z^2] - E|z|^2 = 1 - E|z|^2."""
+    from math import exp, lgamma, pi, sqrt
+    e = sqrt(d) * exp(lgamma(d / 2) - lgamma((d + 1) / 2)) / sqrt(pi)
+    c, t, mse, _ = oracle.lloyd_max_sphere(d, 1)
+    np.testing.assert_allclose(c, [-e, e], rtol=1e-12)  # quadrature: ~1e-13 at d = 256
+    assert t[0] == 0.0
+    assert abs(mse - (1 - e * e)) < 1e-12
+
+
+@pytest.mark.parametrize("d,b", [(64, 2), (128, 3), (256, 4), (64, 4)])
+def test_sphere_codebook_against_scipy_beta(d, b):
+    """Cell masses against scipy's Beta CDF and each centroid against the
+    conditional mean integrated from scipy's Beta density (both independent of
+    the oracle's density and quadrature); E[z^2] = MSE + sum_k P_k c_k^2 = 1."""
+    a = (d - 1) / 2.0
+    r = np.sqrt(d)
+    law = stats.beta(a, a, loc=-r, scale=2 * r)  # z = sqrt(d) (2 B - 1)
+    c, t, mse, _ = oracle.lloyd_max_sphere(d, b)
+    edges = np.concatenate(([-r], t, [r]))
+    P = np.diff(law.cdf(edges))
+    assert abs(P.sum() - 1) < 1e-12
+    for k in range(len(c)):
+        lo, hi = edges[k], edges[k + 1]
+        m1, _ = integrate.quad(lambda z: z * law.pdf(z), lo, hi, epsabs=1e-14, epsrel=1e-12, limit=200)
+        assert abs(m1 / P[k] - c[k]) < 1e-9 * max(1.0, abs(c[k]))
+    assert abs(mse + float(np.sum(P * c * c)) - 1.0) < 1e-11
+
+
+def test_sphere_codebook_tends_to_the_gaussian_one():
+    """u_1 sqrt(d) -> N(0, 1): the d-exact codebook approaches the Gaussian
+    Lloyd-Max codebook, with an O(1/d) gap (4x smaller for 4x larger d)."""
+    cg = oracle.lloyd_max(3)[0]
+    gaps = [np.max(np.abs(oracle.lloyd_max_sphere(d, 3)[0] - cg)) for d in (512, 2048)]
+    assert gaps[0] < 6e-3
+    assert 3.0 < gaps[0] / gaps[1] < 5.0
+
+
+def test_sphere_codebook_mse_on_random_unit_vectors():
+    """Coordinates of uniformly random unit vectors (scaled by sqrt(d)): the
+    d-exact codebook's empirical MSE matches its analytic MSE and is below the
+    Gaussian codebook's on the same coordinates (it is optimal for that law)."""
+    d, b, n = 64, 3, 40000
+    rng = np.random.default_rng(11)
+    g = rng.standard_normal((n, d))
+    z = np.sqrt(d) * g / np.linalg.norm(g, axis=1, keepdims=True)
+    cs, ts, mse_s, _ = oracle.lloyd_max_sphere(d, b)
+    cg, tg, _, _ = oracle.lloyd_max(b)
+    err_s = np.mean((z - cs[np.searchsorted(ts, z, side="right")]) ** 2)
+    err_g = np.mean((z - cg[np.searchsorted(tg, z, side="right")]) ** 2)
+    assert abs(err_s - mse_s) < 4e-4  # ~ 6 standard errors over n * d = 2.56e6 coordinates
+    assert err_s < err_g
