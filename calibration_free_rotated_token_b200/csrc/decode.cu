@@ -87,10 +87,26 @@ __global__ void __launch_bounds__(kDecThreads) qproj_kernel(const __grid_constan
     fwht_smem<D>(sq);
     for (int j = threadIdx.x; j < D; j += blockDim.x) a.qrot[bh * D + j] = sq[j];
     if (QJL) {
+        // row i of S by 16-byte loads, eight in flight at a time
         for (int i = threadIdx.x; i < D; i += blockDim.x) {
-            const __half* Si = a.S + static_cast<int64_t>(i) * D;
+            const uint4* Si = reinterpret_cast<const uint4*>(a.S + static_cast<int64_t>(i) * D);
             float acc = 0.f;
-            for (int j = 0; j < D; ++j) acc = fmaf(__half2float(Si[j]), sq[j], acc);
+#pragma unroll
+            for (int j0 = 0; j0 < D / 8; j0 += 8) {
+                uint4 w[8];
+#pragma unroll
+                for (int u = 0; u < 8 && j0 + u < D / 8; ++u) w[u] = Si[j0 + u];
+#pragma unroll
+                for (int u = 0; u < 8 && j0 + u < D / 8; ++u) {
+                    const __half2* hw = reinterpret_cast<const __half2*>(&w[u]);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 sv = __half22float2(hw[k]);
+                        const int j = 8 * (j0 + u) + 2 * k;
+                        acc = fmaf(sv.y, sq[j + 1], fmaf(sv.x, sq[j], acc));
+                    }
+                }
+            }
             a.qproj[bh * D + i] = acc;
         }
     }

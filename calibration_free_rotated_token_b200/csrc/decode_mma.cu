@@ -179,12 +179,32 @@ __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__
         __syncthreads();
     }
     if (QJL) {
-        for (int e = tid; e < G * M; e += kThreads) {
-            const int h = e / M, i = e % M;
-            const __half* Si = a.S + static_cast<int64_t>(i) * D;
-            float acc = 0.f;
-            for (int j = 0; j < D; ++j) acc = fmaf(__half2float(Si[j]), sq[h][j], acc);
-            sp[h][i] = acc;
+        // p = S q' for every head of the group: thread i reads row i of S
+        // once (16-byte loads, all in flight together) and feeds all G heads.
+        for (int i = tid; i < M; i += kThreads) {
+            const uint4* Si = reinterpret_cast<const uint4*>(a.S + static_cast<int64_t>(i) * D);
+            float acc[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll
+            for (int j0 = 0; j0 < D / 8; j0 += 8) {
+                uint4 w[8];
+#pragma unroll
+                for (int u = 0; u < 8 && j0 + u < D / 8; ++u) w[u] = Si[j0 + u];
+#pragma unroll
+                for (int u = 0; u < 8 && j0 + u < D / 8; ++u) {
+                    const __half2* hw = reinterpret_cast<const __half2*>(&w[u]);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 sv = __half22float2(hw[k]);
+                        const int j = 8 * (j0 + u) + 2 * k;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) acc[h] = fmaf(sv.y, sq[h][j + 1], fmaf(sv.x, sq[h][j], acc[h]));
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) sp[h][i] = acc[h];
         }
         __syncthreads();
     }
