@@ -333,46 +333,76 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const __gri
     constexpr int PART = 2 + D + M;
     __shared__ float sA[D], sB[M];
     __shared__ float sf[512];
-    __shared__ float sL, sM;
+    __shared__ float sred[kDecThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t bh = blockIdx.x;
-    const float* pp = a.part + bh * a.nsplit * PART;
-    if (threadIdx.x == 0) {
-        float mx = -INFINITY;
-        for (int s = 0; s < a.nsplit; ++s)
-            if (pp[s * PART + 1] > 0.f) mx = fmaxf(mx, pp[s * PART]);
-        float L = 0.f;
-        for (int s = 0; s < a.nsplit; ++s) {
-            const float f = (pp[s * PART + 1] > 0.f) ? __expf(pp[s * PART] - mx) : 0.f;
-            sf[s] = f;
-            L += f * pp[s * PART + 1];
+    const int ns = a.nsplit;
+    const float* pp = a.part + bh * ns * PART;
+    // block-wide max (op 0) or sum (op 1) of one value per thread
+    auto block_reduce = [&](float v, int op) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float w = __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            v = op == 0 ? fmaxf(v, w) : v + w;
         }
-        sL = L;
-        sM = mx;
-    }
-    __syncthreads();
-    const float L = sL;
+        __syncthreads();  // sred is free (an earlier reduction has been read)
+        if (lane == 0) sred[wid] = v;
+        __syncthreads();
+        float r = sred[0];
+        for (int k = 1; k < kDecThreads / 32; ++k) r = op == 0 ? fmaxf(r, sred[k]) : r + sred[k];
+        return r;
+    };
+    // running max over the splits that saw tokens, then L = sum_s e^(M_s - max) L_s
+    float mx = -INFINITY;
+    for (int s = tid; s < ns; s += blockDim.x)
+        if (pp[s * PART + 1] > 0.f) mx = fmaxf(mx, pp[s * PART]);
+    mx = block_reduce(mx, 0);
+    float lp = 0.f;
+    for (int s = tid; s < ns; s += blockDim.x)
+        if (pp[s * PART + 1] > 0.f) lp += __expf(pp[s * PART] - mx) * pp[s * PART + 1];
+    const float L = block_reduce(lp, 1);
     if (!(L > 0.f)) {
-        for (int j = threadIdx.x; j < D; j += blockDim.x) a.out[bh * D + j] = 0.f;
+        for (int j = tid; j < D; j += blockDim.x) a.out[bh * D + j] = 0.f;
         return;
     }
-    for (int e = threadIdx.x; e < D + (QJL ? M : 0); e += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < a.nsplit; ++s) acc = fmaf(sf[s], pp[s * PART + 2 + e], acc);
-        if (e < D) sA[e] = acc;
-        else sB[e - D] = acc;
+    // weighted sums of A and B over the splits, 512 split factors at a time
+    constexpr int NE = (D + (QJL ? M : 0) + kDecThreads - 1) / kDecThreads;
+    float acc[NE];
+#pragma unroll
+    for (int k = 0; k < NE; ++k) acc[k] = 0.f;
+    for (int c0 = 0; c0 < ns; c0 += 512) {
+        const int nc = min(512, ns - c0);
+        for (int s = tid; s < nc; s += blockDim.x) {
+            const float* ps = pp + static_cast<int64_t>(c0 + s) * PART;
+            sf[s] = ps[1] > 0.f ? __expf(ps[0] - mx) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < NE; ++k) {
+            const int e = tid + k * kDecThreads;
+            if (e < D + (QJL ? M : 0))
+                for (int s = 0; s < nc; ++s) acc[k] = fmaf(sf[s], pp[static_cast<int64_t>(c0 + s) * PART + 2 + e], acc[k]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int k = 0; k < NE; ++k) {
+        const int e = tid + k * kDecThreads;
+        if (e < D) sA[e] = acc[k];
+        else if (e < D + (QJL ? M : 0)) sB[e - D] = acc[k];
     }
     __syncthreads();
     // v = A + sqrt(pi/2)/m S^T B, in place in sA
     float vj[(D + kDecThreads - 1) / kDecThreads];
     int k = 0;
     for (int j = threadIdx.x; j < D; j += blockDim.x, ++k) {
-        float acc = sA[j];
+        float v = sA[j];
         if (QJL) {
             float st = 0.f;
             for (int i = 0; i < M; ++i) st = fmaf(__half2float(a.S[static_cast<int64_t>(i) * D + j]), sB[i], st);
-            acc = fmaf(kSqrtHalfPi / M, st, acc);
+            v = fmaf(kSqrtHalfPi / M, st, v);
         }
-        vj[k] = acc;
+        vj[k] = v;
     }
     __syncthreads();
     k = 0;
