@@ -364,6 +364,39 @@ def nsn_quantize(k: Constants, x, mean_in=None) -> dict:
     return dict(codes=codes, norm_x=nx, norm_w=nw, mean_half=mean_half, mean_f64=mean_f64, z=z)
 
 
+def nsn_dequantize(k: Constants, codes, norm_x, norm_w, mean_half) -> np.ndarray:
+    """Vectors stored by the NSN front end, reconstructed from its byproducts
+    (NSNQuant section 1: x = s1 (s2 v + o) with s1 = ||x||/sqrt(d), s2 v = w):
+    x_hat = ||x||/sqrt(d) (w_hat + o_blk), w_hat the plain dequantization of the
+    codes with norm ||w|| (no QJL), o_blk the fp16 mean of the vector's block of
+    128 tokens.  codes [n, d]; norm_x, norm_w [n]; mean_half [ceil(n/128), d] fp16 bits."""
+    codes = _c(codes, np.int32)
+    n, d = codes.shape
+    w = dequantize(k, codes, None, norm_w, np.zeros(n), use_qjl=False)
+    o = half_bits_to_double(np.asarray(mean_half, np.uint16).reshape(-1, d))
+    o = np.repeat(o, NSN_BLOCK, axis=0)[:n]
+    return (np.asarray(norm_x, np.float64) / np.sqrt(d))[:, None] * (w + o)
+
+
+def nsn_decode_attend(k: Constants, q, kcache: dict, vcache: dict, kmean, vmean, scale: float,
+                      want_logits: bool = True):
+    """Attention of G queries ([G, d]) over NSN-stored keys and values of one
+    KV head (NSNQuant section 4: attention from the byproducts).  Each cache is
+    a dict with ``codes`` [T, d], ``norm_x`` and ``norm_w`` [T] (the stored
+    fp16-widened values); kmean / vmean are the fp16 block means [ceil(T/128), d].
+    Softmax in fp64 over the reconstructed vectors (nsn_dequantize)."""
+    q = _c(np.atleast_2d(q), np.float64)
+    Kh = nsn_dequantize(k, kcache["codes"], kcache["norm_x"], kcache["norm_w"], kmean)
+    Vh = nsn_dequantize(k, vcache["codes"], vcache["norm_x"], vcache["norm_w"], vmean)
+    G, d = q.shape
+    if Kh.shape[0] == 0:
+        return (np.zeros((G, 0)) if want_logits else None), np.zeros((G, d))
+    logits = scale * (q @ Kh.T)
+    e = np.exp(logits - logits.max(axis=1, keepdims=True))
+    out = (e @ Vh) / e.sum(axis=1, keepdims=True)
+    return (logits if want_logits else None), out
+
+
 # ----------------------------------------------------------------------------
 # Packed cache layout (see module docstring)
 # ----------------------------------------------------------------------------
