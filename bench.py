@@ -397,13 +397,56 @@ def bench_nsn(args, dist):
     bytes_per_vec = 2 * d + h.b * d // 8 + 4 + 2 * d / 128
     gbs = H * T * bytes_per_vec / (ms / steps / 1e3) / 1e9
     hbm, src = peaks()
+    del xs, codes, norms, means
+
+    # ---- decode attention over NSN caches: 4 sequences of this workload (keys per token,
+    # values in blocks of 32), 32 query heads on the 8 KV heads, one bf16 query token ----
+    NB, hq = 4, 4 * H
+    kc = torch.empty((NB * H, T, h.b, d // 32), dtype=torch.int32, device="cuda")
+    vc = torch.empty((NB * H, T // 32, h.b, d), dtype=torch.int32, device="cuda")
+    kn = torch.empty((NB * H, T, 2), dtype=torch.float16, device="cuda")
+    vn = torch.empty_like(kn)
+    km = torch.empty((NB * H, T // 128, d), dtype=torch.float16, device="cuda")
+    vm = torch.empty_like(km)
+    for bi in range(NB):
+        sl = slice(bi * H, (bi + 1) * H)
+        X = wl.nsn_tokens(H, T, d, c["seed"] + 100 + 2 * bi + 1000 * dist.rank, device="cuda")
+        kvq.kvq_nsn_quantize(h, X, kc[sl], kn[sl], km[sl], stream=stream)
+        X = wl.nsn_tokens(H, T, d, c["seed"] + 101 + 2 * bi + 1000 * dist.rank, device="cuda")
+        kvq.kvq_nsn_quantize(h, X, vc[sl], vn[sl], vm[sl], stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
+        del X
+    q = wl.queries(NB, hq, d, c["seed"] + 7, device="cuda", std=d ** -0.5)
+    out = torch.empty((NB, hq, d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(kvq.kvq_decode_workspace(h, NB, hq, H, T), dtype=torch.uint8, device="cuda")
+    seq = torch.full((NB,), T, dtype=torch.int32, device="cuda")
+    kcache = kvq.make_cache(kc, None, kn, T, kvq.KVQ_LAYOUT_TOKEN)
+    vcache = kvq.make_cache(vc, None, vn, T, kvq.KVQ_LAYOUT_BLOCK32)
+
+    def dstep(i):
+        kvq.kvq_nsn_decode_attend(h, q, H, kcache, vcache, km, vm, seq, T, 1.0, out, ws, stream=stream)
+
+    for i in range(3):
+        dstep(i)
+    code, bits = kvq.kvq_status(h)
+    if code != 0:
+        raise RuntimeError(f"nsn decode status {code} bits {bits}")
+    dsteps = max(5, steps // 2)
+    ms_d = timed(dist, dstep, dsteps, stream)
+    cache_bytes = NB * H * T * 2 * (h.b * d // 8 + 4 + 2 * d / 128)
+    dgbs = cache_bytes / (ms_d / dsteps / 1e3) / 1e9
     h.close()
     return {"metric": "NSN quantize tokens/s", "value": dist.world * T * steps / (ms / 1e3), "unit": "tokens/s",
             "ms_per_step": ms / steps, "workload": "8 heads x 65536 tokens x d128 bf16, b=2, no QJL",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "frac_of_spec_8tbs": round(gbs / SPEC_HBM_GBS, 4),
                          "traffic": traffic_record("nsn_quantize"),
-                         "peak_source": f"{src} hbm_gbs (copy)"}}
+                         "peak_source": f"{src} hbm_gbs (copy)"},
+            "decode": {"metric": "NSN packed-cache decode-attn GB/s", "value": round(dist.world * dgbs, 1),
+                       "unit": "GB/s", "frac_of_hbm": round(dgbs / hbm, 4), "ms_per_step": ms_d / dsteps,
+                       "steps": dsteps, "cache_bytes_per_step": int(cache_bytes),
+                       "workload": "4 sequences x 8 KV heads x 65536 tokens of the NSN workload (b=2, keys per "
+                                   "token, values in blocks of 32, fp16 block means), 32 query heads, one bf16 "
+                                   "query token, kvq_nsn_decode_attend"}}
 
 
 def bench_sweep(args, dist):

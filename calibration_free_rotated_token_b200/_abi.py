@@ -35,7 +35,7 @@ STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
 EXPORTED = (
     "kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize", "kvq_decode_workspace",
     "kvq_decode_attend", "kvq_decode_attend_noalloc", "kvq_status", "kvq_last_error", "kvq_get_constants",
-    "kvq_get_info", "kvq_codebook",
+    "kvq_get_info", "kvq_codebook", "kvq_nsn_decode_attend",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -77,7 +77,7 @@ def load() -> ctypes.CDLL:
         L.kvq_init.argtypes = [ctypes.POINTER(P), I, I, U64, U32]
         L.kvq_destroy.argtypes = [P]
         L.kvq_quantize.argtypes = [P, P, I, I64, I64, I, P, P, P, P]
-        L.kvq_nsn_quantize.argtypes = [P, P, I, I64, I64, P, P, P, P]
+        L.kvq_nsn_quantize.argtypes = [P, P, I, I64, I64, I, P, P, P, P]
         L.kvq_quantize_batch.argtypes = [P, I, ctypes.POINTER(KvqQuantJob), P]
         L.kvq_decode_workspace.argtypes = [P, I, I, I, I64]
         L.kvq_decode_workspace.restype = SZ
@@ -90,10 +90,12 @@ def load() -> ctypes.CDLL:
         L.kvq_get_constants.argtypes = [P, P, P, P, P]
         L.kvq_get_info.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(U32)]
         L.kvq_codebook.argtypes = [I, I, U32, P, P]
+        L.kvq_nsn_decode_attend.argtypes = [P, P, I, I, I, I, ctypes.POINTER(KvqCache), ctypes.POINTER(KvqCache),
+                                            P, P, P, I64, ctypes.c_float, P, P, P, SZ, P]
         for name in ("kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize",
                      "kvq_decode_attend",
                      "kvq_decode_attend_noalloc", "kvq_status", "kvq_get_constants", "kvq_get_info",
-                     "kvq_codebook"):
+                     "kvq_codebook", "kvq_nsn_decode_attend"):
             getattr(L, name).restype = I
         _lib = L
         return L
@@ -251,8 +253,9 @@ def kvq_quantize_batch(h: Handle, jobs, stream=None):
     _check(load().kvq_quantize_batch(h.ptr, len(jobs), arr, _stream(stream)))
 
 
-def kvq_nsn_quantize(h: Handle, x: torch.Tensor, codes, norms, block_mean, stream=None):
-    """x: [n_heads, n_tok, d] contiguous, n_tok % 128 == 0."""
+def kvq_nsn_quantize(h: Handle, x: torch.Tensor, codes, norms, block_mean, stream=None,
+                     layout: int = KVQ_LAYOUT_TOKEN):
+    """x: [n_heads, n_tok, d] contiguous, n_tok % 128 == 0; layout token (keys) or block-32 (values)."""
     if x.dim() != 3 or x.shape[-1] != h.d:
         raise ValueError(f"x must be [heads, tokens, {h.d}]")
     _need(x, "x")
@@ -260,7 +263,7 @@ def kvq_nsn_quantize(h: Handle, x: torch.Tensor, codes, norms, block_mean, strea
     _need(codes, "codes", numel=H * T * h.b * h.d // 32)
     _need(norms, "norms", dtype=torch.float16, numel=2 * H * T)
     _need(block_mean, "block_mean", dtype=torch.float16, numel=H * (T // 128) * h.d)
-    _check(load().kvq_nsn_quantize(h.ptr, _ptr(x), _DTYPES[x.dtype], H, T, _ptr(codes), _ptr(norms),
+    _check(load().kvq_nsn_quantize(h.ptr, _ptr(x), _DTYPES[x.dtype], H, T, layout, _ptr(codes), _ptr(norms),
                                    _ptr(block_mean), _stream(stream)))
 
 
@@ -291,6 +294,29 @@ def kvq_decode_attend(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vc
     _check(load().kvq_decode_attend(h.ptr, _ptr(q), _DTYPES[q.dtype], B, hq, hkv, ctypes.byref(kcache),
                                     ctypes.byref(vcache), _ptr(seq_len), max_T, float(scale), _ptr(logits),
                                     _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def kvq_nsn_decode_attend(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vcache: KvqCache,
+                          k_block_mean: torch.Tensor, v_block_mean: torch.Tensor, seq_len: torch.Tensor,
+                          max_T: int, scale: float, out: torch.Tensor, workspace: torch.Tensor,
+                          logits: torch.Tensor | None = None, stream=None):
+    """kvq_decode_attend over caches from kvq_nsn_quantize; block means fp16 [streams, capacity/128, d]."""
+    if q.dim() != 3 or q.shape[-1] != h.d:
+        raise ValueError(f"q must be [batch, hq, {h.d}]")
+    _need(q, "q")
+    B, hq, _ = q.shape
+    _need(seq_len, "seq_len", dtype=torch.int32, numel=B)
+    _need(out, "out", dtype=torch.float32, numel=B * hq * h.d)
+    _need(workspace, "workspace")
+    _need(k_block_mean, "k_block_mean", dtype=torch.float16)
+    _need(v_block_mean, "v_block_mean", dtype=torch.float16)
+    if logits is not None:
+        _need(logits, "logits", dtype=torch.float32, numel=B * hq * max_T)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().kvq_nsn_decode_attend(h.ptr, _ptr(q), _DTYPES[q.dtype], B, hq, hkv, ctypes.byref(kcache),
+                                        ctypes.byref(vcache), _ptr(k_block_mean), _ptr(v_block_mean),
+                                        _ptr(seq_len), max_T, float(scale), _ptr(logits), _ptr(out),
+                                        _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def kvq_decode_attend_noalloc(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vcache: KvqCache,

@@ -450,8 +450,8 @@ int kvq_quantize_batch(kvq_handle h, int count, const kvq_quant_job* jobs, void*
     return KVQ_OK;
 }
 
-int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, uint32_t* codes,
-                     uint16_t* norms, uint16_t* block_mean, void* stream) {
+int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, int layout,
+                     uint32_t* codes, uint16_t* norms, uint16_t* block_mean, void* stream) {
     g_err.clear();
     if (int e = check_handle(h)) return e;
     if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "the NSN front end takes a handle without KVQ_QJL");
@@ -460,8 +460,8 @@ int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, in
     if (h->d > 128) return fail(KVQ_EUNSUPPORTED, "the NSN front end is built for d <= 128");
     if (n_heads * n_tok == 0) return KVQ_OK;
     if (!block_mean || !aligned(block_mean, 2)) return fail(KVQ_EINVAL, "block_mean must be non-null");
-    return quantize_common(h, x, dtype, n_heads * n_tok, h->d, KVQ_LAYOUT_TOKEN, codes, nullptr, norms, block_mean,
-                           true, stream);
+    return quantize_common(h, x, dtype, n_heads * n_tok, h->d, layout, codes, nullptr, norms, block_mean, true,
+                           stream);
 }
 
 size_t kvq_decode_workspace(kvq_handle h, int batch, int hq, int hkv, int64_t max_T) {
@@ -512,8 +512,12 @@ int decode_check(kvq_handle h, int dtype, int batch, int hq, int hkv, const kvq_
 
 int decode_launch(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
                   const kvq_cache* v, const int32_t* seq_len, int64_t max_T, float scale, float* logits,
-                  float* out, void* workspace, int ns, int64_t chunk, void* stream) {
+                  float* out, void* workspace, int ns, int64_t chunk, void* stream, const uint16_t* kmean = nullptr,
+                  const uint16_t* vmean = nullptr) {
     kvq::DecodeArgs a{};
+    a.nsn = kmean != nullptr;
+    a.kmean = reinterpret_cast<const __half*>(kmean);
+    a.vmean = reinterpret_cast<const __half*>(vmean);
     a.batch = batch;
     a.hq = hq;
     a.hkv = hkv;
@@ -578,6 +582,29 @@ int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq,
     if (ws_bytes < need) return fail(KVQ_EINVAL, "workspace too small: need " + std::to_string(need) + " bytes");
     return decode_launch(h, q, dtype, batch, hq, hkv, k, v, seq_len, max_T, scale, logits, out, workspace, ns, chunk,
                          stream);
+}
+
+int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
+                          const kvq_cache* v, const uint16_t* k_block_mean, const uint16_t* v_block_mean,
+                          const int32_t* seq_len, int64_t max_T, float scale, float* logits, float* out,
+                          void* workspace, size_t ws_bytes, void* stream) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
+    if (h->b > 2) return fail(KVQ_EUNSUPPORTED, "decode over NSN caches is built for b <= 2");
+    int ns = 0;
+    int64_t chunk = 0;
+    size_t need = 0;
+    if (int e = decode_check(h, dtype, batch, hq, hkv, k, v, q, seq_len, max_T, scale, out, &ns, &chunk, &need))
+        return e;
+    if (k->capacity % 128 != 0 || v->capacity % 128 != 0)
+        return fail(KVQ_EINVAL, "NSN cache capacities must be multiples of 128 (one block mean per 128 tokens)");
+    if (!k_block_mean || !v_block_mean || !aligned(k_block_mean, 16) || !aligned(v_block_mean, 16))
+        return fail(KVQ_EINVAL, "block means must be non-null and 16-byte aligned");
+    if (!workspace || !aligned(workspace, 16)) return fail(KVQ_EINVAL, "workspace must be non-null and 16-byte aligned");
+    if (ws_bytes < need) return fail(KVQ_EINVAL, "workspace too small: need " + std::to_string(need) + " bytes");
+    return decode_launch(h, q, dtype, batch, hq, hkv, k, v, seq_len, max_T, scale, logits, out, workspace, ns, chunk,
+                         stream, k_block_mean, v_block_mean);
 }
 
 int kvq_decode_attend_noalloc(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv,

@@ -326,8 +326,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     }
 }
 
-// Merge the splits of one (batch, query head) and rotate back.
-template <int D, bool QJL>
+// Merge the splits of one (batch, query head) and rotate back.  NSN: the
+// second vector of each partial is the block-mean term O (no QJL), added
+// after the inverse rotation: out = delta .* H A / (d L) + O / L.
+template <int D, bool QJL, bool NSN = false>
 __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int M = D;
     constexpr int PART = 2 + D + M;
@@ -366,7 +368,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const __gri
         return;
     }
     // weighted sums of A and B over the splits, 512 split factors at a time
-    constexpr int NE = (D + (QJL ? M : 0) + kDecThreads - 1) / kDecThreads;
+    constexpr int EXTRA = (QJL || NSN) ? M : 0;  // entries of the second vector
+    constexpr int NE = (D + EXTRA + kDecThreads - 1) / kDecThreads;
     float acc[NE];
 #pragma unroll
     for (int k = 0; k < NE; ++k) acc[k] = 0.f;
@@ -380,7 +383,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const __gri
 #pragma unroll
         for (int k = 0; k < NE; ++k) {
             const int e = tid + k * kDecThreads;
-            if (e < D + (QJL ? M : 0))
+            if (e < D + EXTRA)
                 for (int s = 0; s < nc; ++s) acc[k] = fmaf(sf[s], pp[static_cast<int64_t>(c0 + s) * PART + 2 + e], acc[k]);
         }
         __syncthreads();
@@ -389,7 +392,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const __gri
     for (int k = 0; k < NE; ++k) {
         const int e = tid + k * kDecThreads;
         if (e < D) sA[e] = acc[k];
-        else if (e < D + (QJL ? M : 0)) sB[e - D] = acc[k];
+        else if (e < D + EXTRA) sB[e - D] = acc[k];
     }
     __syncthreads();
     // v = A + sqrt(pi/2)/m S^T B, in place in sA
@@ -410,7 +413,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const __gri
     __syncthreads();
     fwht_smem<D>(sA);
     const float inv = 1.0f / (static_cast<float>(D) * L);
-    for (int j = threadIdx.x; j < D; j += blockDim.x) a.out[bh * D + j] = sign_of(a.pair_sign, j) * sA[j] * inv;
+    for (int j = threadIdx.x; j < D; j += blockDim.x)
+        a.out[bh * D + j] = sign_of(a.pair_sign, j) * sA[j] * inv + (NSN ? sB[j] / L : 0.f);
 }
 
 template <int D, int B, bool QJL>
@@ -498,13 +502,23 @@ cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s,
     if (decode_uses_mma(h)) {
         cudaError_t e = launch_decode_mma(h, a, s);
         if (e != cudaSuccess) return e;
+        const unsigned nbh = static_cast<unsigned>(a.batch * a.hq);
         switch (h->d) {
-            case 64: qjl ? decode_combine_kernel<64, true><<<a.batch * a.hq, kDecThreads, 0, s>>>(a)
-                         : decode_combine_kernel<64, false><<<a.batch * a.hq, kDecThreads, 0, s>>>(a); break;
-            case 128: qjl ? decode_combine_kernel<128, true><<<a.batch * a.hq, kDecThreads, 0, s>>>(a)
-                          : decode_combine_kernel<128, false><<<a.batch * a.hq, kDecThreads, 0, s>>>(a); break;
-            default: qjl ? decode_combine_kernel<256, true><<<a.batch * a.hq, kDecThreads, 0, s>>>(a)
-                         : decode_combine_kernel<256, false><<<a.batch * a.hq, kDecThreads, 0, s>>>(a); break;
+            case 64:
+                if (a.nsn) decode_combine_kernel<64, false, true><<<nbh, kDecThreads, 0, s>>>(a);
+                else if (qjl) decode_combine_kernel<64, true><<<nbh, kDecThreads, 0, s>>>(a);
+                else decode_combine_kernel<64, false><<<nbh, kDecThreads, 0, s>>>(a);
+                break;
+            case 128:
+                if (a.nsn) decode_combine_kernel<128, false, true><<<nbh, kDecThreads, 0, s>>>(a);
+                else if (qjl) decode_combine_kernel<128, true><<<nbh, kDecThreads, 0, s>>>(a);
+                else decode_combine_kernel<128, false><<<nbh, kDecThreads, 0, s>>>(a);
+                break;
+            default:
+                if (a.nsn) decode_combine_kernel<256, false, true><<<nbh, kDecThreads, 0, s>>>(a);
+                else if (qjl) decode_combine_kernel<256, true><<<nbh, kDecThreads, 0, s>>>(a);
+                else decode_combine_kernel<256, false><<<nbh, kDecThreads, 0, s>>>(a);
+                break;
         }
         return cudaGetLastError();
     }

@@ -87,6 +87,12 @@ __device__ __forceinline__ float load_elem(const void* p, int64_t i) {
     return __uint_as_float(static_cast<uint32_t>(u) << 16);
 }
 
+__device__ __forceinline__ float load_elem_rt(const void* p, int dt, int64_t i) {
+    if (dt == 0) return reinterpret_cast<const float*>(p)[i];
+    const uint16_t u = reinterpret_cast<const uint16_t*>(p)[i];
+    return dt == 1 ? __half2float(__ushort_as_half(u)) : __uint_as_float(static_cast<uint32_t>(u) << 16);
+}
+
 // Warp-level integer products: d(16x8, s32) += a(16x32, u8, row) * b(32x8, s8 or u8, col).
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint2 b) {
     asm volatile(
@@ -274,8 +280,10 @@ __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__
     }
 }
 
-// Shared-memory plan of the split kernel.
-template <int D, int B, bool QJL, int G>
+// Shared-memory plan of the split kernel.  NSN: caches written by the NSN
+// front end (no QJL), whose stages also carry the fp16 block means of keys
+// and values (one D-vector per 128 tokens).
+template <int D, int B, bool QJL, int G, bool NSN = false>
 struct MmaSmem {
     static constexpr int M = D;
     static constexpr int TC = DTile<D>::TC;
@@ -290,17 +298,21 @@ struct MmaSmem {
     static constexpr int kVc = (TC / 32) * B * D * 4;      // value codes (block-32)
     static constexpr int kVq = QJL ? (TC / 32) * M * 4 : 0;
     static constexpr int kVn = TC * 4;
-    static constexpr int kStage = kKc + kKq + kKn + kVc + kVq + kVn;
+    static constexpr int kKm = NSN ? ((TC + 127) / 128) * D * 2 : 0;  // key block means
+    static constexpr int kVm = kKm;                                    // value block means
+    static constexpr int kStage = kKc + kKq + kKn + kVc + kVq + kVn + kKm + kVm;
     static constexpr int kFrag = KS * NTK * 32 * 8;        // query fragments
     static constexpr int kLog = GP * TC * 4;               // logits of the sub-chunk
     static constexpr int kWfrag = (TC / 32) * RT * 32 * 16;  // weight digits, per kind
-    static constexpr int kBytes = 2 * kStage + kFrag + kLog + 2 * kWfrag + 1024;
+    static constexpr int kMisc = NSN ? 1536 : 1024;
+    static constexpr int kBytes = 2 * kStage + kFrag + kLog + 2 * kWfrag + kMisc;
     static constexpr bool kQfReg = KS * NTK <= 24;         // query fragments held in registers
 };
 
-template <int D, int B, bool QJL, int G>
+template <int D, int B, bool QJL, int G, bool NSN = false>
 __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_constant__ DecodeArgs a) {
-    using L = MmaSmem<D, B, QJL, G>;
+    static_assert(!(NSN && QJL), "NSN caches carry no QJL sketch");
+    using L = MmaSmem<D, B, QJL, G, NSN>;
     using HC = HeadCfg<G>;
     constexpr int M = D, TC = L::TC, NTK = L::NTK, RT = L::RT, KS = L::KS, GP = L::GP, CPL = HC::CPL;
     constexpr int KWT = B * D / 32;           // code words per token (key layout)
@@ -319,6 +331,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     float* sred = reinterpret_cast<float*>(misc + 16);      // 96 floats: [4 warps][GP][3] or [4 warps][16]
     float* shead = sred + 96;                                // [GP][8]: item sums (5..7)
     float* sstat = shead + GP * 8;                           // [GP][8]: -, alpha, sig_w/128, sig_wq/128
+    float* sqo = sstat + GP * 8;                             // NSN: [GP][2] scale/sqrt(d) <q, o_k> per block
+    float* sbeta = sqo + GP * 2;                             // NSN: [4 warps][GP][2] sums of e ||x||/sqrt(d)
+    const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
     const uint32_t msk_lo = kLowBits << t, msk_hi = kLowBits << (t + 4);
@@ -351,6 +366,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
         const uint8_t* vc = reinterpret_cast<const uint8_t*>(a.vcodes) + stream * (a.vcap / 32) * B * D * 4;
         const uint8_t* vq = QJL ? reinterpret_cast<const uint8_t*>(a.vqjl) + stream * (a.vcap / 32) * M * 4 : nullptr;
         const uint8_t* vn = reinterpret_cast<const uint8_t*>(a.vnorms) + stream * a.vcap * 4;
+        // NSN: block means, [capacity / 128][D] fp16 per stream
+        const uint8_t* km = NSN ? reinterpret_cast<const uint8_t*>(a.kmean) + stream * (a.kcap / 128) * D * 2 : nullptr;
+        const uint8_t* vm = NSN ? reinterpret_cast<const uint8_t*>(a.vmean) + stream * (a.vcap / 128) * D * 2 : nullptr;
 
         // ---- item set-up (the previous item is done with shared memory) ----
         __syncthreads();
@@ -374,6 +392,19 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                 hk3[hh] = f * kappa * qs[3];
             }
         }
+        // NSN: warp w holds the query of head w (and w + 4 when G = 8) in the
+        // original domain, lane coordinates lane + 32 i, for <q, o_k> per block
+        constexpr int QQ = (NSN && G == 8) ? 2 : 1;
+        float qv[QQ][NSN ? D / 32 : 1];
+        if constexpr (NSN) {
+#pragma unroll
+            for (int qq = 0; qq < QQ; ++qq) {
+                const int h = warp + 4 * qq;
+#pragma unroll
+                for (int i = 0; i < D / 32; ++i)
+                    qv[qq][i] = h < G ? load_elem_rt(a.q, a.qdtype, (qh0 + h) * D + lane + 32 * i) : 0.f;
+            }
+        }
         // running max per head (the same in every thread) and this thread's
         // partial sums of exp, code weights and QJL weights (rescaled with it)
         float mrun[GP], pe[GP], pw[GP], pq[GP];
@@ -391,8 +422,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             const int64_t nt = (have + 31) / 32 * 32;  // <= capacity - tb (capacity is a multiple of 32)
             uint8_t* st = smem + (sc & 1) * L::kStage;
             uint64_t* b = &bar[sc & 1];
+            const int64_t nblk = NSN ? (nt + 127) / 128 : 0;  // block means of the sub-chunk
             const uint32_t bytes = static_cast<uint32_t>(nt * (B * D / 8 + (QJL ? M / 8 : 0) + 4) +
-                                                         (nt / 32) * (B * D * 4 + (QJL ? M * 4 : 0)) + nt * 4);
+                                                         (nt / 32) * (B * D * 4 + (QJL ? M * 4 : 0)) + nt * 4 +
+                                                         2 * nblk * D * 2);
             mbar_arrive_expect_tx(b, bytes);
             bulk_load(st, kc + tb * (B * D / 8), static_cast<uint32_t>(nt * (B * D / 8)), b);
             if (QJL) bulk_load(st + L::kKc, kq + tb * (M / 8), static_cast<uint32_t>(nt * (M / 8)), b);
@@ -404,6 +437,12 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                           static_cast<uint32_t>((nt / 32) * M * 4), b);
             bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq, vn + tb * 4, static_cast<uint32_t>(nt * 4),
                       b);
+            if (NSN) {
+                const uint32_t mb = static_cast<uint32_t>(nblk * D * 2);
+                bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq + L::kVn, km + (tb / 128) * D * 2, mb, b);
+                bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq + L::kVn + L::kKm, vm + (tb / 128) * D * 2,
+                          mb, b);
+            }
             return true;
         };
         bool armed0 = false, armed1 = false;
@@ -445,6 +484,26 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             const uint32_t* sVc = reinterpret_cast<const uint32_t*>(st + L::kKc + L::kKq + L::kKn);
             const uint32_t* sVq = reinterpret_cast<const uint32_t*>(st + L::kKc + L::kKq + L::kKn + L::kVc);
             const __half2* sVn = reinterpret_cast<const __half2*>(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq);
+            const __half* sKm = reinterpret_cast<const __half*>(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq + L::kVn);
+            const __half* sVm = sKm + L::kKm / 2;
+            if constexpr (NSN) {
+                // scale/sqrt(d) <q_h, o_k> for each 128-token block of the sub-chunk
+                // (an unloaded block gives a value no valid token uses)
+#pragma unroll
+                for (int qq = 0; qq < QQ; ++qq)
+#pragma unroll
+                    for (int blk = 0; blk < (TC + 127) / 128; ++blk) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int i = 0; i < D / 32; ++i)
+                            acc = fmaf(qv[qq][i], __half2float(sKm[blk * D + lane + 32 * i]), acc);
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+                        const int h = warp + 4 * qq;
+                        if (lane == 0 && h < GP) sqo[h * 2 + blk] = acc * a.scale * inv_sqrt_d;
+                    }
+                __syncthreads();
+            }
 
             // ---------------- phase K: logits of the sub-chunk ----------------
             float lmax[HH];
@@ -535,7 +594,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                                          static_cast<float>(accq[n1][2 * rr] * 128 + accq[n1][2 * rr + 1]));
                                 inner = fmaf(nk.y, fmaf(hk2[hh], xq, -hk3[hh]), inner);
                             }
-                            l = (h < G && tl < nval) ? nk.x * inner : -INFINITY;
+                            // NSN: l = scale ||x||/sqrt(d) (||w||/d <q', c> + <q, o>)
+                            const float lt = NSN ? nk.x * fmaf(nk.y * inv_sqrt_d, inner, sqo[h * 2 + (tl >> 7)])
+                                                 : nk.x * inner;
+                            l = (h < G && tl < nval) ? lt : -INFINITY;
                             lmax[hh] = fmaxf(lmax[hh], l);
                         }
                         if (h < GP) slog[h * TC + tl] = l;
@@ -551,7 +613,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                 for (int tl = tid; tl < TC; tl += kThreads) {
                     if (tl < nval) {
                         const float2 nv = __half22float2(sVn[tl]);
-                        nmx = fmaxf(nmx, nv.x);
+                        nmx = fmaxf(nmx, NSN ? nv.x * nv.y * inv_sqrt_d : nv.x);
                         ngx = fmaxf(ngx, nv.x * nv.y);
                     }
                 }
@@ -630,13 +692,18 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                 const float fac = static_cast<float>(1 << (7 - s));
                 uint8_t* bc = reinterpret_cast<uint8_t*>(swc) + (u >> 3);
                 uint8_t* bq = reinterpret_cast<uint8_t*>(swq) + (u >> 3);
+                // NSN: the code weight is e ||x|| ||w|| / sqrt(d); the block mean
+                // enters with e ||x|| / sqrt(d), summed per head over the block
+                const float nwc = NSN ? nv.x * nv.y * inv_sqrt_d : nv.x;
+                float eb[NSN ? GP : 1];
 #pragma unroll
                 for (int h = 0; h < GP; ++h) {
                     uint32_t xc, xq = 0u;
                     {
                         const float ex = __expf(slog[h * TC + tl] - mnew[h]);
                         const float e = (valid && h < G) ? ex : 0.f;
-                        const float wc = e * nv.x;
+                        if (NSN) eb[NSN ? h : 0] = e * nv.x * inv_sqrt_d;
+                        const float wc = e * nwc;
                         const float wq = wc * nv.y;
                         pe[h] += e;
                         pw[h] += wc;
@@ -653,6 +720,16 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                             ((((bb * RT + rt) * 32 + 4 * (rl & 7) + (s & 3)) * 4 + (rl >> 3) + 2 * (s >> 2)) << 2);
                         bc[off] = static_cast<uint8_t>(xc >> (8 * k));
                         if (QJL) bq[off] = static_cast<uint8_t>(xq >> (8 * k));
+                    }
+                }
+                if constexpr (NSN) {
+                    // every token of this pass is in block tl >> 7 (tl = tid + 128 i)
+#pragma unroll
+                    for (int h = 0; h < GP; ++h) {
+                        float v = eb[h];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                        if (lane == 0) sbeta[(warp * GP + h) * 2 + (tl >> 7)] = v;
                     }
                 }
             }
@@ -758,6 +835,23 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                             if (B == 2) code = fmaf(coef1, vals[1 % NPV], code);
                             accA[nt][c] = fmaf(accA[nt][c], alpha, sgw * code);
                             if (QJL) accB[nt][c] = fmaf(accB[nt][c], alpha, sgq * 2.f * vals[NPV - 1]);
+                            if (NSN) {
+                                // O += sum_blk beta_blk o_v,blk on this lane's (head, coordinate),
+                                // in the original (unrotated) coordinates; unloaded blocks are skipped
+                                const int col = (G <= 4) ? 2 * t + (g >= 4 ? 1 : 0) : 2 * t + c;
+                                const int coord = warp * (D / 4) + NTV * col + nt;
+                                float add = 0.f;
+#pragma unroll
+                                for (int blk = 0; blk < (TC + 127) / 128; ++blk) {
+                                    if (nval > blk * 128) {
+                                        float bsum = 0.f;
+#pragma unroll
+                                        for (int w = 0; w < 4; ++w) bsum += sbeta[(w * GP + head) * 2 + blk];
+                                        add = fmaf(bsum, __half2float(sVm[blk * D + coord]), add);
+                                    }
+                                }
+                                accB[nt][c] = fmaf(accB[nt][c], alpha, add);
+                            }
                         }
                     }
                 }
@@ -824,6 +918,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                         const int coord = warp * (D / 4) + NTV * col + nt;
                         pp[2 + coord] = c0 * hs[6] + accA[nt][c];
                         if (QJL) pp[2 + D + coord] = accB[nt][c] - hs[7];
+                        if (NSN) pp[2 + D + coord] = accB[nt][c];
                     }
             }
 #pragma unroll
@@ -838,10 +933,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     }
 }
 
-template <int D, int B, bool QJL, int G>
+template <int D, int B, bool QJL, int G, bool NSN = false>
 int ctas_per_sm_g() {
-    using L = MmaSmem<D, B, QJL, G>;
-    auto kern = decode_mma_kernel<D, B, QJL, G>;
+    using L = MmaSmem<D, B, QJL, G, NSN>;
+    auto kern = decode_mma_kernel<D, B, QJL, G, NSN>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess) return 1;
     int n = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, L::kBytes) != cudaSuccess || n < 1) n = 1;
@@ -866,11 +961,28 @@ cudaError_t launch_mma_g(const DecodeArgs& a, int grid, cudaStream_t s) {
         case 1: qfrag_kernel<D, B, QJL, G, 1><<<groups, kThreads, 0, s>>>(a); break;
         default: qfrag_kernel<D, B, QJL, G, 2><<<groups, kThreads, 0, s>>>(a); break;
     }
+    const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit;
+    if constexpr (!QJL) {
+        if (a.nsn) {
+            // NSN caches: the same split plan, on this variant's own persistent grid
+            using LN = MmaSmem<D, B, false, G, true>;
+            auto kn = decode_mma_kernel<D, B, false, G, true>;
+            cudaError_t e = cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, LN::kBytes);
+            if (e != cudaSuccess) return e;
+            int sms = 148, dev = 0;
+            cudaGetDevice(&dev);
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            const int64_t gn = static_cast<int64_t>(ctas_per_sm_g<D, B, false, G, true>()) * sms;
+            const int64_t n = items < gn ? items : gn;
+            if (n <= 0) return cudaSuccess;
+            kn<<<static_cast<unsigned>(n), kThreads, LN::kBytes, s>>>(a);
+            return cudaGetLastError();
+        }
+    }
     using L = MmaSmem<D, B, QJL, G>;
     auto kern = decode_mma_kernel<D, B, QJL, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
-    const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit;
     const int64_t n = items < grid ? items : grid;
     if (n <= 0) return cudaSuccess;
     kern<<<static_cast<unsigned>(n), kThreads, L::kBytes, s>>>(a);

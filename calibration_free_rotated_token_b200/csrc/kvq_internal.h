@@ -98,6 +98,11 @@ struct DecodeArgs {
     const __half* S;
     float centroid[kMaxLevels];
     uint32_t pair_sign[128];
+    // NSN caches (no QJL): fp16 block means, [capacity / 128][d] per stream;
+    // the partials' second vector then holds the block-mean term O.
+    int nsn;
+    const __half* kmean;
+    const __half* vmean;
 };
 
 // Bytes of workspace and number of splits for a decode of these sizes.

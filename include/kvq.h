@@ -185,12 +185,14 @@ int kvq_quantize_batch(kvq_handle h, int count, const kvq_quant_job* jobs, void*
  *   x           device, [n_heads][n_tok][d] contiguous, dtype as above.
  *   n_tok       tokens per head, a multiple of 128 (the full-precision tail
  *               of a real cache stays outside, NSNQuant section 4).
+ *   layout      KVQ_LAYOUT_TOKEN (keys) or KVQ_LAYOUT_BLOCK32 (values; blocks
+ *               of 32 tokens never straddle heads since n_tok % 128 == 0).
  *   codes       device, n_heads * n_tok * b * d/32 uint32.
  *   norms       device, n_heads * n_tok * 2 fp16.
  *   block_mean  device, n_heads * (n_tok/128) * d fp16.
  * Requires a handle without KVQ_QJL (KVQ_EINVAL otherwise).
  */
-int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok,
+int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, int layout,
                      uint32_t* codes, uint16_t* norms, uint16_t* block_mean, void* stream);
 
 /* One packed cache (keys or values) of batch * hkv streams, each holding up
@@ -242,6 +244,30 @@ int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq,
 /* Bytes of the fixed decode scratch built into the library (see
  * kvq_decode_attend_noalloc). */
 #define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * kvq_nsn_decode_attend -- kvq_decode_attend over caches written by
+ * kvq_nsn_quantize (NSNQuant section 4: attention straight from the stored
+ * byproducts).  A stored vector stands for
+ *   x_hat = ||x||/sqrt(d) (w_hat + o_blk),
+ * where w_hat is the codebook vector rotated back and scaled to ||w|| (the
+ * plain dequantization with norm ||w||), and o_blk is the fp16 mean of its
+ * block of 128 tokens.  So
+ *   l_t = scale ||x_t||/sqrt(d) (||w_t||/d <q', c[code_t]> + <q, o_blk(t)>),
+ *   out = sum_t p_t x_hat(v_t).
+ * Arguments as kvq_decode_attend, and:
+ *   k, v          norms hold (fp16 ||x||, fp16 ||w||); codes as usual; no QJL.
+ *   k_block_mean, v_block_mean
+ *                 device, fp16; per stream capacity/128 blocks of d, stream
+ *                 (bi, hi) at block (bi * hkv + hi) * capacity/128, 16-byte
+ *                 aligned.  Capacities must be multiples of 128.
+ * The workspace size is kvq_decode_workspace's.  Requires a handle without
+ * KVQ_QJL (KVQ_EINVAL) and b <= 2 (KVQ_EUNSUPPORTED otherwise).
+ */
+int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
+                          const kvq_cache* v, const uint16_t* k_block_mean, const uint16_t* v_block_mean,
+                          const int32_t* seq_len, int64_t max_T, float scale, float* logits, float* out,
+                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * kvq_decode_attend_noalloc -- kvq_decode_attend without a caller-provided

@@ -15,7 +15,7 @@ import oracle
 from calibration_free_rotated_token_b200 import _abi as kvq
 from calibration_free_rotated_token_b200 import workloads as wl
 
-from .parity import CODE_BAND, max_excluded, to_np_f16bits, to_np_u32, ulp_distance_f16
+from .parity import CODE_BAND, assert_close, max_excluded, to_np_f16bits, to_np_u32, ulp_distance_f16
 
 pytestmark = pytest.mark.gpu
 
@@ -111,3 +111,142 @@ def test_nsn_workload_full_size_sampled():
     sl = slice(c["tokens"] - 128, c["tokens"])
     check_head(k, x[-1, sl].double().cpu().numpy(), to_np_u32(codes[-1, sl]), to_np_f16bits(norms[-1, sl]),
                to_np_f16bits(means[-1, -1:]))
+
+
+def test_nsn_block32_layout_matches_token_layout():
+    """Values are stored in the block-32 layout: the same bits, norms and block means."""
+    d, b = 128, 2
+    x = wl.nsn_tokens(2, 256, d, seed=9).cuda()
+    with kvq.Handle(d, b, 3, qjl=False) as h:
+        c0, n0, m0 = run_nsn(h, x)
+        c1 = torch.empty((2, 256 // 32, b, d), dtype=torch.int32, device="cuda")
+        n1 = torch.empty_like(n0)
+        m1 = torch.empty_like(m0)
+        kvq.kvq_nsn_quantize(h, x, c1, n1, m1, layout=kvq.KVQ_LAYOUT_BLOCK32)
+        assert kvq.kvq_status(h)[0] == 0
+    for hh in range(2):
+        np.testing.assert_array_equal(oracle.unpack_codes_block32(to_np_u32(c1[hh]), b, d, 256),
+                                      oracle.unpack_codes(to_np_u32(c0[hh]).reshape(256, -1), b, d))
+    assert torch.equal(n0, n1) and torch.equal(m0, m1)
+
+
+# ---------------------------------------------------------------------------
+# Decode attention over NSN caches (kvq_nsn_decode_attend)
+# ---------------------------------------------------------------------------
+def _nsn_oracle_stream(k, X):
+    """The oracle's NSN cache of one stream X [T, d] (T % 128 == 0): packed key and value
+    records, norms, block means, and the stored values the oracle decodes from."""
+    r = oracle.nsn_quantize(k, X)
+    nb = np.stack([r["norm_x"].astype(np.float16), r["norm_w"].astype(np.float16)], axis=1)
+    stored = dict(codes=r["codes"], norm_x=nb[:, 0].astype(np.float64), norm_w=nb[:, 1].astype(np.float64))
+    return r, nb, stored
+
+
+def check_nsn_decode(d, b, batch, hq, hkv, seq_len, cap, qdtype=torch.bfloat16, seed=5):
+    k = oracle.make_constants(d, b, seed)
+    G = hq // hkv
+    S = batch * hkv
+    kc = torch.zeros((S, cap, b, d // 32), dtype=torch.int32)
+    vc = torch.zeros((S, cap // 32, b, d), dtype=torch.int32)
+    kn = torch.zeros((S, cap, 2), dtype=torch.float16)
+    vn = torch.zeros_like(kn)
+    km = torch.zeros((S, cap // 128, d), dtype=torch.float16)
+    vm = torch.zeros_like(km)
+    kst, vst = [], []
+    for s in range(S):
+        K = wl.nsn_tokens(1, cap, d, seed=700 + s)[0].double().numpy()
+        V = wl.nsn_tokens(1, cap, d, seed=900 + s)[0].double().numpy()
+        rk, nbk, sk = _nsn_oracle_stream(k, K)
+        rv, nbv, sv = _nsn_oracle_stream(k, V)
+        kc[s] = torch.from_numpy(oracle.pack_codes(rk["codes"], b).view(np.int32))
+        vc[s] = torch.from_numpy(oracle.pack_codes_block32(rv["codes"], b).view(np.int32).reshape(cap // 32, b, d))
+        kn[s] = torch.from_numpy(nbk)
+        vn[s] = torch.from_numpy(nbv)
+        km[s] = torch.from_numpy(rk["mean_half"].view(np.float16))
+        vm[s] = torch.from_numpy(rv["mean_half"].view(np.float16))
+        kst.append((sk, rk["mean_half"]))
+        vst.append((sv, rv["mean_half"]))
+    q = wl.queries(batch, hq, d, seed=77, dtype=qdtype)
+    scale = 1 / np.sqrt(d)
+    max_T = max(seq_len)
+    with kvq.Handle(d, b, seed, qjl=False) as h:
+        kcd, vcd, knd, vnd, kmd, vmd = (t.cuda() for t in (kc, vc, kn, vn, km, vm))
+        kcache = kvq.make_cache(kcd, None, knd, cap, 0)
+        vcache = kvq.make_cache(vcd, None, vnd, cap, 1)
+        out = torch.empty((batch, hq, d), dtype=torch.float32, device="cuda")
+        logits = torch.empty((batch, hq, max_T), dtype=torch.float32, device="cuda")
+        ws = torch.empty(kvq.kvq_decode_workspace(h, batch, hq, hkv, max_T), dtype=torch.uint8, device="cuda")
+        sl = torch.tensor(seq_len, dtype=torch.int32, device="cuda")
+        kvq.kvq_nsn_decode_attend(h, q.cuda(), hkv, kcache, vcache, kmd, vmd, sl, max_T, scale, out, ws, logits)
+        code, bits = kvq.kvq_status(h)
+        assert code == 0, (code, bits)
+        out, logits = out.cpu().numpy(), logits.cpu().numpy()
+    qd = q.double().numpy()
+    for bi in range(batch):
+        T = seq_len[bi]
+        nblk = (T + 127) // 128
+        for hk in range(hkv):
+            s = bi * hkv + hk
+            sk = {key: v[:T] for key, v in kst[s][0].items()}
+            sv = {key: v[:T] for key, v in vst[s][0].items()}
+            lr, orf = oracle.nsn_decode_attend(k, qd[bi, hk * G:(hk + 1) * G], sk, sv, kst[s][1][:nblk],
+                                               vst[s][1][:nblk], scale)
+            assert_close(out[bi, hk * G:(hk + 1) * G], orf, f"nsn out b{bi} kvh{hk}")
+            if T > 0:
+                assert_close(logits[bi, hk * G:(hk + 1) * G, :T], lr, f"nsn logits b{bi} kvh{hk}")
+            assert np.all(logits[bi, hk * G:(hk + 1) * G, T:] == -np.inf)
+
+
+@pytest.mark.parametrize("d,b,batch,hq,hkv,seq_len,cap", [
+    (128, 2, 2, 8, 2, [1000, 300], 1024),    # GQA 4:1, ragged contexts, partial blocks
+    (64, 1, 1, 4, 4, [640], 640),            # GQA 1:1
+    (128, 2, 1, 16, 2, [2000], 2048),        # GQA 8:1
+    (256, 2, 1, 4, 2, [513], 640),           # 128-token sub-chunks (one block each)
+    (128, 1, 2, 4, 1, [0, 129], 256),        # an empty context
+])
+def test_nsn_decode_matches_oracle(d, b, batch, hq, hkv, seq_len, cap):
+    check_nsn_decode(d, b, batch, hq, hkv, seq_len, cap)
+
+
+def test_nsn_decode_long_context():
+    """Many splits merged exactly, the block-mean term included."""
+    check_nsn_decode(128, 2, 1, 4, 1, [20480], 20480)
+
+
+def test_nsn_decode_workload_full_size_sampled():
+    """The NSN workload (8 heads x 65536 tokens, b=2) quantized by the CUDA NSN front end, keys per
+    token and values in blocks of 32, then decoded by 32 query heads (GQA 4:1, one token); two
+    sampled KV heads against the oracle's decode of the same stored cache."""
+    c = wl.NSN
+    H, T, d = c["heads"], c["tokens"], c["d"]
+    k = oracle.make_constants(d, c["b"], c["handle_seed"])
+    X = wl.nsn_tokens(H, T, d, c["seed"], device="cuda")
+    Y = wl.nsn_tokens(H, T, d, c["seed"] + 1, device="cuda")
+    with kvq.Handle(d, c["b"], c["handle_seed"], qjl=False) as h:
+        kc = torch.empty((H, T, h.b, d // 32), dtype=torch.int32, device="cuda")
+        vc = torch.empty((H, T // 32, h.b, d), dtype=torch.int32, device="cuda")
+        kn = torch.empty((H, T, 2), dtype=torch.float16, device="cuda")
+        vn = torch.empty_like(kn)
+        km = torch.empty((H, T // 128, d), dtype=torch.float16, device="cuda")
+        vm = torch.empty_like(km)
+        kvq.kvq_nsn_quantize(h, X, kc, kn, km)
+        kvq.kvq_nsn_quantize(h, Y, vc, vn, vm, layout=kvq.KVQ_LAYOUT_BLOCK32)
+        q = wl.queries(1, 4 * H, d, seed=78, device="cuda")
+        out = torch.empty((1, 4 * H, d), dtype=torch.float32, device="cuda")
+        ws = torch.empty(kvq.kvq_decode_workspace(h, 1, 4 * H, H, T), dtype=torch.uint8, device="cuda")
+        sl = torch.tensor([T], dtype=torch.int32, device="cuda")
+        kvq.kvq_nsn_decode_attend(h, q, H, kvq.make_cache(kc, None, kn, T, 0), kvq.make_cache(vc, None, vn, T, 1),
+                                  km, vm, sl, T, d ** -0.5, out, ws)
+        assert kvq.kvq_status(h)[0] == 0
+    qd = q.double().cpu().numpy()
+    out = out.cpu().numpy()
+    for hk in (2, 7):
+        nk = oracle.half_bits_to_double(to_np_f16bits(kn[hk]).reshape(T, 2))
+        nv = oracle.half_bits_to_double(to_np_f16bits(vn[hk]).reshape(T, 2))
+        sk = dict(codes=oracle.unpack_codes(to_np_u32(kc[hk]).reshape(T, -1), c["b"], d), norm_x=nk[:, 0],
+                  norm_w=nk[:, 1])
+        sv = dict(codes=oracle.unpack_codes_block32(to_np_u32(vc[hk]), c["b"], d, T), norm_x=nv[:, 0],
+                  norm_w=nv[:, 1])
+        _, orf = oracle.nsn_decode_attend(k, qd[0, 4 * hk:4 * hk + 4], sk, sv, to_np_f16bits(km[hk]),
+                                          to_np_f16bits(vm[hk]), d ** -0.5, want_logits=False)
+        assert_close(out[0, 4 * hk:4 * hk + 4], orf, f"nsn workload out kvh{hk}")

@@ -170,7 +170,7 @@ def test_host_side_argument_errors():
         assert code == kvq.KVQ_EINVAL
         with pytest.raises(ValueError):
             kvq.kvq_quantize(h, x[:, :64], codes, qjl, norms)
-    assert kvq.load().kvq_nsn_quantize(h.ptr if False else None, None, 0, 1, 128, None, None, None, None) \
+    assert kvq.load().kvq_nsn_quantize(h.ptr if False else None, None, 0, 1, 128, 0, None, None, None, None) \
         == kvq.KVQ_EINVAL
 
 
