@@ -35,7 +35,7 @@ STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
 EXPORTED = (
     "kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize", "kvq_decode_workspace",
     "kvq_decode_attend", "kvq_decode_attend_noalloc", "kvq_status", "kvq_last_error", "kvq_get_constants",
-    "kvq_get_info", "kvq_codebook", "kvq_nsn_decode_attend",
+    "kvq_get_info", "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -51,6 +51,17 @@ class KvqError(RuntimeError):
 class KvqCache(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("qjl", ctypes.c_void_p), ("norms", ctypes.c_void_p),
                 ("capacity", ctypes.c_int64), ("layout", ctypes.c_int32)]
+
+
+class KvqDecodeDesc(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("batch", ctypes.c_int32),
+                ("hq", ctypes.c_int32), ("hkv", ctypes.c_int32), ("k", ctypes.POINTER(KvqCache)),
+                ("v", ctypes.POINTER(KvqCache)), ("k_block_mean", ctypes.c_void_p),
+                ("v_block_mean", ctypes.c_void_p), ("k_window", ctypes.c_void_p), ("v_window", ctypes.c_void_p),
+                ("window_cap", ctypes.c_int64), ("window_len", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
+                ("max_T", ctypes.c_int64), ("scale", ctypes.c_float), ("logits", ctypes.c_void_p),
+                ("logits_ld", ctypes.c_int64), ("out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("ws_bytes", ctypes.c_size_t)]
 
 
 class KvqQuantJob(ctypes.Structure):
@@ -90,12 +101,13 @@ def load() -> ctypes.CDLL:
         L.kvq_get_constants.argtypes = [P, P, P, P, P]
         L.kvq_get_info.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(U32)]
         L.kvq_codebook.argtypes = [I, I, U32, P, P]
+        L.kvq_decode_attend_ex.argtypes = [P, ctypes.POINTER(KvqDecodeDesc), P]
         L.kvq_nsn_decode_attend.argtypes = [P, P, I, I, I, I, ctypes.POINTER(KvqCache), ctypes.POINTER(KvqCache),
                                             P, P, P, I64, ctypes.c_float, P, P, P, SZ, P]
         for name in ("kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize",
                      "kvq_decode_attend",
                      "kvq_decode_attend_noalloc", "kvq_status", "kvq_get_constants", "kvq_get_info",
-                     "kvq_codebook", "kvq_nsn_decode_attend"):
+                     "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex"):
             getattr(L, name).restype = I
         _lib = L
         return L
@@ -317,6 +329,38 @@ def kvq_nsn_decode_attend(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache
                                         ctypes.byref(vcache), _ptr(k_block_mean), _ptr(v_block_mean),
                                         _ptr(seq_len), max_T, float(scale), _ptr(logits), _ptr(out),
                                         _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def kvq_decode_attend_ex(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vcache: KvqCache,
+                         seq_len: torch.Tensor, max_T: int, scale: float, out: torch.Tensor, workspace: torch.Tensor,
+                         k_window: torch.Tensor | None = None, v_window: torch.Tensor | None = None,
+                         window_len: torch.Tensor | None = None, k_block_mean: torch.Tensor | None = None,
+                         v_block_mean: torch.Tensor | None = None, logits: torch.Tensor | None = None,
+                         logits_ld: int = 0, stream=None):
+    """Decode over a packed cache (plain or NSN) and an optional fp16 residual window
+    ([batch * hkv, window_cap, d]); window_len int32 [batch] on the device."""
+    if q.dim() != 3 or q.shape[-1] != h.d:
+        raise ValueError(f"q must be [batch, hq, {h.d}]")
+    _need(q, "q")
+    B, hq, _ = q.shape
+    _need(seq_len, "seq_len", dtype=torch.int32, numel=B)
+    _need(out, "out", dtype=torch.float32, numel=B * hq * h.d)
+    _need(workspace, "workspace")
+    cap = 0
+    if k_window is not None or v_window is not None:
+        _need(k_window, "k_window", dtype=torch.float16)
+        _need(v_window, "v_window", dtype=torch.float16)
+        _need(window_len, "window_len", dtype=torch.int32, numel=B)
+        cap = k_window.shape[-2]
+        if k_window.numel() != B * hkv * cap * h.d or v_window.shape != k_window.shape:
+            raise ValueError("windows must be [batch * hkv, window_cap, d]")
+    if logits is not None:
+        _need(logits, "logits", dtype=torch.float32, numel=B * hq * (logits_ld or (max_T + cap)))
+    d = KvqDecodeDesc(_ptr(q), _DTYPES[q.dtype], B, hq, hkv, ctypes.pointer(kcache), ctypes.pointer(vcache),
+                      _ptr(k_block_mean), _ptr(v_block_mean), _ptr(k_window), _ptr(v_window), cap,
+                      _ptr(window_len), _ptr(seq_len), max_T, float(scale), _ptr(logits), logits_ld, _ptr(out),
+                      _ptr(workspace), workspace.numel() * workspace.element_size())
+    _check(load().kvq_decode_attend_ex(h.ptr, ctypes.byref(d), _stream(stream)))
 
 
 def kvq_decode_attend_noalloc(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vcache: KvqCache,

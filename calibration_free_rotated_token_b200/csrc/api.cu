@@ -55,6 +55,8 @@ cudaError_t launch_quantize_any(int d, int b, bool qjl, bool nsn, const CUtensor
 }  // namespace
 }  // namespace kvq
 
+static_assert(kvq::kMaxWindow == KVQ_MAX_WINDOW, "window bound of the header and the kernels");
+
 namespace {
 
 thread_local std::string g_err;
@@ -510,20 +512,39 @@ int decode_check(kvq_handle h, int dtype, int batch, int hq, int hkv, const kvq_
     return KVQ_OK;
 }
 
+// Optional parts of a decode call: NSN block means, a residual window, the
+// logits row stride.
+struct DecodeExtras {
+    const uint16_t* kmean = nullptr;
+    const uint16_t* vmean = nullptr;
+    const uint16_t* kwin = nullptr;
+    const uint16_t* vwin = nullptr;
+    int64_t win_cap = 0;
+    const int32_t* win_len = nullptr;
+    int64_t logits_ld = 0;
+};
+
 int decode_launch(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
                   const kvq_cache* v, const int32_t* seq_len, int64_t max_T, float scale, float* logits,
-                  float* out, void* workspace, int ns, int64_t chunk, void* stream, const uint16_t* kmean = nullptr,
-                  const uint16_t* vmean = nullptr) {
+                  float* out, void* workspace, int ns, int64_t chunk, void* stream,
+                  const DecodeExtras& x = DecodeExtras()) {
     kvq::DecodeArgs a{};
-    a.nsn = kmean != nullptr;
-    a.kmean = reinterpret_cast<const __half*>(kmean);
-    a.vmean = reinterpret_cast<const __half*>(vmean);
+    a.nsn = x.kmean != nullptr;
+    a.kmean = reinterpret_cast<const __half*>(x.kmean);
+    a.vmean = reinterpret_cast<const __half*>(x.vmean);
+    a.kwin = reinterpret_cast<const __half*>(x.kwin);
+    a.vwin = reinterpret_cast<const __half*>(x.vwin);
+    a.win_cap = x.win_cap;
+    a.win_len = x.win_len;
+    a.win_dim = h->d;
+    a.logits_ld = x.logits_ld > 0 ? x.logits_ld : max_T;
     a.batch = batch;
     a.hq = hq;
     a.hkv = hkv;
     a.G = hq / hkv;
     a.max_T = max_T;
-    a.nsplit = ns;
+    a.nsplit_run = ns;
+    a.nsplit = ns + (x.kwin != nullptr ? 1 : 0);  // the window's partial is the last split
     a.chunk = chunk;
     a.q = q;
     a.qdtype = dtype;
@@ -542,7 +563,7 @@ int decode_launch(kvq_handle h, const void* q, int dtype, int batch, int hq, int
     const int64_t bh = static_cast<int64_t>(batch) * hq;
     const int64_t streams = static_cast<int64_t>(batch) * hkv;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    size_t off = static_cast<size_t>(bh * ns * (2 + h->d + h->m)) * sizeof(float);
+    size_t off = static_cast<size_t>(bh * (ns + 1) * (2 + h->d + h->m)) * sizeof(float);
     off = (off + 255) / 256 * 256;
     a.part = reinterpret_cast<float*>(ws);
     if (kvq::decode_uses_mma(h)) {
@@ -603,8 +624,53 @@ int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int
         return fail(KVQ_EINVAL, "block means must be non-null and 16-byte aligned");
     if (!workspace || !aligned(workspace, 16)) return fail(KVQ_EINVAL, "workspace must be non-null and 16-byte aligned");
     if (ws_bytes < need) return fail(KVQ_EINVAL, "workspace too small: need " + std::to_string(need) + " bytes");
+    DecodeExtras x;
+    x.kmean = k_block_mean;
+    x.vmean = v_block_mean;
     return decode_launch(h, q, dtype, batch, hq, hkv, k, v, seq_len, max_T, scale, logits, out, workspace, ns, chunk,
-                         stream, k_block_mean, v_block_mean);
+                         stream, x);
+}
+
+int kvq_decode_attend_ex(kvq_handle h, const kvq_decode_desc* d, void* stream) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    if (!d) return fail(KVQ_EINVAL, "null descriptor");
+    int ns = 0;
+    int64_t chunk = 0;
+    size_t need = 0;
+    if (int e = decode_check(h, d->dtype, d->batch, d->hq, d->hkv, d->k, d->v, d->q, d->seq_len, d->max_T, d->scale,
+                             d->out, &ns, &chunk, &need))
+        return e;
+    DecodeExtras x;
+    if (d->k_block_mean || d->v_block_mean) {
+        if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
+        if (h->b > 2) return fail(KVQ_EUNSUPPORTED, "decode over NSN caches is built for b <= 2");
+        if (!d->k_block_mean || !d->v_block_mean || !aligned(d->k_block_mean, 16) || !aligned(d->v_block_mean, 16))
+            return fail(KVQ_EINVAL, "block means must both be non-null and 16-byte aligned");
+        if (d->k->capacity % 128 != 0 || d->v->capacity % 128 != 0)
+            return fail(KVQ_EINVAL, "NSN cache capacities must be multiples of 128 (one block mean per 128 tokens)");
+        x.kmean = d->k_block_mean;
+        x.vmean = d->v_block_mean;
+    }
+    if (d->k_window || d->v_window) {
+        if (!d->k_window || !d->v_window || !d->window_len || !aligned(d->k_window, 16) || !aligned(d->v_window, 16))
+            return fail(KVQ_EINVAL, "the window needs k_window, v_window (16-byte aligned) and window_len");
+        if (d->window_cap < 1 || d->window_cap > KVQ_MAX_WINDOW)
+            return fail(KVQ_EINVAL, "window_cap must be in 1.." + std::to_string(KVQ_MAX_WINDOW));
+        x.kwin = d->k_window;
+        x.vwin = d->v_window;
+        x.win_cap = d->window_cap;
+        x.win_len = d->window_len;
+    }
+    const int64_t row = d->max_T + (x.kwin ? d->window_cap : 0);
+    if (d->logits && d->logits_ld != 0 && d->logits_ld < row)
+        return fail(KVQ_EINVAL, "logits_ld must be at least max_T (+ window_cap with a window)");
+    x.logits_ld = d->logits_ld != 0 ? d->logits_ld : row;
+    if (!d->workspace || !aligned(d->workspace, 16))
+        return fail(KVQ_EINVAL, "workspace must be non-null and 16-byte aligned");
+    if (d->ws_bytes < need) return fail(KVQ_EINVAL, "workspace too small: need " + std::to_string(need) + " bytes");
+    return decode_launch(h, d->q, d->dtype, d->batch, d->hq, d->hkv, d->k, d->v, d->seq_len, d->max_T, d->scale,
+                         d->logits, d->out, d->workspace, ns, chunk, stream, x);
 }
 
 int kvq_decode_attend_noalloc(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv,

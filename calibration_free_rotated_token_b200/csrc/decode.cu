@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         }
         if (a.logits != nullptr && mine && t < t1e) {
 #pragma unroll
-            for (int g = 0; g < G; ++g) a.logits[(qh0 + g) * a.max_T + t] = l[g];
+            for (int g = 0; g < G; ++g) a.logits[(qh0 + g) * a.logits_ld + t] = l[g];
         }
         // stage the value bit planes (blocks of 32 tokens) and norms of this tile
         {
@@ -326,6 +326,91 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     }
 }
 
+__device__ __forceinline__ float load_any(const void* p, int dt, int64_t i) {
+    if (dt == 0) return reinterpret_cast<const float*>(p)[i];
+    const uint16_t u = reinterpret_cast<const uint16_t*>(p)[i];
+    return dt == 1 ? __half2float(__ushort_as_half(u)) : __uint_as_float(static_cast<uint32_t>(u) << 16);
+}
+
+// The full-precision residual window of one (sequence, KV head) as one more
+// split partial (NSNQuant section 4: the newest tokens stay unquantized until
+// a block is flushed): exact fp32 logits of its fp16 keys, its own max M and
+// sum L, and y = sum_t e_t v_t.  Stored so that the combine's arithmetic
+// gives y back: A = H (delta .* y) (delta .* H A / d = y), or for NSN caches
+// the block-mean slot O = y.  An empty window leaves M = -inf, L = 0.
+template <int D, int G, bool NSN>
+__global__ void __launch_bounds__(kDecThreads) decode_window_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int PART = 2 + 2 * D;
+    __shared__ float sq[G][D];
+    __shared__ float sl[G][kMaxWindow];
+    __shared__ float sy[D];
+    __shared__ float smx[G], ssum[G];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t stream = blockIdx.x;
+    const int bi = static_cast<int>(stream / a.hkv), hk = static_cast<int>(stream % a.hkv);
+    const int64_t qh0 = static_cast<int64_t>(bi) * a.hq + static_cast<int64_t>(hk) * G;
+    const int n = static_cast<int>(min(max(static_cast<int64_t>(a.win_len[bi]), int64_t(0)), a.win_cap));
+    const __half* kw = a.kwin + stream * a.win_cap * D;
+    const __half* vw = a.vwin + stream * a.win_cap * D;
+    for (int e = tid; e < G * D; e += blockDim.x) sq[e / D][e % D] = load_any(a.q, a.qdtype, qh0 * D + e);
+    __syncthreads();
+    // logits, one (token, head) per thread
+    for (int e = tid; e < n * G; e += blockDim.x) {
+        const int t = e / G, h = e % G;
+        const __half2* kr = reinterpret_cast<const __half2*>(kw + static_cast<int64_t>(t) * D);
+        float acc = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < D / 2; ++j) {
+            const float2 kv = __half22float2(kr[j]);
+            acc = fmaf(kv.y, sq[h][2 * j + 1], fmaf(kv.x, sq[h][2 * j], acc));
+        }
+        const float l = a.scale * acc;
+        sl[h][t] = l;
+        if (a.logits != nullptr) a.logits[(qh0 + h) * a.logits_ld + a.max_T + t] = l;
+    }
+    __syncthreads();
+    // per head (one warp each): max, weights e = exp(l - max), their sum
+    for (int h = warp; h < G; h += blockDim.x / 32) {
+        float m = -INFINITY;
+        for (int t = lane; t < n; t += 32) m = fmaxf(m, sl[h][t]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        float sum = 0.f;
+        for (int t = lane; t < n; t += 32) {
+            const float e = __expf(sl[h][t] - m);
+            sl[h][t] = e;
+            sum += e;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        if (lane == 0) {
+            smx[h] = m;
+            ssum[h] = sum;
+        }
+    }
+    __syncthreads();
+    for (int h = 0; h < G; ++h) {
+        float* pp = a.part + ((qh0 + h) * a.nsplit + (a.nsplit - 1)) * PART;
+        // y = sum_t e_t v_t, one coordinate per thread (coalesced rows of V)
+        for (int j = tid; j < D; j += blockDim.x) {
+            float acc = 0.f;
+            for (int t = 0; t < n; ++t) acc = fmaf(sl[h][t], __half2float(vw[static_cast<int64_t>(t) * D + j]), acc);
+            sy[j] = NSN ? acc : sign_of(a.pair_sign, j) * acc;
+        }
+        __syncthreads();
+        if (!NSN) fwht_smem<D>(sy);  // A = H (delta .* y)
+        for (int j = tid; j < D; j += blockDim.x) {
+            pp[2 + j] = NSN ? 0.f : sy[j];
+            pp[2 + D + j] = NSN ? sy[j] : 0.f;
+        }
+        if (tid == 0) {
+            pp[0] = n > 0 ? smx[h] : -INFINITY;
+            pp[1] = n > 0 ? ssum[h] : 0.f;
+        }
+        __syncthreads();
+    }
+}
+
 // Merge the splits of one (batch, query head) and rotate back.  NSN: the
 // second vector of each partial is the block-mean term O (no QJL), added
 // after the inverse rotation: out = delta .* H A / (d L) + O / L.
@@ -426,12 +511,16 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
         case 1: qproj_kernel<D, 1, QJL><<<nbh, block, 0, s>>>(a); break;
         default: qproj_kernel<D, 2, QJL><<<nbh, block, 0, s>>>(a); break;
     }
-    const dim3 grid(a.nsplit, a.hkv, a.batch);
+    const dim3 grid(a.nsplit_run, a.hkv, a.batch);
     switch (a.G) {
         case 1: decode_split_kernel<D, B, QJL, 1><<<grid, block, 0, s>>>(a); break;
         case 2: decode_split_kernel<D, B, QJL, 2><<<grid, block, 0, s>>>(a); break;
         case 4: decode_split_kernel<D, B, QJL, 4><<<grid, block, 0, s>>>(a); break;
         default: decode_split_kernel<D, B, QJL, 8><<<grid, block, 0, s>>>(a); break;
+    }
+    if (a.kwin != nullptr) {
+        const cudaError_t e = launch_decode_window(nullptr, a, s);
+        if (e != cudaSuccess) return e;
     }
     decode_combine_kernel<D, QJL><<<nbh, block, 0, s>>>(a);
     return cudaGetLastError();
@@ -484,8 +573,9 @@ void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, in
     *nsplit = static_cast<int>(ns);
     *chunk = ch;
     const int64_t bh = static_cast<int64_t>(batch) * hq;
-    // partials first (both paths), then the path's query data
-    size_t bytes = static_cast<size_t>(bh * ns * (2 + h->d + h->m)) * sizeof(float);
+    // partials first (both paths; one more split for a residual window), then
+    // the path's query data
+    size_t bytes = static_cast<size_t>(bh * (ns + 1) * (2 + h->d + h->m)) * sizeof(float);
     bytes = (bytes + 255) / 256 * 256;
     if (decode_uses_mma(h)) {
         bytes += static_cast<size_t>(bh) * 4 * sizeof(float);
@@ -502,6 +592,10 @@ cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s,
     if (decode_uses_mma(h)) {
         cudaError_t e = launch_decode_mma(h, a, s);
         if (e != cudaSuccess) return e;
+        if (a.kwin != nullptr) {
+            e = launch_decode_window(h, a, s);
+            if (e != cudaSuccess) return e;
+        }
         const unsigned nbh = static_cast<unsigned>(a.batch * a.hq);
         switch (h->d) {
             case 64:
@@ -529,6 +623,34 @@ cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s,
         default:
             if (why) *why = "unsupported head dimension";
             return cudaErrorInvalidValue;
+    }
+}
+
+namespace {
+template <int D, int G>
+cudaError_t window_g(const DecodeArgs& a, cudaStream_t s) {
+    const unsigned n = static_cast<unsigned>(a.batch * a.hkv);
+    if (a.nsn) decode_window_kernel<D, G, true><<<n, kDecThreads, 0, s>>>(a);
+    else decode_window_kernel<D, G, false><<<n, kDecThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+template <int D>
+cudaError_t window_d(const DecodeArgs& a, cudaStream_t s) {
+    switch (a.G) {
+        case 1: return window_g<D, 1>(a, s);
+        case 2: return window_g<D, 2>(a, s);
+        case 4: return window_g<D, 4>(a, s);
+        default: return window_g<D, 8>(a, s);
+    }
+}
+}  // namespace
+
+cudaError_t launch_decode_window(const kvq_ctx*, const DecodeArgs& a, cudaStream_t s) {
+    const int D = static_cast<int>(a.win_dim);
+    switch (D) {
+        case 64: return window_d<64>(a, s);
+        case 128: return window_d<128>(a, s);
+        default: return window_d<256>(a, s);
     }
 }
 

@@ -349,11 +349,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     }
     uint32_t phase[2] = {0u, 0u};
     bool alive = true;
-    const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit;
+    const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit_run;
 
     for (int64_t item = blockIdx.x; item < items && alive; item += gridDim.x) {
-        const int split = static_cast<int>(item % a.nsplit);
-        const int64_t stream = item / a.nsplit;
+        const int split = static_cast<int>(item % a.nsplit_run);
+        const int64_t stream = item / a.nsplit_run;
         const int hk = static_cast<int>(stream % a.hkv), bi = static_cast<int>(stream / a.hkv);
         const int64_t T = min(static_cast<int64_t>(max(a.seq_len[bi], 0)), a.max_T);
         const int64_t t0 = static_cast<int64_t>(split) * a.chunk;
@@ -601,7 +601,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                             lmax[hh] = fmaxf(lmax[hh], l);
                         }
                         if (h < GP) slog[h * TC + tl] = l;
-                        if (a.logits != nullptr && h < G && tl < nval_e) a.logits[(qh0 + h) * a.max_T + tb + tl] = l;
+                        if (a.logits != nullptr && h < G && tl < nval_e) a.logits[(qh0 + h) * a.logits_ld + tb + tl] = l;
                     }
                 }
             }
@@ -961,7 +961,7 @@ cudaError_t launch_mma_g(const DecodeArgs& a, int grid, cudaStream_t s) {
         case 1: qfrag_kernel<D, B, QJL, G, 1><<<groups, kThreads, 0, s>>>(a); break;
         default: qfrag_kernel<D, B, QJL, G, 2><<<groups, kThreads, 0, s>>>(a); break;
     }
-    const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit;
+    const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit_run;
     if constexpr (!QJL) {
         if (a.nsn) {
             // NSN caches: the same split plan, on this variant's own persistent grid

@@ -103,7 +103,23 @@ struct DecodeArgs {
     int nsn;
     const __half* kmean;
     const __half* vmean;
+    // Splits over the packed cache (nsplit counts one more when a window is
+    // attended: its partial is split nsplit - 1); row stride of `logits`.
+    int nsplit_run;
+    int64_t logits_ld;
+    // Full-precision residual window (optional): fp16 [streams][win_cap][d]
+    // keys and values, win_len[batch] tokens each.
+    const __half* kwin;
+    const __half* vwin;
+    int64_t win_cap;
+    const int32_t* win_len;
+    int win_dim;                      // d of the handle (selects the window kernel)
 };
+
+constexpr int kMaxWindow = 256;  // tokens of a residual window (KVQ_MAX_WINDOW)
+
+// Exact attention partial of the residual window of every (sequence, KV head).
+cudaError_t launch_decode_window(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s);
 
 // Bytes of workspace and number of splits for a decode of these sizes.
 void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, int* nsplit, int64_t* chunk,

@@ -269,6 +269,49 @@ int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int
                           const int32_t* seq_len, int64_t max_T, float scale, float* logits, float* out,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/* Most tokens a residual window may hold (kvq_decode_desc.window_cap). */
+#define KVQ_MAX_WINDOW 256
+
+/* Every argument of a decode call, for kvq_decode_attend_ex. */
+typedef struct kvq_decode_desc {
+    const void* q;                   /* as kvq_decode_attend */
+    int dtype;
+    int batch, hq, hkv;
+    const kvq_cache* k;
+    const kvq_cache* v;
+    const uint16_t* k_block_mean;    /* NSN caches (as kvq_nsn_decode_attend), or NULL */
+    const uint16_t* v_block_mean;
+    const uint16_t* k_window;        /* residual window, fp16 [batch * hkv][window_cap][d], or NULL */
+    const uint16_t* v_window;
+    int64_t window_cap;              /* 1..KVQ_MAX_WINDOW when a window is given */
+    const int32_t* window_len;       /* device, [batch]: tokens in each sequence's window */
+    const int32_t* seq_len;          /* device, [batch]: tokens in the packed cache */
+    int64_t max_T;
+    float scale;
+    float* logits;                   /* nullable; row (bi, head) at (bi * hq + head) * logits_ld */
+    int64_t logits_ld;               /* 0: max_T (+ window_cap with a window) */
+    float* out;
+    void* workspace;
+    size_t ws_bytes;
+} kvq_decode_desc;
+
+/*
+ * kvq_decode_attend_ex -- decode attention over a packed cache, optionally
+ * followed by a full-precision residual window (NSNQuant section 4: the newest
+ * tokens stay in fp16 until a block of them is flushed into the packed cache),
+ * for plain or NSN caches.  The softmax runs over the packed tokens [0,
+ * seq_len) then the window tokens [0, window_len) of each sequence; window
+ * keys and values are used exactly (fp32 arithmetic on the fp16 values).
+ * Window logits go to columns max_T + i of the logits rows.  Flushing a full
+ * window is kvq_quantize (or kvq_nsn_quantize) of its tokens into the packed
+ * arrays at offset seq_len (a multiple of 32; of 128 for NSN caches).
+ * The workspace size is kvq_decode_workspace's (it covers the window).
+ * Errors: as kvq_decode_attend and kvq_nsn_decode_attend; KVQ_EINVAL for a
+ * window without all its parts or with window_cap outside 1..KVQ_MAX_WINDOW,
+ * and for logits_ld too small.
+ */
+int kvq_decode_attend_ex(kvq_handle h, const kvq_decode_desc* desc, void* stream);
+
 /*
  * kvq_decode_attend_noalloc -- kvq_decode_attend without a caller-provided
  * workspace.  The pages have no counterpart of this call: it exists for

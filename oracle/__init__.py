@@ -364,6 +364,38 @@ def nsn_quantize(k: Constants, x, mean_in=None) -> dict:
     return dict(codes=codes, norm_x=nx, norm_w=nw, mean_half=mean_half, mean_f64=mean_f64, z=z)
 
 
+def window_decode_attend(k: Constants, q, kcache: dict, vcache: dict, kwin, vwin, scale: float,
+                         use_qjl: bool = True, nsn: tuple | None = None):
+    """Attention over a packed cache followed by a full-precision residual
+    window (NSNQuant section 4: the newest tokens stay unquantized until a
+    block is flushed).  The packed part is scored as in decode_attend (or
+    nsn_decode_attend when ``nsn`` = (kmean, vmean)); the window's keys and
+    values ([n_win, d], the stored fp16 values widened) are used exactly.
+    One softmax over all packed then window tokens.  Returns (logits over the
+    packed then window tokens [G, T + n_win], out [G, d])."""
+    q = _c(np.atleast_2d(q), np.float64)
+    G, d = q.shape
+    if nsn is None:
+        lp, _ = decode_attend(k, q, kcache, vcache, scale, use_qjl, want_logits=True)
+        T = lp.shape[1]
+        vh = (dequantize(k, vcache["codes"], vcache.get("bits"), vcache["norm"], vcache["gamma"], use_qjl)
+              if T > 0 else np.zeros((0, d)))
+    else:
+        lp, _ = nsn_decode_attend(k, q, kcache, vcache, nsn[0], nsn[1], scale, want_logits=True)
+        T = lp.shape[1]
+        vh = (nsn_dequantize(k, vcache["codes"], vcache["norm_x"], vcache["norm_w"], nsn[1])
+              if T > 0 else np.zeros((0, d)))
+    kw = np.asarray(kwin, np.float64).reshape(-1, d)
+    vw = np.asarray(vwin, np.float64).reshape(-1, d)
+    lw = scale * (q @ kw.T)
+    logits = np.concatenate([lp, lw], axis=1)
+    vals = np.concatenate([vh, vw], axis=0)
+    if logits.shape[1] == 0:
+        return logits, np.zeros((G, d))
+    e = np.exp(logits - logits.max(axis=1, keepdims=True))
+    return logits, (e @ vals) / e.sum(axis=1, keepdims=True)
+
+
 def nsn_dequantize(k: Constants, codes, norm_x, norm_w, mean_half) -> np.ndarray:
     """Vectors stored by the NSN front end, reconstructed from its byproducts
     (NSNQuant section 1: x = s1 (s2 v + o) with s1 = ||x||/sqrt(d), s2 v = w):

@@ -73,3 +73,63 @@ def test_empty_context_gives_zero_output():
                  gamma=np.zeros(0))
     _, o = oracle.decode_attend(k, np.ones((2, 64)), empty, empty, 1.0, True)
     assert (o == 0).all()
+
+
+# ---------------------------------------------------------------------------
+# packed cache + full-precision residual window
+# ---------------------------------------------------------------------------
+def _packed(k, X, qjl):
+    q = oracle.quantize(k, X, qjl)
+    st = dict(codes=q["codes"], norm=q["norm"].astype(np.float16).astype(np.float64),
+              gamma=q["gamma"].astype(np.float16).astype(np.float64))
+    if qjl:
+        st["bits"] = q["bits"]
+    return st
+
+
+def test_window_decode_empty_window_is_packed_decode():
+    d = 64
+    k = oracle.make_constants(d, 2, 2)
+    rng = np.random.default_rng(12)
+    kst, vst = _packed(k, rng.standard_normal((300, d)), True), _packed(k, rng.standard_normal((300, d)), True)
+    q = rng.standard_normal((2, d))
+    lr, orf = oracle.decode_attend(k, q, kst, vst, 0.2, True)
+    lw, ow = oracle.window_decode_attend(k, q, kst, vst, np.zeros((0, d)), np.zeros((0, d)), 0.2, True)
+    np.testing.assert_allclose(lw, lr, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(ow, orf, rtol=1e-12, atol=1e-13)
+
+
+def test_window_decode_only_window_is_exact_attention():
+    d = 32
+    k = oracle.make_constants(d, 1, 2)
+    rng = np.random.default_rng(13)
+    empty = dict(codes=np.zeros((0, d), np.int32), norm=np.zeros(0), gamma=np.zeros(0), bits=np.zeros((0, d)))
+    Kw, Vw = rng.standard_normal((50, d)), rng.standard_normal((50, d))
+    q = rng.standard_normal((3, d))
+    lw, ow = oracle.window_decode_attend(k, q, empty, empty, Kw, Vw, 0.5, True)
+    for g in range(3):
+        l = np.array([0.5 * q[g] @ Kw[t] for t in range(50)])
+        w = np.exp(l - l.max())
+        np.testing.assert_allclose(lw[g], l, rtol=1e-13)
+        np.testing.assert_allclose(ow[g], (w[:, None] * Vw).sum(0) / w.sum(), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("qjl", [True, False])
+def test_window_decode_is_attention_over_reconstructed_then_window_tokens(qjl):
+    """One softmax over the packed tokens (as reconstructed vectors, q . k_hat) followed by the
+    window tokens, written out directly."""
+    d, T, W = 64, 200, 37
+    k = oracle.make_constants(d, 2, 3)
+    rng = np.random.default_rng(14)
+    K, V = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    kst, vst = _packed(k, K, qjl), _packed(k, V, qjl)
+    Kh = oracle.dequantize(k, kst["codes"], kst.get("bits"), kst["norm"], kst["gamma"], qjl)
+    Vh = oracle.dequantize(k, vst["codes"], vst.get("bits"), vst["norm"], vst["gamma"], qjl)
+    Kw, Vw = rng.standard_normal((W, d)), rng.standard_normal((W, d))
+    q = rng.standard_normal((2, d))
+    lw, ow = oracle.window_decode_attend(k, q, kst, vst, Kw, Vw, 0.3, qjl)
+    Kall, Vall = np.vstack([Kh, Kw]), np.vstack([Vh, Vw])
+    l = 0.3 * q @ Kall.T
+    e = np.exp(l - l.max(1, keepdims=True))
+    np.testing.assert_allclose(lw, l, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(ow, (e @ Vall) / e.sum(1, keepdims=True), rtol=1e-10, atol=1e-11)
