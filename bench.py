@@ -359,11 +359,32 @@ def bench_decode(args, dist):
     cache_bytes = S * T * 2 * (h.b * d // 8 + d // 8 + 4)
     gbs = cache_bytes / (ms / steps / 1e3) / 1e9
     hbm, src = peaks()
+
+    # the same call with a 128-token fp16 residual window per (sequence, KV head)
+    W = 128
+    kw = wl.llama_keys(S, W, d, c["q_seed"] + 1, device="cuda").half()
+    vw = wl.llama_values(S, W, d, c["q_seed"] + 2, device="cuda").half()
+    wl_len = torch.full((B,), W, dtype=torch.int32, device="cuda")
+
+    def wstep(i):
+        kvq.kvq_decode_attend_ex(h, q, hkv, kcache, vcache, seq, T, c["scale"], out, ws, k_window=kw, v_window=vw,
+                                 window_len=wl_len, stream=stream)
+
+    for i in range(3):
+        wstep(i)
+    code, bits = kvq.kvq_status(h)
+    if code != 0:
+        raise RuntimeError(f"window decode status {code} bits {bits}")
+    ms_w = timed(dist, wstep, steps, stream)
     h.close()
     return {"metric": "packed-cache decode-attn GB/s", "value": round(dist.world * gbs, 1), "unit": "GB/s",
             "frac_of_hbm": round(gbs / hbm, 4), "ms_per_step": ms / steps, "steps": steps,
             "workload": f"batch 16, 32 query / 8 KV heads, d 128, {T}-token contexts, b=2 + QJL, one bf16 query token",
             "cache_bytes_per_step": cache_bytes, "launches_per_step": 3,
+            "with_window": {"window_tokens": W, "ms_per_step": ms_w / steps, "launches_per_step": 4,
+                            "bytes_per_step": int(cache_bytes + S * W * d * 2 * 2),
+                            "note": "kvq_decode_attend_ex: the packed cache plus a 128-token fp16 window per "
+                                    "(sequence, KV head), attended exactly"},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "frac_of_spec_8tbs": round(gbs / SPEC_HBM_GBS, 4),
                          "traffic": traffic_record("decode_split"),

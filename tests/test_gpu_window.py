@@ -157,3 +157,52 @@ def test_flush_append_cycle():
         _, orf = oracle.window_decode_attend(k, qd[0, s * G:(s + 1) * G], kst, vst, kwin[s, :n].double().cpu().numpy(),
                                              vwin[s, :n].double().cpu().numpy(), 1 / np.sqrt(d), True)
         assert_close(out[0, s * G:(s + 1) * G], orf, f"out kvh{s}")
+
+
+def test_window_over_nsn_cache_matches_oracle():
+    """An NSN cache (oracle-built) followed by a 128-token fp16 window: the window's value sum
+    enters the block-mean slot of its partial."""
+    from .test_gpu_nsn import _nsn_oracle_stream
+    d, b, hkv, hq, cap, T, W = 128, 2, 2, 8, 512, 384, 77
+    k = oracle.make_constants(d, b, 5)
+    G = hq // hkv
+    kc = torch.zeros((hkv, cap, b, d // 32), dtype=torch.int32)
+    vc = torch.zeros((hkv, cap // 32, b, d), dtype=torch.int32)
+    kn = torch.zeros((hkv, cap, 2), dtype=torch.float16)
+    vn = torch.zeros_like(kn)
+    km = torch.zeros((hkv, cap // 128, d), dtype=torch.float16)
+    vm = torch.zeros_like(km)
+    st = []
+    for s in range(hkv):
+        rk, nbk, sk = _nsn_oracle_stream(k, wl.nsn_tokens(1, cap, d, seed=1500 + s)[0].double().numpy())
+        rv, nbv, sv = _nsn_oracle_stream(k, wl.nsn_tokens(1, cap, d, seed=1600 + s)[0].double().numpy())
+        kc[s] = torch.from_numpy(oracle.pack_codes(rk["codes"], b).view(np.int32))
+        vc[s] = torch.from_numpy(oracle.pack_codes_block32(rv["codes"], b).view(np.int32).reshape(cap // 32, b, d))
+        kn[s], vn[s] = torch.from_numpy(nbk), torch.from_numpy(nbv)
+        km[s] = torch.from_numpy(rk["mean_half"].view(np.float16))
+        vm[s] = torch.from_numpy(rv["mean_half"].view(np.float16))
+        st.append((sk, sv, rk["mean_half"], rv["mean_half"]))
+    kw = wl.nsn_tokens(hkv, 128, d, seed=1700).to(torch.float16)
+    vw = wl.nsn_tokens(hkv, 128, d, seed=1701).to(torch.float16)
+    q = wl.queries(1, hq, d, seed=81)
+    with kvq.Handle(d, b, 5, qjl=False) as h:
+        out = torch.empty((1, hq, d), dtype=torch.float32, device="cuda")
+        ws = torch.empty(kvq.kvq_decode_workspace(h, 1, hq, hkv, cap), dtype=torch.uint8, device="cuda")
+        kcd, vcd, knd, vnd, kmd, vmd = (t.cuda() for t in (kc, vc, kn, vn, km, vm))
+        kvq.kvq_decode_attend_ex(h, q.cuda(), hkv, kvq.make_cache(kcd, None, knd, cap, 0),
+                                 kvq.make_cache(vcd, None, vnd, cap, 1),
+                                 torch.tensor([T], dtype=torch.int32, device="cuda"), cap, d ** -0.5, out, ws,
+                                 k_window=kw.cuda(), v_window=vw.cuda(),
+                                 window_len=torch.tensor([W], dtype=torch.int32, device="cuda"),
+                                 k_block_mean=kmd, v_block_mean=vmd)
+        assert kvq.kvq_status(h)[0] == 0
+        out = out.cpu().numpy()
+    qd = q.double().numpy()
+    for s in range(hkv):
+        sk, sv, mk, mv = st[s]
+        sk = {key: v[:T] for key, v in sk.items()}
+        sv = {key: v[:T] for key, v in sv.items()}
+        _, orf = oracle.window_decode_attend(k, qd[0, s * G:(s + 1) * G], sk, sv, kw[s, :W].double().numpy(),
+                                             vw[s, :W].double().numpy(), d ** -0.5, False,
+                                             nsn=(mk[:T // 128], mv[:T // 128]))
+        assert_close(out[0, s * G:(s + 1) * G], orf, f"nsn + window out kvh{s}")
