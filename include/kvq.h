@@ -2,12 +2,15 @@
  * kvq.h -- C ABI of the B200 (sm_100a) rotated-token KV-cache quantizer.
  *
  * The method (TurboQuant form, calibration free):
- *   quantize  x -> ||x||, z = H (delta .* x) / ||x||, b-bit Gaussian Lloyd-Max
- *             codes of z, residual r = z - c[code], 1-bit QJL sketch
- *             sign(S r), fp16 norms (||x||, ||r||);
+ *   quantize  x -> ||x||, z = H (delta .* x) / ||x||, b-bit Lloyd-Max codes
+ *             of z (for N(0,1), or for the exact Beta law of a rotated unit
+ *             coordinate with KVQ_BETA_CODEBOOK), residual r = z - c[code],
+ *             1-bit QJL sketch sign(S r), fp16 norms (||x||, ||r||);
+ *             optionally behind the NSN front end (kvq_nsn_quantize);
  *   decode    rotate each query once, logits straight from the packed codes
  *             plus the QJL correction, softmax, weighted sum of the decoded
- *             values, all over the packed cache.
+ *             values, all over the packed cache (plain or NSN), optionally
+ *             followed by an fp16 residual window of the newest tokens.
  * Sources: "O Que E TurboQuant?" (TurboQuant blog), sections "Estagio 1:
  * Rotacao Aleatoria + Compressao PolarQuant", "Estagio 2: Correcao Residual
  * QJL" and "Como Implementar"; "PolarQuant: Optimal Gaussian Weight
@@ -208,7 +211,9 @@ typedef struct kvq_cache {
     int32_t layout;         /* KVQ_LAYOUT_TOKEN (keys) or KVQ_LAYOUT_BLOCK32 (values) */
 } kvq_cache;
 
-/* Bytes of device workspace kvq_decode_attend needs for these sizes. */
+/* Bytes of device workspace a decode call (kvq_decode_attend,
+ * kvq_nsn_decode_attend, kvq_decode_attend_ex with or without a residual
+ * window) needs for these sizes; computed on the host, no device work. */
 size_t kvq_decode_workspace(kvq_handle h, int batch, int hq, int hkv, int64_t max_T);
 
 /*
