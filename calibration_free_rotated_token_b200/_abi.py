@@ -35,7 +35,7 @@ STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
 EXPORTED = (
     "kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize", "kvq_decode_workspace",
     "kvq_decode_attend", "kvq_decode_attend_noalloc", "kvq_status", "kvq_last_error", "kvq_get_constants",
-    "kvq_get_info", "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex",
+    "kvq_get_info", "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex", "kvq_probe_wait_timeout",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -102,12 +102,13 @@ def load() -> ctypes.CDLL:
         L.kvq_get_info.argtypes = [P, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(U32)]
         L.kvq_codebook.argtypes = [I, I, U32, P, P]
         L.kvq_decode_attend_ex.argtypes = [P, ctypes.POINTER(KvqDecodeDesc), P]
+        L.kvq_probe_wait_timeout.argtypes = [P, U32, P]
         L.kvq_nsn_decode_attend.argtypes = [P, P, I, I, I, I, ctypes.POINTER(KvqCache), ctypes.POINTER(KvqCache),
                                             P, P, P, I64, ctypes.c_float, P, P, P, SZ, P]
         for name in ("kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize",
                      "kvq_decode_attend",
                      "kvq_decode_attend_noalloc", "kvq_status", "kvq_get_constants", "kvq_get_info",
-                     "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex"):
+                     "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex", "kvq_probe_wait_timeout"):
             getattr(L, name).restype = I
         _lib = L
         return L
@@ -390,6 +391,11 @@ def kvq_status(h: Handle, stream=None) -> tuple[int, int]:
     bits = ctypes.c_uint32()
     code = load().kvq_status(h.ptr, _stream(stream), ctypes.byref(bits))
     return code, bits.value
+
+
+def kvq_probe_wait_timeout(h: Handle, polls: int = 4096, stream=None):
+    """One kernel whose bounded mbarrier wait runs out; kvq_status then reports KVQ_ETIMEOUT."""
+    _check(load().kvq_probe_wait_timeout(h.ptr, polls, _stream(stream)))
 
 
 def kvq_last_error() -> str:

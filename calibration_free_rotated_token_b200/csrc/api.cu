@@ -693,6 +693,15 @@ int kvq_decode_attend_noalloc(kvq_handle h, const void* q, int dtype, int batch,
                          stream);
 }
 
+int kvq_probe_wait_timeout(kvq_handle h, uint32_t polls, void* stream) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    if (polls == 0 || polls > (1u << 20)) return fail(KVQ_EINVAL, "polls must be in 1..2^20");
+    const cudaError_t e = kvq::launch_wait_timeout_probe(h->d_status, polls, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "wait-timeout probe launch");
+    return KVQ_OK;
+}
+
 int kvq_status(kvq_handle h, void* stream, uint32_t* bits) {
     g_err.clear();
     if (int e = check_handle(h)) return e;

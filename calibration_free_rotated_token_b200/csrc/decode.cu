@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "kvq_internal.h"
+#include "sm100.cuh"
 
 namespace kvq {
 
@@ -652,6 +653,23 @@ cudaError_t launch_decode_window(const kvq_ctx*, const DecodeArgs& a, cudaStream
         case 128: return window_d<128>(a, s);
         default: return window_d<256>(a, s);
     }
+}
+
+// The bounded-wait path on its own: one thread waits on an mbarrier that no
+// one arrives on, for `polls` polls, then records the timeout in the status
+// word and returns (the same helper every kernel's waits use).
+__global__ void wait_timeout_probe_kernel(uint32_t* status, uint32_t polls) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_wait_n(&bar, 0u, status, polls);
+    }
+}
+
+cudaError_t launch_wait_timeout_probe(uint32_t* status, uint32_t polls, cudaStream_t s) {
+    wait_timeout_probe_kernel<<<1, 32, 0, s>>>(status, polls);
+    return cudaGetLastError();
 }
 
 }  // namespace kvq

@@ -118,6 +118,9 @@ struct DecodeArgs {
 
 constexpr int kMaxWindow = 256;  // tokens of a residual window (KVQ_MAX_WINDOW)
 
+// One bounded mbarrier wait that cannot complete (a test of the timeout path).
+cudaError_t launch_wait_timeout_probe(uint32_t* status, uint32_t polls, cudaStream_t s);
+
 // Exact attention partial of the residual window of every (sequence, KV head).
 cudaError_t launch_decode_window(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s);
 

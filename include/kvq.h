@@ -346,6 +346,16 @@ int kvq_decode_attend_noalloc(kvq_handle h, const void* q, int dtype, int batch,
                               float scale, float* logits, float* out, void* stream);
 
 /*
+ * kvq_probe_wait_timeout -- launch one CTA whose mbarrier wait cannot
+ * complete (nothing arrives on it), bounded by `polls` polls (1..2^20), with
+ * the same bounded-wait helper every kernel uses.  When the bound runs out
+ * the kernel sets KVQ_STATUS_TIMEOUT in the handle's status word and returns,
+ * so the next kvq_status reports KVQ_ETIMEOUT and the context stays usable.
+ * It exercises the failure path without a fault.  Asynchronous on `stream`.
+ */
+int kvq_probe_wait_timeout(kvq_handle h, uint32_t polls, void* stream);
+
+/*
  * kvq_status -- synchronise `stream`, read and clear the handle's device
  * status word.  Returns KVQ_OK, KVQ_ENONFINITE or KVQ_ETIMEOUT (the most
  * severe condition seen); *bits (nullable, host) receives the raw

@@ -302,3 +302,19 @@ def test_quantize_beta_codebook_matches_oracle(d, b, qjl, dtype, n):
         codes, qj, norms = run_quantize(h, x.cuda())
     compare_quantize(k, x.double().numpy(), to_np_u32(codes), to_np_u32(qj) if qjl else None,
                      to_np_f16bits(norms), qjl)
+
+
+
+def test_bounded_wait_runs_out_and_the_context_stays_usable():
+    """A wait on an mbarrier nothing arrives on gives up after its poll bound: the status word
+    reports the timeout (read on the host), and the next launches run normally."""
+    with kvq.Handle(128, 2, 1, qjl=True) as h:
+        kvq.kvq_probe_wait_timeout(h, 4096)
+        code, bits = kvq.kvq_status(h)
+        assert code == kvq.KVQ_ETIMEOUT and bits & kvq.STATUS_TIMEOUT
+        x = wl.sweep_tokens(300, 128, seed=11)
+        codes, qj, norms = run_quantize(h, x.cuda())
+        compare_quantize(constants(128, 2, 1), x.double().numpy(), to_np_u32(codes), to_np_u32(qj),
+                         to_np_f16bits(norms), True)
+        with pytest.raises(kvq.KvqError):
+            kvq.kvq_probe_wait_timeout(h, 0)
