@@ -333,82 +333,85 @@ __device__ __forceinline__ float load_any(const void* p, int dt, int64_t i) {
     return dt == 1 ? __half2float(__ushort_as_half(u)) : __uint_as_float(static_cast<uint32_t>(u) << 16);
 }
 
-// The full-precision residual window of one (sequence, KV head) as one more
+// The full-precision residual window of one (sequence, query head) as one more
 // split partial (NSNQuant section 4: the newest tokens stay unquantized until
 // a block is flushed): exact fp32 logits of its fp16 keys, its own max M and
 // sum L, and y = sum_t e_t v_t.  Stored so that the combine's arithmetic
 // gives y back: A = H (delta .* y) (delta .* H A / d = y), or for NSN caches
 // the block-mean slot O = y.  An empty window leaves M = -inf, L = 0.
-template <int D, int G, bool NSN>
+template <int D, bool NSN>
 __global__ void __launch_bounds__(kDecThreads) decode_window_kernel(const __grid_constant__ DecodeArgs a) {
+    // G = hq / hkv query heads (CTAs) read the same KV head's window
     constexpr int PART = 2 + 2 * D;
-    __shared__ float sq[G][D];
-    __shared__ float sl[G][kMaxWindow];
+    __shared__ float sq[D];
+    __shared__ float sl[kMaxWindow];
     __shared__ float sy[D];
-    __shared__ float smx[G], ssum[G];
+    __shared__ float sred[kDecThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t stream = blockIdx.x;
-    const int bi = static_cast<int>(stream / a.hkv), hk = static_cast<int>(stream % a.hkv);
-    const int64_t qh0 = static_cast<int64_t>(bi) * a.hq + static_cast<int64_t>(hk) * G;
+    const int64_t qh = blockIdx.x;  // bi * hq + head
+    const int bi = static_cast<int>(qh / a.hq);
+    const int hk = static_cast<int>((qh % a.hq) / a.G);
+    const int64_t stream = static_cast<int64_t>(bi) * a.hkv + hk;
     const int n = static_cast<int>(min(max(static_cast<int64_t>(a.win_len[bi]), int64_t(0)), a.win_cap));
     const __half* kw = a.kwin + stream * a.win_cap * D;
     const __half* vw = a.vwin + stream * a.win_cap * D;
-    for (int e = tid; e < G * D; e += blockDim.x) sq[e / D][e % D] = load_any(a.q, a.qdtype, qh0 * D + e);
+    for (int j = tid; j < D; j += blockDim.x) sq[j] = load_any(a.q, a.qdtype, qh * D + j);
     __syncthreads();
-    // logits, one (token, head) per thread
-    for (int e = tid; e < n * G; e += blockDim.x) {
-        const int t = e / G, h = e % G;
-        const __half2* kr = reinterpret_cast<const __half2*>(kw + static_cast<int64_t>(t) * D);
+    // logits, one token per thread (the key row in 16-byte loads)
+    float mx = -INFINITY;
+    for (int t = tid; t < n; t += blockDim.x) {
+        const uint4* kr = reinterpret_cast<const uint4*>(kw + static_cast<int64_t>(t) * D);
         float acc = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < D / 2; ++j) {
-            const float2 kv = __half22float2(kr[j]);
-            acc = fmaf(kv.y, sq[h][2 * j + 1], fmaf(kv.x, sq[h][2 * j], acc));
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 w = kr[c];
+            const __half2* hw = reinterpret_cast<const __half2*>(&w);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 kv = __half22float2(hw[k]);
+                acc = fmaf(kv.y, sq[8 * c + 2 * k + 1], fmaf(kv.x, sq[8 * c + 2 * k], acc));
+            }
         }
         const float l = a.scale * acc;
-        sl[h][t] = l;
-        if (a.logits != nullptr) a.logits[(qh0 + h) * a.logits_ld + a.max_T + t] = l;
+        sl[t] = l;
+        mx = fmaxf(mx, l);
+        if (a.logits != nullptr) a.logits[qh * a.logits_ld + a.max_T + t] = l;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (lane == 0) sred[warp] = mx;
+    __syncthreads();
+    mx = sred[0];
+    for (int w = 1; w < kDecThreads / 32; ++w) mx = fmaxf(mx, sred[w]);
+    float sum = 0.f;
+    for (int t = tid; t < n; t += blockDim.x) {
+        const float e = __expf(sl[t] - mx);
+        sl[t] = e;
+        sum += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    __syncthreads();  // every thread has read sred (the max)
+    if (lane == 0) sred[warp] = sum;
+    __syncthreads();
+    float L = 0.f;
+    for (int w = 0; w < kDecThreads / 32; ++w) L += sred[w];
+    // y = sum_t e_t v_t, one coordinate per thread (coalesced rows of V)
+    for (int j = tid; j < D; j += blockDim.x) {
+        float acc = 0.f;
+        for (int t = 0; t < n; ++t) acc = fmaf(sl[t], __half2float(vw[static_cast<int64_t>(t) * D + j]), acc);
+        sy[j] = NSN ? acc : sign_of(a.pair_sign, j) * acc;
     }
     __syncthreads();
-    // per head (one warp each): max, weights e = exp(l - max), their sum
-    for (int h = warp; h < G; h += blockDim.x / 32) {
-        float m = -INFINITY;
-        for (int t = lane; t < n; t += 32) m = fmaxf(m, sl[h][t]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        float sum = 0.f;
-        for (int t = lane; t < n; t += 32) {
-            const float e = __expf(sl[h][t] - m);
-            sl[h][t] = e;
-            sum += e;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        if (lane == 0) {
-            smx[h] = m;
-            ssum[h] = sum;
-        }
+    if (!NSN) fwht_smem<D>(sy);  // A = H (delta .* y)
+    float* pp = a.part + (qh * a.nsplit + (a.nsplit - 1)) * PART;
+    for (int j = tid; j < D; j += blockDim.x) {
+        pp[2 + j] = NSN ? 0.f : sy[j];
+        pp[2 + D + j] = NSN ? sy[j] : 0.f;
     }
-    __syncthreads();
-    for (int h = 0; h < G; ++h) {
-        float* pp = a.part + ((qh0 + h) * a.nsplit + (a.nsplit - 1)) * PART;
-        // y = sum_t e_t v_t, one coordinate per thread (coalesced rows of V)
-        for (int j = tid; j < D; j += blockDim.x) {
-            float acc = 0.f;
-            for (int t = 0; t < n; ++t) acc = fmaf(sl[h][t], __half2float(vw[static_cast<int64_t>(t) * D + j]), acc);
-            sy[j] = NSN ? acc : sign_of(a.pair_sign, j) * acc;
-        }
-        __syncthreads();
-        if (!NSN) fwht_smem<D>(sy);  // A = H (delta .* y)
-        for (int j = tid; j < D; j += blockDim.x) {
-            pp[2 + j] = NSN ? 0.f : sy[j];
-            pp[2 + D + j] = NSN ? sy[j] : 0.f;
-        }
-        if (tid == 0) {
-            pp[0] = n > 0 ? smx[h] : -INFINITY;
-            pp[1] = n > 0 ? ssum[h] : 0.f;
-        }
-        __syncthreads();
+    if (tid == 0) {
+        pp[0] = n > 0 ? mx : -INFINITY;
+        pp[1] = n > 0 ? L : 0.f;
     }
 }
 
@@ -628,21 +631,12 @@ cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s,
 }
 
 namespace {
-template <int D, int G>
-cudaError_t window_g(const DecodeArgs& a, cudaStream_t s) {
-    const unsigned n = static_cast<unsigned>(a.batch * a.hkv);
-    if (a.nsn) decode_window_kernel<D, G, true><<<n, kDecThreads, 0, s>>>(a);
-    else decode_window_kernel<D, G, false><<<n, kDecThreads, 0, s>>>(a);
-    return cudaGetLastError();
-}
 template <int D>
 cudaError_t window_d(const DecodeArgs& a, cudaStream_t s) {
-    switch (a.G) {
-        case 1: return window_g<D, 1>(a, s);
-        case 2: return window_g<D, 2>(a, s);
-        case 4: return window_g<D, 4>(a, s);
-        default: return window_g<D, 8>(a, s);
-    }
+    const unsigned n = static_cast<unsigned>(a.batch * a.hq);
+    if (a.nsn) decode_window_kernel<D, true><<<n, kDecThreads, 0, s>>>(a);
+    else decode_window_kernel<D, false><<<n, kDecThreads, 0, s>>>(a);
+    return cudaGetLastError();
 }
 }  // namespace
 

@@ -121,7 +121,7 @@ constexpr int kMaxWindow = 256;  // tokens of a residual window (KVQ_MAX_WINDOW)
 // One bounded mbarrier wait that cannot complete (a test of the timeout path).
 cudaError_t launch_wait_timeout_probe(uint32_t* status, uint32_t polls, cudaStream_t s);
 
-// Exact attention partial of the residual window of every (sequence, KV head).
+// Exact attention partial of the residual window for every (sequence, query head).
 cudaError_t launch_decode_window(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s);
 
 // Bytes of workspace and number of splits for a decode of these sizes.
