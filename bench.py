@@ -524,7 +524,8 @@ def bench_sweep(args, dist):
                              "quantize_kernel": "quantize_tc_kernel" if d <= 128 else "quantize_kernel",
                              "decode_us": round(ms_d / steps * 1e3, 2), "decode_gbs": round(d_gbs, 1),
                              "decode_frac": round(d_gbs / hbm, 4),
-                             "decode_kernel": "decode_mma_kernel" if b <= 2 else "decode_split_kernel"})
+                             "decode_kernel": ("decode_mma_kernel" if b <= 2 or (b == 3 and d <= 128)
+                                               else "decode_split_kernel")})
                 h.close()
                 del outK, outV, kcache, vcache, ws
         del X

@@ -157,11 +157,51 @@ __device__ __forceinline__ void mma_u8u8(int (&d)[4], const uint32_t (&a)[4], ui
 // column g = (head (g >> 1) + 4 (nt >> 1), digit (g & 1) + 2 (nt & 1)); K
 // index 4t + i is coordinate 32w + t + 8i with factor 2^(7 - t), K index
 // 16 + 4t + i is coordinate 32w + t + 4 + 8i with factor 2^(3 - t).
+// Plane form of a symmetric codebook of 2^B levels (B <= 3):
+//   c[code] = cst + sum_v coef[v] plane_v(code),
+// plane_v = bit v of the code for v < B, and for B = 3 a fourth plane
+// bit0 ^ bit1 ^ bit2.  In +-1 variables s_p = 2 bit_p - 1 a codebook with
+// c[~k] = -c[k] is an odd function, so its multilinear form has only the odd
+// terms: sum_p a_p s_p (B <= 2: exactly the planes), plus a_3 s0 s1 s2 for
+// B = 3, and s0 s1 s2 = 2 (bit0 ^ bit1 ^ bit2) - 1.
+template <int B>
+struct PlaneCoefs {
+    static constexpr int PV = (B == 3) ? 4 : B;  // code planes, the parity plane included
+    float cst;
+    float coef[PV];
+};
+template <int B>
+__device__ __forceinline__ PlaneCoefs<B> plane_coefs(const float* c) {
+    PlaneCoefs<B> r;
+    if constexpr (B <= 2) {
+        r.cst = c[0];
+        r.coef[0] = c[1] - c[0];
+        if constexpr (B == 2) r.coef[1] = c[2] - c[0];
+    } else {
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float s0 = (k & 1) ? 1.f : -1.f, s1 = (k & 2) ? 1.f : -1.f, s2 = (k & 4) ? 1.f : -1.f;
+            a0 = fmaf(c[k], s0, a0);
+            a1 = fmaf(c[k], s1, a1);
+            a2 = fmaf(c[k], s2, a2);
+            a3 = fmaf(c[k], s0 * s1 * s2, a3);
+        }
+        r.cst = -0.125f * (a0 + a1 + a2 + a3);
+        r.coef[0] = 0.25f * a0;
+        r.coef[1] = 0.25f * a1;
+        r.coef[2] = 0.25f * a2;
+        r.coef[3] = 0.25f * a3;
+    }
+    return r;
+}
+
 template <int D, int B, bool QJL, int G, int DT>
 __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int M = D;
     constexpr int NTK = HeadCfg<G>::NTK;
-    constexpr int KS = (B + (QJL ? 1 : 0)) * (D / 32);
+    constexpr int PV = PlaneCoefs<B>::PV;
+    constexpr int KS = (PV + (QJL ? 1 : 0)) * (D / 32);
     __shared__ float sq[G][D];
     __shared__ float sp[G][QJL ? M : 1];
     __shared__ float ssig[G][2];
@@ -214,11 +254,12 @@ __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__
         }
         __syncthreads();
     }
-    // plane coefficients: c[code] = c0 + coef0 bit0 (+ coef1 bit1)
-    const float c0 = a.centroid[0];
-    const float coef0 = a.centroid[1] - c0;
-    const float coef1 = (B == 2) ? a.centroid[2] - c0 : 0.f;
-    const float cmax = fmaxf(fabsf(coef0), fabsf(coef1));
+    // plane coefficients: c[code] = cst + sum_v coef[v] plane_v
+    const PlaneCoefs<B> pc = plane_coefs<B>(a.centroid);
+    const float c0 = pc.cst;
+    float cmax = 0.f;
+#pragma unroll
+    for (int v = 0; v < PV; ++v) cmax = fmaxf(cmax, fabsf(pc.coef[v]));
     for (int h = tid / 32; h < G; h += kThreads / 32) {
         const int ln = tid % 32;
         float mq = 0.f, mp = 0.f, s_q = 0.f, s_p = 0.f;
@@ -258,8 +299,10 @@ __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__
         uint32_t b[2] = {0u, 0u};
         if (h < G) {
             const int plane = ks / (D / 32), w = ks % (D / 32);
-            const bool is_q = plane >= B;
-            const float coef = (plane == 0) ? coef0 : coef1;
+            const bool is_q = plane >= PV;
+            float coef = 0.f;
+#pragma unroll
+            for (int v = 0; v < PV; ++v) coef = (plane == v) ? pc.coef[v] : coef;
             const float sig = is_q ? ssig[h][1] : ssig[h][0];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -290,7 +333,7 @@ struct MmaSmem {
     static constexpr int NTK = HeadCfg<G>::NTK;
     static constexpr int RT = HeadCfg<G>::RT;
     static constexpr int GP = HeadCfg<G>::GP;
-    static constexpr int KS = (B + (QJL ? 1 : 0)) * (D / 32);
+    static constexpr int KS = (PlaneCoefs<B>::PV + (QJL ? 1 : 0)) * (D / 32);
     // staging of one sub-chunk
     static constexpr int kKc = TC * B * D / 8;             // key codes (token layout)
     static constexpr int kKq = QJL ? TC * M / 8 : 0;       // key sign bits
@@ -316,9 +359,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     using HC = HeadCfg<G>;
     constexpr int M = D, TC = L::TC, NTK = L::NTK, RT = L::RT, KS = L::KS, GP = L::GP, CPL = HC::CPL;
     constexpr int KWT = B * D / 32;           // code words per token (key layout)
+    constexpr int PV = PlaneCoefs<B>::PV;     // code planes incl. the parity plane (B = 3)
+    constexpr int KWV = PV * D / 32;          // code-plane words per token, the parity plane included
     constexpr int QWT = QJL ? M / 32 : 0;     // sign words per token
     constexpr int NTV = D / 32;               // value n-tiles per warp (D/4 coordinates / 8)
-    constexpr int NPV = B + (QJL ? 1 : 0);
+    constexpr int NPV = PV + (QJL ? 1 : 0);
     constexpr bool QF_REG = L::kQfReg;
     constexpr int HH = (G == 8) ? 2 : 1;      // query heads per lane in the logit epilogue
     extern __shared__ __align__(128) uint8_t smem[];
@@ -338,8 +383,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
     const uint32_t msk_lo = kLowBits << t, msk_hi = kLowBits << (t + 4);
     const float kappa = kSqrtHalfPi / M;
-    const float coef0 = a.centroid[1] - a.centroid[0];
-    const float coef1 = (B == 2) ? a.centroid[2] - a.centroid[0] : 0.f;
+    const PlaneCoefs<B> pc = plane_coefs<B>(a.centroid);
 
     for (int e = tid; e < 2 * L::kWfrag / 4; e += kThreads) swc[e] = 0u;  // padding rows stay zero
     if (tid == 0) {
@@ -514,34 +558,47 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                 int accc[2][NTK][4], accq[NTK][4];  // code K-steps alternate between two chains
                 if (mt * 16 < nval) {
                     uint32_t w0[KS], w1[KS];
+                    if constexpr (KWT % 4 == 0) {  // token records of 16-byte multiples
 #pragma unroll
-                    for (int q4 = 0; q4 < KWT / 4; ++q4) {
-                        const uint4 x0 = reinterpret_cast<const uint4*>(sKc + tl0 * KWT)[q4];
-                        const uint4 x1 = reinterpret_cast<const uint4*>(sKc + tl1 * KWT)[q4];
-                        w0[4 * q4] = x0.x; w0[4 * q4 + 1] = x0.y; w0[4 * q4 + 2] = x0.z; w0[4 * q4 + 3] = x0.w;
-                        w1[4 * q4] = x1.x; w1[4 * q4 + 1] = x1.y; w1[4 * q4 + 2] = x1.z; w1[4 * q4 + 3] = x1.w;
+                        for (int q4 = 0; q4 < KWT / 4; ++q4) {
+                            const uint4 x0 = reinterpret_cast<const uint4*>(sKc + tl0 * KWT)[q4];
+                            const uint4 x1 = reinterpret_cast<const uint4*>(sKc + tl1 * KWT)[q4];
+                            w0[4 * q4] = x0.x; w0[4 * q4 + 1] = x0.y; w0[4 * q4 + 2] = x0.z; w0[4 * q4 + 3] = x0.w;
+                            w1[4 * q4] = x1.x; w1[4 * q4 + 1] = x1.y; w1[4 * q4 + 2] = x1.z; w1[4 * q4 + 3] = x1.w;
+                        }
+                    } else {  // 8-byte multiples (d = 64 with 1 or 3 bits)
+#pragma unroll
+                        for (int q2 = 0; q2 < KWT / 2; ++q2) {
+                            const uint2 x0 = reinterpret_cast<const uint2*>(sKc + tl0 * KWT)[q2];
+                            const uint2 x1 = reinterpret_cast<const uint2*>(sKc + tl1 * KWT)[q2];
+                            w0[2 * q2] = x0.x; w0[2 * q2 + 1] = x0.y;
+                            w1[2 * q2] = x1.x; w1[2 * q2 + 1] = x1.y;
+                        }
                     }
+                    if constexpr (PV > B) {
+                        // the parity plane: bit0 ^ bit1 ^ bit2 of every coordinate
 #pragma unroll
-                    for (int k = KWT / 4 * 4; k < KWT; ++k) {
-                        w0[k] = sKc[tl0 * KWT + k];
-                        w1[k] = sKc[tl1 * KWT + k];
+                        for (int w = 0; w < D / 32; ++w) {
+                            w0[KWT + w] = w0[w] ^ w0[D / 32 + w] ^ w0[2 * (D / 32) + w];
+                            w1[KWT + w] = w1[w] ^ w1[D / 32 + w] ^ w1[2 * (D / 32) + w];
+                        }
                     }
                     if (QJL) {
 #pragma unroll
                         for (int k = 0; k < QWT; k += 2) {
                             const uint2 x0 = reinterpret_cast<const uint2*>(sKq + tl0 * QWT)[k / 2];
                             const uint2 x1 = reinterpret_cast<const uint2*>(sKq + tl1 * QWT)[k / 2];
-                            w0[KWT + k] = x0.x; w0[KWT + k + 1] = x0.y;
-                            w1[KWT + k] = x1.x; w1[KWT + k + 1] = x1.y;
+                            w0[KWV + k] = x0.x; w0[KWV + k + 1] = x0.y;
+                            w1[KWV + k] = x1.x; w1[KWV + k + 1] = x1.y;
                         }
                     }
                     // code and QJL K-steps interleaved: 2 NTK independent accumulators
 #pragma unroll
-                    for (int i = 0; i < KWT || i < QWT; ++i) {
+                    for (int i = 0; i < KWV || i < QWT; ++i) {
 #pragma unroll
                         for (int kind = 0; kind < 2; ++kind) {
-                            if (kind == 0 ? (i >= KWT) : (i >= QWT)) continue;
-                            const int ks = kind == 0 ? i : KWT + i;
+                            if (kind == 0 ? (i >= KWV) : (i >= QWT)) continue;
+                            const int ks = kind == 0 ? i : KWV + i;
                             const uint4 af = make_uint4(w0[ks] & msk_lo, w1[ks] & msk_lo, w0[ks] & msk_hi,
                                                         w1[ks] & msk_hi);
 #pragma unroll
@@ -558,7 +615,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                             }
                         }
                     }
-                    if (KWT < 2) {
+                    if (KWV < 2) {
 #pragma unroll
                         for (int nt = 0; nt < NTK; ++nt)
 #pragma unroll
@@ -750,21 +807,32 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                         aw[rt] = reinterpret_cast<const uint4*>(swc)[(bb * RT + rt) * 32 + lane];
                         if (QJL) aq[rt] = reinterpret_cast<const uint4*>(swq)[(bb * RT + rt) * 32 + lane];
                     }
+                    uint32_t wr[3][NTV];  // real planes' words, for the parity plane (B = 3)
 #pragma unroll
                     for (int p = 0; p < NPV; ++p) {
-                        const uint32_t* src = (p < B) ? sVc + (bb * B + p) * D + cbase : sVq + bb * M + cbase;
                         uint32_t wv[NTV];
-                        if (NTV % 4 == 0) {
+                        if (PV > B && p == B) {
 #pragma unroll
-                            for (int q4 = 0; q4 < NTV / 4; ++q4) {
-                                const uint4 x = reinterpret_cast<const uint4*>(src)[q4];
-                                wv[4 * q4] = x.x; wv[4 * q4 + 1] = x.y; wv[4 * q4 + 2] = x.z; wv[4 * q4 + 3] = x.w;
-                            }
+                            for (int nt = 0; nt < NTV; ++nt) wv[nt] = wr[0][nt] ^ wr[1][nt] ^ wr[2][nt];
                         } else {
+                            const uint32_t* src = (p < B) ? sVc + (bb * B + p) * D + cbase : sVq + bb * M + cbase;
+                            if (NTV % 4 == 0) {
 #pragma unroll
-                            for (int q2 = 0; q2 < NTV / 2; ++q2) {
-                                const uint2 x = reinterpret_cast<const uint2*>(src)[q2];
-                                wv[2 * q2] = x.x; wv[2 * q2 + 1] = x.y;
+                                for (int q4 = 0; q4 < NTV / 4; ++q4) {
+                                    const uint4 x = reinterpret_cast<const uint4*>(src)[q4];
+                                    wv[4 * q4] = x.x; wv[4 * q4 + 1] = x.y; wv[4 * q4 + 2] = x.z;
+                                    wv[4 * q4 + 3] = x.w;
+                                }
+                            } else {
+#pragma unroll
+                                for (int q2 = 0; q2 < NTV / 2; ++q2) {
+                                    const uint2 x = reinterpret_cast<const uint2*>(src)[q2];
+                                    wv[2 * q2] = x.x; wv[2 * q2 + 1] = x.y;
+                                }
+                            }
+                            if (PV > B && p < B) {
+#pragma unroll
+                                for (int nt = 0; nt < NTV; ++nt) wr[p < 3 ? p : 0][nt] = wv[nt];
                             }
                         }
 #pragma unroll
@@ -772,7 +840,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                             const uint2 bv = make_uint2(wv[nt] & msk_lo, wv[nt] & msk_hi);
 #pragma unroll
                             for (int rt = 0; rt < RT; ++rt) {
-                                const uint4 af = (p < B) ? aw[rt] : aq[(QJL ? rt : 0)];
+                                const uint4 af = (p < PV) ? aw[rt] : aq[(QJL ? rt : 0)];
                                 if (first) mma_u8u8_qz(accv[p][nt][rt], af, bv);
                                 else mma_u8u8_q(accv[p][nt][rt], af, bv);
                             }
@@ -831,8 +899,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                                            fmaf(static_cast<float>(d2), 65536.f, static_cast<float>(d1 * 256u + d0)));
                         }
                         if (head < G) {
-                            float code = coef0 * vals[0];
-                            if (B == 2) code = fmaf(coef1, vals[1 % NPV], code);
+                            float code = pc.coef[0] * vals[0];
+#pragma unroll
+                            for (int v = 1; v < PV; ++v) code = fmaf(pc.coef[v], vals[v], code);
                             accA[nt][c] = fmaf(accA[nt][c], alpha, sgw * code);
                             if (QJL) accB[nt][c] = fmaf(accB[nt][c], alpha, sgq * 2.f * vals[NPV - 1]);
                             if (NSN) {
@@ -909,7 +978,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             if (head < G) {
                 float* pp = a.part + ((qh0 + head) * a.nsplit + split) * PART;
                 const float* hs = shead + head * 8;
-                const float c0 = a.centroid[0];
+                const float c0 = pc.cst;
 #pragma unroll
                 for (int nt = 0; nt < NTV; ++nt)
 #pragma unroll
@@ -1014,6 +1083,10 @@ cudaError_t launch_mma_d(const DecodeArgs& a, int grid, cudaStream_t s) {
         case 256 * 16 + 4: return FN<256, 1, false>(__VA_ARGS__);           \
         case 256 * 16 + 5: return FN<256, 1, true>(__VA_ARGS__);            \
         case 256 * 16 + 8: return FN<256, 2, false>(__VA_ARGS__);           \
+        case 64 * 16 + 12: return FN<64, 3, false>(__VA_ARGS__);            \
+        case 64 * 16 + 13: return FN<64, 3, true>(__VA_ARGS__);             \
+        case 128 * 16 + 12: return FN<128, 3, false>(__VA_ARGS__);          \
+        case 128 * 16 + 13: return FN<128, 3, true>(__VA_ARGS__);           \
         case 256 * 16 + 9: return FN<256, 2, true>(__VA_ARGS__);            \
         default: break;                                                     \
     }
@@ -1047,7 +1120,8 @@ cudaError_t launch_decode_mma(const kvq_ctx* h, const DecodeArgs& a, cudaStream_
 
 size_t decode_mma_qfrag_bytes(const kvq_ctx* h, int G) {
     const int NTK = (G <= 4) ? 2 : 4;
-    const int KS = (h->b + ((h->flags & 1u) ? 1 : 0)) * (h->d / 32);
+    const int PV = h->b == 3 ? 4 : h->b;  // code planes, the 3-bit parity plane included
+    const int KS = (PV + ((h->flags & 1u) ? 1 : 0)) * (h->d / 32);
     return static_cast<size_t>(KS) * NTK * 32 * 8;
 }
 

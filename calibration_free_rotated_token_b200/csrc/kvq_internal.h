@@ -130,12 +130,15 @@ void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, in
 
 cudaError_t launch_decode(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s, std::string* why);
 
-// Tensor-core decode path (1- and 2-bit codebooks): query fragments + split kernel.
+// Tensor-core decode path (1- and 2-bit codebooks, and 3-bit at d <= 128): query fragments + split kernel.
 cudaError_t launch_decode_mma(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s);
 size_t decode_mma_qfrag_bytes(const kvq_ctx* h, int G);
 // Resident CTAs of the tensor-core split kernel on the device (its persistent grid).
 int decode_mma_grid(const kvq_ctx* h, int G);
-inline bool decode_uses_mma(const kvq_ctx* h) { return h->b <= 2; }
+// 3-bit codebooks take four code planes (the parity plane included); at
+// d = 256 their operands no longer fit the register file, so they stay on the
+// CUDA-core path there.
+inline bool decode_uses_mma(const kvq_ctx* h) { return h->b <= 2 || (h->b == 3 && h->d <= 128); }
 
 // Size of the fixed scratch of kvq_decode_attend_noalloc (mirrors
 // KVQ_NOALLOC_SCRATCH_BYTES of kvq.h) and its address on `device`, which
