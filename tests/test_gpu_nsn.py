@@ -203,6 +203,8 @@ def check_nsn_decode(d, b, batch, hq, hkv, seq_len, cap, qdtype=torch.bfloat16, 
     (128, 2, 1, 16, 2, [2000], 2048),        # GQA 8:1
     (256, 2, 1, 4, 2, [513], 640),           # 128-token sub-chunks (one block each)
     (128, 1, 2, 4, 1, [0, 129], 256),        # an empty context
+    (128, 3, 1, 8, 2, [700], 768),           # 3 bits (parity plane)
+    (64, 3, 1, 4, 1, [384], 384),
 ])
 def test_nsn_decode_matches_oracle(d, b, batch, hq, hkv, seq_len, cap):
     check_nsn_decode(d, b, batch, hq, hkv, seq_len, cap)
