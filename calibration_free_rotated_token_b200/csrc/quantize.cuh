@@ -17,13 +17,12 @@
 //   transform is taken at load time).  The FWHT runs entirely in registers:
 //   no shuffles, no shared-memory round trips.
 // * Codes are written as bit planes built in registers; the residual r is
-//   split into fp16 hi + lo and stored into tensor memory (thread = TMEM lane
-//   = MMA row), and one elected thread issues tcgen05 MMAs
-//   D(128 x m) = A_hi S^T + A_lo S^T with S (fp16, exact) resident in shared
-//   memory.  The epilogue reads its own accumulator row back from TMEM and
-//   packs the sign bits.  S is an exact fp16 operand and r is carried to
-//   ~22 bits, so the sign of (S r)_i is exact wherever |(S r)_i| is above a
-//   few 1e-5 * ||r||.
+//   rounded once to fp16 and stored into tensor memory (thread = TMEM lane =
+//   MMA row), and one elected thread issues tcgen05 MMAs D(128 x m) = A S^T
+//   with S (fp16, exact) resident in shared memory.  The epilogue reads its
+//   own accumulator row back from TMEM and packs the sign bits.  The error of
+//   (S r)_i is about 2e-4 ||r||, so a sign can differ from the exact one
+//   outside a 1e-3 ||r|| band only through a 5-sigma error (~1e-11 per bit).
 // * Every wait on an mbarrier is bounded; the outcome is agreed on by the
 //   whole warpgroup (barrier reduction) so no thread is left at a barrier.
 #pragma once
@@ -293,26 +292,22 @@ __device__ __forceinline__ float codes_and_residual(float2 (&v)[NV / 2], float i
     return rr.x + rr.y;
 }
 
-// Residual (2*NP coordinates) as fp16 hi/lo pairs into tensor memory: A_hi
-// from column t_hi, A_lo from t_lo (two fp16 per 32-bit column, even
-// coordinate in the low half).
+// Residual (2*NP coordinates) as one fp16 term into tensor memory from
+// column t_hi (two fp16 per 32-bit column, even coordinate in the low half).
+// S is exact in fp16 and r is rounded once, so (S r)_i carries an error of
+// about 2e-4 ||r|| (fp32 accumulation): a sign can differ from the exact one
+// outside a 1e-3 ||r|| band only through a 5-sigma error, ~1e-11 per bit.
 template <int NP>
-__device__ __forceinline__ void store_residual_tmem(const float2 (&v)[NP], uint32_t t_hi, uint32_t t_lo) {
-    const float2 m1 = make_float2(-1.f, -1.f);
+__device__ __forceinline__ void store_residual_tmem(const float2 (&v)[NP], uint32_t t_hi) {
 #pragma unroll
     for (int cc = 0; cc < NP / 32; ++cc) {
-        uint32_t hi[32], lo[32];
+        uint32_t hi[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const float2 r = v[32 * cc + i];
-            const __half2 hh = __float22half2_rn(r);
-            const float2 rem = __ffma2_rn(__half22float2(hh), m1, r);
-            const __half2 ll = __float22half2_rn(rem);
+            const __half2 hh = __float22half2_rn(v[32 * cc + i]);
             hi[i] = *reinterpret_cast<const uint32_t*>(&hh);
-            lo[i] = *reinterpret_cast<const uint32_t*>(&ll);
         }
         tmem_st32(t_hi + cc * 32, hi);
-        tmem_st32(t_lo + cc * 32, lo);
     }
 }
 
@@ -338,20 +333,17 @@ __device__ __forceinline__ void qjl_bits_from_tmem(uint32_t taddr, uint32_t (&qw
     }
 }
 
-// Issue the QJL MMAs of one tile: acc(128 x N) = A_hi S^T + A_lo S^T.
+// Issue the QJL MMAs of one tile: acc(128 x N) = A S^T, A the fp16 residual.
 // K = KD coordinates, S resident in shared memory as KD/64 K-chunks of
 // N rows x 128 bytes (128-byte swizzle).
 template <int N, int KD>
-__device__ __forceinline__ void issue_qjl_mma(uint32_t acc, uint32_t a_hi, uint32_t a_lo, uint32_t s_smem) {
+__device__ __forceinline__ void issue_qjl_mma(uint32_t acc, uint32_t a_hi, uint32_t s_smem) {
     constexpr uint32_t idesc = idesc_f16_f32(kTileRows, N);
 #pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll
-        for (int ks = 0; ks < KD / 16; ++ks) {
-            const uint32_t boff = (ks / 4) * (N * 128) + (ks % 4) * 32;
-            const uint64_t bd = smem_desc_sw128(s_smem + boff);
-            mma_f16_ts(acc, (pass ? a_lo : a_hi) + ks * 8, bd, idesc, (pass | ks) ? 1u : 0u);
-        }
+    for (int ks = 0; ks < KD / 16; ++ks) {
+        const uint32_t boff = (ks / 4) * (N * 128) + (ks % 4) * 32;
+        const uint64_t bd = smem_desc_sw128(s_smem + boff);
+        mma_f16_ts(acc, a_hi + ks * 8, bd, idesc, ks ? 1u : 0u);
     }
 }
 
@@ -473,7 +465,7 @@ __global__ void __launch_bounds__(256, 1)
         const int r = tid & 127;
         const uint32_t bar_id = 1 + w;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tb = tmem + w * (2 * D);  // A_hi @ +0, A_lo @ +D/2, acc @ +D
+        const uint32_t tb = tmem + w * (2 * D);  // A (fp16 pairs) @ +0, acc @ +D
         if (r == 0) {
             prefetch_tmap(&map);
             for (int64_t i = w; i < kStages; i += 2) issue_tile(i);
@@ -590,13 +582,13 @@ __global__ void __launch_bounds__(256, 1)
                 // tile was computed; finish its epilogue now, which also frees the
                 // A and accumulator columns for this tile.
                 if (pend && !finish_pending()) break;
-                store_residual_tmem<D / 2>(v, tb + lane_base, tb + lane_base + D / 2);
+                store_residual_tmem<D / 2>(v, tb + lane_base);
                 tmem_wait_st();
                 tc_fence_before();
                 named_bar_sync(bar_id, 128);
                 if (r == 0) {
                     tc_fence_after();
-                    issue_qjl_mma<D, D>(tb + D, tb, tb + D / 2, smem_u32(sS));
+                    issue_qjl_mma<D, D>(tb + D, tb, smem_u32(sS));
                     mma_commit(&mmadone[w]);
                 }
                 pend = true;
@@ -648,15 +640,15 @@ __global__ void __launch_bounds__(256, 1)
             const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
             xch[h * 128 + r] = rr;
             if (QJL) {
-                // A_hi columns [0,128), A_lo [128,256), acc [256,512)
-                store_residual_tmem<64>(v, tmem + lane_base + h * 64, tmem + lane_base + 128 + h * 64);
+                // A columns [0,128) (two fp16 per column), acc [256,512)
+                store_residual_tmem<64>(v, tmem + lane_base + h * 64);
                 tmem_wait_st();
                 tc_fence_before();
             }
             named_bar_sync(3, 256);
             if (QJL && tid == 0) {
                 tc_fence_after();
-                issue_qjl_mma<256, 256>(tmem + 256, tmem, tmem + 128, smem_u32(sS));
+                issue_qjl_mma<256, 256>(tmem + 256, tmem, smem_u32(sS));
                 mma_commit(&mmadone[0]);
             }
             if (a.layout == 0) {
