@@ -10,8 +10,11 @@
 //   B = sum w n gamma sgn_v                                   (decode_split_kernel)
 //   merge the splits exactly, out = delta .* H (A + sqrt(pi/2)/m S^T B) / (d L)
 //                                                              (decode_combine_kernel)
-// Three launches on one stream; the split partials live in the caller's
-// workspace.  No kernel waits on another CTA.
+// Three launches on one stream (a fourth, decode_window_kernel, for a
+// residual window); the split partials live in the caller's workspace.  No
+// kernel waits on another CTA.  This file holds the CUDA-core path (4-bit
+// codebooks, and 3-bit at d = 256), the combine and window kernels shared
+// with the tensor-core path of decode_mma.cu, and the split plan.
 #include <cfloat>
 #include <mutex>
 

@@ -1,5 +1,6 @@
 // decode_mma.cu -- decode attention on the tensor cores (warp-level integer
-// MMA), for 1- and 2-bit codebooks.
+// MMA), for 1- and 2-bit codebooks and 3-bit ones at d <= 128; plain caches
+// (with or without QJL) and NSN caches.
 //
 // Method (TurboQuant blog, "Como Implementar": the query is rotated once and
 // the logits come straight from the stored indices; PolarQuant section 2:
@@ -11,7 +12,8 @@
 // Design (sm_100a, one GPU):
 // * A symmetric codebook of 2^b <= 4 levels is affine in the stored bit
 //   planes: c[code] = c0 + (c1 - c0) bit0 + (c2 - c0) bit1 (the bit0*bit1
-//   coefficient c3 - c2 - c1 + c0 vanishes by symmetry).  So every dot
+//   coefficient c3 - c2 - c1 + c0 vanishes by symmetry); a 3-bit one is
+//   affine in its three planes plus their parity (PlaneCoefs).  So every dot
 //   product above is a constant plus plain sums of 0/1 planes, and both
 //   contractions run as exact integer tensor-core products (m16n8k32):
 //   - keys:   D(16 tokens x 8) += A(16 tokens x 32 coords) B(32 coords x 8),
@@ -1110,7 +1112,7 @@ int decode_mma_grid(const kvq_ctx* h, int G) {
     return n;
 }
 
-// Query fragments + split kernel of the tensor-core path (b <= 2).
+// Query fragments + split kernel of the tensor-core path (decode_uses_mma).
 cudaError_t launch_decode_mma(const kvq_ctx* h, const DecodeArgs& a, cudaStream_t s) {
     const bool qjl = (h->flags & 1u) != 0;
     const int grid = decode_mma_grid(h, a.G);
