@@ -248,33 +248,22 @@ def test_sweep_decode_full_size_sampled(d, b, qjl):
 
 def test_decode_more_than_512_splits():
     """One stream of 528384 tokens: the tensor-core path splits it into 516 items of 1024 tokens,
-    so the combine merges more split partials than it caches at once.  The cache comes from the
-    CUDA quantizer; the oracle decodes the same stored cache (unpacked), one query per KV head."""
-    d, b, T, hkv = 128, 2, 528384, 1
+    so the combine merges more split partials than it caches at once.  The cache is the oracle's
+    own quantization of 4096 seeded keys and values, repeated 129 times along the context."""
+    d, b, rep = 128, 2, 129
     k = constants(d, b, 1)
+    K = wl.sweep_tokens(4096, d, seed=601).double().numpy()
+    V = wl.sweep_tokens(4096, d, seed=602).double().numpy()
+    ck, qk, nk, sk = oracle_cache(k, K, True)
+    cv, qv, nv, sv = oracle_cache(k, V, True, layout=1)
+    T = 4096 * rep
+    tile = lambda a: np.concatenate([a] * rep, axis=0)
+    kst = {key: tile(v) for key, v in sk.items()}
+    vst = {key: tile(v) for key, v in sv.items()}
+    q = wl.queries(1, 1, d, seed=603)
     with kvq.Handle(d, b, 1, qjl=True) as h:
-        K = wl.sweep_tokens(hkv * T, d, seed=601, device="cuda")
-        V = wl.sweep_tokens(hkv * T, d, seed=602, device="cuda")
-        kc_, kq_, kn_ = kvq.alloc_packed(h, hkv * T)
-        vc_, vq_, vn_ = kvq.alloc_packed(h, hkv * T, layout=1)
-        kvq.kvq_quantize_batch(h, [(K, kc_, kq_, kn_, 0), (V, vc_, vq_, vn_, 1)])
-        del K, V
-        q = wl.queries(1, hkv, d, seed=603, device="cuda")
-        kc = kvq.make_cache(kc_, kq_, kn_, T, 0)
-        vc = kvq.make_cache(vc_, vq_, vn_, T, 1)
-        out, _ = run_decode(h, q, hkv, kc, vc, [T], T, 1 / np.sqrt(d), want_logits=False)
-        codes_k, bits_k, norms_k = to_np_u32(kc_), to_np_u32(kq_), to_np_f16bits(kn_)
-        codes_v, bits_v, norms_v = to_np_u32(vc_), to_np_u32(vq_), to_np_f16bits(vn_)
-    qd = q.double().cpu().numpy()
-    for s in range(hkv):
-        sl = slice(s * T, (s + 1) * T)
-        nk = oracle.half_bits_to_double(norms_k.reshape(-1, 2)[sl])
-        nv = oracle.half_bits_to_double(norms_v.reshape(-1, 2)[sl])
-        kst = dict(codes=oracle.unpack_codes(codes_k.reshape(hkv * T, -1)[sl], b, d),
-                   bits=oracle.unpack_bits(bits_k.reshape(hkv * T, -1)[sl], d), norm=nk[:, 0], gamma=nk[:, 1])
-        blk = slice(s * T // 32, (s + 1) * T // 32)
-        vst = dict(codes=oracle.unpack_codes_block32(codes_v.reshape(hkv * T // 32, -1)[blk], b, d, T),
-                   bits=oracle.unpack_bits_block32(bits_v.reshape(hkv * T // 32, -1)[blk], d, T),
-                   norm=nv[:, 0], gamma=nv[:, 1])
-        _, orf = oracle.decode_attend(k, qd[0, s:s + 1], kst, vst, 1 / np.sqrt(d), True, want_logits=False)
-        assert_close(out[0, s:s + 1], orf, f"out kv head {s}")
+        kc, _kt = upload_streams(h, [(tile(ck), tile(qk), tile(nk))], T, 0)
+        vc, _vt = upload_streams(h, [(tile(cv), tile(qv), tile(nv))], T, 1)
+        out, _ = run_decode(h, q.cuda(), 1, kc, vc, [T], T, 1 / np.sqrt(d), want_logits=False)
+    _, orf = oracle.decode_attend(k, q[0].double().numpy(), kst, vst, 1 / np.sqrt(d), True, want_logits=False)
+    assert_close(out[0], orf, "out over 516 splits")

@@ -217,14 +217,16 @@ def test_nsn_decode_long_context():
 
 def test_nsn_decode_workload_full_size_sampled():
     """The NSN workload (8 heads x 65536 tokens, b=2) quantized by the CUDA NSN front end, keys per
-    token and values in blocks of 32, then decoded by 32 query heads (GQA 4:1, one token); two
-    sampled KV heads against the oracle's decode of the same stored cache."""
+    token and values in blocks of 32, then decoded by 32 query heads (GQA 4:1, one token).  One
+    sampled KV head is checked against the oracle's NSN quantization on sampled blocks and then
+    replaced by the oracle's own NSN cache, whose decode the oracle recomputes."""
     c = wl.NSN
-    H, T, d = c["heads"], c["tokens"], c["d"]
-    k = oracle.make_constants(d, c["b"], c["handle_seed"])
+    H, T, d, b = c["heads"], c["tokens"], c["d"], c["b"]
+    hs = 5
+    k = oracle.make_constants(d, b, c["handle_seed"])
     X = wl.nsn_tokens(H, T, d, c["seed"], device="cuda")
     Y = wl.nsn_tokens(H, T, d, c["seed"] + 1, device="cuda")
-    with kvq.Handle(d, c["b"], c["handle_seed"], qjl=False) as h:
+    with kvq.Handle(d, b, c["handle_seed"], qjl=False) as h:
         kc = torch.empty((H, T, h.b, d // 32), dtype=torch.int32, device="cuda")
         vc = torch.empty((H, T // 32, h.b, d), dtype=torch.int32, device="cuda")
         kn = torch.empty((H, T, 2), dtype=torch.float16, device="cuda")
@@ -233,6 +235,21 @@ def test_nsn_decode_workload_full_size_sampled():
         vm = torch.empty_like(km)
         kvq.kvq_nsn_quantize(h, X, kc, kn, km)
         kvq.kvq_nsn_quantize(h, Y, vc, vn, vm, layout=kvq.KVQ_LAYOUT_BLOCK32)
+        assert kvq.kvq_status(h)[0] == 0
+        Xs = X[hs].double().cpu().numpy()
+        Ys = Y[hs].double().cpu().numpy()
+        for blk in (0, 77, T // 128 - 1):  # the CUDA records of the sampled head, against the oracle
+            sl = slice(blk * 128, (blk + 1) * 128)
+            check_head(k, Xs[sl], to_np_u32(kc[hs, sl]), to_np_f16bits(kn[hs, sl]), to_np_f16bits(km[hs, blk:blk + 1]))
+        # the sampled head's cache becomes the oracle's own
+        rk, nbk, sk = _nsn_oracle_stream(k, Xs)
+        rv, nbv, sv = _nsn_oracle_stream(k, Ys)
+        kc[hs] = torch.from_numpy(oracle.pack_codes(rk["codes"], b).view(np.int32)).cuda()
+        vc[hs] = torch.from_numpy(oracle.pack_codes_block32(rv["codes"], b).view(np.int32).reshape(T // 32, b, d)).cuda()
+        kn[hs] = torch.from_numpy(nbk).cuda()
+        vn[hs] = torch.from_numpy(nbv).cuda()
+        km[hs] = torch.from_numpy(rk["mean_half"].view(np.float16)).cuda()
+        vm[hs] = torch.from_numpy(rv["mean_half"].view(np.float16)).cuda()
         q = wl.queries(1, 4 * H, d, seed=78, device="cuda")
         out = torch.empty((1, 4 * H, d), dtype=torch.float32, device="cuda")
         ws = torch.empty(kvq.kvq_decode_workspace(h, 1, 4 * H, H, T), dtype=torch.uint8, device="cuda")
@@ -242,13 +259,7 @@ def test_nsn_decode_workload_full_size_sampled():
         assert kvq.kvq_status(h)[0] == 0
     qd = q.double().cpu().numpy()
     out = out.cpu().numpy()
-    for hk in (2, 7):
-        nk = oracle.half_bits_to_double(to_np_f16bits(kn[hk]).reshape(T, 2))
-        nv = oracle.half_bits_to_double(to_np_f16bits(vn[hk]).reshape(T, 2))
-        sk = dict(codes=oracle.unpack_codes(to_np_u32(kc[hk]).reshape(T, -1), c["b"], d), norm_x=nk[:, 0],
-                  norm_w=nk[:, 1])
-        sv = dict(codes=oracle.unpack_codes_block32(to_np_u32(vc[hk]), c["b"], d, T), norm_x=nv[:, 0],
-                  norm_w=nv[:, 1])
-        _, orf = oracle.nsn_decode_attend(k, qd[0, 4 * hk:4 * hk + 4], sk, sv, to_np_f16bits(km[hk]),
-                                          to_np_f16bits(vm[hk]), d ** -0.5, want_logits=False)
-        assert_close(out[0, 4 * hk:4 * hk + 4], orf, f"nsn workload out kvh{hk}")
+    _, orf = oracle.nsn_decode_attend(k, qd[0, 4 * hs:4 * hs + 4], sk, sv, rk["mean_half"], rv["mean_half"],
+                                      d ** -0.5, want_logits=False)
+    assert_close(out[0, 4 * hs:4 * hs + 4], orf, f"nsn workload out kvh{hs}")
+    assert np.isfinite(out).all()

@@ -9,7 +9,7 @@ import oracle
 from calibration_free_rotated_token_b200 import _abi as kvq
 from calibration_free_rotated_token_b200 import workloads as wl
 
-from .parity import assert_close, oracle_cache, to_np_f16bits, to_np_u32
+from .parity import assert_close, compare_quantize, oracle_cache, to_np_f16bits, to_np_u32
 from .test_gpu_decode import constants, upload_streams
 
 pytestmark = pytest.mark.gpu
@@ -96,8 +96,9 @@ def test_window_rejects_bad_arguments():
 def test_flush_append_cycle():
     """Tokens arrive one by one into a 32-token fp16 window; a full window is flushed by
     kvq_quantize_batch into the packed arrays at offset seq_len (keys per token, values in
-    blocks of 32).  The incrementally built cache equals one quantize over all flushed tokens,
-    and decode over packed + window equals the oracle over the same stored cache."""
+    blocks of 32).  The incrementally built cache equals one quantize over all flushed tokens and
+    matches the oracle's quantization of them; decoding the oracle's own cache of those tokens
+    plus the live window then matches the oracle's window decode."""
     d, b, W, steps = 128, 2, 32, 203
     hkv, hq = 2, 8
     cap = 256
@@ -128,32 +129,37 @@ def test_flush_append_cycle():
                 T += W
                 n = 0
         assert kvq.kvq_status(h)[0] == 0
-        # the same tokens quantized at once (the fp16 values the window held)
+        assert T == 192 and n == 11
+        caches = []
         for s in range(hkv):
+            Kf = X[s, :T].half()
+            Vf = Y[s, :T].half()
+            # the same tokens quantized at once
             c1, q1, n1 = kvq.alloc_packed(h, T)
-            kvq.kvq_quantize(h, X[s, :T].half(), c1, q1, n1)
+            kvq.kvq_quantize(h, Kf, c1, q1, n1)
             assert torch.equal(c1.reshape(T, -1), kcodes[s, :T].reshape(T, -1))
             assert torch.equal(q1.reshape(T, -1), kqjl[s, :T].reshape(T, -1)) and torch.equal(n1, kn[s, :T])
+            # the flushed records against the oracle's quantization of the same fp16 tokens
+            Kd, Vd = Kf.double().cpu().numpy(), Vf.double().cpu().numpy()
+            compare_quantize(k, Kd, to_np_u32(kcodes[s, :T]), to_np_u32(kqjl[s, :T]), to_np_f16bits(kn[s, :T]), True)
+            compare_quantize(k, Vd, to_np_u32(vcodes[s, :T // 32]), to_np_u32(vqjl[s, :T // 32]),
+                             to_np_f16bits(vn[s, :T]), True, layout=1)
+            caches.append((oracle_cache(k, Kd, True), oracle_cache(k, Vd, True, layout=1)))
+        # decode the oracle's own cache of the flushed tokens, plus the live window
+        kc_, _kt = upload_streams(h, [c[0][:3] for c in caches], cap, 0)
+        vc_, _vt = upload_streams(h, [c[1][:3] for c in caches], cap, 1)
         q = wl.queries(1, hq, d, seed=80, device="cuda")
         out = torch.empty((1, hq, d), dtype=torch.float32, device="cuda")
         ws = torch.empty(kvq.kvq_decode_workspace(h, 1, hq, hkv, cap), dtype=torch.uint8, device="cuda")
-        kvq.kvq_decode_attend_ex(h, q, hkv, kvq.make_cache(kcodes, kqjl, kn, cap, 0),
-                                 kvq.make_cache(vcodes, vqjl, vn, cap, 1),
-                                 torch.tensor([T], dtype=torch.int32, device="cuda"), cap, 1 / np.sqrt(d), out, ws,
-                                 k_window=kwin, v_window=vwin,
+        kvq.kvq_decode_attend_ex(h, q, hkv, kc_, vc_, torch.tensor([T], dtype=torch.int32, device="cuda"), cap,
+                                 1 / np.sqrt(d), out, ws, k_window=kwin, v_window=vwin,
                                  window_len=torch.tensor([n], dtype=torch.int32, device="cuda"))
         assert kvq.kvq_status(h)[0] == 0
-    assert T == 192 and n == 11
     G = hq // hkv
     qd = q.double().cpu().numpy()
     out = out.cpu().numpy()
     for s in range(hkv):
-        nk = oracle.half_bits_to_double(to_np_f16bits(kn[s, :T]).reshape(T, 2))
-        nv = oracle.half_bits_to_double(to_np_f16bits(vn[s, :T]).reshape(T, 2))
-        kst = dict(codes=oracle.unpack_codes(to_np_u32(kcodes[s, :T]).reshape(T, -1), b, d),
-                   bits=oracle.unpack_bits(to_np_u32(kqjl[s, :T]).reshape(T, -1), d), norm=nk[:, 0], gamma=nk[:, 1])
-        vst = dict(codes=oracle.unpack_codes_block32(to_np_u32(vcodes[s, :T // 32]), b, d, T),
-                   bits=oracle.unpack_bits_block32(to_np_u32(vqjl[s, :T // 32]), d, T), norm=nv[:, 0], gamma=nv[:, 1])
+        kst, vst = caches[s][0][3], caches[s][1][3]
         _, orf = oracle.window_decode_attend(k, qd[0, s * G:(s + 1) * G], kst, vst, kwin[s, :n].double().cpu().numpy(),
                                              vwin[s, :n].double().cpu().numpy(), 1 / np.sqrt(d), True)
         assert_close(out[0, s * G:(s + 1) * G], orf, f"out kvh{s}")
