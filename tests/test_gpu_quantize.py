@@ -318,3 +318,36 @@ def test_bounded_wait_runs_out_and_the_context_stays_usable():
                          to_np_f16bits(norms), True)
         with pytest.raises(kvq.KvqError):
             kvq.kvq_probe_wait_timeout(h, 0)
+
+
+def test_size_limits_are_rejected_on_the_host():
+    """More than 2^31 - 128 vectors in one call (the kernels index rows in 32 bits) is rejected
+    before anything is read or launched, alone and inside a batch; so is a negative count."""
+    with kvq.Handle(128, 2, 1, qjl=True) as h:
+        L = kvq.load()
+        big = (1 << 31) - 127
+        assert L.kvq_quantize(h.ptr, None, kvq.KVQ_BF16, big, 128, 0, None, None, None, None) == kvq.KVQ_EINVAL
+        assert "2^31" in kvq.kvq_last_error()
+        assert L.kvq_quantize(h.ptr, None, kvq.KVQ_BF16, -1, 128, 0, None, None, None, None) == kvq.KVQ_EINVAL
+        x = torch.randn(64, 128, device="cuda", dtype=torch.bfloat16)
+        good = kvq.alloc_packed(h, 64)
+        good[0].fill_(7)
+        jobs = (kvq.KvqQuantJob * 2)(kvq._job(h, x, *good, 0), kvq._job(h, x, *good, 0))
+        jobs[1].n = big
+        assert L.kvq_quantize_batch(h.ptr, 2, jobs, None) == kvq.KVQ_EINVAL
+        torch.cuda.synchronize()
+        assert (good[0] == 7).all()
+        # decode: hq not a multiple of hkv, and a GQA ratio that is not built
+        out = torch.empty(1, 6, 128, device="cuda")
+        ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+        c, qj, n = kvq.alloc_packed(h, 128)
+        kc = kvq.make_cache(c, qj, n, 128, 0)
+        vc_, vq_, vn_ = kvq.alloc_packed(h, 128, layout=1)
+        vc = kvq.make_cache(vc_, vq_, vn_, 128, 1)
+        sl = torch.tensor([128], dtype=torch.int32, device="cuda")
+        q6 = torch.randn(1, 6, 128, device="cuda", dtype=torch.bfloat16)
+        with pytest.raises(kvq.KvqError):
+            kvq.kvq_decode_attend(h, q6, 4, kc, vc, sl, 128, 1.0, out, ws)
+        q3 = torch.randn(1, 3, 128, device="cuda", dtype=torch.bfloat16)
+        with pytest.raises(kvq.KvqError):  # hq / hkv = 3 is not built
+            kvq.kvq_decode_attend(h, q3, 1, kc, vc, sl, 128, 1.0, out[:, :3], ws)
