@@ -218,6 +218,20 @@ def traffic_record(kernel: str):
     return rec.get("dram_bytes_per_launch")
 
 
+def parity_record():
+    """Boundary-excluded code counts per workload, pooled by the parity tests
+    (tests/test_gpu_boundary_rates.py, written with KVQ_PARITY_RECORD) and
+    committed under profiles/; null when absent."""
+    p = os.path.join(ROOT, "profiles", "parity_boundary.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    return {"bar": j.get("bar"), "source": "profiles/parity_boundary.json",
+            "workloads": {k: {"excluded": v["excluded"], "coords": v["coords"], "rate": float(f"{v['rate']:.3g}")}
+                          for k, v in j.get("workloads", {}).items()}}
+
+
 # ----------------------------------------------------------------------------
 # our implementation
 # ----------------------------------------------------------------------------
@@ -610,18 +624,16 @@ def run_ours(args):
         dist.close()
         return
     q = bench_quantize(args, dist)
-    extra = {}
-    if not args.no_decode:
-        extra["decode_attn"] = bench_decode(args, dist)
-    if not args.no_nsn:
-        extra["nsn_quantize"] = bench_nsn(args, dist)
-    if not args.no_sweep:
-        extra["sweep"] = bench_sweep(args, dist)
+    sweep = None if args.no_sweep else bench_sweep(args, dist)
+    nsn = None if args.no_nsn else bench_nsn(args, dist)
+    dec = None if args.no_decode else bench_decode(args, dist)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         cpu = cpu_baseline(q["sample_input"], args.cpu_vectors)
     if dist.rank == 0:
         value = whole_job_rate(dist.world, q["tokens_per_step"] * args.steps, q["ms"])
+        # The long per-configuration sweep goes first and the headline figures last, so that
+        # a reader who keeps only the end of the line still has both halves of the metric.
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": q["ms"] / args.steps, "higher_is_better": True,
@@ -633,11 +645,20 @@ def run_ours(args):
                        "vectors_per_step": q["vectors_per_step"],
                        "l2": "4 rotating input copies per rank (4 x 134 MB > 126 MB L2)",
                        "parallelism": f"dp{dist.world} (independent layers per rank, no collective)"},
-            "roofline": q["roofline"], "tensor": q["tensor"], "cpu_baseline": cpu, "e2e": q["e2e"],
-            "gpu_launches": q["launches"],
-            "clocks": q["clocks"],
         }
-        line.update(extra)
+        if sweep is not None:
+            line["sweep"] = sweep
+        if nsn is not None:
+            line["nsn_quantize"] = nsn
+        line["tensor"] = q["tensor"]
+        line["parity_boundary"] = parity_record()
+        if dec is not None:
+            line["decode_attn"] = dec
+        line.update({"cpu_baseline": cpu, "e2e": q["e2e"], "gpu_launches": q["launches"], "clocks": q["clocks"],
+                     "roofline": q["roofline"]})
+        if dec is not None:
+            line["decode_gbs"] = dec["value"]
+            line["decode_frac_of_hbm"] = dec["frac_of_hbm"]
         print(json.dumps(line), flush=True)
     dist.close()
 

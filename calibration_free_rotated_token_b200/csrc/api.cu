@@ -688,8 +688,13 @@ int kvq_decode_attend_noalloc(kvq_handle h, const void* q, int dtype, int batch,
         return fail(KVQ_EINVAL, "these sizes need " + std::to_string(need) + " bytes of decode scratch, more than the " +
                                     std::to_string(kvq::kNoAllocScratchBytes) +
                                     " bytes built into the library; use kvq_decode_attend with a workspace");
+    // check_handle (in decode_check) made sure h->device is current; the
+    // scratch address is looked up for, and cached under, the current device.
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != h->device)
+        return fail(KVQ_EINVAL, "the handle's device is not the current device");
     void* scratch = nullptr;
-    const cudaError_t e = kvq::noalloc_scratch(h->device, &scratch);
+    const cudaError_t e = kvq::noalloc_scratch(cur, &scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the decode scratch");
     return decode_launch(h, q, dtype, batch, hq, hkv, k, v, seq_len, max_T, scale, logits, out, scratch, ns, chunk,
                          stream);

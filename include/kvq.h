@@ -24,6 +24,11 @@
  *  - Return 0 (KVQ_OK) on success or a negative KVQ_E* code; the message of
  *    the last failure on the calling thread is kvq_last_error().  Nothing is
  *    thrown across the ABI and no kernel traps.
+ *  - A handle belongs to the CUDA device that was current at kvq_init.
+ *    Every call that launches work or reads the device (all but kvq_init,
+ *    kvq_destroy, kvq_codebook, kvq_get_info, kvq_get_constants and
+ *    kvq_last_error) requires that device to be current and returns
+ *    KVQ_EINVAL, before any launch, when another device is current.
  *  - Pointer arguments named as "device" must point to device memory of the
  *    current CUDA device; the caller allocates and owns every input, output
  *    and workspace buffer.  The handle owns only its constants.

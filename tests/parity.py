@@ -21,13 +21,33 @@ import oracle
 CODE_BAND = 1e-5
 CODE_EXCL_MAX_FRAC = 1e-4
 
+# Boundary-excluded coordinates pooled per workload.  The stated bar ("fewer
+# than 1e-4 of all coordinates") is a rate: it is checked on the count pooled
+# over every coordinate a workload's tests compare (pooled_check), not per
+# call, where a few coordinates of noise on a small sample would decide it.
+POOL: dict = {}
+_POOL_LOCK = __import__("threading").Lock()
 
-def max_excluded(n_coords: int) -> float:
-    """Allowed count of boundary-excluded coordinates: the stated rate 1e-4,
-    plus a 5-sigma Poisson margin so that small samples do not fail on
-    counting noise (at 1e6 coordinates the margin is 5% of the rate)."""
-    lam = CODE_EXCL_MAX_FRAC * n_coords
-    return lam + 5.0 * lam ** 0.5 + 3.0
+
+def pool_add(name: str, excluded: int, coords: int) -> None:
+    with _POOL_LOCK:
+        e = POOL.setdefault(name, [0, 0])
+        e[0] += int(excluded)
+        e[1] += int(coords)
+
+
+def pooled(name: str) -> dict:
+    ex, n = POOL.get(name, (0, 0))
+    return {"excluded": ex, "coords": n, "rate": (ex / n) if n else 0.0}
+
+
+def pooled_check(name: str) -> dict:
+    """The pooled count of a workload against the stated rate, with no margin."""
+    r = pooled(name)
+    assert r["coords"] > 0, f"nothing pooled for {name}"
+    assert r["excluded"] <= CODE_EXCL_MAX_FRAC * r["coords"], \
+        f"{name}: {r['excluded']} boundary-excluded coordinates of {r['coords']} (rate {r['rate']:.2e} > 1e-4)"
+    return r
 QJL_BAND = 1e-3
 ATOL, RTOL = 1e-4, 2e-3
 
@@ -46,8 +66,9 @@ def ulp_distance_f16(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
 
 
 def compare_quantize(k: oracle.Constants, x: np.ndarray, codes_g, qjl_g, norms_g, use_qjl: bool,
-                     ref: dict | None = None, layout: int = 0) -> dict:
-    """Checks one quantize call (layout 0: one record per vector, 1: block-32); returns counts."""
+                     ref: dict | None = None, layout: int = 0, pool: str | None = None) -> dict:
+    """Checks one quantize call (layout 0: one record per vector, 1: block-32); returns counts.
+    The boundary-excluded count is added to the workload `pool` (checked by pooled_check)."""
     x = np.asarray(x, np.float64)
     n, d = x.shape
     if ref is None:
@@ -60,7 +81,8 @@ def compare_quantize(k: oracle.Constants, x: np.ndarray, codes_g, qjl_g, norms_g
     near[ref["norm"] == 0] = False  # a zero vector has a defined all-zero record: compared exactly
     bad = (codes != ref["codes"]) & ~near
     assert bad.sum() == 0, f"{bad.sum()} codes differ outside the boundary band (first at {np.argwhere(bad)[:5]})"
-    assert near.sum() <= max_excluded(near.size), f"{near.sum()} excluded coordinates of {near.size}"
+    if pool is not None:
+        pool_add(pool, near.sum(), near.size)
     # excluded coordinates must hold one of the two codes adjacent to a nearby threshold
     if near.any():
         zc = ref["z"][near]
@@ -99,9 +121,24 @@ def assert_close(got: np.ndarray, want: np.ndarray, what: str):
     return worst
 
 
+def oracle_quantize_threads(k: oracle.Constants, x: np.ndarray, use_qjl: bool) -> dict:
+    """oracle.quantize of the rows of x, over row ranges on the host cores (the C oracle runs
+    without the interpreter lock; the ranges share nothing), concatenated in order."""
+    import concurrent.futures as cf
+    import os
+
+    x = np.asarray(x, np.float64)
+    parts = [p for p in np.array_split(x, max(1, min(os.cpu_count() or 1, 32))) if p.shape[0]]
+    if len(parts) <= 1:
+        return oracle.quantize(k, x, use_qjl)
+    with cf.ThreadPoolExecutor(max_workers=len(parts)) as ex:
+        outs = list(ex.map(lambda p: oracle.quantize(k, p, use_qjl), parts))
+    return {key: np.concatenate([o[key] for o in outs]) for key in outs[0]}
+
+
 def oracle_cache(k: oracle.Constants, x: np.ndarray, use_qjl: bool, layout: int = 0):
     """The oracle's own packed cache of x: (codes u32, qjl u32 or None, norms fp16, widened dict)."""
-    q = oracle.quantize(k, x, use_qjl)
+    q = oracle_quantize_threads(k, x, use_qjl)
     if layout == 0:
         codes = oracle.pack_codes(q["codes"], k.b)
         qjl = oracle.pack_bits(q["bits"]) if use_qjl else None

@@ -129,12 +129,21 @@ def test_decode_beta_codebook_matches_oracle(d, b, qjl, batch, hq, hkv, seq_len,
     check_case(d, b, qjl, batch, hq, hkv, seq_len, cap, scale=1 / np.sqrt(d), beta=True)
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+@pytest.mark.parametrize("qjl", [True, False])
+def test_decode_every_sweep_kernel(d, b, qjl):
+    """Every (d, b, QJL) the sweep decodes, at its GQA 1:1 (one query per KV head): two sequences
+    of 4500 and 4133 tokens (several splits and sub-chunks, ragged tails), logits and outputs."""
+    check_case(d, b, qjl, 2, 1, 1, [4500, 4133], 4512, scale=1 / np.sqrt(d), qdtype=torch.bfloat16, seed=4)
+
+
 def test_long_context_split_merge():
     """A context long enough for many splits (exact merge of the split partials)."""
     check_case(128, 2, True, 1, 4, 1, [20000], 20000, scale=1.0 / np.sqrt(128))
 
 
-def _sampled_stream_decode(B, hq, hkv, T, sample, check_rows=1024):
+def _sampled_stream_decode(B, hq, hkv, T, sample, check_rows=1024, want_logits=True):
     """Cache of B x hkv streams of T tokens from the CUDA quantizer (Llama-layer generator);
     one sampled (sequence, KV head) is checked against the oracle's quantization on sampled
     rows and then replaced by the oracle's own cache, whose decode the oracle recomputes."""
@@ -178,10 +187,13 @@ def _sampled_stream_decode(B, hq, hkv, T, sample, check_rows=1024):
         q = wl.queries(B, hq, d, c["q_seed"], device="cuda", std=c["q_std"])
         kc = kvq.make_cache(kcodes, kqjl, knorm, T, 0)
         vc = kvq.make_cache(vcodes, vqjl, vnorm, T, 1)
-        out, _ = run_decode(h, q, hkv, kc, vc, [T] * B, T, c["scale"], want_logits=False)
+        out, logits = run_decode(h, q, hkv, kc, vc, [T] * B, T, c["scale"], want_logits=want_logits)
     qs = q[sample[0], sample[1] * G:(sample[1] + 1) * G].double().cpu().numpy()
-    _, orf = oracle.decode_attend(k, qs, sk, sv, c["scale"], True, want_logits=False)
+    lr, orf = oracle.decode_attend(k, qs, sk, sv, c["scale"], True, want_logits=want_logits)
     assert_close(out[sample[0], sample[1] * G:(sample[1] + 1) * G], orf, "out (sampled stream)")
+    if want_logits:
+        assert_close(logits[sample[0], sample[1] * G:(sample[1] + 1) * G], lr, "logits (sampled stream)")
+        assert np.isfinite(logits).all()
     assert np.isfinite(out).all()
 
 

@@ -25,20 +25,29 @@ def _cache(h, S, T, seed, layout):
     parts = [kvq.alloc_packed(h, T, layout=layout) for _ in range(S)]
     for s in range(S):
         kvq.kvq_quantize(h, x[s], *parts[s], layout=layout)
-    return [torch.stack([p[i] for p in parts]) for i in range(3)]
+    return [torch.stack([p[i] for p in parts]) if parts[0][i] is not None else None for i in range(3)]
 
 
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
-    d, B, hq, hkv, T = 128, 2, 8, 2, 3008
-    with kvq.Handle(d, 2, 1, qjl=True) as h:
-        kt = _cache(h, B * hkv, T, seed=5, layout=0)
-        vt = _cache(h, B * hkv, T, seed=6, layout=1)
-        kc = kvq.make_cache(*kt, T, 0)
-        vc = kvq.make_cache(*vt, T, 1)
-        seq = torch.tensor([T, 1777], dtype=torch.int32, device="cuda")
-        ws = torch.empty(kvq.kvq_decode_workspace(h, B, hq, hkv, T), dtype=torch.uint8, device="cuda")
-        assert ws.numel() <= kvq.NOALLOC_SCRATCH_BYTES
-        for call in range(2):
+@pytest.mark.parametrize("b,qjl,Ts", [
+    (2, True, (3008, 3008)),   # tensor-core path, the same sizes twice
+    (2, True, (3008, 1056)),   # tensor-core path, fewer splits on the second call
+    (4, True, (3008, 1056)),   # CUDA-core path (its own carving of the scratch), fewer splits next
+    (3, False, (640, 2048)),   # 3-bit tensor-core path without QJL, more splits next
+])
+def test_noalloc_matches_workspace_entry_point_on_two_calls(b, qjl, Ts):
+    """Two calls in a row, each against kvq_decode_attend on the same inputs; when the second
+    call's context is shorter, nothing it reads may come from the first call's leftovers."""
+    d, B, hq, hkv = 128, 2, 8, 2
+    cap = max(Ts)
+    with kvq.Handle(d, b, 1, qjl=qjl) as h:
+        kt = _cache(h, B * hkv, cap, seed=5, layout=0)
+        vt = _cache(h, B * hkv, cap, seed=6, layout=1)
+        kc = kvq.make_cache(*kt, cap, 0)
+        vc = kvq.make_cache(*vt, cap, 1)
+        for call, T in enumerate(Ts):
+            seq = torch.tensor([T, min(1777, T - 33)], dtype=torch.int32, device="cuda")
+            ws = torch.empty(kvq.kvq_decode_workspace(h, B, hq, hkv, T), dtype=torch.uint8, device="cuda")
+            assert ws.numel() <= kvq.NOALLOC_SCRATCH_BYTES
             q = wl.queries(B, hq, d, seed=100 + call, device="cuda")
             ref = torch.empty((B, hq, d), dtype=torch.float32, device="cuda")
             ref_l = torch.empty((B, hq, T), dtype=torch.float32, device="cuda")
