@@ -88,6 +88,10 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_double, P, P]
             L.orc_nsn_quantize.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P,
                                            ctypes.c_int64, P, P, P, P, P, P, P]
+            L.orc_nsn_dq_rec_bytes.restype = ctypes.c_int
+            L.orc_nsn_dq_rec_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
+            L.orc_nsn_dq_quantize.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, ctypes.c_int64,
+                                              P, P, P, P, P, P, P, P, P]
             _lib = L
     return _lib
 
@@ -423,6 +427,84 @@ def nsn_decode_attend(k: Constants, q, kcache: dict, vcache: dict, kmean, vmean,
     G, d = q.shape
     if Kh.shape[0] == 0:
         return (np.zeros((G, 0)) if want_logits else None), np.zeros((G, d))
+    logits = scale * (q @ Kh.T)
+    e = np.exp(logits - logits.max(axis=1, keepdims=True))
+    out = (e @ Vh) / e.sum(axis=1, keepdims=True)
+    return (logits if want_logits else None), out
+
+
+# ----------------------------------------------------------------------------
+# NSN with double quantization of its side data (NSNQuant section 3)
+# ----------------------------------------------------------------------------
+def nsn_dq_rec_bytes(d: int, blk: int = NSN_BLOCK) -> int:
+    """Bytes of one block's side record (see orc_nsn_dq_quantize)."""
+    return int(lib().orc_nsn_dq_rec_bytes(d, blk))
+
+
+def nsn_dq_quantize(k: Constants, x, side_in=None, blk: int = NSN_BLOCK) -> dict:
+    """NSN front end with 4-bit norm and mean codes + the quantizer (no QJL) on one head's
+    tokens ([n_tok, d], n_tok % blk == 0).  side_in (uint8 [n_tok/blk, rec_bytes]) replaces the
+    side records this function would write (their steps and codes are then used as given)."""
+    x = _c(x, np.float64)
+    n, d = x.shape
+    assert n % blk == 0
+    nb = n // blk
+    R = nsn_dq_rec_bytes(d, blk)
+    codes = np.empty((n, d), np.int32)
+    nw = np.empty(n, np.float64)
+    side = np.empty((nb, R), np.uint8)
+    n1 = np.empty(n, np.float64)
+    oh = np.empty((nb, d), np.float64)
+    of = np.empty((nb, d), np.float64)
+    nx = np.empty(n, np.float64)
+    z = np.empty((n, d), np.float64)
+    si = None if side_in is None else _c(side_in, np.uint8).reshape(nb, R)
+    lib().orc_nsn_dq_quantize(d, k.b, blk, _p(k.delta), _p(k.centroids), _p(k.thresholds), _p(x), n, _p(si),
+                              _p(codes), _p(nw), _p(side), _p(n1), _p(oh), _p(of), _p(nx), _p(z))
+    return dict(codes=codes, norm_w=nw, side=side, n1=n1, o_hat=oh, mean_f64=of, norm_x=nx, z=z)
+
+
+def nsn_dq_unpack(side, d: int, blk: int = NSN_BLOCK):
+    """The stored scales and means of side records ([nb, rec_bytes] uint8), decoded as the
+    format defines them: n1 = q nstep (exact), o_hat = fp32(lo + step q).  Returns
+    (n1 [nb * blk], o_hat [nb, d]) in float64."""
+    side = np.asarray(side, np.uint8).reshape(-1, nsn_dq_rec_bytes(d, blk))
+    nb = side.shape[0]
+    f16 = lambda lo, hi: (side[:, lo].astype(np.uint16) | (side[:, hi].astype(np.uint16) << 8)).view(np.float16)
+    lo = f16(0, 1).astype(np.float64)
+    st = f16(2, 3).astype(np.float64)
+    ns = f16(4, 5).astype(np.float64)
+    ob = side[:, 8:8 + d // 2]
+    qo = np.stack([ob & 15, ob >> 4], axis=2).reshape(nb, d).astype(np.float64)
+    nbt = side[:, 8 + d // 2:8 + d // 2 + blk // 2]
+    qn = np.stack([nbt & 15, nbt >> 4], axis=2).reshape(nb, blk).astype(np.float64)
+    o_hat = (lo[:, None] + st[:, None] * qo).astype(np.float32).astype(np.float64)
+    n1 = (qn * ns[:, None]).reshape(-1)
+    return n1, o_hat
+
+
+def nsn_dq_dequantize(k: Constants, codes, norm_w, side, blk: int = NSN_BLOCK) -> np.ndarray:
+    """Vectors stored with double-quantized side data: x_hat = n1/sqrt(d) (w_hat + o_hat)."""
+    codes = _c(codes, np.int32)
+    n, d = codes.shape
+    n1, o_hat = nsn_dq_unpack(side, d, blk)
+    w = dequantize(k, codes, None, norm_w, np.zeros(n), use_qjl=False)
+    o = np.repeat(o_hat, blk, axis=0)[:n]
+    return (n1[:n] / np.sqrt(d))[:, None] * (w + o)
+
+
+def nsn_dq_decode_attend(k: Constants, q, kcache: dict, vcache: dict, kside, vside, scale: float,
+                         want_logits: bool = True):
+    """Attention of G queries over keys and values stored with double-quantized NSN side
+    data; caches hold ``codes`` [T, d] and ``norm_w`` [T] (fp16-widened).  Softmax in fp64
+    over the reconstructed vectors (nsn_dq_dequantize)."""
+    q = _c(np.atleast_2d(q), np.float64)
+    G, d = q.shape
+    T = np.asarray(kcache["codes"]).reshape(-1, d).shape[0]
+    if T == 0:
+        return (np.zeros((G, 0)) if want_logits else None), np.zeros((G, d))
+    Kh = nsn_dq_dequantize(k, kcache["codes"], kcache["norm_w"], kside)[:T]
+    Vh = nsn_dq_dequantize(k, vcache["codes"], vcache["norm_w"], vside)[:T]
     logits = scale * (q @ Kh.T)
     e = np.exp(logits - logits.max(axis=1, keepdims=True))
     out = (e @ Vh) / e.sum(axis=1, keepdims=True)

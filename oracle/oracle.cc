@@ -457,4 +457,120 @@ void orc_nsn_quantize(int d, int b, int blk, const int8_t* delta, const double* 
     }
 }
 
+// ---------------------------------------------------------------------------
+// NSN front end with double quantization of its side data ([NSN] sec. 3,
+// "Double Quantization": the NSN parameters -- the mean o and the scale s1 --
+// are themselves quantized to 4 bits).  The pages give no format; the reading
+// (recorded with the design notes) is, per block of `blk` tokens of one head:
+//   s1:  4-bit linear codes of the token norms on the block's own step
+//        nstep = fp16(max_t ||x_t|| / 15):  q = 0 for a zero token, else
+//        q = clamp(rint(||x|| / nstep), 1, 15);  n1 = q * nstep  (exact);
+//   u_t = sqrt(d) x_t / n1_t              (0 for q = 0)
+//   o   = mean over the block of u_t, per channel;
+//   o:   4-bit linear codes on [lo, lo + 15 step] with lo = fp16(min_j o_j),
+//        step = fp16((max_j o_j - min_j o_j) / 15):
+//        q_j = clamp(rint((o_j - lo) / step), 0, 15)  (0 when step = 0),
+//        o_hat_j = fp32(lo + step q_j)   (the exact sum rounded once to fp32)
+//   w_t = u_t - o_hat, quantized like the plain NSN front end (no QJL);
+//   stored: codes, fp16 ||w_t||, and one side record per block:
+//     bytes [0,2) fp16 lo, [2,4) fp16 step, [4,6) fp16 nstep, [6,8) zero,
+//     [8, 8 + d/2) o codes (byte i: channel 2i low nibble, 2i+1 high),
+//     [8 + d/2, 8 + d/2 + blk/2) norm codes (byte i: token 2i low, 2i+1 high),
+//     zero padding to a multiple of 16 bytes (rec_bytes).
+// The stored values are the ones the transform used, so x_t = n1_t / sqrt(d)
+// (w_t + o_hat) exactly before w_t is coded.  side_in (nullable) replaces
+// this function's side records by given ones (codes and steps), so that the
+// rest can be recomputed for a record another implementation wrote.
+// Outputs: codes[n_tok*d], norm_w[n_tok], side_out[(n_tok/blk)*rec_bytes],
+// n1[n_tok], o_hat[(n_tok/blk)*d], o_f64[(n_tok/blk)*d] (unquantized
+// means), norm_x[n_tok] (unquantized norms), z_out (nullable).
+// ---------------------------------------------------------------------------
+int orc_nsn_dq_rec_bytes(int d, int blk) { return (8 + d / 2 + blk / 2 + 15) / 16 * 16; }
+
+void orc_nsn_dq_quantize(int d, int b, int blk, const int8_t* delta, const double* centroid,
+                         const double* threshold, const double* x, int64_t n_tok, const uint8_t* side_in,
+                         int32_t* codes, double* norm_w, uint8_t* side_out, double* n1, double* o_hat,
+                         double* o_f64, double* norm_x, double* z_out) {
+    const int R = orc_nsn_dq_rec_bytes(d, blk);
+    std::vector<double> u((size_t)blk * d), o(d), w(d);
+    const double sqd = std::sqrt((double)d);
+    for (int64_t b0 = 0; b0 < n_tok; b0 += blk) {
+        const int64_t bi = b0 / blk;
+        uint8_t* rec = side_out + bi * R;
+        for (int e = 0; e < R; ++e) rec[e] = 0;
+        // token norms and their 4-bit codes
+        double mx = 0.0;
+        for (int t = 0; t < blk; ++t) {
+            const double* xv = x + (b0 + t) * d;
+            double ss = 0.0;
+            for (int j = 0; j < d; ++j) ss += xv[j] * xv[j];
+            norm_x[b0 + t] = std::sqrt(ss);
+            mx = std::fmax(mx, norm_x[b0 + t]);
+        }
+        uint16_t nstep16 = orc_double_to_half(mx / 15.0);
+        if (side_in) nstep16 = (uint16_t)(side_in[bi * R + 4] | (side_in[bi * R + 5] << 8));
+        const double nstep = orc_half_to_double(nstep16);
+        rec[4] = (uint8_t)(nstep16 & 0xFF);
+        rec[5] = (uint8_t)(nstep16 >> 8);
+        for (int t = 0; t < blk; ++t) {
+            int q;
+            if (side_in) {
+                const uint8_t by = side_in[bi * R + 8 + d / 2 + t / 2];
+                q = (t & 1) ? (by >> 4) : (by & 15);
+            } else if (norm_x[b0 + t] == 0.0 || nstep == 0.0) {
+                q = 0;
+            } else {
+                q = (int)std::nearbyint(norm_x[b0 + t] / nstep);
+                q = q < 1 ? 1 : (q > 15 ? 15 : q);
+            }
+            rec[8 + d / 2 + t / 2] |= (uint8_t)(q << ((t & 1) * 4));
+            n1[b0 + t] = q * nstep;
+            const double* xv = x + (b0 + t) * d;
+            for (int j = 0; j < d; ++j) u[(size_t)t * d + j] = (q == 0) ? 0.0 : sqd * xv[j] / n1[b0 + t];
+        }
+        // channel means and their 4-bit codes
+        double lo = INFINITY, hi = -INFINITY;
+        for (int j = 0; j < d; ++j) {
+            double s = 0.0;
+            for (int t = 0; t < blk; ++t) s += u[(size_t)t * d + j];
+            o[j] = s / blk;
+            o_f64[bi * d + j] = o[j];
+            lo = std::fmin(lo, o[j]);
+            hi = std::fmax(hi, o[j]);
+        }
+        uint16_t lo16 = orc_double_to_half(lo), st16 = orc_double_to_half((hi - lo) / 15.0);
+        if (side_in) {
+            lo16 = (uint16_t)(side_in[bi * R] | (side_in[bi * R + 1] << 8));
+            st16 = (uint16_t)(side_in[bi * R + 2] | (side_in[bi * R + 3] << 8));
+        }
+        const double lov = orc_half_to_double(lo16), stv = orc_half_to_double(st16);
+        rec[0] = (uint8_t)(lo16 & 0xFF);
+        rec[1] = (uint8_t)(lo16 >> 8);
+        rec[2] = (uint8_t)(st16 & 0xFF);
+        rec[3] = (uint8_t)(st16 >> 8);
+        for (int j = 0; j < d; ++j) {
+            int q;
+            if (side_in) {
+                const uint8_t by = side_in[bi * R + 8 + j / 2];
+                q = (j & 1) ? (by >> 4) : (by & 15);
+            } else if (stv == 0.0) {
+                q = 0;
+            } else {
+                q = (int)std::nearbyint((o[j] - lov) / stv);
+                q = q < 0 ? 0 : (q > 15 ? 15 : q);
+            }
+            rec[8 + j / 2] |= (uint8_t)(q << ((j & 1) * 4));
+            o_hat[bi * d + j] = (double)(float)(lov + stv * q);
+        }
+        // the shifted tokens, coded without QJL
+        for (int t = 0; t < blk; ++t) {
+            for (int j = 0; j < d; ++j) w[j] = u[(size_t)t * d + j] - o_hat[bi * d + j];
+            double nw = 0.0, gam = 0.0;
+            orc_quantize(d, b, 0, 0, delta, nullptr, centroid, threshold, w.data(), 1, codes + (b0 + t) * d, nullptr,
+                         &nw, &gam, z_out ? z_out + (b0 + t) * d : nullptr, nullptr);
+            norm_w[b0 + t] = nw;
+        }
+    }
+}
+
 }  // extern "C"
