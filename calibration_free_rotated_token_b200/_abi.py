@@ -36,6 +36,7 @@ EXPORTED = (
     "kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize", "kvq_decode_workspace",
     "kvq_decode_attend", "kvq_decode_attend_noalloc", "kvq_status", "kvq_last_error", "kvq_get_constants",
     "kvq_get_info", "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex", "kvq_probe_wait_timeout",
+    "kvq_nsn_dq_side_bytes", "kvq_nsn_dq_quantize", "kvq_nsn_dq_decode_attend",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -105,10 +106,16 @@ def load() -> ctypes.CDLL:
         L.kvq_probe_wait_timeout.argtypes = [P, U32, P]
         L.kvq_nsn_decode_attend.argtypes = [P, P, I, I, I, I, ctypes.POINTER(KvqCache), ctypes.POINTER(KvqCache),
                                             P, P, P, I64, ctypes.c_float, P, P, P, SZ, P]
+        L.kvq_nsn_dq_side_bytes.argtypes = [I]
+        L.kvq_nsn_dq_side_bytes.restype = SZ
+        L.kvq_nsn_dq_quantize.argtypes = [P, P, I, I64, I64, I, P, P, P, P]
+        L.kvq_nsn_dq_decode_attend.argtypes = [P, P, I, I, I, I, ctypes.POINTER(KvqCache), ctypes.POINTER(KvqCache),
+                                               P, P, P, I64, ctypes.c_float, P, P, P, SZ, P]
         for name in ("kvq_init", "kvq_destroy", "kvq_quantize", "kvq_quantize_batch", "kvq_nsn_quantize",
                      "kvq_decode_attend",
                      "kvq_decode_attend_noalloc", "kvq_status", "kvq_get_constants", "kvq_get_info",
-                     "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex", "kvq_probe_wait_timeout"):
+                     "kvq_codebook", "kvq_nsn_decode_attend", "kvq_decode_attend_ex", "kvq_probe_wait_timeout",
+                     "kvq_nsn_dq_quantize", "kvq_nsn_dq_decode_attend"):
             getattr(L, name).restype = I
         _lib = L
         return L
@@ -280,6 +287,26 @@ def kvq_nsn_quantize(h: Handle, x: torch.Tensor, codes, norms, block_mean, strea
                                    _ptr(block_mean), _stream(stream)))
 
 
+def kvq_nsn_dq_side_bytes(d: int) -> int:
+    """Bytes of one side record of the double-quantized NSN front end (0 for an unsupported d)."""
+    return int(load().kvq_nsn_dq_side_bytes(d))
+
+
+def kvq_nsn_dq_quantize(h: Handle, x: torch.Tensor, codes, wnorms, side, stream=None,
+                        layout: int = KVQ_LAYOUT_TOKEN):
+    """x: [n_heads, n_tok, d] fp16/bf16, n_tok % 128 == 0; wnorms fp16 [n_heads * n_tok];
+    side uint8 [n_heads * n_tok/128, kvq_nsn_dq_side_bytes(d)]."""
+    if x.dim() != 3 or x.shape[-1] != h.d:
+        raise ValueError(f"x must be [heads, tokens, {h.d}]")
+    _need(x, "x")
+    H, T, _ = x.shape
+    _need(codes, "codes", numel=H * T * h.b * h.d // 32)
+    _need(wnorms, "wnorms", dtype=torch.float16, numel=H * T)
+    _need(side, "side", dtype=torch.uint8, numel=H * (T // 128) * kvq_nsn_dq_side_bytes(h.d))
+    _check(load().kvq_nsn_dq_quantize(h.ptr, _ptr(x), _DTYPES[x.dtype], H, T, layout, _ptr(codes), _ptr(wnorms),
+                                      _ptr(side), _stream(stream)))
+
+
 def kvq_decode_workspace(h: Handle, batch: int, hq: int, hkv: int, max_T: int) -> int:
     return int(load().kvq_decode_workspace(h.ptr, batch, hq, hkv, max_T))
 
@@ -330,6 +357,30 @@ def kvq_nsn_decode_attend(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache
                                         ctypes.byref(vcache), _ptr(k_block_mean), _ptr(v_block_mean),
                                         _ptr(seq_len), max_T, float(scale), _ptr(logits), _ptr(out),
                                         _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def kvq_nsn_dq_decode_attend(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vcache: KvqCache,
+                             k_side: torch.Tensor, v_side: torch.Tensor, seq_len: torch.Tensor, max_T: int,
+                             scale: float, out: torch.Tensor, workspace: torch.Tensor,
+                             logits: torch.Tensor | None = None, stream=None):
+    """kvq_decode_attend over caches from kvq_nsn_dq_quantize (norms = fp16 ||w|| per token; side
+    records uint8 [streams, capacity/128, kvq_nsn_dq_side_bytes(d)])."""
+    if q.dim() != 3 or q.shape[-1] != h.d:
+        raise ValueError(f"q must be [batch, hq, {h.d}]")
+    _need(q, "q")
+    B, hq, _ = q.shape
+    _need(seq_len, "seq_len", dtype=torch.int32, numel=B)
+    _need(out, "out", dtype=torch.float32, numel=B * hq * h.d)
+    _need(workspace, "workspace")
+    _need(k_side, "k_side", dtype=torch.uint8)
+    _need(v_side, "v_side", dtype=torch.uint8)
+    if logits is not None:
+        _need(logits, "logits", dtype=torch.float32, numel=B * hq * max_T)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(load().kvq_nsn_dq_decode_attend(h.ptr, _ptr(q), _DTYPES[q.dtype], B, hq, hkv, ctypes.byref(kcache),
+                                           ctypes.byref(vcache), _ptr(k_side), _ptr(v_side), _ptr(seq_len), max_T,
+                                           float(scale), _ptr(logits), _ptr(out), _ptr(workspace), ws_bytes,
+                                           _stream(stream)))
 
 
 def kvq_decode_attend_ex(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache, vcache: KvqCache,

@@ -282,7 +282,7 @@ int check_job(kvq_handle h, const QJob& j, bool nsn, CUtensorMap* map) {
 // One launch over one stream (j1 == nullptr) or two streams of the same
 // dtype (the tensor-core kernel's tiles of j0, then those of j1).
 int launch_jobs(kvq_handle h, const QJob& j0, const CUtensorMap& m0, const QJob* j1, const CUtensorMap* m1,
-                uint16_t* block_mean, bool nsn, void* stream) {
+                uint16_t* block_mean, bool nsn, void* stream, uint8_t* side = nullptr) {
     kvq::QuantArgs a{};
     a.n = j0.rows;
     a.layout = j0.layout;
@@ -300,6 +300,7 @@ int launch_jobs(kvq_handle h, const QJob& j0, const CUtensorMap& m0, const QJob*
         a.norms1 = reinterpret_cast<__half2*>(j1->norms);
     }
     a.block_mean = reinterpret_cast<__half*>(block_mean);
+    a.side = side;
     a.S = h->d_S;
     a.status = h->d_status;
     fill_common(h, a.centroid, a.threshold, a.pair_sign);
@@ -315,14 +316,18 @@ int launch_jobs(kvq_handle h, const QJob& j0, const CUtensorMap& m0, const QJob*
 }
 
 int quantize_common(kvq_handle h, const void* x, int dtype, int64_t rows, int64_t ld, int layout, uint32_t* codes,
-                    uint32_t* qjl, uint16_t* norms, uint16_t* block_mean, bool nsn, void* stream) {
+                    uint32_t* qjl, uint16_t* norms, uint16_t* block_mean, bool nsn, void* stream,
+                    uint8_t* side = nullptr) {
     if (int e = check_handle(h)) return e;
     const QJob j{x, dtype, rows, ld, layout, codes, qjl, norms};
     CUtensorMap map;
     if (int e = check_job(h, j, nsn, &map)) return e;
     if (rows == 0) return KVQ_OK;
-    return launch_jobs(h, j, map, nullptr, nullptr, block_mean, nsn, stream);
+    return launch_jobs(h, j, map, nullptr, nullptr, block_mean, nsn, stream, side);
 }
+
+// Bytes of one side record of the double-quantized NSN front end (d = 64, 128).
+size_t dq_side_bytes(int d) { return static_cast<size_t>((8 + d / 2 + 64 + 15) / 16 * 16); }
 
 }  // namespace
 
@@ -466,6 +471,25 @@ int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, in
                            stream);
 }
 
+size_t kvq_nsn_dq_side_bytes(int d) { return (d == 64 || d == 128) ? dq_side_bytes(d) : 0; }
+
+int kvq_nsn_dq_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, int layout,
+                        uint32_t* codes, uint16_t* wnorms, uint8_t* side, void* stream) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "the NSN front end takes a handle without KVQ_QJL");
+    if (n_heads < 0 || n_tok < 0) return fail(KVQ_EINVAL, "negative size");
+    if (n_tok % 128 != 0) return fail(KVQ_EINVAL, "n_tok must be a multiple of 128 (NSN blocks of 128 tokens)");
+    if (h->d > 128) return fail(KVQ_EUNSUPPORTED, "the NSN front end is built for d <= 128");
+    if (dtype != KVQ_F16 && dtype != KVQ_BF16)
+        return fail(dtype == KVQ_F32 ? KVQ_EUNSUPPORTED : KVQ_EINVAL,
+                    "double-quantized NSN side data are built for fp16 and bf16 input");
+    if (n_heads * n_tok == 0) return KVQ_OK;
+    if (!side || !aligned(side, 16)) return fail(KVQ_EINVAL, "side must be non-null and 16-byte aligned");
+    return quantize_common(h, x, dtype, n_heads * n_tok, h->d, layout, codes, nullptr, wnorms, nullptr, true,
+                           stream, side);
+}
+
 size_t kvq_decode_workspace(kvq_handle h, int batch, int hq, int hkv, int64_t max_T) {
     if (!h || batch <= 0 || hq <= 0 || hkv <= 0 || max_T < 0) return 0;
     int ns = 0;
@@ -515,6 +539,7 @@ int decode_check(kvq_handle h, int dtype, int batch, int hq, int hkv, const kvq_
 // Optional parts of a decode call: NSN block means, a residual window, the
 // logits row stride.
 struct DecodeExtras {
+    bool dq = false;  // kmean / vmean are double-quantized side records; norms hold fp16 ||w||
     const uint16_t* kmean = nullptr;
     const uint16_t* vmean = nullptr;
     const uint16_t* kwin = nullptr;
@@ -530,6 +555,7 @@ int decode_launch(kvq_handle h, const void* q, int dtype, int batch, int hq, int
                   const DecodeExtras& x = DecodeExtras()) {
     kvq::DecodeArgs a{};
     a.nsn = x.kmean != nullptr;
+    a.nsn_dq = x.dq ? 1 : 0;
     a.kmean = reinterpret_cast<const __half*>(x.kmean);
     a.vmean = reinterpret_cast<const __half*>(x.vmean);
     a.kwin = reinterpret_cast<const __half*>(x.kwin);
@@ -628,6 +654,34 @@ int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int
     DecodeExtras x;
     x.kmean = k_block_mean;
     x.vmean = v_block_mean;
+    return decode_launch(h, q, dtype, batch, hq, hkv, k, v, seq_len, max_T, scale, logits, out, workspace, ns, chunk,
+                         stream, x);
+}
+
+int kvq_nsn_dq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
+                             const kvq_cache* v, const uint8_t* k_side, const uint8_t* v_side, const int32_t* seq_len,
+                             int64_t max_T, float scale, float* logits, float* out, void* workspace, size_t ws_bytes,
+                             void* stream) {
+    g_err.clear();
+    if (int e = check_handle(h)) return e;
+    if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
+    if (!kvq::decode_uses_mma(h) || h->d > 128)
+        return fail(KVQ_EUNSUPPORTED, "decode over double-quantized NSN caches is built for d <= 128 and b <= 3");
+    int ns = 0;
+    int64_t chunk = 0;
+    size_t need = 0;
+    if (int e = decode_check(h, dtype, batch, hq, hkv, k, v, q, seq_len, max_T, scale, out, &ns, &chunk, &need))
+        return e;
+    if (k->capacity % 128 != 0 || v->capacity % 128 != 0)
+        return fail(KVQ_EINVAL, "NSN cache capacities must be multiples of 128 (one side record per 128 tokens)");
+    if (!k_side || !v_side || !aligned(k_side, 16) || !aligned(v_side, 16))
+        return fail(KVQ_EINVAL, "side records must be non-null and 16-byte aligned");
+    if (!workspace || !aligned(workspace, 16)) return fail(KVQ_EINVAL, "workspace must be non-null and 16-byte aligned");
+    if (ws_bytes < need) return fail(KVQ_EINVAL, "workspace too small: need " + std::to_string(need) + " bytes");
+    DecodeExtras x;
+    x.dq = true;
+    x.kmean = reinterpret_cast<const uint16_t*>(k_side);
+    x.vmean = reinterpret_cast<const uint16_t*>(v_side);
     return decode_launch(h, q, dtype, batch, hq, hkv, k, v, seq_len, max_T, scale, logits, out, workspace, ns, chunk,
                          stream, x);
 }

@@ -35,6 +35,7 @@
 //   the running-max rescale).
 // * Every mbarrier wait is bounded; all threads take the same decision.
 #include <cfloat>
+#include <type_traits>
 
 #include "kvq_internal.h"
 #include "sm100.cuh"
@@ -325,10 +326,18 @@ __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__
     }
 }
 
+// Bytes of one block's side record of a double-quantized NSN cache: fp16
+// offset, step and norm step, 4-bit codes of the D block means and of the 128
+// token norms, padded to a multiple of 16 bytes.
+__host__ __device__ constexpr int dq_rec_bytes(int D) { return (8 + D / 2 + 64 + 15) / 16 * 16; }
+
 // Shared-memory plan of the split kernel.  NSN: caches written by the NSN
 // front end (no QJL), whose stages also carry the fp16 block means of keys
-// and values (one D-vector per 128 tokens).
-template <int D, int B, bool QJL, int G, bool NSN = false>
+// and values (one D-vector per 128 tokens).  DQ (with NSN): the caches hold
+// fp16 ||w|| per token and one side record per 128 tokens instead; the stage
+// carries them as stored, and each sub-chunk expands them into fp32 norms
+// (n1, ||w||) per token and fp32 block means in the expansion area.
+template <int D, int B, bool QJL, int G, bool NSN = false, bool DQ = false>
 struct MmaSmem {
     static constexpr int M = D;
     static constexpr int TC = DTile<D>::TC;
@@ -339,25 +348,29 @@ struct MmaSmem {
     // staging of one sub-chunk
     static constexpr int kKc = TC * B * D / 8;             // key codes (token layout)
     static constexpr int kKq = QJL ? TC * M / 8 : 0;       // key sign bits
-    static constexpr int kKn = TC * 4;                     // key norms
+    static constexpr int kKn = DQ ? TC * 2 : TC * 4;       // key norms
     static constexpr int kVc = (TC / 32) * B * D * 4;      // value codes (block-32)
     static constexpr int kVq = QJL ? (TC / 32) * M * 4 : 0;
-    static constexpr int kVn = TC * 4;
-    static constexpr int kKm = NSN ? ((TC + 127) / 128) * D * 2 : 0;  // key block means
-    static constexpr int kVm = kKm;                                    // value block means
+    static constexpr int kVn = kKn;
+    static constexpr int kNblk = (TC + 127) / 128;
+    static constexpr int kKm = NSN ? kNblk * (DQ ? dq_rec_bytes(D) : D * 2) : 0;  // key block means
+    static constexpr int kVm = kKm;                                                // value block means
     static constexpr int kStage = kKc + kKq + kKn + kVc + kVq + kVn + kKm + kVm;
+    static constexpr int kXp = DQ ? 2 * TC * 8 + 2 * kNblk * D * 4 : 0;           // DQ expansion area
     static constexpr int kFrag = KS * NTK * 32 * 8;        // query fragments
     static constexpr int kLog = GP * TC * 4;               // logits of the sub-chunk
     static constexpr int kWfrag = (TC / 32) * RT * 32 * 16;  // weight digits, per kind
     static constexpr int kMisc = NSN ? 1536 : 1024;
-    static constexpr int kBytes = 2 * kStage + kFrag + kLog + 2 * kWfrag + kMisc;
+    static constexpr int kBytes = 2 * kStage + kFrag + kLog + 2 * kWfrag + kMisc + kXp;
     static constexpr bool kQfReg = KS * NTK <= 24;         // query fragments held in registers
 };
 
-template <int D, int B, bool QJL, int G, bool NSN = false>
+template <int D, int B, bool QJL, int G, bool NSN = false, bool DQ = false>
 __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_constant__ DecodeArgs a) {
     static_assert(!(NSN && QJL), "NSN caches carry no QJL sketch");
-    using L = MmaSmem<D, B, QJL, G, NSN>;
+    static_assert(!DQ || NSN, "double-quantized side data belong to NSN caches");
+    using L = MmaSmem<D, B, QJL, G, NSN, DQ>;
+    constexpr int RB = dq_rec_bytes(D);
     using HC = HeadCfg<G>;
     constexpr int M = D, TC = L::TC, NTK = L::NTK, RT = L::RT, KS = L::KS, GP = L::GP, CPL = HC::CPL;
     constexpr int KWT = B * D / 32;           // code words per token (key layout)
@@ -380,6 +393,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     float* sstat = shead + GP * 8;                           // [GP][8]: -, alpha, sig_w/128, sig_wq/128
     float* sqo = sstat + GP * 8;                             // NSN: [GP][2] scale/sqrt(d) <q, o_k> per block
     float* sbeta = sqo + GP * 2;                             // NSN: [4 warps][GP][2] sums of e ||x||/sqrt(d)
+    // DQ: per sub-chunk, (n1, ||w||) per token and the block means, in fp32
+    float2* xkn = reinterpret_cast<float2*>(misc + L::kMisc);
+    float2* xvn = xkn + (DQ ? L::TC : 0);
+    float* xkm = reinterpret_cast<float*>(xvn + (DQ ? L::TC : 0));
+    float* xvm = xkm + (DQ ? L::kNblk * D : 0);
     const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
@@ -408,13 +426,15 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
         const int64_t qh0 = static_cast<int64_t>(bi) * a.hq + static_cast<int64_t>(hk) * G;
         const uint8_t* kc = reinterpret_cast<const uint8_t*>(a.kcodes) + stream * a.kcap * (B * D / 8);
         const uint8_t* kq = QJL ? reinterpret_cast<const uint8_t*>(a.kqjl) + stream * a.kcap * (M / 8) : nullptr;
-        const uint8_t* kn = reinterpret_cast<const uint8_t*>(a.knorms) + stream * a.kcap * 4;
+        constexpr int NB = DQ ? 2 : 4;  // norm bytes per token
+        const uint8_t* kn = reinterpret_cast<const uint8_t*>(a.knorms) + stream * a.kcap * NB;
         const uint8_t* vc = reinterpret_cast<const uint8_t*>(a.vcodes) + stream * (a.vcap / 32) * B * D * 4;
         const uint8_t* vq = QJL ? reinterpret_cast<const uint8_t*>(a.vqjl) + stream * (a.vcap / 32) * M * 4 : nullptr;
-        const uint8_t* vn = reinterpret_cast<const uint8_t*>(a.vnorms) + stream * a.vcap * 4;
-        // NSN: block means, [capacity / 128][D] fp16 per stream
-        const uint8_t* km = NSN ? reinterpret_cast<const uint8_t*>(a.kmean) + stream * (a.kcap / 128) * D * 2 : nullptr;
-        const uint8_t* vm = NSN ? reinterpret_cast<const uint8_t*>(a.vmean) + stream * (a.vcap / 128) * D * 2 : nullptr;
+        const uint8_t* vn = reinterpret_cast<const uint8_t*>(a.vnorms) + stream * a.vcap * NB;
+        // NSN: block means, [capacity / 128][D] fp16 per stream (DQ: side records of RB bytes)
+        constexpr int MB = DQ ? RB : D * 2;  // bytes per block
+        const uint8_t* km = NSN ? reinterpret_cast<const uint8_t*>(a.kmean) + stream * (a.kcap / 128) * MB : nullptr;
+        const uint8_t* vm = NSN ? reinterpret_cast<const uint8_t*>(a.vmean) + stream * (a.vcap / 128) * MB : nullptr;
 
         // ---- item set-up (the previous item is done with shared memory) ----
         __syncthreads();
@@ -469,24 +489,24 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             uint8_t* st = smem + (sc & 1) * L::kStage;
             uint64_t* b = &bar[sc & 1];
             const int64_t nblk = NSN ? (nt + 127) / 128 : 0;  // block means of the sub-chunk
-            const uint32_t bytes = static_cast<uint32_t>(nt * (B * D / 8 + (QJL ? M / 8 : 0) + 4) +
-                                                         (nt / 32) * (B * D * 4 + (QJL ? M * 4 : 0)) + nt * 4 +
-                                                         2 * nblk * D * 2);
+            const uint32_t bytes = static_cast<uint32_t>(nt * (B * D / 8 + (QJL ? M / 8 : 0) + NB) +
+                                                         (nt / 32) * (B * D * 4 + (QJL ? M * 4 : 0)) + nt * NB +
+                                                         2 * nblk * MB);
             mbar_arrive_expect_tx(b, bytes);
             bulk_load(st, kc + tb * (B * D / 8), static_cast<uint32_t>(nt * (B * D / 8)), b);
             if (QJL) bulk_load(st + L::kKc, kq + tb * (M / 8), static_cast<uint32_t>(nt * (M / 8)), b);
-            bulk_load(st + L::kKc + L::kKq, kn + tb * 4, static_cast<uint32_t>(nt * 4), b);
+            bulk_load(st + L::kKc + L::kKq, kn + tb * NB, static_cast<uint32_t>(nt * NB), b);
             bulk_load(st + L::kKc + L::kKq + L::kKn, vc + (tb / 32) * B * D * 4,
                       static_cast<uint32_t>((nt / 32) * B * D * 4), b);
             if (QJL)
                 bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc, vq + (tb / 32) * M * 4,
                           static_cast<uint32_t>((nt / 32) * M * 4), b);
-            bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq, vn + tb * 4, static_cast<uint32_t>(nt * 4),
+            bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq, vn + tb * NB, static_cast<uint32_t>(nt * NB),
                       b);
             if (NSN) {
-                const uint32_t mb = static_cast<uint32_t>(nblk * D * 2);
-                bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq + L::kVn, km + (tb / 128) * D * 2, mb, b);
-                bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq + L::kVn + L::kKm, vm + (tb / 128) * D * 2,
+                const uint32_t mb = static_cast<uint32_t>(nblk * MB);
+                bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq + L::kVn, km + (tb / 128) * MB, mb, b);
+                bulk_load(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq + L::kVn + L::kKm, vm + (tb / 128) * MB,
                           mb, b);
             }
             return true;
@@ -532,6 +552,39 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             const __half2* sVn = reinterpret_cast<const __half2*>(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq);
             const __half* sKm = reinterpret_cast<const __half*>(st + L::kKc + L::kKq + L::kKn + L::kVc + L::kVq + L::kVn);
             const __half* sVm = sKm + L::kKm / 2;
+            if constexpr (DQ) {
+                // Expand the sub-chunk's stored side data: n1 = q nstep and ||w|| per token,
+                // o_hat = fp32(lo + step q) per block and channel (keys and values).
+                const uint8_t* rk = reinterpret_cast<const uint8_t*>(sKm);
+                const uint8_t* rv = rk + L::kKm;
+                const __half* wk = reinterpret_cast<const __half*>(sKn);
+                const __half* wv = reinterpret_cast<const __half*>(sVn);
+                auto f16at = [](const uint8_t* p) { return __half2float(*reinterpret_cast<const __half*>(p)); };
+                for (int tl = tid; tl < L::TC; tl += kThreads) {
+                    const int bi = tl >> 7, tt = tl & 127;
+                    const uint8_t* hk = rk + bi * RB;
+                    const uint8_t* hv = rv + bi * RB;
+                    const int qk = (hk[8 + D / 2 + tt / 2] >> ((tt & 1) * 4)) & 15;
+                    const int qv2 = (hv[8 + D / 2 + tt / 2] >> ((tt & 1) * 4)) & 15;
+                    xkn[tl] = make_float2(static_cast<float>(qk) * f16at(hk + 4), __half2float(wk[tl]));
+                    xvn[tl] = make_float2(static_cast<float>(qv2) * f16at(hv + 4), __half2float(wv[tl]));
+                }
+                for (int e = tid; e < L::kNblk * D; e += kThreads) {
+                    const int bi = e / D, j = e % D;
+                    const uint8_t* hk = rk + bi * RB;
+                    const uint8_t* hv = rv + bi * RB;
+                    const int qk = (hk[8 + j / 2] >> ((j & 1) * 4)) & 15;
+                    const int qv2 = (hv[8 + j / 2] >> ((j & 1) * 4)) & 15;
+                    xkm[e] = fmaf(f16at(hk + 2), static_cast<float>(qk), f16at(hk));
+                    xvm[e] = fmaf(f16at(hv + 2), static_cast<float>(qv2), f16at(hv));
+                }
+                __syncthreads();
+            }
+            // stored norms (||x|| or n1, then ||r|| or ||w||) and block means, as fp32
+            auto knorm = [&](int tl) -> float2 { return DQ ? xkn[tl] : __half22float2(sKn[tl]); };
+            auto vnorm = [&](int tl) -> float2 { return DQ ? xvn[tl] : __half22float2(sVn[tl]); };
+            auto kmean = [&](int i) -> float { return DQ ? xkm[i] : __half2float(sKm[i]); };
+            auto vmean = [&](int i) -> float { return DQ ? xvm[i] : __half2float(sVm[i]); };
             if constexpr (NSN) {
                 // scale/sqrt(d) <q_h, o_k> for each 128-token block of the sub-chunk
                 // (an unloaded block gives a value no valid token uses)
@@ -542,7 +595,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                         float acc = 0.f;
 #pragma unroll
                         for (int i = 0; i < D / 32; ++i)
-                            acc = fmaf(qv[qq][i], __half2float(sKm[blk * D + lane + 32 * i]), acc);
+                            acc = fmaf(qv[qq][i], kmean(blk * D + lane + 32 * i), acc);
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
                         const int h = warp + 4 * qq;
@@ -645,7 +698,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                                                   16384.f,
                                                   static_cast<float>((accc[0][n1][2 * rr] + accc[1][n1][2 * rr]) * 128 +
                                                                      accc[0][n1][2 * rr + 1] + accc[1][n1][2 * rr + 1]));
-                            const float2 nk = __half22float2(sKn[tl]);
+                            const float2 nk = knorm(tl);
                             float inner = fmaf(hk1[hh], xc, hk0[hh]);
                             if (QJL) {
                                 const float xq =
@@ -671,7 +724,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                 float nmx = 0.f, ngx = 0.f;
                 for (int tl = tid; tl < TC; tl += kThreads) {
                     if (tl < nval) {
-                        const float2 nv = __half22float2(sVn[tl]);
+                        const float2 nv = vnorm(tl);
                         nmx = fmaxf(nmx, NSN ? nv.x * nv.y * inv_sqrt_d : nv.x);
                         ngx = fmaxf(ngx, nv.x * nv.y);
                     }
@@ -746,7 +799,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             // (r>>3) + 2((u&7)>>2), byte u>>3 of row r's fragment.
             for (int tl = tid; tl < TC; tl += kThreads) {
                 const bool valid = tl < nval;
-                const float2 nv = valid ? __half22float2(sVn[tl]) : make_float2(0.f, 0.f);
+                const float2 nv = valid ? vnorm(tl) : make_float2(0.f, 0.f);
                 const int u = tl & 31, bb = tl >> 5, s = u & 7;
                 const float fac = static_cast<float>(1 << (7 - s));
                 uint8_t* bc = reinterpret_cast<uint8_t*>(swc) + (u >> 3);
@@ -918,7 +971,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                                         float bsum = 0.f;
 #pragma unroll
                                         for (int w = 0; w < 4; ++w) bsum += sbeta[(w * GP + head) * 2 + blk];
-                                        add = fmaf(bsum, __half2float(sVm[blk * D + coord]), add);
+                                        add = fmaf(bsum, vmean(blk * D + coord), add);
                                     }
                                 }
                                 accB[nt][c] = fmaf(accB[nt][c], alpha, add);
@@ -1004,10 +1057,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     }
 }
 
-template <int D, int B, bool QJL, int G, bool NSN = false>
+template <int D, int B, bool QJL, int G, bool NSN = false, bool DQ = false>
 int ctas_per_sm_g() {
-    using L = MmaSmem<D, B, QJL, G, NSN>;
-    auto kern = decode_mma_kernel<D, B, QJL, G, NSN>;
+    using L = MmaSmem<D, B, QJL, G, NSN, DQ>;
+    auto kern = decode_mma_kernel<D, B, QJL, G, NSN, DQ>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess) return 1;
     int n = 1;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, L::kBytes) != cudaSuccess || n < 1) n = 1;
@@ -1035,19 +1088,24 @@ cudaError_t launch_mma_g(const DecodeArgs& a, int grid, cudaStream_t s) {
     const int64_t items = static_cast<int64_t>(a.batch) * a.hkv * a.nsplit_run;
     if constexpr (!QJL) {
         if (a.nsn) {
-            // NSN caches: the same split plan, on this variant's own persistent grid
-            using LN = MmaSmem<D, B, false, G, true>;
-            auto kn = decode_mma_kernel<D, B, false, G, true>;
-            cudaError_t e = cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, LN::kBytes);
-            if (e != cudaSuccess) return e;
-            int sms = 148, dev = 0;
-            cudaGetDevice(&dev);
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            const int64_t gn = static_cast<int64_t>(ctas_per_sm_g<D, B, false, G, true>()) * sms;
-            const int64_t n = items < gn ? items : gn;
-            if (n <= 0) return cudaSuccess;
-            kn<<<static_cast<unsigned>(n), kThreads, LN::kBytes, s>>>(a);
-            return cudaGetLastError();
+            // NSN caches (fp16 or double-quantized side data): the same split
+            // plan, on the variant's own persistent grid
+            auto run = [&](auto dq) -> cudaError_t {
+                constexpr bool DQ = decltype(dq)::value;
+                using LN = MmaSmem<D, B, false, G, true, DQ>;
+                auto kn = decode_mma_kernel<D, B, false, G, true, DQ>;
+                cudaError_t e = cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, LN::kBytes);
+                if (e != cudaSuccess) return e;
+                int sms = 148, dev = 0;
+                cudaGetDevice(&dev);
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+                const int64_t gn = static_cast<int64_t>(ctas_per_sm_g<D, B, false, G, true, DQ>()) * sms;
+                const int64_t n = items < gn ? items : gn;
+                if (n <= 0) return cudaSuccess;
+                kn<<<static_cast<unsigned>(n), kThreads, LN::kBytes, s>>>(a);
+                return cudaGetLastError();
+            };
+            return a.nsn_dq ? run(std::true_type()) : run(std::false_type());
         }
     }
     using L = MmaSmem<D, B, QJL, G>;

@@ -46,6 +46,7 @@ struct QuantArgs {
     uint32_t* qjl;                    // [n][d/32] or null
     __half2* norms;                   // [n]
     __half* block_mean;               // NSN: [n/128][d]
+    uint8_t* side;                    // NSN with double quantization: one side record per 128 rows (else null)
     const __half* S;                  // [m][d] fp16 (global), copied to smem per CTA
     uint32_t* status;
     float centroid[kMaxLevels];
@@ -103,6 +104,9 @@ struct DecodeArgs {
     int nsn;
     const __half* kmean;
     const __half* vmean;
+    // NSN caches with double-quantized side data: the norms arrays hold fp16
+    // ||w|| per token and kmean / vmean point at the side records.
+    int nsn_dq;
     // Splits over the packed cache (nsplit counts one more when a window is
     // attended: its partial is split nsplit - 1); row stride of `logits`.
     int nsplit_run;

@@ -26,6 +26,14 @@ cudaError_t by_dtype(const CUtensorMap& map, const CUtensorMap& map1, int dtype,
     if constexpr (NSN && (QJL || D > 128)) {
         return cudaErrorNotSupported;
     } else if constexpr (NSN) {
+        // double-quantized side data (a.side): 16-bit input only
+        if (a.side != nullptr) {
+            switch (dtype) {
+                case DT_F16: return launch_quantize_tc<D, B, false, DT_F16, true, true>(map, map1, a, sms, s);
+                case DT_BF16: return launch_quantize_tc<D, B, false, DT_BF16, true, true>(map, map1, a, sms, s);
+                default: return cudaErrorNotSupported;
+            }
+        }
         switch (dtype) {
             case DT_F32: return launch_quantize_t<D, B, false, DT_F32, true>(map, a, sms, s);
             case DT_F16: return launch_quantize_tc<D, B, false, DT_F16, true>(map, map1, a, sms, s);

@@ -60,14 +60,234 @@ struct TcCfg {
     static_assert(kStages >= kWG, "one stage per warpgroup at least");
 };
 
-// Sign word of 32 accumulator values: bit i = [u_i >= 0].
+// Column order of the rotated vector and of the residual in tensor memory.
+// Within each group of 32 columns, column 32c + 2i + e holds coordinate
+// 32c + i + 16e (i < 16, e in {0, 1}).  A register pair (2i, 2i + 1) of a
+// 32-column load then holds coordinates i and i + 16 of the group, so the
+// packed fp32x2 operations act on the two 16-bit halves of a packed word and
+// every plane word is two 16-bit chains joined by one byte permute.  The
+// rotation matrix's rows and the residual's K order (S's columns) follow the
+// same permutation, so the products are unchanged.
+__host__ __device__ constexpr int col_coord(int col) { return (col & ~31) + ((col & 31) >> 1) + ((col & 1) << 4); }
+
+// Sign word of 32 accumulator values: bit i = [u_i >= 0] (two 16-bit chains).
 __device__ __forceinline__ uint32_t sign_word(const uint32_t (&u)[32]) {
-    uint32_t b[4] = {0, 0, 0, 0};
+    uint32_t lo = 0, hi = 0;
 #pragma unroll
-    for (int i = 7; i >= 0; --i)
+    for (int i = 15; i >= 0; --i) {
+        lo = __funnelshift_l(u[i], lo, 1);
+        hi = __funnelshift_l(u[16 + i], hi, 1);
+    }
+    return ~__byte_perm(lo, hi, 0x5410);
+}
+
+// Per-lane constants of the 32 x 32 bit transpose (bit_transpose32).
+struct Transpose32 {
+    uint32_t sel16, sel8;      // byte selectors of the 16- and 8-bit stages
+    uint32_t rot[3], keep[3];  // rotate amount and kept-bit mask of the 4-, 2- and 1-bit stages
+    __device__ __forceinline__ explicit Transpose32(int lane) {
+        sel16 = (lane & 16) ? 0x3276u : 0x5410u;
+        sel8 = (lane & 8) ? 0x3715u : 0x6240u;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) b[q] = __funnelshift_l(u[8 * q + i], b[q], 1);
-    return ~(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24));
+        for (int k = 0; k < 3; ++k) {
+            const int s = 4 >> k;
+            const uint32_t m = k == 0 ? 0x0F0F0F0Fu : (k == 1 ? 0x33333333u : 0x55555555u);
+            const bool hi = (lane & s) != 0;
+            rot[k] = hi ? 32u - s : static_cast<uint32_t>(s);
+            keep[k] = hi ? ~m : m;
+        }
+    }
+};
+
+// 32 x 32 bit transpose across the warp: lane i enters with row i (bit j =
+// column j) and leaves with column i (bit j = row j).  Each of the five
+// stages swaps the off-diagonal s x s blocks with the partner lane i ^ s:
+// one shuffle, then a byte permute (s = 16, 8) or a rotate and a bit select
+// (s = 4, 2, 1; the bits rotated around the word land in positions the
+// select does not keep).
+__device__ __forceinline__ uint32_t bit_transpose32(uint32_t x, const Transpose32& t) {
+    uint32_t y = __shfl_xor_sync(0xFFFFFFFFu, x, 16);
+    x = __byte_perm(x, y, t.sel16);
+    y = __shfl_xor_sync(0xFFFFFFFFu, x, 8);
+    x = __byte_perm(x, y, t.sel8);
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        y = __shfl_xor_sync(0xFFFFFFFFu, x, 4 >> k);
+        const uint32_t r = __funnelshift_l(y, y, t.rot[k]);
+        x = (x & t.keep[k]) | (r & ~t.keep[k]);
+    }
+    return x;
+}
+
+// Block-32 store of NW words per lane (lane = vector of the block of 32):
+// lane i writes the transposed word of coordinate (or QJL row) 32w + i.
+template <int NW>
+__device__ __forceinline__ void store_block32_t(uint32_t* dst, const uint32_t* words, uint32_t mask, int lane,
+                                                bool store) {
+    const Transpose32 t(lane);
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const uint32_t x = bit_transpose32(words[w] & mask, t);
+        if (store) dst[32 * w + lane] = x;
+    }
+}
+
+// Codebook constants of the coding pass for B bits (symmetric codebook,
+// H = 2^(B-1) levels per sign): the positive decision levels tau_1..tau_{H-1}
+// (tau_j = t[H-1+j]) and the centroid magnitudes mu_0..mu_{H-1}.  The
+// magnitude index idx = #{j : |z| >= tau_j} is found by a binary search
+// whose bit at each level is s = sat(g * K + 1) with g = |y| - (level) * n:
+// exactly 0 or 1, since a nonzero g is at least |y| 2^-24 (the two terms are
+// within a factor of two near a level) and K = 2^40 / n.  The level of the
+// next step and mu_idx are multilinear in the bits found, so they are fused
+// multiply-adds on the FMA pipe (no branch, select or indexed load).
+template <int B>
+struct CodeTab {
+    static constexpr int H = 1 << (B - 1);
+    float lev[H > 1 ? H - 1 : 1];  // multilinear coefficients of the levels (times n per vector)
+    float mu[H];                   // multilinear coefficients of mu_idx
+    __device__ __forceinline__ explicit CodeTab(const QuantArgs& a) {
+        float tau[H], m[H];
+#pragma unroll
+        for (int j = 0; j < H; ++j) {
+            tau[j] = j > 0 ? a.threshold[H - 1 + j] : 0.f;
+            m[j] = a.centroid[H + j];
+        }
+        if constexpr (B == 1) {
+            lev[0] = 0.f;
+            mu[0] = m[0];
+        } else if constexpr (B == 2) {
+            lev[0] = tau[1];
+            mu[0] = m[0];
+            mu[1] = m[1] - m[0];
+        } else if constexpr (B == 3) {
+            lev[0] = tau[2];                              // level 1
+            lev[1] = tau[1];                              // level 2: tau_1 + s1 (tau_3 - tau_1)
+            lev[2] = tau[3] - tau[1];
+            mu[0] = m[0];                                 // mu = s0 (s1 X + a1) + (s1 (m2 - m0) + m0)
+            mu[1] = m[1] - m[0];
+            mu[2] = m[2] - m[0];
+            mu[3] = m[3] - m[2] - m[1] + m[0];
+        } else {
+            lev[0] = tau[4];                              // level 1
+            lev[1] = tau[2];                              // level 2: tau_2 + s2 (tau_6 - tau_2)
+            lev[2] = tau[6] - tau[2];
+            lev[3] = tau[1];                              // level 3: tau_1 + s1 (tau_3 - tau_1)
+            lev[4] = tau[3] - tau[1];                     //   + s2 (tau_5 - tau_1) + s1 s2 X
+            lev[5] = tau[5] - tau[1];
+            lev[6] = tau[7] - tau[5] - tau[3] + tau[1];
+            // mu = s0 A(s1, s2) + Bv(s1, s2), A and Bv bilinear
+            mu[0] = m[0];
+            mu[1] = m[2] - m[0];
+            mu[2] = m[4] - m[0];
+            mu[3] = m[6] - m[4] - m[2] + m[0];
+            const float a0 = m[1] - m[0], a2 = m[3] - m[2], a4 = m[5] - m[4], a6 = m[7] - m[6];
+            mu[4] = a0;
+            mu[5] = a2 - a0;
+            mu[6] = a4 - a0;
+            mu[7] = a6 - a4 - a2 + a0;
+        }
+    }
+};
+
+// Per-vector constants: 1/n, K = 2^40/n and the levels scaled by n.
+template <int B>
+struct VecTab {
+    float2 inv2;
+    float K;
+    float lev[CodeTab<B>::H > 1 ? CodeTab<B>::H - 1 : 1];
+    __device__ __forceinline__ VecTab(const CodeTab<B>& c, float nrm, float inv) {
+        inv2 = make_float2(inv, inv);
+        // (bounded so that a vector whose norm is below 2^-86 -- stored as an fp16
+        // norm of 0 -- cannot make it overflow)
+        K = fminf(inv * 0x1p40f, 0x1p126f);
+#pragma unroll
+        for (int j = 0; j < (CodeTab<B>::H > 1 ? CodeTab<B>::H - 1 : 1); ++j) lev[j] = c.lev[j] * nrm;
+    }
+};
+
+__device__ __forceinline__ float2 sat_bits(float2 y, float level, float K) {
+    return make_float2(__saturatef(fmaf(fabsf(y.x) - level, K, 1.0f)), __saturatef(fmaf(fabsf(y.y) - level, K, 1.0f)));
+}
+__device__ __forceinline__ float2 sat_bits2(float2 y, float2 level, float K) {
+    return make_float2(__saturatef(fmaf(fabsf(y.x) - level.x, K, 1.0f)),
+                       __saturatef(fmaf(fabsf(y.y) - level.y, K, 1.0f)));
+}
+__device__ __forceinline__ float2 f2s(float v) { return make_float2(v, v); }
+
+// Codes and residual of one 32-column group of this thread's vector.
+// v[i] = (y of coordinate i, y of coordinate 16 + i) of the group (column
+// order above); y = H D x unnormalised, n = ||x||.  Out: the B plane words of
+// the group (token layout: bit i = coordinate i of the group), the fp16
+// residual r = y/n - c[code] as 16 packed pairs (pair i = coordinates i and
+// 16 + i), and ||r||^2 accumulated into rr.
+// Plane words: the top plane is [y >= 0]; plane p < B-1 is bit p of the code,
+// which is (magnitude-index bit p) XOR (sign bit of y).
+template <int B>
+__device__ __forceinline__ void code_group(const float2 (&v)[16], const CodeTab<B>& ct, const VecTab<B>& vt,
+                                           uint32_t (&hres)[16], uint32_t (&words)[B], float2& rr) {
+    constexpr int NB = B > 1 ? B - 1 : 1;
+    uint32_t sl = 0, sh = 0;
+    float2 acc[NB];
+#pragma unroll
+    for (int p = 0; p < NB; ++p) acc[p] = make_float2(0.f, 0.f);
+    const float2 two = f2s(2.0f);
+#pragma unroll
+    for (int i = 15; i >= 0; --i) {
+        const float2 y = v[i];
+        sl = push_sign(sl, y.x);
+        sh = push_sign(sh, y.y);
+        float2 mu;
+        if constexpr (B == 1) {
+            mu = f2s(ct.mu[0]);
+        } else if constexpr (B == 2) {
+            const float2 s0 = sat_bits(y, vt.lev[0], vt.K);
+            acc[0] = __ffma2_rn(acc[0], two, s0);
+            mu = __ffma2_rn(s0, f2s(ct.mu[1]), f2s(ct.mu[0]));
+        } else if constexpr (B == 3) {
+            const float2 s1 = sat_bits(y, vt.lev[0], vt.K);
+            const float2 l2 = __ffma2_rn(s1, f2s(vt.lev[2]), f2s(vt.lev[1]));
+            const float2 s0 = sat_bits2(y, l2, vt.K);
+            acc[1] = __ffma2_rn(acc[1], two, s1);
+            acc[0] = __ffma2_rn(acc[0], two, s0);
+            const float2 hiA = __ffma2_rn(s1, f2s(ct.mu[3]), f2s(ct.mu[1]));
+            const float2 loB = __ffma2_rn(s1, f2s(ct.mu[2]), f2s(ct.mu[0]));
+            mu = __ffma2_rn(s0, hiA, loB);
+        } else {
+            const float2 s2 = sat_bits(y, vt.lev[0], vt.K);
+            const float2 l2 = __ffma2_rn(s2, f2s(vt.lev[2]), f2s(vt.lev[1]));
+            const float2 s1 = sat_bits2(y, l2, vt.K);
+            const float2 la = __ffma2_rn(s2, f2s(vt.lev[6]), f2s(vt.lev[4]));
+            const float2 lb = __ffma2_rn(s2, f2s(vt.lev[5]), f2s(vt.lev[3]));
+            const float2 l3 = __ffma2_rn(s1, la, lb);
+            const float2 s0 = sat_bits2(y, l3, vt.K);
+            acc[2] = __ffma2_rn(acc[2], two, s2);
+            acc[1] = __ffma2_rn(acc[1], two, s1);
+            acc[0] = __ffma2_rn(acc[0], two, s0);
+            const float2 ba = __ffma2_rn(s2, f2s(ct.mu[3]), f2s(ct.mu[1]));
+            const float2 bb = __ffma2_rn(s2, f2s(ct.mu[2]), f2s(ct.mu[0]));
+            const float2 bv = __ffma2_rn(s1, ba, bb);
+            const float2 aa = __ffma2_rn(s2, f2s(ct.mu[7]), f2s(ct.mu[5]));
+            const float2 ab = __ffma2_rn(s2, f2s(ct.mu[6]), f2s(ct.mu[4]));
+            const float2 av = __ffma2_rn(s1, aa, ab);
+            mu = __ffma2_rn(s0, av, bv);
+        }
+        // -c[code] = -(sign of y) mu (mu > 0): one bit select per coordinate
+        const float2 nc = make_float2(u2f(f2u(mu.x) | (~f2u(y.x) & 0x80000000u)),
+                                      u2f(f2u(mu.y) | (~f2u(y.y) & 0x80000000u)));
+        const float2 r = __ffma2_rn(y, vt.inv2, nc);
+        rr = __ffma2_rn(r, r, rr);
+        const __half2 hh = __float22half2_rn(r);
+        hres[i] = *reinterpret_cast<const uint32_t*>(&hh);
+    }
+    const uint32_t sw = __byte_perm(sl, sh, 0x5410);  // sign bits of y (1 = negative)
+    words[B - 1] = ~sw;
+#pragma unroll
+    for (int p = 0; p < B - 1; ++p) {
+        // the chains hold integers < 2^16: adding 2^23 puts them in the low mantissa bits
+        const float2 t = __fadd2_rn(acc[p], f2s(0x1p23f));
+        words[p] = __byte_perm(f2u(t.x), f2u(t.y), 0x5410) ^ sw;
+    }
 }
 
 // Sum of squares of row r of a 16-bit stage (boxes of 64 elements x 128
@@ -103,12 +323,14 @@ __device__ __forceinline__ float stage_elem(const uint8_t* sp, int t, int j) {
     return (DT == DT_BF16) ? u2f(static_cast<uint32_t>(hv) << 16) : __half2float(*reinterpret_cast<const __half*>(&hv));
 }
 
-template <int D, int B, bool QJL, int DT, bool NSN = false>
+template <int D, int B, bool QJL, int DT, bool NSN = false, bool DQ = false>
 __global__ void __launch_bounds__(512, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap map, const __grid_constant__ CUtensorMap map1,
                        const __grid_constant__ QuantArgs a) {
     static_assert(!(NSN && QJL), "NSN front end: no QJL");
+    static_assert(!DQ || NSN, "double quantization is of the NSN side data");
     using C = TcCfg<D, QJL, NSN>;
+    constexpr int RB = (8 + D / 2 + 64 + 15) / 16 * 16;  // DQ: side record bytes per block
     constexpr int NS = C::kStages;
     constexpr int kWpp = D / 32;
     constexpr uint32_t kIdescH = idesc_16bit_f32(kTileRows, D, DT == DT_BF16);
@@ -126,7 +348,7 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t* iss = reinterpret_cast<uint32_t*>(qbar + 4);  // [8] loads issued per stage
     uint32_t* con = iss + 8;                                // [8] loads consumed per stage
     uint32_t* tmem_slot = con + 8;
-    float* nsn_aux = reinterpret_cast<float*>(aux + 1024);  // NSN: [4 warpgroups][640]
+    float* nsn_aux = reinterpret_cast<float*>(aux + 1024);  // NSN: [4 warpgroups][648]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -147,21 +369,23 @@ __global__ void __launch_bounds__(512, 1)
         }
         fence_mbar_init();
     }
-    // H D as the B operand (row n = output coordinate, K = input coordinate):
-    // entry (n, k) = (-1)^popcount(n & k) delta_k.  K-chunk kc (64 entries)
-    // of row n at sHD + kc*D*128 + n*128, 16-byte chunk c at c ^ (n & 7).
+    // H D as the B operand (row n = output column n, which holds coordinate
+    // col_coord(n); K = input coordinate): entry (n, k) =
+    // (-1)^popcount(col_coord(n) & k) delta_k.  K-chunk kc (64 entries) of row
+    // n at sHD + kc*D*128 + n*128, 16-byte chunk c at c ^ (n & 7).
     {
         const uint32_t one = (DT == DT_BF16) ? 0x3F80u : 0x3C00u;
         for (int e = tid; e < D * D / 8; e += C::kThreads) {
             const int n = e / (D / 8), cc = e % (D / 8);
             const int kc = cc / 8, c16 = cc % 8;
+            const int jn = col_coord(n);
             uint32_t w4[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int k = 8 * cc + 2 * q;
                 const uint32_t ps = a.pair_sign[k >> 1];
-                const uint32_t s0 = ((__popc(n & k) & 1u) << 15) ^ (ps & 0x8000u);
-                const uint32_t s1 = ((__popc(n & (k + 1)) & 1u) << 15) ^ ((ps >> 16) & 0x8000u);
+                const uint32_t s0 = ((__popc(jn & k) & 1u) << 15) ^ (ps & 0x8000u);
+                const uint32_t s1 = ((__popc(jn & (k + 1)) & 1u) << 15) ^ ((ps >> 16) & 0x8000u);
                 w4[q] = (one | s0) | ((one | s1) << 16);
             }
             *reinterpret_cast<uint4*>(sHD + kc * (D * 128) + n * 128 + ((c16 ^ (n & 7)) << 4)) =
@@ -169,12 +393,23 @@ __global__ void __launch_bounds__(512, 1)
         }
     }
     if (QJL) {
-        // S is written once at handle creation, before any launch.
-        const uint4* gS = reinterpret_cast<const uint4*>(a.S);
+        // S (written once at handle creation, before any launch) with its
+        // columns in the residual's K order: K index kk is coordinate
+        // col_coord(kk), so 8 consecutive K entries are two runs of 4
+        // consecutive columns of S (coordinates i.. and 16 + i..).
+        const uint16_t* gS = reinterpret_cast<const uint16_t*>(a.S);
         for (int e = tid; e < D * D / 8; e += C::kThreads) {
             const int n = e / (D / 8), cc = e % (D / 8);
             const int kc = cc / 8, c16 = cc % 8;
-            *reinterpret_cast<uint4*>(sS + kc * (D * 128) + n * 128 + ((c16 ^ (n & 7)) << 4)) = gS[e];
+            uint32_t w4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int kk = 8 * cc + 2 * q;
+                w4[q] = static_cast<uint32_t>(gS[n * D + col_coord(kk)]) |
+                        (static_cast<uint32_t>(gS[n * D + col_coord(kk + 1)]) << 16);
+            }
+            *reinterpret_cast<uint4*>(sS + kc * (D * 128) + n * 128 + ((c16 ^ (n & 7)) << 4)) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
     }
     fence_proxy_async_smem();
@@ -221,6 +456,7 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t tcol = tmem + static_cast<uint32_t>(wg * 128);  // this warpgroup's 128 columns
     const uint32_t tl = tcol + lane_base;                            // ... at this thread's lane
     uint32_t hpar = 0, qpar = 0;
+    const CodeTab<B> ctab(a);
 
     for (int64_t i = wg;; i += C::kWG) {
         const int64_t tile_g = blockIdx.x + i * G;
@@ -254,16 +490,42 @@ __global__ void __launch_bounds__(512, 1)
         // sc = sqrt(D)/||x||, block mean o of u = sc x per channel, fp16(o),
         // and ho = H (delta .* fp16(o)), so that H D w = sc y - ho.
         float nx = 0.f, sc = 0.f;
-        float* xch = nsn_aux + wg * 640;  // [128] sc per token
+        float* xch = nsn_aux + wg * 648;  // [128] sc per token
         float* so = xch + 128;            // [D] delta .* fp16(o)
-        float* ho = xch + 256;            // [D] H (delta .* fp16(o))
+        float* ho = xch + 256;            // [D] H (delta .* fp16(o)), in tensor-memory column order
         float2* opart = reinterpret_cast<float2*>(xch + 384);  // [128 / (D/2)][D/2] partial channel sums
+        float* red = xch + 640;           // DQ: [4] block max of ||x|| / [2][4] channel min, max
         if constexpr (NSN) {
             const uint8_t* sp = stage0 + st * C::kTileBytes;
             const float ssx0 = stage_row_sumsq<D, DT>(sp, r);
             nx = sqrtf(ssx0);
             flag_norm(ssx0, nx, a.status);
-            sc = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
+            uint8_t* rec = DQ ? a.side + tile * RB : nullptr;  // DQ: this block's side record
+            if constexpr (!DQ) {
+                sc = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
+            } else {
+                // 4-bit norm codes on the block's step nstep = fp16(max ||x|| / 15):
+                // q = 0 for a zero token, else clamp(rint(||x|| / nstep), 1, 15);
+                // the transform divides by n1 = q nstep, the stored value
+                float m = nx;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+                if (lane == 0) red[warp & 3] = m;
+                named_bar_sync(bar_id, 128);
+                const float mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+                const __half ns16 = __float2half_rn(mx / 15.0f);
+                const float ns = __half2float(ns16);
+                int qn = 0;
+                if (nx > 0.f && ns > 0.f) qn = min(max(__float2int_rn(nx / ns), 1), 15);
+                sc = qn > 0 ? sqrtf(static_cast<float>(D)) / (static_cast<float>(qn) * ns) : 0.f;
+                const int qp = __shfl_down_sync(0xFFFFFFFFu, qn, 1);
+                if (tile * kTileRows < n_s) {
+                    if ((r & 1) == 0) rec[8 + D / 2 + r / 2] = static_cast<uint8_t>(qn | (qp << 4));
+                    if (r == 0) *reinterpret_cast<__half*>(rec + 4) = ns16;
+                    if (r < 2) rec[6 + r] = 0;
+                    if (r >= 2 && r < 2 + (RB - 8 - D / 2 - 64)) rec[8 + D / 2 + 64 + (r - 2)] = 0;
+                }
+            }
             xch[r] = sc;
             named_bar_sync(bar_id, 128);
             {
@@ -284,6 +546,7 @@ __global__ void __launch_bounds__(512, 1)
                 opart[q * P + p] = acc;
             }
             named_bar_sync(bar_id, 128);
+            float om = 0.f;  // channel r's block mean (r < D)
             if (r < D) {
                 constexpr int P = D / 2, Q = kTileRows / P;
                 float acc = 0.f;
@@ -292,11 +555,54 @@ __global__ void __launch_bounds__(512, 1)
                     const float2 pq = opart[q * P + r / 2];
                     acc += (r & 1) ? pq.y : pq.x;
                 }
-                const __half o16 = __float2half_rn(acc * (1.0f / kTileRows));
-                if (tile * kTileRows < n_s) a.block_mean[tile * D + r] = o16;
-                const uint32_t ps = a.pair_sign[r >> 1];
-                const bool neg = ((ps >> ((r & 1) ? 31 : 15)) & 1u) != 0;
-                so[r] = neg ? -__half2float(o16) : __half2float(o16);
+                om = acc * (1.0f / kTileRows);
+                if constexpr (!DQ) {
+                    const __half o16 = __float2half_rn(om);
+                    if (tile * kTileRows < n_s) a.block_mean[tile * D + r] = o16;
+                    const uint32_t ps = a.pair_sign[r >> 1];
+                    const bool neg = ((ps >> ((r & 1) ? 31 : 15)) & 1u) != 0;
+                    so[r] = neg ? -__half2float(o16) : __half2float(o16);
+                } else {
+                    float mn = om, mxo = om;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+                        mxo = fmaxf(mxo, __shfl_xor_sync(0xFFFFFFFFu, mxo, o));
+                    }
+                    if (lane == 0) {
+                        red[warp & 3] = mn;
+                        red[4 + (warp & 3)] = mxo;
+                    }
+                }
+            }
+            if constexpr (DQ) {
+                // 4-bit mean codes on [lo, lo + 15 step], lo = fp16(min o),
+                // step = fp16((max o - min o) / 15); o_hat = fp32(lo + step q)
+                named_bar_sync(bar_id, 128);
+                if (r < D) {
+                    float lo = red[0], hi = red[4];
+#pragma unroll
+                    for (int w = 1; w < D / 32; ++w) {
+                        lo = fminf(lo, red[w]);
+                        hi = fmaxf(hi, red[4 + w]);
+                    }
+                    const __half lo16 = __float2half_rn(lo), st16 = __float2half_rn((hi - lo) / 15.0f);
+                    const float lof = __half2float(lo16), stf = __half2float(st16);
+                    int qo = 0;
+                    if (stf > 0.f) qo = min(max(__float2int_rn((om - lof) / stf), 0), 15);
+                    const float oh = fmaf(stf, static_cast<float>(qo), lof);
+                    const int qp = __shfl_down_sync(0xFFFFFFFFu, qo, 1);
+                    if (tile * kTileRows < n_s) {
+                        if ((r & 1) == 0) rec[8 + r / 2] = static_cast<uint8_t>(qo | (qp << 4));
+                        if (r == 0) {
+                            *reinterpret_cast<__half*>(rec) = lo16;
+                            *reinterpret_cast<__half*>(rec + 2) = st16;
+                        }
+                    }
+                    const uint32_t ps = a.pair_sign[r >> 1];
+                    const bool neg = ((ps >> ((r & 1) ? 31 : 15)) & 1u) != 0;
+                    so[r] = neg ? -oh : oh;
+                }
             }
             named_bar_sync(bar_id, 128);
             if ((warp & 3) == 0) {
@@ -322,7 +628,10 @@ __global__ void __launch_bounds__(512, 1)
                         v[k] = (lane & hl) ? o - v[k] : v[k] + o;
                     }
 #pragma unroll
-                for (int k = 0; k < VPL; ++k) ho[VPL * lane + k] = v[k];
+                for (int k = 0; k < VPL; ++k) {
+                    const int j = VPL * lane + k;  // coordinate j sits in column (j&~31) + 2(j&15) + ((j>>4)&1)
+                    ho[(j & ~31) + ((j & 15) << 1) + ((j >> 4) & 1)] = v[k];
+                }
             }
             named_bar_sync(bar_id, 128);
         }
@@ -356,12 +665,12 @@ __global__ void __launch_bounds__(512, 1)
         const float nrm = sqrtf(ssx);  // ||x||, or ||w|| for NSN
         if (!NSN) flag_norm(ssx, nrm, a.status);
         const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
-
         // ---- pass 2: codes, residual (fp16 into columns [16c, 16c + 16)) ----
-        // Chunk c + 1 loads while chunk c is coded; the residual of chunk c
-        // goes to columns that chunks 0 .. c/2 occupied, all read already.
+        // Group c + 1 loads while group c is coded; the residual of group c
+        // goes to columns that groups 0 .. c/2 occupied, all read already.
         uint32_t planes[B][kWpp];
-        float rr = 0.f;
+        float2 rr2 = make_float2(0.f, 0.f);
+        const VecTab<B> vt(ctab, nrm, inv);
         tmem_ld32(tl, ybuf[0]);
         tmem_wait_ld();
 #pragma unroll
@@ -376,21 +685,17 @@ __global__ void __launch_bounds__(512, 1)
                     v[k] = __ffma2_rn(v[k], make_float2(sc, sc), make_float2(-h2.x, -h2.y));
                 }
             }
-            uint32_t pl[B][1];
-            rr += codes_and_residual<32, B>(v, inv, a, pl);
+            uint32_t hres[16], w[B];
+            code_group<B>(v, ctab, vt, hres, w, rr2);
 #pragma unroll
-            for (int p = 0; p < B; ++p) planes[p][c] = pl[p][0];
-            if (QJL) {
-                uint32_t hi[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const __half2 hh = __float22half2_rn(v[k]);
-                    hi[k] = *reinterpret_cast<const uint32_t*>(&hh);
-                }
-                tmem_st16(tl + 16 * c, hi);
-            }
+            for (int p = 0; p < B; ++p) planes[p][c] = w[p];
+            // Stored without QJL too (except behind the NSN front end): consuming
+            // the residual group by group keeps the register allocation within
+            // the 128 registers of a thread.
+            if (!NSN) tmem_st16(tl + 16 * c, hres);
             if (c + 1 < NC) tmem_wait_ld();
         }
+        const float rr = rr2.x + rr2.y;
         const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
         const int64_t vidx = tile * kTileRows + r;
         const bool valid = vidx < n_s;
@@ -405,12 +710,14 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t m = valid ? zmask : 0u;
 #pragma unroll
             for (int p = 0; p < B; ++p)
-                store_block32<kWpp>(codes_s + (blk * B + p) * D, planes[p], m, lane, blk * 32 < n_s);
+                store_block32_t<kWpp>(codes_s + (blk * B + p) * D, planes[p], m, lane, blk * 32 < n_s);
         }
         if (valid) {
             const float g = nrm > 0.f ? sqrtf(rr) : 0.f;
-            norms_s[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
-                                : __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
+            if constexpr (DQ) reinterpret_cast<__half*>(norms_s)[vidx] = __float2half_rn(nrm);  // ||w|| only
+            else
+                norms_s[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
+                                    : __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
         }
 
         if (QJL) {
@@ -454,7 +761,7 @@ __global__ void __launch_bounds__(512, 1)
                 if (valid) store_words<kWpp>(qjl_s + vidx * kWpp, qw, zmask);
             } else {
                 const int64_t blk = tile * 4 + (warp & 3);
-                store_block32<kWpp>(qjl_s + blk * D, qw, valid ? zmask : 0u, lane, blk * 32 < n_s);
+                store_block32_t<kWpp>(qjl_s + blk * D, qw, valid ? zmask : 0u, lane, blk * 32 < n_s);
             }
         }
         // The next rotation MMA rewrites this warpgroup's columns; the barrier
@@ -474,11 +781,11 @@ __global__ void __launch_bounds__(512, 1)
     }
 }
 
-template <int D, int B, bool QJL, int DT, bool NSN = false>
+template <int D, int B, bool QJL, int DT, bool NSN = false, bool DQ = false>
 cudaError_t launch_quantize_tc(const CUtensorMap& map, const CUtensorMap& map1, const QuantArgs& a, int num_sms,
                                cudaStream_t s) {
     using C = TcCfg<D, QJL, NSN>;
-    auto kern = quantize_tc_kernel<D, B, QJL, DT, NSN>;
+    auto kern = quantize_tc_kernel<D, B, QJL, DT, NSN, DQ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int64_t grid = a.ntiles < num_sms ? a.ntiles : num_sms;

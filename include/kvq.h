@@ -280,6 +280,62 @@ int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int
                           const int32_t* seq_len, int64_t max_T, float scale, float* logits, float* out,
                           void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Double-quantized NSN side data (NSNQuant section 3, "Double Quantization":
+ * the NSN parameters -- the mean o and the scale s1 -- are themselves stored
+ * with 4 bits).  The pages give no format; this library's, per block of 128
+ * tokens of one head, is one side record of kvq_nsn_dq_side_bytes(d) bytes:
+ *   bytes [0,2) fp16 lo, [2,4) fp16 step, [4,6) fp16 nstep, [6,8) zero;
+ *   [8, 8 + d/2)        4-bit codes q_j of the block means (byte i: channel
+ *                       2i in the low nibble, 2i+1 in the high one);
+ *   [8 + d/2, + 64)     4-bit codes q_t of the 128 token norms (byte i: token
+ *                       2i low nibble, 2i+1 high);
+ *   zero padding to a multiple of 16 bytes (144 bytes at d = 128, 112 at 64).
+ * The stored values are   n1_t = q_t nstep   (q_t = 0 only for a zero token)
+ *                         o_hat_j = fp32(lo + step q_j)   (one rounding),
+ * and the transform uses them: u_t = sqrt(d) x_t / n1_t, w_t = u_t - o_hat,
+ * so a token is exactly n1_t/sqrt(d) (w_t + o_hat) before w_t is coded.
+ * Codes:  nstep = fp16(max_t ||x_t|| / 15), q_t = clamp(rint(||x_t||/nstep),
+ * 1, 15);  lo = fp16(min_j o_j), step = fp16((max_j o_j - min_j o_j) / 15),
+ * q_j = clamp(rint((o_j - lo) / step), 0, 15) (0 when step = 0);  o is the
+ * block mean of u.  Per token only fp16 ||w_t|| is stored besides the codes:
+ * 0.195 bits per element of side data at d = 128 with 128-token blocks,
+ * against 0.375 with fp16 ||x||, ||w|| and fp16 means.
+ */
+
+/* Bytes of one side record for head dimension d (64 or 128; else 0). */
+size_t kvq_nsn_dq_side_bytes(int d);
+
+/*
+ * kvq_nsn_dq_quantize -- kvq_nsn_quantize with the side data double-quantized
+ * as described above.
+ *   x, n_heads, n_tok, layout, codes   as kvq_nsn_quantize (fp16 or bf16 x).
+ *   wnorms   device, n_heads * n_tok fp16 (||w_t||), 4-byte aligned.
+ *   side     device, n_heads * (n_tok/128) records of kvq_nsn_dq_side_bytes(d)
+ *            bytes, 16-byte aligned.
+ * Requires a handle without KVQ_QJL (KVQ_EINVAL) and d <= 128; fp32 input
+ * returns KVQ_EUNSUPPORTED.
+ */
+int kvq_nsn_dq_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, int layout,
+                        uint32_t* codes, uint16_t* wnorms, uint8_t* side, void* stream);
+
+/*
+ * kvq_nsn_dq_decode_attend -- kvq_nsn_decode_attend over caches written by
+ * kvq_nsn_dq_quantize: a stored vector stands for
+ *   x_hat = n1/sqrt(d) (w_hat + o_hat_blk),
+ * with n1 and o_hat decoded from the side records as above.
+ *   k, v      norms hold fp16 ||w|| per token (capacity entries per stream);
+ *             codes as usual; capacities multiples of 128.
+ *   k_side, v_side  device, per stream capacity/128 side records, stream
+ *             (bi, hi) at record (bi * hkv + hi) * capacity/128, 16-byte aligned.
+ * Other arguments, workspace and errors as kvq_nsn_decode_attend; built for
+ * d <= 128.
+ */
+int kvq_nsn_dq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
+                             const kvq_cache* v, const uint8_t* k_side, const uint8_t* v_side, const int32_t* seq_len,
+                             int64_t max_T, float scale, float* logits, float* out, void* workspace, size_t ws_bytes,
+                             void* stream);
+
 /* Most tokens a residual window may hold (kvq_decode_desc.window_cap). */
 #define KVQ_MAX_WINDOW 256
 

@@ -91,7 +91,7 @@ def lib() -> ctypes.CDLL:
             L.orc_nsn_dq_rec_bytes.restype = ctypes.c_int
             L.orc_nsn_dq_rec_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
             L.orc_nsn_dq_quantize.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, ctypes.c_int64,
-                                              P, P, P, P, P, P, P, P, P]
+                                              P, ctypes.c_int, P, P, P, P, P, P, P, P]
             _lib = L
     return _lib
 
@@ -441,10 +441,11 @@ def nsn_dq_rec_bytes(d: int, blk: int = NSN_BLOCK) -> int:
     return int(lib().orc_nsn_dq_rec_bytes(d, blk))
 
 
-def nsn_dq_quantize(k: Constants, x, side_in=None, blk: int = NSN_BLOCK) -> dict:
+def nsn_dq_quantize(k: Constants, x, side_in=None, blk: int = NSN_BLOCK, parts: int = 3) -> dict:
     """NSN front end with 4-bit norm and mean codes + the quantizer (no QJL) on one head's
-    tokens ([n_tok, d], n_tok % blk == 0).  side_in (uint8 [n_tok/blk, rec_bytes]) replaces the
-    side records this function would write (their steps and codes are then used as given)."""
+    tokens ([n_tok, d], n_tok % blk == 0).  side_in (uint8 [n_tok/blk, rec_bytes]) replaces parts
+    of the side records this function would write, which are then used as given: parts bit 0 the
+    norm step and codes, bit 1 the mean offset, step and codes."""
     x = _c(x, np.float64)
     n, d = x.shape
     assert n % blk == 0
@@ -460,7 +461,7 @@ def nsn_dq_quantize(k: Constants, x, side_in=None, blk: int = NSN_BLOCK) -> dict
     z = np.empty((n, d), np.float64)
     si = None if side_in is None else _c(side_in, np.uint8).reshape(nb, R)
     lib().orc_nsn_dq_quantize(d, k.b, blk, _p(k.delta), _p(k.centroids), _p(k.thresholds), _p(x), n, _p(si),
-                              _p(codes), _p(nw), _p(side), _p(n1), _p(oh), _p(of), _p(nx), _p(z))
+                              int(parts), _p(codes), _p(nw), _p(side), _p(n1), _p(oh), _p(of), _p(nx), _p(z))
     return dict(codes=codes, norm_w=nw, side=side, n1=n1, o_hat=oh, mean_f64=of, norm_x=nx, z=z)
 
 

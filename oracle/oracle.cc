@@ -479,8 +479,10 @@ void orc_nsn_quantize(int d, int b, int blk, const int8_t* delta, const double* 
 //     zero padding to a multiple of 16 bytes (rec_bytes).
 // The stored values are the ones the transform used, so x_t = n1_t / sqrt(d)
 // (w_t + o_hat) exactly before w_t is coded.  side_in (nullable) replaces
-// this function's side records by given ones (codes and steps), so that the
-// rest can be recomputed for a record another implementation wrote.
+// parts of this function's side records by given ones, so that the rest can
+// be recomputed for a record another implementation wrote: side_parts bit 0
+// takes the norm step and codes from side_in, bit 1 the mean offset, step
+// and codes.
 // Outputs: codes[n_tok*d], norm_w[n_tok], side_out[(n_tok/blk)*rec_bytes],
 // n1[n_tok], o_hat[(n_tok/blk)*d], o_f64[(n_tok/blk)*d] (unquantized
 // means), norm_x[n_tok] (unquantized norms), z_out (nullable).
@@ -489,9 +491,10 @@ int orc_nsn_dq_rec_bytes(int d, int blk) { return (8 + d / 2 + blk / 2 + 15) / 1
 
 void orc_nsn_dq_quantize(int d, int b, int blk, const int8_t* delta, const double* centroid,
                          const double* threshold, const double* x, int64_t n_tok, const uint8_t* side_in,
-                         int32_t* codes, double* norm_w, uint8_t* side_out, double* n1, double* o_hat,
+                         int side_parts, int32_t* codes, double* norm_w, uint8_t* side_out, double* n1, double* o_hat,
                          double* o_f64, double* norm_x, double* z_out) {
     const int R = orc_nsn_dq_rec_bytes(d, blk);
+    const bool in_n = side_in && (side_parts & 1), in_o = side_in && (side_parts & 2);
     std::vector<double> u((size_t)blk * d), o(d), w(d);
     const double sqd = std::sqrt((double)d);
     for (int64_t b0 = 0; b0 < n_tok; b0 += blk) {
@@ -508,13 +511,13 @@ void orc_nsn_dq_quantize(int d, int b, int blk, const int8_t* delta, const doubl
             mx = std::fmax(mx, norm_x[b0 + t]);
         }
         uint16_t nstep16 = orc_double_to_half(mx / 15.0);
-        if (side_in) nstep16 = (uint16_t)(side_in[bi * R + 4] | (side_in[bi * R + 5] << 8));
+        if (in_n) nstep16 = (uint16_t)(side_in[bi * R + 4] | (side_in[bi * R + 5] << 8));
         const double nstep = orc_half_to_double(nstep16);
         rec[4] = (uint8_t)(nstep16 & 0xFF);
         rec[5] = (uint8_t)(nstep16 >> 8);
         for (int t = 0; t < blk; ++t) {
             int q;
-            if (side_in) {
+            if (in_n) {
                 const uint8_t by = side_in[bi * R + 8 + d / 2 + t / 2];
                 q = (t & 1) ? (by >> 4) : (by & 15);
             } else if (norm_x[b0 + t] == 0.0 || nstep == 0.0) {
@@ -539,7 +542,7 @@ void orc_nsn_dq_quantize(int d, int b, int blk, const int8_t* delta, const doubl
             hi = std::fmax(hi, o[j]);
         }
         uint16_t lo16 = orc_double_to_half(lo), st16 = orc_double_to_half((hi - lo) / 15.0);
-        if (side_in) {
+        if (in_o) {
             lo16 = (uint16_t)(side_in[bi * R] | (side_in[bi * R + 1] << 8));
             st16 = (uint16_t)(side_in[bi * R + 2] | (side_in[bi * R + 3] << 8));
         }
@@ -550,7 +553,7 @@ void orc_nsn_dq_quantize(int d, int b, int blk, const int8_t* delta, const doubl
         rec[3] = (uint8_t)(st16 >> 8);
         for (int j = 0; j < d; ++j) {
             int q;
-            if (side_in) {
+            if (in_o) {
                 const uint8_t by = side_in[bi * R + 8 + j / 2];
                 q = (j & 1) ? (by >> 4) : (by & 15);
             } else if (stv == 0.0) {
