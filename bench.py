@@ -469,6 +469,51 @@ def bench_nsn(args, dist):
     ms_d = timed(dist, dstep, dsteps, stream)
     cache_bytes = NB * H * T * 2 * (h.b * d // 8 + 4 + 2 * d / 128)
     dgbs = cache_bytes / (ms_d / dsteps / 1e3) / 1e9
+    del kc, vc, kn, vn, km, vm
+
+    # ---- the same with double-quantized side data (4-bit norm and mean codes, fp16 ||w||) ----
+    R = kvq.kvq_nsn_dq_side_bytes(d)
+    xs = [wl.nsn_tokens(H, T, d, c["seed"] + i + 1000 * dist.rank, device="cuda") for i in range(4)]
+    codes = torch.empty((H, T, h.b, d // 32), dtype=torch.int32, device="cuda")
+    wn = torch.empty((H, T), dtype=torch.float16, device="cuda")
+    side = torch.empty((H, T // 128, R), dtype=torch.uint8, device="cuda")
+
+    def qstep_dq(i):
+        kvq.kvq_nsn_dq_quantize(h, xs[i % 4], codes, wn, side, stream=stream)
+
+    for i in range(3):
+        qstep_dq(i)
+    ms_q = timed(dist, qstep_dq, steps, stream)
+    q_bytes = H * T * (2 * d + h.b * d // 8 + 2) + H * (T // 128) * R
+    q_gbs = q_bytes / (ms_q / steps / 1e3) / 1e9
+    del xs, codes, wn, side
+    kc = torch.empty((NB * H, T, h.b, d // 32), dtype=torch.int32, device="cuda")
+    vc = torch.empty((NB * H, T // 32, h.b, d), dtype=torch.int32, device="cuda")
+    kn = torch.empty((NB * H, T), dtype=torch.float16, device="cuda")
+    vn = torch.empty_like(kn)
+    ks = torch.empty((NB * H, T // 128, R), dtype=torch.uint8, device="cuda")
+    vs = torch.empty_like(ks)
+    for bi in range(NB):
+        sl = slice(bi * H, (bi + 1) * H)
+        X = wl.nsn_tokens(H, T, d, c["seed"] + 100 + 2 * bi + 1000 * dist.rank, device="cuda")
+        kvq.kvq_nsn_dq_quantize(h, X, kc[sl], kn[sl], ks[sl], stream=stream)
+        X = wl.nsn_tokens(H, T, d, c["seed"] + 101 + 2 * bi + 1000 * dist.rank, device="cuda")
+        kvq.kvq_nsn_dq_quantize(h, X, vc[sl], vn[sl], vs[sl], stream=stream, layout=kvq.KVQ_LAYOUT_BLOCK32)
+        del X
+    kcache = kvq.make_cache(kc, None, kn, T, kvq.KVQ_LAYOUT_TOKEN)
+    vcache = kvq.make_cache(vc, None, vn, T, kvq.KVQ_LAYOUT_BLOCK32)
+
+    def dstep_dq(i):
+        kvq.kvq_nsn_dq_decode_attend(h, q, H, kcache, vcache, ks, vs, seq, T, 1.0, out, ws, stream=stream)
+
+    for i in range(3):
+        dstep_dq(i)
+    code, bits = kvq.kvq_status(h)
+    if code != 0:
+        raise RuntimeError(f"nsn dq status {code} bits {bits}")
+    ms_dd = timed(dist, dstep_dq, dsteps, stream)
+    dq_cache = NB * H * T * 2 * (h.b * d // 8 + 2) + NB * H * (T // 128) * 2 * R
+    dq_dgbs = dq_cache / (ms_dd / dsteps / 1e3) / 1e9
     h.close()
     return {"metric": "NSN quantize tokens/s", "value": dist.world * T * steps / (ms / 1e3), "unit": "tokens/s",
             "ms_per_step": ms / steps, "workload": "8 heads x 65536 tokens x d128 bf16, b=2, no QJL",
@@ -481,7 +526,15 @@ def bench_nsn(args, dist):
                        "steps": dsteps, "cache_bytes_per_step": int(cache_bytes),
                        "workload": "4 sequences x 8 KV heads x 65536 tokens of the NSN workload (b=2, keys per "
                                    "token, values in blocks of 32, fp16 block means), 32 query heads, one bf16 "
-                                   "query token, kvq_nsn_decode_attend"}}
+                                   "query token, kvq_nsn_decode_attend"},
+            "double_quantized": {
+                "quantize_ms_per_step": ms_q / steps, "quantize_gbs": round(q_gbs, 1),
+                "quantize_frac_of_hbm": round(q_gbs / hbm, 4), "quantize_bytes_per_step": int(q_bytes),
+                "decode_gbs": round(dist.world * dq_dgbs, 1), "decode_frac_of_hbm": round(dq_dgbs / hbm, 4),
+                "decode_ms_per_step": ms_dd / dsteps, "decode_cache_bytes_per_step": int(dq_cache),
+                "side_bits_per_element": round((R / 128 + 2) * 8 / d, 4),
+                "workload": "the same NSN workload through kvq_nsn_dq_quantize (4-bit token-norm and block-mean "
+                            "codes in one side record per 128 tokens, fp16 ||w||) and kvq_nsn_dq_decode_attend"}}
 
 
 def bench_sweep(args, dist):
