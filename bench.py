@@ -297,6 +297,32 @@ def bench_quantize(args, dist):
                tensor=tensor_record(2 * n, d, avg_launch_s),
                clocks=clk.summary())
 
+    # ---- the same step with the rotation on the CUDA cores: the in-register
+    # transform kernel (one launch for K, one for V), for comparison ----
+    hc = kvq.Handle(d, b, c["handle_seed"], qjl=True, cuda_core_rotation=True)
+
+    def step_cc(i):
+        K, V = copies[i % 4]
+        kvq.kvq_quantize_batch(hc, [(K, *outK, kvq.KVQ_LAYOUT_TOKEN), (V, *outV, kvq.KVQ_LAYOUT_BLOCK32)],
+                               stream=stream)
+
+    for i in range(args.warmup):
+        step_cc(i)
+    ms_cc = timed(dist, step_cc, args.steps, stream)
+    code, bits = kvq.kvq_status(hc)
+    if code != 0:
+        raise RuntimeError(f"quantize (CUDA-core rotation) status {code} bits {bits}")
+    hc.close()
+    cc_s = ms_cc / args.steps / 1e3
+    res["rotation"] = {
+        "tensor_core_us_per_step": round(avg_launch_s * 1e6, 2),
+        "cuda_core_us_per_step": round(cc_s * 1e6, 2),
+        "cuda_core_gbs": round(per_launch_bytes / cc_s / 1e9, 1),
+        "cuda_core_frac_of_hbm": round(per_launch_bytes / cc_s / 1e9 / hbm, 4),
+        "speedup_of_tensor_core_rotation": round(cc_s / avg_launch_s, 3),
+        "note": "the same layer step (K and V, same outputs under the same parity rules) with KVQ_CUDA_CORE_ROTATION: "
+                "quantize_kernel with the in-register Walsh-Hadamard transform, one launch per job"}
+
     # ---- end to end through the binding with host buffers ----
     Kh = copies[0][0].cpu().pin_memory()
     Vh = copies[0][1].cpu().pin_memory()
@@ -704,6 +730,7 @@ def run_ours(args):
         if nsn is not None:
             line["nsn_quantize"] = nsn
         line["tensor"] = q["tensor"]
+        line["rotation"] = q["rotation"]
         line["parity_boundary"] = parity_record()
         if dec is not None:
             line["decode_attn"] = dec

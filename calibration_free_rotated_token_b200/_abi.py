@@ -27,6 +27,7 @@ KVQ_ENONFINITE = -5
 KVQ_ETIMEOUT = -6
 KVQ_QJL = 1
 KVQ_BETA_CODEBOOK = 2
+KVQ_CUDA_CORE_ROTATION = 4
 KVQ_F32, KVQ_F16, KVQ_BF16 = 0, 1, 2
 KVQ_LAYOUT_TOKEN, KVQ_LAYOUT_BLOCK32 = 0, 1
 STATUS_NONFINITE, STATUS_NORM_OVERFLOW, STATUS_TIMEOUT = 1, 2, 4
@@ -152,10 +153,12 @@ def _need(t, name, dtype=None, numel=None, device=True):
 class Handle:
     """Owns a kvq_handle; ``d``, ``b``, ``m``, ``qjl`` mirror kvq_get_info."""
 
-    def __init__(self, d: int, b: int, seed: int, qjl: bool = True, beta: bool = False):
+    def __init__(self, d: int, b: int, seed: int, qjl: bool = True, beta: bool = False,
+                 cuda_core_rotation: bool = False):
         L = load()
         h = ctypes.c_void_p()
-        flags = (KVQ_QJL if qjl else 0) | (KVQ_BETA_CODEBOOK if beta else 0)
+        flags = ((KVQ_QJL if qjl else 0) | (KVQ_BETA_CODEBOOK if beta else 0) |
+                 (KVQ_CUDA_CORE_ROTATION if cuda_core_rotation else 0))
         _check(L.kvq_init(ctypes.byref(h), d, b, seed & (2**64 - 1), flags))
         self._h = h
         dd, bb, mm, ff = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_uint32()

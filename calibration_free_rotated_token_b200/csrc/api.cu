@@ -301,6 +301,7 @@ int launch_jobs(kvq_handle h, const QJob& j0, const CUtensorMap& m0, const QJob*
     }
     a.block_mean = reinterpret_cast<__half*>(block_mean);
     a.side = side;
+    a.cuda_core_rotation = (h->flags & KVQ_CUDA_CORE_ROTATION) != 0 && !nsn;
     a.S = h->d_S;
     a.status = h->d_status;
     fill_common(h, a.centroid, a.threshold, a.pair_sign);
@@ -341,7 +342,7 @@ int kvq_init(kvq_handle* out, int d, int b, uint64_t seed, uint32_t flags) {
     *out = nullptr;
     if (d != 64 && d != 128 && d != 256) return fail(KVQ_EINVAL, "d must be 64, 128 or 256");
     if (b < 1 || b > 4) return fail(KVQ_EINVAL, "b must be in 1..4");
-    if (flags & ~(KVQ_QJL | KVQ_BETA_CODEBOOK)) return fail(KVQ_EINVAL, "unknown flag bits");
+    if (flags & ~(KVQ_QJL | KVQ_BETA_CODEBOOK | KVQ_CUDA_CORE_ROTATION)) return fail(KVQ_EINVAL, "unknown flag bits");
     kvq_ctx* h = new (std::nothrow) kvq_ctx();
     if (!h) return fail(KVQ_ENOMEM, "host allocation failed");
     cudaGetDevice(&h->device);
@@ -384,7 +385,7 @@ int kvq_codebook(int d, int b, uint32_t flags, float* centroids, float* threshol
     g_err.clear();
     if (d != 64 && d != 128 && d != 256) return fail(KVQ_EINVAL, "d must be 64, 128 or 256");
     if (b < 1 || b > 4) return fail(KVQ_EINVAL, "b must be in 1..4");
-    if (flags & ~(KVQ_QJL | KVQ_BETA_CODEBOOK)) return fail(KVQ_EINVAL, "unknown flag bits");
+    if (flags & ~(KVQ_QJL | KVQ_BETA_CODEBOOK | KVQ_CUDA_CORE_ROTATION)) return fail(KVQ_EINVAL, "unknown flag bits");
     if (!centroids || !thresholds) return fail(KVQ_EINVAL, "centroids and thresholds must be non-null");
     std::vector<double> c, t;
     if (flags & KVQ_BETA_CODEBOOK) lloyd_max_sphere_codebook(d, b, &c, &t);
@@ -448,7 +449,7 @@ int kvq_quantize_batch(kvq_handle h, int count, const kvq_quant_job* jobs, void*
     }
     for (size_t i = 0; i < js.size();) {
         const bool pair = i + 1 < js.size() && js[i].dtype == js[i + 1].dtype &&
-                          kvq::quantize_pairs(h->d, js[i].dtype, false);
+                          kvq::quantize_pairs(h->d, js[i].dtype, false) && !(h->flags & KVQ_CUDA_CORE_ROTATION);
         if (int e = launch_jobs(h, js[i], maps[i], pair ? &js[i + 1] : nullptr, pair ? &maps[i + 1] : nullptr,
                                 nullptr, false, stream))
             return e;

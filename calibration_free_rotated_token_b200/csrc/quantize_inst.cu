@@ -3,7 +3,8 @@
 // per supported pair so that the twelve instantiations compile in parallel.
 // 16-bit input with d <= 128 (with or without the NSN front end) takes the
 // tensor-core rotation kernel (quantize_tc.cuh); fp32 input and d = 256 take
-// the kernel with the in-register transform (quantize.cuh).
+// the kernel with the in-register transform (quantize.cuh), which 16-bit input
+// at d <= 128 takes too when the handle asks for the CUDA-core rotation.
 #include "quantize_tc.cuh"
 
 #ifndef KVQ_D
@@ -45,11 +46,19 @@ cudaError_t by_dtype(const CUtensorMap& map, const CUtensorMap& map1, int dtype,
                 if constexpr (D <= 128) return launch_quantize_t<D, B, QJL, DT_F32, NSN>(map, a, sms, s);
                 else return cudaErrorNotSupported;
             case DT_F16:
-                if constexpr (D <= 128 && !NSN) return launch_quantize_tc<D, B, QJL, DT_F16>(map, map1, a, sms, s);
-                else return launch_quantize_t<D, B, QJL, DT_F16, NSN>(map, a, sms, s);
+                if constexpr (D <= 128 && !NSN) {
+                    if (a.cuda_core_rotation) return launch_quantize_t<D, B, QJL, DT_F16, false>(map, a, sms, s);
+                    return launch_quantize_tc<D, B, QJL, DT_F16>(map, map1, a, sms, s);
+                } else {
+                    return launch_quantize_t<D, B, QJL, DT_F16, NSN>(map, a, sms, s);
+                }
             default:
-                if constexpr (D <= 128 && !NSN) return launch_quantize_tc<D, B, QJL, DT_BF16>(map, map1, a, sms, s);
-                else return launch_quantize_t<D, B, QJL, DT_BF16, NSN>(map, a, sms, s);
+                if constexpr (D <= 128 && !NSN) {
+                    if (a.cuda_core_rotation) return launch_quantize_t<D, B, QJL, DT_BF16, false>(map, a, sms, s);
+                    return launch_quantize_tc<D, B, QJL, DT_BF16>(map, map1, a, sms, s);
+                } else {
+                    return launch_quantize_t<D, B, QJL, DT_BF16, NSN>(map, a, sms, s);
+                }
         }
     }
 }

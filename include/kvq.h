@@ -87,6 +87,14 @@ extern "C" {
  * vector scaled by sqrt(d) (Beta((d-1)/2, (d-1)/2) on [-1, 1], stretched to
  * [-sqrt(d), sqrt(d)]; TurboQuant blog, "Estágio 1") instead of N(0, 1). */
 #define KVQ_BETA_CODEBOOK 2u
+/* Rotation on the CUDA cores: kvq_quantize / kvq_quantize_batch with 16-bit
+ * input at d <= 128 rotate by the in-register Walsh-Hadamard transform (the
+ * kernel fp32 input and d = 256 use) instead of the tensor-core product
+ * X (H D)^T.  Same outputs under the same rules (codes exact outside the
+ * decision-level band, norms within one fp16 ulp); one launch per job.  For
+ * comparing the two rotations at one configuration; the NSN entry points
+ * ignore it. */
+#define KVQ_CUDA_CORE_ROTATION 4u
 
 /* ---- element types of inputs ------------------------------------------ */
 #define KVQ_F32 0
@@ -113,7 +121,7 @@ typedef struct kvq_ctx* kvq_handle;
  *   b      Lloyd-Max bits per coordinate, 1..4.
  *   seed   seeds the SplitMix64 streams: Rademacher signs use `seed`, the
  *          Gaussian projection S (d x d, rounded to fp16) uses `seed + 1`.
- *   flags  KVQ_QJL and/or KVQ_BETA_CODEBOOK, or 0.
+ *   flags  KVQ_QJL, KVQ_BETA_CODEBOOK and/or KVQ_CUDA_CORE_ROTATION, or 0.
  * Synchronous.  Allocates device memory for the constants and a status
  * word.  Errors: KVQ_EINVAL, KVQ_ENOMEM, KVQ_ECUDA.
  */

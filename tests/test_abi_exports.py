@@ -76,3 +76,9 @@ def test_library_codebook_matches_oracle_on_host(lib, beta):
     assert lib.kvq_codebook(96, 2, 0, buf, buf) == _abi.KVQ_EINVAL
     assert lib.kvq_codebook(128, 2, 8, buf, buf) == _abi.KVQ_EINVAL
     assert lib.kvq_codebook(128, 2, 0, None, buf) == _abi.KVQ_EINVAL
+    # the rotation flag is a valid flag and leaves the codebook unchanged
+    ref = (C.c_float * 16)()
+    assert lib.kvq_codebook(128, 3, 0, ref, buf) == _abi.KVQ_OK
+    got = (C.c_float * 16)()
+    assert lib.kvq_codebook(128, 3, _abi.KVQ_CUDA_CORE_ROTATION | _abi.KVQ_QJL, got, buf) == _abi.KVQ_OK
+    assert list(got)[:8] == list(ref)[:8]

@@ -251,6 +251,33 @@ def test_quantize_batch_matches_oracle_and_single_calls(d, b, qjl, j0, j1):
                 assert torch.equal(q1, qj)
 
 
+@pytest.mark.parametrize("d,b,qjl,dtype,n,layout", [
+    (128, 2, True, torch.bfloat16, 1000, 0),
+    (128, 2, True, torch.bfloat16, 777, 1),
+    (64, 3, False, torch.float16, 257, 0),
+    (128, 4, True, torch.float16, 300, 0),
+    (64, 1, True, torch.bfloat16, 129, 1),
+])
+def test_cuda_core_rotation_matches_oracle(d, b, qjl, dtype, n, layout):
+    """KVQ_CUDA_CORE_ROTATION: 16-bit input at d <= 128 through the in-register transform kernel, under the
+    same parity rules; a layer's K and V through kvq_quantize_batch (one launch per job)."""
+    x = wl.sweep_tokens(n, d, seed=500 + d + b, dtype=dtype)
+    x[1] = 0
+    k = constants(d, b, 9)
+    with kvq.Handle(d, b, 9, qjl=qjl, cuda_core_rotation=True) as h:
+        codes, qj, norms = run_quantize(h, x.cuda(), layout=layout)
+        compare_quantize(k, x.double().numpy(), to_np_u32(codes), to_np_u32(qj) if qjl else None,
+                         to_np_f16bits(norms), qjl, layout=layout)
+        y = wl.sweep_tokens(n + 64, d, seed=600 + d + b, dtype=dtype)
+        outs = [kvq.alloc_packed(h, t.shape[0], layout=lay) for t, lay in ((x, 0), (y, 1))]
+        kvq.kvq_quantize_batch(h, [(t.cuda(), *o, lay) for t, o, lay in zip((x, y), outs, (0, 1))])
+        code, bits = kvq.kvq_status(h)
+        assert code == 0, (code, bits)
+    for t, (c, q, nn), lay in zip((x, y), outs, (0, 1)):
+        compare_quantize(k, t.double().numpy(), to_np_u32(c), to_np_u32(q) if qjl else None, to_np_f16bits(nn),
+                         qjl, layout=lay)
+
+
 def test_quantize_batch_empty_jobs_and_three_streams():
     d, b = 128, 2
     xs = [wl.sweep_tokens(n, d, seed=400 + n, dtype=torch.bfloat16) for n in (200, 0, 130, 64)]
