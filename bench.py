@@ -204,6 +204,35 @@ def timed(dist: Dist, fn, steps: int, stream) -> float:
     return dist.max(e0.elapsed_time(e1))
 
 
+_L2_FLUSH = None
+
+
+def timed_flushed(dist: Dist, fn, steps: int, stream) -> float:
+    """Milliseconds for `steps` calls of fn(i) whose data would fit in L2: each
+    call is timed alone on the device, after a 256 MB write (twice the L2) has
+    evicted the previous call's data; the sum over the calls, max over ranks."""
+    global _L2_FLUSH
+    if _L2_FLUSH is None:
+        _L2_FLUSH = torch.empty(64 << 20, dtype=torch.int32, device="cuda")
+    dist.barrier()
+    torch.cuda.synchronize()
+    evs = []
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            _L2_FLUSH.fill_(i)
+            # as in timed(): the host enqueues the call before the device reaches it
+            torch.cuda._sleep(HEAD_START_CYCLES // 8)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(i)
+            e1.record(stream)
+            evs.append((e0, e1))
+    torch.cuda.synchronize()
+    dist.barrier()
+    return dist.max(sum(a.elapsed_time(b) for a, b in evs))
+
+
 def traffic_record(kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if it matches the current build."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -492,7 +521,7 @@ def bench_nsn(args, dist):
     if code != 0:
         raise RuntimeError(f"nsn decode status {code} bits {bits}")
     dsteps = max(5, steps // 2)
-    ms_d = timed(dist, dstep, dsteps, stream)
+    ms_d = timed_flushed(dist, dstep, dsteps, stream)
     cache_bytes = NB * H * T * 2 * (h.b * d // 8 + 4 + 2 * d / 128)
     dgbs = cache_bytes / (ms_d / dsteps / 1e3) / 1e9
     del kc, vc, kn, vn, km, vm
@@ -537,7 +566,7 @@ def bench_nsn(args, dist):
     code, bits = kvq.kvq_status(h)
     if code != 0:
         raise RuntimeError(f"nsn dq status {code} bits {bits}")
-    ms_dd = timed(dist, dstep_dq, dsteps, stream)
+    ms_dd = timed_flushed(dist, dstep_dq, dsteps, stream)
     dq_cache = NB * H * T * 2 * (h.b * d // 8 + 2) + NB * H * (T // 128) * 2 * R
     dq_dgbs = dq_cache / (ms_dd / dsteps / 1e3) / 1e9
     h.close()
@@ -550,6 +579,7 @@ def bench_nsn(args, dist):
             "decode": {"metric": "NSN packed-cache decode-attn GB/s", "value": round(dist.world * dgbs, 1),
                        "unit": "GB/s", "frac_of_hbm": round(dgbs / hbm, 4), "ms_per_step": ms_d / dsteps,
                        "steps": dsteps, "cache_bytes_per_step": int(cache_bytes),
+                       "l2": "each call timed alone after a 256 MB write evicts L2 (the cache is about L2's size)",
                        "workload": "4 sequences x 8 KV heads x 65536 tokens of the NSN workload (b=2, keys per "
                                    "token, values in blocks of 32, fp16 block means), 32 query heads, one bf16 "
                                    "query token, kvq_nsn_decode_attend"},
@@ -559,6 +589,7 @@ def bench_nsn(args, dist):
                 "decode_gbs": round(dist.world * dq_dgbs, 1), "decode_frac_of_hbm": round(dq_dgbs / hbm, 4),
                 "decode_ms_per_step": ms_dd / dsteps, "decode_cache_bytes_per_step": int(dq_cache),
                 "side_bits_per_element": round((R / 128 + 2) * 8 / d, 4),
+                "l2": "decode calls timed alone after a 256 MB write evicts L2",
                 "workload": "the same NSN workload through kvq_nsn_dq_quantize (4-bit token-norm and block-mean "
                             "codes in one side record per 128 tokens, fp16 ||w||) and kvq_nsn_dq_decode_attend"}}
 
@@ -603,7 +634,7 @@ def bench_sweep(args, dist):
 
                 for i in range(3):
                     dstep(i)
-                ms_d = timed(dist, dstep, steps, stream)
+                ms_d = timed_flushed(dist, dstep, steps, stream)
                 code, bits = kvq.kvq_status(h)
                 if code != 0:
                     raise RuntimeError(f"sweep d={d} b={b} qjl={qjl}: status {code} bits {bits}")
@@ -627,6 +658,8 @@ def bench_sweep(args, dist):
                         "over them: 8 KV heads x "
                         "131072 tokens, one bf16 query per head",
             "bytes": "quantize: 2d in + the packed record out per vector; decode: the K and V records read",
+            "l2": "quantize: two 2^20-vector inputs per call (256 MB-1 GB); decode: each call timed alone after a "
+                  "256 MB write evicts L2 (the caches, 28-109 MB, fit in it)",
             "peak": hbm, "peak_source": f"{src} hbm_gbs (copy)", "steps": steps, "rows": rows}
 
 

@@ -558,13 +558,32 @@ void decode_plan(const kvq_ctx* h, int batch, int hq, int hkv, int64_t max_T, in
     int64_t ch;
     if (decode_uses_mma(h)) {
         // Persistent grid over (stream, split) items: about 16 items per
-        // resident CTA keeps the last round short; splits of at least 1024
-        // tokens amortise the per-item set-up.
+        // resident CTA keeps the last round short; splits are multiples of 256
+        // tokens and at least 1024 (amortising the per-item set-up).  When even
+        // 1024-token splits leave fewer than 3 rounds of items over the grid
+        // (few streams), a short last round costs a large share of the call:
+        // then the split is the one, up to 4x longer, whose rounds cost least,
+        // counting an item as its tokens plus a set-up worth kItemCost tokens.
+        constexpr int64_t kItemCost = 384;
         const int64_t grid = decode_mma_grid(h, hkv > 0 ? hq / hkv : 1);
-        const int64_t target = 16 * grid;
-        ch = (streams * max_T + target - 1) / (target > 0 ? target : 1);
-        ch = (ch + 255) / 256 * 256;
-        if (ch < 1024) ch = 1024;
+        const int64_t g = grid > 0 ? grid : 1;
+        const int64_t target = 16 * g;
+        int64_t lo = (streams * max_T + target - 1) / target;
+        lo = (lo + 255) / 256 * 256;
+        if (lo < 1024) lo = 1024;
+        ch = lo;
+        if (streams * ((max_T + lo - 1) / lo) < 3 * g) {
+            const int64_t mx = (max_T + 255) / 256 * 256;
+            int64_t best_cost = -1;
+            for (int64_t c = lo; c <= 4 * lo && (c == lo || c <= mx); c += 256) {
+                const int64_t rounds = (streams * ((max_T + c - 1) / c) + g - 1) / g;
+                const int64_t cost = rounds * (c + kItemCost);
+                if (best_cost < 0 || cost < best_cost) {
+                    ch = c;
+                    best_cost = cost;
+                }
+            }
+        }
         if ((max_T + ch - 1) / ch > 4096) ch = ((max_T + 4095) / 4096 + 255) / 256 * 256;
     } else {
         int64_t want = (4 * static_cast<int64_t>(sms) + streams - 1) / (streams > 0 ? streams : 1);
