@@ -57,7 +57,10 @@ struct DTile {
 
 template <int G>
 struct HeadCfg {
-    static constexpr int NTK = (G <= 4) ? 2 : 4;  // key n-tiles: 4 digit columns per head
+    // key n-tiles (4 digit columns per head): G <= 2 takes one n-tile of two
+    // heads (column g = head g / 4, digit g % 4), G = 4 two and G = 8 four
+    // (column g of n-tile nt = head g / 2 + 4 (nt / 2), digit g % 2 + 2 (nt % 2))
+    static constexpr int NTK = (G <= 2) ? 1 : (G <= 4) ? 2 : 4;
     static constexpr int RT = (G <= 4) ? 1 : 2;   // value m-tiles: 4 digit rows per head
     static constexpr int GP = (G <= 4) ? 4 : 8;   // heads incl. padding
     static constexpr int CPL = (G <= 4) ? 1 : 2;  // value columns merged per lane
@@ -297,8 +300,8 @@ __global__ void __launch_bounds__(kThreads) qfrag_kernel(const __grid_constant__
     for (int e = tid; e < KS * NTK * 32; e += kThreads) {
         const int lane = e % 32, nt = (e / 32) % NTK, ks = e / (32 * NTK);
         const int g = lane >> 2, t = lane & 3;
-        const int h = (g >> 1) + 4 * (nt >> 1);
-        const int dig = (g & 1) + 2 * (nt & 1);
+        const int h = (NTK == 1) ? (g >> 2) : (g >> 1) + 4 * (nt >> 1);
+        const int dig = (NTK == 1) ? (g & 3) : (g & 1) + 2 * (nt & 1);
         uint32_t b[2] = {0u, 0u};
         if (h < G) {
             const int plane = ks / (D / 32), w = ks % (D / 32);
@@ -362,7 +365,9 @@ struct MmaSmem {
     static constexpr int kWfrag = (TC / 32) * RT * 32 * 16;  // weight digits, per kind
     static constexpr int kMisc = NSN ? 1536 : 1024;
     static constexpr int kBytes = 2 * kStage + kFrag + kLog + 2 * kWfrag + kMisc + kXp;
-    static constexpr bool kQfReg = KS * NTK <= 24;         // query fragments held in registers
+    // query fragments held in registers (at G <= 2 under the same K-step bound
+    // as with two n-tiles: more live fragments cost a resident CTA per SM)
+    static constexpr bool kQfReg = KS * (NTK == 1 ? 2 : NTK) <= 24;
 };
 
 template <int D, int B, bool QJL, int G, bool NSN = false, bool DQ = false>
@@ -442,12 +447,13 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             const uint2* gf = a.qfrag + stream * KS * NTK * 32;
             for (int e = tid; e < KS * NTK * 32; e += kThreads) sfrag[e] = gf[e];
         }
-        // logit constants of this lane's heads t (and t + 4):
+        // logit constants of this lane's heads t (and t + 4); with one key
+        // n-tile (G <= 2) head t / 2:
         // l = n (k0 + k1 xc + n_gamma (k2 xq - k3)), scale / d folded in
         float hk0[HH], hk1[HH], hk2[HH], hk3[HH];
 #pragma unroll
         for (int hh = 0; hh < HH; ++hh) {
-            const int h = t + 4 * hh;
+            const int h = (NTK == 1) ? (t >> 1) : t + 4 * hh;
             hk0[hh] = hk1[hh] = hk2[hh] = hk3[hh] = 0.f;
             if (h < G) {
                 const float* qs = a.qscal + (qh0 + h) * 4;
@@ -683,37 +689,55 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                         for (int r = 0; r < 4; ++r) accc[0][nt][r] = accc[1][nt][r] = accq[nt][r] = 0;
                 }
                 // epilogue: thread t owns head t (and t + 4 when G = 8); its
-                // columns hold the four digits of the head
+                // columns hold the four digits of the head.  With one key
+                // n-tile (G <= 2) lanes t and t ^ 1 hold digits 0, 1 and 2, 3 of
+                // head t / 2: one exchange completes both, and the even lane
+                // keeps the logit.
+                const bool own = (NTK > 1) || ((t & 1) == 0);
 #pragma unroll
                 for (int hh = 0; hh < HH; ++hh) {
-                    const int h = t + 4 * hh;
+                    const int h = (NTK == 1) ? (t >> 1) : t + 4 * hh;
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr) {
                         const int tl = rr ? tl1 : tl0;
                         float l;
                         {
-                            const int n0 = 2 * hh, n1 = 2 * hh + 1;
-                            const float xc = fmaf(static_cast<float>((accc[0][n0][2 * rr] + accc[1][n0][2 * rr]) * 128 +
-                                                                     accc[0][n0][2 * rr + 1] + accc[1][n0][2 * rr + 1]),
-                                                  16384.f,
-                                                  static_cast<float>((accc[0][n1][2 * rr] + accc[1][n1][2 * rr]) * 128 +
-                                                                     accc[0][n1][2 * rr + 1] + accc[1][n1][2 * rr + 1]));
+                            float xc, xq = 0.f;
+                            if constexpr (NTK == 1) {
+                                const int mine = (accc[0][0][2 * rr] + accc[1][0][2 * rr]) * 128 + accc[0][0][2 * rr + 1] +
+                                                 accc[1][0][2 * rr + 1];
+                                const int other = __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
+                                xc = fmaf(static_cast<float>((t & 1) ? other : mine), 16384.f,
+                                          static_cast<float>((t & 1) ? mine : other));
+                                if (QJL) {
+                                    const int mq = accq[0][2 * rr] * 128 + accq[0][2 * rr + 1];
+                                    const int oq = __shfl_xor_sync(0xFFFFFFFFu, mq, 1);
+                                    xq = fmaf(static_cast<float>((t & 1) ? oq : mq), 16384.f,
+                                              static_cast<float>((t & 1) ? mq : oq));
+                                }
+                            } else {
+                                const int n0 = 2 * hh, n1 = 2 * hh + 1;
+                                xc = fmaf(static_cast<float>((accc[0][n0][2 * rr] + accc[1][n0][2 * rr]) * 128 +
+                                                             accc[0][n0][2 * rr + 1] + accc[1][n0][2 * rr + 1]),
+                                          16384.f,
+                                          static_cast<float>((accc[0][n1][2 * rr] + accc[1][n1][2 * rr]) * 128 +
+                                                             accc[0][n1][2 * rr + 1] + accc[1][n1][2 * rr + 1]));
+                                if (QJL)
+                                    xq = fmaf(static_cast<float>(accq[n0][2 * rr] * 128 + accq[n0][2 * rr + 1]), 16384.f,
+                                              static_cast<float>(accq[n1][2 * rr] * 128 + accq[n1][2 * rr + 1]));
+                            }
                             const float2 nk = knorm(tl);
                             float inner = fmaf(hk1[hh], xc, hk0[hh]);
-                            if (QJL) {
-                                const float xq =
-                                    fmaf(static_cast<float>(accq[n0][2 * rr] * 128 + accq[n0][2 * rr + 1]), 16384.f,
-                                         static_cast<float>(accq[n1][2 * rr] * 128 + accq[n1][2 * rr + 1]));
-                                inner = fmaf(nk.y, fmaf(hk2[hh], xq, -hk3[hh]), inner);
-                            }
+                            if (QJL) inner = fmaf(nk.y, fmaf(hk2[hh], xq, -hk3[hh]), inner);
                             // NSN: l = scale ||x||/sqrt(d) (||w||/d <q', c> + <q, o>)
                             const float lt = NSN ? nk.x * fmaf(nk.y * inv_sqrt_d, inner, sqo[h * 2 + (tl >> 7)])
                                                  : nk.x * inner;
-                            l = (h < G && tl < nval) ? lt : -INFINITY;
+                            l = (own && h < G && tl < nval) ? lt : -INFINITY;
                             lmax[hh] = fmaxf(lmax[hh], l);
                         }
-                        if (h < GP) slog[h * TC + tl] = l;
-                        if (a.logits != nullptr && h < G && tl < nval_e) a.logits[(qh0 + h) * a.logits_ld + tb + tl] = l;
+                        if (own && h < GP) slog[h * TC + tl] = l;
+                        if (own && a.logits != nullptr && h < G && tl < nval_e)
+                            a.logits[(qh0 + h) * a.logits_ld + tb + tl] = l;
                     }
                 }
             }
@@ -741,7 +765,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                 if (g == 0) {
 #pragma unroll
                     for (int hh = 0; hh < HH; ++hh)
-                        if (t + 4 * hh < GP) sred[warp * 16 + t + 4 * hh] = lmax[hh];
+                        if (NTK == 1) sred[warp * 16 + ((t & 1) ? 2 + (t >> 1) : (t >> 1))] = lmax[hh];  // odd lanes: -inf
+                        else if (t + 4 * hh < GP) sred[warp * 16 + t + 4 * hh] = lmax[hh];
                 }
                 if (lane == 0) {
                     sred[warp * 16 + 8] = nmx;
@@ -1179,7 +1204,7 @@ cudaError_t launch_decode_mma(const kvq_ctx* h, const DecodeArgs& a, cudaStream_
 }
 
 size_t decode_mma_qfrag_bytes(const kvq_ctx* h, int G) {
-    const int NTK = (G <= 4) ? 2 : 4;
+    const int NTK = (G <= 2) ? 1 : (G <= 4) ? 2 : 4;
     const int PV = h->b == 3 ? 4 : h->b;  // code planes, the 3-bit parity plane included
     const int KS = (PV + ((h->flags & 1u) ? 1 : 0)) * (h->d / 32);
     return static_cast<size_t>(KS) * NTK * 32 * 8;
