@@ -63,7 +63,7 @@ class KvqDecodeDesc(ctypes.Structure):
                 ("window_cap", ctypes.c_int64), ("window_len", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
                 ("max_T", ctypes.c_int64), ("scale", ctypes.c_float), ("logits", ctypes.c_void_p),
                 ("logits_ld", ctypes.c_int64), ("out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-                ("ws_bytes", ctypes.c_size_t)]
+                ("ws_bytes", ctypes.c_size_t), ("k_side", ctypes.c_void_p), ("v_side", ctypes.c_void_p)]
 
 
 class KvqQuantJob(ctypes.Structure):
@@ -391,8 +391,10 @@ def kvq_decode_attend_ex(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache,
                          k_window: torch.Tensor | None = None, v_window: torch.Tensor | None = None,
                          window_len: torch.Tensor | None = None, k_block_mean: torch.Tensor | None = None,
                          v_block_mean: torch.Tensor | None = None, logits: torch.Tensor | None = None,
-                         logits_ld: int = 0, stream=None):
-    """Decode over a packed cache (plain or NSN) and an optional fp16 residual window
+                         logits_ld: int = 0, stream=None, k_side: torch.Tensor | None = None,
+                         v_side: torch.Tensor | None = None):
+    """Decode over a packed cache (plain, NSN with fp16 block means, or NSN with
+    double-quantized side records) and an optional fp16 residual window
     ([batch * hkv, window_cap, d]); window_len int32 [batch] on the device."""
     if q.dim() != 3 or q.shape[-1] != h.d:
         raise ValueError(f"q must be [batch, hq, {h.d}]")
@@ -414,7 +416,7 @@ def kvq_decode_attend_ex(h: Handle, q: torch.Tensor, hkv: int, kcache: KvqCache,
     d = KvqDecodeDesc(_ptr(q), _DTYPES[q.dtype], B, hq, hkv, ctypes.pointer(kcache), ctypes.pointer(vcache),
                       _ptr(k_block_mean), _ptr(v_block_mean), _ptr(k_window), _ptr(v_window), cap,
                       _ptr(window_len), _ptr(seq_len), max_T, float(scale), _ptr(logits), logits_ld, _ptr(out),
-                      _ptr(workspace), workspace.numel() * workspace.element_size())
+                      _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(k_side), _ptr(v_side))
     _check(load().kvq_decode_attend_ex(h.ptr, ctypes.byref(d), _stream(stream)))
 
 

@@ -698,6 +698,20 @@ int kvq_decode_attend_ex(kvq_handle h, const kvq_decode_desc* d, void* stream) {
                              d->out, &ns, &chunk, &need))
         return e;
     DecodeExtras x;
+    if (d->k_side || d->v_side) {
+        if (d->k_block_mean || d->v_block_mean)
+            return fail(KVQ_EINVAL, "side records and block means describe different caches: give one kind");
+        if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
+        if (!kvq::decode_uses_mma(h) || h->d > 128)
+            return fail(KVQ_EUNSUPPORTED, "decode over double-quantized NSN caches is built for d <= 128 and b <= 3");
+        if (!d->k_side || !d->v_side || !aligned(d->k_side, 16) || !aligned(d->v_side, 16))
+            return fail(KVQ_EINVAL, "side records must both be non-null and 16-byte aligned");
+        if (d->k->capacity % 128 != 0 || d->v->capacity % 128 != 0)
+            return fail(KVQ_EINVAL, "NSN cache capacities must be multiples of 128 (one side record per 128 tokens)");
+        x.dq = true;
+        x.kmean = reinterpret_cast<const uint16_t*>(d->k_side);
+        x.vmean = reinterpret_cast<const uint16_t*>(d->v_side);
+    }
     if (d->k_block_mean || d->v_block_mean) {
         if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
         if (!kvq::decode_uses_mma(h))

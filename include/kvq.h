@@ -368,22 +368,28 @@ typedef struct kvq_decode_desc {
     float* out;
     void* workspace;
     size_t ws_bytes;
+    /* NSN caches with double-quantized side data (as kvq_nsn_dq_decode_attend:
+     * the norms hold fp16 ||w||), or NULL; not together with block means. */
+    const uint8_t* k_side;
+    const uint8_t* v_side;
 } kvq_decode_desc;
 
 /*
  * kvq_decode_attend_ex -- decode attention over a packed cache, optionally
  * followed by a full-precision residual window (NSNQuant section 4: the newest
  * tokens stay in fp16 until a block of them is flushed into the packed cache),
- * for plain or NSN caches.  The softmax runs over the packed tokens [0,
+ * for plain caches, NSN caches with fp16 block means, or NSN caches with
+ * double-quantized side records (k_side / v_side).  The softmax runs over the packed tokens [0,
  * seq_len) then the window tokens [0, window_len) of each sequence; window
  * keys and values are used exactly (fp32 arithmetic on the fp16 values).
  * Window logits go to columns max_T + i of the logits rows.  Flushing a full
- * window is kvq_quantize (or kvq_nsn_quantize) of its tokens into the packed
- * arrays at offset seq_len (a multiple of 32; of 128 for NSN caches).
+ * window is kvq_quantize (or kvq_nsn_quantize, kvq_nsn_dq_quantize) of its
+ * tokens into the packed arrays at offset seq_len (a multiple of 32; of 128
+ * for NSN caches).
  * The workspace size is kvq_decode_workspace's (it covers the window).
  * Errors: as kvq_decode_attend and kvq_nsn_decode_attend; KVQ_EINVAL for a
  * window without all its parts or with window_cap outside 1..KVQ_MAX_WINDOW,
- * and for logits_ld too small.
+ * for logits_ld too small, and for side records given with block means.
  */
 int kvq_decode_attend_ex(kvq_handle h, const kvq_decode_desc* desc, void* stream);
 

@@ -369,17 +369,22 @@ def nsn_quantize(k: Constants, x, mean_in=None) -> dict:
 
 
 def window_decode_attend(k: Constants, q, kcache: dict, vcache: dict, kwin, vwin, scale: float,
-                         use_qjl: bool = True, nsn: tuple | None = None):
+                         use_qjl: bool = True, nsn: tuple | None = None, dq: tuple | None = None):
     """Attention over a packed cache followed by a full-precision residual
     window (NSNQuant section 4: the newest tokens stay unquantized until a
     block is flushed).  The packed part is scored as in decode_attend (or
-    nsn_decode_attend when ``nsn`` = (kmean, vmean)); the window's keys and
-    values ([n_win, d], the stored fp16 values widened) are used exactly.
-    One softmax over all packed then window tokens.  Returns (logits over the
-    packed then window tokens [G, T + n_win], out [G, d])."""
+    nsn_decode_attend when ``nsn`` = (kmean, vmean), or nsn_dq_decode_attend
+    when ``dq`` = (kside, vside)); the window's keys and values ([n_win, d],
+    the stored fp16 values widened) are used exactly.  One softmax over all
+    packed then window tokens.  Returns (logits over the packed then window
+    tokens [G, T + n_win], out [G, d])."""
     q = _c(np.atleast_2d(q), np.float64)
     G, d = q.shape
-    if nsn is None:
+    if dq is not None:
+        lp, _ = nsn_dq_decode_attend(k, q, kcache, vcache, dq[0], dq[1], scale, want_logits=True)
+        T = lp.shape[1]
+        vh = nsn_dq_dequantize(k, vcache["codes"], vcache["norm_w"], dq[1])[:T] if T > 0 else np.zeros((0, d))
+    elif nsn is None:
         lp, _ = decode_attend(k, q, kcache, vcache, scale, use_qjl, want_logits=True)
         T = lp.shape[1]
         vh = (dequantize(k, vcache["codes"], vcache.get("bits"), vcache["norm"], vcache["gamma"], use_qjl)

@@ -271,3 +271,71 @@ def test_nsn_dq_workload_full_size_sampled():
                                          want_logits=False)
     assert_close(out.cpu().numpy()[0, 4 * hs:4 * hs + 4], orf, "nsn-dq out (sampled head)")
     print("nsn_dq", pooled_check("nsn_dq"))
+
+
+def test_window_over_a_double_quantized_cache_matches_oracle():
+    """kvq_decode_attend_ex over an oracle-built double-quantized cache (ragged contexts) followed by fp16
+    windows of different lengths: one softmax over the packed then the window tokens."""
+    d, b, batch, hq, hkv, cap, wcap = 128, 2, 2, 8, 2, 512, 96
+    seq_len, win_len = [384, 200], [77, 0]
+    k = oracle.make_constants(d, b, 6)
+    G, S = hq // hkv, batch * hkv
+    R = oracle.nsn_dq_rec_bytes(d)
+    kc = torch.zeros((S, cap, b, d // 32), dtype=torch.int32)
+    vc = torch.zeros((S, cap // 32, b, d), dtype=torch.int32)
+    kn = torch.zeros((S, cap), dtype=torch.float16)
+    vn = torch.zeros_like(kn)
+    ks = torch.zeros((S, cap // 128, R), dtype=torch.uint8)
+    vs = torch.zeros_like(ks)
+    st = []
+    for s in range(S):
+        rk, wk, sk = _dq_oracle_stream(k, wl.nsn_tokens(1, cap, d, seed=1100 + s)[0].double().numpy())
+        rv, wv, sv = _dq_oracle_stream(k, wl.nsn_tokens(1, cap, d, seed=1200 + s)[0].double().numpy())
+        kc[s] = torch.from_numpy(oracle.pack_codes(rk["codes"], b).view(np.int32))
+        vc[s] = torch.from_numpy(oracle.pack_codes_block32(rv["codes"], b).view(np.int32).reshape(cap // 32, b, d))
+        kn[s], vn[s] = torch.from_numpy(wk), torch.from_numpy(wv)
+        ks[s], vs[s] = torch.from_numpy(rk["side"]), torch.from_numpy(rv["side"])
+        st.append((sk, sv, rk["side"], rv["side"]))
+    kw = wl.nsn_tokens(S, wcap, d, seed=1300).to(torch.float16)
+    vw = wl.nsn_tokens(S, wcap, d, seed=1301).to(torch.float16)
+    q = wl.queries(batch, hq, d, seed=83)
+    max_T = max(seq_len)
+    with kvq.Handle(d, b, 6, qjl=False) as h:
+        out = torch.empty((batch, hq, d), dtype=torch.float32, device="cuda")
+        logits = torch.empty((batch, hq, max_T + wcap), dtype=torch.float32, device="cuda")
+        ws = torch.empty(kvq.kvq_decode_workspace(h, batch, hq, hkv, max_T), dtype=torch.uint8, device="cuda")
+        kcd, vcd, knd, vnd, ksd, vsd = (t.cuda() for t in (kc, vc, kn, vn, ks, vs))
+        kvq.kvq_decode_attend_ex(h, q.cuda(), hkv, kvq.make_cache(kcd, None, knd, cap, 0),
+                                 kvq.make_cache(vcd, None, vnd, cap, 1),
+                                 torch.tensor(seq_len, dtype=torch.int32, device="cuda"), max_T, d ** -0.5, out, ws,
+                                 k_window=kw.cuda(), v_window=vw.cuda(),
+                                 window_len=torch.tensor(win_len, dtype=torch.int32, device="cuda"),
+                                 logits=logits, k_side=ksd, v_side=vsd)
+        assert kvq.kvq_status(h)[0] == 0
+        # side records and block means together are refused
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_decode_attend_ex(h, q.cuda(), hkv, kvq.make_cache(kcd, None, knd, cap, 0),
+                                     kvq.make_cache(vcd, None, vnd, cap, 1),
+                                     torch.tensor(seq_len, dtype=torch.int32, device="cuda"), max_T, d ** -0.5, out,
+                                     ws, k_block_mean=torch.zeros((S, cap // 128, d), dtype=torch.float16,
+                                                                  device="cuda"),
+                                     v_block_mean=torch.zeros((S, cap // 128, d), dtype=torch.float16, device="cuda"),
+                                     k_side=ksd, v_side=vsd)
+        assert e.value.code == kvq.KVQ_EINVAL
+        out, logits = out.cpu().numpy(), logits.cpu().numpy()
+    qd = q.double().numpy()
+    for bi in range(batch):
+        T, W = seq_len[bi], win_len[bi]
+        for hk in range(hkv):
+            s = bi * hkv + hk
+            sk, sv, rks, rvs = st[s]
+            sk = {key: v[:T] for key, v in sk.items()}
+            sv = {key: v[:T] for key, v in sv.items()}
+            lr, orf = oracle.window_decode_attend(k, qd[bi, hk * G:(hk + 1) * G], sk, sv,
+                                                  kw[s, :W].double().numpy(), vw[s, :W].double().numpy(), d ** -0.5,
+                                                  False, dq=(rks, rvs))
+            assert_close(out[bi, hk * G:(hk + 1) * G], orf, f"dq + window out b{bi} kvh{hk}")
+            assert_close(logits[bi, hk * G:(hk + 1) * G, :T], lr[:, :T], f"dq + window packed logits b{bi} kvh{hk}")
+            if W:
+                assert_close(logits[bi, hk * G:(hk + 1) * G, max_T:max_T + W], lr[:, T:],
+                             f"dq + window window logits b{bi} kvh{hk}")

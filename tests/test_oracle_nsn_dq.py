@@ -141,3 +141,30 @@ def test_double_quantization_keeps_the_reconstruction_quality():
     xp = oracle.dequantize(k, qp["codes"], None, qp["norm"], qp["gamma"], False)
     c0, c1, cp = cos(x, x0), cos(x, x1), cos(x, xp)
     assert c1 > c0 - 0.005 and c1 > cp + 0.05, (c0, c1, cp)
+
+
+def test_window_over_a_double_quantized_cache():
+    """A double-quantized NSN cache followed by an exact window: with an empty window it is the cache's decode;
+    in general one softmax over the tokens rebuilt from the stored values, then the window tokens."""
+    d, T, W, G = 64, 256, 37, 2
+    k = oracle.make_constants(d, 2, 12)
+    rk = oracle.nsn_dq_quantize(k, _tokens(T, d, 21))
+    rv = oracle.nsn_dq_quantize(k, _tokens(T, d, 22))
+    kc = dict(codes=rk["codes"], norm_w=rk["norm_w"].astype(np.float16).astype(np.float64))
+    vc = dict(codes=rv["codes"], norm_w=rv["norm_w"].astype(np.float16).astype(np.float64))
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((G, d)) / 8
+    kw = rng.standard_normal((W, d)).astype(np.float16).astype(np.float64)
+    vw = rng.standard_normal((W, d)).astype(np.float16).astype(np.float64)
+    l0, o0 = oracle.window_decode_attend(k, q, kc, vc, np.zeros((0, d)), np.zeros((0, d)), 0.3, False,
+                                         dq=(rk["side"], rv["side"]))
+    l1, o1 = oracle.nsn_dq_decode_attend(k, q, kc, vc, rk["side"], rv["side"], 0.3)
+    np.testing.assert_array_equal(l0, l1)
+    np.testing.assert_allclose(o0, o1, rtol=1e-13, atol=1e-15)
+    l, o = oracle.window_decode_attend(k, q, kc, vc, kw, vw, 0.3, False, dq=(rk["side"], rv["side"]))
+    Kh = np.concatenate([oracle.nsn_dq_dequantize(k, kc["codes"], kc["norm_w"], rk["side"]), kw])
+    Vh = np.concatenate([oracle.nsn_dq_dequantize(k, vc["codes"], vc["norm_w"], rv["side"]), vw])
+    lw = 0.3 * q @ Kh.T
+    e = np.exp(lw - lw.max(1, keepdims=True))
+    np.testing.assert_allclose(l, lw, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(o, (e @ Vh) / e.sum(1, keepdims=True), rtol=1e-11, atol=1e-13)
