@@ -639,8 +639,6 @@ int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int
     g_err.clear();
     if (int e = check_handle(h)) return e;
     if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
-    if (!kvq::decode_uses_mma(h))
-        return fail(KVQ_EUNSUPPORTED, "decode over NSN caches is built for b <= 2, and b = 3 at d <= 128");
     int ns = 0;
     int64_t chunk = 0;
     size_t need = 0;
@@ -714,8 +712,6 @@ int kvq_decode_attend_ex(kvq_handle h, const kvq_decode_desc* d, void* stream) {
     }
     if (d->k_block_mean || d->v_block_mean) {
         if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
-        if (!kvq::decode_uses_mma(h))
-        return fail(KVQ_EUNSUPPORTED, "decode over NSN caches is built for b <= 2, and b = 3 at d <= 128");
         if (!d->k_block_mean || !d->v_block_mean || !aligned(d->k_block_mean, 16) || !aligned(d->v_block_mean, 16))
             return fail(KVQ_EINVAL, "block means must both be non-null and 16-byte aligned");
         if (d->k->capacity % 128 != 0 || d->v->capacity % 128 != 0)

@@ -125,8 +125,13 @@ __device__ __forceinline__ int code_at(const uint32_t* planes, int words_per_pla
 }
 
 // One (split, kv head, batch) per block: tokens [split*chunk, (split+1)*chunk).
-template <int D, int B, bool QJL, int G>
+// NSN (no QJL): caches written by the NSN front end, fp16 block means per 128
+// tokens (NSNQuant sections 1 and 4): the logit is scale ||x||/sqrt(d)
+// (||w||/d <q', c[code]> + <q, o_blk>), the code weights are e ||x|| ||w|| / sqrt(d)
+// and the block means enter the partial's second vector with e ||x|| / sqrt(d).
+template <int D, int B, bool QJL, int G, bool NSN = false>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
+    static_assert(!(NSN && QJL), "NSN caches carry no QJL sketch");
     constexpr int M = D;                 // QJL rows
     constexpr int WP = D / 32;           // words per plane
     constexpr int KW = B * WP;           // code words per vector
@@ -145,6 +150,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     __shared__ float svn[TT], svg[TT];
     __shared__ float sred[G][kDecThreads / 32];
     __shared__ float smax[G], salpha[G], ssum[G];
+    constexpr int NBT = TT / 128;                      // NSN blocks per tile
+    __shared__ float sq0[NSN ? G : 1][NSN ? D : 1];    // NSN: the query in the original domain
+    __shared__ float sqo[G][NBT];                      // NSN: scale/sqrt(d) <q, o_blk> of the tile's blocks
+    __shared__ float sbeta[G][NBT];                    // NSN: sum of e ||x|| / sqrt(d) per block of the tile
+    const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
 
     const int64_t T = min(static_cast<int64_t>(max(a.seq_len[bi], 0)), a.max_T);
     const int64_t t0 = static_cast<int64_t>(split) * a.chunk;
@@ -157,6 +167,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     if (QJL)
         for (int e = tid; e < G * M; e += blockDim.x) spq[e / M][e % M] = a.qproj[(qh0 + e / M) * M + e % M];
     if (tid < (1 << B)) scb[tid] = a.centroid[tid];
+    if constexpr (NSN) {
+        for (int e = tid; e < G * D; e += blockDim.x) {
+            const int64_t i = (qh0 + e / D) * D + e % D;
+            const uint16_t u = reinterpret_cast<const uint16_t*>(a.q)[a.qdtype == 0 ? 0 : i];
+            sq0[e / D][e % D] = a.qdtype == 0 ? reinterpret_cast<const float*>(a.q)[i]
+                                : a.qdtype == 1 ? __half2float(__ushort_as_half(u))
+                                                : __uint_as_float(static_cast<uint32_t>(u) << 16);
+        }
+    }
     if (tid < G) {
         smax[tid] = -INFINITY;
         ssum[tid] = 0.f;
@@ -175,8 +194,26 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     const uint32_t* vq = QJL ? a.vqjl + stream * (a.vcap / 32) * M : nullptr;
     const __half2* vn = a.vnorms + stream * a.vcap;
     const float kappa = kSqrtHalfPi / M;
+    const __half* kmean = NSN ? a.kmean + stream * (a.kcap / 128) * D : nullptr;
+    const __half* vmean = NSN ? a.vmean + stream * (a.vcap / 128) * D : nullptr;
 
     for (int64_t tb = t0; tb < t1e; tb += TT) {
+        if constexpr (NSN) {
+            // scale/sqrt(d) <q_g, o_blk> for the tile's blocks (tb is a multiple of 128); a
+            // block past the cache's tokens gives a value no valid token uses
+            const int warp = tid >> 5, lane = tid & 31;
+            for (int pr = warp; pr < G * NBT; pr += kDecThreads / 32) {
+                const int g = pr / NBT, bq = pr % NBT;
+                const int64_t blk = tb / 128 + bq;
+                float acc = 0.f;
+                if (blk * 128 < t1)
+                    for (int j = lane; j < D; j += 32) acc = fmaf(sq0[g][j], __half2float(kmean[blk * D + j]), acc);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                if (lane == 0) sqo[g][bq] = acc * a.scale * inv_sqrt_d;
+            }
+            __syncthreads();
+        }
         // ---- phase A: logits, one token per thread ----
         const int64_t t = tb + tid;
         const bool mine = tid < TT;
@@ -206,8 +243,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
                     for (int g = 0; g < G; ++g) accq[g] = fmaf(spq[g][i], s, accq[g]);
                 }
             }
+            if constexpr (NSN) {
 #pragma unroll
-            for (int g = 0; g < G; ++g) l[g] = a.scale * (nk.x / D) * (acc[g] + (QJL ? kappa * nk.y * accq[g] : 0.f));
+                for (int g = 0; g < G; ++g)
+                    l[g] = nk.x * fmaf(a.scale * inv_sqrt_d * (nk.y / D), acc[g], sqo[g][tid >> 7]);
+            } else {
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+                    l[g] = a.scale * (nk.x / D) * (acc[g] + (QJL ? kappa * nk.y * accq[g] : 0.f));
+            }
         } else {
 #pragma unroll
             for (int g = 0; g < G; ++g) l[g] = -INFINITY;
@@ -226,9 +270,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
                 for (int e = tid; e < nblk * M; e += kDecThreads) (&svq[0][0])[e] = vq[blk0 * M + e];
         }
         if (mine && t < t1) {
+            // NSN: the code weight factor ||x|| ||w|| / sqrt(d) and the block-mean factor ||x|| / sqrt(d)
             const float2 nv = __half22float2(vn[t]);
-            svn[tid] = nv.x;
-            svg[tid] = nv.y;
+            svn[tid] = NSN ? nv.x * nv.y * inv_sqrt_d : nv.x;
+            svg[tid] = NSN ? nv.x * inv_sqrt_d : nv.y;
         }
         // ---- phase B: tile max, running max, weights ----
 #pragma unroll
@@ -264,6 +309,25 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
             for (int k = 0; k < kDecThreads / 32; ++k) s += sred[tid][k];
             ssum[tid] = ssum[tid] * salpha[tid] + s;
         }
+        if constexpr (NSN) {
+            // sum of e ||x|| / sqrt(d) over each block of the tile: token tid is in block tid / 128
+            __syncthreads();  // sred is reused
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float b = (mine && tb + tid < t1) ? sw[g][tid] * svg[tid] : 0.f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
+                if ((tid & 31) == 0) sred[g][tid >> 5] = b;
+            }
+            __syncthreads();
+            if (tid < G * NBT) {
+                const int g = tid / NBT, bq = tid % NBT;
+                float b = 0.f;
+                for (int k = bq * 4; k < bq * 4 + 4 && k < kDecThreads / 32; ++k) b += sred[g][k];
+                sbeta[g][bq] = b;
+            }
+            __syncthreads();
+        }
         // ---- phase C: value sums, one coordinate (or QJL row) per thread ----
         const int ntok = static_cast<int>(min(static_cast<int64_t>(TT), t1 - tb > 0 ? t1 - tb : 0));
 #pragma unroll
@@ -293,6 +357,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
                     if (second) accA2[g] += acc[g];
                     else accA[g] += acc[g];
                 }
+                if constexpr (NSN) {
+                    // O_j += sum over the tile's blocks of beta o_v,blk[j] (second vector of the partial)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        float o = 0.f;
+                        for (int bq = 0; bq < NBT; ++bq) {
+                            const int64_t blk = tb / 128 + bq;
+                            if (blk * 128 < t1) o = fmaf(sbeta[g][bq], __half2float(vmean[blk * D + j]), o);
+                        }
+                        if (second) accB2[g] += o;
+                        else accB[g] += o;
+                    }
+                }
             } else {
                 const int i = role - D;
                 float acc[G];
@@ -319,8 +396,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             float* pp = a.part + ((qh0 + g) * a.nsplit + split) * PART;
-            if (role < D) pp[2 + role] = k ? accA2[g] : accA[g];
-            else pp[2 + role] = k ? accB2[g] : accB[g];
+            if (role < D) {
+                pp[2 + role] = k ? accA2[g] : accA[g];
+                if (NSN) pp[2 + D + role] = k ? accB2[g] : accB[g];  // the block-mean term O
+            } else {
+                pp[2 + role] = k ? accB2[g] : accB[g];
+            }
         }
     }
     if (tid < G) {
@@ -519,17 +600,31 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
         default: qproj_kernel<D, 2, QJL><<<nbh, block, 0, s>>>(a); break;
     }
     const dim3 grid(a.nsplit_run, a.hkv, a.batch);
-    switch (a.G) {
-        case 1: decode_split_kernel<D, B, QJL, 1><<<grid, block, 0, s>>>(a); break;
-        case 2: decode_split_kernel<D, B, QJL, 2><<<grid, block, 0, s>>>(a); break;
-        case 4: decode_split_kernel<D, B, QJL, 4><<<grid, block, 0, s>>>(a); break;
-        default: decode_split_kernel<D, B, QJL, 8><<<grid, block, 0, s>>>(a); break;
+    bool nsn = false;
+    if constexpr (!QJL) nsn = a.nsn != 0;
+    if (nsn) {
+        if constexpr (!QJL) {
+            switch (a.G) {
+                case 1: decode_split_kernel<D, B, false, 1, true><<<grid, block, 0, s>>>(a); break;
+                case 2: decode_split_kernel<D, B, false, 2, true><<<grid, block, 0, s>>>(a); break;
+                case 4: decode_split_kernel<D, B, false, 4, true><<<grid, block, 0, s>>>(a); break;
+                default: decode_split_kernel<D, B, false, 8, true><<<grid, block, 0, s>>>(a); break;
+            }
+        }
+    } else {
+        switch (a.G) {
+            case 1: decode_split_kernel<D, B, QJL, 1><<<grid, block, 0, s>>>(a); break;
+            case 2: decode_split_kernel<D, B, QJL, 2><<<grid, block, 0, s>>>(a); break;
+            case 4: decode_split_kernel<D, B, QJL, 4><<<grid, block, 0, s>>>(a); break;
+            default: decode_split_kernel<D, B, QJL, 8><<<grid, block, 0, s>>>(a); break;
+        }
     }
     if (a.kwin != nullptr) {
         const cudaError_t e = launch_decode_window(nullptr, a, s);
         if (e != cudaSuccess) return e;
     }
-    decode_combine_kernel<D, QJL><<<nbh, block, 0, s>>>(a);
+    if (nsn) decode_combine_kernel<D, false, true><<<nbh, block, 0, s>>>(a);
+    else decode_combine_kernel<D, QJL><<<nbh, block, 0, s>>>(a);
     return cudaGetLastError();
 }
 

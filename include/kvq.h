@@ -280,8 +280,8 @@ int kvq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq,
  *                 (bi, hi) at block (bi * hkv + hi) * capacity/128, 16-byte
  *                 aligned.  Capacities must be multiples of 128.
  * The workspace size is kvq_decode_workspace's.  Requires a handle without
- * KVQ_QJL (KVQ_EINVAL) and b <= 2, or b = 3 at d <= 128 (KVQ_EUNSUPPORTED
- * otherwise).
+ * KVQ_QJL (KVQ_EINVAL); every (d, b) is built (b <= 2, and b = 3 at d <= 128,
+ * on the tensor-core path, the rest on the CUDA cores).
  */
 int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
                           const kvq_cache* v, const uint16_t* k_block_mean, const uint16_t* v_block_mean,

@@ -207,6 +207,11 @@ def check_nsn_decode(d, b, batch, hq, hkv, seq_len, cap, qdtype=torch.bfloat16, 
     (128, 1, 2, 4, 1, [0, 129], 256),        # an empty context
     (128, 3, 1, 8, 2, [700], 768),           # 3 bits (parity plane)
     (64, 3, 1, 4, 1, [384], 384),
+    # CUDA-core path (4-bit codebooks, 3 bits at d = 256)
+    (128, 4, 2, 8, 2, [1000, 300], 1024),    # GQA 4:1, ragged contexts, partial blocks
+    (64, 4, 1, 4, 4, [640], 640),            # GQA 1:1
+    (256, 3, 1, 8, 1, [700], 768),           # GQA 8:1, 128-token tiles
+    (256, 4, 2, 4, 2, [0, 300], 384),        # an empty context
 ])
 def test_nsn_decode_matches_oracle(d, b, batch, hq, hkv, seq_len, cap):
     check_nsn_decode(d, b, batch, hq, hkv, seq_len, cap)
