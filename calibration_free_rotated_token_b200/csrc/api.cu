@@ -465,7 +465,8 @@ int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, in
     if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "the NSN front end takes a handle without KVQ_QJL");
     if (n_heads < 0 || n_tok < 0) return fail(KVQ_EINVAL, "negative size");
     if (n_tok % 128 != 0) return fail(KVQ_EINVAL, "n_tok must be a multiple of 128 (NSN blocks of 128 tokens)");
-    if (h->d > 128) return fail(KVQ_EUNSUPPORTED, "the NSN front end is built for d <= 128");
+    if (h->d > 128 && dtype == KVQ_F32)
+        return fail(KVQ_EUNSUPPORTED, "the NSN front end at d = 256 is built for fp16 and bf16 input");
     if (n_heads * n_tok == 0) return KVQ_OK;
     if (!block_mean || !aligned(block_mean, 2)) return fail(KVQ_EINVAL, "block_mean must be non-null");
     return quantize_common(h, x, dtype, n_heads * n_tok, h->d, layout, codes, nullptr, norms, block_mean, true,

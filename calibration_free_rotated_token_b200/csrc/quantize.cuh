@@ -54,10 +54,11 @@ struct QCfg {
     static constexpr int kStages = kCoop ? kStagesCap : (kStagesCap & ~1);
     static constexpr int kThreads = 256;
     static constexpr int kTmemCols = !QJL ? 0 : (kCoop ? 512 : (4 * D < 32 ? 32 : 4 * D));
-    static constexpr int kAuxBytes = 4096;
+    static constexpr int kAuxBytes = NSN ? 8192 : 4096;
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kSBytes + kAuxBytes;
     static_assert(kStages >= 1, "input tile does not fit in shared memory");
-    static_assert(!(NSN && (QJL || kCoop)), "NSN front end: no QJL, D <= 128");
+    static_assert(!(NSN && QJL), "NSN front end: no QJL");
+    static_assert(!(NSN && kCoop && DT == DT_F32), "NSN front end at D = 256: 16-bit input");
 };
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
@@ -629,10 +630,64 @@ __global__ void __launch_bounds__(256, 1)
 
             float2 v[64];
             const float ss = load_row_coop<DT>(sp, r, h, v, a.pair_sign);
-            named_bar_sync(3, 256);
-            if (tid == 0) issue_tile(i + kStages);
-            const float nrm = sqrtf(ss);
-            if (h == 0) flag_norm(ss, nrm, a.status);
+            float nrm, nx = 0.f;
+            if constexpr (NSN) {
+                // NSN front end (NSNQuant sections 1-2) on a 128-token block: u = sqrt(D) x / ||x||,
+                // o = the fp16 channel means of u, w = u - o.  The loaded v is this half of the top
+                // butterfly of delta .* x, which is linear: the half of delta .* w is sc v - bo with
+                // bo the same butterfly of delta .* o; ||w||^2 is half the sum of both halves' squares.
+                float* ssc = reinterpret_cast<float*>(aux + 2048);  // [128] sc per row
+                float* sbo = reinterpret_cast<float*>(aux + 2560);  // [2][128] butterflies of delta .* o
+                float* swx = reinterpret_cast<float*>(aux + 3584);  // [2][128] half sums of squares
+                nx = sqrtf(ss);
+                if (h == 0) flag_norm(ss, nx, a.status);
+                const float sc = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
+                if (h == 0) ssc[r] = sc;
+                named_bar_sync(3, 256);
+                {
+                    // block mean of channel j = tid over the tile's rows
+                    const int j = tid;
+                    float acc = 0.f;
+                    for (int t = 0; t < kTileRows; ++t) {
+                        const uint8_t* p = sp + (j / 64) * 16384 + t * 128 + ((((j % 64) / 8) ^ (t & 7)) << 4) + (j % 8) * 2;
+                        const uint16_t hv = *reinterpret_cast<const uint16_t*>(p);
+                        const float xt = (DT == DT_BF16) ? u2f(static_cast<uint32_t>(hv) << 16)
+                                                         : __half2float(*reinterpret_cast<const __half*>(&hv));
+                        acc = fmaf(xt, ssc[t], acc);
+                    }
+                    const __half o16 = __float2half_rn(acc * (1.0f / kTileRows));
+                    so16[j] = o16;
+                    a.block_mean[tile * D + j] = o16;
+                }
+                named_bar_sync(3, 256);
+                if (tid == 0) issue_tile(i + kStages);  // the stage is read
+                {
+                    // sbo[hh][j] = delta_j o_j + (-1)^hh delta_{j+128} o_{j+128}
+                    const int hh = tid >> 7, j = tid & 127;
+                    auto sgn = [&](int c) {
+                        return ((a.pair_sign[c >> 1] >> ((c & 1) ? 31 : 15)) & 1u) ? -1.f : 1.f;
+                    };
+                    const float lo = sgn(j) * __half2float(so16[j]);
+                    const float hi = sgn(j + 128) * __half2float(so16[j + 128]);
+                    sbo[hh * 128 + j] = hh ? lo - hi : lo + hi;
+                }
+                named_bar_sync(3, 256);
+                const float2 sc2 = make_float2(sc, sc);
+                const float2* bo2 = reinterpret_cast<const float2*>(sbo + h * 128);
+#pragma unroll
+                for (int k = 0; k < 64; ++k) {
+                    const float2 b = bo2[k];
+                    v[k] = __ffma2_rn(v[k], sc2, make_float2(-b.x, -b.y));
+                }
+                swx[h * 128 + r] = sumsq(v);
+                named_bar_sync(3, 256);
+                nrm = sqrtf(0.5f * (swx[r] + swx[128 + r]));
+            } else {
+                named_bar_sync(3, 256);
+                if (tid == 0) issue_tile(i + kStages);
+                nrm = sqrtf(ss);
+                if (h == 0) flag_norm(ss, nrm, a.status);
+            }
             fwht<64>(v);
             const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
             uint32_t planes[B][4];
@@ -667,7 +722,8 @@ __global__ void __launch_bounds__(256, 1)
             if (valid) {
                 if (h == 0) {
                     const float g = nrm > 0.f ? sqrtf(xch[r] + xch[128 + r]) : 0.f;
-                    a.norms[vidx] = __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
+                    a.norms[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
+                                        : __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
                 }
             }
             if (QJL) {

@@ -24,8 +24,16 @@ namespace {
 template <int D, int B, bool QJL, bool NSN>
 cudaError_t by_dtype(const CUtensorMap& map, const CUtensorMap& map1, int dtype, const QuantArgs& a, int sms,
                      cudaStream_t s) {
-    if constexpr (NSN && (QJL || D > 128)) {
+    if constexpr (NSN && QJL) {
         return cudaErrorNotSupported;
+    } else if constexpr (NSN && D > 128) {
+        // d = 256: the in-register transform kernel, 16-bit input, fp16 side data
+        if (a.side != nullptr) return cudaErrorNotSupported;
+        switch (dtype) {
+            case DT_F16: return launch_quantize_t<D, B, false, DT_F16, true>(map, a, sms, s);
+            case DT_BF16: return launch_quantize_t<D, B, false, DT_BF16, true>(map, a, sms, s);
+            default: return cudaErrorNotSupported;
+        }
     } else if constexpr (NSN) {
         // double-quantized side data (a.side): 16-bit input only
         if (a.side != nullptr) {

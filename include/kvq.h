@@ -206,7 +206,8 @@ int kvq_quantize_batch(kvq_handle h, int count, const kvq_quant_job* jobs, void*
  *   codes       device, n_heads * n_tok * b * d/32 uint32.
  *   norms       device, n_heads * n_tok * 2 fp16.
  *   block_mean  device, n_heads * (n_tok/128) * d fp16.
- * Requires a handle without KVQ_QJL (KVQ_EINVAL otherwise).
+ * Requires a handle without KVQ_QJL (KVQ_EINVAL otherwise); at d = 256 the
+ * input must be fp16 or bf16 (fp32 returns KVQ_EUNSUPPORTED).
  */
 int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, int layout,
                      uint32_t* codes, uint16_t* norms, uint16_t* block_mean, void* stream);

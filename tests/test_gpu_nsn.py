@@ -68,7 +68,9 @@ def check_head(k, x, codes_g, norms_g, means_g, pool=None):
 
 
 @pytest.mark.parametrize("d,b,dtype", [(128, 2, torch.bfloat16), (128, 1, torch.float16), (64, 3, torch.float32),
-                                       (64, 4, torch.bfloat16)])
+                                       (64, 4, torch.bfloat16),
+                                       # d = 256: the in-register transform kernel, two threads per vector
+                                       (256, 2, torch.bfloat16), (256, 3, torch.float16), (256, 4, torch.bfloat16)])
 def test_nsn_matches_oracle(d, b, dtype):
     x = wl.nsn_tokens(2, 512, d, seed=d + b, dtype=dtype)
     x[1, 130] = 0  # a zero token inside a block
@@ -270,3 +272,11 @@ def test_nsn_decode_workload_full_size_sampled():
                                       d ** -0.5, want_logits=False)
     assert_close(out[0, 4 * hs:4 * hs + 4], orf, f"nsn workload out kvh{hs}")
     assert np.isfinite(out).all()
+
+
+def test_nsn_front_end_at_d256_rejects_fp32():
+    with kvq.Handle(256, 2, 3, qjl=False) as h:
+        x = torch.randn(1, 128, 256, device="cuda", dtype=torch.float32)
+        with pytest.raises(kvq.KvqError) as e:
+            run_nsn(h, x)
+        assert e.value.code == kvq.KVQ_EUNSUPPORTED
