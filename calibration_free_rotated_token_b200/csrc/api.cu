@@ -473,7 +473,7 @@ int kvq_nsn_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, in
                            stream);
 }
 
-size_t kvq_nsn_dq_side_bytes(int d) { return (d == 64 || d == 128) ? dq_side_bytes(d) : 0; }
+size_t kvq_nsn_dq_side_bytes(int d) { return (d == 64 || d == 128 || d == 256) ? dq_side_bytes(d) : 0; }
 
 int kvq_nsn_dq_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, int layout,
                         uint32_t* codes, uint16_t* wnorms, uint8_t* side, void* stream) {
@@ -482,7 +482,6 @@ int kvq_nsn_dq_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads,
     if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "the NSN front end takes a handle without KVQ_QJL");
     if (n_heads < 0 || n_tok < 0) return fail(KVQ_EINVAL, "negative size");
     if (n_tok % 128 != 0) return fail(KVQ_EINVAL, "n_tok must be a multiple of 128 (NSN blocks of 128 tokens)");
-    if (h->d > 128) return fail(KVQ_EUNSUPPORTED, "the NSN front end is built for d <= 128");
     if (dtype != KVQ_F16 && dtype != KVQ_BF16)
         return fail(dtype == KVQ_F32 ? KVQ_EUNSUPPORTED : KVQ_EINVAL,
                     "double-quantized NSN side data are built for fp16 and bf16 input");
@@ -665,8 +664,6 @@ int kvq_nsn_dq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, 
     g_err.clear();
     if (int e = check_handle(h)) return e;
     if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
-    if (!kvq::decode_uses_mma(h) || h->d > 128)
-        return fail(KVQ_EUNSUPPORTED, "decode over double-quantized NSN caches is built for d <= 128 and b <= 3");
     int ns = 0;
     int64_t chunk = 0;
     size_t need = 0;
@@ -701,8 +698,6 @@ int kvq_decode_attend_ex(kvq_handle h, const kvq_decode_desc* d, void* stream) {
         if (d->k_block_mean || d->v_block_mean)
             return fail(KVQ_EINVAL, "side records and block means describe different caches: give one kind");
         if (h->flags & KVQ_QJL) return fail(KVQ_EINVAL, "NSN caches carry no QJL sketch: use a handle without KVQ_QJL");
-        if (!kvq::decode_uses_mma(h) || h->d > 128)
-            return fail(KVQ_EUNSUPPORTED, "decode over double-quantized NSN caches is built for d <= 128 and b <= 3");
         if (!d->k_side || !d->v_side || !aligned(d->k_side, 16) || !aligned(d->v_side, 16))
             return fail(KVQ_EINVAL, "side records must both be non-null and 16-byte aligned");
         if (d->k->capacity % 128 != 0 || d->v->capacity % 128 != 0)

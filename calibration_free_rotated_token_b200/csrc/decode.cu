@@ -18,6 +18,8 @@
 #include <cfloat>
 #include <mutex>
 
+#include <type_traits>
+
 #include "kvq_internal.h"
 #include "sm100.cuh"
 
@@ -129,9 +131,14 @@ __device__ __forceinline__ int code_at(const uint32_t* planes, int words_per_pla
 // tokens (NSNQuant sections 1 and 4): the logit is scale ||x||/sqrt(d)
 // (||w||/d <q', c[code]> + <q, o_blk>), the code weights are e ||x|| ||w|| / sqrt(d)
 // and the block means enter the partial's second vector with e ||x|| / sqrt(d).
-template <int D, int B, bool QJL, int G, bool NSN = false>
+// DQ (with NSN): the norms hold fp16 ||w|| per token and the block means are
+// side records (4-bit codes of ||x|| and of the means, NSNQuant section 3):
+// ||x|| reads as n1 = q nstep and the mean as o_hat = lo + step q.
+template <int D, int B, bool QJL, int G, bool NSN = false, bool DQ = false>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
     static_assert(!(NSN && QJL), "NSN caches carry no QJL sketch");
+    static_assert(!DQ || NSN, "double-quantized side data belong to NSN caches");
+    constexpr int RB = (8 + D / 2 + 64 + 15) / 16 * 16;  // DQ: bytes of one side record
     constexpr int M = D;                 // QJL rows
     constexpr int WP = D / 32;           // words per plane
     constexpr int KW = B * WP;           // code words per vector
@@ -194,8 +201,41 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     const uint32_t* vq = QJL ? a.vqjl + stream * (a.vcap / 32) * M : nullptr;
     const __half2* vn = a.vnorms + stream * a.vcap;
     const float kappa = kSqrtHalfPi / M;
-    const __half* kmean = NSN ? a.kmean + stream * (a.kcap / 128) * D : nullptr;
-    const __half* vmean = NSN ? a.vmean + stream * (a.vcap / 128) * D : nullptr;
+    const __half* kmean = (NSN && !DQ) ? a.kmean + stream * (a.kcap / 128) * D : nullptr;
+    const __half* vmean = (NSN && !DQ) ? a.vmean + stream * (a.vcap / 128) * D : nullptr;
+    const uint8_t* krec = DQ ? reinterpret_cast<const uint8_t*>(a.kmean) + stream * (a.kcap / 128) * RB : nullptr;
+    const uint8_t* vrec = DQ ? reinterpret_cast<const uint8_t*>(a.vmean) + stream * (a.vcap / 128) * RB : nullptr;
+    auto f16at = [](const uint8_t* p) { return __half2float(*reinterpret_cast<const __half*>(p)); };
+    auto nib = [](const uint8_t* p, int i) { return static_cast<float>((p[i >> 1] >> ((i & 1) * 4)) & 15); };
+    // block mean of channel j (fp16 as stored, or o_hat from the record) and the stored norms of token t
+    auto kmean_at = [&](int64_t blk, int j) {
+        if constexpr (DQ) {
+            const uint8_t* r = krec + blk * RB;
+            return fmaf(f16at(r + 2), nib(r + 8, j), f16at(r));
+        } else {
+            return __half2float(kmean[blk * D + j]);
+        }
+    };
+    auto vmean_at = [&](int64_t blk, int j) {
+        if constexpr (DQ) {
+            const uint8_t* r = vrec + blk * RB;
+            return fmaf(f16at(r + 2), nib(r + 8, j), f16at(r));
+        } else {
+            return __half2float(vmean[blk * D + j]);
+        }
+    };
+    // DQ norms: one fp16 ||w|| per token (the stream's base in fp16 units)
+    const __half* knh = reinterpret_cast<const __half*>(a.knorms) + stream * a.kcap;
+    const __half* vnh = reinterpret_cast<const __half*>(a.vnorms) + stream * a.vcap;
+    auto norms_at = [&](bool key, int64_t tt) -> float2 {
+        if constexpr (DQ) {
+            const uint8_t* r = (key ? krec : vrec) + (tt >> 7) * RB;
+            const float n1 = nib(r + 8 + D / 2, static_cast<int>(tt & 127)) * f16at(r + 4);
+            return make_float2(n1, __half2float((key ? knh : vnh)[tt]));
+        } else {
+            return __half22float2((key ? kn : vn)[tt]);
+        }
+    };
 
     for (int64_t tb = t0; tb < t1e; tb += TT) {
         if constexpr (NSN) {
@@ -207,7 +247,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
                 const int64_t blk = tb / 128 + bq;
                 float acc = 0.f;
                 if (blk * 128 < t1)
-                    for (int j = lane; j < D; j += 32) acc = fmaf(sq0[g][j], __half2float(kmean[blk * D + j]), acc);
+                    for (int j = lane; j < D; j += 32) acc = fmaf(sq0[g][j], kmean_at(blk, j), acc);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
                 if (lane == 0) sqo[g][bq] = acc * a.scale * inv_sqrt_d;
@@ -231,7 +271,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 #pragma unroll
                 for (int g = 0; g < G; ++g) acc[g] = fmaf(sqr[g][j], c, acc[g]);
             }
-            const float2 nk = __half22float2(kn[t]);
+            const float2 nk = norms_at(true, t);
             if (QJL) {
                 uint32_t qw[QJL ? QW : 1];
 #pragma unroll
@@ -271,7 +311,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         }
         if (mine && t < t1) {
             // NSN: the code weight factor ||x|| ||w|| / sqrt(d) and the block-mean factor ||x|| / sqrt(d)
-            const float2 nv = __half22float2(vn[t]);
+            const float2 nv = norms_at(false, t);
             svn[tid] = NSN ? nv.x * nv.y * inv_sqrt_d : nv.x;
             svg[tid] = NSN ? nv.x * inv_sqrt_d : nv.y;
         }
@@ -364,7 +404,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
                         float o = 0.f;
                         for (int bq = 0; bq < NBT; ++bq) {
                             const int64_t blk = tb / 128 + bq;
-                            if (blk * 128 < t1) o = fmaf(sbeta[g][bq], __half2float(vmean[blk * D + j]), o);
+                            if (blk * 128 < t1) o = fmaf(sbeta[g][bq], vmean_at(blk, j), o);
                         }
                         if (second) accB2[g] += o;
                         else accB[g] += o;
@@ -604,12 +644,17 @@ cudaError_t launch_d(const DecodeArgs& a, cudaStream_t s) {
     if constexpr (!QJL) nsn = a.nsn != 0;
     if (nsn) {
         if constexpr (!QJL) {
-            switch (a.G) {
-                case 1: decode_split_kernel<D, B, false, 1, true><<<grid, block, 0, s>>>(a); break;
-                case 2: decode_split_kernel<D, B, false, 2, true><<<grid, block, 0, s>>>(a); break;
-                case 4: decode_split_kernel<D, B, false, 4, true><<<grid, block, 0, s>>>(a); break;
-                default: decode_split_kernel<D, B, false, 8, true><<<grid, block, 0, s>>>(a); break;
-            }
+            auto run = [&](auto dq) {
+                constexpr bool DQ = decltype(dq)::value;
+                switch (a.G) {
+                    case 1: decode_split_kernel<D, B, false, 1, true, DQ><<<grid, block, 0, s>>>(a); break;
+                    case 2: decode_split_kernel<D, B, false, 2, true, DQ><<<grid, block, 0, s>>>(a); break;
+                    case 4: decode_split_kernel<D, B, false, 4, true, DQ><<<grid, block, 0, s>>>(a); break;
+                    default: decode_split_kernel<D, B, false, 8, true, DQ><<<grid, block, 0, s>>>(a); break;
+                }
+            };
+            if (a.nsn_dq) run(std::true_type());
+            else run(std::false_type());
         }
     } else {
         switch (a.G) {

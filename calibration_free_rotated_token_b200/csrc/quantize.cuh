@@ -639,9 +639,39 @@ __global__ void __launch_bounds__(256, 1)
                 float* ssc = reinterpret_cast<float*>(aux + 2048);  // [128] sc per row
                 float* sbo = reinterpret_cast<float*>(aux + 2560);  // [2][128] butterflies of delta .* o
                 float* swx = reinterpret_cast<float*>(aux + 3584);  // [2][128] half sums of squares
+                float* sof = reinterpret_cast<float*>(aux + 4608);  // [256] the subtracted means o (fp32)
+                float* sred = reinterpret_cast<float*>(aux + 5632); // [2][8] block reductions
+                // With double quantization (side records, NSNQuant section 3) the transform uses the
+                // stored values: n1 = q nstep for ||x|| and o_hat = lo + step q for the mean.
+                const bool dq = a.side != nullptr;
+                constexpr int RB = (8 + D / 2 + 64 + 15) / 16 * 16;
+                uint8_t* rec = dq ? a.side + tile * RB : nullptr;
                 nx = sqrtf(ss);
                 if (h == 0) flag_norm(ss, nx, a.status);
-                const float sc = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
+                float sc = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
+                if (dq) {
+                    // 4-bit norm codes on nstep = fp16(max ||x|| / 15) of the block
+                    float m = nx;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+                    if (lane == 0) sred[warp] = m;
+                    named_bar_sync(3, 256);
+                    float mx = sred[0];
+#pragma unroll
+                    for (int k = 1; k < 8; ++k) mx = fmaxf(mx, sred[k]);
+                    const __half ns16 = __float2half_rn(mx / 15.0f);
+                    const float nsf = __half2float(ns16);
+                    int qn = 0;
+                    if (nx > 0.f && nsf > 0.f) qn = min(max(__float2int_rn(nx / nsf), 1), 15);
+                    sc = qn > 0 ? sqrtf(static_cast<float>(D)) / (static_cast<float>(qn) * nsf) : 0.f;
+                    const int qp = __shfl_down_sync(0xFFFFFFFFu, qn, 1);
+                    if (h == 0) {
+                        if ((r & 1) == 0) rec[8 + D / 2 + r / 2] = static_cast<uint8_t>(qn | (qp << 4));
+                        if (r == 0) *reinterpret_cast<__half*>(rec + 4) = ns16;
+                        if (r < 2) rec[6 + r] = 0;
+                        if (r >= 2 && r < 2 + (RB - 8 - D / 2 - 64)) rec[8 + D / 2 + 64 + (r - 2)] = 0;
+                    }
+                }
                 if (h == 0) ssc[r] = sc;
                 named_bar_sync(3, 256);
                 {
@@ -655,9 +685,42 @@ __global__ void __launch_bounds__(256, 1)
                                                          : __half2float(*reinterpret_cast<const __half*>(&hv));
                         acc = fmaf(xt, ssc[t], acc);
                     }
-                    const __half o16 = __float2half_rn(acc * (1.0f / kTileRows));
-                    so16[j] = o16;
-                    a.block_mean[tile * D + j] = o16;
+                    const float om = acc * (1.0f / kTileRows);
+                    if (!dq) {
+                        const __half o16 = __float2half_rn(om);
+                        sof[j] = __half2float(o16);
+                        a.block_mean[tile * D + j] = o16;
+                    } else {
+                        // 4-bit mean codes on [lo, lo + 15 step], lo = fp16(min o), step = fp16((max - min) / 15)
+                        float mn = om, mo = om;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) {
+                            mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+                            mo = fmaxf(mo, __shfl_xor_sync(0xFFFFFFFFu, mo, o));
+                        }
+                        if (lane == 0) {
+                            sred[warp] = mn;
+                            sred[8 + warp] = mo;
+                        }
+                        named_bar_sync(3, 256);
+                        float lo = sred[0], hi = sred[8];
+#pragma unroll
+                        for (int k = 1; k < 8; ++k) {
+                            lo = fminf(lo, sred[k]);
+                            hi = fmaxf(hi, sred[8 + k]);
+                        }
+                        const __half lo16 = __float2half_rn(lo), st16 = __float2half_rn((hi - lo) / 15.0f);
+                        const float lof = __half2float(lo16), stf = __half2float(st16);
+                        int qo = 0;
+                        if (stf > 0.f) qo = min(max(__float2int_rn((om - lof) / stf), 0), 15);
+                        sof[j] = fmaf(stf, static_cast<float>(qo), lof);
+                        const int qp = __shfl_down_sync(0xFFFFFFFFu, qo, 1);
+                        if ((j & 1) == 0) rec[8 + j / 2] = static_cast<uint8_t>(qo | (qp << 4));
+                        if (j == 0) {
+                            *reinterpret_cast<__half*>(rec) = lo16;
+                            *reinterpret_cast<__half*>(rec + 2) = st16;
+                        }
+                    }
                 }
                 named_bar_sync(3, 256);
                 if (tid == 0) issue_tile(i + kStages);  // the stage is read
@@ -667,8 +730,8 @@ __global__ void __launch_bounds__(256, 1)
                     auto sgn = [&](int c) {
                         return ((a.pair_sign[c >> 1] >> ((c & 1) ? 31 : 15)) & 1u) ? -1.f : 1.f;
                     };
-                    const float lo = sgn(j) * __half2float(so16[j]);
-                    const float hi = sgn(j + 128) * __half2float(so16[j + 128]);
+                    const float lo = sgn(j) * sof[j];
+                    const float hi = sgn(j + 128) * sof[j + 128];
                     sbo[hh * 128 + j] = hh ? lo - hi : lo + hi;
                 }
                 named_bar_sync(3, 256);
@@ -722,8 +785,11 @@ __global__ void __launch_bounds__(256, 1)
             if (valid) {
                 if (h == 0) {
                     const float g = nrm > 0.f ? sqrtf(xch[r] + xch[128 + r]) : 0.f;
-                    a.norms[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
-                                        : __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
+                    if (NSN && a.side != nullptr)
+                        reinterpret_cast<__half*>(a.norms)[vidx] = __float2half_rn(nrm);  // ||w|| only
+                    else
+                        a.norms[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
+                                            : __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
                 }
             }
             if (QJL) {

@@ -27,8 +27,7 @@ cudaError_t by_dtype(const CUtensorMap& map, const CUtensorMap& map1, int dtype,
     if constexpr (NSN && QJL) {
         return cudaErrorNotSupported;
     } else if constexpr (NSN && D > 128) {
-        // d = 256: the in-register transform kernel, 16-bit input, fp16 side data
-        if (a.side != nullptr) return cudaErrorNotSupported;
+        // d = 256: the in-register transform kernel, 16-bit input (side records when a.side is given)
         switch (dtype) {
             case DT_F16: return launch_quantize_t<D, B, false, DT_F16, true>(map, a, sms, s);
             case DT_BF16: return launch_quantize_t<D, B, false, DT_BF16, true>(map, a, sms, s);

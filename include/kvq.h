@@ -299,7 +299,8 @@ int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int
  *                       2i in the low nibble, 2i+1 in the high one);
  *   [8 + d/2, + 64)     4-bit codes q_t of the 128 token norms (byte i: token
  *                       2i low nibble, 2i+1 high);
- *   zero padding to a multiple of 16 bytes (144 bytes at d = 128, 112 at 64).
+ *   zero padding to a multiple of 16 bytes (144 bytes at d = 128, 112 at 64,
+ *   208 at 256).
  * The stored values are   n1_t = q_t nstep   (q_t = 0 only for a zero token)
  *                         o_hat_j = fp32(lo + step q_j)   (one rounding),
  * and the transform uses them: u_t = sqrt(d) x_t / n1_t, w_t = u_t - o_hat,
@@ -312,7 +313,7 @@ int kvq_nsn_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int
  * against 0.375 with fp16 ||x||, ||w|| and fp16 means.
  */
 
-/* Bytes of one side record for head dimension d (64 or 128; else 0). */
+/* Bytes of one side record for head dimension d (64, 128 or 256; else 0). */
 size_t kvq_nsn_dq_side_bytes(int d);
 
 /*
@@ -322,8 +323,8 @@ size_t kvq_nsn_dq_side_bytes(int d);
  *   wnorms   device, n_heads * n_tok fp16 (||w_t||), 4-byte aligned.
  *   side     device, n_heads * (n_tok/128) records of kvq_nsn_dq_side_bytes(d)
  *            bytes, 16-byte aligned.
- * Requires a handle without KVQ_QJL (KVQ_EINVAL) and d <= 128; fp32 input
- * returns KVQ_EUNSUPPORTED.
+ * Requires a handle without KVQ_QJL (KVQ_EINVAL); fp32 input returns
+ * KVQ_EUNSUPPORTED.
  */
 int kvq_nsn_dq_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads, int64_t n_tok, int layout,
                         uint32_t* codes, uint16_t* wnorms, uint8_t* side, void* stream);
@@ -337,8 +338,8 @@ int kvq_nsn_dq_quantize(kvq_handle h, const void* x, int dtype, int64_t n_heads,
  *             codes as usual; capacities multiples of 128.
  *   k_side, v_side  device, per stream capacity/128 side records, stream
  *             (bi, hi) at record (bi * hkv + hi) * capacity/128, 16-byte aligned.
- * Other arguments, workspace and errors as kvq_nsn_decode_attend; built for
- * d <= 128.
+ * Other arguments, workspace and errors as kvq_nsn_decode_attend; every
+ * (d, b) is built.
  */
 int kvq_nsn_dq_decode_attend(kvq_handle h, const void* q, int dtype, int batch, int hq, int hkv, const kvq_cache* k,
                              const kvq_cache* v, const uint8_t* k_side, const uint8_t* v_side, const int32_t* seq_len,

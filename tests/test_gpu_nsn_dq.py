@@ -115,7 +115,9 @@ def run_dq(h, x, layout=0):
 
 
 @pytest.mark.parametrize("d,b,dtype", [(128, 2, torch.bfloat16), (128, 1, torch.float16), (64, 3, torch.bfloat16),
-                                       (64, 2, torch.float16), (128, 4, torch.bfloat16)])
+                                       (64, 2, torch.float16), (128, 4, torch.bfloat16),
+                                       # d = 256: the in-register transform kernel, two threads per vector
+                                       (256, 2, torch.bfloat16), (256, 4, torch.float16)])
 def test_nsn_dq_matches_oracle(d, b, dtype):
     x = wl.nsn_tokens(2, 512, d, seed=30 + d + b, dtype=dtype)
     x[1, 130] = 0  # a zero token inside a block
@@ -154,7 +156,7 @@ def test_nsn_dq_rejects_unbuilt_and_invalid_calls():
             kvq.kvq_nsn_dq_quantize(h, torch.randn(1, 100, 128, device="cuda", dtype=torch.bfloat16), codes, wn,
                                     side)
     assert kvq.kvq_nsn_dq_side_bytes(128) == 144 and kvq.kvq_nsn_dq_side_bytes(64) == 112
-    assert kvq.kvq_nsn_dq_side_bytes(256) == 0
+    assert kvq.kvq_nsn_dq_side_bytes(256) == 208 and kvq.kvq_nsn_dq_side_bytes(96) == 0
 
 
 def _dq_oracle_stream(k, X):
@@ -221,6 +223,11 @@ def check_dq_decode(d, b, batch, hq, hkv, seq_len, cap, qdtype=torch.bfloat16, s
     (128, 2, 1, 16, 2, [2000], 2048),        # GQA 8:1
     (128, 1, 2, 4, 1, [0, 129], 256),        # an empty context
     (128, 3, 1, 8, 2, [700], 768),           # 3 bits (parity plane)
+    (256, 2, 1, 4, 2, [513], 640),           # d = 256 on the tensor cores (128-token sub-chunks)
+    # CUDA-core path: 4-bit codebooks, 3 bits at d = 256
+    (128, 4, 2, 8, 2, [1000, 300], 1024),
+    (64, 4, 1, 4, 4, [640], 640),
+    (256, 3, 2, 4, 1, [0, 700], 768),        # an empty context
 ])
 def test_nsn_dq_decode_matches_oracle(d, b, batch, hq, hkv, seq_len, cap):
     check_dq_decode(d, b, batch, hq, hkv, seq_len, cap)
