@@ -688,7 +688,7 @@ def bench_sweep(args, dist):
                              "quantize_us_per_2e20": round(ms_q / (2 * steps) * 1e3, 2),
                              "quantize_gbs": round(q_gbs, 1),
                              "quantize_frac": round(q_gbs / hbm, 4),
-                             "quantize_kernel": "quantize_tc_kernel" if d <= 128 else "quantize_kernel",
+                             "quantize_kernel": "quantize_tc_kernel" if d <= 128 or not qjl else "quantize_kernel",
                              "decode_us": round(ms_d / steps * 1e3, 2), "decode_gbs": round(d_gbs, 1),
                              "decode_frac": round(d_gbs / hbm, 4),
                              "decode_kernel": ("decode_mma_kernel" if b <= 2 or (b == 3 and d <= 128)

@@ -449,7 +449,8 @@ int kvq_quantize_batch(kvq_handle h, int count, const kvq_quant_job* jobs, void*
     }
     for (size_t i = 0; i < js.size();) {
         const bool pair = i + 1 < js.size() && js[i].dtype == js[i + 1].dtype &&
-                          kvq::quantize_pairs(h->d, js[i].dtype, false) && !(h->flags & KVQ_CUDA_CORE_ROTATION);
+                          kvq::quantize_pairs(h->d, js[i].dtype, false, (h->flags & KVQ_QJL) != 0) &&
+                          !(h->flags & KVQ_CUDA_CORE_ROTATION);
         if (int e = launch_jobs(h, js[i], maps[i], pair ? &js[i + 1] : nullptr, pair ? &maps[i + 1] : nullptr,
                                 nullptr, false, stream))
             return e;

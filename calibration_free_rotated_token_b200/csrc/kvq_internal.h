@@ -70,8 +70,8 @@ struct QuantArgs {
 cudaError_t launch_quantize(const kvq_ctx* h, const CUtensorMap& map, int dtype, bool nsn, const QuantArgs& a,
                             cudaStream_t s, std::string* why);
 // True when two streams of vectors can share one launch (the tensor-core
-// kernel: 16-bit input, d <= 128, no NSN front end).
-inline bool quantize_pairs(int d, int dtype, bool nsn) { return d <= 128 && dtype != 0 && !nsn; }
+// kernel: 16-bit input, no NSN front end, d <= 128 or d = 256 without QJL).
+inline bool quantize_pairs(int d, int dtype, bool nsn, bool qjl) { return dtype != 0 && !nsn && (d <= 128 || !qjl); }
 
 struct DecodeArgs {
     int batch, hq, hkv, G;            // G = hq / hkv

@@ -58,7 +58,7 @@ struct QCfg {
     static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kSBytes + kAuxBytes;
     static_assert(kStages >= 1, "input tile does not fit in shared memory");
     static_assert(!(NSN && QJL), "NSN front end: no QJL");
-    static_assert(!(NSN && kCoop && DT == DT_F32), "NSN front end at D = 256: 16-bit input");
+    static_assert(!(NSN && kCoop), "NSN front end at D = 256: the tensor-core kernel");
 };
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
@@ -630,127 +630,10 @@ __global__ void __launch_bounds__(256, 1)
 
             float2 v[64];
             const float ss = load_row_coop<DT>(sp, r, h, v, a.pair_sign);
-            float nrm, nx = 0.f;
-            if constexpr (NSN) {
-                // NSN front end (NSNQuant sections 1-2) on a 128-token block: u = sqrt(D) x / ||x||,
-                // o = the fp16 channel means of u, w = u - o.  The loaded v is this half of the top
-                // butterfly of delta .* x, which is linear: the half of delta .* w is sc v - bo with
-                // bo the same butterfly of delta .* o; ||w||^2 is half the sum of both halves' squares.
-                float* ssc = reinterpret_cast<float*>(aux + 2048);  // [128] sc per row
-                float* sbo = reinterpret_cast<float*>(aux + 2560);  // [2][128] butterflies of delta .* o
-                float* swx = reinterpret_cast<float*>(aux + 3584);  // [2][128] half sums of squares
-                float* sof = reinterpret_cast<float*>(aux + 4608);  // [256] the subtracted means o (fp32)
-                float* sred = reinterpret_cast<float*>(aux + 5632); // [2][8] block reductions
-                // With double quantization (side records, NSNQuant section 3) the transform uses the
-                // stored values: n1 = q nstep for ||x|| and o_hat = lo + step q for the mean.
-                const bool dq = a.side != nullptr;
-                constexpr int RB = (8 + D / 2 + 64 + 15) / 16 * 16;
-                uint8_t* rec = dq ? a.side + tile * RB : nullptr;
-                nx = sqrtf(ss);
-                if (h == 0) flag_norm(ss, nx, a.status);
-                float sc = nx > 0.f ? sqrtf(static_cast<float>(D)) / nx : 0.f;
-                if (dq) {
-                    // 4-bit norm codes on nstep = fp16(max ||x|| / 15) of the block
-                    float m = nx;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-                    if (lane == 0) sred[warp] = m;
-                    named_bar_sync(3, 256);
-                    float mx = sred[0];
-#pragma unroll
-                    for (int k = 1; k < 8; ++k) mx = fmaxf(mx, sred[k]);
-                    const __half ns16 = __float2half_rn(mx / 15.0f);
-                    const float nsf = __half2float(ns16);
-                    int qn = 0;
-                    if (nx > 0.f && nsf > 0.f) qn = min(max(__float2int_rn(nx / nsf), 1), 15);
-                    sc = qn > 0 ? sqrtf(static_cast<float>(D)) / (static_cast<float>(qn) * nsf) : 0.f;
-                    const int qp = __shfl_down_sync(0xFFFFFFFFu, qn, 1);
-                    if (h == 0) {
-                        if ((r & 1) == 0) rec[8 + D / 2 + r / 2] = static_cast<uint8_t>(qn | (qp << 4));
-                        if (r == 0) *reinterpret_cast<__half*>(rec + 4) = ns16;
-                        if (r < 2) rec[6 + r] = 0;
-                        if (r >= 2 && r < 2 + (RB - 8 - D / 2 - 64)) rec[8 + D / 2 + 64 + (r - 2)] = 0;
-                    }
-                }
-                if (h == 0) ssc[r] = sc;
-                named_bar_sync(3, 256);
-                {
-                    // block mean of channel j = tid over the tile's rows
-                    const int j = tid;
-                    float acc = 0.f;
-                    for (int t = 0; t < kTileRows; ++t) {
-                        const uint8_t* p = sp + (j / 64) * 16384 + t * 128 + ((((j % 64) / 8) ^ (t & 7)) << 4) + (j % 8) * 2;
-                        const uint16_t hv = *reinterpret_cast<const uint16_t*>(p);
-                        const float xt = (DT == DT_BF16) ? u2f(static_cast<uint32_t>(hv) << 16)
-                                                         : __half2float(*reinterpret_cast<const __half*>(&hv));
-                        acc = fmaf(xt, ssc[t], acc);
-                    }
-                    const float om = acc * (1.0f / kTileRows);
-                    if (!dq) {
-                        const __half o16 = __float2half_rn(om);
-                        sof[j] = __half2float(o16);
-                        a.block_mean[tile * D + j] = o16;
-                    } else {
-                        // 4-bit mean codes on [lo, lo + 15 step], lo = fp16(min o), step = fp16((max - min) / 15)
-                        float mn = om, mo = om;
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) {
-                            mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-                            mo = fmaxf(mo, __shfl_xor_sync(0xFFFFFFFFu, mo, o));
-                        }
-                        if (lane == 0) {
-                            sred[warp] = mn;
-                            sred[8 + warp] = mo;
-                        }
-                        named_bar_sync(3, 256);
-                        float lo = sred[0], hi = sred[8];
-#pragma unroll
-                        for (int k = 1; k < 8; ++k) {
-                            lo = fminf(lo, sred[k]);
-                            hi = fmaxf(hi, sred[8 + k]);
-                        }
-                        const __half lo16 = __float2half_rn(lo), st16 = __float2half_rn((hi - lo) / 15.0f);
-                        const float lof = __half2float(lo16), stf = __half2float(st16);
-                        int qo = 0;
-                        if (stf > 0.f) qo = min(max(__float2int_rn((om - lof) / stf), 0), 15);
-                        sof[j] = fmaf(stf, static_cast<float>(qo), lof);
-                        const int qp = __shfl_down_sync(0xFFFFFFFFu, qo, 1);
-                        if ((j & 1) == 0) rec[8 + j / 2] = static_cast<uint8_t>(qo | (qp << 4));
-                        if (j == 0) {
-                            *reinterpret_cast<__half*>(rec) = lo16;
-                            *reinterpret_cast<__half*>(rec + 2) = st16;
-                        }
-                    }
-                }
-                named_bar_sync(3, 256);
-                if (tid == 0) issue_tile(i + kStages);  // the stage is read
-                {
-                    // sbo[hh][j] = delta_j o_j + (-1)^hh delta_{j+128} o_{j+128}
-                    const int hh = tid >> 7, j = tid & 127;
-                    auto sgn = [&](int c) {
-                        return ((a.pair_sign[c >> 1] >> ((c & 1) ? 31 : 15)) & 1u) ? -1.f : 1.f;
-                    };
-                    const float lo = sgn(j) * sof[j];
-                    const float hi = sgn(j + 128) * sof[j + 128];
-                    sbo[hh * 128 + j] = hh ? lo - hi : lo + hi;
-                }
-                named_bar_sync(3, 256);
-                const float2 sc2 = make_float2(sc, sc);
-                const float2* bo2 = reinterpret_cast<const float2*>(sbo + h * 128);
-#pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    const float2 b = bo2[k];
-                    v[k] = __ffma2_rn(v[k], sc2, make_float2(-b.x, -b.y));
-                }
-                swx[h * 128 + r] = sumsq(v);
-                named_bar_sync(3, 256);
-                nrm = sqrtf(0.5f * (swx[r] + swx[128 + r]));
-            } else {
-                named_bar_sync(3, 256);
-                if (tid == 0) issue_tile(i + kStages);
-                nrm = sqrtf(ss);
-                if (h == 0) flag_norm(ss, nrm, a.status);
-            }
+            named_bar_sync(3, 256);
+            if (tid == 0) issue_tile(i + kStages);
+            const float nrm = sqrtf(ss);
+            if (h == 0) flag_norm(ss, nrm, a.status);
             fwht<64>(v);
             const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
             uint32_t planes[B][4];
@@ -782,15 +665,9 @@ __global__ void __launch_bounds__(256, 1)
                     store_block32<4>(a.codes + (blk * B + p) * 256 + h * 128, planes[p], valid ? zmask : 0u, lane,
                                      blk * 32 < a.n);
             }
-            if (valid) {
-                if (h == 0) {
-                    const float g = nrm > 0.f ? sqrtf(xch[r] + xch[128 + r]) : 0.f;
-                    if (NSN && a.side != nullptr)
-                        reinterpret_cast<__half*>(a.norms)[vidx] = __float2half_rn(nrm);  // ||w|| only
-                    else
-                        a.norms[vidx] = NSN ? __halves2half2(__float2half_rn(nx), __float2half_rn(nrm))
-                                            : __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
-                }
+            if (valid && h == 0) {
+                const float g = nrm > 0.f ? sqrtf(xch[r] + xch[128 + r]) : 0.f;
+                a.norms[vidx] = __halves2half2(__float2half_rn(nrm), __float2half_rn(g));
             }
             if (QJL) {
                 const bool okm = mbar_wait(&mmadone[0], static_cast<uint32_t>(jlocal & 1), a.status);

@@ -1,5 +1,6 @@
 // quantize_tc.cuh -- the quantize kernel (and its NSN front end) with the
-// rotation on the tensor cores, for 16-bit input and d <= 128.
+// rotation on the tensor cores, for 16-bit input: d <= 128, and d = 256
+// without QJL.
 //
 // Method (TurboQuant blog, "Estagio 1" and "Estagio 2"; PolarQuant section 2),
 // per vector x: y = H (delta .* x) (unnormalised Sylvester Hadamard, so
@@ -17,6 +18,12 @@
 //   and whole tiles; a thread owns one vector (its TMEM lane).  Each stage of
 //   the x ring belongs to one warpgroup; it is free as soon as the rotation
 //   MMA has read it, and the warpgroup refills it then.
+// * d = 256 (no QJL: S would not fit beside the stages): H of order 256 is
+//   [[H', H'], [H', -H']] with H' of order 128, so the rotation is two
+//   products P = X1 (H' D1)^T and Q = X2 (H' D2)^T over the two halves of x
+//   (64 KB of B operands instead of 128 KB), and the passes read
+//   y = (P + Q, P - Q) group by group.  Two warpgroups of 256 columns each,
+//   two 64 KB stages.
 // * Pass 1 reads y back (32 columns at a time) for ||y||^2; pass 2 reads it
 //   again, forms codes and the residual chunk by chunk and writes the fp16
 //   residual into the already consumed columns [0, d/2).
@@ -44,20 +51,32 @@ struct TcCfg {
     static constexpr int kTileBytes = kTileRows * D * 2;   // 16-bit input
     static constexpr int kBoxBytes = 128 * kTileRows;      // 64 elements x 128 rows
     static constexpr int kBoxes = D * 2 / 128;
-    static constexpr int kMatBytes = D * D * 2;            // H D or S, 16-bit, K-major, swizzled
-    static constexpr int kWG = 4;
+    // The rotation is kNMat products of N = K = kNB: at d = 256 the two
+    // 128-coordinate halves x1, x2 of x give P = (H D1) x1 and Q = (H D2) x2
+    // (H of order 128, D1, D2 the two halves of the sign diagonal), and the
+    // Sylvester recursion puts the rotated vector together as (P + Q, P - Q).
+    static constexpr int kNB = D > 128 ? 128 : D;
+    static constexpr int kNMat = D / kNB;
+    static constexpr int kMatBytes = kNMat * kNB * kNB * 2;  // H D blocks, 16-bit, K-major, swizzled
+    static constexpr int kSBytes = QJL ? D * D * 2 : 0;      // S, same layout
+    static constexpr int kCols = D > 128 ? 256 : 128;        // tensor-memory columns per warpgroup
+    static constexpr int kWG = 512 / kCols;
     static constexpr int kThreads = 128 * kWG;
-    static constexpr int kAuxBytes = NSN ? 12288 : 1024;  // NSN: per-warpgroup scale, partial means, mean, rotated mean
+    // NSN scratch floats per warpgroup: scale [128], mean [D], rotated mean [D],
+    // partial channel sums [1024], reductions [8]
+    static constexpr int kNsnF = 1160 + 2 * D;
+    static constexpr int kAuxBytes = NSN ? 24576 : 1024;
     static constexpr int kBudget = 225 * 1024;
-    static constexpr int kStagesRaw = (kBudget - kMatBytes - (QJL ? kMatBytes : 0) - kAuxBytes) / kTileBytes;
-    // Tile i goes to warpgroup i % 4 and stage i % kStages; with kStages a
-    // multiple of 4 every stage belongs to one warpgroup, which consumes its
+    static constexpr int kStagesRaw = (kBudget - kMatBytes - kSBytes - kAuxBytes) / kTileBytes;
+    // Tile i goes to warpgroup i % kWG and stage i % kStages; with kStages a
+    // multiple of kWG every stage belongs to one warpgroup, which consumes its
     // phases strictly in order (a parity wait can never see a stale phase).
     static constexpr int kStages = (kStagesRaw > 8 ? 8 : kStagesRaw) / kWG * kWG;
-    static constexpr int kSmemBytes = 1024 + kStages * kTileBytes + kMatBytes + (QJL ? kMatBytes : 0) + kAuxBytes;
+    static constexpr int kSmemBytes = 1024 + kStages * kTileBytes + kMatBytes + kSBytes + kAuxBytes;
     static constexpr int kQN = 64;                          // rows of S per QJL MMA
-    static_assert(D == 64 || D == 128, "tensor-core rotation: d in {64, 128}");
+    static_assert(D == 64 || D == 128 || (D == 256 && !QJL), "tensor-core rotation: d in {64, 128}, or 256 without QJL");
     static_assert(kStages >= kWG, "one stage per warpgroup at least");
+    static_assert(1024 + kWG * kNsnF * 4 <= kAuxBytes || !NSN, "NSN scratch");
 };
 
 // Column order of the rotated vector and of the residual in tensor memory.
@@ -324,7 +343,7 @@ __device__ __forceinline__ float stage_elem(const uint8_t* sp, int t, int j) {
 }
 
 template <int D, int B, bool QJL, int DT, bool NSN = false, bool DQ = false>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(TcCfg<D, QJL, NSN>::kThreads, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap map, const __grid_constant__ CUtensorMap map1,
                        const __grid_constant__ QuantArgs a) {
     static_assert(!(NSN && QJL), "NSN front end: no QJL");
@@ -333,7 +352,8 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int RB = (8 + D / 2 + 64 + 15) / 16 * 16;  // DQ: side record bytes per block
     constexpr int NS = C::kStages;
     constexpr int kWpp = D / 32;
-    constexpr uint32_t kIdescH = idesc_16bit_f32(kTileRows, D, DT == DT_BF16);
+    constexpr int NB = C::kNB;
+    constexpr uint32_t kIdescH = idesc_16bit_f32(kTileRows, NB, DT == DT_BF16);
     constexpr uint32_t kIdescQ = idesc_16bit_f32(kTileRows, C::kQN, false);
 
     extern __shared__ uint8_t smem_raw[];
@@ -341,14 +361,14 @@ __global__ void __launch_bounds__(512, 1)
     uint8_t* stage0 = smem;
     uint8_t* sHD = smem + NS * C::kTileBytes;
     uint8_t* sS = sHD + C::kMatBytes;
-    uint8_t* aux = sS + (QJL ? C::kMatBytes : 0);
+    uint8_t* aux = sS + C::kSBytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(aux);    // [8]
     uint64_t* hbar = full + 8;                              // [4] rotation MMA done
     uint64_t* qbar = hbar + 4;                              // [4] QJL MMA done
     uint32_t* iss = reinterpret_cast<uint32_t*>(qbar + 4);  // [8] loads issued per stage
     uint32_t* con = iss + 8;                                // [8] loads consumed per stage
     uint32_t* tmem_slot = con + 8;
-    float* nsn_aux = reinterpret_cast<float*>(aux + 1024);  // NSN: [4 warpgroups][648]
+    float* nsn_aux = reinterpret_cast<float*>(aux + 1024);  // NSN: [warpgroups][kNsnF]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -369,26 +389,28 @@ __global__ void __launch_bounds__(512, 1)
         }
         fence_mbar_init();
     }
-    // H D as the B operand (row n = output column n, which holds coordinate
-    // col_coord(n); K = input coordinate): entry (n, k) =
-    // (-1)^popcount(col_coord(n) & k) delta_k.  K-chunk kc (64 entries) of row
-    // n at sHD + kc*D*128 + n*128, 16-byte chunk c at c ^ (n & 7).
+    // Block m of H D as the B operand (row n = output column n, which holds
+    // coordinate col_coord(n); K = input coordinate k of the block's half):
+    // entry (n, k) = (-1)^popcount(col_coord(n) & k) delta_{m NB + k}.  K-chunk
+    // kc (64 entries) of row n at sHD + m*NB*NB*2 + kc*NB*128 + n*128, 16-byte
+    // chunk c at c ^ (n & 7).
     {
         const uint32_t one = (DT == DT_BF16) ? 0x3F80u : 0x3C00u;
-        for (int e = tid; e < D * D / 8; e += C::kThreads) {
-            const int n = e / (D / 8), cc = e % (D / 8);
+        for (int e = tid; e < C::kNMat * NB * NB / 8; e += C::kThreads) {
+            const int m = e / (NB * NB / 8), em = e % (NB * NB / 8);
+            const int n = em / (NB / 8), cc = em % (NB / 8);
             const int kc = cc / 8, c16 = cc % 8;
             const int jn = col_coord(n);
             uint32_t w4[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int k = 8 * cc + 2 * q;
-                const uint32_t ps = a.pair_sign[k >> 1];
+                const uint32_t ps = a.pair_sign[(m * NB + k) >> 1];
                 const uint32_t s0 = ((__popc(jn & k) & 1u) << 15) ^ (ps & 0x8000u);
                 const uint32_t s1 = ((__popc(jn & (k + 1)) & 1u) << 15) ^ ((ps >> 16) & 0x8000u);
                 w4[q] = (one | s0) | ((one | s1) << 16);
             }
-            *reinterpret_cast<uint4*>(sHD + kc * (D * 128) + n * 128 + ((c16 ^ (n & 7)) << 4)) =
+            *reinterpret_cast<uint4*>(sHD + m * (NB * NB * 2) + kc * (NB * 128) + n * 128 + ((c16 ^ (n & 7)) << 4)) =
                 make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
     }
@@ -453,7 +475,7 @@ __global__ void __launch_bounds__(512, 1)
 
     const uint32_t bar_id = 1 + wg;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tcol = tmem + static_cast<uint32_t>(wg * 128);  // this warpgroup's 128 columns
+    const uint32_t tcol = tmem + static_cast<uint32_t>(wg * C::kCols);  // this warpgroup's columns
     const uint32_t tl = tcol + lane_base;                            // ... at this thread's lane
     uint32_t hpar = 0, qpar = 0;
     const CodeTab<B> ctab(a);
@@ -474,15 +496,22 @@ __global__ void __launch_bounds__(512, 1)
         if (named_bar_or(bar_id, 128, !ok)) break;
         if (r == 0) {
             con[st] += 1;
-            // ---- rotation: Y = X (H D)^T into columns [0, D) ----
+            // ---- rotation: Y = X (H D)^T into columns [0, D) (d = 256: P, Q) ----
             tc_fence_after();
             const uint32_t xs = smem_u32(stage0 + st * C::kTileBytes);
-            const uint32_t hs = smem_u32(sHD);
+            // (read through an opaque move so that the B descriptors are formed
+            // here, not hoisted out of the tile loop into registers held throughout)
+            uint32_t hs;
+            asm volatile("mov.b32 %0, %1;" : "=r"(hs) : "r"(smem_u32(sHD)));
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t aoff = (ks / 4) * C::kBoxBytes + (ks % 4) * 32;
-                const uint32_t boff = (ks / 4) * (D * 128) + (ks % 4) * 32;
-                mma_f16_ss(tcol, smem_desc_sw128(xs + aoff), smem_desc_sw128(hs + boff), kIdescH, ks > 0 ? 1u : 0u);
+            for (int m = 0; m < C::kNMat; ++m) {
+#pragma unroll
+                for (int ks = 0; ks < NB / 16; ++ks) {
+                    const uint32_t aoff = (m * (NB / 64) + ks / 4) * C::kBoxBytes + (ks % 4) * 32;
+                    const uint32_t boff = m * (NB * NB * 2) + (ks / 4) * (NB * 128) + (ks % 4) * 32;
+                    mma_f16_ss(tcol + m * NB, smem_desc_sw128(xs + aoff), smem_desc_sw128(hs + boff), kIdescH,
+                               ks > 0 ? 1u : 0u);
+                }
             }
             mma_commit(&hbar[wg]);
         }
@@ -490,11 +519,11 @@ __global__ void __launch_bounds__(512, 1)
         // sc = sqrt(D)/||x||, block mean o of u = sc x per channel, fp16(o),
         // and ho = H (delta .* fp16(o)), so that H D w = sc y - ho.
         float nx = 0.f, sc = 0.f;
-        float* xch = nsn_aux + wg * 648;  // [128] sc per token
-        float* so = xch + 128;            // [D] delta .* fp16(o)
-        float* ho = xch + 256;            // [D] H (delta .* fp16(o)), in tensor-memory column order
-        float2* opart = reinterpret_cast<float2*>(xch + 384);  // [128 / (D/2)][D/2] partial channel sums
-        float* red = xch + 640;           // DQ: [4] block max of ||x|| / [2][4] channel min, max
+        float* xch = nsn_aux + wg * C::kNsnF;  // [128] sc per token
+        float* so = xch + 128;                  // [D] delta .* fp16(o)
+        float* ho = xch + 128 + D;              // [D] H (delta .* fp16(o)), in tensor-memory column order
+        float* opart = xch + 128 + 2 * D;       // [1024 / D][D] partial channel sums
+        float* red = xch + 1152 + 2 * D;        // DQ: [4] block max of ||x|| / [2][4] channel min, max
         if constexpr (NSN) {
             const uint8_t* sp = stage0 + st * C::kTileBytes;
             const float ssx0 = stage_row_sumsq<D, DT>(sp, r);
@@ -529,41 +558,58 @@ __global__ void __launch_bounds__(512, 1)
             xch[r] = sc;
             named_bar_sync(bar_id, 128);
             {
-                // thread r: channel pair p, tokens of group q (fp32x2 sums)
-                constexpr int P = D / 2, Q = kTileRows / P, TPQ = kTileRows / Q;
-                const int p = r % P, q = r / P;
-                const int j0 = 2 * p;
-                float2 acc = make_float2(0.f, 0.f);
+                // thread r: channels 8o .. 8o + 7 (one 16-byte chunk of a row) over
+                // the tokens of group q; four independent fp32x2 sums
+                constexpr int NO = D / 8, QG = kTileRows / NO, TPG = kTileRows / QG;
+                const int o = r % NO, q = r / NO;
+                const uint8_t* cb = sp + (o / 8) * 16384;
+                float2 acc[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll 4
-                for (int t = q * TPQ; t < (q + 1) * TPQ; ++t) {
-                    const uint32_t wd = *reinterpret_cast<const uint32_t*>(
-                        sp + (j0 / 64) * 16384 + t * 128 + ((((j0 % 64) / 8) ^ (t & 7)) << 4) + (j0 % 8) * 2);
-                    const float2 xv = (DT == DT_BF16) ? make_float2(u2f(wd << 16), u2f(wd & 0xFFFF0000u))
-                                                      : __half22float2(*reinterpret_cast<const __half2*>(&wd));
+                for (int t = q * TPG; t < (q + 1) * TPG; ++t) {
+                    const uint4 wv = *reinterpret_cast<const uint4*>(cb + t * 128 + (((o % 8) ^ (t & 7)) << 4));
+                    const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
                     const float sct = xch[t];
-                    acc = __ffma2_rn(xv, make_float2(sct, sct), acc);
+                    const float2 s2 = make_float2(sct, sct);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 xv = (DT == DT_BF16)
+                                              ? make_float2(u2f(w4[k] << 16), u2f(w4[k] & 0xFFFF0000u))
+                                              : __half22float2(*reinterpret_cast<const __half2*>(&w4[k]));
+                        acc[k] = __ffma2_rn(xv, s2, acc[k]);
+                    }
                 }
-                opart[q * P + p] = acc;
+                float4* dst = reinterpret_cast<float4*>(opart + q * D + 8 * o);
+                dst[0] = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+                dst[1] = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
             }
             named_bar_sync(bar_id, 128);
-            float om = 0.f;  // channel r's block mean (r < D)
+            // thread r holds the block means of channels r + 128 k (k < kCh; r < D)
+            constexpr int kCh = (D + 127) / 128;
+            float om[kCh];
             if (r < D) {
-                constexpr int P = D / 2, Q = kTileRows / P;
-                float acc = 0.f;
+                constexpr int QG = kTileRows / (D / 8);
+                float mn = INFINITY, mxo = -INFINITY;
 #pragma unroll
-                for (int q = 0; q < Q; ++q) {
-                    const float2 pq = opart[q * P + r / 2];
-                    acc += (r & 1) ? pq.y : pq.x;
+                for (int k = 0; k < kCh; ++k) {
+                    const int ch = r + 128 * k;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int q = 0; q < QG; ++q) acc += opart[q * D + ch];
+                    om[k] = acc * (1.0f / kTileRows);
+                    if constexpr (!DQ) {
+                        const __half o16 = __float2half_rn(om[k]);
+                        if (tile * kTileRows < n_s) a.block_mean[tile * D + ch] = o16;
+                        const uint32_t ps = a.pair_sign[ch >> 1];
+                        const bool neg = ((ps >> ((ch & 1) ? 31 : 15)) & 1u) != 0;
+                        so[ch] = neg ? -__half2float(o16) : __half2float(o16);
+                    } else {
+                        mn = fminf(mn, om[k]);
+                        mxo = fmaxf(mxo, om[k]);
+                    }
                 }
-                om = acc * (1.0f / kTileRows);
-                if constexpr (!DQ) {
-                    const __half o16 = __float2half_rn(om);
-                    if (tile * kTileRows < n_s) a.block_mean[tile * D + r] = o16;
-                    const uint32_t ps = a.pair_sign[r >> 1];
-                    const bool neg = ((ps >> ((r & 1) ? 31 : 15)) & 1u) != 0;
-                    so[r] = neg ? -__half2float(o16) : __half2float(o16);
-                } else {
-                    float mn = om, mxo = om;
+                if constexpr (DQ) {
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) {
                         mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
@@ -580,28 +626,33 @@ __global__ void __launch_bounds__(512, 1)
                 // step = fp16((max o - min o) / 15); o_hat = fp32(lo + step q)
                 named_bar_sync(bar_id, 128);
                 if (r < D) {
+                    constexpr int kMW = (D < 128 ? D : 128) / 32;  // warps holding channels
                     float lo = red[0], hi = red[4];
 #pragma unroll
-                    for (int w = 1; w < D / 32; ++w) {
+                    for (int w = 1; w < kMW; ++w) {
                         lo = fminf(lo, red[w]);
                         hi = fmaxf(hi, red[4 + w]);
                     }
                     const __half lo16 = __float2half_rn(lo), st16 = __float2half_rn((hi - lo) / 15.0f);
                     const float lof = __half2float(lo16), stf = __half2float(st16);
-                    int qo = 0;
-                    if (stf > 0.f) qo = min(max(__float2int_rn((om - lof) / stf), 0), 15);
-                    const float oh = fmaf(stf, static_cast<float>(qo), lof);
-                    const int qp = __shfl_down_sync(0xFFFFFFFFu, qo, 1);
-                    if (tile * kTileRows < n_s) {
-                        if ((r & 1) == 0) rec[8 + r / 2] = static_cast<uint8_t>(qo | (qp << 4));
-                        if (r == 0) {
-                            *reinterpret_cast<__half*>(rec) = lo16;
-                            *reinterpret_cast<__half*>(rec + 2) = st16;
+#pragma unroll
+                    for (int k = 0; k < kCh; ++k) {
+                        const int ch = r + 128 * k;
+                        int qo = 0;
+                        if (stf > 0.f) qo = min(max(__float2int_rn((om[k] - lof) / stf), 0), 15);
+                        const float oh = fmaf(stf, static_cast<float>(qo), lof);
+                        const int qp = __shfl_down_sync(0xFFFFFFFFu, qo, 1);
+                        if (tile * kTileRows < n_s) {
+                            if ((ch & 1) == 0) rec[8 + ch / 2] = static_cast<uint8_t>(qo | (qp << 4));
+                            if (ch == 0) {
+                                *reinterpret_cast<__half*>(rec) = lo16;
+                                *reinterpret_cast<__half*>(rec + 2) = st16;
+                            }
                         }
+                        const uint32_t ps = a.pair_sign[ch >> 1];
+                        const bool neg = ((ps >> ((ch & 1) ? 31 : 15)) & 1u) != 0;
+                        so[ch] = neg ? -oh : oh;
                     }
-                    const uint32_t ps = a.pair_sign[r >> 1];
-                    const bool neg = ((ps >> ((r & 1) ? 31 : 15)) & 1u) != 0;
-                    so[r] = neg ? -oh : oh;
                 }
             }
             named_bar_sync(bar_id, 128);
@@ -641,61 +692,148 @@ __global__ void __launch_bounds__(512, 1)
         if (r == 0) issue_tile(i + NS);  // the stage has been read
         tc_fence_after();
 
-        // ---- pass 1: ||y||^2 = D ||x||^2 (the next chunk loads while one is summed) ----
-        constexpr int NC = D / 32;
-        uint32_t ybuf[2][32];
-        float2 acc2 = make_float2(0.f, 0.f);
-        tmem_ld32(tl, ybuf[0]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            if (c + 1 < NC) tmem_ld32(tl + 32 * (c + 1), ybuf[(c + 1) & 1]);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                float2 y = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
-                if constexpr (NSN) {
-                    const float2 h2 = reinterpret_cast<const float2*>(ho)[16 * c + k];
-                    y = __ffma2_rn(y, make_float2(sc, sc), make_float2(-h2.x, -h2.y));  // H D w
-                }
-                acc2 = __ffma2_rn(y, y, acc2);
-            }
-            if (c + 1 < NC) tmem_wait_ld();
-        }
-        const float ssx = (acc2.x + acc2.y) * (1.0f / D);
-        const float nrm = sqrtf(ssx);  // ||x||, or ||w|| for NSN
-        if (!NSN) flag_norm(ssx, nrm, a.status);
-        const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
-        // ---- pass 2: codes, residual (fp16 into columns [16c, 16c + 16)) ----
-        // Group c + 1 loads while group c is coded; the residual of group c
-        // goes to columns that groups 0 .. c/2 occupied, all read already.
+        float nrm, rr;
         uint32_t planes[B][kWpp];
-        float2 rr2 = make_float2(0.f, 0.f);
-        const VecTab<B> vt(ctab, nrm, inv);
-        tmem_ld32(tl, ybuf[0]);
-        tmem_wait_ld();
+        if constexpr (C::kNMat == 1) {
+            // ---- pass 1: ||y||^2 = D ||x||^2 (the next chunk loads while one is summed) ----
+            constexpr int NC = D / 32;
+            uint32_t ybuf[2][32];
+            float2 acc2 = make_float2(0.f, 0.f);
+            tmem_ld32(tl, ybuf[0]);
+            tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            if (c + 1 < NC) tmem_ld32(tl + 32 * (c + 1), ybuf[(c + 1) & 1]);
-            float2 v[16];
+            for (int c = 0; c < NC; ++c) {
+                if (c + 1 < NC) tmem_ld32(tl + 32 * (c + 1), ybuf[(c + 1) & 1]);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                v[k] = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
-                if constexpr (NSN) {
-                    const float2 h2 = reinterpret_cast<const float2*>(ho)[16 * c + k];
-                    v[k] = __ffma2_rn(v[k], make_float2(sc, sc), make_float2(-h2.x, -h2.y));
+                for (int k = 0; k < 16; ++k) {
+                    float2 y = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
+                    if constexpr (NSN) {
+                        const float2 h2 = reinterpret_cast<const float2*>(ho)[16 * c + k];
+                        y = __ffma2_rn(y, make_float2(sc, sc), make_float2(-h2.x, -h2.y));  // H D w
+                    }
+                    acc2 = __ffma2_rn(y, y, acc2);
                 }
+                if (c + 1 < NC) tmem_wait_ld();
             }
-            uint32_t hres[16], w[B];
-            code_group<B>(v, ctab, vt, hres, w, rr2);
+            const float ssx = (acc2.x + acc2.y) * (1.0f / D);
+            nrm = sqrtf(ssx);  // ||x||, or ||w|| for NSN
+            if (!NSN) flag_norm(ssx, nrm, a.status);
+            const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+            // ---- pass 2: codes, residual (fp16 into columns [16c, 16c + 16)) ----
+            // Group c + 1 loads while group c is coded; the residual of group c
+            // goes to columns that groups 0 .. c/2 occupied, all read already.
+            float2 rr2 = make_float2(0.f, 0.f);
+            const VecTab<B> vt(ctab, nrm, inv);
+            tmem_ld32(tl, ybuf[0]);
+            tmem_wait_ld();
 #pragma unroll
-            for (int p = 0; p < B; ++p) planes[p][c] = w[p];
-            // Stored without QJL too (except behind the NSN front end): consuming
-            // the residual group by group keeps the register allocation within
-            // the 128 registers of a thread.
-            if (!NSN) tmem_st16(tl + 16 * c, hres);
-            if (c + 1 < NC) tmem_wait_ld();
+            for (int c = 0; c < NC; ++c) {
+                if (c + 1 < NC) tmem_ld32(tl + 32 * (c + 1), ybuf[(c + 1) & 1]);
+                float2 v[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    v[k] = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
+                    if constexpr (NSN) {
+                        const float2 h2 = reinterpret_cast<const float2*>(ho)[16 * c + k];
+                        v[k] = __ffma2_rn(v[k], make_float2(sc, sc), make_float2(-h2.x, -h2.y));
+                    }
+                }
+                uint32_t hres[16], w[B];
+                code_group<B>(v, ctab, vt, hres, w, rr2);
+#pragma unroll
+                for (int p = 0; p < B; ++p) planes[p][c] = w[p];
+                // Stored without QJL too (except behind the NSN front end): consuming
+                // the residual group by group keeps the register allocation within
+                // the 128 registers of a thread.
+                if (!NSN) tmem_st16(tl + 16 * c, hres);
+                if (c + 1 < NC) tmem_wait_ld();
+            }
+            rr = rr2.x + rr2.y;
+        } else {
+            // ---- d = 256: columns [0, 128) hold P, [128, 256) Q; group c < 4 of
+            // the rotated vector is P_c + Q_c, group 4 + c is P_c - Q_c ----
+            const float2 m1 = make_float2(-1.f, -1.f);
+            const float2 sc2 = make_float2(sc, sc);
+            const float2* ho2 = reinterpret_cast<const float2*>(ho);
+            // y of group (c, half) from the loaded P and Q words, pair k
+            auto ypair = [&](const uint32_t(&pw)[32], const uint32_t(&qw)[32], int c, int half, int k) {
+                const float2 pv = make_float2(u2f(pw[2 * k]), u2f(pw[2 * k + 1]));
+                const float2 qv = make_float2(u2f(qw[2 * k]), u2f(qw[2 * k + 1]));
+                float2 y = half ? __ffma2_rn(qv, m1, pv) : __fadd2_rn(pv, qv);
+                if constexpr (NSN) {
+                    const float2 h2 = ho2[16 * (4 * half + c) + k];
+                    y = __ffma2_rn(y, sc2, make_float2(-h2.x, -h2.y));  // H D w
+                }
+                return y;
+            };
+            // One buffer: both halves of group c are formed from P_c and Q_c,
+            // then P_{c+1} and Q_{c+1} load into the same registers while
+            // group c is summed or coded.
+            // (pin2 keeps the formed values from being computed after the next
+            // load, which would keep the old P and Q words live beside it)
+            auto pin2 = [](float2& v) { asm volatile("" : "+f"(v.x), "+f"(v.y)); };
+            uint32_t pb[32], qb[32];
+            // ---- pass 1: ||y||^2 ----
+            float2 acc2 = make_float2(0.f, 0.f);
+            tmem_ld32(tl, pb);
+            tmem_ld32(tl + 128, qb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float2 yt[16], yb[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    yt[k] = ypair(pb, qb, c, 0, k);
+                    yb[k] = ypair(pb, qb, c, 1, k);
+                    pin2(yt[k]);
+                    pin2(yb[k]);
+                }
+                if (c + 1 < 4) {
+                    tmem_ld32(tl + 32 * (c + 1), pb);
+                    tmem_ld32(tl + 128 + 32 * (c + 1), qb);
+                }
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    acc2 = __ffma2_rn(yt[k], yt[k], acc2);
+                    acc2 = __ffma2_rn(yb[k], yb[k], acc2);
+                }
+                if (c + 1 < 4) tmem_wait_ld();
+            }
+            const float ssx = (acc2.x + acc2.y) * (1.0f / D);
+            nrm = sqrtf(ssx);  // ||x||, or ||w|| for NSN
+            if (!NSN) flag_norm(ssx, nrm, a.status);
+            const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+            // ---- pass 2: codes of both halves of each group (no QJL: the residual is only summed) ----
+            float2 rr2 = make_float2(0.f, 0.f);
+            const VecTab<B> vt(ctab, nrm, inv);
+            tmem_ld32(tl, pb);
+            tmem_ld32(tl + 128, qb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float2 yt[16], yb[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    yt[k] = ypair(pb, qb, c, 0, k);
+                    yb[k] = ypair(pb, qb, c, 1, k);
+                    pin2(yt[k]);
+                    pin2(yb[k]);
+                }
+                if (c + 1 < 4) {
+                    tmem_ld32(tl + 32 * (c + 1), pb);
+                    tmem_ld32(tl + 128 + 32 * (c + 1), qb);
+                }
+                uint32_t hres[16], w[B];
+                code_group<B>(yt, ctab, vt, hres, w, rr2);
+#pragma unroll
+                for (int p = 0; p < B; ++p) planes[p][c] = w[p];
+                code_group<B>(yb, ctab, vt, hres, w, rr2);
+#pragma unroll
+                for (int p = 0; p < B; ++p) planes[p][4 + c] = w[p];
+                if (c + 1 < 4) tmem_wait_ld();
+            }
+            rr = rr2.x + rr2.y;
         }
-        const float rr = rr2.x + rr2.y;
         const uint32_t zmask = nrm > 0.f ? 0xFFFFFFFFu : 0u;
         const int64_t vidx = tile * kTileRows + r;
         const bool valid = vidx < n_s;

@@ -88,12 +88,12 @@ extern "C" {
  * [-sqrt(d), sqrt(d)]; TurboQuant blog, "Estágio 1") instead of N(0, 1). */
 #define KVQ_BETA_CODEBOOK 2u
 /* Rotation on the CUDA cores: kvq_quantize / kvq_quantize_batch with 16-bit
- * input at d <= 128 rotate by the in-register Walsh-Hadamard transform (the
- * kernel fp32 input and d = 256 use) instead of the tensor-core product
- * X (H D)^T.  Same outputs under the same rules (codes exact outside the
- * decision-level band, norms within one fp16 ulp); one launch per job.  For
- * comparing the two rotations at one configuration; the NSN entry points
- * ignore it. */
+ * input, wherever the tensor-core product X (H D)^T would run (d <= 128, and
+ * d = 256 without KVQ_QJL), rotate by the in-register Walsh-Hadamard
+ * transform instead (the kernel that fp32 input and d = 256 with QJL use).
+ * Same outputs under the same rules (codes exact outside the decision-level
+ * band, norms within one fp16 ulp); one launch per job.  For comparing the
+ * two rotations at one configuration; the NSN entry points ignore it. */
 #define KVQ_CUDA_CORE_ROTATION 4u
 
 /* ---- element types of inputs ------------------------------------------ */
@@ -179,10 +179,11 @@ typedef struct kvq_quant_job {
 /*
  * kvq_quantize_batch -- kvq_quantize of `count` streams of vectors (for
  * instance the keys and the values of one layer) in as few launches as the
- * kernels allow: two consecutive non-empty jobs of the same 16-bit dtype at
- * d <= 128 share one launch, whose tiles are those of the first job then
- * those of the second; the others take one launch each.  The outputs are
- * exactly those of one kvq_quantize call per job.
+ * kernels allow: two consecutive non-empty jobs of the same 16-bit dtype
+ * share one launch (at d <= 128, and at d = 256 without KVQ_QJL), whose
+ * tiles are those of the first job then those of the second; the others
+ * take one launch each.  The outputs are exactly those of one kvq_quantize
+ * call per job.
  *   count  >= 0; jobs  host array of `count` descriptors (read during the
  *          call only).  Every job is checked before anything is launched;
  *          an error names the job ("job i: ...") and launches nothing.

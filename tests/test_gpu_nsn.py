@@ -69,7 +69,7 @@ def check_head(k, x, codes_g, norms_g, means_g, pool=None):
 
 @pytest.mark.parametrize("d,b,dtype", [(128, 2, torch.bfloat16), (128, 1, torch.float16), (64, 3, torch.float32),
                                        (64, 4, torch.bfloat16),
-                                       # d = 256: the in-register transform kernel, two threads per vector
+                                       # d = 256: the rotation as two 128-wide tensor-core products
                                        (256, 2, torch.bfloat16), (256, 3, torch.float16), (256, 4, torch.bfloat16)])
 def test_nsn_matches_oracle(d, b, dtype):
     x = wl.nsn_tokens(2, 512, d, seed=d + b, dtype=dtype)
@@ -117,9 +117,10 @@ def test_nsn_workload_full_size_sampled():
                to_np_f16bits(means[-1, -1:]))
 
 
-def test_nsn_block32_layout_matches_token_layout():
+@pytest.mark.parametrize("d", [128, 256])
+def test_nsn_block32_layout_matches_token_layout(d):
     """Values are stored in the block-32 layout: the same bits, norms and block means."""
-    d, b = 128, 2
+    b = 2
     x = wl.nsn_tokens(2, 256, d, seed=9).cuda()
     with kvq.Handle(d, b, 3, qjl=False) as h:
         c0, n0, m0 = run_nsn(h, x)

@@ -116,8 +116,8 @@ def run_dq(h, x, layout=0):
 
 @pytest.mark.parametrize("d,b,dtype", [(128, 2, torch.bfloat16), (128, 1, torch.float16), (64, 3, torch.bfloat16),
                                        (64, 2, torch.float16), (128, 4, torch.bfloat16),
-                                       # d = 256: the in-register transform kernel, two threads per vector
-                                       (256, 2, torch.bfloat16), (256, 4, torch.float16)])
+                                       # d = 256: the rotation as two 128-wide tensor-core products
+                                       (256, 2, torch.bfloat16), (256, 4, torch.float16), (256, 1, torch.bfloat16)])
 def test_nsn_dq_matches_oracle(d, b, dtype):
     x = wl.nsn_tokens(2, 512, d, seed=30 + d + b, dtype=dtype)
     x[1, 130] = 0  # a zero token inside a block
@@ -131,8 +131,9 @@ def test_nsn_dq_matches_oracle(d, b, dtype):
     assert (_nib(side[1].cpu().numpy(), 8 + d // 2, 128)[1, 2] == 0)  # token 130 = block 1, row 2
 
 
-def test_nsn_dq_block32_layout_matches_token_layout():
-    d, b = 128, 2
+@pytest.mark.parametrize("d", [128, 256])
+def test_nsn_dq_block32_layout_matches_token_layout(d):
+    b = 2
     x = wl.nsn_tokens(2, 256, d, seed=9).cuda()
     with kvq.Handle(d, b, 3, qjl=False) as h:
         c0, w0, s0 = run_dq(h, x)

@@ -226,7 +226,8 @@ BATCH_CASES = [
     (64, 1, False, (torch.float16, 129, 1), (torch.float16, 2000, 0)),    # fused, block-32 first
     (128, 4, True, (torch.bfloat16, 31, 0), (torch.bfloat16, 33, 1)),     # fused, both under one tile
     (128, 3, True, (torch.bfloat16, 515, 0), (torch.float16, 257, 1)),    # dtypes differ: two launches
-    (256, 2, True, (torch.bfloat16, 300, 0), (torch.bfloat16, 300, 1)),   # d = 256: two launches
+    (256, 2, True, (torch.bfloat16, 300, 0), (torch.bfloat16, 300, 1)),   # d = 256 with QJL: two launches
+    (256, 4, False, (torch.float16, 700, 1), (torch.float16, 129, 0)),    # d = 256 without QJL: fused
     (128, 2, False, (torch.float32, 100, 0), (torch.float32, 70, 1)),     # fp32: two launches
 ]
 
@@ -257,10 +258,13 @@ def test_quantize_batch_matches_oracle_and_single_calls(d, b, qjl, j0, j1):
     (64, 3, False, torch.float16, 257, 0),
     (128, 4, True, torch.float16, 300, 0),
     (64, 1, True, torch.bfloat16, 129, 1),
+    (256, 2, False, torch.bfloat16, 300, 0),
+    (256, 3, False, torch.float16, 129, 1),
 ])
 def test_cuda_core_rotation_matches_oracle(d, b, qjl, dtype, n, layout):
-    """KVQ_CUDA_CORE_ROTATION: 16-bit input at d <= 128 through the in-register transform kernel, under the
-    same parity rules; a layer's K and V through kvq_quantize_batch (one launch per job)."""
+    """KVQ_CUDA_CORE_ROTATION: 16-bit input, wherever the tensor-core rotation would run (d <= 128, and d = 256
+    without QJL), through the in-register transform kernel, under the same parity rules; a layer's K and V
+    through kvq_quantize_batch (one launch per job)."""
     x = wl.sweep_tokens(n, d, seed=500 + d + b, dtype=dtype)
     x[1] = 0
     k = constants(d, b, 9)
