@@ -47,7 +47,7 @@ struct QuantArgs {
     __half2* norms;                   // [n]
     __half* block_mean;               // NSN: [n/128][d]
     uint8_t* side;                    // NSN with double quantization: one side record per 128 rows (else null)
-    int cuda_core_rotation;           // 16-bit input, d <= 128: the in-register transform kernel instead
+    int cuda_core_rotation;           // plain 16-bit input: the in-register transform kernel instead of tcgen05
     const __half* S;                  // [m][d] fp16 (global), copied to smem per CTA
     uint32_t* status;
     float centroid[kMaxLevels];

@@ -692,6 +692,12 @@ __global__ void __launch_bounds__(TcCfg<D, QJL, NSN>::kThreads, 1)
         if (r == 0) issue_tile(i + NS);  // the stage has been read
         tc_fence_after();
 
+        // -ho for the pair idx of the rotated vector (column order), read as the
+        // 16-byte chunk holding pairs idx & ~1 and idx | 1 (one load serves both)
+        auto ho_neg = [&](int idx) {
+            const float4 hq = reinterpret_cast<const float4*>(ho)[idx >> 1];
+            return (idx & 1) ? make_float2(-hq.z, -hq.w) : make_float2(-hq.x, -hq.y);
+        };
         float nrm, rr;
         uint32_t planes[B][kWpp];
         if constexpr (C::kNMat == 1) {
@@ -707,10 +713,7 @@ __global__ void __launch_bounds__(TcCfg<D, QJL, NSN>::kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     float2 y = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
-                    if constexpr (NSN) {
-                        const float2 h2 = reinterpret_cast<const float2*>(ho)[16 * c + k];
-                        y = __ffma2_rn(y, make_float2(sc, sc), make_float2(-h2.x, -h2.y));  // H D w
-                    }
+                    if constexpr (NSN) y = __ffma2_rn(y, make_float2(sc, sc), ho_neg(16 * c + k));  // H D w
                     acc2 = __ffma2_rn(y, y, acc2);
                 }
                 if (c + 1 < NC) tmem_wait_ld();
@@ -733,10 +736,7 @@ __global__ void __launch_bounds__(TcCfg<D, QJL, NSN>::kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     v[k] = make_float2(u2f(ybuf[c & 1][2 * k]), u2f(ybuf[c & 1][2 * k + 1]));
-                    if constexpr (NSN) {
-                        const float2 h2 = reinterpret_cast<const float2*>(ho)[16 * c + k];
-                        v[k] = __ffma2_rn(v[k], make_float2(sc, sc), make_float2(-h2.x, -h2.y));
-                    }
+                    if constexpr (NSN) v[k] = __ffma2_rn(v[k], make_float2(sc, sc), ho_neg(16 * c + k));
                 }
                 uint32_t hres[16], w[B];
                 code_group<B>(v, ctab, vt, hres, w, rr2);
@@ -754,16 +754,12 @@ __global__ void __launch_bounds__(TcCfg<D, QJL, NSN>::kThreads, 1)
             // the rotated vector is P_c + Q_c, group 4 + c is P_c - Q_c ----
             const float2 m1 = make_float2(-1.f, -1.f);
             const float2 sc2 = make_float2(sc, sc);
-            const float2* ho2 = reinterpret_cast<const float2*>(ho);
             // y of group (c, half) from the loaded P and Q words, pair k
             auto ypair = [&](const uint32_t(&pw)[32], const uint32_t(&qw)[32], int c, int half, int k) {
                 const float2 pv = make_float2(u2f(pw[2 * k]), u2f(pw[2 * k + 1]));
                 const float2 qv = make_float2(u2f(qw[2 * k]), u2f(qw[2 * k + 1]));
                 float2 y = half ? __ffma2_rn(qv, m1, pv) : __fadd2_rn(pv, qv);
-                if constexpr (NSN) {
-                    const float2 h2 = ho2[16 * (4 * half + c) + k];
-                    y = __ffma2_rn(y, sc2, make_float2(-h2.x, -h2.y));  // H D w
-                }
+                if constexpr (NSN) y = __ffma2_rn(y, sc2, ho_neg(16 * (4 * half + c) + k));  // H D w
                 return y;
             };
             // One buffer: both halves of group c are formed from P_c and Q_c,
