@@ -114,6 +114,12 @@ def test_tiny_reference_workload():
     (256, 4, False, 1, 2, 1, [129], 160, torch.bfloat16),
     (128, 1, False, 1, 2, 2, [300], 320, torch.bfloat16),            # tensor-core path, GQA 1:1
     (128, 2, False, 2, 4, 1, [900, 64], 960, torch.float16),          # tensor-core path without QJL
+    (256, 1, True, 1, 4, 1, [700], 704, torch.bfloat16),              # d = 256, 1 bit: tensor-core path
+    (256, 1, False, 2, 2, 2, [300, 45], 320, torch.float16),          # ... without QJL, ragged
+    (256, 3, True, 1, 8, 2, [513], 544, torch.bfloat16),              # d = 256, 3 bits: CUDA-core path
+    (256, 3, False, 2, 4, 4, [1, 260], 288, torch.bfloat16),          # ... one-token context
+    (128, 4, True, 1, 8, 2, [600], 608, torch.bfloat16),              # 4 bits with QJL: CUDA-core path
+    (64, 4, True, 2, 4, 1, [333, 0], 352, torch.float16),             # ... d = 64, an empty context
 ])
 def test_decode_matches_oracle(d, b, qjl, batch, hq, hkv, seq_len, cap, qdt):
     check_case(d, b, qjl, batch, hq, hkv, seq_len, cap, scale=1 / np.sqrt(d), qdtype=qdt)
@@ -209,7 +215,7 @@ def test_decode_workload_full_size_sampled():
 
 
 @pytest.mark.parametrize("d,b,qjl", [(64, 1, False), (64, 3, True), (128, 2, True), (128, 4, False),
-                                     (256, 2, False)])
+                                     (256, 2, False), (256, 3, True), (256, 1, False)])
 def test_sweep_decode_full_size_sampled(d, b, qjl):
     """Bit-width / head-dim sweep: the 1,048,576 bf16 vectors (1% x10) as 8 KV heads x 131072 tokens,
     quantized as K and V by the CUDA path, one N(0,1) query per KV head; one sampled head is checked
