@@ -52,6 +52,8 @@ def parse():
                     help="context length of the decode measurement (default: the workload's 131072)")
     ap.add_argument("--soak", type=float, default=1.5,
                     help="seconds of untimed steps under the clock sampler before the timed region")
+    ap.add_argument("--sweep-rows", default=None,
+                    help="run only these sweep rows, as d:b:qjl[,d:b:qjl...] (qjl 0 or 1; for profiler captures)")
     return ap.parse_args()
 
 
@@ -649,14 +651,21 @@ def bench_sweep(args, dist):
     hbm, src = peaks()
     stream = torch.cuda.current_stream()
     steps = max(5, args.steps // 3)
+    keep = None
+    if args.sweep_rows:
+        keep = {tuple(int(v) for v in r.split(":")) for r in args.sweep_rows.split(",")}
     rows = []
     for d in c["dims"]:
+        if keep is not None and not any(k[0] == d for k in keep):
+            continue
         X = [wl.sweep_tokens(n, d, c["seed"] + 2 * d + i + 1000 * dist.rank, device="cuda") for i in range(2)]
         q = wl.queries(1, hkv, d, c["seed"] + 7 * d, device="cuda")
         seq = torch.full((1,), T, dtype=torch.int32, device="cuda")
         out = torch.empty((1, hkv, d), dtype=torch.float32, device="cuda")
         for b in c["bits"]:
             for qjl in c["qjl"]:
+                if keep is not None and (d, b, int(qjl)) not in keep:
+                    continue
                 h = kvq.Handle(d, b, c["handle_seed"], qjl=qjl)
                 outK = kvq.alloc_packed(h, n)
                 outV = kvq.alloc_packed(h, n, layout=kvq.KVQ_LAYOUT_BLOCK32)
