@@ -769,33 +769,59 @@ __global__ void __launch_bounds__(TcCfg<D, QJL, NSN>::kThreads, 1)
             // load, which would keep the old P and Q words live beside it)
             auto pin2 = [](float2& v) { asm volatile("" : "+f"(v.x), "+f"(v.y)); };
             uint32_t pb[32], qb[32];
-            // ---- pass 1: ||y||^2 ----
+            // ---- pass 1: ||y||^2 (without the NSN shift, 2 (||P||^2 + ||Q||^2)) ----
             float2 acc2 = make_float2(0.f, 0.f);
             tmem_ld32(tl, pb);
             tmem_ld32(tl + 128, qb);
             tmem_wait_ld();
+            if constexpr (!NSN) {
+                float2 accq = make_float2(0.f, 0.f);
+                // P_{c+1} loads while Q_c is summed
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float2 yt[16], yb[16];
+                for (int c = 0; c < 4; ++c) {
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    yt[k] = ypair(pb, qb, c, 0, k);
-                    yb[k] = ypair(pb, qb, c, 1, k);
-                    pin2(yt[k]);
-                    pin2(yb[k]);
-                }
-                if (c + 1 < 4) {
-                    tmem_ld32(tl + 32 * (c + 1), pb);
-                    tmem_ld32(tl + 128 + 32 * (c + 1), qb);
-                }
+                    for (int k = 0; k < 16; ++k) {
+                        const float2 pv = make_float2(u2f(pb[2 * k]), u2f(pb[2 * k + 1]));
+                        acc2 = __ffma2_rn(pv, pv, acc2);
+                    }
+                    pin2(acc2);
+                    if (c + 1 < 4) tmem_ld32(tl + 32 * (c + 1), pb);
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    acc2 = __ffma2_rn(yt[k], yt[k], acc2);
-                    acc2 = __ffma2_rn(yb[k], yb[k], acc2);
+                    for (int k = 0; k < 16; ++k) {
+                        const float2 qv = make_float2(u2f(qb[2 * k]), u2f(qb[2 * k + 1]));
+                        accq = __ffma2_rn(qv, qv, accq);
+                    }
+                    pin2(accq);
+                    if (c + 1 < 4) {
+                        tmem_ld32(tl + 128 + 32 * (c + 1), qb);
+                        tmem_wait_ld();
+                    }
                 }
-                if (c + 1 < 4) tmem_wait_ld();
+                acc2 = __fadd2_rn(acc2, accq);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float2 yt[16], yb[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        yt[k] = ypair(pb, qb, c, 0, k);
+                        yb[k] = ypair(pb, qb, c, 1, k);
+                        pin2(yt[k]);
+                        pin2(yb[k]);
+                    }
+                    if (c + 1 < 4) {
+                        tmem_ld32(tl + 32 * (c + 1), pb);
+                        tmem_ld32(tl + 128 + 32 * (c + 1), qb);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        acc2 = __ffma2_rn(yt[k], yt[k], acc2);
+                        acc2 = __ffma2_rn(yb[k], yb[k], acc2);
+                    }
+                    if (c + 1 < 4) tmem_wait_ld();
+                }
             }
-            const float ssx = (acc2.x + acc2.y) * (1.0f / D);
+            const float ssx = (acc2.x + acc2.y) * ((NSN ? 1.0f : 2.0f) / D);
             nrm = sqrtf(ssx);  // ||x||, or ||w|| for NSN
             if (!NSN) flag_norm(ssx, nrm, a.status);
             const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
